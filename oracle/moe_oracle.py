@@ -1,0 +1,245 @@
+"""CPU oracle for the sparse Mixture-of-Experts layer forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Only tests/, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import or run this module; the product
+path (the CUDA library and its Python binding) never does.
+
+It is a plain, slow, float64 NumPy restatement of the layer defined on the
+page "Mixture of experts" (rayaq.ca/ml-models/mixture-of-experts):
+
+  * section "Replacing the feed-forward block", eq. h = W_r x, p = softmax(h),
+    y = sum_{i in TopK(h)} g_i(x) E_i(x);
+  * section "Top-k gating": keep the k largest logits, largest first; Switch
+    gate (k = 1) = the chosen expert's full-softmax probability; renormalised
+    gate = softmax over the k chosen logits;
+  * section "The load-balancing loss": L_aux / alpha = E * sum_i f_i P_i with
+    f_i the share of tokens whose top choice is i and P_i the mean router
+    probability; router z-loss = mean over tokens of (log sum_j exp h_j)^2;
+  * section "Capacity and dropped tokens": capacity = tokens/experts x
+    capacity factor; slots are filled in position order and the overflow is
+    dropped (the layer's output for a dropped assignment is zero; the caller's
+    residual carries the input);
+  * section "Implementation": SwiGLU expert w2(silu(w1 x) * w3 x); the router
+    is computed in float32; the gated expert outputs are summed per token.
+
+Readings where the page is silent (each is listed with its reason in the
+design notes of this repository):
+  - ties in top-k go to the lower expert index;
+  - capacity C = ceil(capacity_factor * T * k / E) (equal to the page's
+    formula at k = 1); capacity_factor <= 0 means dropless;
+  - slot priority is token order alone (a token's second choice can take a
+    slot before a later token's first choice);
+  - f_i counts first choices of all T tokens before any dropping; P_i is the
+    full softmax over all E experts;
+  - gates are not renormalised after drops;
+  - the ReLU expert is w2(relu(w1 x)) (the feed-forward block of the same
+    page's "Problem" section, with no biases, like the SwiGLU listing);
+  - router logits are rounded once to fp32 and every routing decision is
+    taken on those fp32 values.
+
+Parity pins: every function here is pinned by tests/test_oracle_pins.py
+against closed forms, brute force, library routines and the page's stated
+special cases (see that file's docstrings).
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Sequence
+
+import numpy as np
+
+ACT_RELU, ACT_SWIGLU = 0, 1
+GATE_SWITCH, GATE_RENORM = 0, 1
+
+
+def router_logits(x, W_r, b_r=None) -> np.ndarray:
+    """Router logits h = W_r x (+ b) per token, as fp32.
+
+    "Replacing the feed-forward block": the router is one linear layer with E
+    rows.  Accumulated in float64 and rounded once to float32 ("compute the
+    router in float32", section "Implementation").
+    x: [T][d], W_r: [E][d], b_r: [E] or None.  Returns float32 [T][E].
+    """
+    h = np.asarray(x, np.float64) @ np.asarray(W_r, np.float64).T
+    if b_r is not None:
+        h = h + np.asarray(b_r, np.float64)[None, :]
+    return h.astype(np.float32)
+
+
+def softmax_lse(h32: np.ndarray):
+    """Full softmax p over the E experts and the log-sum-exp of each token.
+
+    p = softmax(h) ("Replacing the feed-forward block"); lse = log sum_j exp h_j
+    (the z-loss term of "The load-balancing loss").  float64 from the fp32 logits.
+    """
+    h = np.asarray(h32, np.float64)
+    if h.shape[0] == 0:
+        return np.zeros_like(h), np.zeros(0)
+    m = h.max(axis=1, keepdims=True)
+    e = np.exp(h - m)
+    Z = e.sum(axis=1, keepdims=True)
+    return e / Z, (m + np.log(Z))[:, 0]
+
+
+def top_k(h32: np.ndarray, k: int) -> np.ndarray:
+    """Indices of the k largest logits of each token, largest first.
+
+    "Top-k gating": the router keeps the k largest logits.  Selection is done
+    k times on the fp32 values: take the largest remaining logit; among equal
+    logits (+0 and -0 compare equal) the lower expert index wins.
+    Returns int64 [T][k].
+    """
+    h = np.asarray(h32, np.float64).copy()
+    T = h.shape[0]
+    idx = np.empty((T, k), np.int64)
+    rows = np.arange(T)
+    for j in range(k):
+        sel = np.argmax(h, axis=1)  # first index among equal maxima
+        idx[:, j] = sel
+        h[rows, sel] = -np.inf
+    return idx
+
+
+def gates(h32: np.ndarray, p: np.ndarray, idx: np.ndarray, gate_mode: int) -> np.ndarray:
+    """Gate value of each chosen expert ("Top-k gating").
+
+    SWITCH: g_j = p[idx_j], the full-softmax probability (below 1 for E > 1).
+    RENORM: g = softmax over the k chosen logits, which equals the chosen
+    full-softmax probabilities divided by their sum.
+    Returns float64 [T][k].
+    """
+    rows = np.arange(idx.shape[0])[:, None]
+    if gate_mode == GATE_SWITCH:
+        return p[rows, idx]
+    sel = np.asarray(h32, np.float64)[rows, idx]
+    if sel.shape[0] == 0:
+        return sel
+    e = np.exp(sel - sel[:, :1])  # idx[:, 0] holds the largest logit
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def expert_capacity(capacity_factor: float, T: int, k: int, E: int) -> Optional[int]:
+    """Slots per expert ("Capacity and dropped tokens").
+
+    The page's rule is tokens/experts x capacity factor; with k assignments per
+    token the assignments per expert are T*k/E, so C = ceil(cf * T * k / E)
+    (identical at k = 1).  cf <= 0 means no capacity limit (dropless).
+    """
+    if capacity_factor <= 0:
+        return None
+    return int(math.ceil(float(capacity_factor) * T * k / E))
+
+
+def assign_slots(idx: np.ndarray, E: int, C: Optional[int]):
+    """Capacity enforcement with position-order dropping.
+
+    "Capacity and dropped tokens": an expert's slots are filled in position
+    order and the assignments beyond its capacity are dropped.  The rank of
+    assignment (t, j) is the number of earlier assignments to the same expert
+    in token order (a token holds each expert at most once).  Kept iff
+    rank < C.  The kept assignments of expert e occupy rows
+    offsets[e] .. offsets[e+1]-1 of the expert-sorted dispatch buffer, in token
+    order; dest_row is that row, or -1 when dropped.
+    """
+    T, k = idx.shape
+    flat = idx.reshape(-1)
+    rank = np.zeros(flat.shape, np.int64)
+    counts = np.zeros(E, np.int64)
+    for e in range(E):
+        hit = flat == e
+        n = int(hit.sum())
+        rank[hit] = np.arange(n)
+        counts[e] = n
+    kept = np.ones(flat.shape, bool) if C is None else rank < C
+    kept_counts = counts if C is None else np.minimum(counts, C)
+    offsets = np.concatenate([[0], np.cumsum(kept_counts)]).astype(np.int64)
+    dest = np.where(kept, offsets[flat] + rank, -1)
+    return {
+        "counts": counts,
+        "kept_counts": kept_counts,
+        "offsets": offsets,
+        "rank": rank.reshape(T, k),
+        "kept": kept.reshape(T, k),
+        "dest_row": dest.reshape(T, k),
+        "dropped": int((~kept).sum()),
+    }
+
+
+def expert_ffn(xr: np.ndarray, W1e, W3e, W2e, act: int) -> np.ndarray:
+    """One expert on a batch of rows.
+
+    SWIGLU ("Implementation"): w2(silu(w1 x) * w3 x), silu(u) = u / (1 + e^-u).
+    RELU: w2(relu(w1 x)).  Weights in nn.Linear (out, in) layout:
+    W1e/W3e [d_ff][d], W2e [d][d_ff].  float64.
+    """
+    a = xr @ np.asarray(W1e, np.float64).T
+    if act == ACT_RELU:
+        hdn = np.maximum(a, 0.0)
+    else:
+        b = xr @ np.asarray(W3e, np.float64).T
+        hdn = a / (1.0 + np.exp(-a)) * b
+    return hdn @ np.asarray(W2e, np.float64).T
+
+
+def aux_and_z(p: np.ndarray, lse: np.ndarray, idx: np.ndarray, E: int):
+    """Unscaled load-balancing loss and router z-loss ("The load-balancing loss").
+
+    aux = E * sum_i f_i P_i, f_i = share of the T tokens whose first choice is
+    i (counted before capacity), P_i = mean full-softmax probability of i.
+    z = mean over tokens of lse^2.  The caller applies alpha = 0.01 and 1e-3.
+    T = 0 gives aux = z = 0.
+    """
+    T = p.shape[0]
+    if T == 0:
+        return 0.0, 0.0
+    f = np.bincount(idx[:, 0], minlength=E).astype(np.float64) / T
+    P = p.mean(axis=0)
+    return float(E * np.sum(f * P)), float(np.mean(lse ** 2))
+
+
+def moe_forward(x, W_r, b_r, W1, W3, W2, *, k: int, gate_mode: int, act: int,
+                capacity_factor: float, rows: Optional[Sequence[int]] = None,
+                logits: Optional[np.ndarray] = None) -> dict:
+    """The whole layer: routing for every token, y for every token or for ``rows``.
+
+    x: [T][d]; W_r: [E][d]; b_r: [E] or None; W1, W3: [E][d_ff][d] (W3 None for
+    ReLU); W2: [E][d][d_ff]; any float dtype (bf16 values come in widened).
+    ``logits``: route from these fp32 logits instead of computing W_r x.
+    ``rows``: compute y only for these tokens (routing, capacity and losses are
+    always global; y_t depends on x_t and the global routing only).
+
+    y_t = sum over kept assignments (t, j), in slot order j, of
+    g_tj * E_{idx_tj}(x_t); a token with all assignments dropped gets y_t = 0.
+    """
+    x = np.asarray(x)
+    T = x.shape[0]
+    E = np.asarray(W_r).shape[0]
+    h32 = router_logits(x, W_r, b_r) if logits is None else np.asarray(logits, np.float32)
+    p, lse = softmax_lse(h32)
+    idx = top_k(h32, k)
+    g = gates(h32, p, idx, gate_mode)
+    C = expert_capacity(capacity_factor, T, k, E)
+    slots = assign_slots(idx, E, C)
+    aux, z = aux_and_z(p, lse, idx, E)
+
+    want = np.arange(T) if rows is None else np.asarray(rows, np.int64)
+    d = x.shape[1]
+    # contrib[i, j] = g_tj * E_{idx_tj}(x_t) for token t = want[i] (0 if dropped)
+    contrib = np.zeros((len(want), k, d), np.float64)
+    ew = idx[want]                      # [n][k] experts of the wanted tokens
+    kw = slots["kept"][want]            # [n][k] kept flags
+    for e in range(E):
+        ii, jj = np.nonzero((ew == e) & kw)
+        if ii.size == 0:
+            continue
+        ts = want[ii]
+        out = expert_ffn(np.asarray(x[ts], np.float64), W1[e],
+                         None if W3 is None else W3[e], W2[e], act)
+        contrib[ii, jj] = g[ts, jj][:, None] * out
+    y = np.zeros((len(want), d), np.float64)
+    for j in range(k):                  # slot order
+        y += contrib[:, j]
+    res = {"logits": h32, "p": p, "lse": lse, "idx": idx, "gate": g, "capacity": C,
+           "y": y, "rows": want, "aux": aux, "z": z}
+    res.update(slots)
+    return res

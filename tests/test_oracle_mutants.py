@@ -1,0 +1,132 @@
+"""Each plausible mistake planted in the oracle must fail at least one pin.
+
+The mutants live only here, on the CPU; they patch the oracle module for the
+duration of one check.  This shows the pins in test_oracle_pins.py would catch
+a dropped term, a wrong sign, a wrong index or tie rule, a transposed operand,
+an off-by-one capacity or a wrong slot priority.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import oracle.moe_oracle as M
+from tests import test_oracle_pins as P
+
+
+def _top_k_last_index_on_ties(h32, k):
+    h = np.asarray(h32, np.float64)[:, ::-1].copy()
+    E = h.shape[1]
+    idx = np.empty((h.shape[0], k), np.int64)
+    rows = np.arange(h.shape[0])
+    for j in range(k):
+        s = np.argmax(h, axis=1)
+        idx[:, j] = E - 1 - s
+        h[rows, s] = -np.inf
+    return idx
+
+
+def _gates_not_renormalised(h32, p, idx, gate_mode):
+    return p[np.arange(idx.shape[0])[:, None], idx]
+
+
+def _ffn_silu_sign(xr, W1e, W3e, W2e, act):
+    a = xr @ np.asarray(W1e, np.float64).T
+    hdn = np.maximum(a, 0) if act == M.ACT_RELU else a / (1 + np.exp(a)) * (xr @ np.asarray(W3e, np.float64).T)
+    return hdn @ np.asarray(W2e, np.float64).T
+
+
+def _ffn_w1_w3_swapped_roles(xr, W1e, W3e, W2e, act):
+    if act == M.ACT_RELU:
+        return _orig["expert_ffn"](xr, W1e, W3e, W2e, act)
+    a = xr @ np.asarray(W3e, np.float64).T
+    b = xr @ np.asarray(W1e, np.float64).T
+    return (a / (1 + np.exp(-a)) * b) @ np.asarray(W2e, np.float64).T
+
+
+def _aux_without_E(p, lse, idx, E):
+    aux, z = _orig["aux_and_z"](p, lse, idx, E)
+    return aux / E, z
+
+
+def _z_without_square(p, lse, idx, E):
+    aux, _ = _orig["aux_and_z"](p, lse, idx, E)
+    return aux, float(np.mean(lse)) if len(lse) else 0.0
+
+
+def _f_over_all_choices(p, lse, idx, E):
+    T = p.shape[0]
+    f = np.bincount(idx.reshape(-1), minlength=E) / (T * idx.shape[1])
+    return float(E * np.sum(f * p.mean(axis=0))), float(np.mean(lse ** 2))
+
+
+def _slots_off_by_one(idx, E, C):
+    return _orig["assign_slots"](idx, E, None if C is None else C + 1)
+
+
+def _slots_choice_major(idx, E, C):
+    T, k = idx.shape
+    s = _orig["assign_slots"](idx.T.copy(), E, C)  # scans choice j before token t
+    for key in ("rank", "kept", "dest_row"):
+        s[key] = s[key].T.copy()
+    return s
+
+
+def _logits_transposed_router(x, W_r, b_r=None):
+    W = np.asarray(W_r, np.float64)
+    h = np.asarray(x, np.float64) @ (W.T if W.shape[0] != W.shape[1] else W)
+    if b_r is not None:
+        h = h + b_r
+    return h.astype(np.float32)
+
+
+def _logits_dropped_bias(x, W_r, b_r=None):
+    return _orig["router_logits"](x, W_r, None)
+
+
+_orig = {n: getattr(M, n) for n in ("top_k", "gates", "expert_ffn", "aux_and_z", "assign_slots", "router_logits")}
+
+MUTANTS = {
+    "top_k ties to the higher index": ("top_k", _top_k_last_index_on_ties),
+    "renormalised gates left unnormalised": ("gates", _gates_not_renormalised),
+    "silu with the wrong sign": ("expert_ffn", _ffn_silu_sign),
+    "SwiGLU gate/value roles swapped": ("expert_ffn", _ffn_w1_w3_swapped_roles),
+    "aux without the factor E": ("aux_and_z", _aux_without_E),
+    "z-loss without the square": ("aux_and_z", _z_without_square),
+    "f over all k choices": ("aux_and_z", _f_over_all_choices),
+    "capacity off by one": ("assign_slots", _slots_off_by_one),
+    "slots by choice before token": ("assign_slots", _slots_choice_major),
+    "router weight transposed": ("router_logits", _logits_transposed_router),
+    "router bias dropped": ("router_logits", _logits_dropped_bias),
+}
+
+PINS = [
+    lambda: [P.test_top_k_matches_brute_force_with_ties(E) for E in (3, 5)],
+    P.test_top_k_signed_zero_is_a_tie,
+    P.test_renorm_gates_sum_to_one_and_equal_conditional_probabilities,
+    P.test_switch_gate_is_max_probability_below_one,
+    P.test_closed_form_golden_routing,
+    P.test_router_logits_match_linear_and_are_order_free_on_dyadic_inputs,
+    P.test_aux_is_one_under_uniform_routing,
+    P.test_aux_tends_to_E_when_collapsed,
+    P.test_z_loss_closed_form,
+    P.test_dropless_keeps_everything,
+    lambda: P.test_position_order_dropping_k1(3),
+    P.test_slot_priority_is_token_order_across_choices,
+    P.test_worked_example_reconstruction,
+    lambda: [P.test_single_expert_is_the_dense_ffn(a, g) for a in (0, 1) for g in (0, 1)],
+    lambda: [P.test_k_equals_E_is_the_dense_softmax_mixture(a) for a in (0, 1)],
+]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(M, attr, fn)
+    monkeypatch.setattr(oracle, attr, fn)
+    caught = 0
+    for pin in PINS:
+        try:
+            pin()
+        except (AssertionError, ValueError, IndexError):
+            caught += 1
+    assert caught >= 1, f"no pin fails for mutant: {name}"
