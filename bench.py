@@ -1,0 +1,438 @@
+"""Benchmark of the MoE layer forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one forward pass of the whole layer (router, scan, dispatch, two
+grouped GEMMs, combine, losses) over one batch of the workload's synthetic
+input, resident in HBM.  L2 is flushed (a 256 MiB write) between steps,
+outside the timed events.  Prints ONE JSON line on rank 0.
+
+N > 1 (torchrun): every rank runs an independent replica of the layer on its
+own batch (the layer has no cross-batch exchange), so scaling is weak; the
+time is the max over ranks of each rank's device-timed total.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s on 1 B200 and % of roofline (TFLOP/s or HBM GB/s)"
+DEFAULT_WORKLOAD = "switch_k1"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+STAGE_KERNEL = {"router": "router_kernel", "scan": "scan_kernel", "dispatch": "dispatch_kernel",
+                "gemm1": "grouped_gemm_kernel", "gemm2": "grouped_gemm_kernel", "combine": "combine_kernel"}
+# oracle tokens per CPU-baseline sample, per workload (bounded to ~10-30 s of CPU work)
+CPU_SAMPLE_TOKENS = {"switch_k1": 8192, "mixtral_prefill": 128, "mixtral_decode_t1": 1, "mixtral_decode_t16": 16,
+                     "mixtral_decode_t64": 64, "fine_grained": 2048, "tiny_fp32": 64}
+
+
+# ----------------------------------------------------------------------------- helpers (host only)
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def layer_work(w, kept_counts, hidden="bf16x2"):
+    """Algorithmic FLOPs and bytes of the layer and of each grouped GEMM launch.
+
+    Counts kept assignments only.  Bytes: weights of experts with >= 1 kept
+    row (read once), x read once, y written once, W_r; per GEMM also its own
+    input and output activations (the expert-sorted rows; the hidden
+    activation at 4 bytes per element when held as a hi + lo bf16 pair).
+    """
+    elt = 2 if w.dtype == 1 else 4
+    h_elt = 4 if (w.dtype == 1 and hidden == "bf16x2") else elt
+    S = int(sum(kept_counts))
+    active = sum(1 for c in kept_counts if c > 0)
+    nproj1 = 2 if w.act == 1 else 1
+    w1_bytes = active * nproj1 * w.d_ff * w.d * elt
+    w2_bytes = active * w.d * w.d_ff * elt
+    flops_router = 2.0 * w.T * w.E * w.d
+    flops1 = 2.0 * S * w.d * w.d_ff * nproj1
+    flops2 = 2.0 * S * w.d_ff * w.d
+    gemm1_bytes = w1_bytes + S * w.d * elt + S * w.d_ff * h_elt
+    out2 = S * w.d * (elt if w.k == 1 else 4)
+    gemm2_bytes = w2_bytes + S * w.d_ff * h_elt + out2
+    layer_bytes = w1_bytes + w2_bytes + 2 * w.T * w.d * elt + w.E * w.d * 4
+    return {"S": S, "active_experts": active, "flops_layer": flops_router + flops1 + flops2,
+            "bytes_layer": layer_bytes, "gemm1": {"flops": flops1, "bytes": gemm1_bytes},
+            "gemm2": {"flops": flops2, "bytes": gemm2_bytes}}
+
+
+def kernel_roofline(flops, nbytes, seconds, peaks):
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        a = flops / seconds / 1e12
+        return {"bound": "tensor", "achieved": round(a, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(a / peaks["bf16_tflops"], 4)}
+    a = nbytes / seconds / 1e9
+    return {"bound": "hbm", "achieved": round(a, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(a / peaks["hbm_gbs"], 4)}
+
+
+def source_sha(*rel):
+    h = hashlib.sha256()
+    for r in rel:
+        with open(os.path.join(ROOT, r), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(stage, workload):
+    """dram bytes per launch from the committed ncu summary, if the kernel is unchanged since."""
+    p = os.path.join(ROOT, "profiles", f"{stage}_{workload}.txt")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    src = vals.get("source_files", "").split()
+    if not src or "dram_bytes_per_launch" not in vals:
+        return None
+    if source_sha(*src) != vals.get("source_sha256"):
+        return None
+    return float(vals["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled in the background."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 8:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        win = [p for (t, p) in self.samples if t0 - 0.1 <= t <= t1 + 0.1]
+        if not win and self.samples:
+            mid = 0.5 * (t0 + t1)
+            win = [min(self.samples, key=lambda s: abs(s[0] - mid))[1]]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in win for i in range(4) if p[4 + i].lower().startswith("active")})
+
+        def num(s):
+            try:
+                return float(s)
+            except ValueError:
+                return None
+        sm = [num(p[1]) for p in win if num(p[1]) is not None]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(win[0][2]),
+                "power_w_max": max((num(p[3]) or 0.0) for p in win), "reasons": reasons, "samples": len(win)}
+
+
+def combine_ranks(seconds_local, tokens_local, dist_mod=None):
+    """(max over ranks of the timed seconds, sum over ranks of the tokens)."""
+    if dist_mod is None or not dist_mod.is_initialized():
+        return seconds_local, tokens_local
+    import torch
+    dev = "cuda" if dist_mod.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([seconds_local], dtype=torch.float64, device=dev)
+    n = torch.tensor([float(tokens_local)], dtype=torch.float64, device=dev)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    dist_mod.all_reduce(n, op=dist_mod.ReduceOp.SUM)
+    return float(t.item()), float(n.item())
+
+
+def rank_seed(base_seed, rank):
+    """Each replica draws its own batch of tokens; weights are shared."""
+    return base_seed + 7919 * rank
+
+
+def config_of(w, n_gpus):
+    return {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "k": w.k, "d_ff": w.d_ff,
+            "act": "swiglu" if w.act == 1 else "relu", "gate": "renorm" if w.gate == 1 else "switch",
+            "capacity_factor": w.capacity_factor, "tokens_per_gpu": w.T,
+            "parallelism": "replicas" if n_gpus > 1 else "single",
+            "l2": "flushed between steps (256 MiB write, outside the timed events)"}
+
+
+# ----------------------------------------------------------------------------- CPU (oracle) leg
+def cpu_oracle_run(w, inp, n_tokens):
+    """Time the oracle's forward on the first n_tokens tokens of the batch (full weights)."""
+    import numpy as np
+    import oracle
+
+    class Host:
+        def __init__(self, t):
+            self.t, self.c = t, {}
+
+        def __getitem__(self, e):
+            if e not in self.c:
+                self.c[e] = self.t[e].float().cpu().numpy()
+            return self.c[e]
+    x = inp["x"][:n_tokens].float().cpu().numpy()
+    W_r = inp["W_r"].float().cpu().numpy()
+    b_r = None if inp["b_r"] is None else inp["b_r"].float().cpu().numpy()
+    W1, W2 = Host(inp["W1"]), Host(inp["W2"])
+    W3 = None if inp["W3"] is None else Host(inp["W3"])
+    t0 = time.perf_counter()
+    oracle.moe_forward(x, W_r, b_r, W1, W3, W2, k=w.k, gate_mode=w.gate, act=w.act,
+                       capacity_factor=w.capacity_factor)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(w, inp):
+    n = min(w.T, CPU_SAMPLE_TOKENS.get(w.name, 256))
+    secs = cpu_oracle_run(w, inp, n)
+    return {"value": round(n / secs, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"oracle forward (float64 NumPy) on the first {n} of {w.T} tokens with the full weights; "
+                      f"{secs:.2f} s wall on the host"}
+
+
+# ----------------------------------------------------------------------------- GPU leg
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--hidden", choices=["bf16x2", "bf16"], default="bf16x2",
+                    help="how the expert hidden activation is held (bf16 layers)")
+    args = ap.parse_args()
+
+    import torch
+    import torch.distributed as dist
+    from sparse_mixture_experts_gating_b200 import MoELayer, launch_count, status
+    from sparse_mixture_experts_gating_b200.workloads import WORKLOADS, make_inputs, torch_dtype
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WORKLOADS[args.workload]
+    warmup = max(3, args.warmup)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return reference_arm(args, w, warmup)
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+
+    inp = make_inputs(w, device=dev)
+    if rank > 0:
+        inp["x"] = make_inputs(w.with_(seed=rank_seed(w.seed, rank)), device=dev, weights=False)["x"]
+    layer = MoELayer(w.E, w.k, w.d, w.d_ff, act=w.act, gate_mode=w.gate, capacity_factor=w.capacity_factor,
+                     dtype=torch_dtype(w.dtype), hidden=args.hidden)
+    ws = layer.workspace(w.T, dev)
+    y = torch.empty((w.T, w.d), dtype=inp["x"].dtype, device=dev)
+    stats = (torch.empty(w.E, dtype=torch.int32, device=dev), torch.empty(1, dtype=torch.int32, device=dev),
+             torch.empty(1, dtype=torch.float32, device=dev), torch.empty(1, dtype=torch.float32, device=dev))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    args_fw = (inp["x"], inp["W_r"], inp["b_r"], inp["W1"], inp["W3"], inp["W2"])
+
+    def step(events=None, x=None):
+        a = args_fw if x is None else (x,) + args_fw[1:]
+        layer(*a, out=y, stats=stats, workspace=ws, events=events)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    status()
+
+    K = args.steps
+    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ev_stage = [[torch.cuda.Event(enable_timing=True) for _ in range(12)] for _ in range(K)]
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    sampler = ClockSampler(vis.split(",")[local].strip() if vis else str(local))
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n_launch0 = launch_count()
+    wall0 = time.time()
+    for i in range(K):
+        flush.zero_()
+        ev_step[i][0].record(stream)
+        step(events=ev_stage[i])
+        ev_step[i][1].record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    n_launch = launch_count() - n_launch0
+    time.sleep(0.15)
+    sampler.stop()
+    status()
+
+    step_ms = [a.elapsed_time(b) for a, b in ev_step]
+    total_s = sum(step_ms) / 1e3
+    stage_names = ["router", "scan", "dispatch", "gemm1", "gemm2", "combine"]
+    stage_ms = {}
+    for s_i, name in enumerate(stage_names):
+        if name == "combine" and w.dtype == 1 and w.k == 1:
+            continue
+        stage_ms[name] = statistics.mean(ev[2 * s_i].elapsed_time(ev[2 * s_i + 1]) for ev in ev_stage)
+
+    # end to end through the public API: pinned host x in, y and statistics out, every step
+    x_host = inp["x"].cpu().pin_memory()
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    st_host = [torch.empty(s.shape, dtype=s.dtype).pin_memory() for s in stats]
+    x_dev = torch.empty_like(inp["x"])
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(warmup + K):
+        flush.zero_()
+        if i >= warmup:
+            e2e_ev[i - warmup][0].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x=x_dev)
+        y_host.copy_(y, non_blocking=True)
+        for h, s in zip(st_host, stats):
+            h.copy_(s, non_blocking=True)
+        if i >= warmup:
+            e2e_ev[i - warmup][1].record(stream)
+    torch.cuda.synchronize()
+    status()
+    e2e_s = sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3
+
+    t_max, tokens = combine_ranks(total_s, w.T * K, dist if world > 1 else None)
+    e2e_max, _ = combine_ranks(e2e_s, w.T * K, dist if world > 1 else None)
+
+    counts = stats[0].cpu().tolist()
+    cap = layer.capacity(w.T)
+    kept = [c if cap is None else min(c, cap) for c in counts]
+    work = layer_work(w, kept, args.hidden)
+    peaks, peak_src = load_peaks()
+    dom = max(("gemm1", "gemm2"), key=lambda s: stage_ms[s])
+    roof = kernel_roofline(work[dom]["flops"], work[dom]["bytes"], stage_ms[dom] / 1e3, peaks)
+    roof["kernel"] = f"{STAGE_KERNEL[dom]} ({dom})"
+    roof["peak_source"] = f"{peak_src} ({'bf16_tflops' if roof['bound'] == 'tensor' else 'hbm_gbs'}, burst)"
+    tr = profiled_traffic(dom, w.name)
+    roof["traffic"] = tr
+    ms_step = total_s / K * 1e3
+    floor_s = max(work["flops_layer"] / (peaks["bf16_tflops"] * 1e12), work["bytes_layer"] / (peaks["hbm_gbs"] * 1e9))
+    clocks = sampler.summary(wall0, wall1)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": round(tokens / t_max, 1),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": warmup,
+            "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == 1 else "f32",
+            "data": "synthetic (seeded; shapes and distributions of the workload, random-init weights)",
+            "config": dict(config_of(w, world), hidden=args.hidden),
+            "roofline": roof,
+            "layer_roofline": {"floor_ms": round(floor_s * 1e3, 5), "frac": round(floor_s / (ms_step / 1e3), 4),
+                               "flops": work["flops_layer"], "bytes": work["bytes_layer"],
+                               "kept_assignments": work["S"], "active_experts": work["active_experts"]},
+            "kernels_ms": {k: round(v, 5) for k, v in stage_ms.items()},
+            "e2e": {"value": round(tokens / e2e_max, 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+                    "d2h_bytes_per_step": y_host.numel() * y_host.element_size()
+                    + sum(h.numel() * h.element_size() for h in st_host)},
+            "gpu_launches": int(n_launch),
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, inp)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def reference_arm(args, w, warmup):
+    """The oracle timed on the host cores (rank 0 only): the reference arm of this benchmark."""
+    import torch
+    from sparse_mixture_experts_gating_b200.workloads import make_inputs
+
+    n = min(w.T, max(1, CPU_SAMPLE_TOKENS.get(w.name, 256) // 4))
+    inp = make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
+    for _ in range(warmup):
+        cpu_oracle_run(w, inp, n)
+    secs = [cpu_oracle_run(w, inp, n) for _ in range(args.steps)]
+    total = sum(secs)
+    value = n * args.steps / total
+    cores = blas_threads()
+    line = {
+        "metric": METRIC, "impl": "reference", "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "config": config_of(w, 1),
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: oracle forward (float64 NumPy) on the first {n} of {w.T} tokens"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,201 @@
+/*
+ * moe.h - C ABI of the sparse Mixture-of-Experts layer forward pass (sm_100a).
+ *
+ * The layer is the one defined on the page "Mixture of experts"
+ * (rayaq.ca/ml-models/mixture-of-experts), sections "Replacing the
+ * feed-forward block", "Top-k gating", "The load-balancing loss",
+ * "Capacity and dropped tokens" and "Implementation":
+ *
+ *   h = W_r x (+ b)            router logits, fp32
+ *   p = softmax(h)             full softmax over the E experts
+ *   TopK(h)                    k largest logits, largest first, ties -> lower index
+ *   g                          SWITCH: g_j = p[idx_j]; RENORM: softmax over the k chosen logits
+ *   capacity                   C = ceil(capacity_factor * T * k / E); slots filled in
+ *                              token order; overflow assignments dropped (contribute 0)
+ *   y_t = sum_j kept g_tj * E_{idx_tj}(x_t)   summed in slot order j
+ *   E_e(x) = W2_e relu(W1_e x)            (ReLU experts)
+ *   E_e(x) = W2_e (silu(W1_e x) * W3_e x)  (SwiGLU experts)
+ *   aux = E * sum_i f_i P_i    f_i: share of first choices (before capacity),
+ *                              P_i: mean of p_i over the T tokens (unscaled: the
+ *                              caller multiplies by alpha = 0.01)
+ *   z   = mean_t (log sum_j exp h_tj)^2   (unscaled: the caller multiplies by 1e-3)
+ *
+ * Conventions for every entry point:
+ *   - Tensor arguments are DEVICE pointers owned by the caller, row-major,
+ *     16-byte aligned, and not aliased with one another.
+ *   - bf16 layers: x, W1, W3, W2 and y are bf16; W_r and b_r are fp32.
+ *     fp32 layers: everything is fp32.
+ *   - Weights use the nn.Linear (out, in) layout: W_r [E][d], W1 and W3
+ *     [E][d_ff][d], W2 [E][d][d_ff].
+ *   - Every call is asynchronous on the given CUDA stream (a cudaStream_t
+ *     passed as void*; NULL = the legacy default stream).  moe_forward never
+ *     synchronises and never allocates device memory.
+ *   - Errors detectable on the host are returned before any launch and leave
+ *     the outputs untouched; a message is kept for moe_last_error().
+ *     Errors raised on the device (a bounded wait that ran out) are sticky
+ *     per device and reported by moe_status().
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_layer* moe_handle;
+
+enum { MOE_ACT_RELU = 0, MOE_ACT_SWIGLU = 1 };
+enum { MOE_GATE_SWITCH = 0, MOE_GATE_RENORM = 1 };
+enum { MOE_F32 = 0, MOE_BF16 = 1 };
+enum { MOE_HIDDEN_BF16X2 = 0, MOE_HIDDEN_BF16 = 1 };
+enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* bad shape, mode, null pointer or too small workspace */
+  MOE_ERR_UNSUPPORTED = 2, /* valid layer this build cannot run (alignment, limits) */
+  MOE_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  MOE_ERR_TIMEOUT = 4      /* a device-side bounded wait ran out (kernel gave up) */
+};
+
+/* Kernel stages of one forward call, in launch order (see moe_debug.events). */
+enum {
+  MOE_STAGE_ROUTER = 0,   /* logits, softmax, top-k, gates, per-block counts      */
+  MOE_STAGE_SCAN = 1,     /* per-expert scan, capacity, offsets, losses            */
+  MOE_STAGE_DISPATCH = 2, /* slot ranks, drop mask, permute of x into expert order */
+  MOE_STAGE_GEMM1 = 3,    /* grouped x W1^T (|| x W3^T) with ReLU / SwiGLU         */
+  MOE_STAGE_GEMM2 = 4,    /* grouped h W2^T with the gate                          */
+  MOE_STAGE_COMBINE = 5,  /* slot-order sum per token                              */
+  MOE_NUM_STAGES = 6
+};
+
+/*
+ * Optional debug / profiling hooks for moe_forward.  Every pointer may be
+ * NULL.  Output arrays are device memory of the stated shape:
+ *   logits_in   [T][E] fp32, read : route from these logits instead of W_r x + b
+ *                                   (the "identical logits" parity mode)
+ *   logits_out  [T][E] fp32, write: the fp32 router logits used for routing
+ *   lse_out     [T]    fp32, write: log-sum-exp of each token's logits
+ *   topk_idx    [T][k] int32      : chosen experts, largest logit first
+ *   topk_gate   [T][k] fp32       : gate of each choice
+ *   dest_row    [T][k] int32      : row of (t, j) in the expert-sorted buffer, -1 if dropped
+ *   drop_mask   [T][k] uint8      : 1 if assignment (t, j) was dropped
+ *   expert_offsets [E+1] int32    : first row of each expert in the sorted buffer
+ *   y_f32       [T][d] fp32, write: the output in fp32, before its final rounding to
+ *                                   the layer dtype (y is its round-to-nearest-even image)
+ *   events[2*s], events[2*s+1]    : cudaEvent_t recorded on the stream right before
+ *                                   and after the launches of stage s (MOE_STAGE_*)
+ */
+typedef struct moe_debug {
+  const float* logits_in;
+  float* logits_out;
+  float* lse_out;
+  int32_t* topk_idx;
+  float* topk_gate;
+  int32_t* dest_row;
+  uint8_t* drop_mask;
+  int32_t* expert_offsets;
+  float* y_f32;
+  void* events[2 * MOE_NUM_STAGES];
+} moe_debug;
+
+/*
+ * Create a layer description (host memory only; no device work).
+ *   num_experts E in [1, 256]; 1 <= k <= E and k <= 8; d >= 1; d_ff >= 1;
+ *   act MOE_ACT_*; gate_mode MOE_GATE_*; dtype MOE_F32 or MOE_BF16;
+ *   capacity_factor <= 0 means dropless (no capacity limit).
+ * bf16 layers need d and d_ff to be multiples of 8 (16-byte rows for the
+ * tensor-memory-accelerator loads): otherwise MOE_ERR_UNSUPPORTED.
+ * Returns MOE_OK and *out, or MOE_ERR_INVALID_ARG (out untouched).
+ */
+MOE_API int moe_create(int num_experts, int k, int d, int d_ff, int act, int gate_mode,
+               double capacity_factor, int dtype, moe_handle* out);
+
+/*
+ * bf16 layers: how the hidden activation between the two expert projections
+ * is held (no counterpart on the pages, which fix only the router at fp32):
+ *   MOE_HIDDEN_BF16X2 (default): as the sum of two bf16 numbers hi + lo
+ *     (about 16 significant bits); the second projection runs its tensor-core
+ *     MMAs on both planes, twice the tensor work of that projection.
+ *   MOE_HIDDEN_BF16: one bf16 number (8 significant bits, unit roundoff 2^-8).
+ * Changes moe_workspace_bytes().  fp32 layers ignore it.  Returns MOE_OK or
+ * MOE_ERR_INVALID_ARG.
+ */
+MOE_API int moe_set_hidden_precision(moe_handle h, int mode);
+
+/* Free a handle created by moe_create.  NULL is accepted. */
+MOE_API int moe_destroy(moe_handle h);
+
+/*
+ * Expert capacity for a batch of T tokens: ceil(capacity_factor * T * k / E)
+ * evaluated in double, or -1 for a dropless layer.  Host only.
+ */
+MOE_API int64_t moe_capacity(moe_handle h, int64_t T);
+
+/*
+ * Bytes of device workspace moe_forward needs for T tokens (0 on bad args).
+ * The workspace holds the routing tables and the expert-sorted activations;
+ * it must be 256-byte aligned and is fully rewritten by every call.
+ */
+MOE_API size_t moe_workspace_bytes(moe_handle h, int64_t T);
+
+/*
+ * One forward pass of the layer over T tokens (T >= 0).
+ *   x            [T][d]        layer input (bf16 or fp32)
+ *   W_r          [E][d]  fp32  router weight;   b_r [E] fp32 bias or NULL
+ *   W1           [E][d_ff][d]  first expert projection
+ *   W3           [E][d_ff][d]  SwiGLU value projection; must be NULL for ReLU
+ *   W2           [E][d][d_ff]  second expert projection
+ *   y            [T][d]        output (same dtype as x); 0 for fully dropped tokens
+ *   expert_counts[E]     int32 assignments routed to each expert, before capacity
+ *   dropped      [1]     int32 number of dropped (token, choice) assignments
+ *   aux_loss     [1]     fp32  E * sum_i f_i P_i (unscaled)
+ *   z_loss       [1]     fp32  mean_t lse_t^2 (unscaled)
+ *   workspace, workspace_bytes: device scratch of at least moe_workspace_bytes(h, T)
+ *   dbg          optional hooks (may be NULL)
+ *   stream       cudaStream_t as void*
+ * T = 0 writes zero counts, dropped = 0, aux = z = 0 and launches nothing else.
+ */
+MOE_API int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const float* b_r,
+                const void* W1, const void* W3, const void* W2, void* y,
+                int32_t* expert_counts, int32_t* dropped, float* aux_loss, float* z_loss,
+                void* workspace, size_t workspace_bytes, const moe_debug* dbg, void* stream);
+
+/*
+ * Synchronise `stream` and report the device error word of the current device:
+ * MOE_OK, MOE_ERR_TIMEOUT (a kernel's bounded wait ran out and it returned
+ * early; outputs of that call are undefined) or MOE_ERR_CUDA.  The error
+ * word stays set until moe_clear_status().
+ */
+MOE_API int moe_status(void* stream);
+
+/* Clear the device error word of the current device (synchronous). */
+MOE_API int moe_clear_status(void);
+
+/* Message of the last host-side error of the calling thread ("" if none). */
+MOE_API const char* moe_last_error(void);
+
+/* Kernels launched by this library in the calling process so far. */
+MOE_API uint64_t moe_launch_count(void);
+
+/*
+ * Self-test of the device-side failure path (no counterpart on the pages):
+ * launches one thread that waits on a device flag nothing ever sets, with the
+ * same bounded wait the pipelined kernels use, limited to `limit_ns`
+ * nanoseconds (clamped to [1e3, 2e9]).  When the wait runs out the kernel
+ * records MOE_ERR_TIMEOUT in the device error word and returns, so a
+ * following moe_status() reports MOE_ERR_TIMEOUT and the context stays usable.
+ */
+MOE_API int moe_selftest_timeout(int64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

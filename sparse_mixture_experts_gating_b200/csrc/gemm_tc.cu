@@ -1,0 +1,486 @@
+// Persistent grouped GEMM on the 5th-generation tensor cores (tcgen05 + TMEM),
+// fed by TMA, for the expert FFNs of the MoE layer ("Mixture of experts",
+// rayaq.ca, section "Implementation": each expert runs once on the sub-batch of
+// its tokens; production code sorts tokens by expert and runs one grouped
+// matrix multiply).
+//
+// C_e[m][n] = sum_k A[offsets[e] + m][k] * B_e[n][k] for every expert e, where
+// A holds the expert-sorted rows (ragged groups, offsets on the device) and
+// B_e is the expert's nn.Linear weight [N][K].  Tiles are 128 rows x 256 MMA
+// columns; the tile list is expert-major, then n-tile, then m-tile, so tiles
+// sharing a weight slab run at the same time and the slab is read from HBM once.
+//
+// Warp roles (192 threads, one CTA per SM):
+//   warp 0       TMA producer: A box [128 x 64] + two B boxes [128 x 64] per stage
+//   warp 1       TMEM allocator; lane 0 issues tcgen05.mma (M=128, N=256, K=16)
+//   warps 2..5   epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane per
+//                row), activation or gate, masked stores
+// Pipelines: STAGES-deep smem ring (full/empty mbarriers) and two TMEM
+// accumulators of 256 columns (tmem_full/tmem_empty), so the epilogue of tile i
+// overlaps the MMAs of tile i+1.  Every wait is bounded; a wait that runs out
+// records MOE_ERR_TIMEOUT, raises the CTA's abort flag, drains its in-flight
+// copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = kTileM;               // rows per tile
+constexpr int BK = 64;                   // bf16 per 128-byte smem row
+constexpr int MMA_N = 256;               // columns per MMA / accumulator
+constexpr int MAX_STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;     // 16 KB
+constexpr int B_HALF = 128 * BK * 2;     // 16 KB per B box
+constexpr int NUM_THREADS = 192;
+
+// Pipeline geometry.  SPLIT: the A operand is held as two bf16 planes
+// (hi + lo, about 16 significant bits) and every k-block issues the MMAs of
+// both planes against the same B tile, so one stage holds two A boxes.
+template <bool SPLIT>
+struct Geo {
+  static constexpr int kA = SPLIT ? 2 : 1;
+  static constexpr int STAGES = SPLIT ? 3 : 4;
+  static constexpr int STAGE_BYTES = kA * A_BYTES + 2 * B_HALF;
+};
+constexpr uint32_t TMEM_COLS = 2 * MMA_N;
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, MMA_N);
+constexpr int MAX_E = 256;
+
+struct Params {
+  int E, N, K, n_tiles, bn, num_kb;
+  void* out;
+  void* out_lo;     // SwiGLU/ReLU epilogue with a split hidden activation: the lo plane
+  float* out_f32;
+  const int32_t* offsets;
+  const int32_t* mprefix;
+  const float* row_gate;
+  const int32_t* row_token;
+  unsigned int* err;
+  uint64_t limit_ns;
+};
+
+struct Ctl {
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_slot;
+  volatile int abort;
+  int mprefix[MAX_E + 1];
+  int offsets[MAX_E + 1];
+};
+
+template <bool SPLIT>
+constexpr size_t smem_bytes() {
+  return Geo<SPLIT>::STAGES * Geo<SPLIT>::STAGE_BYTES + sizeof(Ctl) + 1024;
+}
+
+// Tile L -> (expert, m-tile, n-tile); tiles are expert-major, then n, then m.
+__device__ __forceinline__ void decode_tile(int L, const Ctl* c, int E, int n_tiles, int& e, int& mt, int& nt) {
+  int lo = 0, hi = E;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (c->mprefix[mid] * n_tiles <= L) lo = mid; else hi = mid;
+  }
+  e = lo;
+  const int local = L - c->mprefix[e] * n_tiles;
+  const int mtiles = c->mprefix[e + 1] - c->mprefix[e];
+  nt = local / mtiles;
+  mt = local - nt * mtiles;
+}
+
+__device__ __forceinline__ bool wait_or_abort(Ctl* c, uint64_t* bar, uint32_t parity, const Params& p) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (c->abort) return false;
+    if (globaltimer_ns() - t0 > p.limit_ns) {
+      record_error(p.err, DEV_ERR_TIMEOUT);
+      c->abort = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ float silu_mul(float a, float b) { return a / (1.f + __expf(-a)) * b; }
+
+// bf16 pair (hi, lo) with hi = RNE(v) and lo = RNE(v - hi): hi + lo carries
+// about 16 significant bits of v.
+__device__ __forceinline__ void split_bf16(float v0, float v1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+  const float2 hf = __bfloat1622float2(h);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = pack_bf16x2(v0 - hf.x, v1 - hf.y);
+}
+
+// EPI: epilogue (internal.h GemmEpi).  SPLIT: for the first projection the
+// epilogue writes the hidden activation as hi/lo planes; for the second the
+// A operand is read as hi (tmA) + lo (tmA2) planes.
+template <int EPI, bool SPLIT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+                        const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                        const Params p) {
+  constexpr bool A_SPLIT = SPLIT && (EPI == EPI_GATE_F32 || EPI == EPI_GATE_SCATTER_BF16);
+  constexpr bool OUT_SPLIT = SPLIT && (EPI == EPI_RELU_BF16 || EPI == EPI_SWIGLU_BF16);
+  constexpr int STAGES = Geo<A_SPLIT>::STAGES;
+  constexpr int STAGE_BYTES = Geo<A_SPLIT>::STAGE_BYTES;
+  constexpr int B_OFF = Geo<A_SPLIT>::kA * A_BYTES;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* stages = smem_raw + pad;
+  Ctl* ctl = reinterpret_cast<Ctl*>(stages + STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&ctl->tfull[a], 1); mbar_init(&ctl->tempty[a], 128); }
+    mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tmA);
+    if (A_SPLIT) tma_prefetch_desc(&tmA2);
+    tma_prefetch_desc(&tmB0);
+    tma_prefetch_desc(&tmB1);
+  }
+  for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) {
+    ctl->mprefix[i] = p.mprefix[i];
+    ctl->offsets[i] = p.offsets[i];
+  }
+  if (warp == 1) tmem_alloc(&ctl->tmem_slot, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_slot;
+  const int total = ctl->mprefix[p.E] * p.n_tiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_phase[STAGES];
+      bool issued[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) { issued[s] = false; issued_phase[s] = 0; }
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        int e, mt, nt;
+        decode_tile(L, ctl, p.E, p.n_tiles, e, mt, nt);
+        const int row0 = ctl->offsets[e] + mt * BM;
+        const int brow = e * p.N + nt * p.bn;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!wait_or_abort(ctl, &ctl->empty[stage], phase ^ 1u, p)) { ok = false; break; }
+          uint8_t* sa = stages + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
+          tma_load_2d(sa, &tmA, &ctl->full[stage], kb * BK, row0);
+          if (A_SPLIT) tma_load_2d(sa + A_BYTES, &tmA2, &ctl->full[stage], kb * BK, row0);
+          if (EPI == EPI_SWIGLU_BF16) {
+            tma_load_2d(sa + B_OFF, &tmB0, &ctl->full[stage], kb * BK, brow);
+            tma_load_2d(sa + B_OFF + B_HALF, &tmB1, &ctl->full[stage], kb * BK, brow);
+          } else {
+            tma_load_2d(sa + B_OFF, &tmB0, &ctl->full[stage], kb * BK, brow);
+            tma_load_2d(sa + B_OFF + B_HALF, &tmB0, &ctl->full[stage], kb * BK, brow + 128);
+          }
+          issued[stage] = true;
+          issued_phase[stage] = phase;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Drain: every issued copy must have landed before the CTA may exit.
+      for (int s = 0; s < STAGES; ++s)
+        if (issued[s]) mbar_wait(&ctl->full[s], issued_phase[s], p.limit_ns);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        if (!wait_or_abort(ctl, &ctl->tempty[acc], acc_phase ^ 1u, p)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * MMA_N);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!wait_or_abort(ctl, &ctl->full[stage], phase, p)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stages + stage * STAGE_BYTES);
+          const uint32_t sb = sa + B_OFF;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_bf16(d_tmem, sdesc_k_sw128(sa + k * 32), sdesc_k_sw128(sb + k * 32), IDESC,
+                      (kb | k) != 0 ? 1u : 0u);
+          if (A_SPLIT) {
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)
+              umma_bf16(d_tmem, sdesc_k_sw128(sa + A_BYTES + k * 32), sdesc_k_sw128(sb + k * 32), IDESC, 1u);
+          }
+          umma_commit(&ctl->empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&ctl->tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      // Drain: all MMAs of this CTA complete before TMEM is freed.
+      umma_commit(&ctl->drain);
+      mbar_wait(&ctl->drain, 0, p.limit_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int r_in_tile = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x) {
+      int e, mt, nt;
+      decode_tile(L, ctl, p.E, p.n_tiles, e, mt, nt);
+      const bool ok = __all_sync(0xffffffffu, wait_or_abort(ctl, &ctl->tfull[acc], acc_phase, p));
+      if (!ok) break;  // warp-uniform: tcgen05.ld below is .sync.aligned
+      tc_fence_after();
+      const int m_local = mt * BM + r_in_tile;
+      const bool vrow = m_local < ctl->offsets[e + 1] - ctl->offsets[e];
+      const int64_t row = ctl->offsets[e] + m_local;
+      const int n0 = nt * p.bn;
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * MMA_N);
+
+      if (EPI == EPI_SWIGLU_BF16) {
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.N;
+        __nv_bfloat16* out_lo = OUT_SPLIT ? static_cast<__nv_bfloat16*>(p.out_lo) + row * p.N : nullptr;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t ra[32], rb[32];
+          tmem_ld32(tb + c * 32, ra);
+          tmem_ld32(tb + 128 + c * 32, rb);
+          tmem_ld_wait();
+          const int col = n0 + c * 32;
+          if (vrow) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (col + v * 8 < p.N) {
+                uint4 pk, pl;
+                uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
+                uint32_t* wl = reinterpret_cast<uint32_t*>(&pl);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const int j = v * 8 + 2 * i;
+                  const float h0 = silu_mul(__uint_as_float(ra[j]), __uint_as_float(rb[j]));
+                  const float h1 = silu_mul(__uint_as_float(ra[j + 1]), __uint_as_float(rb[j + 1]));
+                  if (OUT_SPLIT) split_bf16(h0, h1, w[i], wl[i]);
+                  else w[i] = pack_bf16x2(h0, h1);
+                }
+                *reinterpret_cast<uint4*>(out + col + v * 8) = pk;
+                if (OUT_SPLIT) *reinterpret_cast<uint4*>(out_lo + col + v * 8) = pl;
+              }
+            }
+          }
+        }
+      } else if (EPI == EPI_RELU_BF16) {
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.N;
+        __nv_bfloat16* out_lo = OUT_SPLIT ? static_cast<__nv_bfloat16*>(p.out_lo) + row * p.N : nullptr;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t ra[32];
+          tmem_ld32(tb + c * 32, ra);
+          tmem_ld_wait();
+          const int col = n0 + c * 32;
+          if (vrow) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (col + v * 8 < p.N) {
+                uint4 pk, pl;
+                uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
+                uint32_t* wl = reinterpret_cast<uint32_t*>(&pl);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const int j = v * 8 + 2 * i;
+                  const float h0 = fmaxf(__uint_as_float(ra[j]), 0.f);
+                  const float h1 = fmaxf(__uint_as_float(ra[j + 1]), 0.f);
+                  if (OUT_SPLIT) split_bf16(h0, h1, w[i], wl[i]);
+                  else w[i] = pack_bf16x2(h0, h1);
+                }
+                *reinterpret_cast<uint4*>(out + col + v * 8) = pk;
+                if (OUT_SPLIT) *reinterpret_cast<uint4*>(out_lo + col + v * 8) = pl;
+              }
+            }
+          }
+        }
+      } else {
+        const float g = vrow ? p.row_gate[row] : 0.f;
+        if (EPI == EPI_GATE_F32) {
+          float* out = static_cast<float*>(p.out) + row * p.N;
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t ra[32];
+            tmem_ld32(tb + c * 32, ra);
+            tmem_ld_wait();
+            const int col = n0 + c * 32;
+            if (vrow) {
+#pragma unroll
+              for (int v = 0; v < 8; ++v) {
+                if (col + v * 4 < p.N) {
+                  float4 o;
+                  o.x = __uint_as_float(ra[v * 4 + 0]) * g;
+                  o.y = __uint_as_float(ra[v * 4 + 1]) * g;
+                  o.z = __uint_as_float(ra[v * 4 + 2]) * g;
+                  o.w = __uint_as_float(ra[v * 4 + 3]) * g;
+                  *reinterpret_cast<float4*>(out + col + v * 4) = o;
+                }
+              }
+            }
+          }
+        } else {  // EPI_GATE_SCATTER_BF16: k == 1, write y[token] directly
+          const int64_t tok = vrow ? p.row_token[row] : 0;
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + tok * p.N;
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t ra[32];
+            tmem_ld32(tb + c * 32, ra);
+            tmem_ld_wait();
+            const int col = n0 + c * 32;
+            if (vrow) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                if (col + v * 8 < p.N) {
+                  uint4 pk;
+                  uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) {
+                    const int j = v * 8 + 2 * i;
+                    w[i] = pack_bf16x2(__uint_as_float(ra[j]) * g, __uint_as_float(ra[j + 1]) * g);
+                  }
+                  *reinterpret_cast<uint4*>(out + col + v * 8) = pk;
+                  if (p.out_f32 != nullptr) {
+                    float* of = p.out_f32 + tok * p.N + col + v * 8;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) of[i] = __uint_as_float(ra[v * 8 + i]) * g;
+                  }
+                }
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&ctl->tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host: tensor maps through the driver entry point (no libcuda link needed).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// Row-major bf16 matrix [rows][cols] -> map with box [128 rows][64 cols], 128B swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI, bool SPLIT>
+cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b0, const CUtensorMap& b1,
+                     const Params& p, int num_sms, cudaStream_t s) {
+  constexpr bool A_SPLIT = SPLIT && (EPI == EPI_GATE_F32 || EPI == EPI_GATE_SCATTER_BF16);
+  constexpr size_t bytes = smem_bytes<A_SPLIT>();
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(bytes));
+  if (e != cudaSuccess) return e;
+  grouped_gemm_kernel<EPI, SPLIT><<<num_sms, NUM_THREADS, bytes, s>>>(a, a2, b0, b1, p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t s, const char** why) {
+  *why = nullptr;
+  if (g.E > MAX_E) { *why = "grouped GEMM supports at most 256 experts"; return cudaErrorInvalidValue; }
+  const bool a_split = g.split && g.A2 != nullptr;
+  CUtensorMap ma, ma2, mb0, mb1;
+  if (!make_map(&ma, g.A, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K)) ||
+      !make_map(&ma2, a_split ? g.A2 : g.A, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K)) ||
+      !make_map(&mb0, g.B0, static_cast<uint64_t>(g.E) * g.N, static_cast<uint64_t>(g.K)) ||
+      !make_map(&mb1, g.epi == EPI_SWIGLU_BF16 ? g.B1 : g.B0, static_cast<uint64_t>(g.E) * g.N,
+                static_cast<uint64_t>(g.K))) {
+    *why = "cuTensorMapEncodeTiled failed (alignment or driver entry point)";
+    return cudaErrorInvalidValue;
+  }
+  Params p;
+  p.E = g.E;
+  p.N = g.N;
+  p.K = g.K;
+  p.bn = (g.epi == EPI_SWIGLU_BF16) ? 128 : 256;
+  p.n_tiles = (g.N + p.bn - 1) / p.bn;
+  p.num_kb = (g.K + BK - 1) / BK;
+  p.out = g.out;
+  p.out_lo = g.out2;
+  p.out_f32 = g.out_f32;
+  p.offsets = g.offsets;
+  p.mprefix = g.mprefix;
+  p.row_gate = g.row_gate;
+  p.row_token = g.row_token;
+  p.err = g.err;
+  p.limit_ns = kWaitLimitNs;
+  if (g.split) {
+    switch (g.epi) {
+      case EPI_RELU_BF16: return launch_t<EPI_RELU_BF16, true>(ma, ma2, mb0, mb1, p, num_sms, s);
+      case EPI_SWIGLU_BF16: return launch_t<EPI_SWIGLU_BF16, true>(ma, ma2, mb0, mb1, p, num_sms, s);
+      case EPI_GATE_F32: return launch_t<EPI_GATE_F32, true>(ma, ma2, mb0, mb1, p, num_sms, s);
+      case EPI_GATE_SCATTER_BF16: return launch_t<EPI_GATE_SCATTER_BF16, true>(ma, ma2, mb0, mb1, p, num_sms, s);
+    }
+  } else {
+    switch (g.epi) {
+      case EPI_RELU_BF16: return launch_t<EPI_RELU_BF16, false>(ma, ma2, mb0, mb1, p, num_sms, s);
+      case EPI_SWIGLU_BF16: return launch_t<EPI_SWIGLU_BF16, false>(ma, ma2, mb0, mb1, p, num_sms, s);
+      case EPI_GATE_F32: return launch_t<EPI_GATE_F32, false>(ma, ma2, mb0, mb1, p, num_sms, s);
+      case EPI_GATE_SCATTER_BF16: return launch_t<EPI_GATE_SCATTER_BF16, false>(ma, ma2, mb0, mb1, p, num_sms, s);
+    }
+  }
+  *why = "unknown epilogue";
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

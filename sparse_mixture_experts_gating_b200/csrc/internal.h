@@ -1,0 +1,91 @@
+// Host-side interface between the translation units of the MoE library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Tokens per router / dispatch block; the per-block partial counts use it.
+constexpr int kRouterTokens = 32;
+// Rows per tensor-core tile (M of one tcgen05.mma).
+constexpr int kTileM = 128;
+
+struct RoutingArgs {
+  int64_t T;
+  int E, k, d, gate_mode;
+  int64_t capacity;  // -1: dropless
+  int nblk;          // ceil(T / kRouterTokens)
+  int x_is_bf16;
+  const void* x;
+  const float* W_r;
+  const float* b_r;
+  const float* logits_in;
+  // workspace
+  int32_t* topk_idx;   // [T][k]
+  float* topk_gate;    // [T][k]
+  int32_t* dest_row;   // [T][k]
+  int32_t* part_hist;  // [E][nblk]
+  int32_t* part_cnt1;  // [E][nblk]
+  float* part_psum;    // [E][nblk]
+  float* part_lse2;    // [nblk]
+  int32_t* blockoff;   // [E][nblk]
+  int32_t* counts;     // [E]   (may alias the user output)
+  int32_t* offsets;    // [E+1]
+  int32_t* mprefix;    // [E+1] prefix of ceil(kept_e / kTileM)
+  int32_t* row_token;  // [S_max]
+  float* row_gate;     // [S_max]
+  void* Xp;            // [S_max][d]
+  // outputs
+  int32_t* dropped;
+  float* aux;
+  float* z;
+  // debug
+  float* logits_out;
+  float* lse_out;
+  uint8_t* drop_mask;
+  int32_t* offsets_out;
+  // k == 1 tensor-core path: the dispatch zeroes y rows of dropped tokens
+  void* y_zero_dropped;
+  float* yf_zero_dropped;  // and the fp32 debug copy of them
+};
+
+cudaError_t launch_router(const RoutingArgs& a, cudaStream_t s);
+cudaError_t launch_scan(const RoutingArgs& a, cudaStream_t s);
+cudaError_t launch_dispatch(const RoutingArgs& a, cudaStream_t s);
+cudaError_t launch_combine(int64_t T, int k, int d, int y_is_bf16, const int32_t* dest_row, const float* Yp,
+                           void* y, float* y_f32, cudaStream_t s);
+
+// Grouped GEMM epilogues
+enum GemmEpi { EPI_RELU_BF16 = 0, EPI_SWIGLU_BF16 = 1, EPI_GATE_F32 = 2, EPI_GATE_SCATTER_BF16 = 3 };
+
+struct GemmArgs {
+  int epi;
+  int E;
+  int N;  // output columns per expert
+  int K;  // reduction length
+  int64_t a_rows;  // rows of the A buffer (S_max)
+  const void* A;   // [a_rows][K]  (the hi plane when split)
+  const void* A2;  // [a_rows][K]  lo plane of a split A operand, else NULL
+  int split;       // first projection: write hi/lo planes; second: read them
+  const void* B0;  // [E][N][K]  (W1, or W2)
+  const void* B1;  // [E][N][K]  (W3 for SwiGLU, else unused)
+  void* out;       // Hp [S][N] | Yp [S][N] fp32 | y [T][N]
+  void* out2;      // lo plane of a split Hp, else NULL
+  float* out_f32;  // scatter epilogue only: optional fp32 copy of y
+  const int32_t* offsets;
+  const int32_t* mprefix;
+  const float* row_gate;
+  const int32_t* row_token;
+  unsigned int* err;
+};
+
+cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t s, const char** why);
+cudaError_t launch_gemm_simt(const GemmArgs& g, int64_t s_max, cudaStream_t s);
+
+cudaError_t launch_selftest_timeout(unsigned int* err, int64_t limit_ns, cudaStream_t s);
+
+void count_launch();
+
+}  // namespace moe

@@ -1,0 +1,370 @@
+// C ABI of the MoE layer forward pass: handle, validation, workspace layout and
+// the launch sequence router -> scan -> dispatch -> GEMM1 -> GEMM2 -> combine,
+// all on the caller's stream with no host synchronisation.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+#include <string>
+
+#include "moe.h"
+#include "common.cuh"
+#include "internal.h"
+
+struct moe_layer {
+  int E, k, d, d_ff, act, gate_mode, dtype;
+  double capacity_factor;
+  int hidden;  // MOE_HIDDEN_*
+};
+
+// Sticky device error word (one per device that loads the library).
+__device__ unsigned int g_moe_error_word = 0;
+
+namespace moe {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+namespace {
+
+thread_local std::string t_err;
+
+int fail(int code, const std::string& msg) {
+  t_err = msg;
+  return code;
+}
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int num_sms = 0;
+  unsigned int* err = nullptr;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Per-device set-up, done once per device with that device current.
+cudaError_t device_info(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (di.err == nullptr) {
+    e = cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_moe_error_word);
+    if (e != cudaSuccess) return e;
+    di.err = static_cast<unsigned int*>(p);
+  }
+  *out = &di;
+  return cudaSuccess;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int64_t capacity_of(const moe_layer& L, int64_t T) {
+  if (!(L.capacity_factor > 0.0)) return -1;
+  const double c = ceil(L.capacity_factor * static_cast<double>(T) * static_cast<double>(L.k) /
+                        static_cast<double>(L.E));
+  if (c > 2147483647.0) return 2147483647;
+  return static_cast<int64_t>(c);
+}
+
+struct Layout {
+  int64_t T, s_max, capacity;
+  int nblk;
+  bool need_yp;
+  bool split;
+  size_t idx, gate, dest, row_token, row_gate, part_hist, part_cnt1, part_psum, part_lse2, blockoff, counts,
+      offsets, mprefix, scal, Xp, Hp, Hp_lo, Yp, total;
+};
+
+Layout make_layout(const moe_layer& L, int64_t T) {
+  Layout w;
+  w.T = T;
+  w.capacity = capacity_of(L, T);
+  const int64_t Tk = T * L.k;
+  w.s_max = Tk;
+  if (w.capacity >= 0) w.s_max = std::min<int64_t>(Tk, static_cast<int64_t>(L.E) * w.capacity);
+  w.nblk = static_cast<int>((T + kRouterTokens - 1) / kRouterTokens);
+  const size_t elt = L.dtype == MOE_BF16 ? 2 : 4;
+  w.need_yp = !(L.dtype == MOE_BF16 && L.k == 1);
+  w.split = L.dtype == MOE_BF16 && L.hidden == MOE_HIDDEN_BF16X2;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
+  w.idx = take(sizeof(int32_t) * Tk);
+  w.gate = take(sizeof(float) * Tk);
+  w.dest = take(sizeof(int32_t) * Tk);
+  w.row_token = take(sizeof(int32_t) * w.s_max);
+  w.row_gate = take(sizeof(float) * w.s_max);
+  w.part_hist = take(sizeof(int32_t) * L.E * static_cast<size_t>(w.nblk));
+  w.part_cnt1 = take(sizeof(int32_t) * L.E * static_cast<size_t>(w.nblk));
+  w.part_psum = take(sizeof(float) * L.E * static_cast<size_t>(w.nblk));
+  w.part_lse2 = take(sizeof(float) * w.nblk);
+  w.blockoff = take(sizeof(int32_t) * L.E * static_cast<size_t>(w.nblk));
+  w.counts = take(sizeof(int32_t) * L.E);
+  w.offsets = take(sizeof(int32_t) * (L.E + 1));
+  w.mprefix = take(sizeof(int32_t) * (L.E + 1));
+  w.scal = take(64);
+  w.Xp = take(elt * static_cast<size_t>(w.s_max) * L.d);
+  w.Hp = take(elt * static_cast<size_t>(w.s_max) * L.d_ff);
+  w.Hp_lo = take(w.split ? elt * static_cast<size_t>(w.s_max) * L.d_ff : 0);
+  w.Yp = take(w.need_yp ? sizeof(float) * static_cast<size_t>(w.s_max) * L.d : 0);
+  w.total = o;
+  return w;
+}
+
+void record(const moe_debug* dbg, int stage, int which, cudaStream_t s) {
+  if (dbg == nullptr) return;
+  void* ev = dbg->events[2 * stage + which];
+  if (ev != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(ev), s);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_create(int num_experts, int k, int d, int d_ff, int act, int gate_mode, double capacity_factor, int dtype,
+               moe_handle* out) {
+  if (out == nullptr) return fail(MOE_ERR_INVALID_ARG, "moe_create: out is NULL");
+  if (num_experts < 1 || num_experts > 256) return fail(MOE_ERR_INVALID_ARG, "moe_create: num_experts must be in [1, 256]");
+  if (k < 1 || k > num_experts || k > 8) return fail(MOE_ERR_INVALID_ARG, "moe_create: need 1 <= k <= min(E, 8)");
+  if (d < 1 || d_ff < 1) return fail(MOE_ERR_INVALID_ARG, "moe_create: d and d_ff must be positive");
+  if (act != MOE_ACT_RELU && act != MOE_ACT_SWIGLU) return fail(MOE_ERR_INVALID_ARG, "moe_create: unknown act");
+  if (gate_mode != MOE_GATE_SWITCH && gate_mode != MOE_GATE_RENORM)
+    return fail(MOE_ERR_INVALID_ARG, "moe_create: unknown gate_mode");
+  if (dtype != MOE_F32 && dtype != MOE_BF16) return fail(MOE_ERR_INVALID_ARG, "moe_create: unknown dtype");
+  if (!(capacity_factor == capacity_factor)) return fail(MOE_ERR_INVALID_ARG, "moe_create: capacity_factor is NaN");
+  if (dtype == MOE_BF16 && (d % 8 != 0 || d_ff % 8 != 0))
+    return fail(MOE_ERR_UNSUPPORTED, "moe_create: bf16 layers need d and d_ff to be multiples of 8");
+  moe_layer* L = new moe_layer{num_experts, k, d, d_ff, act, gate_mode, dtype, capacity_factor, MOE_HIDDEN_BF16X2};
+  *out = L;
+  t_err.clear();
+  return MOE_OK;
+}
+
+int moe_set_hidden_precision(moe_handle h, int mode) {
+  if (h == nullptr) return fail(MOE_ERR_INVALID_ARG, "moe_set_hidden_precision: handle is NULL");
+  if (mode != MOE_HIDDEN_BF16X2 && mode != MOE_HIDDEN_BF16)
+    return fail(MOE_ERR_INVALID_ARG, "moe_set_hidden_precision: unknown mode");
+  h->hidden = mode;
+  return MOE_OK;
+}
+
+int moe_destroy(moe_handle h) {
+  delete h;
+  return MOE_OK;
+}
+
+int64_t moe_capacity(moe_handle h, int64_t T) {
+  if (h == nullptr || T < 0) return -1;
+  return capacity_of(*h, T);
+}
+
+size_t moe_workspace_bytes(moe_handle h, int64_t T) {
+  if (h == nullptr || T < 0) return 0;
+  return make_layout(*h, T).total;
+}
+
+int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const float* b_r, const void* W1,
+                const void* W3, const void* W2, void* y, int32_t* expert_counts, int32_t* dropped, float* aux_loss,
+                float* z_loss, void* workspace, size_t workspace_bytes, const moe_debug* dbg, void* stream) {
+  if (h == nullptr) return fail(MOE_ERR_INVALID_ARG, "moe_forward: handle is NULL");
+  const moe_layer& L = *h;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "moe_forward: T < 0");
+  if (T * L.k > 2147483647LL / 2) return fail(MOE_ERR_UNSUPPORTED, "moe_forward: T * k too large");
+  if (expert_counts == nullptr || dropped == nullptr || aux_loss == nullptr || z_loss == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "moe_forward: a statistics output pointer is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    if (cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * L.E, s) != cudaSuccess ||
+        cudaMemsetAsync(dropped, 0, sizeof(int32_t), s) != cudaSuccess ||
+        cudaMemsetAsync(aux_loss, 0, sizeof(float), s) != cudaSuccess ||
+        cudaMemsetAsync(z_loss, 0, sizeof(float), s) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, std::string("moe_forward: ") + cudaGetErrorString(cudaGetLastError()));
+    t_err.clear();
+    return MOE_OK;
+  }
+  if (x == nullptr || W_r == nullptr || W1 == nullptr || W2 == nullptr || y == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "moe_forward: x, W_r, W1, W2 and y must be non-NULL");
+  if ((L.act == MOE_ACT_SWIGLU) != (W3 != nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "moe_forward: W3 must be given for SwiGLU and NULL for ReLU");
+  const Layout w = make_layout(L, T);
+  if (workspace == nullptr || workspace_bytes < w.total)
+    return fail(MOE_ERR_INVALID_ARG, "moe_forward: workspace missing or smaller than moe_workspace_bytes()");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0)
+    return fail(MOE_ERR_INVALID_ARG, "moe_forward: workspace must be 256-byte aligned");
+  const uintptr_t al = reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y) |
+                       reinterpret_cast<uintptr_t>(W1) | reinterpret_cast<uintptr_t>(W2) |
+                       reinterpret_cast<uintptr_t>(W3);
+  if ((al & 15) != 0) return fail(MOE_ERR_INVALID_ARG, "moe_forward: x, y and weights must be 16-byte aligned");
+  if (L.dtype == MOE_F32 && (w.s_max + 7) / 8 > 65535)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_forward: fp32 layers are limited to 524280 assignments");
+
+  DeviceInfo* di = nullptr;
+  cudaError_t ce = device_info(&di);
+  if (ce != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_forward: ") + cudaGetErrorString(ce));
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  RoutingArgs r;
+  memset(&r, 0, sizeof(r));
+  r.T = T;
+  r.E = L.E;
+  r.k = L.k;
+  r.d = L.d;
+  r.gate_mode = L.gate_mode;
+  r.capacity = w.capacity;
+  r.nblk = w.nblk;
+  r.x_is_bf16 = L.dtype == MOE_BF16;
+  r.x = x;
+  r.W_r = W_r;
+  r.b_r = b_r;
+  r.logits_in = dbg ? dbg->logits_in : nullptr;
+  r.topk_idx = reinterpret_cast<int32_t*>(ws + w.idx);
+  r.topk_gate = reinterpret_cast<float*>(ws + w.gate);
+  r.dest_row = reinterpret_cast<int32_t*>(ws + w.dest);
+  r.part_hist = reinterpret_cast<int32_t*>(ws + w.part_hist);
+  r.part_cnt1 = reinterpret_cast<int32_t*>(ws + w.part_cnt1);
+  r.part_psum = reinterpret_cast<float*>(ws + w.part_psum);
+  r.part_lse2 = reinterpret_cast<float*>(ws + w.part_lse2);
+  r.blockoff = reinterpret_cast<int32_t*>(ws + w.blockoff);
+  r.counts = expert_counts;
+  r.offsets = reinterpret_cast<int32_t*>(ws + w.offsets);
+  r.mprefix = reinterpret_cast<int32_t*>(ws + w.mprefix);
+  r.row_token = reinterpret_cast<int32_t*>(ws + w.row_token);
+  r.row_gate = reinterpret_cast<float*>(ws + w.row_gate);
+  r.Xp = ws + w.Xp;
+  r.dropped = dropped;
+  r.aux = aux_loss;
+  r.z = z_loss;
+  r.logits_out = dbg ? dbg->logits_out : nullptr;
+  r.lse_out = dbg ? dbg->lse_out : nullptr;
+  r.drop_mask = dbg ? dbg->drop_mask : nullptr;
+  r.offsets_out = dbg ? dbg->expert_offsets : nullptr;
+  r.y_zero_dropped = w.need_yp ? nullptr : y;
+  r.yf_zero_dropped = (w.need_yp || dbg == nullptr) ? nullptr : dbg->y_f32;
+
+  const bool tc = L.dtype == MOE_BF16;
+  auto check = [&](cudaError_t e, const char* what) -> int {
+    if (e == cudaSuccess) return MOE_OK;
+    return fail(MOE_ERR_CUDA, std::string("moe_forward: ") + what + ": " + cudaGetErrorString(e));
+  };
+  int rc;
+  record(dbg, MOE_STAGE_ROUTER, 0, s);
+  if ((rc = check(launch_router(r, s), "router")) != MOE_OK) return rc;
+  record(dbg, MOE_STAGE_ROUTER, 1, s);
+  record(dbg, MOE_STAGE_SCAN, 0, s);
+  if ((rc = check(launch_scan(r, s), "scan")) != MOE_OK) return rc;
+  record(dbg, MOE_STAGE_SCAN, 1, s);
+  record(dbg, MOE_STAGE_DISPATCH, 0, s);
+  if ((rc = check(launch_dispatch(r, s), "dispatch")) != MOE_OK) return rc;
+  record(dbg, MOE_STAGE_DISPATCH, 1, s);
+
+  GemmArgs g1;
+  memset(&g1, 0, sizeof(g1));
+  g1.epi = L.act == MOE_ACT_SWIGLU ? EPI_SWIGLU_BF16 : EPI_RELU_BF16;
+  g1.E = L.E;
+  g1.N = L.d_ff;
+  g1.K = L.d;
+  g1.a_rows = w.s_max;
+  g1.A = ws + w.Xp;
+  g1.B0 = W1;
+  g1.B1 = W3;
+  g1.out = ws + w.Hp;
+  g1.split = w.split;
+  g1.out2 = w.split ? static_cast<void*>(ws + w.Hp_lo) : nullptr;
+  g1.offsets = r.offsets;
+  g1.mprefix = r.mprefix;
+  g1.row_gate = r.row_gate;
+  g1.row_token = r.row_token;
+  g1.err = di->err;
+
+  GemmArgs g2 = g1;
+  g2.epi = w.need_yp ? EPI_GATE_F32 : EPI_GATE_SCATTER_BF16;
+  g2.N = L.d;
+  g2.K = L.d_ff;
+  g2.A = ws + w.Hp;
+  g2.A2 = w.split ? static_cast<const void*>(ws + w.Hp_lo) : nullptr;
+  g2.out2 = nullptr;
+  g2.B0 = W2;
+  g2.B1 = nullptr;
+  g2.out = w.need_yp ? static_cast<void*>(ws + w.Yp) : y;
+  g2.out_f32 = (w.need_yp || dbg == nullptr) ? nullptr : dbg->y_f32;
+
+  const char* why = nullptr;
+  record(dbg, MOE_STAGE_GEMM1, 0, s);
+  ce = tc ? launch_gemm_tc(g1, di->num_sms, s, &why) : launch_gemm_simt(g1, w.s_max, s);
+  if (why != nullptr) return fail(MOE_ERR_UNSUPPORTED, std::string("moe_forward: ") + why);
+  if ((rc = check(ce, "gemm1")) != MOE_OK) return rc;
+  record(dbg, MOE_STAGE_GEMM1, 1, s);
+  record(dbg, MOE_STAGE_GEMM2, 0, s);
+  ce = tc ? launch_gemm_tc(g2, di->num_sms, s, &why) : launch_gemm_simt(g2, w.s_max, s);
+  if (why != nullptr) return fail(MOE_ERR_UNSUPPORTED, std::string("moe_forward: ") + why);
+  if ((rc = check(ce, "gemm2")) != MOE_OK) return rc;
+  record(dbg, MOE_STAGE_GEMM2, 1, s);
+  if (w.need_yp) {
+    record(dbg, MOE_STAGE_COMBINE, 0, s);
+    if ((rc = check(launch_combine(T, L.k, L.d, L.dtype == MOE_BF16, r.dest_row,
+                                   reinterpret_cast<const float*>(ws + w.Yp), y, dbg ? dbg->y_f32 : nullptr, s),
+                    "combine")) != MOE_OK)
+      return rc;
+    record(dbg, MOE_STAGE_COMBINE, 1, s);
+  }
+  if (dbg != nullptr) {
+    const size_t tk = static_cast<size_t>(T) * L.k;
+    if (dbg->topk_idx && cudaMemcpyAsync(dbg->topk_idx, r.topk_idx, 4 * tk, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "moe_forward: debug copy failed");
+    if (dbg->topk_gate && cudaMemcpyAsync(dbg->topk_gate, r.topk_gate, 4 * tk, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "moe_forward: debug copy failed");
+    if (dbg->dest_row && cudaMemcpyAsync(dbg->dest_row, r.dest_row, 4 * tk, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "moe_forward: debug copy failed");
+  }
+  t_err.clear();
+  return MOE_OK;
+}
+
+int moe_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_status: ") + cudaGetErrorString(e));
+  unsigned int word = 0;
+  e = cudaMemcpyFromSymbol(&word, g_moe_error_word, sizeof(word));
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_status: ") + cudaGetErrorString(e));
+  if (word == DEV_ERR_TIMEOUT) return fail(MOE_ERR_TIMEOUT, "moe_status: a device-side bounded wait ran out");
+  if (word != 0) return fail(MOE_ERR_CUDA, "moe_status: unknown device error word");
+  return MOE_OK;
+}
+
+int moe_clear_status(void) {
+  const unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyToSymbol(g_moe_error_word, &zero, sizeof(zero));
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_clear_status: ") + cudaGetErrorString(e));
+  return MOE_OK;
+}
+
+const char* moe_last_error(void) { return t_err.c_str(); }
+
+uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int moe_selftest_timeout(int64_t limit_ns, void* stream) {
+  DeviceInfo* di = nullptr;
+  cudaError_t ce = device_info(&di);
+  if (ce != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_selftest_timeout: ") + cudaGetErrorString(ce));
+  const int64_t lim = std::min<int64_t>(std::max<int64_t>(limit_ns, 1000), 2000000000LL);
+  ce = launch_selftest_timeout(di->err, lim, static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_selftest_timeout: ") + cudaGetErrorString(ce));
+  return MOE_OK;
+}
+
+}  // extern "C"

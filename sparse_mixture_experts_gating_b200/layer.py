@@ -1,0 +1,141 @@
+"""Python binding of the MoE layer forward pass (torch tensors -> C ABI).
+
+Marshalling only: every step of the layer runs in the CUDA library.  PyTorch
+provides device memory and the current stream.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import MoEDebug, check, lib
+
+ACT = {"relu": 0, "swiglu": 1}
+GATE = {"switch": 0, "renorm": 1}
+DTYPE = {torch.float32: 0, torch.bfloat16: 1}
+HIDDEN = {"bf16x2": 0, "bf16": 1}
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+class MoELayer:
+    """One MoE layer description (E experts, top-k, d -> d_ff -> d experts).
+
+    act: "relu" | "swiglu" (or 0 / 1); gate_mode: "switch" | "renorm" (or 0 / 1);
+    capacity_factor <= 0: dropless; dtype: torch.float32 or torch.bfloat16;
+    hidden (bf16 layers): "bf16x2" keeps the hidden activation as a hi + lo
+    pair of bf16 planes (default), "bf16" as one bf16 plane.
+    """
+
+    def __init__(self, num_experts: int, k: int, d: int, d_ff: int, act="swiglu", gate_mode="renorm",
+                 capacity_factor: float = 0.0, dtype=torch.bfloat16, hidden="bf16x2"):
+        self.E, self.k, self.d, self.d_ff = num_experts, k, d, d_ff
+        self.act = ACT[act] if isinstance(act, str) else int(act)
+        self.gate_mode = GATE[gate_mode] if isinstance(gate_mode, str) else int(gate_mode)
+        self.capacity_factor = float(capacity_factor)
+        self.dtype = dtype
+        h = ctypes.c_void_p()
+        check(lib().moe_create(num_experts, k, d, d_ff, self.act, self.gate_mode, self.capacity_factor,
+                               DTYPE[dtype], ctypes.byref(h)))
+        self._h = h
+        self._ws = None
+        self.hidden = hidden
+        check(lib().moe_set_hidden_precision(h, HIDDEN[hidden]))
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and _lib._LIB is not None:
+            _lib._LIB.moe_destroy(h)
+            self._h = None
+
+    def capacity(self, T: int) -> Optional[int]:
+        c = lib().moe_capacity(self._h, T)
+        return None if c < 0 else int(c)
+
+    def workspace_bytes(self, T: int) -> int:
+        return int(lib().moe_workspace_bytes(self._h, T))
+
+    def workspace(self, T: int, device) -> torch.Tensor:
+        n = self.workspace_bytes(T)
+        if self._ws is None or self._ws.numel() < n or self._ws.device != torch.device(device):
+            self._ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+        return self._ws
+
+    def forward(self, x, W_r, b_r, W1, W3, W2, *, out=None, stats=None, workspace=None,
+                debug: Optional[dict] = None, events=None, stream=None):
+        """Run the layer.  Returns (y, expert_counts, dropped, aux_loss, z_loss) as device tensors.
+
+        debug: optional dict of device tensors named like the fields of
+        moe_debug (logits_in, logits_out, lse_out, topk_idx, topk_gate,
+        dest_row, drop_mask, expert_offsets, y_f32).  events: optional list of
+        2 * 6 torch.cuda.Event recorded around the kernel stages.
+        """
+        T = x.shape[0]
+        dev = x.device
+        y = out if out is not None else torch.empty((T, self.d), dtype=x.dtype, device=dev)
+        if stats is None:
+            stats = (torch.empty(self.E, dtype=torch.int32, device=dev),
+                     torch.empty(1, dtype=torch.int32, device=dev),
+                     torch.empty(1, dtype=torch.float32, device=dev),
+                     torch.empty(1, dtype=torch.float32, device=dev))
+        counts, dropped, aux, z = stats
+        ws = workspace if workspace is not None else self.workspace(T, dev)
+        dbg = None
+        if debug is not None or events is not None:
+            dbg = MoEDebug()
+            for name, t in (debug or {}).items():
+                setattr(dbg, name, _ptr(t))
+            if events is not None:
+                for i, ev in enumerate(events):
+                    if ev is not None:
+                        if not ev.cuda_event:  # torch creates its CUDA event lazily, on first record
+                            ev.record(torch.cuda.current_stream() if stream is None else stream)
+                        dbg.events[i] = ev.cuda_event
+        check(lib().moe_forward(
+            self._h, T, _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(y),
+            _ptr(counts), _ptr(dropped), _ptr(aux), _ptr(z), _ptr(ws), ws.numel(),
+            None if dbg is None else ctypes.byref(dbg), _stream_handle(stream)))
+        return y, counts, dropped, aux, z
+
+    __call__ = forward
+
+    def debug_buffers(self, T: int, device) -> dict:
+        """Device tensors for every output field of moe_debug."""
+        E, k = self.E, self.k
+        return {
+            "logits_out": torch.empty((T, E), dtype=torch.float32, device=device),
+            "lse_out": torch.empty(T, dtype=torch.float32, device=device),
+            "topk_idx": torch.empty((T, k), dtype=torch.int32, device=device),
+            "topk_gate": torch.empty((T, k), dtype=torch.float32, device=device),
+            "dest_row": torch.empty((T, k), dtype=torch.int32, device=device),
+            "drop_mask": torch.empty((T, k), dtype=torch.uint8, device=device),
+            "expert_offsets": torch.empty(E + 1, dtype=torch.int32, device=device),
+            "y_f32": torch.empty((T, self.d), dtype=torch.float32, device=device),
+        }
+
+
+def status(stream=None) -> None:
+    """Synchronise the stream and raise MoEError if a kernel's bounded wait ran out."""
+    check(lib().moe_status(_stream_handle(stream)))
+
+
+def clear_status() -> None:
+    check(lib().moe_clear_status())
+
+
+def launch_count() -> int:
+    return int(lib().moe_launch_count())
+
+
+def selftest_timeout(limit_ns: int, stream=None) -> None:
+    check(lib().moe_selftest_timeout(int(limit_ns), _stream_handle(stream)))

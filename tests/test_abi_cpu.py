@@ -1,0 +1,108 @@
+"""The C-ABI library: it builds, loads, exports every symbol include/moe.h
+declares, and validates arguments on the host.  No compute call is made (no
+GPU is needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+from sparse_mixture_experts_gating_b200 import _build, _lib
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return _lib.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src, flags=re.M)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    assert {"moe_create", "moe_forward", "moe_destroy", "moe_workspace_bytes", "moe_status"} <= set(names)
+    assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def _create(L, *args):
+    h = ctypes.c_void_p()
+    rc = L.moe_create(*args, ctypes.byref(h))
+    return rc, h
+
+
+def test_create_validates_arguments(L):
+    ok, h = _create(L, 8, 2, 4096, 14336, 1, 1, 0.0, 1)
+    assert ok == _lib.MOE_OK and h.value
+    L.moe_destroy(h)
+    bad = [
+        (0, 1, 64, 64, 0, 1, 0.0, 1),      # no experts
+        (257, 1, 64, 64, 0, 1, 0.0, 1),    # too many experts
+        (4, 5, 64, 64, 0, 1, 0.0, 1),      # k > E
+        (16, 9, 64, 64, 0, 1, 0.0, 1),     # k > 8
+        (4, 0, 64, 64, 0, 1, 0.0, 1),      # k = 0
+        (4, 2, 0, 64, 0, 1, 0.0, 1),       # d = 0
+        (4, 2, 64, 64, 2, 1, 0.0, 1),      # unknown act
+        (4, 2, 64, 64, 0, 2, 0.0, 1),      # unknown gate
+        (4, 2, 64, 64, 0, 1, 0.0, 7),      # unknown dtype
+        (4, 2, 64, 64, 0, 1, float("nan"), 1),
+    ]
+    for args in bad:
+        rc, h = _create(L, *args)
+        assert rc == _lib.MOE_ERR_INVALID_ARG, args
+        assert h.value is None
+        assert L.moe_last_error().decode().startswith("moe_create")
+    rc, _ = _create(L, 4, 2, 60, 64, 0, 1, 0.0, 1)  # bf16 rows must be 16-byte multiples
+    assert rc == _lib.MOE_ERR_UNSUPPORTED
+    rc, h = _create(L, 4, 2, 60, 62, 0, 1, 0.0, 0)  # fp32 accepts any width
+    assert rc == _lib.MOE_OK
+    L.moe_destroy(h)
+
+
+def test_capacity_matches_the_oracle(L):
+    rng = np.random.default_rng(3)
+    for _ in range(300):
+        E = int(rng.integers(1, 257)); k = int(rng.integers(1, min(E, 8) + 1))
+        cf = float(rng.choice([0.0, -1.0, 1.0, 1.25, 2.0, rng.uniform(0.01, 4.0)]))
+        T = int(rng.integers(0, 100000))
+        rc, h = _create(L, E, k, 64, 64, 0, 1, cf, 1)
+        assert rc == 0
+        c = L.moe_capacity(h, T)
+        ref = O.expert_capacity(cf, T, k, E)
+        assert (None if c < 0 else c) == ref, (E, k, cf, T)
+        L.moe_destroy(h)
+
+
+def test_workspace_and_forward_validation_without_gpu(L):
+    rc, h = _create(L, 64, 1, 768, 3072, 0, 0, 1.25, 1)
+    assert rc == 0
+    ws = L.moe_workspace_bytes(h, 8192)
+    # Xp + Hp + routing tables at least; capacity 160 bounds the sorted rows
+    assert ws >= 2 * 8192 * (768 + 3072)
+    assert L.moe_workspace_bytes(h, -1) == 0
+    assert L.moe_workspace_bytes(None, 16) == 0
+    p = ctypes.c_void_p(256)
+    # NULL handle, negative T, NULL statistics outputs: rejected before any CUDA call
+    assert L.moe_forward(None, 4, p, p, None, p, None, p, p, p, p, p, p, p, 1 << 30, None, None) == 1
+    assert L.moe_forward(h, -1, p, p, None, p, None, p, p, p, p, p, p, p, 1 << 30, None, None) == 1
+    assert L.moe_forward(h, 4, p, p, None, p, None, p, p, None, p, p, p, p, 1 << 30, None, None) == 1
+    # W3 given for a ReLU layer
+    assert L.moe_forward(h, 4, p, p, None, p, p, p, p, p, p, p, p, p, 1 << 30, None, None) == 1
+    # workspace too small / misaligned
+    assert L.moe_forward(h, 4, p, p, None, p, None, p, p, p, p, p, p, p, 16, None, None) == 1
+    assert L.moe_forward(h, 4, p, p, None, p, None, p, p, p, p, p, p, ctypes.c_void_p(272), 1 << 30,
+                         None, None) == 1
+    assert "workspace" in L.moe_last_error().decode()
+    L.moe_destroy(h)
+    assert L.moe_destroy(None) == 0

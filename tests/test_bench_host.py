@@ -1,0 +1,71 @@
+"""Host-side logic of bench.py (no GPU): rank reduction over gloo with two
+ranks, per-rank seeding, algorithmic work and roofline arithmetic."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from sparse_mixture_experts_gating_b200.workloads import WORKLOADS
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    secs = [0.25, 0.75][rank]
+    t, n = bench.combine_ranks(secs, 1000 * (rank + 1), dist)
+    out[rank] = (t, n)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_combine_ranks_takes_max_time_and_sums_tokens_over_two_gloo_ranks():
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
+        res = dict(out)
+    assert res[0] == res[1] == (0.75, 3000.0)
+
+
+def test_combine_ranks_single_process_is_identity():
+    assert bench.combine_ranks(0.5, 123, None) == (0.5, 123)
+
+
+def test_rank_seeds_differ_and_rank0_keeps_the_workload_seed():
+    seeds = {bench.rank_seed(1235, r) for r in range(8)}
+    assert len(seeds) == 8 and bench.rank_seed(1235, 0) == 1235
+
+
+def test_layer_work_mixtral_prefill_matches_the_closed_form():
+    w = WORKLOADS["mixtral_prefill"]
+    work = bench.layer_work(w, [2048] * 8)
+    S = 16384
+    assert work["gemm1"]["flops"] == 2 * S * 4096 * 14336 * 2
+    assert work["gemm2"]["flops"] == 2 * S * 14336 * 4096
+    # 6 * d * d_ff * T * k for the experts (5.77 TFLOP) plus the router
+    assert abs(work["flops_layer"] - (6 * 4096 * 14336 * 16384 + 2 * 8192 * 8 * 4096)) < 1
+    assert work["bytes_layer"] == 3 * 8 * 4096 * 14336 * 2 + 2 * 8192 * 4096 * 2 + 8 * 4096 * 4
+
+
+def test_kernel_roofline_picks_the_binding_resource():
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0}
+    r = bench.kernel_roofline(flops=1e12, nbytes=1e9, seconds=1e-3, peaks=peaks)
+    assert r["bound"] == "tensor" and r["achieved"] == 1000.0 and abs(r["frac"] - 1000 / 1500) < 1e-4
+    r = bench.kernel_roofline(flops=1e9, nbytes=3e9, seconds=1e-3, peaks=peaks)
+    assert r["bound"] == "hbm" and r["achieved"] == 3000.0 and r["frac"] == 0.5
+
+
+def test_traffic_is_null_without_a_matching_profile(tmp_path, monkeypatch):
+    assert bench.profiled_traffic("gemm1", "no_such_workload") is None
