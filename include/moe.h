@@ -169,6 +169,29 @@ MOE_API int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r
                 void* workspace, size_t workspace_bytes, const moe_debug* dbg, void* stream);
 
 /*
+ * moe_forward for callers that cannot allocate device memory (no counterpart
+ * on the pages): for example a plug-in inside a host framework that owns every
+ * device allocation and offers its extensions no workspace, or a serving loop
+ * that must not enter an allocator on its hot path.  Same arguments and
+ * results as moe_forward, without the workspace and the debug hooks: the
+ * scratch is a 32 MiB array compiled into the library, resident on every GPU
+ * that loads it until the process exits.
+ *   - A call needing more than 32 MiB (moe_workspace_bytes(h, T) > 32 MiB;
+ *     e.g. the 8-expert top-2 d 4096 / d_ff 14336 SwiGLU layer up to T = 204)
+ *     is rejected with MOE_ERR_UNSUPPORTED before any launch.
+ *   - The first call on a device looks up the array's address on that device
+ *     (with it current); make that first call before any stream capture.
+ *   - Every call shares the array and leaves its contents there; calls that
+ *     overlap on the GPU (other streams, other host threads) race on it.
+ *     Nothing in it needs to start at zero.
+ *   - Allocates nothing (no cudaMalloc / cudaFree or allocating routine).
+ */
+MOE_API int moe_forward_static(moe_handle h, int64_t T, const void* x, const float* W_r, const float* b_r,
+                               const void* W1, const void* W3, const void* W2, void* y,
+                               int32_t* expert_counts, int32_t* dropped, float* aux_loss, float* z_loss,
+                               void* stream);
+
+/*
  * Synchronise `stream` and report the device error word of the current device:
  * MOE_OK, MOE_ERR_TIMEOUT (a kernel's bounded wait ran out and it returned
  * early; outputs of that call are undefined) or MOE_ERR_CUDA.  The error

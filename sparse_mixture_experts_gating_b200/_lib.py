@@ -24,6 +24,8 @@ SIGNATURES = {
     "moe_forward": (c_int, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                             c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p,
                             c_void_p]),
+    "moe_forward_static": (c_int, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                   c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "moe_status": (c_int, [c_void_p]),
     "moe_clear_status": (c_int, []),
     "moe_last_error": (c_char_p, []),

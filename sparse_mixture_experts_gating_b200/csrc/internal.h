@@ -88,4 +88,7 @@ cudaError_t launch_selftest_timeout(unsigned int* err, int64_t limit_ns, cudaStr
 
 void count_launch();
 
+// Set the calling thread's moe_last_error() message.
+void set_error_message(const char* msg);
+
 }  // namespace moe

@@ -130,6 +130,9 @@ void record(const moe_debug* dbg, int stage, int which, cudaStream_t s) {
 }
 
 }  // namespace
+
+void set_error_message(const char* msg) { t_err = msg; }
+
 }  // namespace moe
 
 using namespace moe;
