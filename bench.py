@@ -184,6 +184,13 @@ def combine_ranks(seconds_local, tokens_local, dist_mod=None):
     return float(t.item()), float(n.item())
 
 
+def gpu_hold(torch, ms):
+    """Keep the GPU busy for about `ms` so the host can enqueue the timed steps
+    ahead of it; the step events then measure GPU time only (launch latency of
+    the host never shows up as idle GPU time inside a step)."""
+    torch.cuda._sleep(int(ms * 2.0e6))  # cycles at ~2 GHz
+
+
 def rank_seed(base_seed, rank):
     """Each replica draws its own batch of tokens; weights are shared."""
     return base_seed + 7919 * rank
@@ -252,6 +259,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--hidden", choices=["bf16x2", "bf16"], default="bf16x2",
                     help="how the expert hidden activation is held (bf16 layers)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's token count (small cases for profiler captures)")
     args = ap.parse_args()
 
     import torch
@@ -263,6 +272,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     w = WORKLOADS[args.workload]
+    if args.tokens is not None:
+        w = w.with_(T=args.tokens, x_rows_of=None)
     warmup = max(3, args.warmup)
 
     if args.impl == "reference":
@@ -299,8 +310,30 @@ def main():
     status()
 
     K = args.steps
-    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    stage_names = ["router", "scan", "dispatch", "gemm1", "gemm2", "combine"]
+    active = [n for n in stage_names if not (n == "combine" and w.dtype == 1 and w.k == 1)]
+
+    # Untimed profiling pass: every stage bracketed by events -> per-kernel breakdown.
     ev_stage = [[torch.cuda.Event(enable_timing=True) for _ in range(12)] for _ in range(K)]
+    torch.cuda.synchronize()
+    gpu_hold(torch, 2.0 + 0.3 * K)
+    for i in range(K):
+        flush.zero_()
+        step(events=ev_stage[i])
+    torch.cuda.synchronize()
+    stage_ms = {}
+    for s_i, name in enumerate(stage_names):
+        if name in active:
+            stage_ms[name] = statistics.mean(ev[2 * s_i].elapsed_time(ev[2 * s_i + 1]) for ev in ev_stage)
+    dom = max(("gemm1", "gemm2"), key=lambda n: stage_ms[n])
+    dom_i = stage_names.index(dom)
+
+    # Timed region: step events, plus the dominant kernel's own pair (live roofline).
+    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ev_dom = [[None] * 12 for _ in range(K)]
+    for i in range(K):
+        ev_dom[i][2 * dom_i] = torch.cuda.Event(enable_timing=True)
+        ev_dom[i][2 * dom_i + 1] = torch.cuda.Event(enable_timing=True)
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     sampler = ClockSampler(vis.split(",")[local].strip() if vis else str(local))
     sampler.start()
@@ -310,10 +343,11 @@ def main():
     torch.cuda.synchronize()
     n_launch0 = launch_count()
     wall0 = time.time()
+    gpu_hold(torch, 2.0 + 0.2 * K)
     for i in range(K):
         flush.zero_()
         ev_step[i][0].record(stream)
-        step(events=ev_stage[i])
+        step(events=ev_dom[i])
         ev_step[i][1].record(stream)
     torch.cuda.synchronize()
     wall1 = time.time()
@@ -326,12 +360,7 @@ def main():
 
     step_ms = [a.elapsed_time(b) for a, b in ev_step]
     total_s = sum(step_ms) / 1e3
-    stage_names = ["router", "scan", "dispatch", "gemm1", "gemm2", "combine"]
-    stage_ms = {}
-    for s_i, name in enumerate(stage_names):
-        if name == "combine" and w.dtype == 1 and w.k == 1:
-            continue
-        stage_ms[name] = statistics.mean(ev[2 * s_i].elapsed_time(ev[2 * s_i + 1]) for ev in ev_stage)
+    dom_ms = statistics.mean(ev[2 * dom_i].elapsed_time(ev[2 * dom_i + 1]) for ev in ev_dom)
 
     # end to end through the public API: pinned host x in, y and statistics out, every step
     x_host = inp["x"].cpu().pin_memory()
@@ -339,6 +368,8 @@ def main():
     st_host = [torch.empty(s.shape, dtype=s.dtype).pin_memory() for s in stats]
     x_dev = torch.empty_like(inp["x"])
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    torch.cuda.synchronize()
+    gpu_hold(torch, 2.0 + 0.2 * (K + warmup))
     for i in range(warmup + K):
         flush.zero_()
         if i >= warmup:
@@ -362,8 +393,7 @@ def main():
     kept = [c if cap is None else min(c, cap) for c in counts]
     work = layer_work(w, kept, args.hidden)
     peaks, peak_src = load_peaks()
-    dom = max(("gemm1", "gemm2"), key=lambda s: stage_ms[s])
-    roof = kernel_roofline(work[dom]["flops"], work[dom]["bytes"], stage_ms[dom] / 1e3, peaks)
+    roof = kernel_roofline(work[dom]["flops"], work[dom]["bytes"], dom_ms / 1e3, peaks)
     roof["kernel"] = f"{STAGE_KERNEL[dom]} ({dom})"
     roof["peak_source"] = f"{peak_src} ({'bf16_tflops' if roof['bound'] == 'tensor' else 'hbm_gbs'}, burst)"
     tr = profiled_traffic(dom, w.name)

@@ -55,18 +55,7 @@ constexpr uint32_t TMEM_COLS = 2 * MMA_N;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, MMA_N);
 constexpr int MAX_E = 256;
 
-struct Params {
-  int E, N, K, n_tiles, bn, num_kb;
-  void* out;
-  void* out_lo;     // SwiGLU/ReLU epilogue with a split hidden activation: the lo plane
-  float* out_f32;
-  const int32_t* offsets;
-  const int32_t* mprefix;
-  const float* row_gate;
-  const int32_t* row_token;
-  unsigned int* err;
-  uint64_t limit_ns;
-};
+using Params = TcParams;
 
 struct Ctl {
   uint64_t full[MAX_STAGES];
@@ -409,46 +398,52 @@ EncodeTiledFn encode_fn() {
 
 // Row-major bf16 matrix [rows][cols] -> map with box [128 rows][64 cols], 128B swizzle.
 bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  return make_map_bf16(m, base, rows, cols, 128);
+}
+
+}  // namespace
+
+bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), 128};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+namespace {
+
 template <int EPI, bool SPLIT>
-cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b0, const CUtensorMap& b1,
-                     const Params& p, int num_sms, cudaStream_t s) {
+cudaError_t launch_t(const TcGemmPlan& pl, int num_sms, cudaStream_t s) {
   constexpr bool A_SPLIT = SPLIT && (EPI == EPI_GATE_F32 || EPI == EPI_GATE_SCATTER_BF16);
   constexpr size_t bytes = smem_bytes<A_SPLIT>();
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(bytes));
+  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void*>(&grouped_gemm_kernel<EPI, SPLIT>),
+                                      static_cast<int>(bytes));
   if (e != cudaSuccess) return e;
-  grouped_gemm_kernel<EPI, SPLIT><<<num_sms, NUM_THREADS, bytes, s>>>(a, a2, b0, b1, p);
+  grouped_gemm_kernel<EPI, SPLIT><<<num_sms, NUM_THREADS, bytes, s>>>(pl.a, pl.a2, pl.b0, pl.b1, pl.p);
   count_launch();
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t s, const char** why) {
+cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
   *why = nullptr;
   if (g.E > MAX_E) { *why = "grouped GEMM supports at most 256 experts"; return cudaErrorInvalidValue; }
   const bool a_split = g.split && g.A2 != nullptr;
-  CUtensorMap ma, ma2, mb0, mb1;
-  if (!make_map(&ma, g.A, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K)) ||
-      !make_map(&ma2, a_split ? g.A2 : g.A, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K)) ||
-      !make_map(&mb0, g.B0, static_cast<uint64_t>(g.E) * g.N, static_cast<uint64_t>(g.K)) ||
-      !make_map(&mb1, g.epi == EPI_SWIGLU_BF16 ? g.B1 : g.B0, static_cast<uint64_t>(g.E) * g.N,
+  if (!make_map(&pl->a, g.A, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K)) ||
+      !make_map(&pl->a2, a_split ? g.A2 : g.A, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K)) ||
+      !make_map(&pl->b0, g.B0, static_cast<uint64_t>(g.E) * g.N, static_cast<uint64_t>(g.K)) ||
+      !make_map(&pl->b1, g.epi == EPI_SWIGLU_BF16 ? g.B1 : g.B0, static_cast<uint64_t>(g.E) * g.N,
                 static_cast<uint64_t>(g.K))) {
     *why = "cuTensorMapEncodeTiled failed (alignment or driver entry point)";
     return cudaErrorInvalidValue;
   }
-  Params p;
+  Params& p = pl->p;
   p.E = g.E;
   p.N = g.N;
   p.K = g.K;
@@ -464,23 +459,30 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t s, const
   p.row_token = g.row_token;
   p.err = g.err;
   p.limit_ns = kWaitLimitNs;
-  if (g.split) {
-    switch (g.epi) {
-      case EPI_RELU_BF16: return launch_t<EPI_RELU_BF16, true>(ma, ma2, mb0, mb1, p, num_sms, s);
-      case EPI_SWIGLU_BF16: return launch_t<EPI_SWIGLU_BF16, true>(ma, ma2, mb0, mb1, p, num_sms, s);
-      case EPI_GATE_F32: return launch_t<EPI_GATE_F32, true>(ma, ma2, mb0, mb1, p, num_sms, s);
-      case EPI_GATE_SCATTER_BF16: return launch_t<EPI_GATE_SCATTER_BF16, true>(ma, ma2, mb0, mb1, p, num_sms, s);
-    }
-  } else {
-    switch (g.epi) {
-      case EPI_RELU_BF16: return launch_t<EPI_RELU_BF16, false>(ma, ma2, mb0, mb1, p, num_sms, s);
-      case EPI_SWIGLU_BF16: return launch_t<EPI_SWIGLU_BF16, false>(ma, ma2, mb0, mb1, p, num_sms, s);
-      case EPI_GATE_F32: return launch_t<EPI_GATE_F32, false>(ma, ma2, mb0, mb1, p, num_sms, s);
-      case EPI_GATE_SCATTER_BF16: return launch_t<EPI_GATE_SCATTER_BF16, false>(ma, ma2, mb0, mb1, p, num_sms, s);
+  pl->epi = g.epi;
+  pl->split = g.split;
+  if (g.epi < EPI_RELU_BF16 || g.epi > EPI_GATE_SCATTER_BF16) {
+    *why = "unknown epilogue";
+    return cudaErrorInvalidValue;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_gemm_tc(const TcGemmPlan& pl, int num_sms, cudaStream_t s) {
+  if (pl.split) {
+    switch (pl.epi) {
+      case EPI_RELU_BF16: return launch_t<EPI_RELU_BF16, true>(pl, num_sms, s);
+      case EPI_SWIGLU_BF16: return launch_t<EPI_SWIGLU_BF16, true>(pl, num_sms, s);
+      case EPI_GATE_F32: return launch_t<EPI_GATE_F32, true>(pl, num_sms, s);
+      default: return launch_t<EPI_GATE_SCATTER_BF16, true>(pl, num_sms, s);
     }
   }
-  *why = "unknown epilogue";
-  return cudaErrorInvalidValue;
+  switch (pl.epi) {
+    case EPI_RELU_BF16: return launch_t<EPI_RELU_BF16, false>(pl, num_sms, s);
+    case EPI_SWIGLU_BF16: return launch_t<EPI_SWIGLU_BF16, false>(pl, num_sms, s);
+    case EPI_GATE_F32: return launch_t<EPI_GATE_F32, false>(pl, num_sms, s);
+    default: return launch_t<EPI_GATE_SCATTER_BF16, false>(pl, num_sms, s);
+  }
 }
 
 }  // namespace moe

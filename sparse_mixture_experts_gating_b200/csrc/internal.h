@@ -1,6 +1,7 @@
 // Host-side interface between the translation units of the MoE library.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -52,6 +53,16 @@ struct RoutingArgs {
 };
 
 cudaError_t launch_router(const RoutingArgs& a, cudaStream_t s);
+
+// Tensor-core router for bf16 layers with E <= 128: W_r is first split exactly
+// into three bf16 planes [3][E_pad][d] (E_pad = E rounded up to 16) in `wsplit`.
+constexpr int kRouterTcMaxE = 128;
+inline int router_pad_e(int E) { return (E + 15) / 16 * 16; }
+cudaError_t launch_router_tc(const RoutingArgs& a, void* wsplit, int num_sms, unsigned int* err, cudaStream_t s,
+                             const char** why);
+
+// bf16 [rows][cols] tensor map, box [box_rows][64], 128-byte swizzle.
+bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 cudaError_t launch_scan(const RoutingArgs& a, cudaStream_t s);
 cudaError_t launch_dispatch(const RoutingArgs& a, cudaStream_t s);
 cudaError_t launch_combine(int64_t T, int k, int d, int y_is_bf16, const int32_t* dest_row, const float* Yp,
@@ -81,7 +92,33 @@ struct GemmArgs {
   unsigned int* err;
 };
 
-cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t s, const char** why);
+// Kernel parameters of the tensor-core grouped GEMM.
+struct TcParams {
+  int E, N, K, n_tiles, bn, num_kb;
+  void* out;
+  void* out_lo;     // first projection with a split hidden activation: the lo plane
+  float* out_f32;   // scatter epilogue only: optional fp32 copy of y
+  const int32_t* offsets;
+  const int32_t* mprefix;
+  const float* row_gate;
+  const int32_t* row_token;
+  unsigned int* err;
+  uint64_t limit_ns;
+};
+
+// Everything a tensor-core GEMM launch needs, prepared on the host up front.
+struct TcGemmPlan {
+  CUtensorMap a, a2, b0, b1;
+  TcParams p;
+  int epi;
+  int split;
+};
+
+cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* plan, const char** why);
+cudaError_t launch_gemm_tc(const TcGemmPlan& plan, int num_sms, cudaStream_t s);
+
+// Raise a kernel's dynamic shared memory limit, once per (kernel, device, size).
+cudaError_t set_smem_limit_once(const void* kernel, int bytes);
 cudaError_t launch_gemm_simt(const GemmArgs& g, int64_t s_max, cudaStream_t s);
 
 cudaError_t launch_selftest_timeout(unsigned int* err, int64_t limit_ns, cudaStream_t s);

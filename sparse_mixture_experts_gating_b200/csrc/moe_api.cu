@@ -10,7 +10,9 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <set>
 #include <string>
+#include <tuple>
 
 #include "moe.h"
 #include "common.cuh"
@@ -85,7 +87,7 @@ struct Layout {
   bool need_yp;
   bool split;
   size_t idx, gate, dest, row_token, row_gate, part_hist, part_cnt1, part_psum, part_lse2, blockoff, counts,
-      offsets, mprefix, scal, Xp, Hp, Hp_lo, Yp, total;
+      offsets, mprefix, scal, wsplit, Xp, Hp, Hp_lo, Yp, total;
 };
 
 Layout make_layout(const moe_layer& L, int64_t T) {
@@ -115,6 +117,8 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   w.offsets = take(sizeof(int32_t) * (L.E + 1));
   w.mprefix = take(sizeof(int32_t) * (L.E + 1));
   w.scal = take(64);
+  const bool tc_router = L.dtype == MOE_BF16 && L.E <= kRouterTcMaxE;
+  w.wsplit = take(tc_router ? 3 * sizeof(uint16_t) * router_pad_e(L.E) * static_cast<size_t>(L.d) : 0);
   w.Xp = take(elt * static_cast<size_t>(w.s_max) * L.d);
   w.Hp = take(elt * static_cast<size_t>(w.s_max) * L.d_ff);
   w.Hp_lo = take(w.split ? elt * static_cast<size_t>(w.s_max) * L.d_ff : 0);
@@ -132,6 +136,20 @@ void record(const moe_debug* dbg, int stage, int which, cudaStream_t s) {
 }  // namespace
 
 void set_error_message(const char* msg) { t_err = msg; }
+
+cudaError_t set_smem_limit_once(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::set<std::tuple<const void*, int, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const auto key = std::make_tuple(kernel, dev, bytes);
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.count(key)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert(key);
+  return e;
+}
 
 }  // namespace moe
 
@@ -259,22 +277,6 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   r.y_zero_dropped = w.need_yp ? nullptr : y;
   r.yf_zero_dropped = (w.need_yp || dbg == nullptr) ? nullptr : dbg->y_f32;
 
-  const bool tc = L.dtype == MOE_BF16;
-  auto check = [&](cudaError_t e, const char* what) -> int {
-    if (e == cudaSuccess) return MOE_OK;
-    return fail(MOE_ERR_CUDA, std::string("moe_forward: ") + what + ": " + cudaGetErrorString(e));
-  };
-  int rc;
-  record(dbg, MOE_STAGE_ROUTER, 0, s);
-  if ((rc = check(launch_router(r, s), "router")) != MOE_OK) return rc;
-  record(dbg, MOE_STAGE_ROUTER, 1, s);
-  record(dbg, MOE_STAGE_SCAN, 0, s);
-  if ((rc = check(launch_scan(r, s), "scan")) != MOE_OK) return rc;
-  record(dbg, MOE_STAGE_SCAN, 1, s);
-  record(dbg, MOE_STAGE_DISPATCH, 0, s);
-  if ((rc = check(launch_dispatch(r, s), "dispatch")) != MOE_OK) return rc;
-  record(dbg, MOE_STAGE_DISPATCH, 1, s);
-
   GemmArgs g1;
   memset(&g1, 0, sizeof(g1));
   g1.epi = L.act == MOE_ACT_SWIGLU ? EPI_SWIGLU_BF16 : EPI_RELU_BF16;
@@ -306,15 +308,43 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   g2.out = w.need_yp ? static_cast<void*>(ws + w.Yp) : y;
   g2.out_f32 = (w.need_yp || dbg == nullptr) ? nullptr : dbg->y_f32;
 
-  const char* why = nullptr;
+  // Host-side preparation of both GEMM launches happens before the first launch.
+  TcGemmPlan plan1, plan2;
+  if (L.dtype == MOE_BF16) {
+    const char* why = nullptr;
+    if (plan_gemm_tc(g1, &plan1, &why) != cudaSuccess || plan_gemm_tc(g2, &plan2, &why) != cudaSuccess)
+      return fail(MOE_ERR_UNSUPPORTED, std::string("moe_forward: ") + (why ? why : "GEMM plan failed"));
+  }
+
+  const bool tc = L.dtype == MOE_BF16;
+  auto check = [&](cudaError_t e, const char* what) -> int {
+    if (e == cudaSuccess) return MOE_OK;
+    return fail(MOE_ERR_CUDA, std::string("moe_forward: ") + what + ": " + cudaGetErrorString(e));
+  };
+  int rc;
+  record(dbg, MOE_STAGE_ROUTER, 0, s);
+  if (tc && L.E <= kRouterTcMaxE && r.logits_in == nullptr) {
+    const char* why = nullptr;
+    ce = launch_router_tc(r, ws + w.wsplit, di->num_sms, di->err, s, &why);
+    if (why != nullptr) return fail(MOE_ERR_UNSUPPORTED, std::string("moe_forward: ") + why);
+    if ((rc = check(ce, "router")) != MOE_OK) return rc;
+  } else if ((rc = check(launch_router(r, s), "router")) != MOE_OK) {
+    return rc;
+  }
+  record(dbg, MOE_STAGE_ROUTER, 1, s);
+  record(dbg, MOE_STAGE_SCAN, 0, s);
+  if ((rc = check(launch_scan(r, s), "scan")) != MOE_OK) return rc;
+  record(dbg, MOE_STAGE_SCAN, 1, s);
+  record(dbg, MOE_STAGE_DISPATCH, 0, s);
+  if ((rc = check(launch_dispatch(r, s), "dispatch")) != MOE_OK) return rc;
+  record(dbg, MOE_STAGE_DISPATCH, 1, s);
+
   record(dbg, MOE_STAGE_GEMM1, 0, s);
-  ce = tc ? launch_gemm_tc(g1, di->num_sms, s, &why) : launch_gemm_simt(g1, w.s_max, s);
-  if (why != nullptr) return fail(MOE_ERR_UNSUPPORTED, std::string("moe_forward: ") + why);
+  ce = tc ? launch_gemm_tc(plan1, di->num_sms, s) : launch_gemm_simt(g1, w.s_max, s);
   if ((rc = check(ce, "gemm1")) != MOE_OK) return rc;
   record(dbg, MOE_STAGE_GEMM1, 1, s);
   record(dbg, MOE_STAGE_GEMM2, 0, s);
-  ce = tc ? launch_gemm_tc(g2, di->num_sms, s, &why) : launch_gemm_simt(g2, w.s_max, s);
-  if (why != nullptr) return fail(MOE_ERR_UNSUPPORTED, std::string("moe_forward: ") + why);
+  ce = tc ? launch_gemm_tc(plan2, di->num_sms, s) : launch_gemm_simt(g2, w.s_max, s);
   if ((rc = check(ce, "gemm2")) != MOE_OK) return rc;
   record(dbg, MOE_STAGE_GEMM2, 1, s);
   if (w.need_yp) {

@@ -1,0 +1,379 @@
+// Router of bf16 layers on the tensor cores, with fp32 arithmetic:
+//   h = W_r x (+ b)  ("Mixture of experts", rayaq.ca, section "Replacing the
+//   feed-forward block"; the router stays float32 per section "Implementation").
+//
+// W_r (fp32) is split exactly into three bf16 planes w0 + w1 + w2 = W_r (each
+// plane takes the next 8 significant bits of the residual; 3 x 8 = 24 bits =
+// an fp32 significand).  x is bf16, so every product x_c * w_p,c is exact and
+// the tcgen05 MMA accumulates all 3d of them in fp32 in TMEM: an fp32 dot
+// product, not a reduced-precision one.  With dyadic inputs whose partial sums
+// are all representable, the logits are exact in any order.
+//
+// One CTA per 128-token tile (persistent over tiles): warp 0 issues TMA (x box
+// 128 x 64, three plane boxes E_pad x 64), warp 1 issues the MMAs (M 128,
+// N E_pad, K 16; 4 per plane per k-block), warps 2..5 run the epilogue with one
+// token per thread (TMEM lane = token): bias, max, one-pass top-k (ties to the
+// lower expert index), log-sum-exp, gates, and the per-32-token partial counts
+// and sums that the scan kernel reduces (each epilogue warp owns one 32-token
+// router block, the same partition as the CUDA-core router).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int NUM_THREADS = 192;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int MAX_STAGES = 4;
+
+struct RtParams {
+  int64_t T;
+  int E, k, d, gate_mode, num_kb, nblk, n_tiles;
+  const float* b_r;
+  int32_t* topk_idx;
+  float* topk_gate;
+  int32_t* part_hist;
+  int32_t* part_cnt1;
+  float* part_psum;
+  float* part_lse2;
+  float* logits_out;
+  float* lse_out;
+  unsigned int* err;
+  uint64_t limit_ns;
+};
+
+struct RtCtl {
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_slot;
+  volatile int abort;
+  int hist[4][kRouterTcMaxE];
+  int cnt1[4][kRouterTcMaxE];
+};
+
+template <int EP>
+struct RtGeo {
+  static constexpr int B_PLANE = EP * BK * 2;  // one plane box: EP rows x 128 B
+  static constexpr int STAGE_BYTES = A_BYTES + 3 * B_PLANE;
+  static constexpr int STAGES = (200 * 1024 / STAGE_BYTES) < MAX_STAGES ? (200 * 1024 / STAGE_BYTES) : MAX_STAGES;
+  static constexpr uint32_t TMEM_COLS = (2 * EP) <= 32 ? 32 : (2 * EP) <= 64 ? 64 : (2 * EP) <= 128 ? 128
+                                        : (2 * EP) <= 256 ? 256 : 512;
+  static constexpr size_t SMEM = STAGES * STAGE_BYTES + sizeof(RtCtl) + 1024;
+};
+
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Split W_r (fp32 [E][d]) into bf16 planes [3][EP][d]; rows E..EP-1 are zero.
+__global__ void __launch_bounds__(256) split_router_kernel(const float* __restrict__ W, int E, int EP, int d,
+                                                           __nv_bfloat16* __restrict__ planes) {
+  const int64_t n = static_cast<int64_t>(EP) * d;
+  for (int64_t i = blockIdx.x * 256ll + threadIdx.x; i < n; i += static_cast<int64_t>(gridDim.x) * 256) {
+    const int e = static_cast<int>(i / d);
+    const float w = e < E ? W[i] : 0.f;
+    const __nv_bfloat16 w0 = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(w0);
+    const __nv_bfloat16 w1 = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(w1);
+    planes[i] = w0;
+    planes[n + i] = w1;
+    planes[2 * n + i] = __float2bfloat16_rn(r2);
+  }
+}
+
+template <int EP>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                     const RtParams p) {
+  using G = RtGeo<EP>;
+  constexpr int STAGES = G::STAGES;
+  constexpr uint32_t IDESC = idesc_bf16_f32(BM, EP);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* stages = smem_raw + pad;
+  RtCtl* ctl = reinterpret_cast<RtCtl*>(stages + STAGES * G::STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&ctl->tfull[a], 1); mbar_init(&ctl->tempty[a], 128); }
+    mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  for (int i = threadIdx.x; i < 4 * kRouterTcMaxE; i += NUM_THREADS) {
+    (&ctl->hist[0][0])[i] = 0;
+    (&ctl->cnt1[0][0])[i] = 0;
+  }
+  if (warp == 1) tmem_alloc(&ctl->tmem_slot, G::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {  // ---------------------------------------------- TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_phase[STAGES];
+      bool issued[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) { issued[s] = false; issued_phase[s] = 0; }
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait_or_abort(&ctl->empty[stage], phase ^ 1u, &ctl->abort, p.err, p.limit_ns)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = stages + stage * G::STAGE_BYTES;
+          mbar_arrive_expect_tx(&ctl->full[stage], G::STAGE_BYTES);
+          tma_load_2d(sa, &tmX, &ctl->full[stage], kb * BK, tile * BM);
+#pragma unroll
+          for (int pl = 0; pl < 3; ++pl)
+            tma_load_2d(sa + A_BYTES + pl * G::B_PLANE, &tmW, &ctl->full[stage], kb * BK, pl * EP);
+          issued[stage] = true;
+          issued_phase[stage] = phase;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      for (int s = 0; s < STAGES; ++s)
+        if (issued[s]) mbar_wait(&ctl->full[s], issued_phase[s], p.limit_ns);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // ---------------------------------------------- MMA issuer
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait_or_abort(&ctl->tempty[acc], acc_phase ^ 1u, &ctl->abort, p.err, p.limit_ns)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * EP);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait_or_abort(&ctl->full[stage], phase, &ctl->abort, p.err, p.limit_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stages + stage * G::STAGE_BYTES);
+#pragma unroll
+          for (int pl = 0; pl < 3; ++pl) {
+            const uint32_t sb = sa + A_BYTES + pl * G::B_PLANE;
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)
+              umma_bf16(d_tmem, sdesc_k_sw128(sa + k * 32), sdesc_k_sw128(sb + k * 32), IDESC,
+                        (kb | pl | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(&ctl->empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&ctl->tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      umma_commit(&ctl->drain);
+      mbar_wait(&ctl->drain, 0, p.limit_ns);
+    }
+  } else {  // ---------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter = 32-token router block within the tile
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    const int E = p.E, K = p.k;
+    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
+      const bool ok = __all_sync(0xffffffffu,
+                                 mbar_wait_or_abort(&ctl->tfull[acc], acc_phase, &ctl->abort, p.err, p.limit_ns));
+      if (!ok) break;
+      tc_fence_after();
+      const int64_t tok = static_cast<int64_t>(tile) * BM + q * 32 + lane;
+      const bool valid = tok < p.T;
+      const int blk = tile * 4 + q;
+      const bool blk_valid = blk < p.nblk;
+      const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * EP);
+
+      // pass 1: logits, max, top-k (value desc, index asc) in one scan over e
+      float m = -INFINITY;
+      float tv[8];
+      int te[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { tv[j] = -INFINITY; te[j] = 0x7fffffff; }
+#pragma unroll 1
+      for (int c0 = 0; c0 < EP; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(ta + c0, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int e = c0 + i;
+          if (e >= E) break;
+          float h = __uint_as_float(r[i]);
+          if (p.b_r != nullptr) h += __ldg(p.b_r + e);
+          if (h != h) h = -INFINITY;  // NaN logits (out of contract) rank last
+          if (valid && p.logits_out != nullptr) p.logits_out[tok * E + e] = h;
+          m = fmaxf(m, h);
+          if (h > tv[K - 1] || te[K - 1] == 0x7fffffff) {
+            int j = K - 1;
+            while (j > 0 && (tv[j - 1] < h || te[j - 1] == 0x7fffffff)) {
+              tv[j] = tv[j - 1];
+              te[j] = te[j - 1];
+              --j;
+            }
+            tv[j] = h;
+            te[j] = e;
+          }
+        }
+      }
+      // pass 2: sum of exp
+      float s = 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < EP; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(ta + c0, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int e = c0 + i;
+          if (e >= E) break;
+          float h = __uint_as_float(r[i]);
+          if (p.b_r != nullptr) h += __ldg(p.b_r + e);
+          if (h != h) h = -INFINITY;
+          s += expf(h - m);
+        }
+      }
+      const float inv_s = 1.f / s;
+      const float lse = m + logf(s);
+      // pass 3: per-expert probability sums of this 32-token block (fixed shuffle tree)
+#pragma unroll 1
+      for (int c0 = 0; c0 < EP; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(ta + c0, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int e = c0 + i;
+          if (e >= E) break;
+          float h = __uint_as_float(r[i]);
+          if (p.b_r != nullptr) h += __ldg(p.b_r + e);
+          if (h != h) h = -INFINITY;
+          const float ps = warp_sum_f(valid ? expf(h - m) * inv_s : 0.f);
+          if (lane == 0 && blk_valid) p.part_psum[e * p.nblk + blk] = ps;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&ctl->tempty[acc]);  // accumulator consumed
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+
+      // gates, outputs and block counts
+      if (valid) {
+        float den = 0.f;
+        if (p.gate_mode != 0)
+          for (int j = 0; j < K; ++j) den += expf(tv[j] - tv[0]);
+        for (int j = 0; j < K; ++j) {
+          const float g = (p.gate_mode == 0) ? expf(tv[j] - m) * inv_s : expf(tv[j] - tv[0]) / den;
+          const int e = (te[j] >= 0 && te[j] < E) ? te[j] : 0;
+          p.topk_idx[tok * K + j] = te[j];
+          p.topk_gate[tok * K + j] = g;
+          atomicAdd(&ctl->hist[q][e], 1);
+          if (j == 0) atomicAdd(&ctl->cnt1[q][e], 1);
+        }
+        if (p.lse_out != nullptr) p.lse_out[tok] = lse;
+      }
+      const float l2 = warp_sum_f(valid ? lse * lse : 0.f);
+      __syncwarp();
+      if (blk_valid) {
+        if (lane == 0) p.part_lse2[blk] = l2;
+        for (int e = lane; e < E; e += 32) {
+          p.part_hist[e * p.nblk + blk] = ctl->hist[q][e];
+          p.part_cnt1[e * p.nblk + blk] = ctl->cnt1[q][e];
+        }
+      }
+      __syncwarp();
+      for (int e = lane; e < E; e += 32) { ctl->hist[q][e] = 0; ctl->cnt1[q][e] = 0; }
+      __syncwarp();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, G::TMEM_COLS);
+  }
+}
+
+template <int EP>
+cudaError_t launch_ep(const RoutingArgs& a, void* wsplit, int num_sms, unsigned int* err, cudaStream_t s,
+                      const char** why) {
+  using G = RtGeo<EP>;
+  static_assert(G::STAGES >= 2, "router stages");
+  CUtensorMap mx, mw;
+  if (!make_map_bf16(&mx, a.x, static_cast<uint64_t>(a.T), static_cast<uint64_t>(a.d), BM) ||
+      !make_map_bf16(&mw, wsplit, static_cast<uint64_t>(3 * EP), static_cast<uint64_t>(a.d), EP)) {
+    *why = "router: cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  RtParams p;
+  p.T = a.T;
+  p.E = a.E;
+  p.k = a.k;
+  p.d = a.d;
+  p.gate_mode = a.gate_mode;
+  p.num_kb = (a.d + BK - 1) / BK;
+  p.nblk = a.nblk;
+  p.n_tiles = static_cast<int>((a.T + BM - 1) / BM);
+  p.b_r = a.b_r;
+  p.topk_idx = a.topk_idx;
+  p.topk_gate = a.topk_gate;
+  p.part_hist = a.part_hist;
+  p.part_cnt1 = a.part_cnt1;
+  p.part_psum = a.part_psum;
+  p.part_lse2 = a.part_lse2;
+  p.logits_out = a.logits_out;
+  p.lse_out = a.lse_out;
+  p.err = err;
+  p.limit_ns = kWaitLimitNs;
+
+  const int64_t n = static_cast<int64_t>(EP) * a.d;
+  const int sblocks = static_cast<int>((n + 255) / 256 < 4 * num_sms ? (n + 255) / 256 : 4 * num_sms);
+  split_router_kernel<<<sblocks, 256, 0, s>>>(a.W_r, a.E, EP, a.d, static_cast<__nv_bfloat16*>(wsplit));
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = set_smem_limit_once(reinterpret_cast<const void*>(&router_tc_kernel<EP>), static_cast<int>(G::SMEM));
+  if (e != cudaSuccess) return e;
+  const int grid = p.n_tiles < num_sms ? p.n_tiles : num_sms;
+  router_tc_kernel<EP><<<grid, NUM_THREADS, G::SMEM, s>>>(mx, mw, p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_router_tc(const RoutingArgs& a, void* wsplit, int num_sms, unsigned int* err, cudaStream_t s,
+                             const char** why) {
+  *why = nullptr;
+  const int EP = router_pad_e(a.E);
+  if (EP <= 16) return launch_ep<16>(a, wsplit, num_sms, err, s, why);
+  if (EP <= 32) return launch_ep<32>(a, wsplit, num_sms, err, s, why);
+  if (EP <= 64) return launch_ep<64>(a, wsplit, num_sms, err, s, why);
+  if (EP <= 128) return launch_ep<128>(a, wsplit, num_sms, err, s, why);
+  *why = "router: tensor-core router supports at most 128 experts";
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

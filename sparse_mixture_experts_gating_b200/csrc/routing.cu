@@ -229,8 +229,7 @@ template <typename XT, int TE>
 cudaError_t launch_router_t(const RoutingArgs& a, cudaStream_t s) {
   constexpr int EP = 16 * TE;
   const size_t smem = sizeof(float) * (BT * KP + EP * KP + BT * (EP + 1) + 4 * EP + 4) + sizeof(int) * 2 * EP;
-  cudaError_t e = cudaFuncSetAttribute(router_kernel<XT, TE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void*>(&router_kernel<XT, TE>), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   router_kernel<XT, TE><<<a.nblk, RT, smem, s>>>(a);
   count_launch();
