@@ -67,6 +67,8 @@ struct Ctl {
   volatile int abort;
   int mprefix[MAX_E + 1];
   int offsets[MAX_E + 1];
+  // epilogue staging, per epilogue warp: 32 rows x 128 B (+16 B pad)
+  alignas(16) uint8_t stage_out[4][32 * 144];
 };
 
 template <bool SPLIT>
@@ -161,10 +163,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued_phase[STAGES];
-      bool issued[STAGES];
-#pragma unroll
-      for (int s = 0; s < STAGES; ++s) { issued[s] = false; issued_phase[s] = 0; }
+      uint32_t issued = 0, issued_phase = 0;  // per-stage bits: a copy was issued / its phase
       bool ok = true;
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
         int e, mt, nt;
@@ -184,14 +183,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tma_load_2d(sa + B_OFF, &tmB0, &ctl->full[stage], kb * BK, brow);
             tma_load_2d(sa + B_OFF + B_HALF, &tmB0, &ctl->full[stage], kb * BK, brow + 128);
           }
-          issued[stage] = true;
-          issued_phase[stage] = phase;
+          issued |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
       // Drain: every issued copy must have landed before the CTA may exit.
       for (int s = 0; s < STAGES; ++s)
-        if (issued[s]) mbar_wait(&ctl->full[s], issued_phase[s], p.limit_ns);
+        if ((issued >> s) & 1u) mbar_wait(&ctl->full[s], (issued_phase >> s) & 1u, p.limit_ns);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -230,8 +229,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // Each warp owns 32 rows of the tile (its TMEM lane quarter).  Per chunk of
+    // 32 columns a lane computes its row's values, stages them in shared
+    // memory, and the warp then stores the 32 x 32 block with whole-row
+    // coalescing (8 rows x 64 B, or 4 rows x 128 B, per instruction).
+    const int q = warp & 3;
     const int r_in_tile = q * 32 + lane;
+    uint8_t* stg = reinterpret_cast<uint8_t*>(ctl->stage_out[q]);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x) {
@@ -242,125 +246,109 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const int m_local = mt * BM + r_in_tile;
       const bool vrow = m_local < ctl->offsets[e + 1] - ctl->offsets[e];
-      const int64_t row = ctl->offsets[e] + m_local;
+      const int row = ctl->offsets[e] + m_local;  // expert-sorted row of this lane
       const int n0 = nt * p.bn;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * MMA_N);
+      // destination row of each 32-row block row this lane stores (for bf16: rows lane/4 + 8i)
+      int drow[4];
+      bool dval[4];
+      const float g = (EPI == EPI_GATE_F32 || EPI == EPI_GATE_SCATTER_BF16) && vrow ? p.row_gate[row] : 0.f;
+      const int my_dst = (EPI == EPI_GATE_SCATTER_BF16) ? (vrow ? p.row_token[row] : 0) : row;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int src = (lane >> 2) + 8 * i;
+        drow[i] = __shfl_sync(0xffffffffu, my_dst, src);
+        dval[i] = __shfl_sync(0xffffffffu, vrow ? 1 : 0, src) != 0;
+      }
 
-      if (EPI == EPI_SWIGLU_BF16) {
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.N;
-        __nv_bfloat16* out_lo = OUT_SPLIT ? static_cast<__nv_bfloat16*>(p.out_lo) + row * p.N : nullptr;
+      if (EPI == EPI_SWIGLU_BF16 || EPI == EPI_RELU_BF16 || EPI == EPI_GATE_SCATTER_BF16) {
+        constexpr int NCH = (EPI == EPI_SWIGLU_BF16) ? 4 : 8;
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+        __nv_bfloat16* out_lo = static_cast<__nv_bfloat16*>(p.out_lo);
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t ra[32], rb[32];
-          tmem_ld32(tb + c * 32, ra);
-          tmem_ld32(tb + 128 + c * 32, rb);
-          tmem_ld_wait();
-          const int col = n0 + c * 32;
-          if (vrow) {
+        for (int c = 0; c < NCH; ++c) {
+          uint32_t ra[32];
+          uint32_t hi[16], lo[16];
+          if (EPI == EPI_SWIGLU_BF16) {
+            uint32_t rb[32];
+            tmem_ld32(tb + c * 32, ra);
+            tmem_ld32(tb + 128 + c * 32, rb);
+            tmem_ld_wait();
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              if (col + v * 8 < p.N) {
-                uint4 pk, pl;
-                uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
-                uint32_t* wl = reinterpret_cast<uint32_t*>(&pl);
+            for (int i = 0; i < 16; ++i) {
+              const float h0 = silu_mul(__uint_as_float(ra[2 * i]), __uint_as_float(rb[2 * i]));
+              const float h1 = silu_mul(__uint_as_float(ra[2 * i + 1]), __uint_as_float(rb[2 * i + 1]));
+              if (OUT_SPLIT) split_bf16(h0, h1, hi[i], lo[i]);
+              else hi[i] = pack_bf16x2(h0, h1);
+            }
+          } else {
+            tmem_ld32(tb + c * 32, ra);
+            tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const int j = v * 8 + 2 * i;
-                  const float h0 = silu_mul(__uint_as_float(ra[j]), __uint_as_float(rb[j]));
-                  const float h1 = silu_mul(__uint_as_float(ra[j + 1]), __uint_as_float(rb[j + 1]));
-                  if (OUT_SPLIT) split_bf16(h0, h1, w[i], wl[i]);
-                  else w[i] = pack_bf16x2(h0, h1);
-                }
-                *reinterpret_cast<uint4*>(out + col + v * 8) = pk;
-                if (OUT_SPLIT) *reinterpret_cast<uint4*>(out_lo + col + v * 8) = pl;
+            for (int i = 0; i < 16; ++i) {
+              float h0 = __uint_as_float(ra[2 * i]), h1 = __uint_as_float(ra[2 * i + 1]);
+              if (EPI == EPI_RELU_BF16) {
+                h0 = fmaxf(h0, 0.f);
+                h1 = fmaxf(h1, 0.f);
+              } else {
+                h0 *= g;
+                h1 *= g;
               }
+              if (OUT_SPLIT) split_bf16(h0, h1, hi[i], lo[i]);
+              else hi[i] = pack_bf16x2(h0, h1);
+            }
+            if (EPI == EPI_GATE_SCATTER_BF16 && p.out_f32 != nullptr && vrow) {  // debug copy
+              float* of = p.out_f32 + static_cast<int64_t>(my_dst) * p.N + n0 + c * 32;
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (n0 + c * 32 + i < p.N) of[i] = __uint_as_float(ra[i]) * g;
             }
           }
+          const int col = n0 + c * 32;
+#pragma unroll
+          for (int plane = 0; plane < (OUT_SPLIT ? 2 : 1); ++plane) {
+            const uint32_t* src = plane == 0 ? hi : lo;
+            uint4* srow = reinterpret_cast<uint4*>(stg + lane * 80);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) srow[v] = make_uint4(src[4 * v], src[4 * v + 1], src[4 * v + 2], src[4 * v + 3]);
+            __syncwarp();
+            __nv_bfloat16* dst = plane == 0 ? out : out_lo;
+            const int seg = lane & 3;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int rr = (lane >> 2) + 8 * i;
+              if (dval[i] && col + seg * 8 < p.N)
+                *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(drow[i]) * p.N + col + seg * 8) =
+                    *reinterpret_cast<const uint4*>(stg + rr * 80 + seg * 16);
+            }
+            __syncwarp();
+          }
         }
-      } else if (EPI == EPI_RELU_BF16) {
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.N;
-        __nv_bfloat16* out_lo = OUT_SPLIT ? static_cast<__nv_bfloat16*>(p.out_lo) + row * p.N : nullptr;
+      } else {  // EPI_GATE_F32: gated fp32 rows of the expert-sorted buffer
+        float* out = static_cast<float*>(p.out);
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           uint32_t ra[32];
           tmem_ld32(tb + c * 32, ra);
           tmem_ld_wait();
+          float4* srow = reinterpret_cast<float4*>(stg + lane * 144);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            srow[v] = make_float4(__uint_as_float(ra[4 * v]) * g, __uint_as_float(ra[4 * v + 1]) * g,
+                                  __uint_as_float(ra[4 * v + 2]) * g, __uint_as_float(ra[4 * v + 3]) * g);
+          __syncwarp();
           const int col = n0 + c * 32;
-          if (vrow) {
+          const int seg = lane & 7;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              if (col + v * 8 < p.N) {
-                uint4 pk, pl;
-                uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
-                uint32_t* wl = reinterpret_cast<uint32_t*>(&pl);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const int j = v * 8 + 2 * i;
-                  const float h0 = fmaxf(__uint_as_float(ra[j]), 0.f);
-                  const float h1 = fmaxf(__uint_as_float(ra[j + 1]), 0.f);
-                  if (OUT_SPLIT) split_bf16(h0, h1, w[i], wl[i]);
-                  else w[i] = pack_bf16x2(h0, h1);
-                }
-                *reinterpret_cast<uint4*>(out + col + v * 8) = pk;
-                if (OUT_SPLIT) *reinterpret_cast<uint4*>(out_lo + col + v * 8) = pl;
-              }
-            }
+          for (int i = 0; i < 8; ++i) {
+            const int rr = (lane >> 3) + 4 * i;
+            const int dr = __shfl_sync(0xffffffffu, row, rr);
+            const bool dv = __shfl_sync(0xffffffffu, vrow ? 1 : 0, rr) != 0;
+            if (dv && col + seg * 4 < p.N)
+              *reinterpret_cast<float4*>(out + static_cast<int64_t>(dr) * p.N + col + seg * 4) =
+                  *reinterpret_cast<const float4*>(stg + rr * 144 + seg * 16);
           }
-        }
-      } else {
-        const float g = vrow ? p.row_gate[row] : 0.f;
-        if (EPI == EPI_GATE_F32) {
-          float* out = static_cast<float*>(p.out) + row * p.N;
-#pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t ra[32];
-            tmem_ld32(tb + c * 32, ra);
-            tmem_ld_wait();
-            const int col = n0 + c * 32;
-            if (vrow) {
-#pragma unroll
-              for (int v = 0; v < 8; ++v) {
-                if (col + v * 4 < p.N) {
-                  float4 o;
-                  o.x = __uint_as_float(ra[v * 4 + 0]) * g;
-                  o.y = __uint_as_float(ra[v * 4 + 1]) * g;
-                  o.z = __uint_as_float(ra[v * 4 + 2]) * g;
-                  o.w = __uint_as_float(ra[v * 4 + 3]) * g;
-                  *reinterpret_cast<float4*>(out + col + v * 4) = o;
-                }
-              }
-            }
-          }
-        } else {  // EPI_GATE_SCATTER_BF16: k == 1, write y[token] directly
-          const int64_t tok = vrow ? p.row_token[row] : 0;
-          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + tok * p.N;
-#pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t ra[32];
-            tmem_ld32(tb + c * 32, ra);
-            tmem_ld_wait();
-            const int col = n0 + c * 32;
-            if (vrow) {
-#pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                if (col + v * 8 < p.N) {
-                  uint4 pk;
-                  uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
-#pragma unroll
-                  for (int i = 0; i < 4; ++i) {
-                    const int j = v * 8 + 2 * i;
-                    w[i] = pack_bf16x2(__uint_as_float(ra[j]) * g, __uint_as_float(ra[j + 1]) * g);
-                  }
-                  *reinterpret_cast<uint4*>(out + col + v * 8) = pk;
-                  if (p.out_f32 != nullptr) {
-                    float* of = p.out_f32 + tok * p.N + col + v * 8;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) of[i] = __uint_as_float(ra[v * 8 + i]) * g;
-                  }
-                }
-              }
-            }
-          }
+          __syncwarp();
         }
       }
       tc_fence_before();

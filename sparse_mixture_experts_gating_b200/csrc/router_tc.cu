@@ -32,7 +32,7 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int NUM_THREADS = 192;
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int MAX_STAGES = 4;
+constexpr int MAX_STAGES = 8;  // small router tiles: a deep ring hides the TMA round trip
 
 struct RtParams {
   int64_t T;
@@ -60,6 +60,8 @@ struct RtCtl {
   volatile int abort;
   int hist[4][kRouterTcMaxE];
   int cnt1[4][kRouterTcMaxE];
+  float pstage[4][32][17];  // per epilogue warp: 32 tokens x 16 experts of probabilities
+  float bias[kRouterTcMaxE];
 };
 
 template <int EP>
@@ -95,7 +97,9 @@ __global__ void __launch_bounds__(256) split_router_kernel(const float* __restri
   }
 }
 
-template <int EP>
+// K (= top-k) is a template parameter so the running k-best list is indexed
+// statically and lives in registers.
+template <int EP, int K>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const RtParams p) {
@@ -121,6 +125,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     (&ctl->hist[0][0])[i] = 0;
     (&ctl->cnt1[0][0])[i] = 0;
   }
+  for (int e = threadIdx.x; e < kRouterTcMaxE; e += NUM_THREADS)
+    ctl->bias[e] = (p.b_r != nullptr && e < p.E) ? p.b_r[e] : 0.f;
   if (warp == 1) tmem_alloc(&ctl->tmem_slot, G::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
@@ -131,10 +137,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {  // ---------------------------------------------- TMA producer
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued_phase[STAGES];
-      bool issued[STAGES];
-#pragma unroll
-      for (int s = 0; s < STAGES; ++s) { issued[s] = false; issued_phase[s] = 0; }
+      uint32_t issued = 0, issued_phase = 0;  // per-stage bits: a copy was issued / its phase
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
         for (int kb = 0; kb < p.num_kb; ++kb) {
@@ -148,13 +151,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int pl = 0; pl < 3; ++pl)
             tma_load_2d(sa + A_BYTES + pl * G::B_PLANE, &tmW, &ctl->full[stage], kb * BK, pl * EP);
-          issued[stage] = true;
-          issued_phase[stage] = phase;
+          issued |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
       for (int s = 0; s < STAGES; ++s)
-        if (issued[s]) mbar_wait(&ctl->full[s], issued_phase[s], p.limit_ns);
+        if ((issued >> s) & 1u) mbar_wait(&ctl->full[s], (issued_phase >> s) & 1u, p.limit_ns);
     }
   } else if (warp == 1) {
     if (lane == 0) {  // ---------------------------------------------- MMA issuer
@@ -194,7 +197,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int q = warp & 3;  // TMEM lane quarter = 32-token router block within the tile
     int acc = 0;
     uint32_t acc_phase = 0;
-    const int E = p.E, K = p.k;
+    const int E = p.E;
     for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
       const bool ok = __all_sync(0xffffffffu,
                                  mbar_wait_or_abort(&ctl->tfull[acc], acc_phase, &ctl->abort, p.err, p.limit_ns));
@@ -206,12 +209,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool blk_valid = blk < p.nblk;
       const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * EP);
 
-      // pass 1: logits, max, top-k (value desc, index asc) in one scan over e
+      // pass 1: logits, max, top-k (value desc, index asc) in one scan over e.
+      // The k best are kept sorted in registers; a candidate enters by
+      // compare-and-swap down the list (strict >, so an equal logit never
+      // displaces the lower expert index seen first; once an entry moves, the
+      // rest of the list shifts down behind it).
       float m = -INFINITY;
-      float tv[8];
-      int te[8];
+      float tv[K];
+      int te[K];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) { tv[j] = -INFINITY; te[j] = 0x7fffffff; }
+      for (int j = 0; j < K; ++j) { tv[j] = -INFINITY; te[j] = 0x7fffffff; }
 #pragma unroll 1
       for (int c0 = 0; c0 < EP; c0 += 16) {
         uint32_t r[16];
@@ -220,25 +227,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int e = c0 + i;
-          if (e >= E) break;
-          float h = __uint_as_float(r[i]);
-          if (p.b_r != nullptr) h += __ldg(p.b_r + e);
-          if (h != h) h = -INFINITY;  // NaN logits (out of contract) rank last
-          if (valid && p.logits_out != nullptr) p.logits_out[tok * E + e] = h;
-          m = fmaxf(m, h);
-          if (h > tv[K - 1] || te[K - 1] == 0x7fffffff) {
-            int j = K - 1;
-            while (j > 0 && (tv[j - 1] < h || te[j - 1] == 0x7fffffff)) {
-              tv[j] = tv[j - 1];
-              te[j] = te[j - 1];
-              --j;
+          if (e < E) {
+            float h = __uint_as_float(r[i]) + ctl->bias[e];
+            if (h != h) h = -INFINITY;  // NaN logits (out of contract) rank last
+            if (valid && p.logits_out != nullptr) p.logits_out[tok * E + e] = h;
+            m = fmaxf(m, h);
+            if (h > tv[K - 1] || te[K - 1] == 0x7fffffff) {
+              float cv = h;
+              int ce = e;
+              bool shifting = false;
+#pragma unroll
+              for (int j = 0; j < K; ++j) {
+                if (shifting || cv > tv[j] || te[j] == 0x7fffffff) {
+                  shifting = true;
+                  const float tvj = tv[j];
+                  const int tej = te[j];
+                  tv[j] = cv;
+                  te[j] = ce;
+                  cv = tvj;
+                  ce = tej;
+                }
+              }
             }
-            tv[j] = h;
-            te[j] = e;
           }
         }
       }
-      // pass 2: sum of exp
+      // pass 2: s = sum_e exp(h - m)
       float s = 0.f;
 #pragma unroll 1
       for (int c0 = 0; c0 < EP; c0 += 16) {
@@ -248,16 +262,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int e = c0 + i;
-          if (e >= E) break;
-          float h = __uint_as_float(r[i]);
-          if (p.b_r != nullptr) h += __ldg(p.b_r + e);
-          if (h != h) h = -INFINITY;
-          s += expf(h - m);
+          if (e < E) {
+            float h = __uint_as_float(r[i]) + ctl->bias[e];
+            if (h != h) h = -INFINITY;
+            s += expf(h - m);
+          }
         }
       }
       const float inv_s = 1.f / s;
       const float lse = m + logf(s);
-      // pass 3: per-expert probability sums of this 32-token block (fixed shuffle tree)
+      // pass 3: per-expert probability sums of this 32-token block: the warp
+      // stages 32 tokens x 16 experts in shared memory and lane i sums column i
+      // over the tokens in order (fixed order: deterministic).
+      float* stg = &ctl->pstage[q][0][0];
 #pragma unroll 1
       for (int c0 = 0; c0 < EP; c0 += 16) {
         uint32_t r[16];
@@ -266,13 +283,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int e = c0 + i;
-          if (e >= E) break;
-          float h = __uint_as_float(r[i]);
-          if (p.b_r != nullptr) h += __ldg(p.b_r + e);
-          if (h != h) h = -INFINITY;
-          const float ps = warp_sum_f(valid ? expf(h - m) * inv_s : 0.f);
-          if (lane == 0 && blk_valid) p.part_psum[e * p.nblk + blk] = ps;
+          float pe = 0.f;
+          if (valid && e < E) {
+            float h = __uint_as_float(r[i]) + ctl->bias[e];
+            if (h != h) h = -INFINITY;
+            pe = expf(h - m) * inv_s;
+          }
+          stg[lane * 17 + i] = pe;
         }
+        __syncwarp();
+        if (lane < 16 && c0 + lane < E && blk_valid) {
+          float acc_p = 0.f;
+#pragma unroll 8
+          for (int t = 0; t < 32; ++t) acc_p += stg[t * 17 + lane];
+          p.part_psum[(c0 + lane) * p.nblk + blk] = acc_p;
+        }
+        __syncwarp();
       }
       tc_fence_before();
       mbar_arrive(&ctl->tempty[acc]);  // accumulator consumed
@@ -281,8 +307,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // gates, outputs and block counts
       if (valid) {
         float den = 0.f;
-        if (p.gate_mode != 0)
+        if (p.gate_mode != 0) {
+#pragma unroll
           for (int j = 0; j < K; ++j) den += expf(tv[j] - tv[0]);
+        }
+#pragma unroll
         for (int j = 0; j < K; ++j) {
           const float g = (p.gate_mode == 0) ? expf(tv[j] - m) * inv_s : expf(tv[j] - tv[0]) / den;
           const int e = (te[j] >= 0 && te[j] < E) ? te[j] : 0;
@@ -316,7 +345,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <int EP>
+template <int EP, int K>
 cudaError_t launch_ep(const RoutingArgs& a, void* wsplit, int num_sms, unsigned int* err, cudaStream_t s,
                       const char** why) {
   using G = RtGeo<EP>;
@@ -354,12 +383,27 @@ cudaError_t launch_ep(const RoutingArgs& a, void* wsplit, int num_sms, unsigned 
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = set_smem_limit_once(reinterpret_cast<const void*>(&router_tc_kernel<EP>), static_cast<int>(G::SMEM));
+  e = set_smem_limit_once(reinterpret_cast<const void*>(&router_tc_kernel<EP, K>), static_cast<int>(G::SMEM));
   if (e != cudaSuccess) return e;
   const int grid = p.n_tiles < num_sms ? p.n_tiles : num_sms;
-  router_tc_kernel<EP><<<grid, NUM_THREADS, G::SMEM, s>>>(mx, mw, p);
+  router_tc_kernel<EP, K><<<grid, NUM_THREADS, G::SMEM, s>>>(mx, mw, p);
   count_launch();
   return cudaGetLastError();
+}
+
+template <int EP>
+cudaError_t launch_k(const RoutingArgs& a, void* wsplit, int num_sms, unsigned int* err, cudaStream_t s,
+                     const char** why) {
+  switch (a.k) {
+    case 1: return launch_ep<EP, 1>(a, wsplit, num_sms, err, s, why);
+    case 2: return launch_ep<EP, 2>(a, wsplit, num_sms, err, s, why);
+    case 3: return launch_ep<EP, 3>(a, wsplit, num_sms, err, s, why);
+    case 4: return launch_ep<EP, 4>(a, wsplit, num_sms, err, s, why);
+    case 5: return launch_ep<EP, 5>(a, wsplit, num_sms, err, s, why);
+    case 6: return launch_ep<EP, 6>(a, wsplit, num_sms, err, s, why);
+    case 7: return launch_ep<EP, 7>(a, wsplit, num_sms, err, s, why);
+    default: return launch_ep<EP, 8>(a, wsplit, num_sms, err, s, why);
+  }
 }
 
 }  // namespace
@@ -368,10 +412,10 @@ cudaError_t launch_router_tc(const RoutingArgs& a, void* wsplit, int num_sms, un
                              const char** why) {
   *why = nullptr;
   const int EP = router_pad_e(a.E);
-  if (EP <= 16) return launch_ep<16>(a, wsplit, num_sms, err, s, why);
-  if (EP <= 32) return launch_ep<32>(a, wsplit, num_sms, err, s, why);
-  if (EP <= 64) return launch_ep<64>(a, wsplit, num_sms, err, s, why);
-  if (EP <= 128) return launch_ep<128>(a, wsplit, num_sms, err, s, why);
+  if (EP <= 16) return launch_k<16>(a, wsplit, num_sms, err, s, why);
+  if (EP <= 32) return launch_k<32>(a, wsplit, num_sms, err, s, why);
+  if (EP <= 64) return launch_k<64>(a, wsplit, num_sms, err, s, why);
+  if (EP <= 128) return launch_k<128>(a, wsplit, num_sms, err, s, why);
   *why = "router: tensor-core router supports at most 128 experts";
   return cudaErrorInvalidValue;
 }

@@ -253,22 +253,36 @@ __global__ void __launch_bounds__(1024) scan_kernel(RoutingArgs a) {
   __shared__ float s_psum[256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = a.E, nb = a.nblk;
+  constexpr int V = 8;  // blocks per lane loaded ahead of the dependent scan steps
   for (int e = warp; e < E; e += 32) {
     int run = 0, c1 = 0;
     float ps = 0.f;
-    for (int b0 = 0; b0 < nb; b0 += 32) {
-      const int b = b0 + lane;
-      const int h = b < nb ? a.part_hist[e * nb + b] : 0;
-      int incl = h;
+    for (int g0 = 0; g0 < nb; g0 += 32 * V) {
+      int hv[V], cv[V];
+      float pv[V];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
+      for (int v = 0; v < V; ++v) {  // independent loads first
+        const int b = g0 + v * 32 + lane;
+        const bool in = b < nb;
+        hv[v] = in ? a.part_hist[e * nb + b] : 0;
+        cv[v] = in ? a.part_cnt1[e * nb + b] : 0;
+        pv[v] = in ? a.part_psum[e * nb + b] : 0.f;
       }
-      if (b < nb) a.blockoff[e * nb + b] = run + incl - h;
-      run += __shfl_sync(0xffffffffu, incl, 31);
-      c1 += warp_sum_i(b < nb ? a.part_cnt1[e * nb + b] : 0);
-      ps += warp_sum(b < nb ? a.part_psum[e * nb + b] : 0.f);
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        const int b = g0 + v * 32 + lane;
+        if (g0 + v * 32 >= nb) break;
+        int incl = hv[v];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += u;
+        }
+        if (b < nb) a.blockoff[e * nb + b] = run + incl - hv[v];
+        run += __shfl_sync(0xffffffffu, incl, 31);
+        c1 += warp_sum_i(cv[v]);
+        ps += warp_sum(pv[v]);
+      }
     }
     if (lane == 0) { s_counts[e] = run; s_cnt1[e] = c1; s_psum[e] = ps; }
   }
@@ -375,7 +389,15 @@ __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
         const uint4* src = reinterpret_cast<const uint4*>(x + tok * d);
         uint4* dst = reinterpret_cast<uint4*>(Xp + static_cast<int64_t>(dest) * d);
         const int nv = static_cast<int>(static_cast<size_t>(d) * sizeof(XT) / 16);
-        for (int v = lane; v < nv; v += 32) dst[v] = src[v];
+        int v = lane;
+        for (; v + 96 < nv; v += 128) {  // four independent 16-byte loads in flight per lane
+          const uint4 a0 = src[v], a1 = src[v + 32], a2 = src[v + 64], a3 = src[v + 96];
+          dst[v] = a0;
+          dst[v + 32] = a1;
+          dst[v + 64] = a2;
+          dst[v + 96] = a3;
+        }
+        for (; v < nv; v += 32) dst[v] = src[v];
       } else {
         for (int c = lane; c < d; c += 32) Xp[static_cast<int64_t>(dest) * d + c] = x[tok * d + c];
       }
@@ -401,12 +423,16 @@ __global__ void __launch_bounds__(256) combine_kernel(int64_t T, int k, int d, c
   for (int j = 0; j < 8; ++j) dst[j] = j < k ? dest_row[t * k + j] : -1;
   if ((d & 3) == 0) {
     for (int v = lane; v < d / 4; v += 32) {
+      float4 u[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)  // all loads of the slots first (independent), then the ordered sum
+        u[j] = dst[j] >= 0 ? reinterpret_cast<const float4*>(Yp + static_cast<int64_t>(dst[j]) * d)[v]
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (dst[j] < 0) continue;
-        const float4 u = reinterpret_cast<const float4*>(Yp + static_cast<int64_t>(dst[j]) * d)[v];
-        acc.x += u.x; acc.y += u.y; acc.z += u.z; acc.w += u.w;
+        acc.x += u[j].x; acc.y += u[j].y; acc.z += u[j].z; acc.w += u[j].w;
       }
       if (yf != nullptr) reinterpret_cast<float4*>(yf + t * d)[v] = acc;
       if constexpr (sizeof(YT) == 2) {
