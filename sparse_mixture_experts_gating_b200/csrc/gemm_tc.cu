@@ -76,8 +76,12 @@ constexpr size_t smem_bytes() {
   return Geo<SPLIT>::STAGES * Geo<SPLIT>::STAGE_BYTES + sizeof(Ctl) + 1024;
 }
 
-// Tile L -> (expert, m-tile, n-tile); tiles are expert-major, then n, then m.
-__device__ __forceinline__ void decode_tile(int L, const Ctl* c, int E, int n_tiles, int& e, int& mt, int& nt) {
+// Tile L -> (expert, m-tile, n-tile, K range); tiles are expert-major, then n,
+// then m, then K range.
+__device__ __forceinline__ void decode_tile(int L, const Ctl* c, int E, int n_tiles, int ksplit, int& e, int& mt,
+                                            int& nt, int& ks) {
+  ks = L % ksplit;
+  L /= ksplit;
   int lo = 0, hi = E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -106,7 +110,8 @@ __device__ __forceinline__ bool wait_or_abort(Ctl* c, uint64_t* bar, uint32_t pa
   }
 }
 
-__device__ __forceinline__ float silu_mul(float a, float b) { return a / (1.f + __expf(-a)) * b; }
+// silu(a) * b with the fast divide (2 ulp; 0 once 1 + e^-a overflows, the limit of silu).
+__device__ __forceinline__ float silu_mul(float a, float b) { return __fdividef(a, 1.f + __expf(-a)) * b; }
 
 // bf16 pair (hi, lo) with hi = RNE(v) and lo = RNE(v - hi): hi + lo carries
 // about 16 significant bits of v.
@@ -156,7 +161,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_slot;
-  const int total = ctl->mprefix[p.E] * p.n_tiles;
+  const int total = ctl->mprefix[p.E] * p.n_tiles * p.ksplit;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -166,11 +171,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t issued = 0, issued_phase = 0;  // per-stage bits: a copy was issued / its phase
       bool ok = true;
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-        int e, mt, nt;
-        decode_tile(L, ctl, p.E, p.n_tiles, e, mt, nt);
+        int e, mt, nt, ks;
+        decode_tile(L, ctl, p.E, p.n_tiles, p.ksplit, e, mt, nt, ks);
         const int row0 = ctl->offsets[e] + mt * BM;
         const int brow = e * p.N + nt * p.bn;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        const int kb0 = ks * p.kb_per, kb1 = min(p.num_kb, kb0 + p.kb_per);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_or_abort(ctl, &ctl->empty[stage], phase ^ 1u, p)) { ok = false; break; }
           uint8_t* sa = stages + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
@@ -202,7 +208,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!wait_or_abort(ctl, &ctl->tempty[acc], acc_phase ^ 1u, p)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * MMA_N);
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        const int ks = L % p.ksplit;
+        const int kb0 = ks * p.kb_per, kb1 = min(p.num_kb, kb0 + p.kb_per);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_or_abort(ctl, &ctl->full[stage], phase, p)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(stages + stage * STAGE_BYTES);
@@ -210,7 +218,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             umma_bf16(d_tmem, sdesc_k_sw128(sa + k * 32), sdesc_k_sw128(sb + k * 32), IDESC,
-                      (kb | k) != 0 ? 1u : 0u);
+                      (kb != kb0 || k != 0) ? 1u : 0u);
           if (A_SPLIT) {
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k)
@@ -239,13 +247,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x) {
-      int e, mt, nt;
-      decode_tile(L, ctl, p.E, p.n_tiles, e, mt, nt);
+      int e, mt, nt, ks;
+      decode_tile(L, ctl, p.E, p.n_tiles, p.ksplit, e, mt, nt, ks);
       const bool ok = __all_sync(0xffffffffu, wait_or_abort(ctl, &ctl->tfull[acc], acc_phase, p));
       if (!ok) break;  // warp-uniform: tcgen05.ld below is .sync.aligned
       tc_fence_after();
       const int m_local = mt * BM + r_in_tile;
       const bool vrow = m_local < ctl->offsets[e + 1] - ctl->offsets[e];
+      if (!__any_sync(0xffffffffu, vrow)) {  // all 32 rows of this warp lie past the expert's group
+        tc_fence_before();
+        mbar_arrive(&ctl->tempty[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        continue;
+      }
       const int row = ctl->offsets[e] + m_local;  // expert-sorted row of this lane
       const int n0 = nt * p.bn;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * MMA_N);
@@ -324,8 +338,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             __syncwarp();
           }
         }
-      } else {  // EPI_GATE_F32: gated fp32 rows of the expert-sorted buffer
-        float* out = static_cast<float*>(p.out);
+      } else {  // EPI_GATE_F32: gated fp32 rows of the expert-sorted buffer (partial ks)
+        float* out = static_cast<float*>(p.out) + static_cast<int64_t>(ks) * p.split_stride;
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           uint32_t ra[32];
@@ -438,6 +452,9 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
   p.bn = (g.epi == EPI_SWIGLU_BF16) ? 128 : 256;
   p.n_tiles = (g.N + p.bn - 1) / p.bn;
   p.num_kb = (g.K + BK - 1) / BK;
+  p.ksplit = g.epi == EPI_GATE_F32 ? (g.ksplit < 1 ? 1 : (g.ksplit > p.num_kb ? p.num_kb : g.ksplit)) : 1;
+  p.kb_per = (p.num_kb + p.ksplit - 1) / p.ksplit;
+  p.split_stride = g.split_stride;
   p.out = g.out;
   p.out_lo = g.out2;
   p.out_f32 = g.out_f32;

@@ -58,15 +58,27 @@ cudaError_t launch_router(const RoutingArgs& a, cudaStream_t s);
 // into three bf16 planes [3][E_pad][d] (E_pad = E rounded up to 16) in `wsplit`.
 constexpr int kRouterTcMaxE = 128;
 inline int router_pad_e(int E) { return (E + 15) / 16 * 16; }
-cudaError_t launch_router_tc(const RoutingArgs& a, void* wsplit, int num_sms, unsigned int* err, cudaStream_t s,
-                             const char** why);
+// K ranges of the tensor-core router (split when the 128-token tiles alone
+// cannot occupy the GPU); the split CTAs exchange fp32 partial logits through
+// `partials` ([tiles][ksplit][128][E_pad]) and per-tile tickets.
+int router_ksplit(int64_t T, int d);
+size_t router_partials_bytes(int64_t T, int E, int d);
+cudaError_t launch_router_tc(const RoutingArgs& a, void* wsplit, void* partials, int num_sms, unsigned int* err,
+                             cudaStream_t s, const char** why);
 
 // bf16 [rows][cols] tensor map, box [box_rows][64], 128-byte swizzle.
 bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 cudaError_t launch_scan(const RoutingArgs& a, cudaStream_t s);
 cudaError_t launch_dispatch(const RoutingArgs& a, cudaStream_t s);
+// y_t = sum over kept choices j (in order j) of sum over the ksplit partials
+// (in order) of Yp[partial][dest_row[t][j]].
 cudaError_t launch_combine(int64_t T, int k, int d, int y_is_bf16, const int32_t* dest_row, const float* Yp,
-                           void* y, float* y_f32, cudaStream_t s);
+                           int ksplit, int64_t split_stride, void* y, float* y_f32, cudaStream_t s);
+
+// K ranges of the second projection: split K when the tiles alone cannot
+// occupy the GPU (small token counts), for a 148-SM B200.
+constexpr int kSplitTargetCtas = 148;
+int gemm2_ksplit(int64_t s_max, int E, int d, int d_ff);
 
 // Grouped GEMM epilogues
 enum GemmEpi { EPI_RELU_BF16 = 0, EPI_SWIGLU_BF16 = 1, EPI_GATE_F32 = 2, EPI_GATE_SCATTER_BF16 = 3 };
@@ -84,6 +96,8 @@ struct GemmArgs {
   const void* B1;  // [E][N][K]  (W3 for SwiGLU, else unused)
   void* out;       // Hp [S][N] | Yp [S][N] fp32 | y [T][N]
   void* out2;      // lo plane of a split Hp, else NULL
+  int ksplit;      // EPI_GATE_F32: K is cut into ksplit ranges, partial j written at out + j * split_stride
+  int64_t split_stride;
   float* out_f32;  // scatter epilogue only: optional fp32 copy of y
   const int32_t* offsets;
   const int32_t* mprefix;
@@ -95,6 +109,8 @@ struct GemmArgs {
 // Kernel parameters of the tensor-core grouped GEMM.
 struct TcParams {
   int E, N, K, n_tiles, bn, num_kb;
+  int ksplit, kb_per;      // K ranges per (expert, m-tile, n-tile) and k-blocks in each
+  int64_t split_stride;    // elements between the partial outputs of consecutive K ranges
   void* out;
   void* out_lo;     // first projection with a split hidden activation: the lo plane
   float* out_f32;   // scatter epilogue only: optional fp32 copy of y

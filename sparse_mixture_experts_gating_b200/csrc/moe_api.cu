@@ -73,6 +73,10 @@ cudaError_t device_info(DeviceInfo** out) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+int ksplit_of(const moe_layer& L, int64_t s_max) {
+  return (L.dtype == MOE_BF16 && !(L.k == 1)) ? gemm2_ksplit(s_max, L.E, L.d, L.d_ff) : 1;
+}
+
 int64_t capacity_of(const moe_layer& L, int64_t T) {
   if (!(L.capacity_factor > 0.0)) return -1;
   const double c = ceil(L.capacity_factor * static_cast<double>(T) * static_cast<double>(L.k) /
@@ -86,8 +90,9 @@ struct Layout {
   int nblk;
   bool need_yp;
   bool split;
+  int ksplit;
   size_t idx, gate, dest, row_token, row_gate, part_hist, part_cnt1, part_psum, part_lse2, blockoff, counts,
-      offsets, mprefix, scal, wsplit, Xp, Hp, Hp_lo, Yp, total;
+      offsets, mprefix, scal, wsplit, rpart, Xp, Hp, Hp_lo, Yp, total;
 };
 
 Layout make_layout(const moe_layer& L, int64_t T) {
@@ -119,10 +124,16 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   w.scal = take(64);
   const bool tc_router = L.dtype == MOE_BF16 && L.E <= kRouterTcMaxE;
   w.wsplit = take(tc_router ? 3 * sizeof(uint16_t) * router_pad_e(L.E) * static_cast<size_t>(L.d) : 0);
+  w.rpart = take(tc_router ? router_partials_bytes(T, L.E, L.d) : 0);
   w.Xp = take(elt * static_cast<size_t>(w.s_max) * L.d);
   w.Hp = take(elt * static_cast<size_t>(w.s_max) * L.d_ff);
   w.Hp_lo = take(w.split ? elt * static_cast<size_t>(w.s_max) * L.d_ff : 0);
-  w.Yp = take(w.need_yp ? sizeof(float) * static_cast<size_t>(w.s_max) * L.d : 0);
+  w.ksplit = ksplit_of(L, w.s_max);
+  // Yp holds ksplit partials of s_max rows; reserve the most any smaller batch
+  // needs as well, so a workspace sized for some T serves every smaller batch
+  int64_t yp_rows = w.ksplit * w.s_max;
+  for (int64_t s = 1; s < w.s_max && s <= 256; ++s) yp_rows = std::max<int64_t>(yp_rows, ksplit_of(L, s) * s);
+  w.Yp = take(w.need_yp ? sizeof(float) * static_cast<size_t>(yp_rows) * L.d : 0);
   w.total = o;
   return w;
 }
@@ -136,6 +147,19 @@ void record(const moe_debug* dbg, int stage, int which, cudaStream_t s) {
 }  // namespace
 
 void set_error_message(const char* msg) { t_err = msg; }
+
+int gemm2_ksplit(int64_t s_max, int E, int d, int d_ff) {
+  // most m-tiles the second projection can have: floor(S/128) full ones plus
+  // one partial per expert that holds rows
+  const int64_t mtiles = s_max / kTileM + std::min<int64_t>(E, s_max);
+  const int64_t base = mtiles * ((d + 255) / 256);
+  if (base <= 0 || base * 2 > kSplitTargetCtas) return 1;
+  const int64_t num_kb = (d_ff + 63) / 64;
+  const int64_t ks = std::min<int64_t>(kSplitTargetCtas / base, num_kb / 4);
+  if (ks <= 1) return 1;
+  const int64_t per = (num_kb + ks - 1) / ks;  // no empty K range
+  return static_cast<int>((num_kb + per - 1) / per);
+}
 
 cudaError_t set_smem_limit_once(const void* kernel, int bytes) {
   static std::mutex mu;
@@ -206,6 +230,7 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   const moe_layer& L = *h;
   if (T < 0) return fail(MOE_ERR_INVALID_ARG, "moe_forward: T < 0");
   if (T * L.k > 2147483647LL / 2) return fail(MOE_ERR_UNSUPPORTED, "moe_forward: T * k too large");
+  if (T * static_cast<int64_t>(L.d) >= 4294967296LL) return fail(MOE_ERR_UNSUPPORTED, "moe_forward: T * d too large");
   if (expert_counts == nullptr || dropped == nullptr || aux_loss == nullptr || z_loss == nullptr)
     return fail(MOE_ERR_INVALID_ARG, "moe_forward: a statistics output pointer is NULL");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -307,6 +332,9 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   g2.B1 = nullptr;
   g2.out = w.need_yp ? static_cast<void*>(ws + w.Yp) : y;
   g2.out_f32 = (w.need_yp || dbg == nullptr) ? nullptr : dbg->y_f32;
+  g2.ksplit = w.ksplit;
+  g2.split_stride = static_cast<int64_t>(w.s_max) * L.d;
+  g1.ksplit = 1;
 
   // Host-side preparation of both GEMM launches happens before the first launch.
   TcGemmPlan plan1, plan2;
@@ -325,7 +353,7 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   record(dbg, MOE_STAGE_ROUTER, 0, s);
   if (tc && L.E <= kRouterTcMaxE && r.logits_in == nullptr) {
     const char* why = nullptr;
-    ce = launch_router_tc(r, ws + w.wsplit, di->num_sms, di->err, s, &why);
+    ce = launch_router_tc(r, ws + w.wsplit, ws + w.rpart, di->num_sms, di->err, s, &why);
     if (why != nullptr) return fail(MOE_ERR_UNSUPPORTED, std::string("moe_forward: ") + why);
     if ((rc = check(ce, "router")) != MOE_OK) return rc;
   } else if ((rc = check(launch_router(r, s), "router")) != MOE_OK) {
@@ -350,7 +378,8 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   if (w.need_yp) {
     record(dbg, MOE_STAGE_COMBINE, 0, s);
     if ((rc = check(launch_combine(T, L.k, L.d, L.dtype == MOE_BF16, r.dest_row,
-                                   reinterpret_cast<const float*>(ws + w.Yp), y, dbg ? dbg->y_f32 : nullptr, s),
+                                   reinterpret_cast<const float*>(ws + w.Yp), w.ksplit,
+                                   static_cast<int64_t>(w.s_max) * L.d, y, dbg ? dbg->y_f32 : nullptr, s),
                     "combine")) != MOE_OK)
       return rc;
     record(dbg, MOE_STAGE_COMBINE, 1, s);

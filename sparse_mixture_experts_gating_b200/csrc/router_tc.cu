@@ -37,6 +37,9 @@ constexpr int MAX_STAGES = 8;  // small router tiles: a deep ring hides the TMA 
 struct RtParams {
   int64_t T;
   int E, k, d, gate_mode, num_kb, nblk, n_tiles;
+  int ksplit, kb_per;   // K ranges per tile (1: no split) and k-blocks per range
+  float* partials;      // [n_tiles][ksplit][128][EP] fp32 partial logits
+  int* tickets;         // [n_tiles] ranges finished (zeroed by the split kernel)
   const float* b_r;
   int32_t* topk_idx;
   float* topk_gate;
@@ -58,6 +61,7 @@ struct RtCtl {
   uint64_t drain;
   uint32_t tmem_slot;
   volatile int abort;
+  int last;  // this CTA finished the last K range of the tile
   int hist[4][kRouterTcMaxE];
   int cnt1[4][kRouterTcMaxE];
   float pstage[4][32][17];  // per epilogue warp: 32 tokens x 16 experts of probabilities
@@ -82,8 +86,11 @@ __device__ __forceinline__ float warp_sum_f(float v) {
 
 // Split W_r (fp32 [E][d]) into bf16 planes [3][EP][d]; rows E..EP-1 are zero.
 __global__ void __launch_bounds__(256) split_router_kernel(const float* __restrict__ W, int E, int EP, int d,
-                                                           __nv_bfloat16* __restrict__ planes) {
+                                                           __nv_bfloat16* __restrict__ planes, int* tickets,
+                                                           int n_tickets) {
   const int64_t n = static_cast<int64_t>(EP) * d;
+  if (tickets != nullptr)
+    for (int i = blockIdx.x * 256 + threadIdx.x; i < n_tickets; i += gridDim.x * 256) tickets[i] = 0;
   for (int64_t i = blockIdx.x * 256ll + threadIdx.x; i < n; i += static_cast<int64_t>(gridDim.x) * 256) {
     const int e = static_cast<int>(i / d);
     const float w = e < E ? W[i] : 0.f;
@@ -139,8 +146,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued = 0, issued_phase = 0;  // per-stage bits: a copy was issued / its phase
       bool ok = true;
-      for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+      for (int u = blockIdx.x; u < p.n_tiles * p.ksplit && ok; u += gridDim.x) {
+        const int tile = u / p.ksplit, ks = u - tile * p.ksplit;
+        const int kb0 = ks * p.kb_per, kb1 = min(p.num_kb, kb0 + p.kb_per);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_or_abort(&ctl->empty[stage], phase ^ 1u, &ctl->abort, p.err, p.limit_ns)) {
             ok = false;
             break;
@@ -164,11 +173,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+      for (int u = blockIdx.x; u < p.n_tiles * p.ksplit && ok; u += gridDim.x) {
         if (!mbar_wait_or_abort(&ctl->tempty[acc], acc_phase ^ 1u, &ctl->abort, p.err, p.limit_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * EP);
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        const int ks = u % p.ksplit;
+        const int kb0 = ks * p.kb_per, kb1 = min(p.num_kb, kb0 + p.kb_per);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_or_abort(&ctl->full[stage], phase, &ctl->abort, p.err, p.limit_ns)) {
             ok = false;
             break;
@@ -181,7 +192,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k)
               umma_bf16(d_tmem, sdesc_k_sw128(sa + k * 32), sdesc_k_sw128(sb + k * 32), IDESC,
-                        (kb | pl | k) != 0 ? 1u : 0u);
+                        (kb != kb0 || pl != 0 || k != 0) ? 1u : 0u);
           }
           umma_commit(&ctl->empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -198,11 +209,65 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     const int E = p.E;
-    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
+    for (int u = blockIdx.x; u < p.n_tiles * p.ksplit; u += gridDim.x) {
+      const int tile = u / p.ksplit, ks = u - tile * p.ksplit;
       const bool ok = __all_sync(0xffffffffu,
                                  mbar_wait_or_abort(&ctl->tfull[acc], acc_phase, &ctl->abort, p.err, p.limit_ns));
       if (!ok) break;
       tc_fence_after();
+      if (p.ksplit > 1) {
+        // Publish this K range's partial logits (row = TMEM lane); the CTA that
+        // finishes a tile's last range sums all ranges in order back into its
+        // accumulator and runs the epilogue; the others release theirs.
+        const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * EP);
+        float* prow = p.partials + ((static_cast<int64_t>(tile) * p.ksplit + ks) * BM + q * 32 + lane) * EP;
+#pragma unroll 1
+        for (int c0 = 0; c0 < EP; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(tq + c0, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(prow + c0 + i) = make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                                                                    __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+        }
+        __threadfence();
+        named_barrier(1, 128);  // all 128 rows of this range are written
+        if (threadIdx.x == 64) ctl->last = (atomicAdd(p.tickets + tile, 1) == p.ksplit - 1) ? 1 : 0;
+        named_barrier(1, 128);
+        if (!ctl->last) {
+          tc_fence_before();
+          mbar_arrive(&ctl->tempty[acc]);
+          if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+          continue;
+        }
+        __threadfence();
+        const float* prow0 = p.partials + (static_cast<int64_t>(tile) * p.ksplit * BM + q * 32 + lane) * EP;
+#pragma unroll 1
+        for (int c0 = 0; c0 < EP; c0 += 16) {
+          uint32_t r[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) r[i] = 0u;
+          float sum[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) sum[i] = 0.f;
+          for (int s2 = 0; s2 < p.ksplit; ++s2) {  // fixed order: deterministic
+            const float* src = prow0 + static_cast<int64_t>(s2) * BM * EP + c0;
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+              const float4 v4 = __ldcg(reinterpret_cast<const float4*>(src + i));
+              sum[i] += v4.x;
+              sum[i + 1] += v4.y;
+              sum[i + 2] += v4.z;
+              sum[i + 3] += v4.w;
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(sum[i]);
+          tmem_st16(tq + c0, r);
+        }
+        tmem_st_wait();
+      }
       const int64_t tok = static_cast<int64_t>(tile) * BM + q * 32 + lane;
       const bool valid = tok < p.T;
       const int blk = tile * 4 + q;
@@ -346,8 +411,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 template <int EP, int K>
-cudaError_t launch_ep(const RoutingArgs& a, void* wsplit, int num_sms, unsigned int* err, cudaStream_t s,
-                      const char** why) {
+cudaError_t launch_ep(const RoutingArgs& a, void* wsplit, void* partials, int num_sms, unsigned int* err,
+                      cudaStream_t s, const char** why) {
   using G = RtGeo<EP>;
   static_assert(G::STAGES >= 2, "router stages");
   CUtensorMap mx, mw;
@@ -365,6 +430,11 @@ cudaError_t launch_ep(const RoutingArgs& a, void* wsplit, int num_sms, unsigned 
   p.num_kb = (a.d + BK - 1) / BK;
   p.nblk = a.nblk;
   p.n_tiles = static_cast<int>((a.T + BM - 1) / BM);
+  p.ksplit = router_ksplit(a.T, a.d);
+  p.kb_per = (p.num_kb + p.ksplit - 1) / p.ksplit;
+  p.partials = static_cast<float*>(partials);
+  p.tickets = reinterpret_cast<int*>(static_cast<uint8_t*>(partials) +
+                                     static_cast<size_t>(p.n_tiles) * p.ksplit * BM * EP * sizeof(float));
   p.b_r = a.b_r;
   p.topk_idx = a.topk_idx;
   p.topk_gate = a.topk_gate;
@@ -379,43 +449,72 @@ cudaError_t launch_ep(const RoutingArgs& a, void* wsplit, int num_sms, unsigned 
 
   const int64_t n = static_cast<int64_t>(EP) * a.d;
   const int sblocks = static_cast<int>((n + 255) / 256 < 4 * num_sms ? (n + 255) / 256 : 4 * num_sms);
-  split_router_kernel<<<sblocks, 256, 0, s>>>(a.W_r, a.E, EP, a.d, static_cast<__nv_bfloat16*>(wsplit));
+  split_router_kernel<<<sblocks, 256, 0, s>>>(a.W_r, a.E, EP, a.d, static_cast<__nv_bfloat16*>(wsplit),
+                                              p.ksplit > 1 ? p.tickets : nullptr, p.n_tiles);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = set_smem_limit_once(reinterpret_cast<const void*>(&router_tc_kernel<EP, K>), static_cast<int>(G::SMEM));
   if (e != cudaSuccess) return e;
-  const int grid = p.n_tiles < num_sms ? p.n_tiles : num_sms;
+  const int units = p.n_tiles * p.ksplit;
+  const int grid = units < num_sms ? units : num_sms;
   router_tc_kernel<EP, K><<<grid, NUM_THREADS, G::SMEM, s>>>(mx, mw, p);
   count_launch();
   return cudaGetLastError();
 }
 
 template <int EP>
-cudaError_t launch_k(const RoutingArgs& a, void* wsplit, int num_sms, unsigned int* err, cudaStream_t s,
-                     const char** why) {
+cudaError_t launch_k(const RoutingArgs& a, void* wsplit, void* partials, int num_sms, unsigned int* err,
+                     cudaStream_t s, const char** why) {
   switch (a.k) {
-    case 1: return launch_ep<EP, 1>(a, wsplit, num_sms, err, s, why);
-    case 2: return launch_ep<EP, 2>(a, wsplit, num_sms, err, s, why);
-    case 3: return launch_ep<EP, 3>(a, wsplit, num_sms, err, s, why);
-    case 4: return launch_ep<EP, 4>(a, wsplit, num_sms, err, s, why);
-    case 5: return launch_ep<EP, 5>(a, wsplit, num_sms, err, s, why);
-    case 6: return launch_ep<EP, 6>(a, wsplit, num_sms, err, s, why);
-    case 7: return launch_ep<EP, 7>(a, wsplit, num_sms, err, s, why);
-    default: return launch_ep<EP, 8>(a, wsplit, num_sms, err, s, why);
+    case 1: return launch_ep<EP, 1>(a, wsplit, partials, num_sms, err, s, why);
+    case 2: return launch_ep<EP, 2>(a, wsplit, partials, num_sms, err, s, why);
+    case 3: return launch_ep<EP, 3>(a, wsplit, partials, num_sms, err, s, why);
+    case 4: return launch_ep<EP, 4>(a, wsplit, partials, num_sms, err, s, why);
+    case 5: return launch_ep<EP, 5>(a, wsplit, partials, num_sms, err, s, why);
+    case 6: return launch_ep<EP, 6>(a, wsplit, partials, num_sms, err, s, why);
+    case 7: return launch_ep<EP, 7>(a, wsplit, partials, num_sms, err, s, why);
+    default: return launch_ep<EP, 8>(a, wsplit, partials, num_sms, err, s, why);
   }
 }
 
 }  // namespace
 
-cudaError_t launch_router_tc(const RoutingArgs& a, void* wsplit, int num_sms, unsigned int* err, cudaStream_t s,
-                             const char** why) {
+int router_ksplit(int64_t T, int d) {
+  const int64_t tiles = (T + BM - 1) / BM;
+  const int64_t num_kb = (d + BK - 1) / BK;
+  if (tiles <= 0 || tiles > 16) return 1;  // none, or enough tiles: the exchange would cost more than it saves
+  int64_t ks = kSplitTargetCtas / tiles;
+  if (ks > 16) ks = 16;
+  if (ks > num_kb / 2) ks = num_kb / 2;
+  if (ks <= 1) return 1;
+  const int64_t per = (num_kb + ks - 1) / ks;  // no empty K range
+  return static_cast<int>((num_kb + per - 1) / per);
+}
+
+size_t router_partials_bytes(int64_t T, int E, int d) {
+  // the largest need over every batch size up to T, so a workspace sized for
+  // some T serves every smaller batch too
+  size_t best = 0;
+  const int64_t max_tiles = (T + BM - 1) / BM;
+  for (int64_t tiles = 1; tiles <= max_tiles && tiles <= 16; ++tiles) {
+    const int ks = router_ksplit(tiles * BM, d);
+    if (ks <= 1) continue;
+    const size_t need = static_cast<size_t>(tiles) * ks * BM * router_pad_e(E) * sizeof(float) +
+                        static_cast<size_t>(tiles) * 4;
+    if (need > best) best = need;
+  }
+  return best;
+}
+
+cudaError_t launch_router_tc(const RoutingArgs& a, void* wsplit, void* partials, int num_sms, unsigned int* err,
+                             cudaStream_t s, const char** why) {
   *why = nullptr;
   const int EP = router_pad_e(a.E);
-  if (EP <= 16) return launch_k<16>(a, wsplit, num_sms, err, s, why);
-  if (EP <= 32) return launch_k<32>(a, wsplit, num_sms, err, s, why);
-  if (EP <= 64) return launch_k<64>(a, wsplit, num_sms, err, s, why);
-  if (EP <= 128) return launch_k<128>(a, wsplit, num_sms, err, s, why);
+  if (EP <= 16) return launch_k<16>(a, wsplit, partials, num_sms, err, s, why);
+  if (EP <= 32) return launch_k<32>(a, wsplit, partials, num_sms, err, s, why);
+  if (EP <= 64) return launch_k<64>(a, wsplit, partials, num_sms, err, s, why);
+  if (EP <= 128) return launch_k<128>(a, wsplit, partials, num_sms, err, s, why);
   *why = "router: tensor-core router supports at most 128 experts";
   return cudaErrorInvalidValue;
 }

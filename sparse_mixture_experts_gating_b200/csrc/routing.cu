@@ -410,50 +410,78 @@ __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Combine: one warp per token; y_t = sum_{j kept} Yp[dest_row[t][j]], j ascending.
+// Combine: y_t = sum over kept choices j (ascending) of the slot's row of Yp
+// (summed over its K-range partials in order).  One thread per token and
+// group of 4 columns, so small batches still spread over many warps.
 template <typename YT>
 __global__ void __launch_bounds__(256) combine_kernel(int64_t T, int k, int d, const int32_t* __restrict__ dest_row,
-                                                      const float* __restrict__ Yp, YT* __restrict__ y,
-                                                      float* __restrict__ yf) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + warp;
-  if (t >= T) return;
-  int dst[8];
+                                                      const float* __restrict__ Yp, int ksplit, int64_t split_stride,
+                                                      YT* __restrict__ y, float* __restrict__ yf) {
+  const uint32_t vpr = static_cast<uint32_t>(d) >> 2;  // float4 groups per row (d % 4 == 0 on this path)
+  const uint32_t i = blockIdx.x * 256u + threadIdx.x;    // T * d / 4 < 2^32 (checked on the host)
+  if (i >= static_cast<uint32_t>(T) * vpr) return;
+  const uint32_t t32 = i / vpr;
+  const int64_t t = t32;
+  const int v = static_cast<int>(i - t32 * vpr);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (ksplit == 1) {
+    float4 u[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) dst[j] = j < k ? dest_row[t * k + j] : -1;
-  if ((d & 3) == 0) {
-    for (int v = lane; v < d / 4; v += 32) {
-      float4 u[8];
+    for (int j = 0; j < 8; ++j) {  // all loads first (independent), then the ordered sum
+      const int dst = j < k ? dest_row[t * k + j] : -1;
+      u[j] = dst >= 0 ? reinterpret_cast<const float4*>(Yp + static_cast<int64_t>(dst) * d)[v]
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 #pragma unroll
-      for (int j = 0; j < 8; ++j)  // all loads of the slots first (independent), then the ordered sum
-        u[j] = dst[j] >= 0 ? reinterpret_cast<const float4*>(Yp + static_cast<int64_t>(dst[j]) * d)[v]
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (dst[j] < 0) continue;
-        acc.x += u[j].x; acc.y += u[j].y; acc.z += u[j].z; acc.w += u[j].w;
-      }
-      if (yf != nullptr) reinterpret_cast<float4*>(yf + t * d)[v] = acc;
-      if constexpr (sizeof(YT) == 2) {
-        uint2 o;
-        o.x = pack_bf16x2(acc.x, acc.y);
-        o.y = pack_bf16x2(acc.z, acc.w);
-        reinterpret_cast<uint2*>(y + t * d)[v] = o;
-      } else {
-        reinterpret_cast<float4*>(y + t * d)[v] = acc;
-      }
+    for (int j = 0; j < 8; ++j) {
+      acc.x += u[j].x; acc.y += u[j].y; acc.z += u[j].z; acc.w += u[j].w;
     }
   } else {
-    for (int c = lane; c < d; c += 32) {
-      float acc = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (dst[j] >= 0) acc += Yp[static_cast<int64_t>(dst[j]) * d + c];
-      y[t * d + c] = YT(acc);
-      if (yf != nullptr) yf[t * d + c] = acc;
+    for (int j = 0; j < k; ++j) {
+      const int dst = dest_row[t * k + j];
+      if (dst < 0) continue;
+      float4 sj = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int ks = 0; ks < ksplit; ++ks) {
+        const float4 u = reinterpret_cast<const float4*>(Yp + static_cast<int64_t>(ks) * split_stride +
+                                                         static_cast<int64_t>(dst) * d)[v];
+        sj.x += u.x; sj.y += u.y; sj.z += u.z; sj.w += u.w;
+      }
+      acc.x += sj.x; acc.y += sj.y; acc.z += sj.z; acc.w += sj.w;
     }
   }
+  if (yf != nullptr) reinterpret_cast<float4*>(yf + t * d)[v] = acc;
+  if constexpr (sizeof(YT) == 2) {
+    uint2 o;
+    o.x = pack_bf16x2(acc.x, acc.y);
+    o.y = pack_bf16x2(acc.z, acc.w);
+    reinterpret_cast<uint2*>(y + t * d)[v] = o;
+  } else {
+    reinterpret_cast<float4*>(y + t * d)[v] = acc;
+  }
+}
+
+// Scalar combine for rows whose width is not a multiple of 4 (fp32 layers).
+template <typename YT>
+__global__ void __launch_bounds__(256) combine_scalar_kernel(int64_t T, int k, int d,
+                                                             const int32_t* __restrict__ dest_row,
+                                                             const float* __restrict__ Yp, int ksplit,
+                                                             int64_t split_stride, YT* __restrict__ y,
+                                                             float* __restrict__ yf) {
+  const uint32_t i = blockIdx.x * 256u + threadIdx.x;  // T * d < 2^32 (checked on the host)
+  if (i >= static_cast<uint32_t>(T) * static_cast<uint32_t>(d)) return;
+  const uint32_t t32 = i / static_cast<uint32_t>(d);
+  const int64_t t = t32;
+  const int c = static_cast<int>(i - t32 * static_cast<uint32_t>(d));
+  float acc = 0.f;
+  for (int j = 0; j < k; ++j) {
+    const int dst = dest_row[t * k + j];
+    if (dst < 0) continue;
+    float sj = 0.f;
+    for (int ks = 0; ks < ksplit; ++ks) sj += Yp[static_cast<int64_t>(ks) * split_stride + static_cast<int64_t>(dst) * d + c];
+    acc += sj;
+  }
+  y[t * d + c] = YT(acc);
+  if (yf != nullptr) yf[t * d + c] = acc;
 }
 
 // ---------------------------------------------------------------------------
@@ -489,12 +517,24 @@ cudaError_t launch_dispatch(const RoutingArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_combine(int64_t T, int k, int d, int y_is_bf16, const int32_t* dest_row, const float* Yp,
-                           void* y, float* y_f32, cudaStream_t s) {
-  const unsigned grid = static_cast<unsigned>((T + 7) / 8);
-  if (y_is_bf16)
-    combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(T, k, d, dest_row, Yp, static_cast<__nv_bfloat16*>(y), y_f32);
-  else
-    combine_kernel<float><<<grid, 256, 0, s>>>(T, k, d, dest_row, Yp, static_cast<float*>(y), y_f32);
+                           int ksplit, int64_t split_stride, void* y, float* y_f32, cudaStream_t s) {
+  if ((d & 3) == 0) {
+    const unsigned grid = static_cast<unsigned>((T * (d / 4) + 255) / 256);
+    if (y_is_bf16)
+      combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(T, k, d, dest_row, Yp, ksplit, split_stride,
+                                                          static_cast<__nv_bfloat16*>(y), y_f32);
+    else
+      combine_kernel<float><<<grid, 256, 0, s>>>(T, k, d, dest_row, Yp, ksplit, split_stride,
+                                                 static_cast<float*>(y), y_f32);
+  } else {
+    const unsigned grid = static_cast<unsigned>((T * d + 255) / 256);
+    if (y_is_bf16)
+      combine_scalar_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(T, k, d, dest_row, Yp, ksplit, split_stride,
+                                                                 static_cast<__nv_bfloat16*>(y), y_f32);
+    else
+      combine_scalar_kernel<float><<<grid, 256, 0, s>>>(T, k, d, dest_row, Yp, ksplit, split_stride,
+                                                        static_cast<float*>(y), y_f32);
+  }
   count_launch();
   return cudaGetLastError();
 }

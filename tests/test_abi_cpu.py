@@ -106,3 +106,34 @@ def test_workspace_and_forward_validation_without_gpu(L):
     assert "workspace" in L.moe_last_error().decode()
     L.moe_destroy(h)
     assert L.moe_destroy(None) == 0
+
+
+def test_workspace_sizing_is_defined_for_every_batch_size(L):
+    """Host-only sizing (no GPU): every T from 0 up, several layer shapes, both
+    hidden precisions; sizes never shrink as T grows."""
+    shapes = [(8, 2, 4096, 14336, 1, 1, 0.0, 1), (64, 1, 768, 3072, 0, 0, 1.25, 1),
+              (128, 4, 2048, 768, 1, 1, 2.0, 1), (4, 2, 32, 64, 0, 1, 0.0, 0), (256, 8, 64, 64, 0, 0, 0.5, 1),
+              (3, 2, 1032, 1160, 1, 1, 0.0, 1)]
+    for args in shapes:
+        rc, h = _create(L, *args)
+        assert rc == 0
+        for mode in (0, 1):
+            assert L.moe_set_hidden_precision(h, mode) == 0
+            prev = 0
+            for T in list(range(0, 300)) + [511, 512, 513, 2047, 2048, 2049, 8192, 16384]:
+                n = L.moe_workspace_bytes(h, T)
+                assert n >= prev and n % 256 == 0, (args, mode, T, n)
+                prev = n
+        L.moe_destroy(h)
+
+
+def test_static_scratch_limit_stated_in_the_header_holds(L):
+    """The header's example limit of moe_forward_static matches the sizing."""
+    m = re.search(r"d_ff 14336 SwiGLU layer up to T = (\d+)\)", open(HEADER).read())
+    assert m, "example limit not found in include/moe.h"
+    stated = int(m.group(1))
+    rc, h = _create(L, 8, 2, 4096, 14336, 1, 1, 0.0, 1)
+    assert rc == 0
+    lim = 32 << 20
+    assert L.moe_workspace_bytes(h, stated) <= lim < L.moe_workspace_bytes(h, stated + 1)
+    L.moe_destroy(h)

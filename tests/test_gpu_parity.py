@@ -40,6 +40,8 @@ SMALL = [
     ("fp32_swiglu_switch_cap", 301, 48, 6, 3, 40, S, SW, 1.5, F32, "normal"),
     ("fp32_relu_e1", 130, 24, 1, 1, 72, R, SW, 0.0, F32, None),
     ("long_k_ragged", 333, 1032, 4, 2, 1160, S, RN, 0.0, BF, None),
+    ("decode_splitk", 3, 256, 8, 2, 1024, S, RN, 0.0, BF, None),          # K ranges of GEMM2 split
+    ("decode_splitk_ragged", 5, 136, 4, 2, 1160, R, SW, 0.0, BF, "normal"),
 ]
 
 
