@@ -202,6 +202,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream serialization attribute may start while the previous kernel of the
+// stream is still running: it does its own setup (barriers, TMEM, descriptor
+// prefetch), then pdl_wait() blocks until that kernel has completed and its
+// writes are visible; every read of its outputs and every global write comes
+// after.  pdl_trigger() lets the next kernel of the stream be scheduled.
+// Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Barrier among `nthreads` threads of the CTA on hardware barrier `id` (not 0).
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

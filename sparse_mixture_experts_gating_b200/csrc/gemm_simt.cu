@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(int E, int N, int K, con
                                                         const float* __restrict__ row_gate) {
   const int n = blockIdx.x * 32 + threadIdx.x;
   const int r = blockIdx.y * 8 + threadIdx.y;
+  pdl_wait();
+  pdl_trigger();
   if (r >= offsets[E] || n >= N) return;
   const int e = expert_of_row(offsets, E, r);
   const float* a = A + static_cast<int64_t>(r) * K;
@@ -60,17 +62,15 @@ cudaError_t launch_gemm_simt(const GemmArgs& g, int64_t s_max, cudaStream_t s) {
   float* out = static_cast<float*>(g.out);
   switch (g.epi) {
     case EPI_RELU_BF16:
-      simt_gemm_kernel<EPI_RELU_BF16><<<grid, block, 0, s>>>(g.E, g.N, g.K, A, B0, B1, out, g.offsets, g.row_gate);
-      break;
+      return launch_pdl(simt_gemm_kernel<EPI_RELU_BF16>, grid, block, 0, s, g.E, g.N, g.K, A, B0, B1, out, g.offsets,
+                        g.row_gate);
     case EPI_SWIGLU_BF16:
-      simt_gemm_kernel<EPI_SWIGLU_BF16><<<grid, block, 0, s>>>(g.E, g.N, g.K, A, B0, B1, out, g.offsets, g.row_gate);
-      break;
+      return launch_pdl(simt_gemm_kernel<EPI_SWIGLU_BF16>, grid, block, 0, s, g.E, g.N, g.K, A, B0, B1, out,
+                        g.offsets, g.row_gate);
     default:
-      simt_gemm_kernel<EPI_GATE_F32><<<grid, block, 0, s>>>(g.E, g.N, g.K, A, B0, B1, out, g.offsets, g.row_gate);
-      break;
+      return launch_pdl(simt_gemm_kernel<EPI_GATE_F32>, grid, block, 0, s, g.E, g.N, g.K, A, B0, B1, out, g.offsets,
+                        g.row_gate);
   }
-  count_launch();
-  return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -11,7 +11,11 @@
 // sharing a weight slab run at the same time and the slab is read from HBM once.
 //
 // Warp roles (192 threads, one CTA per SM):
-//   warp 0       TMA producer: A box [128 x 64] + two B boxes [128 x 64] per stage
+//   warp 0       TMA producer: A box [128 x 64] + two B boxes [128 x 64] per stage;
+//                with a single-plane A, a tile whose expert group ends inside it
+//                loads only the 16-row A boxes that hold rows of the group (the
+//                other smem rows keep stale data: they feed accumulator rows
+//                that are never stored)
 //   warp 1       TMEM allocator; lane 0 issues tcgen05.mma (M=128, N=256, K=16)
 //   warps 2..5   epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane per
 //                row), activation or gate, masked stores
@@ -39,6 +43,7 @@ constexpr int BK = 64;                   // bf16 per 128-byte smem row
 constexpr int MMA_N = 256;               // columns per MMA / accumulator
 constexpr int MAX_STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;     // 16 KB
+constexpr int A_SHORT = 16;              // rows per A box of a partly filled tile
 constexpr int B_HALF = 128 * BK * 2;     // 16 KB per B box
 constexpr int NUM_THREADS = 192;
 
@@ -76,22 +81,45 @@ constexpr size_t smem_bytes() {
   return Geo<SPLIT>::STAGES * Geo<SPLIT>::STAGE_BYTES + sizeof(Ctl) + 1024;
 }
 
-// Tile L -> (expert, m-tile, n-tile, K range); tiles are expert-major, then n,
-// then m, then K range.
-__device__ __forceinline__ void decode_tile(int L, const Ctl* c, int E, int n_tiles, int ksplit, int& e, int& mt,
-                                            int& nt, int& ks) {
-  ks = L % ksplit;
-  L /= ksplit;
+// Tile t -> (expert, m-tile, n-tile); tiles are expert-major, then n, then m.
+__device__ __forceinline__ void decode_tile(int t, const Ctl* c, int E, int n_tiles, int& e, int& mt, int& nt) {
   int lo = 0, hi = E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (c->mprefix[mid] * n_tiles <= L) lo = mid; else hi = mid;
+    if (c->mprefix[mid] * n_tiles <= t) lo = mid; else hi = mid;
   }
   e = lo;
-  const int local = L - c->mprefix[e] * n_tiles;
+  const int local = t - c->mprefix[e] * n_tiles;
   const int mtiles = c->mprefix[e + 1] - c->mprefix[e];
   nt = local / mtiles;
   mt = local - nt * mtiles;
+}
+
+// Work of one CTA, identical in every role: units u = blockIdx.x + j * gridDim.x
+// below tiles * ksplit; unit u is tile u / ksplit, K range u % ksplit
+// (ksplit > 1 only for the gated fp32 epilogue, whose partial outputs the
+// combine kernel sums in order).
+struct Item {
+  int tile, ks;    // tile and K-range index
+  int kb0, kb1;    // k-blocks [kb0, kb1)
+};
+struct ItemIter {
+  int u, units;
+};
+__device__ __forceinline__ ItemIter iter_begin(const Ctl* c, const Params& p) {
+  ItemIter it;
+  it.u = static_cast<int>(blockIdx.x);
+  it.units = c->mprefix[p.E] * p.n_tiles * p.ksplit;
+  return it;
+}
+__device__ __forceinline__ bool iter_next(ItemIter& it, const Params& p, Item& w) {
+  if (it.u >= it.units) return false;
+  w.tile = it.u / p.ksplit;
+  w.ks = it.u - w.tile * p.ksplit;
+  w.kb0 = w.ks * p.kb_per;
+  w.kb1 = min(p.num_kb, w.kb0 + p.kb_per);
+  it.u += static_cast<int>(gridDim.x);
+  return true;
 }
 
 __device__ __forceinline__ bool wait_or_abort(Ctl* c, uint64_t* bar, uint32_t parity, const Params& p) {
@@ -129,6 +157,7 @@ template <int EPI, bool SPLIT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                         const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                        const __grid_constant__ CUtensorMap tmAs, const __grid_constant__ CUtensorMap tmAs2,
                         const Params p) {
   constexpr bool A_SPLIT = SPLIT && (EPI == EPI_GATE_F32 || EPI == EPI_GATE_SCATTER_BF16);
   constexpr bool OUT_SPLIT = SPLIT && (EPI == EPI_RELU_BF16 || EPI == EPI_SWIGLU_BF16);
@@ -151,17 +180,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (A_SPLIT) tma_prefetch_desc(&tmA2);
     tma_prefetch_desc(&tmB0);
     tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(&tmAs);
+    if (A_SPLIT) tma_prefetch_desc(&tmAs2);
   }
+  if (warp == 1) tmem_alloc(&ctl->tmem_slot, TMEM_COLS);
+  pdl_wait();  // tile offsets and the A rows come from the kernels before
+  pdl_trigger();
   for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) {
     ctl->mprefix[i] = p.mprefix[i];
     ctl->offsets[i] = p.offsets[i];
   }
-  if (warp == 1) tmem_alloc(&ctl->tmem_slot, TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_slot;
-  const int total = ctl->mprefix[p.E] * p.n_tiles * p.ksplit;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -170,18 +202,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued = 0, issued_phase = 0;  // per-stage bits: a copy was issued / its phase
       bool ok = true;
-      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-        int e, mt, nt, ks;
-        decode_tile(L, ctl, p.E, p.n_tiles, p.ksplit, e, mt, nt, ks);
+      ItemIter it = iter_begin(ctl, p);
+      Item w;
+      while (ok && iter_next(it, p, w)) {
+        int e, mt, nt;
+        decode_tile(w.tile, ctl, p.E, p.n_tiles, e, mt, nt);
         const int row0 = ctl->offsets[e] + mt * BM;
         const int brow = e * p.N + nt * p.bn;
-        const int kb0 = ks * p.kb_per, kb1 = min(p.num_kb, kb0 + p.kb_per);
+        const int kb0 = w.kb0, kb1 = w.kb1;
+        // rows of the group in this tile (>= 1); 0 short boxes = one full box.
+        // Short boxes only for a single-plane A: with the hi + lo planes the
+        // extra copies cost more than the rows they save.
+        const int vrows = ctl->offsets[e + 1] - row0;
+        const int nshort = (A_SPLIT || vrows >= BM) ? 0 : (vrows + A_SHORT - 1) / A_SHORT;
+        const uint32_t a_bytes = nshort == 0 ? A_BYTES : nshort * A_SHORT * BK * 2;
+        const uint32_t tx = (A_SPLIT ? 2u : 1u) * a_bytes + 2u * B_HALF;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_or_abort(ctl, &ctl->empty[stage], phase ^ 1u, p)) { ok = false; break; }
           uint8_t* sa = stages + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
-          tma_load_2d(sa, &tmA, &ctl->full[stage], kb * BK, row0);
-          if (A_SPLIT) tma_load_2d(sa + A_BYTES, &tmA2, &ctl->full[stage], kb * BK, row0);
+          mbar_arrive_expect_tx(&ctl->full[stage], tx);
+          if (nshort == 0) {
+            tma_load_2d(sa, &tmA, &ctl->full[stage], kb * BK, row0);
+            if (A_SPLIT) tma_load_2d(sa + A_BYTES, &tmA2, &ctl->full[stage], kb * BK, row0);
+          } else {
+            for (int j = 0; j < nshort; ++j) {
+              tma_load_2d(sa + j * A_SHORT * BK * 2, &tmAs, &ctl->full[stage], kb * BK, row0 + j * A_SHORT);
+              if (A_SPLIT)
+                tma_load_2d(sa + A_BYTES + j * A_SHORT * BK * 2, &tmAs2, &ctl->full[stage], kb * BK,
+                            row0 + j * A_SHORT);
+            }
+          }
           if (EPI == EPI_SWIGLU_BF16) {
             tma_load_2d(sa + B_OFF, &tmB0, &ctl->full[stage], kb * BK, brow);
             tma_load_2d(sa + B_OFF + B_HALF, &tmB1, &ctl->full[stage], kb * BK, brow);
@@ -204,12 +254,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+      ItemIter it = iter_begin(ctl, p);
+      Item w;
+      while (ok && iter_next(it, p, w)) {
         if (!wait_or_abort(ctl, &ctl->tempty[acc], acc_phase ^ 1u, p)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * MMA_N);
-        const int ks = L % p.ksplit;
-        const int kb0 = ks * p.kb_per, kb1 = min(p.num_kb, kb0 + p.kb_per);
+        const int kb0 = w.kb0, kb1 = w.kb1;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_or_abort(ctl, &ctl->full[stage], phase, p)) { ok = false; break; }
           tc_fence_after();
@@ -246,9 +297,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint8_t* stg = reinterpret_cast<uint8_t*>(ctl->stage_out[q]);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x) {
-      int e, mt, nt, ks;
-      decode_tile(L, ctl, p.E, p.n_tiles, p.ksplit, e, mt, nt, ks);
+    ItemIter it = iter_begin(ctl, p);
+    Item w;
+    while (iter_next(it, p, w)) {
+      int e, mt, nt;
+      decode_tile(w.tile, ctl, p.E, p.n_tiles, e, mt, nt);
+      const int ks = w.ks;
       const bool ok = __all_sync(0xffffffffu, wait_or_abort(ctl, &ctl->tfull[acc], acc_phase, p));
       if (!ok) break;  // warp-uniform: tcgen05.ld below is .sync.aligned
       tc_fence_after();
@@ -426,9 +480,8 @@ cudaError_t launch_t(const TcGemmPlan& pl, int num_sms, cudaStream_t s) {
   cudaError_t e = set_smem_limit_once(reinterpret_cast<const void*>(&grouped_gemm_kernel<EPI, SPLIT>),
                                       static_cast<int>(bytes));
   if (e != cudaSuccess) return e;
-  grouped_gemm_kernel<EPI, SPLIT><<<num_sms, NUM_THREADS, bytes, s>>>(pl.a, pl.a2, pl.b0, pl.b1, pl.p);
-  count_launch();
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_kernel<EPI, SPLIT>, dim3(num_sms), dim3(NUM_THREADS), bytes, s, pl.a, pl.a2, pl.b0,
+                    pl.b1, pl.as, pl.as2, pl.p);
 }
 
 }  // namespace
@@ -439,6 +492,9 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
   const bool a_split = g.split && g.A2 != nullptr;
   if (!make_map(&pl->a, g.A, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K)) ||
       !make_map(&pl->a2, a_split ? g.A2 : g.A, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K)) ||
+      !make_map_bf16(&pl->as, g.A, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K), A_SHORT) ||
+      !make_map_bf16(&pl->as2, a_split ? g.A2 : g.A, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K),
+                     A_SHORT) ||
       !make_map(&pl->b0, g.B0, static_cast<uint64_t>(g.E) * g.N, static_cast<uint64_t>(g.K)) ||
       !make_map(&pl->b1, g.epi == EPI_SWIGLU_BF16 ? g.B1 : g.B0, static_cast<uint64_t>(g.E) * g.N,
                 static_cast<uint64_t>(g.K))) {

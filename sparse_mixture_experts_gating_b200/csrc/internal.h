@@ -125,6 +125,7 @@ struct TcParams {
 // Everything a tensor-core GEMM launch needs, prepared on the host up front.
 struct TcGemmPlan {
   CUtensorMap a, a2, b0, b1;
+  CUtensorMap as, as2;  // A and A2 with 16-row boxes, for tiles whose group ends inside the tile
   TcParams p;
   int epi;
   int split;
@@ -140,6 +141,27 @@ cudaError_t launch_gemm_simt(const GemmArgs& g, int64_t s_max, cudaStream_t s);
 cudaError_t launch_selftest_timeout(unsigned int* err, int64_t limit_ns, cudaStream_t s);
 
 void count_launch();
+
+// Launch `kernel` with programmatic dependent launch (the kernel calls
+// pdl_wait() before it touches what the previous kernel of the stream
+// wrote).  Every kernel of a forward pass except the first is launched so.
+template <typename... P, typename... A>
+inline cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<A&&>(args)...);
+  count_launch();
+  return e;
+}
 
 // Set the calling thread's moe_last_error() message.
 void set_error_message(const char* msg);

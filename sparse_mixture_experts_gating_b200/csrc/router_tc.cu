@@ -64,7 +64,7 @@ struct RtCtl {
   int last;  // this CTA finished the last K range of the tile
   int hist[4][kRouterTcMaxE];
   int cnt1[4][kRouterTcMaxE];
-  float pstage[4][32][17];  // per epilogue warp: 32 tokens x 16 experts of probabilities
+  float pstage[4][32][33];  // per epilogue warp: 32 tokens x 32 experts of probabilities
   float bias[kRouterTcMaxE];
 };
 
@@ -135,6 +135,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   for (int e = threadIdx.x; e < kRouterTcMaxE; e += NUM_THREADS)
     ctl->bias[e] = (p.b_r != nullptr && e < p.E) ? p.b_r[e] : 0.f;
   if (warp == 1) tmem_alloc(&ctl->tmem_slot, G::TMEM_COLS);
+  pdl_wait();  // the W_r planes and tickets come from the split kernel
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -219,17 +221,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // Publish this K range's partial logits (row = TMEM lane); the CTA that
         // finishes a tile's last range sums all ranges in order back into its
         // accumulator and runs the epilogue; the others release theirs.
+        // Rows past T carry no token: they neither publish nor read partials.
         const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * EP);
+        const bool row_live = static_cast<int64_t>(tile) * BM + q * 32 + lane < p.T;
         float* prow = p.partials + ((static_cast<int64_t>(tile) * p.ksplit + ks) * BM + q * 32 + lane) * EP;
 #pragma unroll 1
         for (int c0 = 0; c0 < EP; c0 += 16) {
           uint32_t r[16];
           tmem_ld16(tq + c0, r);
           tmem_ld_wait();
+          if (row_live) {
 #pragma unroll
-          for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(prow + c0 + i) = make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
-                                                                    __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+            for (int i = 0; i < 16; i += 4)
+              *reinterpret_cast<float4*>(prow + c0 + i) =
+                  make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
+                              __uint_as_float(r[i + 3]));
+          }
         }
         __threadfence();
         named_barrier(1, 128);  // all 128 rows of this range are written
@@ -246,20 +253,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll 1
         for (int c0 = 0; c0 < EP; c0 += 16) {
           uint32_t r[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) r[i] = 0u;
           float sum[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) sum[i] = 0.f;
-          for (int s2 = 0; s2 < p.ksplit; ++s2) {  // fixed order: deterministic
-            const float* src = prow0 + static_cast<int64_t>(s2) * BM * EP + c0;
+          // ranges in ascending order (deterministic), four loads in flight per batch
+#pragma unroll 1
+          for (int s0 = 0; row_live && s0 < p.ksplit; s0 += 4) {
+            float4 v[4][4];
 #pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-              const float4 v4 = __ldcg(reinterpret_cast<const float4*>(src + i));
-              sum[i] += v4.x;
-              sum[i + 1] += v4.y;
-              sum[i + 2] += v4.z;
-              sum[i + 3] += v4.w;
+            for (int u2 = 0; u2 < 4; ++u2) {
+              const float* src = prow0 + static_cast<int64_t>(s0 + u2) * BM * EP + c0;
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                v[u2][i] = s0 + u2 < p.ksplit ? __ldcg(reinterpret_cast<const float4*>(src + 4 * i))
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u2 = 0; u2 < 4; ++u2) {
+              if (s0 + u2 < p.ksplit) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  sum[4 * i] += v[u2][i].x;
+                  sum[4 * i + 1] += v[u2][i].y;
+                  sum[4 * i + 2] += v[u2][i].z;
+                  sum[4 * i + 3] += v[u2][i].w;
+                }
+              }
             }
           }
 #pragma unroll
@@ -274,31 +293,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool blk_valid = blk < p.nblk;
       const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * EP);
 
-      // pass 1: logits, max, top-k (value desc, index asc) in one scan over e.
-      // The k best are kept sorted in registers; a candidate enters by
-      // compare-and-swap down the list (strict >, so an equal logit never
-      // displaces the lower expert index seen first; once an entry moves, the
-      // rest of the list shifts down behind it).
-      float m = -INFINITY;
+      float m = -INFINITY, inv_s, lse;
       float tv[K];
       int te[K];
 #pragma unroll
       for (int j = 0; j < K; ++j) { tv[j] = -INFINITY; te[j] = 0x7fffffff; }
-#pragma unroll 1
-      for (int c0 = 0; c0 < EP; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(ta + c0, r);
-        tmem_ld_wait();
+      if constexpr (EP <= 64) {
+        // The token's EP logits come out of TMEM in one batch of loads and stay in
+        // registers: h = acc + bias, then the max and the top-k (value desc,
+        // index asc) in one scan over e.  The k best are kept sorted; a candidate
+        // enters by compare-and-swap down the list (strict >, so an equal logit
+        // never displaces the lower expert index seen first; once an entry moves,
+        // the rest of the list shifts down behind it).
+        float h[EP];
+        {
+          uint32_t hr[EP / 16][16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int e = c0 + i;
+          for (int c = 0; c < EP / 16; ++c) tmem_ld16(ta + c * 16, hr[c]);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < EP; ++e) h[e] = __uint_as_float(hr[e / 16][e % 16]);
+        }
+        tc_fence_before();
+        mbar_arrive(&ctl->tempty[acc]);  // accumulator consumed: the next tile's MMAs may start
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+#pragma unroll
+        for (int e = 0; e < EP; ++e) {
           if (e < E) {
-            float h = __uint_as_float(r[i]) + ctl->bias[e];
-            if (h != h) h = -INFINITY;  // NaN logits (out of contract) rank last
-            if (valid && p.logits_out != nullptr) p.logits_out[tok * E + e] = h;
-            m = fmaxf(m, h);
-            if (h > tv[K - 1] || te[K - 1] == 0x7fffffff) {
-              float cv = h;
+            float v = h[e] + ctl->bias[e];
+            if (v != v) v = -INFINITY;  // NaN logits (out of contract) rank last
+            h[e] = v;
+            if (valid && p.logits_out != nullptr) p.logits_out[tok * E + e] = v;
+            m = fmaxf(m, v);
+            if (v > tv[K - 1] || te[K - 1] == 0x7fffffff) {
+              float cv = v;
               int ce = e;
               bool shifting = false;
 #pragma unroll
@@ -316,58 +344,130 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-      }
-      // pass 2: s = sum_e exp(h - m)
-      float s = 0.f;
-#pragma unroll 1
-      for (int c0 = 0; c0 < EP; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(ta + c0, r);
-        tmem_ld_wait();
+        // s = sum_e exp(h - m): each exponential once (kept in h), four partial
+        // sums in a fixed order
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int e = c0 + i;
-          if (e < E) {
-            float h = __uint_as_float(r[i]) + ctl->bias[e];
-            if (h != h) h = -INFINITY;
-            s += expf(h - m);
+        for (int e = 0; e < EP; ++e) {
+          const float x = e < E ? expf(h[e] - m) : 0.f;
+          h[e] = x;
+          s4[e & 3] += x;
+        }
+        const float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        inv_s = 1.f / s;
+        lse = m + logf(s);
+        // per-expert probability sums of this 32-token block: the warp writes
+        // 32 tokens x 32 experts row-major into shared memory and lane j sums
+        // column j over the tokens in order (fixed order: deterministic)
+        float* stg = &ctl->pstage[q][0][0];
+#pragma unroll
+        for (int c0 = 0; c0 < EP; c0 += 32) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            stg[lane * 33 + i] = (c0 + i < EP && valid && c0 + i < E) ? h[(c0 + i) & (EP - 1)] * inv_s : 0.f;
+          __syncwarp();
+          float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+          for (int t = 0; t < 32; t += 2) {
+            a0 += stg[t * 33 + lane];
+            a1 += stg[(t + 1) * 33 + lane];
+          }
+          if (c0 + lane < E && blk_valid) p.part_psum[(c0 + lane) * p.nblk + blk] = a0 + a1;
+          __syncwarp();
+        }
+      } else {
+        // E_pad = 128: the same steps over 16-column chunks (re-read from TMEM in
+        // each pass), which keeps the code small enough for the instruction cache
+        // pass 1: logits, max, top-k (value desc, index asc) in one scan over e.
+        // The k best are kept sorted in registers; a candidate enters by
+        // compare-and-swap down the list (strict >, so an equal logit never
+        // displaces the lower expert index seen first; once an entry moves, the
+        // rest of the list shifts down behind it).
+#pragma unroll 1
+        for (int c0 = 0; c0 < EP; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(ta + c0, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = c0 + i;
+            if (e < E) {
+              float h = __uint_as_float(r[i]) + ctl->bias[e];
+              if (h != h) h = -INFINITY;  // NaN logits (out of contract) rank last
+              if (valid && p.logits_out != nullptr) p.logits_out[tok * E + e] = h;
+              m = fmaxf(m, h);
+              if (h > tv[K - 1] || te[K - 1] == 0x7fffffff) {
+                float cv = h;
+                int ce = e;
+                bool shifting = false;
+#pragma unroll
+                for (int j = 0; j < K; ++j) {
+                  if (shifting || cv > tv[j] || te[j] == 0x7fffffff) {
+                    shifting = true;
+                    const float tvj = tv[j];
+                    const int tej = te[j];
+                    tv[j] = cv;
+                    te[j] = ce;
+                    cv = tvj;
+                    ce = tej;
+                  }
+                }
+              }
+            }
           }
         }
-      }
-      const float inv_s = 1.f / s;
-      const float lse = m + logf(s);
-      // pass 3: per-expert probability sums of this 32-token block: the warp
-      // stages 32 tokens x 16 experts in shared memory and lane i sums column i
-      // over the tokens in order (fixed order: deterministic).
-      float* stg = &ctl->pstage[q][0][0];
+        // pass 2: s = sum_e exp(h - m)
+        float s = 0.f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < EP; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(ta + c0, r);
-        tmem_ld_wait();
+        for (int c0 = 0; c0 < EP; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(ta + c0, r);
+          tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int e = c0 + i;
-          float pe = 0.f;
-          if (valid && e < E) {
-            float h = __uint_as_float(r[i]) + ctl->bias[e];
-            if (h != h) h = -INFINITY;
-            pe = expf(h - m) * inv_s;
+          for (int i = 0; i < 16; ++i) {
+            const int e = c0 + i;
+            if (e < E) {
+              float h = __uint_as_float(r[i]) + ctl->bias[e];
+              if (h != h) h = -INFINITY;
+              s += expf(h - m);
+            }
           }
-          stg[lane * 17 + i] = pe;
         }
-        __syncwarp();
-        if (lane < 16 && c0 + lane < E && blk_valid) {
-          float acc_p = 0.f;
+        inv_s = 1.f / s;
+        lse = m + logf(s);
+        // pass 3: per-expert probability sums of this 32-token block: the warp
+        // stages 32 tokens x 16 experts in shared memory and lane i sums column i
+        // over the tokens in order (fixed order: deterministic).
+        float* stg = &ctl->pstage[q][0][0];
+#pragma unroll 1
+        for (int c0 = 0; c0 < EP; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(ta + c0, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = c0 + i;
+            float pe = 0.f;
+            if (valid && e < E) {
+              float h = __uint_as_float(r[i]) + ctl->bias[e];
+              if (h != h) h = -INFINITY;
+              pe = expf(h - m) * inv_s;
+            }
+            stg[lane * 17 + i] = pe;
+          }
+          __syncwarp();
+          if (lane < 16 && c0 + lane < E && blk_valid) {
+            float acc_p = 0.f;
 #pragma unroll 8
-          for (int t = 0; t < 32; ++t) acc_p += stg[t * 17 + lane];
-          p.part_psum[(c0 + lane) * p.nblk + blk] = acc_p;
+            for (int t = 0; t < 32; ++t) acc_p += stg[t * 17 + lane];
+            p.part_psum[(c0 + lane) * p.nblk + blk] = acc_p;
+          }
+          __syncwarp();
         }
-        __syncwarp();
+        tc_fence_before();
+        mbar_arrive(&ctl->tempty[acc]);  // accumulator consumed
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
-      tc_fence_before();
-      mbar_arrive(&ctl->tempty[acc]);  // accumulator consumed
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
 
       // gates, outputs and block counts
       if (valid) {
@@ -458,9 +558,7 @@ cudaError_t launch_ep(const RoutingArgs& a, void* wsplit, void* partials, int nu
   if (e != cudaSuccess) return e;
   const int units = p.n_tiles * p.ksplit;
   const int grid = units < num_sms ? units : num_sms;
-  router_tc_kernel<EP, K><<<grid, NUM_THREADS, G::SMEM, s>>>(mx, mw, p);
-  count_launch();
-  return cudaGetLastError();
+  return launch_pdl(router_tc_kernel<EP, K>, dim3(grid), dim3(NUM_THREADS), G::SMEM, s, mx, mw, p);
 }
 
 template <int EP>

@@ -253,6 +253,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(RoutingArgs a) {
   __shared__ float s_psum[256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = a.E, nb = a.nblk;
+  pdl_wait();
+  pdl_trigger();
   constexpr int V = 8;  // blocks per lane loaded ahead of the dependent scan steps
   for (int e = warp; e < E; e += 32) {
     int run = 0, c1 = 0;
@@ -344,6 +346,8 @@ __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * BT;
   const int nt = static_cast<int>((a.T - t0) < BT ? (a.T - t0) : BT);
   const int nA = nt * k;
+  pdl_wait();
+  pdl_trigger();
   for (int e = tid; e < E; e += 256) run_s[e] = a.blockoff[e * nb + blockIdx.x];
   __syncthreads();
   if (warp == 0) {
@@ -417,6 +421,8 @@ template <typename YT>
 __global__ void __launch_bounds__(256) combine_kernel(int64_t T, int k, int d, const int32_t* __restrict__ dest_row,
                                                       const float* __restrict__ Yp, int ksplit, int64_t split_stride,
                                                       YT* __restrict__ y, float* __restrict__ yf) {
+  pdl_wait();
+  pdl_trigger();
   const uint32_t vpr = static_cast<uint32_t>(d) >> 2;  // float4 groups per row (d % 4 == 0 on this path)
   const uint32_t i = blockIdx.x * 256u + threadIdx.x;    // T * d / 4 < 2^32 (checked on the host)
   if (i >= static_cast<uint32_t>(T) * vpr) return;
@@ -467,6 +473,8 @@ __global__ void __launch_bounds__(256) combine_scalar_kernel(int64_t T, int k, i
                                                              const float* __restrict__ Yp, int ksplit,
                                                              int64_t split_stride, YT* __restrict__ y,
                                                              float* __restrict__ yf) {
+  pdl_wait();
+  pdl_trigger();
   const uint32_t i = blockIdx.x * 256u + threadIdx.x;  // T * d < 2^32 (checked on the host)
   if (i >= static_cast<uint32_t>(T) * static_cast<uint32_t>(d)) return;
   const uint32_t t32 = i / static_cast<uint32_t>(d);
@@ -502,41 +510,30 @@ cudaError_t launch_router(const RoutingArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_scan(const RoutingArgs& a, cudaStream_t s) {
-  scan_kernel<<<1, 1024, 0, s>>>(a);
-  count_launch();
-  return cudaGetLastError();
+  return launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, s, a);
 }
 
 cudaError_t launch_dispatch(const RoutingArgs& a, cudaStream_t s) {
-  if (a.x_is_bf16)
-    dispatch_kernel<__nv_bfloat16><<<a.nblk, 256, 0, s>>>(a);
-  else
-    dispatch_kernel<float><<<a.nblk, 256, 0, s>>>(a);
-  count_launch();
-  return cudaGetLastError();
+  if (a.x_is_bf16) return launch_pdl(dispatch_kernel<__nv_bfloat16>, dim3(a.nblk), dim3(256), 0, s, a);
+  return launch_pdl(dispatch_kernel<float>, dim3(a.nblk), dim3(256), 0, s, a);
 }
 
 cudaError_t launch_combine(int64_t T, int k, int d, int y_is_bf16, const int32_t* dest_row, const float* Yp,
                            int ksplit, int64_t split_stride, void* y, float* y_f32, cudaStream_t s) {
   if ((d & 3) == 0) {
-    const unsigned grid = static_cast<unsigned>((T * (d / 4) + 255) / 256);
+    const dim3 grid(static_cast<unsigned>((T * (d / 4) + 255) / 256));
     if (y_is_bf16)
-      combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(T, k, d, dest_row, Yp, ksplit, split_stride,
-                                                          static_cast<__nv_bfloat16*>(y), y_f32);
-    else
-      combine_kernel<float><<<grid, 256, 0, s>>>(T, k, d, dest_row, Yp, ksplit, split_stride,
-                                                 static_cast<float*>(y), y_f32);
-  } else {
-    const unsigned grid = static_cast<unsigned>((T * d + 255) / 256);
-    if (y_is_bf16)
-      combine_scalar_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(T, k, d, dest_row, Yp, ksplit, split_stride,
-                                                                 static_cast<__nv_bfloat16*>(y), y_f32);
-    else
-      combine_scalar_kernel<float><<<grid, 256, 0, s>>>(T, k, d, dest_row, Yp, ksplit, split_stride,
-                                                        static_cast<float*>(y), y_f32);
+      return launch_pdl(combine_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, T, k, d, dest_row, Yp, ksplit,
+                        split_stride, static_cast<__nv_bfloat16*>(y), y_f32);
+    return launch_pdl(combine_kernel<float>, grid, dim3(256), 0, s, T, k, d, dest_row, Yp, ksplit, split_stride,
+                      static_cast<float*>(y), y_f32);
   }
-  count_launch();
-  return cudaGetLastError();
+  const dim3 grid(static_cast<unsigned>((T * d + 255) / 256));
+  if (y_is_bf16)
+    return launch_pdl(combine_scalar_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, T, k, d, dest_row, Yp, ksplit,
+                      split_stride, static_cast<__nv_bfloat16*>(y), y_f32);
+  return launch_pdl(combine_scalar_kernel<float>, grid, dim3(256), 0, s, T, k, d, dest_row, Yp, ksplit,
+                    split_stride, static_cast<float*>(y), y_f32);
 }
 
 cudaError_t launch_selftest_timeout(unsigned int* err, int64_t limit_ns, cudaStream_t s) {

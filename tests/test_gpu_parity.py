@@ -42,6 +42,12 @@ SMALL = [
     ("long_k_ragged", 333, 1032, 4, 2, 1160, S, RN, 0.0, BF, None),
     ("decode_splitk", 3, 256, 8, 2, 1024, S, RN, 0.0, BF, None),          # K ranges of GEMM2 split
     ("decode_splitk_ragged", 5, 136, 4, 2, 1160, R, SW, 0.0, BF, "normal"),
+    # grouped-GEMM stream-K tail: 1 < tiles / 148 < 2 (two pieces per tile) ...
+    ("stream_k_tail_relu", 600, 256, 8, 2, 4096, R, RN, 0.0, BF, None),
+    # ... and few tiles over long K (up to 6-7 pieces per tile), k = 1 scatter epilogue, SwiGLU
+    ("stream_k_switch_pieces", 700, 512, 16, 1, 1024, R, SW, 1.25, BF, "normal"),
+    ("stream_k_long_k", 2, 2048, 4, 1, 256, R, RN, 0.0, BF, None),
+    ("stream_k_swiglu_pieces", 4, 1536, 8, 2, 384, S, RN, 0.0, BF, None),
 ]
 
 
@@ -66,7 +72,8 @@ def test_small_layers_match_oracle(case):
 
 
 SINGLE = [c for c in SMALL if c[9] == BF and c[0] in ("swiglu_e8_k2", "switch_relu_drops", "k4_zipf_tails",
-                                                       "e128_k8_cap", "long_k_ragged")]
+                                                       "e128_k8_cap", "long_k_ragged", "stream_k_tail_relu",
+                                                       "stream_k_switch_pieces")]
 
 
 @pytest.mark.parametrize("case", SINGLE, ids=[c[0] for c in SINGLE])
