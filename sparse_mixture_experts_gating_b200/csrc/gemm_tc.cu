@@ -222,8 +222,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint8_t* sa = stages + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&ctl->full[stage], tx);
           if (nshort == 0) {
-            tma_load_2d(sa, &tmA, &ctl->full[stage], kb * BK, row0);
-            if (A_SPLIT) tma_load_2d(sa + A_BYTES, &tmA2, &ctl->full[stage], kb * BK, row0);
+            if (A_SPLIT) tma_load_3d(sa, &tmA, &ctl->full[stage], kb * BK, row0, 0);  // hi and lo planes
+            else tma_load_2d(sa, &tmA, &ctl->full[stage], kb * BK, row0);
           } else {
             for (int j = 0; j < nshort; ++j) {
               tma_load_2d(sa + j * A_SHORT * BK * 2, &tmAs, &ctl->full[stage], kb * BK, row0 + j * A_SHORT);
@@ -236,8 +236,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tma_load_2d(sa + B_OFF, &tmB0, &ctl->full[stage], kb * BK, brow);
             tma_load_2d(sa + B_OFF + B_HALF, &tmB1, &ctl->full[stage], kb * BK, brow);
           } else {
-            tma_load_2d(sa + B_OFF, &tmB0, &ctl->full[stage], kb * BK, brow);
-            tma_load_2d(sa + B_OFF + B_HALF, &tmB0, &ctl->full[stage], kb * BK, brow + 128);
+            tma_load_2d(sa + B_OFF, &tmB0, &ctl->full[stage], kb * BK, brow);  // 256-row box
           }
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -459,6 +458,19 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
 
 }  // namespace
 
+bool make_map_planes_bf16(CUtensorMap* m, const void* base, uint64_t plane_stride, uint64_t rows, uint64_t cols,
+                          uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[3] = {cols, rows, 2};
+  const cuuint64_t strides[2] = {cols * 2, plane_stride};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(BK), box_rows, 2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
@@ -490,14 +502,26 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
   *why = nullptr;
   if (g.E > MAX_E) { *why = "grouped GEMM supports at most 256 experts"; return cudaErrorInvalidValue; }
   const bool a_split = g.split && g.A2 != nullptr;
-  if (!make_map(&pl->a, g.A, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K)) ||
-      !make_map(&pl->a2, a_split ? g.A2 : g.A, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K)) ||
-      !make_map_bf16(&pl->as, g.A, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K), A_SHORT) ||
-      !make_map_bf16(&pl->as2, a_split ? g.A2 : g.A, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K),
-                     A_SHORT) ||
-      !make_map(&pl->b0, g.B0, static_cast<uint64_t>(g.E) * g.N, static_cast<uint64_t>(g.K)) ||
-      !make_map(&pl->b1, g.epi == EPI_SWIGLU_BF16 ? g.B1 : g.B0, static_cast<uint64_t>(g.E) * g.N,
-                static_cast<uint64_t>(g.K))) {
+  const bool swiglu = g.epi == EPI_SWIGLU_BF16;
+  const uint64_t a_rows = static_cast<uint64_t>(g.a_rows), K = static_cast<uint64_t>(g.K);
+  const uint64_t b_rows = static_cast<uint64_t>(g.E) * g.N;
+  // a split A is read through one 3D map over both planes (the lo plane must
+  // follow the hi plane at a 16-byte multiple)
+  const intptr_t plane_stride = static_cast<const uint8_t*>(g.A2) - static_cast<const uint8_t*>(g.A);
+  if (a_split && (plane_stride <= 0 || plane_stride % 16 != 0 ||
+                  static_cast<uint64_t>(plane_stride) < a_rows * K * 2)) {
+    *why = "grouped GEMM: the lo plane of the A operand must follow the hi plane";
+    return cudaErrorInvalidValue;
+  }
+  const bool maps_ok =
+      (a_split ? make_map_planes_bf16(&pl->a, g.A, static_cast<uint64_t>(plane_stride), a_rows, K, 128)
+               : make_map(&pl->a, g.A, a_rows, K)) &&
+      make_map(&pl->a2, a_split ? g.A2 : g.A, a_rows, K) && make_map_bf16(&pl->as, g.A, a_rows, K, A_SHORT) &&
+      make_map_bf16(&pl->as2, a_split ? g.A2 : g.A, a_rows, K, A_SHORT) &&
+      // B: two 128-row boxes (W1 and W3) for SwiGLU, else one 256-row box
+      make_map_bf16(&pl->b0, g.B0, b_rows, K, swiglu ? 128 : 256) &&
+      make_map(&pl->b1, swiglu ? g.B1 : g.B0, b_rows, K);
+  if (!maps_ok) {
     *why = "cuTensorMapEncodeTiled failed (alignment or driver entry point)";
     return cudaErrorInvalidValue;
   }

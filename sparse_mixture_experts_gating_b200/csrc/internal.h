@@ -68,6 +68,11 @@ cudaError_t launch_router_tc(const RoutingArgs& a, void* wsplit, void* partials,
 
 // bf16 [rows][cols] tensor map, box [box_rows][64], 128-byte swizzle.
 bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// Two bf16 planes [2][rows][cols], plane_stride bytes apart -> 3D map with box
+// [2 planes][box_rows][64 cols], 128-byte swizzle: one copy lands plane 0's
+// [box_rows x 64] tile followed by plane 1's.
+bool make_map_planes_bf16(CUtensorMap* m, const void* base, uint64_t plane_stride, uint64_t rows, uint64_t cols,
+                          uint32_t box_rows);
 cudaError_t launch_scan(const RoutingArgs& a, cudaStream_t s);
 cudaError_t launch_dispatch(const RoutingArgs& a, cudaStream_t s);
 // y_t = sum over kept choices j (in order j) of sum over the ksplit partials

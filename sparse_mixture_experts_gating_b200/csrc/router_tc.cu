@@ -159,9 +159,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint8_t* sa = stages + stage * G::STAGE_BYTES;
           mbar_arrive_expect_tx(&ctl->full[stage], G::STAGE_BYTES);
           tma_load_2d(sa, &tmX, &ctl->full[stage], kb * BK, tile * BM);
+          if (3 * EP <= 256) {  // the three planes in one box
+            tma_load_2d(sa + A_BYTES, &tmW, &ctl->full[stage], kb * BK, 0);
+          } else {
 #pragma unroll
-          for (int pl = 0; pl < 3; ++pl)
-            tma_load_2d(sa + A_BYTES + pl * G::B_PLANE, &tmW, &ctl->full[stage], kb * BK, pl * EP);
+            for (int pl = 0; pl < 3; ++pl)
+              tma_load_2d(sa + A_BYTES + pl * G::B_PLANE, &tmW, &ctl->full[stage], kb * BK, pl * EP);
+          }
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -517,7 +521,8 @@ cudaError_t launch_ep(const RoutingArgs& a, void* wsplit, void* partials, int nu
   static_assert(G::STAGES >= 2, "router stages");
   CUtensorMap mx, mw;
   if (!make_map_bf16(&mx, a.x, static_cast<uint64_t>(a.T), static_cast<uint64_t>(a.d), BM) ||
-      !make_map_bf16(&mw, wsplit, static_cast<uint64_t>(3 * EP), static_cast<uint64_t>(a.d), EP)) {
+      !make_map_bf16(&mw, wsplit, static_cast<uint64_t>(3 * EP), static_cast<uint64_t>(a.d),
+                     3 * EP <= 256 ? 3 * EP : EP)) {
     *why = "router: cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
