@@ -35,6 +35,9 @@ struct RoutingArgs {
   int32_t* counts;     // [E]   (may alias the user output)
   int32_t* offsets;    // [E+1]
   int32_t* mprefix;    // [E+1] prefix of ceil(kept_e / kTileM)
+  int32_t* tot_cnt1;   // [E]   first-choice count of each expert (scan)
+  float* tot_psum;     // [E]   probability sum of each expert (scan)
+  int32_t* scan_ticket;  // zeroed by the router; the scan's last block resets it
   int32_t* row_token;  // [S_max]
   float* row_gate;     // [S_max]
   void* Xp;            // [S_max][d]

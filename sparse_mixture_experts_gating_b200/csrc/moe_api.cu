@@ -121,7 +121,7 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   w.counts = take(sizeof(int32_t) * L.E);
   w.offsets = take(sizeof(int32_t) * (L.E + 1));
   w.mprefix = take(sizeof(int32_t) * (L.E + 1));
-  w.scal = take(64);
+  w.scal = take(sizeof(int32_t) * L.E + sizeof(float) * L.E + 64);  // scan totals and ticket
   const bool tc_router = L.dtype == MOE_BF16 && L.E <= kRouterTcMaxE;
   w.wsplit = take(tc_router ? 3 * sizeof(uint16_t) * router_pad_e(L.E) * static_cast<size_t>(L.d) : 0);
   w.rpart = take(tc_router ? router_partials_bytes(T, L.E, L.d) : 0);
@@ -290,6 +290,9 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   r.offsets = reinterpret_cast<int32_t*>(ws + w.offsets);
   r.mprefix = reinterpret_cast<int32_t*>(ws + w.mprefix);
   r.row_token = reinterpret_cast<int32_t*>(ws + w.row_token);
+  r.tot_cnt1 = reinterpret_cast<int32_t*>(ws + w.scal);
+  r.tot_psum = reinterpret_cast<float*>(ws + w.scal + sizeof(int32_t) * L.E);
+  r.scan_ticket = reinterpret_cast<int32_t*>(ws + w.scal + (sizeof(int32_t) + sizeof(float)) * L.E);
   r.row_gate = reinterpret_cast<float*>(ws + w.row_gate);
   r.Xp = ws + w.Xp;
   r.dropped = dropped;

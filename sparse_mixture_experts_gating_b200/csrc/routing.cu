@@ -73,6 +73,7 @@ __global__ void __launch_bounds__(RT) router_kernel(RoutingArgs a) {
   const XT* x = static_cast<const XT*>(a.x);
 
   for (int e = tid; e < EP; e += RT) { cnt1_s[e] = 0; hist_s[e] = 0; }
+  if (blockIdx.x == 0 && tid == 0) *a.scan_ticket = 0;
 
   if (a.logits_in == nullptr) {
     const int tg = tid >> 4, eg = tid & 15;
@@ -246,90 +247,157 @@ cudaError_t launch_router_x(const RoutingArgs& a, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------------------
-// Scan: one block of 1024 threads.  Warp w owns experts w, w+32, ...
-__global__ void __launch_bounds__(1024) scan_kernel(RoutingArgs a) {
-  __shared__ int s_counts[256];
-  __shared__ int s_cnt1[256];
-  __shared__ float s_psum[256];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// Scan: one block per expert e.  Each thread takes a contiguous run of the
+// router blocks, so the exclusive prefix of e's per-block counts (the stable
+// rank base of each block, in token order) is one block-wide scan; e's totals
+// (routed count, first-choice count, probability sum) go to the workspace.
+// The block that finishes last (ticket) turns the totals into capacity,
+// expert offsets, tile prefix, dropped count, aux loss and z-loss, all summed
+// in a fixed order.
+constexpr int SCAN_T = 256;
+constexpr int kScanSingleBlocks = 8;  // up to 256 tokens: one block, one expert per thread
+
+__device__ __forceinline__ int block_exscan_int(int v, int* s_warp, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < SCAN_T / 32 ? s_warp[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += u;
+    }
+    if (lane < SCAN_T / 32) s_warp[lane] = wi - w;  // exclusive warp bases
+    if (lane == SCAN_T / 32 - 1) s_warp[SCAN_T / 32] = wi;
+  }
+  __syncthreads();
+  const int r = s_warp[warp] + incl - v;
+  total = s_warp[SCAN_T / 32];
+  __syncthreads();
+  return r;
+}
+
+// Sum over the block in a fixed tree order (deterministic).
+template <typename F>
+__device__ __forceinline__ F block_sum(F v, F* s_red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  F t = 0;
+  if (threadIdx.x == 0)
+    for (int w = 0; w < SCAN_T / 32; ++w) t += s_red[w];
+  __syncthreads();
+  return t;  // valid in thread 0
+}
+
+// Capacity, expert offsets, tile prefix, dropped count, aux loss and z-loss
+// from the per-expert totals (thread e < E holds expert e's), by all SCAN_T
+// threads of one block.
+__device__ __forceinline__ void scan_finalize(const RoutingArgs& a, int cnt, int c1, float ps, int* s_warp,
+                                              int* s_redi, double* s_redd) {
+  const int tid = threadIdx.x, E = a.E, nb = a.nblk;
+  const int kept =
+      tid < E ? ((a.capacity < 0) ? cnt : static_cast<int>((int64_t)cnt < a.capacity ? (int64_t)cnt : a.capacity))
+              : 0;
+  const int mt = (kept + kTileM - 1) / kTileM;
+  int total_kept = 0, total_tiles = 0;
+  const int off = block_exscan_int(kept, s_warp, total_kept);
+  const int mp = block_exscan_int(mt, s_warp, total_tiles);
+  if (tid < E) {
+    a.counts[tid] = cnt;
+    a.offsets[tid] = off;
+    a.mprefix[tid] = mp;
+    if (a.offsets_out != nullptr) a.offsets_out[tid] = off;
+  }
+  const int drop = block_sum<int>(tid < E ? cnt - kept : 0, s_redi);
+  const double auxp =
+      block_sum<double>(tid < E ? static_cast<double>(c1) * static_cast<double>(ps) : 0.0, s_redd);
+  double zs = 0.0;
+  for (int b = tid; b < nb; b += SCAN_T) zs += static_cast<double>(a.part_lse2[b]);
+  zs = block_sum<double>(zs, s_redd);
+  if (tid == 0) {
+    a.offsets[E] = total_kept;
+    a.mprefix[E] = total_tiles;
+    if (a.offsets_out != nullptr) a.offsets_out[E] = total_kept;
+    *a.dropped = drop;
+    const double T = static_cast<double>(a.T);
+    *a.aux = static_cast<float>(static_cast<double>(E) * auxp / (T * T));
+    *a.z = static_cast<float>(zs / T);
+  }
+}
+
+// SINGLE (few router blocks): one block, thread e walks expert e's blocks in
+// order.  Otherwise one block per expert as described above.
+template <bool SINGLE>
+__global__ void __launch_bounds__(SCAN_T) scan_kernel(RoutingArgs a) {
+  __shared__ int s_warp[SCAN_T / 32 + 1];
+  __shared__ float s_redf[SCAN_T / 32];
+  __shared__ double s_redd[SCAN_T / 32];
+  __shared__ int s_redi[SCAN_T / 32];
+  __shared__ int s_last;
+  const int tid = threadIdx.x;
   const int E = a.E, nb = a.nblk;
   pdl_wait();
   pdl_trigger();
-  constexpr int V = 8;  // blocks per lane loaded ahead of the dependent scan steps
-  for (int e = warp; e < E; e += 32) {
-    int run = 0, c1 = 0;
+  if constexpr (SINGLE) {
+    int cnt = 0, c1 = 0;
     float ps = 0.f;
-    for (int g0 = 0; g0 < nb; g0 += 32 * V) {
-      int hv[V], cv[V];
-      float pv[V];
-#pragma unroll
-      for (int v = 0; v < V; ++v) {  // independent loads first
-        const int b = g0 + v * 32 + lane;
-        const bool in = b < nb;
-        hv[v] = in ? a.part_hist[e * nb + b] : 0;
-        cv[v] = in ? a.part_cnt1[e * nb + b] : 0;
-        pv[v] = in ? a.part_psum[e * nb + b] : 0.f;
-      }
-#pragma unroll
-      for (int v = 0; v < V; ++v) {
-        const int b = g0 + v * 32 + lane;
-        if (g0 + v * 32 >= nb) break;
-        int incl = hv[v];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int u = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += u;
-        }
-        if (b < nb) a.blockoff[e * nb + b] = run + incl - hv[v];
-        run += __shfl_sync(0xffffffffu, incl, 31);
-        c1 += warp_sum_i(cv[v]);
-        ps += warp_sum(pv[v]);
+    if (tid < E) {
+      const int64_t row = static_cast<int64_t>(tid) * nb;
+#pragma unroll 4
+      for (int b = 0; b < nb; ++b) {
+        a.blockoff[row + b] = cnt;
+        cnt += a.part_hist[row + b];
+        c1 += a.part_cnt1[row + b];
+        ps += a.part_psum[row + b];
       }
     }
-    if (lane == 0) { s_counts[e] = run; s_cnt1[e] = c1; s_psum[e] = ps; }
+    scan_finalize(a, cnt, c1, ps, s_warp, s_redi, s_redd);
+    return;
+  }
+  const int e = blockIdx.x;
+  // this thread's run of router blocks [b0, b1)
+  const int per = (nb + SCAN_T - 1) / SCAN_T;
+  const int b0 = min(nb, tid * per), b1 = min(nb, b0 + per);
+  const int32_t* hist = a.part_hist + static_cast<int64_t>(e) * nb;
+  int h_run = 0, c1 = 0;
+  float ps = 0.f;
+  for (int b = b0; b < b1; ++b) {
+    h_run += hist[b];
+    c1 += a.part_cnt1[static_cast<int64_t>(e) * nb + b];
+    ps += a.part_psum[static_cast<int64_t>(e) * nb + b];
+  }
+  int count = 0;
+  int base = block_exscan_int(h_run, s_warp, count);
+  for (int b = b0; b < b1; ++b) {
+    a.blockoff[static_cast<int64_t>(e) * nb + b] = base;
+    base += hist[b];
+  }
+  const int c1_tot = block_sum<int>(c1, s_redi);
+  const float ps_tot = block_sum<float>(ps, s_redf);
+  if (tid == 0) {
+    a.counts[e] = count;
+    a.tot_cnt1[e] = c1_tot;
+    a.tot_psum[e] = ps_tot;
+    __threadfence();
+    s_last = atomicAdd(a.scan_ticket, 1) == E - 1;
   }
   __syncthreads();
-  if (warp == 0) {
-    int base = 0, tiles = 0, drop = 0;
-    double auxp = 0.0;
-    for (int e0 = 0; e0 < E; e0 += 32) {
-      const int e = e0 + lane;
-      const int cnt = e < E ? s_counts[e] : 0;
-      const int kept = (a.capacity < 0) ? cnt : static_cast<int>((int64_t)cnt < a.capacity ? (int64_t)cnt : a.capacity);
-      const int mt = (kept + kTileM - 1) / kTileM;
-      int ik = kept, im = mt;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, ik, o);
-        const int w = __shfl_up_sync(0xffffffffu, im, o);
-        if (lane >= o) { ik += u; im += w; }
-      }
-      if (e < E) {
-        a.counts[e] = cnt;
-        a.offsets[e] = base + ik - kept;
-        a.mprefix[e] = tiles + im - mt;
-        if (a.offsets_out != nullptr) a.offsets_out[e] = base + ik - kept;
-        auxp += static_cast<double>(s_cnt1[e]) * static_cast<double>(s_psum[e]);
-      }
-      base += __shfl_sync(0xffffffffu, ik, 31);
-      tiles += __shfl_sync(0xffffffffu, im, 31);
-      drop += warp_sum_i(cnt - kept);
-    }
-    auxp = warp_sum_d(auxp);
-    if (lane == 0) {
-      a.offsets[E] = base;
-      a.mprefix[E] = tiles;
-      if (a.offsets_out != nullptr) a.offsets_out[E] = base;
-      *a.dropped = drop;
-      const double T = static_cast<double>(a.T);
-      *a.aux = static_cast<float>(static_cast<double>(E) * auxp / (T * T));
-    }
-  } else if (warp == 1) {
-    double zs = 0.0;
-    for (int b = lane; b < nb; b += 32) zs += static_cast<double>(a.part_lse2[b]);
-    zs = warp_sum_d(zs);
-    if (lane == 0) *a.z = static_cast<float>(zs / static_cast<double>(a.T));
-  }
+  if (!s_last) return;
+  __threadfence();
+  // the last block
+  scan_finalize(a, tid < E ? __ldcg(a.counts + tid) : 0, tid < E ? __ldcg(a.tot_cnt1 + tid) : 0,
+                tid < E ? __ldcg(a.tot_psum + tid) : 0.f, s_warp, s_redi, s_redd);
+  if (tid == 0) *a.scan_ticket = 0;  // ready for the next call
 }
 
 // ---------------------------------------------------------------------------
@@ -393,15 +461,15 @@ __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
         const uint4* src = reinterpret_cast<const uint4*>(x + tok * d);
         uint4* dst = reinterpret_cast<uint4*>(Xp + static_cast<int64_t>(dest) * d);
         const int nv = static_cast<int>(static_cast<size_t>(d) * sizeof(XT) / 16);
-        int v = lane;
-        for (; v + 96 < nv; v += 128) {  // four independent 16-byte loads in flight per lane
-          const uint4 a0 = src[v], a1 = src[v + 32], a2 = src[v + 64], a3 = src[v + 96];
-          dst[v] = a0;
-          dst[v + 32] = a1;
-          dst[v + 64] = a2;
-          dst[v + 96] = a3;
+        for (int v0 = lane; v0 < nv; v0 += 128) {  // up to four 16-byte loads in flight per lane
+          uint4 c[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (v0 + 32 * q < nv) c[q] = src[v0 + 32 * q];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (v0 + 32 * q < nv) dst[v0 + 32 * q] = c[q];
         }
-        for (; v < nv; v += 32) dst[v] = src[v];
       } else {
         for (int c = lane; c < d; c += 32) Xp[static_cast<int64_t>(dest) * d + c] = x[tok * d + c];
       }
@@ -415,54 +483,78 @@ __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
 
 // ---------------------------------------------------------------------------
 // Combine: y_t = sum over kept choices j (ascending) of the slot's row of Yp
-// (summed over its K-range partials in order).  One thread per token and
-// group of 4 columns, so small batches still spread over many warps.
-template <typename YT>
-__global__ void __launch_bounds__(256) combine_kernel(int64_t T, int k, int d, const int32_t* __restrict__ dest_row,
+// (summed over its K-range partials in order).  A thread owns CU groups of 4
+// columns (grid-strided, so every load instruction of a warp is one run of
+// 512 bytes); the destinations and all CU * K row loads are issued before the
+// ordered sums, so each thread keeps 8 loads in flight.  Small batches use
+// CU = 1 (WIDE false) to spread over more blocks.
+template <typename YT, int K, bool WIDE>
+__global__ void __launch_bounds__(256) combine_kernel(int64_t T, int d, const int32_t* __restrict__ dest_row,
                                                       const float* __restrict__ Yp, int ksplit, int64_t split_stride,
                                                       YT* __restrict__ y, float* __restrict__ yf) {
+  constexpr int CU = (!WIDE || K >= 8) ? 1 : 8 / K;
   pdl_wait();
   pdl_trigger();
   const uint32_t vpr = static_cast<uint32_t>(d) >> 2;  // float4 groups per row (d % 4 == 0 on this path)
-  const uint32_t i = blockIdx.x * 256u + threadIdx.x;    // T * d / 4 < 2^32 (checked on the host)
-  if (i >= static_cast<uint32_t>(T) * vpr) return;
-  const uint32_t t32 = i / vpr;
-  const int64_t t = t32;
-  const int v = static_cast<int>(i - t32 * vpr);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const uint32_t n = static_cast<uint32_t>(T) * vpr;   // T * d / 4 < 2^32 (checked on the host)
+  const uint32_t stride = gridDim.x * 256u;
+  uint32_t tok[CU];
+  int v[CU], dst[CU][K];
+#pragma unroll
+  for (int u = 0; u < CU; ++u) {
+    const uint32_t i = blockIdx.x * 256u + threadIdx.x + u * stride;
+    tok[u] = i < n ? i / vpr : 0xffffffffu;
+    v[u] = i < n ? static_cast<int>(i - tok[u] * vpr) : 0;
+#pragma unroll
+    for (int j = 0; j < K; ++j) dst[u][j] = i < n ? dest_row[static_cast<int64_t>(tok[u]) * K + j] : -1;
+  }
+  float4 acc[CU];
   if (ksplit == 1) {
-    float4 u[8];
+    float4 r[CU][K];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {  // all loads first (independent), then the ordered sum
-      const int dst = j < k ? dest_row[t * k + j] : -1;
-      u[j] = dst >= 0 ? reinterpret_cast<const float4*>(Yp + static_cast<int64_t>(dst) * d)[v]
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+    for (int u = 0; u < CU; ++u)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      acc.x += u[j].x; acc.y += u[j].y; acc.z += u[j].z; acc.w += u[j].w;
+      for (int j = 0; j < K; ++j)
+        r[u][j] = dst[u][j] >= 0 ? reinterpret_cast<const float4*>(Yp + static_cast<int64_t>(dst[u][j]) * d)[v[u]]
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < CU; ++u) {
+      acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < K; ++j) {
+        acc[u].x += r[u][j].x; acc[u].y += r[u][j].y; acc[u].z += r[u][j].z; acc[u].w += r[u][j].w;
+      }
     }
   } else {
-    for (int j = 0; j < k; ++j) {
-      const int dst = dest_row[t * k + j];
-      if (dst < 0) continue;
-      float4 sj = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int ks = 0; ks < ksplit; ++ks) {
-        const float4 u = reinterpret_cast<const float4*>(Yp + static_cast<int64_t>(ks) * split_stride +
-                                                         static_cast<int64_t>(dst) * d)[v];
-        sj.x += u.x; sj.y += u.y; sj.z += u.z; sj.w += u.w;
+#pragma unroll
+    for (int u = 0; u < CU; ++u) {
+      acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < K; ++j) {
+        if (dst[u][j] < 0) continue;
+        float4 sj = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int ks = 0; ks < ksplit; ++ks) {
+          const float4 q = reinterpret_cast<const float4*>(Yp + static_cast<int64_t>(ks) * split_stride +
+                                                           static_cast<int64_t>(dst[u][j]) * d)[v[u]];
+          sj.x += q.x; sj.y += q.y; sj.z += q.z; sj.w += q.w;
+        }
+        acc[u].x += sj.x; acc[u].y += sj.y; acc[u].z += sj.z; acc[u].w += sj.w;
       }
-      acc.x += sj.x; acc.y += sj.y; acc.z += sj.z; acc.w += sj.w;
     }
   }
-  if (yf != nullptr) reinterpret_cast<float4*>(yf + t * d)[v] = acc;
-  if constexpr (sizeof(YT) == 2) {
-    uint2 o;
-    o.x = pack_bf16x2(acc.x, acc.y);
-    o.y = pack_bf16x2(acc.z, acc.w);
-    reinterpret_cast<uint2*>(y + t * d)[v] = o;
-  } else {
-    reinterpret_cast<float4*>(y + t * d)[v] = acc;
+#pragma unroll
+  for (int u = 0; u < CU; ++u) {
+    if (tok[u] == 0xffffffffu) continue;
+    const int64_t t = tok[u];
+    if (yf != nullptr) reinterpret_cast<float4*>(yf + t * d)[v[u]] = acc[u];
+    if constexpr (sizeof(YT) == 2) {
+      uint2 o;
+      o.x = pack_bf16x2(acc[u].x, acc[u].y);
+      o.y = pack_bf16x2(acc[u].z, acc[u].w);
+      reinterpret_cast<uint2*>(y + t * d)[v[u]] = o;
+    } else {
+      reinterpret_cast<float4*>(y + t * d)[v[u]] = acc[u];
+    }
   }
 }
 
@@ -510,7 +602,8 @@ cudaError_t launch_router(const RoutingArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_scan(const RoutingArgs& a, cudaStream_t s) {
-  return launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, s, a);
+  if (a.nblk <= kScanSingleBlocks) return launch_pdl(scan_kernel<true>, dim3(1), dim3(SCAN_T), 0, s, a);
+  return launch_pdl(scan_kernel<false>, dim3(a.E), dim3(SCAN_T), 0, s, a);
 }
 
 cudaError_t launch_dispatch(const RoutingArgs& a, cudaStream_t s) {
@@ -518,15 +611,40 @@ cudaError_t launch_dispatch(const RoutingArgs& a, cudaStream_t s) {
   return launch_pdl(dispatch_kernel<float>, dim3(a.nblk), dim3(256), 0, s, a);
 }
 
+namespace {
+template <int K>
+cudaError_t launch_combine_k(int64_t T, int d, int y_is_bf16, const int32_t* dest_row, const float* Yp, int ksplit,
+                             int64_t split_stride, void* y, float* y_f32, cudaStream_t s) {
+  constexpr int CU = K >= 8 ? 1 : 8 / K;
+  const int64_t groups = T * (d / 4);
+  // wide threads only when the grid still covers every SM several times over
+  const bool wide = groups >= static_cast<int64_t>(256) * CU * 148 * 4;
+  const int cu = wide ? CU : 1;
+  const dim3 grid(static_cast<unsigned>((groups + 256 * cu - 1) / (256 * cu)));
+  if (y_is_bf16) {
+    auto kern = wide ? combine_kernel<__nv_bfloat16, K, true> : combine_kernel<__nv_bfloat16, K, false>;
+    return launch_pdl(kern, grid, dim3(256), 0, s, T, d, dest_row, Yp, ksplit, split_stride,
+                      static_cast<__nv_bfloat16*>(y), y_f32);
+  }
+  auto kern = wide ? combine_kernel<float, K, true> : combine_kernel<float, K, false>;
+  return launch_pdl(kern, grid, dim3(256), 0, s, T, d, dest_row, Yp, ksplit, split_stride, static_cast<float*>(y),
+                    y_f32);
+}
+}  // namespace
+
 cudaError_t launch_combine(int64_t T, int k, int d, int y_is_bf16, const int32_t* dest_row, const float* Yp,
                            int ksplit, int64_t split_stride, void* y, float* y_f32, cudaStream_t s) {
   if ((d & 3) == 0) {
-    const dim3 grid(static_cast<unsigned>((T * (d / 4) + 255) / 256));
-    if (y_is_bf16)
-      return launch_pdl(combine_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, T, k, d, dest_row, Yp, ksplit,
-                        split_stride, static_cast<__nv_bfloat16*>(y), y_f32);
-    return launch_pdl(combine_kernel<float>, grid, dim3(256), 0, s, T, k, d, dest_row, Yp, ksplit, split_stride,
-                      static_cast<float*>(y), y_f32);
+    switch (k) {
+      case 1: return launch_combine_k<1>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
+      case 2: return launch_combine_k<2>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
+      case 3: return launch_combine_k<3>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
+      case 4: return launch_combine_k<4>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
+      case 5: return launch_combine_k<5>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
+      case 6: return launch_combine_k<6>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
+      case 7: return launch_combine_k<7>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
+      default: return launch_combine_k<8>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
+    }
   }
   const dim3 grid(static_cast<unsigned>((T * d + 255) / 256));
   if (y_is_bf16)
