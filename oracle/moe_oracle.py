@@ -213,9 +213,45 @@ def aux_and_z(p: np.ndarray, lse: np.ndarray, idx: np.ndarray, E: int):
     return float(E * np.sum(f * P)), float(np.mean(lse ** 2))
 
 
+def balance_losses(p: np.ndarray, idx: np.ndarray, E: int) -> dict:
+    """Alternative load-balancing statistics, unscaled (the caller applies its
+    coefficient, e.g. 0.01).
+
+    * ``cv_counts``: the coefficient of variation (standard deviation over
+      mean, over the E experts) of the expert assignment counts, all k choices
+      counted before capacity -- page "Mixture of Experts (MoE)"
+      (inferensys.com, self-hosted large language models), training-challenge
+      bullets: "a coefficient of 0.01 multiplied by the coefficient of
+      variation of expert assignment counts".
+    * ``cv2_probs``: the squared coefficient of variation of the router
+      probabilities aggregated per expert (P_i, the mean full-softmax
+      probability) -- page "Mixture of Experts (MoE) Language Models"
+      (chipfoundryservices.com), "Load Balancing and Training": cv^2 of the
+      router probabilities.
+    * ``aux_all_choices``: the Switch loss of "Mixture of experts" (rayaq.ca),
+      section "The load-balancing loss", with f_i the share of all T*k
+      assignments (not only first choices) routed to i.
+
+    Readings: standard deviation and variance are of the E values themselves
+    (population moments, divided by E); T = 0 gives zeros.
+    """
+    T, k = idx.shape
+    if T == 0:
+        return {"aux_all_choices": 0.0, "cv_counts": 0.0, "cv2_probs": 0.0}
+    counts = np.bincount(idx.ravel(), minlength=E).astype(np.float64)
+    P = p.astype(np.float64).mean(axis=0)
+    mean_c = counts.mean()
+    cv_counts = float(np.sqrt(np.mean((counts - mean_c) ** 2)) / mean_c)
+    mean_p = P.mean()
+    cv2_probs = float(np.mean((P - mean_p) ** 2) / mean_p ** 2)
+    aux_all = float(E * np.sum(counts / (T * k) * P))
+    return {"aux_all_choices": aux_all, "cv_counts": cv_counts, "cv2_probs": cv2_probs}
+
+
 def moe_forward(x, W_r, b_r, W1, W3, W2, *, k: int, gate_mode: int, act: int,
                 capacity_factor: float, rows: Optional[Sequence[int]] = None,
-                logits: Optional[np.ndarray] = None, hidden_bf16: bool = False) -> dict:
+                logits: Optional[np.ndarray] = None, hidden_bf16: bool = False,
+                shared: Optional[tuple] = None) -> dict:
     """The whole layer: routing for every token, y for every token or for ``rows``.
 
     x: [T][d]; W_r: [E][d]; b_r: [E] or None; W1, W3: [E][d_ff][d] (W3 None for
@@ -224,9 +260,18 @@ def moe_forward(x, W_r, b_r, W1, W3, W2, *, k: int, gate_mode: int, act: int,
     ``rows``: compute y only for these tokens (routing, capacity and losses are
     always global; y_t depends on x_t and the global routing only).
     ``hidden_bf16``: round each expert's hidden activation to bf16 (see expert_ffn).
+    ``shared``: (W1s, W3s, W2s), each with n_s experts shaped like W1, W3, W2:
+    shared experts that every token visits ("Mixture of experts", section
+    "Total versus active parameters": "shared experts every token visits").
+    Reading: a shared expert is an FFN of the same shape and activation as the
+    routed ones, applied to every token with weight 1, outside routing,
+    capacity and the losses; its output is added after the routed sum, in
+    shared-expert order, so a token whose routed assignments were all dropped
+    still gets it.
 
     y_t = sum over kept assignments (t, j), in slot order j, of
-    g_tj * E_{idx_tj}(x_t); a token with all assignments dropped gets y_t = 0.
+    g_tj * E_{idx_tj}(x_t), plus sum_s S_s(x_t); a token with all routed
+    assignments dropped and no shared experts gets y_t = 0.
     """
     x = np.asarray(x)
     T = x.shape[0]
@@ -256,7 +301,13 @@ def moe_forward(x, W_r, b_r, W1, W3, W2, *, k: int, gate_mode: int, act: int,
     y = np.zeros((len(want), d), np.float64)
     for j in range(k):                  # slot order
         y += contrib[:, j]
+    if shared is not None:
+        W1s, W3s, W2s = shared
+        xs = np.asarray(x[want], np.float64)
+        for si in range(len(W1s)):      # shared-expert order, after the routed sum
+            y += expert_ffn(xs, W1s[si], None if W3s is None else W3s[si], W2s[si], act, hidden_bf16)
     res = {"logits": h32, "p": p, "lse": lse, "idx": idx, "gate": g, "capacity": C,
            "y": y, "rows": want, "aux": aux, "z": z}
+    res.update(balance_losses(p, idx, E))
     res.update(slots)
     return res

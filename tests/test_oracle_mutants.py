@@ -3,7 +3,8 @@
 The mutants live only here, on the CPU; they patch the oracle module for the
 duration of one check.  This shows the pins in test_oracle_pins.py would catch
 a dropped term, a wrong sign, a wrong index or tie rule, a transposed operand,
-an off-by-one capacity or a wrong slot priority.
+an off-by-one capacity, a wrong slot priority, a wrong moment in the balance
+statistics or shared experts applied to the wrong tokens or weights.
 """
 import numpy as np
 import pytest
@@ -83,7 +84,47 @@ def _logits_dropped_bias(x, W_r, b_r=None):
     return _orig["router_logits"](x, W_r, None)
 
 
-_orig = {n: getattr(M, n) for n in ("top_k", "gates", "expert_ffn", "aux_and_z", "assign_slots", "router_logits")}
+def _balance_sample_std(p, idx, E):
+    r = _orig["balance_losses"](p, idx, E)
+    counts = np.bincount(idx.ravel(), minlength=E).astype(np.float64)
+    if len(idx) and E > 1:
+        r["cv_counts"] = float(counts.std(ddof=1) / counts.mean())
+    return r
+
+
+def _balance_cv_not_squared(p, idx, E):
+    r = _orig["balance_losses"](p, idx, E)
+    r["cv2_probs"] = float(np.sqrt(r["cv2_probs"]))
+    return r
+
+
+def _balance_first_choices_only(p, idx, E):
+    r = _orig["balance_losses"](p, idx, E)
+    if len(idx):
+        f = np.bincount(idx[:, 0], minlength=E) / len(idx)
+        r["aux_all_choices"] = float(E * np.sum(f * p.mean(axis=0)))
+    return r
+
+
+def _shared_only_for_kept_tokens(*args, shared=None, **kw):
+    r = _orig["moe_forward"](*args, shared=None, **kw)
+    if shared is not None:
+        full = _orig["moe_forward"](*args, shared=shared, **kw)
+        keep = r["kept"][r["rows"]].any(axis=1)
+        r["y"] = np.where(keep[:, None], full["y"], r["y"])
+    return r
+
+
+def _shared_weighted_by_gate(*args, shared=None, **kw):
+    r = _orig["moe_forward"](*args, shared=None, **kw)
+    if shared is not None:
+        full = _orig["moe_forward"](*args, shared=shared, **kw)
+        r["y"] = r["y"] + r["gate"][r["rows"], :1] * (full["y"] - r["y"])
+    return r
+
+
+_orig = {n: getattr(M, n) for n in ("top_k", "gates", "expert_ffn", "aux_and_z", "assign_slots", "router_logits",
+                                     "balance_losses", "moe_forward")}
 
 MUTANTS = {
     "top_k ties to the higher index": ("top_k", _top_k_last_index_on_ties),
@@ -97,6 +138,11 @@ MUTANTS = {
     "slots by choice before token": ("assign_slots", _slots_choice_major),
     "router weight transposed": ("router_logits", _logits_transposed_router),
     "router bias dropped": ("router_logits", _logits_dropped_bias),
+    "CV with the sample standard deviation": ("balance_losses", _balance_sample_std),
+    "cv^2 left unsquared": ("balance_losses", _balance_cv_not_squared),
+    "all-choices loss over first choices": ("balance_losses", _balance_first_choices_only),
+    "shared experts skipped for dropped tokens": ("moe_forward", _shared_only_for_kept_tokens),
+    "shared experts scaled by the gate": ("moe_forward", _shared_weighted_by_gate),
 }
 
 PINS = [
@@ -115,6 +161,12 @@ PINS = [
     P.test_worked_example_reconstruction,
     lambda: [P.test_single_expert_is_the_dense_ffn(a, g) for a in (0, 1) for g in (0, 1)],
     lambda: [P.test_k_equals_E_is_the_dense_softmax_mixture(a) for a in (0, 1)],
+    P.test_balance_losses_are_zero_and_one_under_uniform_routing,
+    P.test_balance_losses_closed_forms_when_collapsed,
+    P.test_all_choices_loss_equals_switch_loss_at_k1_and_counts_every_choice,
+    lambda: [P.test_shared_expert_with_silent_routed_experts_is_the_dense_ffn(a) for a in (0, 1)],
+    P.test_shared_copy_of_the_single_expert_doubles_the_output,
+    P.test_dropped_tokens_still_get_the_shared_experts,
 ]
 
 

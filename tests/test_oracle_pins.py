@@ -156,6 +156,54 @@ def test_z_loss_closed_form():
         assert z == pytest.approx((c + math.log(E)) ** 2, rel=1e-12)
 
 
+def test_balance_losses_are_zero_and_one_under_uniform_routing():
+    """Uniform routing: equal assignment counts and equal P_i give a coefficient
+    of variation 0, cv^2 0, and the all-choices Switch loss E*sum f P = 1."""
+    for E, k in [(4, 1), (8, 2), (16, 4)]:
+        T = 8 * E
+        idx = np.stack([(np.arange(T) + j) % E for j in range(k)], axis=1)  # each expert k*T/E times
+        p = np.full((T, E), 1.0 / E)
+        r = O.balance_losses(p, idx, E)
+        assert r["cv_counts"] == pytest.approx(0.0, abs=1e-15)
+        assert r["cv2_probs"] == pytest.approx(0.0, abs=1e-15)
+        assert r["aux_all_choices"] == pytest.approx(1.0, abs=1e-12)
+
+
+def test_balance_losses_closed_forms_when_collapsed():
+    """All T tokens to expert 0 with probability 1 (k = 1): counts (T, 0, ..., 0)
+    have mean T/E and standard deviation (T/E) sqrt(E - 1), so CV = sqrt(E - 1);
+    P = e_0 gives cv^2 = E - 1; the all-choices loss equals E."""
+    for E in (2, 5, 8, 64):
+        T = 3 * E
+        idx = np.zeros((T, 1), np.int64)
+        p = np.zeros((T, E)); p[:, 0] = 1.0
+        r = O.balance_losses(p, idx, E)
+        assert r["cv_counts"] == pytest.approx(math.sqrt(E - 1), rel=1e-12)
+        assert r["cv2_probs"] == pytest.approx(E - 1, rel=1e-12)
+        assert r["aux_all_choices"] == pytest.approx(E, rel=1e-12)
+
+
+def test_all_choices_loss_equals_switch_loss_at_k1_and_counts_every_choice():
+    """k = 1: first choices are all choices, so the two losses agree; k = 2 with
+    second choices on one expert: f over all choices differs from first choices."""
+    E, T, d = 6, 40, 9
+    x = rng.normal(size=(T, d)); W_r = rng.normal(size=(E, d))
+    z = np.zeros((E, 2, d)), np.zeros((E, d, 2))
+    r = O.moe_forward(x, W_r, None, z[0], None, z[1], k=1, gate_mode=O.GATE_SWITCH, act=O.ACT_RELU,
+                      capacity_factor=0.0)
+    assert r["aux_all_choices"] == pytest.approx(r["aux"], rel=1e-12)
+    # hand-made: first choices uniform over experts 0..3, every second choice = expert 5
+    T2 = 8
+    idx = np.stack([np.arange(T2) % 4, np.full(T2, 5)], axis=1)
+    P = np.arange(1.0, E + 1) / np.sum(np.arange(1.0, E + 1))   # non-uniform, so f matters
+    p = np.tile(P, (T2, 1))
+    bl = O.balance_losses(p, idx, E)
+    counts = np.array([2, 2, 2, 2, 0, 8], float)
+    assert bl["aux_all_choices"] == pytest.approx(E * np.sum(counts / 16 * P), rel=1e-12)
+    assert bl["aux_all_choices"] != pytest.approx(E * np.sum(np.array([2, 2, 2, 2, 0, 0]) / 8 * P), rel=1e-6)
+    assert bl["cv_counts"] == pytest.approx(counts.std() / counts.mean(), rel=1e-12)
+
+
 # ---------------------------------------------------------------- capacity
 def test_capacity_formula():
     """Capacity and dropped tokens: C = tokens/experts x factor (x k for top-k)."""
@@ -262,7 +310,8 @@ def test_sampled_rows_equal_full_rows_and_dropped_tokens_are_zero():
     rows = [0, 5, 59, 31]
     part = O.moe_forward(x, W_r, None, W1, None, W2, k=k, gate_mode=O.GATE_RENORM,
                          act=O.ACT_RELU, capacity_factor=0.5, rows=rows)
-    np.testing.assert_array_equal(part["y"], full["y"][rows])
+    # equal up to fp64 rounding: BLAS may sum a 4-row batch in another order than a 60-row one
+    np.testing.assert_allclose(part["y"], full["y"][rows], rtol=1e-13, atol=1e-13)
     gone = ~full["kept"].any(axis=1)
     assert gone.any() and np.all(full["y"][gone] == 0)
     # a partially dropped token keeps its surviving gate as it is (no renormalisation)
@@ -302,3 +351,52 @@ def test_hidden_bf16_is_exact_when_the_hidden_values_are_bf16_numbers():
     np.testing.assert_array_equal(a["y"], b["y"])
     h = rng.normal(size=5000) * 10
     assert np.all(np.abs(O.round_to_bf16(h) - h) <= (2.0 ** -8 + 2.0 ** -23) * np.abs(h))  # unit roundoff 2^-8, via fp32
+
+
+# ---------------------------------------------------------------- shared experts
+@pytest.mark.parametrize("act", [O.ACT_RELU, O.ACT_SWIGLU])
+def test_shared_expert_with_silent_routed_experts_is_the_dense_ffn(act):
+    """Routed experts whose output is zero (W2 = 0): y is the sum of the shared
+    experts' dense FFNs, for every token."""
+    T, d, dff, E, ns = 19, 8, 12, 4, 2
+    x = rng.normal(size=(T, d)); W_r = rng.normal(size=(E, d))
+    W1 = rng.normal(size=(E, dff, d)); W3 = rng.normal(size=(E, dff, d)); W2 = np.zeros((E, d, dff))
+    S1 = rng.normal(size=(ns, dff, d)); S3 = rng.normal(size=(ns, dff, d)); S2 = rng.normal(size=(ns, d, dff))
+    r = O.moe_forward(x, W_r, None, W1, W3 if act else None, W2, k=2, gate_mode=O.GATE_RENORM, act=act,
+                      capacity_factor=0.0, shared=(S1, S3 if act else None, S2))
+    ref = sum(_torch_ffn(torch.tensor(x), torch.tensor(S1[s]), torch.tensor(S3[s]), torch.tensor(S2[s]), act)
+              for s in range(ns))
+    np.testing.assert_allclose(r["y"], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_shared_copy_of_the_single_expert_doubles_the_output():
+    """E = 1, k = 1 (gate 1) and one shared expert with the same weights: y = 2 FFN(x)."""
+    T, d, dff = 11, 6, 10
+    x = rng.normal(size=(T, d)); W_r = rng.normal(size=(1, d))
+    W1 = rng.normal(size=(1, dff, d)); W2 = rng.normal(size=(1, d, dff))
+    r = O.moe_forward(x, W_r, None, W1, None, W2, k=1, gate_mode=O.GATE_RENORM, act=O.ACT_RELU,
+                      capacity_factor=0.0, shared=(W1.copy(), None, W2.copy()))
+    ref = _torch_ffn(torch.tensor(x), torch.tensor(W1[0]), None, torch.tensor(W2[0]), O.ACT_RELU)
+    np.testing.assert_allclose(r["y"], 2 * ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_dropped_tokens_still_get_the_shared_experts():
+    """Capacity drops routed assignments only: a token with every routed choice
+    dropped gets exactly the shared output; routing, counts and losses do not
+    see the shared experts."""
+    T, d, dff, E, k = 50, 8, 12, 4, 2
+    x = rng.normal(size=(T, d)); W_r = rng.normal(size=(E, d))
+    W1 = rng.normal(size=(E, dff, d)); W2 = rng.normal(size=(E, d, dff))
+    S1 = rng.normal(size=(1, dff, d)); S2 = rng.normal(size=(1, d, dff))
+    plain = O.moe_forward(x, W_r, None, W1, None, W2, k=k, gate_mode=O.GATE_RENORM, act=O.ACT_RELU,
+                          capacity_factor=0.25)
+    sh = O.moe_forward(x, W_r, None, W1, None, W2, k=k, gate_mode=O.GATE_RENORM, act=O.ACT_RELU,
+                       capacity_factor=0.25, shared=(S1, None, S2))
+    gone = ~plain["kept"].any(axis=1)
+    assert gone.sum() > 0
+    shared_out = _torch_ffn(torch.tensor(x), torch.tensor(S1[0]), None, torch.tensor(S2[0]), O.ACT_RELU).numpy()
+    np.testing.assert_allclose(sh["y"][gone], shared_out[gone], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sh["y"], plain["y"] + shared_out, rtol=1e-12, atol=1e-12)
+    for key in ("idx", "counts", "dest_row", "kept"):
+        np.testing.assert_array_equal(sh[key], plain[key])
+    assert (sh["aux"], sh["z"], sh["dropped"]) == (plain["aux"], plain["z"], plain["dropped"])
