@@ -50,15 +50,17 @@ def load_peaks():
 def layer_work(w, kept_counts, hidden="bf16x2"):
     """Algorithmic FLOPs and bytes of the layer and of each grouped GEMM launch.
 
-    Counts kept assignments only.  Bytes: weights of experts with >= 1 kept
-    row (read once), x read once, y written once, W_r; per GEMM also its own
-    input and output activations (the expert-sorted rows; the hidden
-    activation at 4 bytes per element when held as a hi + lo bf16 pair).
+    Counts kept assignments only, plus T rows per shared expert.  Bytes:
+    weights of experts with >= 1 kept row and of every shared expert (read
+    once), x read once, y written once, W_r; per GEMM also its own input and
+    output activations (the expert-sorted rows; the hidden activation at 4
+    bytes per element when held as a hi + lo bf16 pair).
     """
     elt = 2 if w.dtype == 1 else 4
     h_elt = 4 if (w.dtype == 1 and hidden == "bf16x2") else elt
-    S = int(sum(kept_counts))
-    active = sum(1 for c in kept_counts if c > 0)
+    n_sh = getattr(w, "n_shared", 0)
+    S = int(sum(kept_counts)) + n_sh * w.T
+    active = sum(1 for c in kept_counts if c > 0) + n_sh
     nproj1 = 2 if w.act == 1 else 1
     w1_bytes = active * nproj1 * w.d_ff * w.d * elt
     w2_bytes = active * w.d * w.d_ff * elt
@@ -66,7 +68,7 @@ def layer_work(w, kept_counts, hidden="bf16x2"):
     flops1 = 2.0 * S * w.d * w.d_ff * nproj1
     flops2 = 2.0 * S * w.d_ff * w.d
     gemm1_bytes = w1_bytes + S * w.d * elt + S * w.d_ff * h_elt
-    out2 = S * w.d * (elt if w.k == 1 else 4)
+    out2 = S * w.d * (elt if (w.k == 1 and n_sh == 0) else 4)
     gemm2_bytes = w2_bytes + S * w.d_ff * h_elt + out2
     layer_bytes = w1_bytes + w2_bytes + 2 * w.T * w.d * elt + w.E * w.d * 4
     return {"S": S, "active_experts": active, "flops_layer": flops_router + flops1 + flops2,
@@ -197,7 +199,7 @@ def rank_seed(base_seed, rank):
 
 
 def config_of(w, n_gpus):
-    return {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "k": w.k, "d_ff": w.d_ff,
+    return {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "k": w.k, "d_ff": w.d_ff, "n_shared": w.n_shared,
             "act": "swiglu" if w.act == 1 else "relu", "gate": "renorm" if w.gate == 1 else "switch",
             "capacity_factor": w.capacity_factor, "tokens_per_gpu": w.T,
             "parallelism": "replicas" if n_gpus > 1 else "single",
@@ -223,9 +225,13 @@ def cpu_oracle_run(w, inp, n_tokens):
     b_r = None if inp["b_r"] is None else inp["b_r"].float().cpu().numpy()
     W1, W2 = Host(inp["W1"]), Host(inp["W2"])
     W3 = None if inp["W3"] is None else Host(inp["W3"])
+    shared = None
+    if getattr(w, "n_shared", 0):
+        ids = range(w.E, w.E + w.n_shared)
+        shared = ([W1[e] for e in ids], None if W3 is None else [W3[e] for e in ids], [W2[e] for e in ids])
     t0 = time.perf_counter()
     oracle.moe_forward(x, W_r, b_r, W1, W3, W2, k=w.k, gate_mode=w.gate, act=w.act,
-                       capacity_factor=w.capacity_factor)
+                       capacity_factor=w.capacity_factor, shared=shared)
     return time.perf_counter() - t0
 
 
@@ -291,7 +297,7 @@ def main():
     if rank > 0:
         inp["x"] = make_inputs(w.with_(seed=rank_seed(w.seed, rank)), device=dev, weights=False)["x"]
     layer = MoELayer(w.E, w.k, w.d, w.d_ff, act=w.act, gate_mode=w.gate, capacity_factor=w.capacity_factor,
-                     dtype=torch_dtype(w.dtype), hidden=args.hidden)
+                     dtype=torch_dtype(w.dtype), hidden=args.hidden, n_shared=w.n_shared)
     ws = layer.workspace(w.T, dev)
     y = torch.empty((w.T, w.d), dtype=inp["x"].dtype, device=dev)
     stats = (torch.empty(w.E, dtype=torch.int32, device=dev), torch.empty(1, dtype=torch.int32, device=dev),

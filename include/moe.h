@@ -130,6 +130,21 @@ MOE_API int moe_create(int num_experts, int k, int d, int d_ff, int act, int gat
  */
 MOE_API int moe_set_hidden_precision(moe_handle h, int mode);
 
+/*
+ * Shared experts ("Mixture of experts", rayaq.ca, section "Total versus
+ * active parameters": shared experts every token visits).  With n_shared > 0
+ * the layer adds, for every token, the outputs of n_shared more experts of
+ * the same shape and activation, each with weight 1, after the gated routed
+ * sum:  y_t = sum_j g_tj E_{idx_tj}(x_t) + sum_s S_s(x_t).  Their weights
+ * follow the routed experts' in W1, W3 and W2, which then hold E + n_shared
+ * experts (index E + s is shared expert s).  Shared experts take no part in
+ * routing, capacity, expert_counts, dropped or the losses; a token whose
+ * routed choices were all dropped still gets them.  0 <= n_shared <= 8 and
+ * E + n_shared <= 256, else MOE_ERR_INVALID_ARG.  Changes
+ * moe_workspace_bytes().  Default 0.
+ */
+MOE_API int moe_set_shared_experts(moe_handle h, int n_shared);
+
 /* Free a handle created by moe_create.  NULL is accepted. */
 MOE_API int moe_destroy(moe_handle h);
 
@@ -150,7 +165,8 @@ MOE_API size_t moe_workspace_bytes(moe_handle h, int64_t T);
  * One forward pass of the layer over T tokens (T >= 0).
  *   x            [T][d]        layer input (bf16 or fp32)
  *   W_r          [E][d]  fp32  router weight;   b_r [E] fp32 bias or NULL
- *   W1           [E][d_ff][d]  first expert projection
+ *   W1           [E][d_ff][d]  first expert projection ([E + n_shared] rows of
+ *                              experts with shared experts, see moe_set_shared_experts)
  *   W3           [E][d_ff][d]  SwiGLU value projection; must be NULL for ReLU
  *   W2           [E][d][d_ff]  second expert projection
  *   y            [T][d]        output (same dtype as x); 0 for fully dropped tokens
@@ -167,6 +183,26 @@ MOE_API int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r
                 const void* W1, const void* W3, const void* W2, void* y,
                 int32_t* expert_counts, int32_t* dropped, float* aux_loss, float* z_loss,
                 void* workspace, size_t workspace_bytes, const moe_debug* dbg, void* stream);
+
+/*
+ * The alternative load-balancing statistics of the last moe_forward that used
+ * `workspace` with T tokens (stream-ordered on `stream`), unscaled, written as
+ * three fp32 values to the device pointer `out`:
+ *   out[0]  E * sum_i (c_i / (T k)) P_i: the Switch loss with f_i counted over
+ *           all k choices ("Mixture of experts", rayaq.ca, section "The
+ *           load-balancing loss");
+ *   out[1]  the coefficient of variation std(c) / mean(c) of the assignment
+ *           counts c_i (= expert_counts) over the E experts ("Mixture of
+ *           Experts (MoE)", inferensys.com: 0.01 times the coefficient of
+ *           variation of expert assignment counts);
+ *   out[2]  the squared coefficient of variation var(P) / mean(P)^2 of the
+ *           mean router probabilities P_i ("Mixture of Experts (MoE) Language
+ *           Models", chipfoundryservices.com: cv^2 of the router probabilities).
+ * Moments are over the E values (divided by E).  The forward pass computes
+ * them in its reduction at no extra launch; this call copies them (T = 0
+ * writes zeros).  Returns MOE_OK, MOE_ERR_INVALID_ARG or MOE_ERR_CUDA.
+ */
+MOE_API int moe_balance_losses(moe_handle h, int64_t T, const void* workspace, float* out, void* stream);
 
 /*
  * moe_forward for callers that cannot allocate device memory (no counterpart

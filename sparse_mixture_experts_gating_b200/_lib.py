@@ -21,6 +21,8 @@ SIGNATURES = {
     "moe_destroy": (c_int, [c_void_p]),
     "moe_capacity": (c_int64, [c_void_p, c_int64]),
     "moe_workspace_bytes": (c_size_t, [c_void_p, c_int64]),
+    "moe_set_shared_experts": (c_int, [c_void_p, c_int]),
+    "moe_balance_losses": (c_int, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p]),
     "moe_forward": (c_int, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                             c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p,
                             c_void_p]),

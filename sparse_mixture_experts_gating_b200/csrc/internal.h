@@ -38,6 +38,8 @@ struct RoutingArgs {
   int32_t* tot_cnt1;   // [E]   first-choice count of each expert (scan)
   float* tot_psum;     // [E]   probability sum of each expert (scan)
   int32_t* scan_ticket;  // zeroed by the router; the scan's last block resets it
+  float* balance_out;    // [3] aux over all choices, CV of counts, cv^2 of P (scan)
+  int n_shared;          // shared experts: groups E .. E + n_shared - 1 of T rows each
   int32_t* row_token;  // [S_max]
   float* row_gate;     // [S_max]
   void* Xp;            // [S_max][d]
@@ -79,8 +81,10 @@ bool make_map_planes_bf16(CUtensorMap* m, const void* base, uint64_t plane_strid
 cudaError_t launch_scan(const RoutingArgs& a, cudaStream_t s);
 cudaError_t launch_dispatch(const RoutingArgs& a, cudaStream_t s);
 // y_t = sum over kept choices j (in order j) of sum over the ksplit partials
-// (in order) of Yp[partial][dest_row[t][j]].
-cudaError_t launch_combine(int64_t T, int k, int d, int y_is_bf16, const int32_t* dest_row, const float* Yp,
+// (in order) of Yp[partial][dest_row[t][j]], then (in order s) of the rows
+// *shared_base + s * T + t of the n_shared shared experts.
+cudaError_t launch_combine(int64_t T, int k, int d, int y_is_bf16, const int32_t* dest_row, int n_shared,
+                           const int32_t* shared_base, const float* Yp,
                            int ksplit, int64_t split_stride, void* y, float* y_f32, cudaStream_t s);
 
 // K ranges of the second projection: split K when the tiles alone cannot

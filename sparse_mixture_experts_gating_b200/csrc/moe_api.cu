@@ -21,7 +21,8 @@
 struct moe_layer {
   int E, k, d, d_ff, act, gate_mode, dtype;
   double capacity_factor;
-  int hidden;  // MOE_HIDDEN_*
+  int hidden;    // MOE_HIDDEN_*
+  int n_shared;  // shared experts every token visits (weights E .. E + n_shared - 1)
 };
 
 // Sticky device error word (one per device that loads the library).
@@ -73,8 +74,12 @@ cudaError_t device_info(DeviceInfo** out) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// The second projection writes fp32 rows for the combine (k > 1, shared
+// experts, or fp32 layers) instead of scattering bf16 rows straight into y.
+bool need_yp_of(const moe_layer& L) { return !(L.dtype == MOE_BF16 && L.k == 1 && L.n_shared == 0); }
+
 int ksplit_of(const moe_layer& L, int64_t s_max) {
-  return (L.dtype == MOE_BF16 && !(L.k == 1)) ? gemm2_ksplit(s_max, L.E, L.d, L.d_ff) : 1;
+  return (L.dtype == MOE_BF16 && need_yp_of(L)) ? gemm2_ksplit(s_max, L.E + L.n_shared, L.d, L.d_ff) : 1;
 }
 
 int64_t capacity_of(const moe_layer& L, int64_t T) {
@@ -102,9 +107,10 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   const int64_t Tk = T * L.k;
   w.s_max = Tk;
   if (w.capacity >= 0) w.s_max = std::min<int64_t>(Tk, static_cast<int64_t>(L.E) * w.capacity);
+  w.s_max += static_cast<int64_t>(L.n_shared) * T;  // every token's rows of the shared experts
   w.nblk = static_cast<int>((T + kRouterTokens - 1) / kRouterTokens);
   const size_t elt = L.dtype == MOE_BF16 ? 2 : 4;
-  w.need_yp = !(L.dtype == MOE_BF16 && L.k == 1);
+  w.need_yp = need_yp_of(L);
   w.split = L.dtype == MOE_BF16 && L.hidden == MOE_HIDDEN_BF16X2;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
@@ -121,7 +127,8 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   w.counts = take(sizeof(int32_t) * L.E);
   w.offsets = take(sizeof(int32_t) * (L.E + 1));
   w.mprefix = take(sizeof(int32_t) * (L.E + 1));
-  w.scal = take(sizeof(int32_t) * L.E + sizeof(float) * L.E + 64);  // scan totals and ticket
+  // scan totals [E] + [E], the scan ticket, the three balance statistics
+  w.scal = take(sizeof(int32_t) * L.E + sizeof(float) * L.E + 64);
   const bool tc_router = L.dtype == MOE_BF16 && L.E <= kRouterTcMaxE;
   w.wsplit = take(tc_router ? 3 * sizeof(uint16_t) * router_pad_e(L.E) * static_cast<size_t>(L.d) : 0);
   w.rpart = take(tc_router ? router_partials_bytes(T, L.E, L.d) : 0);
@@ -130,9 +137,16 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   w.Hp_lo = take(w.split ? elt * static_cast<size_t>(w.s_max) * L.d_ff : 0);
   w.ksplit = ksplit_of(L, w.s_max);
   // Yp holds ksplit partials of s_max rows; reserve the most any smaller batch
-  // needs as well, so a workspace sized for some T serves every smaller batch
+  // needs as well, so a workspace sized for some T serves every smaller batch.
+  // ksplit(s) depends on s through the m-tile bound floor(s / 128) + min(groups, s),
+  // which changes at every s below the group count and then only at multiples
+  // of 128, and ksplit(s) = 1 once s > 148 * 128; the product ksplit(s) * s
+  // peaks at the last s before each change.
   int64_t yp_rows = w.ksplit * w.s_max;
-  for (int64_t s = 1; s < w.s_max && s <= 256; ++s) yp_rows = std::max<int64_t>(yp_rows, ksplit_of(L, s) * s);
+  const int64_t groups = L.E + L.n_shared;
+  for (int64_t s = 1; s < w.s_max && s <= groups; ++s) yp_rows = std::max<int64_t>(yp_rows, ksplit_of(L, s) * s);
+  for (int64_t s = 127; s < w.s_max && s <= 148 * 128; s += 128)
+    yp_rows = std::max<int64_t>(yp_rows, ksplit_of(L, s) * s);
   w.Yp = take(w.need_yp ? sizeof(float) * static_cast<size_t>(yp_rows) * L.d : 0);
   w.total = o;
   return w;
@@ -194,7 +208,8 @@ int moe_create(int num_experts, int k, int d, int d_ff, int act, int gate_mode, 
   if (!(capacity_factor == capacity_factor)) return fail(MOE_ERR_INVALID_ARG, "moe_create: capacity_factor is NaN");
   if (dtype == MOE_BF16 && (d % 8 != 0 || d_ff % 8 != 0))
     return fail(MOE_ERR_UNSUPPORTED, "moe_create: bf16 layers need d and d_ff to be multiples of 8");
-  moe_layer* L = new moe_layer{num_experts, k, d, d_ff, act, gate_mode, dtype, capacity_factor, MOE_HIDDEN_BF16X2};
+  moe_layer* L =
+      new moe_layer{num_experts, k, d, d_ff, act, gate_mode, dtype, capacity_factor, MOE_HIDDEN_BF16X2, 0};
   *out = L;
   t_err.clear();
   return MOE_OK;
@@ -205,6 +220,33 @@ int moe_set_hidden_precision(moe_handle h, int mode) {
   if (mode != MOE_HIDDEN_BF16X2 && mode != MOE_HIDDEN_BF16)
     return fail(MOE_ERR_INVALID_ARG, "moe_set_hidden_precision: unknown mode");
   h->hidden = mode;
+  return MOE_OK;
+}
+
+int moe_set_shared_experts(moe_handle h, int n_shared) {
+  if (h == nullptr) return fail(MOE_ERR_INVALID_ARG, "moe_set_shared_experts: handle is NULL");
+  if (n_shared < 0 || n_shared > 8 || h->E + n_shared > 256)
+    return fail(MOE_ERR_INVALID_ARG, "moe_set_shared_experts: need 0 <= n_shared <= 8 and E + n_shared <= 256");
+  h->n_shared = n_shared;
+  return MOE_OK;
+}
+
+int moe_balance_losses(moe_handle h, int64_t T, const void* workspace, float* out, void* stream) {
+  if (h == nullptr || T < 0 || out == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "moe_balance_losses: NULL handle or output, or T < 0");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (T == 0) {
+    e = cudaMemsetAsync(out, 0, 3 * sizeof(float), s);
+  } else {
+    if (workspace == nullptr) return fail(MOE_ERR_INVALID_ARG, "moe_balance_losses: workspace is NULL");
+    const Layout w = make_layout(*h, T);
+    const uint8_t* src = static_cast<const uint8_t*>(workspace) + w.scal +
+                         (sizeof(int32_t) + sizeof(float)) * h->E + 16;
+    e = cudaMemcpyAsync(out, src, 3 * sizeof(float), cudaMemcpyDeviceToDevice, s);
+  }
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_balance_losses: ") + cudaGetErrorString(e));
+  t_err.clear();
   return MOE_OK;
 }
 
@@ -293,6 +335,8 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   r.tot_cnt1 = reinterpret_cast<int32_t*>(ws + w.scal);
   r.tot_psum = reinterpret_cast<float*>(ws + w.scal + sizeof(int32_t) * L.E);
   r.scan_ticket = reinterpret_cast<int32_t*>(ws + w.scal + (sizeof(int32_t) + sizeof(float)) * L.E);
+  r.balance_out = reinterpret_cast<float*>(ws + w.scal + (sizeof(int32_t) + sizeof(float)) * L.E + 16);
+  r.n_shared = L.n_shared;
   r.row_gate = reinterpret_cast<float*>(ws + w.row_gate);
   r.Xp = ws + w.Xp;
   r.dropped = dropped;
@@ -308,7 +352,7 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   GemmArgs g1;
   memset(&g1, 0, sizeof(g1));
   g1.epi = L.act == MOE_ACT_SWIGLU ? EPI_SWIGLU_BF16 : EPI_RELU_BF16;
-  g1.E = L.E;
+  g1.E = L.E + L.n_shared;  // routed groups, then one group of T rows per shared expert
   g1.N = L.d_ff;
   g1.K = L.d;
   g1.a_rows = w.s_max;
@@ -380,7 +424,7 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   record(dbg, MOE_STAGE_GEMM2, 1, s);
   if (w.need_yp) {
     record(dbg, MOE_STAGE_COMBINE, 0, s);
-    if ((rc = check(launch_combine(T, L.k, L.d, L.dtype == MOE_BF16, r.dest_row,
+    if ((rc = check(launch_combine(T, L.k, L.d, L.dtype == MOE_BF16, r.dest_row, L.n_shared, r.offsets + L.E,
                                    reinterpret_cast<const float*>(ws + w.Yp), w.ksplit,
                                    static_cast<int64_t>(w.s_max) * L.d, y, dbg ? dbg->y_f32 : nullptr, s),
                     "combine")) != MOE_OK)

@@ -299,39 +299,70 @@ __device__ __forceinline__ F block_sum(F v, F* s_red) {
   return t;  // valid in thread 0
 }
 
-// Capacity, expert offsets, tile prefix, dropped count, aux loss and z-loss
-// from the per-expert totals (thread e < E holds expert e's), by all SCAN_T
-// threads of one block.
+// Sum over the block in a fixed tree order, returned to every thread.
+template <typename F>
+__device__ __forceinline__ F block_sum_all(F v, F* s_red, F* s_out) {
+  const F t = block_sum<F>(v, s_red);
+  if (threadIdx.x == 0) *s_out = t;
+  __syncthreads();
+  const F r = *s_out;
+  __syncthreads();
+  return r;
+}
+
+// Capacity, expert offsets, tile prefix, dropped count, aux loss, z-loss and
+// the alternative balance statistics from the per-expert totals (thread e < E
+// holds routed expert e's; threads E .. E + n_shared - 1 stand for the shared
+// experts' groups of T rows, which take no part in capacity, counts or
+// losses), by all SCAN_T threads of one block.
 __device__ __forceinline__ void scan_finalize(const RoutingArgs& a, int cnt, int c1, float ps, int* s_warp,
-                                              int* s_redi, double* s_redd) {
+                                              int* s_redi, double* s_redd, double* s_bcast) {
   const int tid = threadIdx.x, E = a.E, nb = a.nblk;
-  const int kept =
-      tid < E ? ((a.capacity < 0) ? cnt : static_cast<int>((int64_t)cnt < a.capacity ? (int64_t)cnt : a.capacity))
-              : 0;
+  const int groups = E + a.n_shared;
+  const bool routed = tid < E;
+  int kept = 0;
+  if (routed) kept = (a.capacity < 0) ? cnt : static_cast<int>((int64_t)cnt < a.capacity ? (int64_t)cnt : a.capacity);
+  else if (tid < groups) kept = static_cast<int>(a.T);
   const int mt = (kept + kTileM - 1) / kTileM;
-  int total_kept = 0, total_tiles = 0;
-  const int off = block_exscan_int(kept, s_warp, total_kept);
+  int total_rows = 0, total_tiles = 0;
+  const int off = block_exscan_int(kept, s_warp, total_rows);
   const int mp = block_exscan_int(mt, s_warp, total_tiles);
-  if (tid < E) {
-    a.counts[tid] = cnt;
+  if (routed) a.counts[tid] = cnt;
+  if (tid < groups) {
     a.offsets[tid] = off;
     a.mprefix[tid] = mp;
-    if (a.offsets_out != nullptr) a.offsets_out[tid] = off;
   }
-  const int drop = block_sum<int>(tid < E ? cnt - kept : 0, s_redi);
-  const double auxp =
-      block_sum<double>(tid < E ? static_cast<double>(c1) * static_cast<double>(ps) : 0.0, s_redd);
+  // the debug copy holds the routed experts' offsets [E + 1] (offsets[E] = kept routed
+  // rows: the total without shared experts, else thread E's prefix; E < 256 then)
+  if (a.offsets_out != nullptr) {
+    if (tid < E) a.offsets_out[tid] = off;
+    if (a.n_shared == 0 ? tid == 0 : tid == E) a.offsets_out[E] = a.n_shared == 0 ? total_rows : off;
+  }
+  const int drop = block_sum<int>(routed ? cnt - kept : 0, s_redi);
+  const double T = static_cast<double>(a.T);
+  const double Pe = routed ? static_cast<double>(ps) / T : 0.0;  // mean router probability of e
+  const double auxp = block_sum<double>(routed ? static_cast<double>(c1) * static_cast<double>(ps) : 0.0, s_redd);
+  // alternative balance statistics (population moments over the E experts)
+  const double mean_c = block_sum_all<double>(routed ? static_cast<double>(cnt) : 0.0, s_redd, s_bcast) / E;
+  const double mean_p = block_sum_all<double>(Pe, s_redd, s_bcast) / E;
+  const double dc = routed ? static_cast<double>(cnt) - mean_c : 0.0;
+  const double dp = routed ? Pe - mean_p : 0.0;
+  const double var_c = block_sum<double>(dc * dc, s_redd) / E;
+  const double var_p = block_sum<double>(dp * dp, s_redd) / E;
+  const double aux_all =
+      block_sum<double>(routed ? static_cast<double>(cnt) / (T * a.k) * Pe : 0.0, s_redd) * E;
   double zs = 0.0;
   for (int b = tid; b < nb; b += SCAN_T) zs += static_cast<double>(a.part_lse2[b]);
   zs = block_sum<double>(zs, s_redd);
   if (tid == 0) {
-    a.offsets[E] = total_kept;
-    a.mprefix[E] = total_tiles;
-    if (a.offsets_out != nullptr) a.offsets_out[E] = total_kept;
+    a.offsets[groups] = total_rows;
+    a.mprefix[groups] = total_tiles;
     *a.dropped = drop;
-    const double T = static_cast<double>(a.T);
     *a.aux = static_cast<float>(static_cast<double>(E) * auxp / (T * T));
     *a.z = static_cast<float>(zs / T);
+    a.balance_out[0] = static_cast<float>(aux_all);
+    a.balance_out[1] = static_cast<float>(mean_c > 0.0 ? sqrt(var_c) / mean_c : 0.0);
+    a.balance_out[2] = static_cast<float>(mean_p > 0.0 ? var_p / (mean_p * mean_p) : 0.0);
   }
 }
 
@@ -343,6 +374,7 @@ __global__ void __launch_bounds__(SCAN_T) scan_kernel(RoutingArgs a) {
   __shared__ float s_redf[SCAN_T / 32];
   __shared__ double s_redd[SCAN_T / 32];
   __shared__ int s_redi[SCAN_T / 32];
+  __shared__ double s_bcast;
   __shared__ int s_last;
   const int tid = threadIdx.x;
   const int E = a.E, nb = a.nblk;
@@ -361,7 +393,7 @@ __global__ void __launch_bounds__(SCAN_T) scan_kernel(RoutingArgs a) {
         ps += a.part_psum[row + b];
       }
     }
-    scan_finalize(a, cnt, c1, ps, s_warp, s_redi, s_redd);
+    scan_finalize(a, cnt, c1, ps, s_warp, s_redi, s_redd, &s_bcast);
     return;
   }
   const int e = blockIdx.x;
@@ -396,7 +428,7 @@ __global__ void __launch_bounds__(SCAN_T) scan_kernel(RoutingArgs a) {
   __threadfence();
   // the last block
   scan_finalize(a, tid < E ? __ldcg(a.counts + tid) : 0, tid < E ? __ldcg(a.tot_cnt1 + tid) : 0,
-                tid < E ? __ldcg(a.tot_psum + tid) : 0.f, s_warp, s_redi, s_redd);
+                tid < E ? __ldcg(a.tot_psum + tid) : 0.f, s_warp, s_redi, s_redd, &s_bcast);
   if (tid == 0) *a.scan_ticket = 0;  // ready for the next call
 }
 
@@ -453,30 +485,48 @@ __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
   XT* Xp = static_cast<XT*>(a.Xp);
   XT* yz = static_cast<XT*>(a.y_zero_dropped);
   const bool vec = (static_cast<size_t>(d) * sizeof(XT)) % 16 == 0;
+  // one warp copies one row of x (token tok) to row `dest` of the sorted buffer
+  auto copy_row = [&](int64_t tok, int64_t dest) {
+    if (vec) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + tok * d);
+      uint4* dst = reinterpret_cast<uint4*>(Xp + dest * d);
+      const int nv = static_cast<int>(static_cast<size_t>(d) * sizeof(XT) / 16);
+      for (int v0 = lane; v0 < nv; v0 += 128) {  // up to four 16-byte loads in flight per lane
+        uint4 c[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (v0 + 32 * q < nv) c[q] = src[v0 + 32 * q];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (v0 + 32 * q < nv) dst[v0 + 32 * q] = c[q];
+      }
+    } else {
+      for (int c = lane; c < d; c += 32) Xp[dest * d + c] = x[tok * d + c];
+    }
+  };
   for (int ai = warp; ai < nA; ai += 8) {
     const int dest = dest_s[ai];
     const int64_t tok = t0 + ai / k;
     if (dest >= 0) {
-      if (vec) {
-        const uint4* src = reinterpret_cast<const uint4*>(x + tok * d);
-        uint4* dst = reinterpret_cast<uint4*>(Xp + static_cast<int64_t>(dest) * d);
-        const int nv = static_cast<int>(static_cast<size_t>(d) * sizeof(XT) / 16);
-        for (int v0 = lane; v0 < nv; v0 += 128) {  // up to four 16-byte loads in flight per lane
-          uint4 c[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (v0 + 32 * q < nv) c[q] = src[v0 + 32 * q];
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (v0 + 32 * q < nv) dst[v0 + 32 * q] = c[q];
-        }
-      } else {
-        for (int c = lane; c < d; c += 32) Xp[static_cast<int64_t>(dest) * d + c] = x[tok * d + c];
-      }
+      copy_row(tok, dest);
     } else if (yz != nullptr) {  // k == 1: a dropped token's output row is zero
       for (int c = lane; c < d; c += 32) yz[tok * d + c] = XT(0.f);
       if (a.yf_zero_dropped != nullptr)
         for (int c = lane; c < d; c += 32) a.yf_zero_dropped[tok * d + c] = 0.f;
+    }
+  }
+  // shared experts: every token of the block, gate 1, rows offsets[E] + s * T + t
+  if (a.n_shared > 0) {
+    const int64_t base = a.offsets[E];
+    for (int q = warp; q < nt * a.n_shared; q += 8) {
+      const int si = q / nt;
+      const int64_t tok = t0 + (q - si * nt);
+      const int64_t row = base + si * a.T + tok;
+      if (lane == 0) {
+        a.row_token[row] = static_cast<int32_t>(tok);
+        a.row_gate[row] = 1.f;
+      }
+      copy_row(tok, row);
     }
   }
 }
@@ -490,6 +540,7 @@ __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
 // CU = 1 (WIDE false) to spread over more blocks.
 template <typename YT, int K, bool WIDE>
 __global__ void __launch_bounds__(256) combine_kernel(int64_t T, int d, const int32_t* __restrict__ dest_row,
+                                                      int n_shared, const int32_t* __restrict__ shared_base,
                                                       const float* __restrict__ Yp, int ksplit, int64_t split_stride,
                                                       YT* __restrict__ y, float* __restrict__ yf) {
   constexpr int CU = (!WIDE || K >= 8) ? 1 : 8 / K;
@@ -542,6 +593,22 @@ __global__ void __launch_bounds__(256) combine_kernel(int64_t T, int d, const in
       }
     }
   }
+  if (n_shared > 0) {  // the shared experts' rows, after the routed sum, in order s
+    const int64_t sb = *shared_base;
+    for (int si = 0; si < n_shared; ++si) {
+#pragma unroll
+      for (int u = 0; u < CU; ++u) {
+        if (tok[u] == 0xffffffffu) continue;
+        const int64_t row = sb + static_cast<int64_t>(si) * T + tok[u];
+        float4 sj = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int ks = 0; ks < ksplit; ++ks) {
+          const float4 q = reinterpret_cast<const float4*>(Yp + static_cast<int64_t>(ks) * split_stride + row * d)[v[u]];
+          sj.x += q.x; sj.y += q.y; sj.z += q.z; sj.w += q.w;
+        }
+        acc[u].x += sj.x; acc[u].y += sj.y; acc[u].z += sj.z; acc[u].w += sj.w;
+      }
+    }
+  }
 #pragma unroll
   for (int u = 0; u < CU; ++u) {
     if (tok[u] == 0xffffffffu) continue;
@@ -561,7 +628,8 @@ __global__ void __launch_bounds__(256) combine_kernel(int64_t T, int d, const in
 // Scalar combine for rows whose width is not a multiple of 4 (fp32 layers).
 template <typename YT>
 __global__ void __launch_bounds__(256) combine_scalar_kernel(int64_t T, int k, int d,
-                                                             const int32_t* __restrict__ dest_row,
+                                                             const int32_t* __restrict__ dest_row, int n_shared,
+                                                             const int32_t* __restrict__ shared_base,
                                                              const float* __restrict__ Yp, int ksplit,
                                                              int64_t split_stride, YT* __restrict__ y,
                                                              float* __restrict__ yf) {
@@ -578,6 +646,12 @@ __global__ void __launch_bounds__(256) combine_scalar_kernel(int64_t T, int k, i
     if (dst < 0) continue;
     float sj = 0.f;
     for (int ks = 0; ks < ksplit; ++ks) sj += Yp[static_cast<int64_t>(ks) * split_stride + static_cast<int64_t>(dst) * d + c];
+    acc += sj;
+  }
+  for (int si = 0; si < n_shared; ++si) {  // shared experts after the routed sum
+    const int64_t row = *shared_base + static_cast<int64_t>(si) * T + t;
+    float sj = 0.f;
+    for (int ks = 0; ks < ksplit; ++ks) sj += Yp[static_cast<int64_t>(ks) * split_stride + row * d + c];
     acc += sj;
   }
   y[t * d + c] = YT(acc);
@@ -613,8 +687,9 @@ cudaError_t launch_dispatch(const RoutingArgs& a, cudaStream_t s) {
 
 namespace {
 template <int K>
-cudaError_t launch_combine_k(int64_t T, int d, int y_is_bf16, const int32_t* dest_row, const float* Yp, int ksplit,
-                             int64_t split_stride, void* y, float* y_f32, cudaStream_t s) {
+cudaError_t launch_combine_k(int64_t T, int d, int y_is_bf16, const int32_t* dest_row, int n_shared,
+                             const int32_t* shared_base, const float* Yp, int ksplit, int64_t split_stride, void* y,
+                             float* y_f32, cudaStream_t s) {
   constexpr int CU = K >= 8 ? 1 : 8 / K;
   const int64_t groups = T * (d / 4);
   // wide threads only when the grid still covers every SM several times over
@@ -623,35 +698,52 @@ cudaError_t launch_combine_k(int64_t T, int d, int y_is_bf16, const int32_t* des
   const dim3 grid(static_cast<unsigned>((groups + 256 * cu - 1) / (256 * cu)));
   if (y_is_bf16) {
     auto kern = wide ? combine_kernel<__nv_bfloat16, K, true> : combine_kernel<__nv_bfloat16, K, false>;
-    return launch_pdl(kern, grid, dim3(256), 0, s, T, d, dest_row, Yp, ksplit, split_stride,
+    return launch_pdl(kern, grid, dim3(256), 0, s, T, d, dest_row, n_shared, shared_base, Yp, ksplit, split_stride,
                       static_cast<__nv_bfloat16*>(y), y_f32);
   }
   auto kern = wide ? combine_kernel<float, K, true> : combine_kernel<float, K, false>;
-  return launch_pdl(kern, grid, dim3(256), 0, s, T, d, dest_row, Yp, ksplit, split_stride, static_cast<float*>(y),
-                    y_f32);
+  return launch_pdl(kern, grid, dim3(256), 0, s, T, d, dest_row, n_shared, shared_base, Yp, ksplit, split_stride,
+                    static_cast<float*>(y), y_f32);
 }
 }  // namespace
 
-cudaError_t launch_combine(int64_t T, int k, int d, int y_is_bf16, const int32_t* dest_row, const float* Yp,
-                           int ksplit, int64_t split_stride, void* y, float* y_f32, cudaStream_t s) {
+cudaError_t launch_combine(int64_t T, int k, int d, int y_is_bf16, const int32_t* dest_row, int n_shared,
+                           const int32_t* shared_base, const float* Yp, int ksplit, int64_t split_stride, void* y,
+                           float* y_f32, cudaStream_t s) {
   if ((d & 3) == 0) {
     switch (k) {
-      case 1: return launch_combine_k<1>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
-      case 2: return launch_combine_k<2>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
-      case 3: return launch_combine_k<3>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
-      case 4: return launch_combine_k<4>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
-      case 5: return launch_combine_k<5>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
-      case 6: return launch_combine_k<6>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
-      case 7: return launch_combine_k<7>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
-      default: return launch_combine_k<8>(T, d, y_is_bf16, dest_row, Yp, ksplit, split_stride, y, y_f32, s);
+      case 1:
+        return launch_combine_k<1>(T, d, y_is_bf16, dest_row, n_shared, shared_base, Yp, ksplit, split_stride, y,
+                                     y_f32, s);
+      case 2:
+        return launch_combine_k<2>(T, d, y_is_bf16, dest_row, n_shared, shared_base, Yp, ksplit, split_stride, y,
+                                     y_f32, s);
+      case 3:
+        return launch_combine_k<3>(T, d, y_is_bf16, dest_row, n_shared, shared_base, Yp, ksplit, split_stride, y,
+                                     y_f32, s);
+      case 4:
+        return launch_combine_k<4>(T, d, y_is_bf16, dest_row, n_shared, shared_base, Yp, ksplit, split_stride, y,
+                                     y_f32, s);
+      case 5:
+        return launch_combine_k<5>(T, d, y_is_bf16, dest_row, n_shared, shared_base, Yp, ksplit, split_stride, y,
+                                     y_f32, s);
+      case 6:
+        return launch_combine_k<6>(T, d, y_is_bf16, dest_row, n_shared, shared_base, Yp, ksplit, split_stride, y,
+                                     y_f32, s);
+      case 7:
+        return launch_combine_k<7>(T, d, y_is_bf16, dest_row, n_shared, shared_base, Yp, ksplit, split_stride, y,
+                                     y_f32, s);
+      default:
+        return launch_combine_k<8>(T, d, y_is_bf16, dest_row, n_shared, shared_base, Yp, ksplit, split_stride, y,
+                                     y_f32, s);
     }
   }
   const dim3 grid(static_cast<unsigned>((T * d + 255) / 256));
   if (y_is_bf16)
-    return launch_pdl(combine_scalar_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, T, k, d, dest_row, Yp, ksplit,
-                      split_stride, static_cast<__nv_bfloat16*>(y), y_f32);
-  return launch_pdl(combine_scalar_kernel<float>, grid, dim3(256), 0, s, T, k, d, dest_row, Yp, ksplit,
-                    split_stride, static_cast<float*>(y), y_f32);
+    return launch_pdl(combine_scalar_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, T, k, d, dest_row, n_shared,
+                      shared_base, Yp, ksplit, split_stride, static_cast<__nv_bfloat16*>(y), y_f32);
+  return launch_pdl(combine_scalar_kernel<float>, grid, dim3(256), 0, s, T, k, d, dest_row, n_shared, shared_base,
+                    Yp, ksplit, split_stride, static_cast<float*>(y), y_f32);
 }
 
 cudaError_t launch_selftest_timeout(unsigned int* err, int64_t limit_ns, cudaStream_t s) {

@@ -35,10 +35,12 @@ class MoELayer:
     capacity_factor <= 0: dropless; dtype: torch.float32 or torch.bfloat16;
     hidden (bf16 layers): "bf16x2" keeps the hidden activation as a hi + lo
     pair of bf16 planes (default), "bf16" as one bf16 plane.
+    n_shared: shared experts every token visits; W1, W3, W2 then hold
+    num_experts + n_shared experts, the shared ones last.
     """
 
     def __init__(self, num_experts: int, k: int, d: int, d_ff: int, act="swiglu", gate_mode="renorm",
-                 capacity_factor: float = 0.0, dtype=torch.bfloat16, hidden="bf16x2"):
+                 capacity_factor: float = 0.0, dtype=torch.bfloat16, hidden="bf16x2", n_shared: int = 0):
         self.E, self.k, self.d, self.d_ff = num_experts, k, d, d_ff
         self.act = ACT[act] if isinstance(act, str) else int(act)
         self.gate_mode = GATE[gate_mode] if isinstance(gate_mode, str) else int(gate_mode)
@@ -51,6 +53,8 @@ class MoELayer:
         self._ws = None
         self.hidden = hidden
         check(lib().moe_set_hidden_precision(h, HIDDEN[hidden]))
+        self.n_shared = int(n_shared)
+        check(lib().moe_set_shared_experts(h, self.n_shared))
 
     def __del__(self):
         h = getattr(self, "_h", None)
@@ -108,6 +112,16 @@ class MoELayer:
         return y, counts, dropped, aux, z
 
     __call__ = forward
+
+    def balance_losses(self, T: int, workspace=None, out=None, stream=None) -> torch.Tensor:
+        """The alternative balance statistics of the last forward on ``workspace``
+        (default: this layer's own): a device tensor [aux over all k choices,
+        CV of the assignment counts, cv^2 of the mean router probabilities]."""
+        ws = workspace if workspace is not None else self._ws
+        dev = ws.device if ws is not None else torch.device("cuda")
+        out = out if out is not None else torch.empty(3, dtype=torch.float32, device=dev)
+        check(lib().moe_balance_losses(self._h, T, _ptr(ws), _ptr(out), _stream_handle(stream)))
+        return out
 
     def debug_buffers(self, T: int, device) -> dict:
         """Device tensors for every output field of moe_debug."""

@@ -9,7 +9,9 @@ Shapes follow the workloads the pages describe: a Switch-style k=1 layer
 Mixtral-shaped 8-expert top-2 SwiGLU layer (same page, "Total versus active
 parameters" and "Implementation"), and a fine-grained many-expert layer
 ("2 out of 8 or 128", Mixture of Experts (MoE), inferensys.com
-inference-optimization glossary, first paragraph).
+inference-optimization glossary, first paragraph), also with a shared expert
+("Mixture of experts", rayaq.ca, "Total versus active parameters": shared
+experts every token visits).
 
 Distributions (no dataset exists for any of them):
   x ~ N(0, 1); router rows W_r ~ N(0, 1/d); expert weights ~ N(0, 1/fan_in)
@@ -58,6 +60,7 @@ class Workload:
     dyadic: bool = False
     x_rows_of: Optional[str] = None  # take x as the first T rows of this workload's x
     seed: int = 1234
+    n_shared: int = 0  # shared experts every token visits (weights follow the routed experts')
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -87,6 +90,11 @@ WORKLOADS = {
         Workload("fine_grained", T=16384, d=2048, E=128, k=4, d_ff=768,
                  act=ACT_SWIGLU, gate=GATE_RENORM, capacity_factor=2.0,
                  dtype=DTYPE_BF16, bias="zipf", seed=1238),
+        # the fine-grained layer plus one shared expert of the same shape
+        # ("many small experts plus shared experts every token visits")
+        Workload("fine_grained_shared", T=16384, d=2048, E=128, k=4, d_ff=768,
+                 act=ACT_SWIGLU, gate=GATE_RENORM, capacity_factor=2.0,
+                 dtype=DTYPE_BF16, bias="zipf", seed=1238, n_shared=1),
     ]
 }
 
@@ -119,8 +127,9 @@ def make_inputs(w: Workload, device="cpu", weights=True, x_rows: Optional[int] =
     """Draw the layer inputs of workload ``w`` on ``device``.
 
     Returns a dict with x [T][d], W_r [E][d] (fp32), b_r [E] (fp32) or None,
-    W1 [E][d_ff][d], W3 [E][d_ff][d] (SwiGLU only, else None),
-    W2 [E][d][d_ff].  x and the expert weights have the workload's dtype.
+    W1 [E + n_shared][d_ff][d], W3 [E + n_shared][d_ff][d] (SwiGLU only, else
+    None), W2 [E + n_shared][d][d_ff] (the shared experts last).  x and the
+    expert weights have the workload's dtype.
     """
     dev = torch.device(device)
     dt = torch_dtype(w.dtype)
@@ -145,11 +154,12 @@ def make_inputs(w: Workload, device="cpu", weights=True, x_rows: Optional[int] =
     out = {"x": x.to(dt).contiguous(), "W_r": W_r.contiguous(), "b_r": b_r,
            "W1": None, "W3": None, "W2": None}
     if weights:
-        W1 = _normal((w.E, w.d_ff, w.d), 1.0 / math.sqrt(w.d), dev, w.seed, "W1")
-        W2 = _normal((w.E, w.d, w.d_ff), 1.0 / math.sqrt(w.d_ff), dev, w.seed, "W2")
+        ne = w.E + w.n_shared
+        W1 = _normal((ne, w.d_ff, w.d), 1.0 / math.sqrt(w.d), dev, w.seed, "W1")
+        W2 = _normal((ne, w.d, w.d_ff), 1.0 / math.sqrt(w.d_ff), dev, w.seed, "W2")
         W3 = None
         if w.act == ACT_SWIGLU:
-            W3 = _normal((w.E, w.d_ff, w.d), 1.0 / math.sqrt(w.d), dev, w.seed, "W3")
+            W3 = _normal((ne, w.d_ff, w.d), 1.0 / math.sqrt(w.d), dev, w.seed, "W3")
         if w.dyadic and w.dtype == DTYPE_F32:
             W1 = _round_to_grid(W1, -10, 1.0 - 2.0 ** -10)
             W2 = _round_to_grid(W2, -10, 1.0 - 2.0 ** -10)

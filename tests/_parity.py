@@ -47,7 +47,8 @@ class HostExperts:
 
 def layer_for(w: Workload, hidden: str = "bf16x2") -> MoELayer:
     return MoELayer(w.E, w.k, w.d, w.d_ff, act=w.act, gate_mode=w.gate,
-                    capacity_factor=w.capacity_factor, dtype=torch_dtype(w.dtype), hidden=hidden)
+                    capacity_factor=w.capacity_factor, dtype=torch_dtype(w.dtype), hidden=hidden,
+                    n_shared=w.n_shared)
 
 
 def run_gpu(w: Workload, inp: dict, *, logits_in=None, debug=True, layer=None):
@@ -62,6 +63,8 @@ def run_gpu(w: Workload, inp: dict, *, logits_in=None, debug=True, layer=None):
     status()
     out = {"y_dev": y, "y": np32(y), "counts": counts.cpu().numpy(), "dropped": int(dropped.item()),
            "aux": float(aux.item()), "z": float(z.item())}
+    bl = layer.balance_losses(w.T).cpu().numpy()
+    out.update(aux_all_choices=float(bl[0]), cv_counts=float(bl[1]), cv2_probs=float(bl[2]))
     if dbg:
         for key, t in dbg.items():
             if key != "logits_in":
@@ -76,10 +79,28 @@ def host_inputs(inp: dict):
             "W2": HostExperts(inp["W2"])}
 
 
+class _Shift:
+    """Experts E + s of a HostExperts as a sequence of n shared experts."""
+
+    def __init__(self, he, E, n):
+        self.he, self.E, self.n = he, E, n
+
+    def __len__(self):
+        return self.n
+
+    def __getitem__(self, s):
+        return self.he[self.E + s]
+
+
 def run_oracle(w: Workload, host: dict, rows=None, logits=None, hidden_bf16=False):
+    shared = None
+    if w.n_shared:
+        shared = (_Shift(host["W1"], w.E, w.n_shared),
+                  None if host["W3"] is None else _Shift(host["W3"], w.E, w.n_shared),
+                  _Shift(host["W2"], w.E, w.n_shared))
     return O.moe_forward(host["x"], host["W_r"], host["b_r"], host["W1"], host["W3"], host["W2"],
                          k=w.k, gate_mode=w.gate, act=w.act, capacity_factor=w.capacity_factor,
-                         rows=rows, logits=logits, hidden_bf16=hidden_bf16)
+                         rows=rows, logits=logits, hidden_bf16=hidden_bf16, shared=shared)
 
 
 def assert_routing_equal(g: dict, o: dict):
@@ -95,6 +116,10 @@ def assert_gates_and_losses(g: dict, o: dict):
     np.testing.assert_allclose(g["topk_gate"], o["gate"], rtol=0, atol=2e-6)
     assert abs(g["aux"] - o["aux"]) <= 1e-5 * max(1.0, abs(o["aux"]))
     assert abs(g["z"] - o["z"]) <= 1e-5 * max(1.0, abs(o["z"]))
+    # the alternative balance statistics (fp32 results of fp64 sums of fp32 partials)
+    for key in ("aux_all_choices", "cv_counts", "cv2_probs"):
+        if key in g:
+            assert abs(g[key] - o[key]) <= 1e-5 * max(1.0, abs(o[key])), (key, g[key], o[key])
     if "lse_out" in g:
         np.testing.assert_allclose(g["lse_out"], o["lse"], rtol=2e-6, atol=2e-6)
 

@@ -108,15 +108,38 @@ def test_workspace_and_forward_validation_without_gpu(L):
     assert L.moe_destroy(None) == 0
 
 
+def test_shared_experts_and_balance_losses_validate_arguments(L):
+    rc, h = _create(L, 8, 2, 64, 64, 1, 1, 0.0, 1)
+    assert rc == 0
+    ws0 = L.moe_workspace_bytes(h, 100)
+    for bad in (-1, 9):
+        assert L.moe_set_shared_experts(h, bad) == _lib.MOE_ERR_INVALID_ARG
+    assert L.moe_set_shared_experts(None, 1) == _lib.MOE_ERR_INVALID_ARG
+    assert L.moe_set_shared_experts(h, 2) == 0
+    # two shared experts add 2 * T rows to every expert-sorted buffer
+    assert L.moe_workspace_bytes(h, 100) >= ws0 + 2 * 100 * (64 + 64) * 2
+    rc2, h2 = _create(L, 255, 2, 64, 64, 1, 1, 0.0, 1)
+    assert L.moe_set_shared_experts(h2, 2) == _lib.MOE_ERR_INVALID_ARG  # E + n_shared > 256
+    assert L.moe_set_shared_experts(h2, 1) == 0
+    p = ctypes.c_void_p(256)
+    assert L.moe_balance_losses(None, 4, p, p, None) == _lib.MOE_ERR_INVALID_ARG
+    assert L.moe_balance_losses(h, -1, p, p, None) == _lib.MOE_ERR_INVALID_ARG
+    assert L.moe_balance_losses(h, 4, p, None, None) == _lib.MOE_ERR_INVALID_ARG
+    assert L.moe_balance_losses(h, 4, None, p, None) == _lib.MOE_ERR_INVALID_ARG
+    L.moe_destroy(h)
+    L.moe_destroy(h2)
+
+
 def test_workspace_sizing_is_defined_for_every_batch_size(L):
     """Host-only sizing (no GPU): every T from 0 up, several layer shapes, both
     hidden precisions; sizes never shrink as T grows."""
     shapes = [(8, 2, 4096, 14336, 1, 1, 0.0, 1), (64, 1, 768, 3072, 0, 0, 1.25, 1),
               (128, 4, 2048, 768, 1, 1, 2.0, 1), (4, 2, 32, 64, 0, 1, 0.0, 0), (256, 8, 64, 64, 0, 0, 0.5, 1),
               (3, 2, 1032, 1160, 1, 1, 0.0, 1)]
-    for args in shapes:
+    for i, args in enumerate(shapes):
         rc, h = _create(L, *args)
         assert rc == 0
+        assert L.moe_set_shared_experts(h, min(i % 3, 256 - args[0])) == 0
         for mode in (0, 1):
             assert L.moe_set_hidden_precision(h, mode) == 0
             prev = 0

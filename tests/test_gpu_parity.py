@@ -48,13 +48,21 @@ SMALL = [
     ("stream_k_switch_pieces", 700, 512, 16, 1, 1024, R, SW, 1.25, BF, "normal"),
     ("stream_k_long_k", 2, 2048, 4, 1, 256, R, RN, 0.0, BF, None),
     ("stream_k_swiglu_pieces", 4, 1536, 8, 2, 384, S, RN, 0.0, BF, None),
+    # shared experts (last field: n_shared): k = 2; k = 1 Switch with drops (the
+    # combine path, dropped tokens keep the shared output); fp32; a small batch
+    # whose second projection is split into K-range partials
+    ("shared_k2_swiglu", 500, 128, 8, 2, 256, S, RN, 0.0, BF, None, 1),
+    ("shared_switch_k1_drops", 400, 64, 16, 1, 128, R, SW, 0.5, BF, "normal", 2),
+    ("shared_fp32", 120, 24, 4, 2, 40, S, RN, 1.0, F32, None, 1),
+    ("shared_decode_splitk", 2, 256, 8, 2, 1024, S, RN, 0.0, BF, None, 1),
 ]
 
 
 def _small(case) -> Workload:
-    name, T, d, E, k, d_ff, act, gate, cf, dt, bias = case
+    name, T, d, E, k, d_ff, act, gate, cf, dt, bias = case[:11]
+    n_shared = case[11] if len(case) > 11 else 0
     return Workload(name, T=T, d=d, E=E, k=k, d_ff=d_ff, act=act, gate=gate, capacity_factor=cf, dtype=dt,
-                    bias=bias, dyadic=True, seed=4000 + zlib.crc32(name.encode()) % 1000)
+                    bias=bias, dyadic=True, seed=4000 + zlib.crc32(name.encode()) % 1000, n_shared=n_shared)
 
 
 @pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
@@ -73,7 +81,7 @@ def test_small_layers_match_oracle(case):
 
 SINGLE = [c for c in SMALL if c[9] == BF and c[0] in ("swiglu_e8_k2", "switch_relu_drops", "k4_zipf_tails",
                                                        "e128_k8_cap", "long_k_ragged", "stream_k_tail_relu",
-                                                       "stream_k_switch_pieces")]
+                                                       "stream_k_switch_pieces", "shared_switch_k1_drops")]
 
 
 @pytest.mark.parametrize("case", SINGLE, ids=[c[0] for c in SINGLE])
@@ -194,7 +202,7 @@ def test_device_wait_timeout_is_reported_and_context_survives():
 
 # ---------------------------------------------------------------- full-size workloads
 FULL = ["switch_k1", "mixtral_prefill", "mixtral_decode_t1", "mixtral_decode_t16", "mixtral_decode_t64",
-        "fine_grained"]
+        "fine_grained", "fine_grained_shared"]
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -229,7 +237,7 @@ def test_full_size_identical_logits(name):
     assert_y_close(w, g, o["y"], rows=rows)
 
 
-@pytest.mark.parametrize("name", ["switch_k1", "mixtral_prefill", "fine_grained"])
+@pytest.mark.parametrize("name", ["switch_k1", "mixtral_prefill", "fine_grained", "fine_grained_shared"])
 def test_full_size_bench_configuration(name):
     """The launch the benchmark times (no debug hooks), on the workloads' own inputs.
 
