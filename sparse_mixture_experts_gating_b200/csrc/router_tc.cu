@@ -30,7 +30,7 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;  // producer, MMA, 8 epilogue warps
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int MAX_STAGES = 8;  // small router tiles: a deep ring hides the TMA round trip
 
@@ -64,7 +64,11 @@ struct RtCtl {
   int last;  // this CTA finished the last K range of the tile
   int hist[4][kRouterTcMaxE];
   int cnt1[4][kRouterTcMaxE];
-  float pstage[4][32][33];  // per epilogue warp: 32 tokens x 32 experts of probabilities
+  float pstage[8][32][17];  // per epilogue warp: 32 tokens x 16 experts of probabilities
+  float xm[4][2][32];       // per lane quarter and half: partial max of each token
+  float xs[4][2][32];       // partial exp sums
+  float xtv[4][8][32];      // half 1's top-k list (values, indices)
+  int xte[4][8][32];
   float bias[kRouterTcMaxE];
 };
 
@@ -72,7 +76,7 @@ template <int EP>
 struct RtGeo {
   static constexpr int B_PLANE = EP * BK * 2;  // one plane box: EP rows x 128 B
   static constexpr int STAGE_BYTES = A_BYTES + 3 * B_PLANE;
-  static constexpr int STAGES = (200 * 1024 / STAGE_BYTES) < MAX_STAGES ? (200 * 1024 / STAGE_BYTES) : MAX_STAGES;
+  static constexpr int STAGES = (190 * 1024 / STAGE_BYTES) < MAX_STAGES ? (190 * 1024 / STAGE_BYTES) : MAX_STAGES;
   static constexpr uint32_t TMEM_COLS = (2 * EP) <= 32 ? 32 : (2 * EP) <= 64 ? 64 : (2 * EP) <= 128 ? 128
                                         : (2 * EP) <= 256 ? 256 : 512;
   static constexpr size_t SMEM = STAGES * STAGE_BYTES + sizeof(RtCtl) + 1024;
@@ -122,7 +126,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&ctl->tfull[a], 1); mbar_init(&ctl->tempty[a], 128); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&ctl->tfull[a], 1); mbar_init(&ctl->tempty[a], 256); }
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     fence_mbarrier_init();
@@ -212,7 +216,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait(&ctl->drain, 0, p.limit_ns);
     }
   } else {  // ---------------------------------------------------------- epilogue
-    const int q = warp & 3;  // TMEM lane quarter = 32-token router block within the tile
+    // Eight warps, two per TMEM lane quarter q (= 32-token router block of the
+    // tile).  Warp half hf takes expert columns [c_lo, c_hi): the pair splits
+    // the experts and exchanges, per token, the partial max, the partial top-k
+    // list (half 1 -> half 0) and the partial exp sums through shared memory;
+    // the lower-expert half goes first in every merge and sum, so ties and
+    // summation order are fixed.
+    const int wi = warp - 2;       // 0..7
+    const int q = warp & 3;        // TMEM lane quarter
+    const int hf = wi >> 2;        // 0: lower experts, 1: upper experts
+    constexpr int H = EP / 2 < 16 ? 16 : EP / 2;  // columns per half (EP = 16: half 1 has none)
+    const int c_lo = hf * H;
+    const bool has_cols = c_lo < EP;
+    const int pair_bar = 2 + q;    // named barrier of the warp pair (64 threads)
     int acc = 0;
     uint32_t acc_phase = 0;
     const int E = p.E;
@@ -222,31 +238,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                  mbar_wait_or_abort(&ctl->tfull[acc], acc_phase, &ctl->abort, p.err, p.limit_ns));
       if (!ok) break;
       tc_fence_after();
+      const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * EP);
       if (p.ksplit > 1) {
-        // Publish this K range's partial logits (row = TMEM lane); the CTA that
-        // finishes a tile's last range sums all ranges in order back into its
-        // accumulator and runs the epilogue; the others release theirs.
+        // Publish this K range's partial logits of this half's columns (row =
+        // TMEM lane); the CTA that finishes a tile's last range sums all
+        // ranges in order back into its accumulator; the others release it.
         // Rows past T carry no token: they neither publish nor read partials.
-        const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * EP);
         const bool row_live = static_cast<int64_t>(tile) * BM + q * 32 + lane < p.T;
         float* prow = p.partials + ((static_cast<int64_t>(tile) * p.ksplit + ks) * BM + q * 32 + lane) * EP;
+        if (has_cols) {
 #pragma unroll 1
-        for (int c0 = 0; c0 < EP; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(tq + c0, r);
-          tmem_ld_wait();
-          if (row_live) {
+          for (int c0 = c_lo; c0 < c_lo + H; c0 += 16) {
+            uint32_t r[16];
+            tmem_ld16(tq + c0, r);
+            tmem_ld_wait();
+            if (row_live) {
 #pragma unroll
-            for (int i = 0; i < 16; i += 4)
-              *reinterpret_cast<float4*>(prow + c0 + i) =
-                  make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
-                              __uint_as_float(r[i + 3]));
+              for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<float4*>(prow + c0 + i) =
+                    make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
+                                __uint_as_float(r[i + 3]));
+            }
           }
         }
         __threadfence();
-        named_barrier(1, 128);  // all 128 rows of this range are written
+        named_barrier(1, 256);  // all 128 rows of this range are written
         if (threadIdx.x == 64) ctl->last = (atomicAdd(p.tickets + tile, 1) == p.ksplit - 1) ? 1 : 0;
-        named_barrier(1, 128);
+        named_barrier(1, 256);
         if (!ctl->last) {
           tc_fence_before();
           mbar_arrive(&ctl->tempty[acc]);
@@ -255,226 +273,231 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         __threadfence();
         const float* prow0 = p.partials + (static_cast<int64_t>(tile) * p.ksplit * BM + q * 32 + lane) * EP;
+        if (has_cols) {
 #pragma unroll 1
-        for (int c0 = 0; c0 < EP; c0 += 16) {
-          uint32_t r[16];
-          float sum[16];
+          for (int c0 = c_lo; c0 < c_lo + H; c0 += 16) {
+            uint32_t r[16];
+            float sum[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) sum[i] = 0.f;
-          // ranges in ascending order (deterministic), four loads in flight per batch
+            for (int i = 0; i < 16; ++i) sum[i] = 0.f;
+            // ranges in ascending order (deterministic), four loads in flight per batch
 #pragma unroll 1
-          for (int s0 = 0; row_live && s0 < p.ksplit; s0 += 4) {
-            float4 v[4][4];
+            for (int s0 = 0; row_live && s0 < p.ksplit; s0 += 4) {
+              float4 v[4][4];
 #pragma unroll
-            for (int u2 = 0; u2 < 4; ++u2) {
-              const float* src = prow0 + static_cast<int64_t>(s0 + u2) * BM * EP + c0;
+              for (int u2 = 0; u2 < 4; ++u2) {
+                const float* src = prow0 + static_cast<int64_t>(s0 + u2) * BM * EP + c0;
 #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                v[u2][i] = s0 + u2 < p.ksplit ? __ldcg(reinterpret_cast<const float4*>(src + 4 * i))
-                                              : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+                for (int i = 0; i < 4; ++i)
+                  v[u2][i] = s0 + u2 < p.ksplit ? __ldcg(reinterpret_cast<const float4*>(src + 4 * i))
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+              }
 #pragma unroll
-            for (int u2 = 0; u2 < 4; ++u2) {
-              if (s0 + u2 < p.ksplit) {
+              for (int u2 = 0; u2 < 4; ++u2) {
+                if (s0 + u2 < p.ksplit) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  sum[4 * i] += v[u2][i].x;
-                  sum[4 * i + 1] += v[u2][i].y;
-                  sum[4 * i + 2] += v[u2][i].z;
-                  sum[4 * i + 3] += v[u2][i].w;
+                  for (int i = 0; i < 4; ++i) {
+                    sum[4 * i] += v[u2][i].x;
+                    sum[4 * i + 1] += v[u2][i].y;
+                    sum[4 * i + 2] += v[u2][i].z;
+                    sum[4 * i + 3] += v[u2][i].w;
+                  }
                 }
               }
             }
-          }
 #pragma unroll
-          for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(sum[i]);
-          tmem_st16(tq + c0, r);
+            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(sum[i]);
+            tmem_st16(tq + c0, r);
+          }
+          tmem_st_wait();
         }
-        tmem_st_wait();
       }
       const int64_t tok = static_cast<int64_t>(tile) * BM + q * 32 + lane;
       const bool valid = tok < p.T;
       const int blk = tile * 4 + q;
       const bool blk_valid = blk < p.nblk;
-      const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * EP);
 
-      float m = -INFINITY, inv_s, lse;
-      float tv[K];
-      int te[K];
+      // 1. this half's logits: for up to 32 columns (E_pad <= 64) one batch of
+      // TMEM loads into registers, after which the accumulator is released;
+      // for 64 columns (E_pad = 128) passes over 16-column chunks re-read TMEM
+      // (the register budget of ten warps does not hold 64 logits per thread)
+      constexpr bool REG = H <= 32;
+      float h[REG ? H : 1];
+      if constexpr (REG) {
+        if (has_cols) {
+          uint32_t hr[H / 16][16];
 #pragma unroll
-      for (int j = 0; j < K; ++j) { tv[j] = -INFINITY; te[j] = 0x7fffffff; }
-      if constexpr (EP <= 64) {
-        // The token's EP logits come out of TMEM in one batch of loads and stay in
-        // registers: h = acc + bias, then the max and the top-k (value desc,
-        // index asc) in one scan over e.  The k best are kept sorted; a candidate
-        // enters by compare-and-swap down the list (strict >, so an equal logit
-        // never displaces the lower expert index seen first; once an entry moves,
-        // the rest of the list shifts down behind it).
-        float h[EP];
-        {
-          uint32_t hr[EP / 16][16];
-#pragma unroll
-          for (int c = 0; c < EP / 16; ++c) tmem_ld16(ta + c * 16, hr[c]);
+          for (int c = 0; c < H / 16; ++c) tmem_ld16(tq + c_lo + c * 16, hr[c]);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < EP; ++e) h[e] = __uint_as_float(hr[e / 16][e % 16]);
+          for (int i = 0; i < H; ++i) h[i] = __uint_as_float(hr[i / 16][i % 16]);
         }
         tc_fence_before();
         mbar_arrive(&ctl->tempty[acc]);  // accumulator consumed: the next tile's MMAs may start
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      // logit of column i of this half (from registers or a chunk just loaded)
+      auto logit = [&](float raw, int e) {
+        float v = raw + ctl->bias[e];
+        return v != v ? -INFINITY : v;  // NaN logits (out of contract) rank last
+      };
+
+      // 2. bias, partial max and partial top-k (value desc, index asc): the k
+      // best are kept sorted; a candidate enters by compare-and-swap down the
+      // list (strict >, so an equal logit never displaces the lower index seen
+      // first; once an entry moves, the rest of the list shifts down behind it)
+      float m = -INFINITY;
+      float tv[K];
+      int te[K];
 #pragma unroll
-        for (int e = 0; e < EP; ++e) {
-          if (e < E) {
-            float v = h[e] + ctl->bias[e];
-            if (v != v) v = -INFINITY;  // NaN logits (out of contract) rank last
-            h[e] = v;
-            if (valid && p.logits_out != nullptr) p.logits_out[tok * E + e] = v;
-            m = fmaxf(m, v);
-            if (v > tv[K - 1] || te[K - 1] == 0x7fffffff) {
-              float cv = v;
-              int ce = e;
-              bool shifting = false;
+      for (int j = 0; j < K; ++j) { tv[j] = -INFINITY; te[j] = 0x7fffffff; }
+      auto consider = [&](float v, int e) {
+        if (valid && p.logits_out != nullptr) p.logits_out[tok * E + e] = v;
+        m = fmaxf(m, v);
+        if (v > tv[K - 1] || te[K - 1] == 0x7fffffff) {
+          float cv = v;
+          int ce = e;
+          bool shifting = false;
 #pragma unroll
-              for (int j = 0; j < K; ++j) {
-                if (shifting || cv > tv[j] || te[j] == 0x7fffffff) {
-                  shifting = true;
-                  const float tvj = tv[j];
-                  const int tej = te[j];
-                  tv[j] = cv;
-                  te[j] = ce;
-                  cv = tvj;
-                  ce = tej;
-                }
-              }
+          for (int j = 0; j < K; ++j) {
+            if (shifting || cv > tv[j] || te[j] == 0x7fffffff) {
+              shifting = true;
+              const float tvj = tv[j];
+              const int tej = te[j];
+              tv[j] = cv;
+              te[j] = ce;
+              cv = tvj;
+              ce = tej;
             }
           }
         }
-        // s = sum_e exp(h - m): each exponential once (kept in h), four partial
-        // sums in a fixed order
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      };
+      if constexpr (REG) {
 #pragma unroll
-        for (int e = 0; e < EP; ++e) {
-          const float x = e < E ? expf(h[e] - m) : 0.f;
-          h[e] = x;
-          s4[e & 3] += x;
+        for (int i = 0; i < H; ++i) {
+          const int e = c_lo + i;
+          if (has_cols && e < E) {
+            h[i] = logit(h[i], e);
+            consider(h[i], e);
+          }
         }
-        const float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-        inv_s = 1.f / s;
-        lse = m + logf(s);
-        // per-expert probability sums of this 32-token block: the warp writes
-        // 32 tokens x 32 experts row-major into shared memory and lane j sums
-        // column j over the tokens in order (fixed order: deterministic)
-        float* stg = &ctl->pstage[q][0][0];
+      } else {
+#pragma unroll 1
+        for (int c0 = 0; c0 < H; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(tq + c_lo + c0, r);
+          tmem_ld_wait();
 #pragma unroll
-        for (int c0 = 0; c0 < EP; c0 += 32) {
+          for (int i = 0; i < 16; ++i) {
+            const int e = c_lo + c0 + i;
+            if (e < E) consider(logit(__uint_as_float(r[i]), e), e);
+          }
+        }
+      }
+      // 3. exchange: both halves' max; half 1's list to half 0, which merges
+      // (half 0's experts have the lower indices, so it wins equal values)
+      ctl->xm[q][hf][lane] = m;
+      if (hf == 1) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            stg[lane * 33 + i] = (c0 + i < EP && valid && c0 + i < E) ? h[(c0 + i) & (EP - 1)] * inv_s : 0.f;
-          __syncwarp();
+        for (int j = 0; j < K; ++j) { ctl->xtv[q][j][lane] = tv[j]; ctl->xte[q][j][lane] = te[j]; }
+      }
+      named_barrier(pair_bar, 64);
+      m = fmaxf(ctl->xm[q][0][lane], ctl->xm[q][1][lane]);
+      if (hf == 0) {
+        float bv[K];
+        int be[K];
+#pragma unroll
+        for (int j = 0; j < K; ++j) { bv[j] = ctl->xtv[q][j][lane]; be[j] = ctl->xte[q][j][lane]; }
+        float mv[K];
+        int me[K];
+        int ia = 0, ib = 0;
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+          // take from A unless B's head is strictly larger (or A is exhausted/empty)
+          float av = -INFINITY, bvh = -INFINITY;
+          int ae = 0x7fffffff, beh = 0x7fffffff;
+#pragma unroll
+          for (int t = 0; t < K; ++t) {
+            if (t == ia) { av = tv[t]; ae = te[t]; }
+            if (t == ib) { bvh = bv[t]; beh = be[t]; }
+          }
+          const bool take_b = ia >= K || (ib < K && beh != 0x7fffffff &&
+                                          (ae == 0x7fffffff || bvh > av));
+          mv[j] = take_b ? bvh : av;
+          me[j] = take_b ? beh : ae;
+          if (take_b) ++ib; else ++ia;
+        }
+#pragma unroll
+        for (int j = 0; j < K; ++j) { tv[j] = mv[j]; te[j] = me[j]; }
+      }
+      // 4. s = sum_e exp(h - m): four partial sums per half in a fixed order,
+      // then half 0 + half 1 (registers: each exponential once, kept in h)
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (REG) {
+#pragma unroll
+        for (int i = 0; i < H; ++i) {
+          const float x = (has_cols && c_lo + i < E) ? expf(h[i] - m) : 0.f;
+          h[i] = x;
+          s4[i & 3] += x;
+        }
+      } else {
+#pragma unroll 1
+        for (int c0 = 0; c0 < H; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(tq + c_lo + c0, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = c_lo + c0 + i;
+            s4[i & 3] += e < E ? expf(logit(__uint_as_float(r[i]), e) - m) : 0.f;
+          }
+        }
+      }
+      ctl->xs[q][hf][lane] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      named_barrier(pair_bar, 64);
+      const float s = ctl->xs[q][0][lane] + ctl->xs[q][1][lane];
+      const float inv_s = 1.f / s;
+      const float lse = m + logf(s);
+      // 5. per-expert probability sums of this 32-token block for this half's
+      // experts: 32 tokens x 16 experts through shared memory, lane j < 16
+      // sums column j over the tokens in order (fixed order: deterministic)
+      float* stg = &ctl->pstage[wi][0][0];
+#pragma unroll
+      for (int c0 = 0; c0 < H; c0 += 16) {
+        if constexpr (REG) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            stg[lane * 17 + i] = (valid && has_cols && c_lo + c0 + i < E) ? h[(c0 + i) & (H - 1)] * inv_s : 0.f;
+        } else {
+          uint32_t r[16];
+          tmem_ld16(tq + c_lo + c0, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = c_lo + c0 + i;
+            stg[lane * 17 + i] = (valid && e < E) ? expf(logit(__uint_as_float(r[i]), e) - m) * inv_s : 0.f;
+          }
+        }
+        __syncwarp();
+        if (lane < 16 && has_cols && c_lo + c0 + lane < E && blk_valid) {
           float a0 = 0.f, a1 = 0.f;
 #pragma unroll
           for (int t = 0; t < 32; t += 2) {
-            a0 += stg[t * 33 + lane];
-            a1 += stg[(t + 1) * 33 + lane];
+            a0 += stg[t * 17 + lane];
+            a1 += stg[(t + 1) * 17 + lane];
           }
-          if (c0 + lane < E && blk_valid) p.part_psum[(c0 + lane) * p.nblk + blk] = a0 + a1;
-          __syncwarp();
+          p.part_psum[(c_lo + c0 + lane) * p.nblk + blk] = a0 + a1;
         }
-      } else {
-        // E_pad = 128: the same steps over 16-column chunks (re-read from TMEM in
-        // each pass), which keeps the code small enough for the instruction cache
-        // pass 1: logits, max, top-k (value desc, index asc) in one scan over e.
-        // The k best are kept sorted in registers; a candidate enters by
-        // compare-and-swap down the list (strict >, so an equal logit never
-        // displaces the lower expert index seen first; once an entry moves, the
-        // rest of the list shifts down behind it).
-#pragma unroll 1
-        for (int c0 = 0; c0 < EP; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(ta + c0, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e = c0 + i;
-            if (e < E) {
-              float h = __uint_as_float(r[i]) + ctl->bias[e];
-              if (h != h) h = -INFINITY;  // NaN logits (out of contract) rank last
-              if (valid && p.logits_out != nullptr) p.logits_out[tok * E + e] = h;
-              m = fmaxf(m, h);
-              if (h > tv[K - 1] || te[K - 1] == 0x7fffffff) {
-                float cv = h;
-                int ce = e;
-                bool shifting = false;
-#pragma unroll
-                for (int j = 0; j < K; ++j) {
-                  if (shifting || cv > tv[j] || te[j] == 0x7fffffff) {
-                    shifting = true;
-                    const float tvj = tv[j];
-                    const int tej = te[j];
-                    tv[j] = cv;
-                    te[j] = ce;
-                    cv = tvj;
-                    ce = tej;
-                  }
-                }
-              }
-            }
-          }
-        }
-        // pass 2: s = sum_e exp(h - m)
-        float s = 0.f;
-#pragma unroll 1
-        for (int c0 = 0; c0 < EP; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(ta + c0, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e = c0 + i;
-            if (e < E) {
-              float h = __uint_as_float(r[i]) + ctl->bias[e];
-              if (h != h) h = -INFINITY;
-              s += expf(h - m);
-            }
-          }
-        }
-        inv_s = 1.f / s;
-        lse = m + logf(s);
-        // pass 3: per-expert probability sums of this 32-token block: the warp
-        // stages 32 tokens x 16 experts in shared memory and lane i sums column i
-        // over the tokens in order (fixed order: deterministic).
-        float* stg = &ctl->pstage[q][0][0];
-#pragma unroll 1
-        for (int c0 = 0; c0 < EP; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(ta + c0, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e = c0 + i;
-            float pe = 0.f;
-            if (valid && e < E) {
-              float h = __uint_as_float(r[i]) + ctl->bias[e];
-              if (h != h) h = -INFINITY;
-              pe = expf(h - m) * inv_s;
-            }
-            stg[lane * 17 + i] = pe;
-          }
-          __syncwarp();
-          if (lane < 16 && c0 + lane < E && blk_valid) {
-            float acc_p = 0.f;
-#pragma unroll 8
-            for (int t = 0; t < 32; ++t) acc_p += stg[t * 17 + lane];
-            p.part_psum[(c0 + lane) * p.nblk + blk] = acc_p;
-          }
-          __syncwarp();
-        }
+        __syncwarp();
+      }
+      if constexpr (!REG) {
         tc_fence_before();
         mbar_arrive(&ctl->tempty[acc]);  // accumulator consumed
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
+      if (hf == 1) continue;
 
-      // gates, outputs and block counts
+      // 6. (half 0) gates, outputs and block counts
       if (valid) {
         float den = 0.f;
         if (p.gate_mode != 0) {

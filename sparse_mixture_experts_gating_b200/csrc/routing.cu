@@ -299,24 +299,64 @@ __device__ __forceinline__ F block_sum(F v, F* s_red) {
   return t;  // valid in thread 0
 }
 
-// Sum over the block in a fixed tree order, returned to every thread.
-template <typename F>
-__device__ __forceinline__ F block_sum_all(F v, F* s_red, F* s_out) {
-  const F t = block_sum<F>(v, s_red);
-  if (threadIdx.x == 0) *s_out = t;
+// N sums over the block at once, in a fixed tree order; every thread adds the
+// per-warp partials itself in the same order, so all get the same totals.
+template <int N>
+__device__ __forceinline__ void block_sums(double (&v)[N], double* s_red /* [SCAN_T / 32][N] */) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
+  }
+  if (lane == 0)
+#pragma unroll
+    for (int i = 0; i < N; ++i) s_red[warp * N + i] = v[i];
   __syncthreads();
-  const F r = *s_out;
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    double t = 0.0;
+    for (int w = 0; w < SCAN_T / 32; ++w) t += s_red[w * N + i];
+    v[i] = t;
+  }
   __syncthreads();
-  return r;
+}
+
+// Exclusive prefix sums of two ints over the block (thread order), and their totals.
+__device__ __forceinline__ void block_exscan_int2(int a0, int a1, int* s_warp2 /* [2][SCAN_T / 32 + 1] */,
+                                                  int& r0, int& r1, int& t0, int& t1) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int W = SCAN_T / 32;
+  int i0 = a0, i1 = a1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u0 = __shfl_up_sync(0xffffffffu, i0, o);
+    const int u1 = __shfl_up_sync(0xffffffffu, i1, o);
+    if (lane >= o) { i0 += u0; i1 += u1; }
+  }
+  if (lane == 31) { s_warp2[warp] = i0; s_warp2[W + 1 + warp] = i1; }
+  __syncthreads();
+  int b0 = 0, b1 = 0;
+  t0 = t1 = 0;
+  for (int w = 0; w < W; ++w) {
+    const int w0 = s_warp2[w], w1 = s_warp2[W + 1 + w];
+    if (w < warp) { b0 += w0; b1 += w1; }
+    t0 += w0;
+    t1 += w1;
+  }
+  r0 = b0 + i0 - a0;
+  r1 = b1 + i1 - a1;
+  __syncthreads();
 }
 
 // Capacity, expert offsets, tile prefix, dropped count, aux loss, z-loss and
 // the alternative balance statistics from the per-expert totals (thread e < E
 // holds routed expert e's; threads E .. E + n_shared - 1 stand for the shared
 // experts' groups of T rows, which take no part in capacity, counts or
-// losses), by all SCAN_T threads of one block.
-__device__ __forceinline__ void scan_finalize(const RoutingArgs& a, int cnt, int c1, float ps, int* s_warp,
-                                              int* s_redi, double* s_redd, double* s_bcast) {
+// losses), by all SCAN_T threads of one block.  Sums run in double, in a
+// fixed order.
+__device__ __forceinline__ void scan_finalize(const RoutingArgs& a, int cnt, int c1, float ps, int* s_warp2,
+                                              double* s_red) {
   const int tid = threadIdx.x, E = a.E, nb = a.nblk;
   const int groups = E + a.n_shared;
   const bool routed = tid < E;
@@ -324,9 +364,8 @@ __device__ __forceinline__ void scan_finalize(const RoutingArgs& a, int cnt, int
   if (routed) kept = (a.capacity < 0) ? cnt : static_cast<int>((int64_t)cnt < a.capacity ? (int64_t)cnt : a.capacity);
   else if (tid < groups) kept = static_cast<int>(a.T);
   const int mt = (kept + kTileM - 1) / kTileM;
-  int total_rows = 0, total_tiles = 0;
-  const int off = block_exscan_int(kept, s_warp, total_rows);
-  const int mp = block_exscan_int(mt, s_warp, total_tiles);
+  int off, mp, total_rows, total_tiles;
+  block_exscan_int2(kept, mt, s_warp2, off, mp, total_rows, total_tiles);
   if (routed) a.counts[tid] = cnt;
   if (tid < groups) {
     a.offsets[tid] = off;
@@ -338,31 +377,29 @@ __device__ __forceinline__ void scan_finalize(const RoutingArgs& a, int cnt, int
     if (tid < E) a.offsets_out[tid] = off;
     if (a.n_shared == 0 ? tid == 0 : tid == E) a.offsets_out[E] = a.n_shared == 0 ? total_rows : off;
   }
-  const int drop = block_sum<int>(routed ? cnt - kept : 0, s_redi);
   const double T = static_cast<double>(a.T);
+  const double c = routed ? static_cast<double>(cnt) : 0.0;
   const double Pe = routed ? static_cast<double>(ps) / T : 0.0;  // mean router probability of e
-  const double auxp = block_sum<double>(routed ? static_cast<double>(c1) * static_cast<double>(ps) : 0.0, s_redd);
-  // alternative balance statistics (population moments over the E experts)
-  const double mean_c = block_sum_all<double>(routed ? static_cast<double>(cnt) : 0.0, s_redd, s_bcast) / E;
-  const double mean_p = block_sum_all<double>(Pe, s_redd, s_bcast) / E;
-  const double dc = routed ? static_cast<double>(cnt) - mean_c : 0.0;
-  const double dp = routed ? Pe - mean_p : 0.0;
-  const double var_c = block_sum<double>(dc * dc, s_redd) / E;
-  const double var_p = block_sum<double>(dp * dp, s_redd) / E;
-  const double aux_all =
-      block_sum<double>(routed ? static_cast<double>(cnt) / (T * a.k) * Pe : 0.0, s_redd) * E;
   double zs = 0.0;
   for (int b = tid; b < nb; b += SCAN_T) zs += static_cast<double>(a.part_lse2[b]);
-  zs = block_sum<double>(zs, s_redd);
+  // dropped, sum f1*P (first choices), sum of counts, sum of P, sum counts*P, sum lse^2
+  double v[6] = {routed ? static_cast<double>(cnt - kept) : 0.0,
+                 routed ? static_cast<double>(c1) * static_cast<double>(ps) : 0.0, c, Pe, c * Pe, zs};
+  block_sums<6>(v, s_red);
+  // population moments over the E experts
+  const double mean_c = v[2] / E, mean_p = v[3] / E;
+  const double dc = routed ? c - mean_c : 0.0, dp = routed ? Pe - mean_p : 0.0;
+  double m2[2] = {dc * dc, dp * dp};
+  block_sums<2>(m2, s_red);
   if (tid == 0) {
     a.offsets[groups] = total_rows;
     a.mprefix[groups] = total_tiles;
-    *a.dropped = drop;
-    *a.aux = static_cast<float>(static_cast<double>(E) * auxp / (T * T));
-    *a.z = static_cast<float>(zs / T);
-    a.balance_out[0] = static_cast<float>(aux_all);
-    a.balance_out[1] = static_cast<float>(mean_c > 0.0 ? sqrt(var_c) / mean_c : 0.0);
-    a.balance_out[2] = static_cast<float>(mean_p > 0.0 ? var_p / (mean_p * mean_p) : 0.0);
+    *a.dropped = static_cast<int>(v[0]);
+    *a.aux = static_cast<float>(static_cast<double>(E) * v[1] / (T * T));
+    *a.z = static_cast<float>(v[5] / T);
+    a.balance_out[0] = static_cast<float>(E * v[4] / (T * a.k));
+    a.balance_out[1] = static_cast<float>(mean_c > 0.0 ? sqrt(m2[0] / E) / mean_c : 0.0);
+    a.balance_out[2] = static_cast<float>(mean_p > 0.0 ? (m2[1] / E) / (mean_p * mean_p) : 0.0);
   }
 }
 
@@ -370,11 +407,10 @@ __device__ __forceinline__ void scan_finalize(const RoutingArgs& a, int cnt, int
 // order.  Otherwise one block per expert as described above.
 template <bool SINGLE>
 __global__ void __launch_bounds__(SCAN_T) scan_kernel(RoutingArgs a) {
-  __shared__ int s_warp[SCAN_T / 32 + 1];
+  __shared__ int s_warp[2 * (SCAN_T / 32 + 1)];
   __shared__ float s_redf[SCAN_T / 32];
-  __shared__ double s_redd[SCAN_T / 32];
   __shared__ int s_redi[SCAN_T / 32];
-  __shared__ double s_bcast;
+  __shared__ double s_redd[6 * (SCAN_T / 32)];
   __shared__ int s_last;
   const int tid = threadIdx.x;
   const int E = a.E, nb = a.nblk;
@@ -393,7 +429,7 @@ __global__ void __launch_bounds__(SCAN_T) scan_kernel(RoutingArgs a) {
         ps += a.part_psum[row + b];
       }
     }
-    scan_finalize(a, cnt, c1, ps, s_warp, s_redi, s_redd, &s_bcast);
+    scan_finalize(a, cnt, c1, ps, s_warp, s_redd);
     return;
   }
   const int e = blockIdx.x;
@@ -428,7 +464,7 @@ __global__ void __launch_bounds__(SCAN_T) scan_kernel(RoutingArgs a) {
   __threadfence();
   // the last block
   scan_finalize(a, tid < E ? __ldcg(a.counts + tid) : 0, tid < E ? __ldcg(a.tot_cnt1 + tid) : 0,
-                tid < E ? __ldcg(a.tot_psum + tid) : 0.f, s_warp, s_redi, s_redd, &s_bcast);
+                tid < E ? __ldcg(a.tot_psum + tid) : 0.f, s_warp, s_redd);
   if (tid == 0) *a.scan_ticket = 0;  // ready for the next call
 }
 
