@@ -41,7 +41,7 @@ namespace {
 constexpr int BM = kTileM;               // rows per tile
 constexpr int BK = 64;                   // bf16 per 128-byte smem row
 constexpr int MMA_N = 256;               // columns per MMA / accumulator
-constexpr int MAX_STAGES = 4;
+constexpr int MAX_STAGES = 5;
 constexpr int A_BYTES = BM * BK * 2;     // 16 KB
 constexpr int A_SHORT = 16;              // rows per A box of a partly filled tile
 constexpr int B_HALF = 128 * BK * 2;     // 16 KB per B box
@@ -50,11 +50,17 @@ constexpr int NUM_THREADS = 192;
 // Pipeline geometry.  SPLIT: the A operand is held as two bf16 planes
 // (hi + lo, about 16 significant bits) and every k-block issues the MMAs of
 // both planes against the same B tile, so one stage holds two A boxes.
-template <bool SPLIT>
+// AR: A rows a stage holds (32, 64 or 128).  No expert group has more rows
+// than the batch has tokens, so small batches stage only AR rows of A and fit
+// more stages (more weight bytes in flight per SM) in the same shared memory;
+// the M = 128 MMA still reads 128 rows from the A base, and rows past AR (the
+// next bytes of the stage) only feed accumulator rows that are never stored.
+template <bool SPLIT, int AR>
 struct Geo {
   static constexpr int kA = SPLIT ? 2 : 1;
-  static constexpr int STAGES = SPLIT ? 3 : 4;
-  static constexpr int STAGE_BYTES = kA * A_BYTES + 2 * B_HALF;
+  static constexpr int A_ST = AR * BK * 2;  // one plane of A in a stage
+  static constexpr int STAGE_BYTES = kA * A_ST + 2 * B_HALF;
+  static constexpr int STAGES = (200 * 1024 / STAGE_BYTES) < MAX_STAGES ? (200 * 1024 / STAGE_BYTES) : MAX_STAGES;
 };
 constexpr uint32_t TMEM_COLS = 2 * MMA_N;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, MMA_N);
@@ -76,9 +82,9 @@ struct Ctl {
   alignas(16) uint8_t stage_out[4][32 * 144];
 };
 
-template <bool SPLIT>
+template <bool SPLIT, int AR>
 constexpr size_t smem_bytes() {
-  return Geo<SPLIT>::STAGES * Geo<SPLIT>::STAGE_BYTES + sizeof(Ctl) + 1024;
+  return Geo<SPLIT, AR>::STAGES * Geo<SPLIT, AR>::STAGE_BYTES + sizeof(Ctl) + 1024;
 }
 
 // Tile t -> (expert, m-tile, n-tile); tiles are expert-major, then n, then m.
@@ -153,7 +159,7 @@ __device__ __forceinline__ void split_bf16(float v0, float v1, uint32_t& hi, uin
 // EPI: epilogue (internal.h GemmEpi).  SPLIT: for the first projection the
 // epilogue writes the hidden activation as hi/lo planes; for the second the
 // A operand is read as hi (tmA) + lo (tmA2) planes.
-template <int EPI, bool SPLIT>
+template <int EPI, bool SPLIT, int AR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                         const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
@@ -161,9 +167,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         const Params p) {
   constexpr bool A_SPLIT = SPLIT && (EPI == EPI_GATE_F32 || EPI == EPI_GATE_SCATTER_BF16);
   constexpr bool OUT_SPLIT = SPLIT && (EPI == EPI_RELU_BF16 || EPI == EPI_SWIGLU_BF16);
-  constexpr int STAGES = Geo<A_SPLIT>::STAGES;
-  constexpr int STAGE_BYTES = Geo<A_SPLIT>::STAGE_BYTES;
-  constexpr int B_OFF = Geo<A_SPLIT>::kA * A_BYTES;
+  using G = Geo<A_SPLIT, AR>;
+  constexpr int STAGES = G::STAGES;
+  constexpr int STAGE_BYTES = G::STAGE_BYTES;
+  constexpr int A_ST = G::A_ST;
+  constexpr int B_OFF = G::kA * A_ST;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* stages = smem_raw + pad;
@@ -214,8 +222,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // Short boxes only for a single-plane A: with the hi + lo planes the
         // extra copies cost more than the rows they save.
         const int vrows = ctl->offsets[e + 1] - row0;
-        const int nshort = (A_SPLIT || vrows >= BM) ? 0 : (vrows + A_SHORT - 1) / A_SHORT;
-        const uint32_t a_bytes = nshort == 0 ? A_BYTES : nshort * A_SHORT * BK * 2;
+        const int nshort = (A_SPLIT || vrows >= AR) ? 0 : (vrows + A_SHORT - 1) / A_SHORT;
+        const uint32_t a_bytes = nshort == 0 ? A_ST : nshort * A_SHORT * BK * 2;
         const uint32_t tx = (A_SPLIT ? 2u : 1u) * a_bytes + 2u * B_HALF;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_or_abort(ctl, &ctl->empty[stage], phase ^ 1u, p)) { ok = false; break; }
@@ -228,7 +236,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int j = 0; j < nshort; ++j) {
               tma_load_2d(sa + j * A_SHORT * BK * 2, &tmAs, &ctl->full[stage], kb * BK, row0 + j * A_SHORT);
               if (A_SPLIT)
-                tma_load_2d(sa + A_BYTES + j * A_SHORT * BK * 2, &tmAs2, &ctl->full[stage], kb * BK,
+                tma_load_2d(sa + A_ST + j * A_SHORT * BK * 2, &tmAs2, &ctl->full[stage], kb * BK,
                             row0 + j * A_SHORT);
             }
           }
@@ -272,7 +280,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (A_SPLIT) {
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k)
-              umma_bf16(d_tmem, sdesc_k_sw128(sa + A_BYTES + k * 32), sdesc_k_sw128(sb + k * 32), IDESC, 1u);
+              umma_bf16(d_tmem, sdesc_k_sw128(sa + A_ST + k * 32), sdesc_k_sw128(sb + k * 32), IDESC, 1u);
           }
           umma_commit(&ctl->empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -485,15 +493,23 @@ bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t col
 
 namespace {
 
-template <int EPI, bool SPLIT>
+template <int EPI, bool SPLIT, int AR>
 cudaError_t launch_t(const TcGemmPlan& pl, int num_sms, cudaStream_t s) {
   constexpr bool A_SPLIT = SPLIT && (EPI == EPI_GATE_F32 || EPI == EPI_GATE_SCATTER_BF16);
-  constexpr size_t bytes = smem_bytes<A_SPLIT>();
-  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void*>(&grouped_gemm_kernel<EPI, SPLIT>),
+  constexpr size_t bytes = smem_bytes<A_SPLIT, AR>();
+  static_assert(bytes <= 227 * 1024, "grouped GEMM shared memory");
+  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void*>(&grouped_gemm_kernel<EPI, SPLIT, AR>),
                                       static_cast<int>(bytes));
   if (e != cudaSuccess) return e;
-  return launch_pdl(grouped_gemm_kernel<EPI, SPLIT>, dim3(num_sms), dim3(NUM_THREADS), bytes, s, pl.a, pl.a2, pl.b0,
-                    pl.b1, pl.as, pl.as2, pl.p);
+  return launch_pdl(grouped_gemm_kernel<EPI, SPLIT, AR>, dim3(num_sms), dim3(NUM_THREADS), bytes, s, pl.a, pl.a2,
+                    pl.b0, pl.b1, pl.as, pl.as2, pl.p);
+}
+
+template <int EPI, bool SPLIT>
+cudaError_t launch_ar(const TcGemmPlan& pl, int num_sms, cudaStream_t s) {
+  if (pl.ar == 32) return launch_t<EPI, SPLIT, 32>(pl, num_sms, s);
+  if (pl.ar == 64) return launch_t<EPI, SPLIT, 64>(pl, num_sms, s);
+  return launch_t<EPI, SPLIT, 128>(pl, num_sms, s);
 }
 
 }  // namespace
@@ -503,6 +519,9 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
   if (g.E > MAX_E) { *why = "grouped GEMM supports at most 256 experts"; return cudaErrorInvalidValue; }
   const bool a_split = g.split && g.A2 != nullptr;
   const bool swiglu = g.epi == EPI_SWIGLU_BF16;
+  // A rows per stage: every expert group has at most max_group_rows rows
+  pl->ar = g.max_group_rows <= 32 ? 32 : g.max_group_rows <= 64 ? 64 : 128;
+  const uint32_t ar = static_cast<uint32_t>(pl->ar);
   const uint64_t a_rows = static_cast<uint64_t>(g.a_rows), K = static_cast<uint64_t>(g.K);
   const uint64_t b_rows = static_cast<uint64_t>(g.E) * g.N;
   // a split A is read through one 3D map over both planes (the lo plane must
@@ -514,8 +533,8 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
     return cudaErrorInvalidValue;
   }
   const bool maps_ok =
-      (a_split ? make_map_planes_bf16(&pl->a, g.A, static_cast<uint64_t>(plane_stride), a_rows, K, 128)
-               : make_map(&pl->a, g.A, a_rows, K)) &&
+      (a_split ? make_map_planes_bf16(&pl->a, g.A, static_cast<uint64_t>(plane_stride), a_rows, K, ar)
+               : make_map_bf16(&pl->a, g.A, a_rows, K, ar)) &&
       make_map(&pl->a2, a_split ? g.A2 : g.A, a_rows, K) && make_map_bf16(&pl->as, g.A, a_rows, K, A_SHORT) &&
       make_map_bf16(&pl->as2, a_split ? g.A2 : g.A, a_rows, K, A_SHORT) &&
       // B: two 128-row boxes (W1 and W3) for SwiGLU, else one 256-row box
@@ -556,17 +575,17 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
 cudaError_t launch_gemm_tc(const TcGemmPlan& pl, int num_sms, cudaStream_t s) {
   if (pl.split) {
     switch (pl.epi) {
-      case EPI_RELU_BF16: return launch_t<EPI_RELU_BF16, true>(pl, num_sms, s);
-      case EPI_SWIGLU_BF16: return launch_t<EPI_SWIGLU_BF16, true>(pl, num_sms, s);
-      case EPI_GATE_F32: return launch_t<EPI_GATE_F32, true>(pl, num_sms, s);
-      default: return launch_t<EPI_GATE_SCATTER_BF16, true>(pl, num_sms, s);
+      case EPI_RELU_BF16: return launch_ar<EPI_RELU_BF16, true>(pl, num_sms, s);
+      case EPI_SWIGLU_BF16: return launch_ar<EPI_SWIGLU_BF16, true>(pl, num_sms, s);
+      case EPI_GATE_F32: return launch_ar<EPI_GATE_F32, true>(pl, num_sms, s);
+      default: return launch_ar<EPI_GATE_SCATTER_BF16, true>(pl, num_sms, s);
     }
   }
   switch (pl.epi) {
-    case EPI_RELU_BF16: return launch_t<EPI_RELU_BF16, false>(pl, num_sms, s);
-    case EPI_SWIGLU_BF16: return launch_t<EPI_SWIGLU_BF16, false>(pl, num_sms, s);
-    case EPI_GATE_F32: return launch_t<EPI_GATE_F32, false>(pl, num_sms, s);
-    default: return launch_t<EPI_GATE_SCATTER_BF16, false>(pl, num_sms, s);
+    case EPI_RELU_BF16: return launch_ar<EPI_RELU_BF16, false>(pl, num_sms, s);
+    case EPI_SWIGLU_BF16: return launch_ar<EPI_SWIGLU_BF16, false>(pl, num_sms, s);
+    case EPI_GATE_F32: return launch_ar<EPI_GATE_F32, false>(pl, num_sms, s);
+    default: return launch_ar<EPI_GATE_SCATTER_BF16, false>(pl, num_sms, s);
   }
 }
 

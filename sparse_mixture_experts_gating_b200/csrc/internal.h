@@ -101,6 +101,7 @@ struct GemmArgs {
   int N;  // output columns per expert
   int K;  // reduction length
   int64_t a_rows;  // rows of the A buffer (S_max)
+  int64_t max_group_rows;  // no expert group has more rows (the batch's T)
   const void* A;   // [a_rows][K]  (the hi plane when split)
   const void* A2;  // [a_rows][K]  lo plane of a split A operand, else NULL
   int split;       // first projection: write hi/lo planes; second: read them
@@ -141,6 +142,7 @@ struct TcGemmPlan {
   TcParams p;
   int epi;
   int split;
+  int ar;  // A rows per pipeline stage: 32, 64 or 128
 };
 
 cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* plan, const char** why);

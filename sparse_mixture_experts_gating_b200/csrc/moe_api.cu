@@ -356,6 +356,7 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   g1.N = L.d_ff;
   g1.K = L.d;
   g1.a_rows = w.s_max;
+  g1.max_group_rows = T;  // a token takes each expert at most once; a shared expert's group has T rows
   g1.A = ws + w.Xp;
   g1.B0 = W1;
   g1.B1 = W3;

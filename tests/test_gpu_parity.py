@@ -55,6 +55,9 @@ SMALL = [
     ("shared_switch_k1_drops", 400, 64, 16, 1, 128, R, SW, 0.5, BF, "normal", 2),
     ("shared_fp32", 120, 24, 4, 2, 40, S, RN, 1.0, F32, None, 1),
     ("shared_decode_splitk", 2, 256, 8, 2, 1024, S, RN, 0.0, BF, None, 1),
+    # 33 <= T <= 64: pipeline stages hold 64 rows of A (T <= 32: 32 rows)
+    ("ar64_swiglu", 48, 256, 8, 2, 512, S, RN, 0.0, BF, None),
+    ("ar64_switch_shared", 61, 192, 4, 1, 384, R, SW, 1.0, BF, "normal", 1),
 ]
 
 
@@ -81,7 +84,8 @@ def test_small_layers_match_oracle(case):
 
 SINGLE = [c for c in SMALL if c[9] == BF and c[0] in ("swiglu_e8_k2", "switch_relu_drops", "k4_zipf_tails",
                                                        "e128_k8_cap", "long_k_ragged", "stream_k_tail_relu",
-                                                       "stream_k_switch_pieces", "shared_switch_k1_drops")]
+                                                       "stream_k_switch_pieces", "shared_switch_k1_drops",
+                                                       "one_token", "ar64_swiglu")]
 
 
 @pytest.mark.parametrize("case", SINGLE, ids=[c[0] for c in SINGLE])
