@@ -4,8 +4,8 @@
 
 One step = one forward pass of the whole layer (router, scan, dispatch, two
 grouped GEMMs, combine, losses) over one batch of the workload's synthetic
-input, resident in HBM.  L2 is flushed (a 256 MiB write) between steps,
-outside the timed events.  Prints ONE JSON line on rank 0.
+input, resident in HBM.  L2 is flushed between steps, outside the timed
+events: a 256 MiB write, then a 256 MiB read of another buffer.  Prints ONE JSON line on rank 0.
 
 N > 1 (torchrun): every rank runs an independent replica of the layer on its
 own batch (the layer has no cross-batch exchange), so scaling is weak; the
@@ -203,7 +203,8 @@ def config_of(w, n_gpus):
             "act": "swiglu" if w.act == 1 else "relu", "gate": "renorm" if w.gate == 1 else "switch",
             "capacity_factor": w.capacity_factor, "tokens_per_gpu": w.T,
             "parallelism": "replicas" if n_gpus > 1 else "single",
-            "l2": "flushed between steps (256 MiB write, outside the timed events)"}
+            "l2": "flushed between steps outside the timed events: a 256 MiB write, then a 256 MiB read of "
+                  "another buffer (the write's dirty lines go back to HBM before the step starts)"}
 
 
 # ----------------------------------------------------------------------------- CPU (oracle) leg
@@ -303,6 +304,14 @@ def main():
     stats = (torch.empty(w.E, dtype=torch.int32, device=dev), torch.empty(1, dtype=torch.int32, device=dev),
              torch.empty(1, dtype=torch.float32, device=dev), torch.empty(1, dtype=torch.float32, device=dev))
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_rd = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
+
+    def flush_l2():
+        # a write larger than L2, then a read of another buffer larger than L2:
+        # the write's dirty lines are written back here, outside the timed
+        # events, and the step starts with L2 holding none of its inputs
+        flush.zero_()
+        flush_rd.sum()
     stream = torch.cuda.current_stream()
     args_fw = (inp["x"], inp["W_r"], inp["b_r"], inp["W1"], inp["W3"], inp["W2"])
 
@@ -311,7 +320,7 @@ def main():
         layer(*a, out=y, stats=stats, workspace=ws, events=events)
 
     for _ in range(warmup):
-        flush.zero_()
+        flush_l2()
         step()
     status()
 
@@ -324,7 +333,7 @@ def main():
     torch.cuda.synchronize()
     gpu_hold(torch, 2.0 + 0.3 * K)
     for i in range(K):
-        flush.zero_()
+        flush_l2()
         step(events=ev_stage[i])
     torch.cuda.synchronize()
     stage_ms = {}
@@ -351,7 +360,7 @@ def main():
     wall0 = time.time()
     gpu_hold(torch, 2.0 + 0.2 * K)
     for i in range(K):
-        flush.zero_()
+        flush_l2()
         ev_step[i][0].record(stream)
         step(events=ev_dom[i])
         ev_step[i][1].record(stream)
@@ -377,7 +386,7 @@ def main():
     torch.cuda.synchronize()
     gpu_hold(torch, 2.0 + 0.2 * (K + warmup))
     for i in range(warmup + K):
-        flush.zero_()
+        flush_l2()
         if i >= warmup:
             e2e_ev[i - warmup][0].record(stream)
         x_dev.copy_(x_host, non_blocking=True)
