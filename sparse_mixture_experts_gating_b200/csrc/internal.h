@@ -79,6 +79,12 @@ bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t col
 bool make_map_planes_bf16(CUtensorMap* m, const void* base, uint64_t plane_stride, uint64_t rows, uint64_t cols,
                           uint32_t box_rows);
 cudaError_t launch_scan(const RoutingArgs& a, cudaStream_t s);
+// Batches of at most 32 tokens (one router block): router, scan and dispatch
+// in two launches (fp32 partial logits over d-chunks, then one block for the
+// rest).  `partials` holds route_small_partials_bytes(E).
+constexpr int kRouteSmallMaxT = 32;
+size_t route_small_partials_bytes(int E);
+cudaError_t launch_route_small(const RoutingArgs& a, void* partials, cudaStream_t s);
 cudaError_t launch_dispatch(const RoutingArgs& a, cudaStream_t s);
 // y_t = sum over kept choices j (in order j) of sum over the ksplit partials
 // (in order) of Yp[partial][dest_row[t][j]], then (in order s) of the rows

@@ -97,7 +97,7 @@ struct Layout {
   bool split;
   int ksplit;
   size_t idx, gate, dest, row_token, row_gate, part_hist, part_cnt1, part_psum, part_lse2, blockoff, counts,
-      offsets, mprefix, scal, wsplit, rpart, Xp, Hp, Hp_lo, Yp, total;
+      offsets, mprefix, scal, wsplit, rpart, spart, Xp, Hp, Hp_lo, Yp, total;
 };
 
 Layout make_layout(const moe_layer& L, int64_t T) {
@@ -132,6 +132,7 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   const bool tc_router = L.dtype == MOE_BF16 && L.E <= kRouterTcMaxE;
   w.wsplit = take(tc_router ? 3 * sizeof(uint16_t) * router_pad_e(L.E) * static_cast<size_t>(L.d) : 0);
   w.rpart = take(tc_router ? router_partials_bytes(T, L.E, L.d) : 0);
+  w.spart = take(route_small_partials_bytes(L.E));  // batches of <= 32 tokens (constant: sizes stay monotone)
   w.Xp = take(elt * static_cast<size_t>(w.s_max) * L.d);
   w.Hp = take(elt * static_cast<size_t>(w.s_max) * L.d_ff);
   w.Hp_lo = take(w.split ? elt * static_cast<size_t>(w.s_max) * L.d_ff : 0);
@@ -399,21 +400,32 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   };
   int rc;
   record(dbg, MOE_STAGE_ROUTER, 0, s);
-  if (tc && L.E <= kRouterTcMaxE && r.logits_in == nullptr) {
-    const char* why = nullptr;
-    ce = launch_router_tc(r, ws + w.wsplit, ws + w.rpart, di->num_sms, di->err, s, &why);
-    if (why != nullptr) return fail(MOE_ERR_UNSUPPORTED, std::string("moe_forward: ") + why);
-    if ((rc = check(ce, "router")) != MOE_OK) return rc;
-  } else if ((rc = check(launch_router(r, s), "router")) != MOE_OK) {
-    return rc;
+  if (T <= kRouteSmallMaxT) {
+    // one router block: router, scan and dispatch in two launches (the scan
+    // and dispatch stages of the debug events stay empty)
+    if ((rc = check(launch_route_small(r, ws + w.spart, s), "router")) != MOE_OK) return rc;
+    record(dbg, MOE_STAGE_ROUTER, 1, s);
+    record(dbg, MOE_STAGE_SCAN, 0, s);
+    record(dbg, MOE_STAGE_SCAN, 1, s);
+    record(dbg, MOE_STAGE_DISPATCH, 0, s);
+    record(dbg, MOE_STAGE_DISPATCH, 1, s);
+  } else {
+    if (tc && L.E <= kRouterTcMaxE && r.logits_in == nullptr) {
+      const char* why = nullptr;
+      ce = launch_router_tc(r, ws + w.wsplit, ws + w.rpart, di->num_sms, di->err, s, &why);
+      if (why != nullptr) return fail(MOE_ERR_UNSUPPORTED, std::string("moe_forward: ") + why);
+      if ((rc = check(ce, "router")) != MOE_OK) return rc;
+    } else if ((rc = check(launch_router(r, s), "router")) != MOE_OK) {
+      return rc;
+    }
+    record(dbg, MOE_STAGE_ROUTER, 1, s);
+    record(dbg, MOE_STAGE_SCAN, 0, s);
+    if ((rc = check(launch_scan(r, s), "scan")) != MOE_OK) return rc;
+    record(dbg, MOE_STAGE_SCAN, 1, s);
+    record(dbg, MOE_STAGE_DISPATCH, 0, s);
+    if ((rc = check(launch_dispatch(r, s), "dispatch")) != MOE_OK) return rc;
+    record(dbg, MOE_STAGE_DISPATCH, 1, s);
   }
-  record(dbg, MOE_STAGE_ROUTER, 1, s);
-  record(dbg, MOE_STAGE_SCAN, 0, s);
-  if ((rc = check(launch_scan(r, s), "scan")) != MOE_OK) return rc;
-  record(dbg, MOE_STAGE_SCAN, 1, s);
-  record(dbg, MOE_STAGE_DISPATCH, 0, s);
-  if ((rc = check(launch_dispatch(r, s), "dispatch")) != MOE_OK) return rc;
-  record(dbg, MOE_STAGE_DISPATCH, 1, s);
 
   record(dbg, MOE_STAGE_GEMM1, 0, s);
   ce = tc ? launch_gemm_tc(plan1, di->num_sms, s) : launch_gemm_simt(g1, w.s_max, s);

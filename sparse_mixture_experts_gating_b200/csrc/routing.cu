@@ -568,6 +568,218 @@ __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Small batches (T <= 32: one router block).  Two kernels replace the router,
+// scan and dispatch:
+//   route_small_dot_kernel  grid (DS, E): block (ds, e) sums W_r[e][c] x[t][c]
+//                           over its d-chunk for every token t (fp32, a fixed
+//                           block-tree order) into partial[ds][t][e];
+//   route_small_kernel      one block of SCAN_T threads: logits = the DS
+//                           partials in order (+ bias), then softmax,
+//                           log-sum-exp, top-k and gates (a warp per token,
+//                           lanes over experts), the per-expert totals, the
+//                           scan's capacity / offsets / losses (scan_finalize),
+//                           slot ranks in token order, and the row copies.
+constexpr int SMALL_T = 32;
+constexpr int SMALL_DS_MAX = 16;
+
+template <typename XT>
+__global__ void __launch_bounds__(256) route_small_dot_kernel(RoutingArgs a, int chunk, float* __restrict__ partial) {
+  __shared__ float s_red[8][SMALL_T];
+  const int ds = blockIdx.x, e = blockIdx.y, tid = threadIdx.x;
+  const int T = static_cast<int>(a.T), d = a.d;
+  const XT* x = static_cast<const XT*>(a.x);
+  const float* w = a.W_r + static_cast<int64_t>(e) * d;
+  const int c0 = ds * chunk, c1 = min(d, c0 + chunk);
+  float acc[SMALL_T];
+#pragma unroll
+  for (int t = 0; t < SMALL_T; ++t) acc[t] = 0.f;
+  for (int c = c0 + tid; c < c1; c += 256) {
+    const float wv = w[c];
+#pragma unroll
+    for (int t = 0; t < SMALL_T; ++t)
+      if (t < T) acc[t] = fmaf(wv, to_f32(x[static_cast<int64_t>(t) * d + c]), acc[t]);
+  }
+  const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+  for (int t = 0; t < SMALL_T; ++t) {
+    if (t < T) {
+      float v = acc[t];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) s_red[warp][t] = v;
+    }
+  }
+  __syncthreads();
+  if (tid < T) {
+    float v = 0.f;
+#pragma unroll
+    for (int wi = 0; wi < 8; ++wi) v += s_red[wi][tid];
+    partial[(static_cast<int64_t>(ds) * T + tid) * a.E + e] = v;
+  }
+}
+
+template <typename XT>
+__global__ void __launch_bounds__(SCAN_T) route_small_kernel(RoutingArgs a, int n_ds, const float* __restrict__ partial) {
+  extern __shared__ __align__(16) float sm_h[];  // [T][E]: logits, then probabilities
+  __shared__ int s_idx[SMALL_T * 8];
+  __shared__ float s_gate[SMALL_T * 8];
+  __shared__ int s_hist[256], s_cnt1[256], s_dest[SMALL_T * 8];
+  __shared__ float s_lse2[SMALL_T];
+  __shared__ int s_warp[2 * (SCAN_T / 32 + 1)];
+  __shared__ double s_red[6 * (SCAN_T / 32)];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int T = static_cast<int>(a.T), E = a.E, k = a.k, d = a.d;
+  pdl_wait();
+  pdl_trigger();
+  for (int e = tid; e < 256; e += SCAN_T) { s_hist[e] = 0; s_cnt1[e] = 0; }
+  // logits: partials in d-chunk order, then the bias
+  for (int i = tid; i < T * E; i += SCAN_T) {
+    const int t = i / E, e = i - t * E;
+    float h;
+    if (a.logits_in != nullptr) {
+      h = a.logits_in[i];
+    } else {
+      h = 0.f;
+      for (int ds = 0; ds < n_ds; ++ds) h += partial[(static_cast<int64_t>(ds) * T + t) * E + e];
+      if (a.b_r != nullptr) h += a.b_r[e];
+    }
+    if (h != h) h = -INFINITY;  // NaN logits (out of contract) rank last
+    sm_h[i] = h;
+    if (a.logits_out != nullptr) a.logits_out[i] = h;
+  }
+  __syncthreads();
+  // a warp per token: max, log-sum-exp, top-k (value desc, index asc), gates
+  for (int t = warp; t < T; t += SCAN_T / 32) {
+    float* h = sm_h + t * E;
+    float m = -INFINITY;
+    for (int e = lane; e < E; e += 32) m = fmaxf(m, h[e]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float sl = 0.f;
+    for (int e = lane; e < E; e += 32) sl += expf(h[e] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sl += __shfl_xor_sync(0xffffffffu, sl, o);
+    const float inv_s = 1.f / sl;
+    const float lse = m + logf(sl);
+    uint32_t picked = 0;  // bit i: this lane's expert lane + 32 i is taken
+    float tv0 = 0.f, den = 0.f;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff, bi = -1;
+      for (int i = 0, e = lane; e < E; ++i, e += 32)
+        if (!((picked >> i) & 1u) && (be == 0x7fffffff || h[e] > bv)) { bv = h[e]; be = e; bi = i; }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
+      }
+      if (bi >= 0 && lane + 32 * bi == be) picked |= 1u << bi;
+      if (j == 0) tv0 = bv;
+      const float gsw = expf(bv - m) * inv_s;
+      const float ren = expf(bv - tv0);
+      den += ren;
+      if (lane == 0) {
+        s_idx[t * k + j] = be;
+        s_gate[t * k + j] = a.gate_mode == 0 ? gsw : ren;  // renormalised below
+        a.topk_idx[t * k + j] = be;
+        atomicAdd(&s_hist[be], 1);
+        if (j == 0) atomicAdd(&s_cnt1[be], 1);
+      }
+    }
+    if (lane == 0) {
+      for (int j = 0; j < k; ++j) {
+        if (a.gate_mode != 0) s_gate[t * k + j] /= den;
+        a.topk_gate[t * k + j] = s_gate[t * k + j];
+      }
+      if (a.lse_out != nullptr) a.lse_out[t] = lse;
+      s_lse2[t] = lse * lse;
+    }
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) h[e] = expf(h[e] - m) * inv_s;  // probabilities
+  }
+  __syncthreads();
+  // per-expert totals in token order; z from the token lse^2 in order
+  int cnt = 0, c1 = 0;
+  float ps = 0.f;
+  if (tid < E) {
+    cnt = s_hist[tid];
+    c1 = s_cnt1[tid];
+    for (int t = 0; t < T; ++t) ps += sm_h[t * E + tid];
+  }
+  if (tid == 0) {
+    float z2 = 0.f;
+    for (int t = 0; t < T; ++t) z2 += s_lse2[t];
+    a.part_lse2[0] = z2;
+  }
+  __syncthreads();
+  scan_finalize(a, cnt, c1, ps, s_warp, s_red);  // counts, offsets, tile prefix, dropped, losses
+  // slot ranks in token order (assignment i = t * k + j), kept flags, destinations
+  const int nA = T * k;
+  for (int i = tid; i < nA; i += SCAN_T) {
+    const int e = s_idx[i];
+    int rank = 0;
+    for (int i2 = 0; i2 < i; ++i2) rank += s_idx[i2] == e;
+    const bool kept = a.capacity < 0 || rank < a.capacity;
+    const int dest = kept ? a.offsets[e] + rank : -1;
+    s_dest[i] = dest;
+    a.dest_row[i] = dest;
+    if (a.drop_mask != nullptr) a.drop_mask[i] = kept ? 0 : 1;
+    if (kept) {
+      a.row_token[dest] = i / k;
+      a.row_gate[dest] = s_gate[i];
+    }
+  }
+  __syncthreads();
+  // row copies (a warp per row): kept assignments, then the shared experts' rows
+  const XT* x = static_cast<const XT*>(a.x);
+  XT* Xp = static_cast<XT*>(a.Xp);
+  XT* yz = static_cast<XT*>(a.y_zero_dropped);
+  const bool vec = (static_cast<size_t>(d) * sizeof(XT)) % 16 == 0;
+  auto copy_row = [&](int64_t tok, int64_t dest) {
+    if (vec) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + tok * d);
+      uint4* dst = reinterpret_cast<uint4*>(Xp + dest * d);
+      const int nv = static_cast<int>(static_cast<size_t>(d) * sizeof(XT) / 16);
+      for (int v0 = lane; v0 < nv; v0 += 128) {
+        uint4 c[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (v0 + 32 * q < nv) c[q] = src[v0 + 32 * q];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (v0 + 32 * q < nv) dst[v0 + 32 * q] = c[q];
+      }
+    } else {
+      for (int c = lane; c < d; c += 32) Xp[dest * d + c] = x[tok * d + c];
+    }
+  };
+  for (int i = warp; i < nA; i += SCAN_T / 32) {
+    const int64_t tok = i / k;
+    if (s_dest[i] >= 0) {
+      copy_row(tok, s_dest[i]);
+    } else if (yz != nullptr) {  // k == 1: a dropped token's output row is zero
+      for (int c = lane; c < d; c += 32) yz[tok * d + c] = XT(0.f);
+      if (a.yf_zero_dropped != nullptr)
+        for (int c = lane; c < d; c += 32) a.yf_zero_dropped[tok * d + c] = 0.f;
+    }
+  }
+  if (a.n_shared > 0) {
+    const int64_t base = a.offsets[E];
+    for (int q = warp; q < T * a.n_shared; q += SCAN_T / 32) {
+      const int si = q / T;
+      const int64_t tok = q - si * T;
+      const int64_t row = base + si * static_cast<int64_t>(T) + tok;
+      if (lane == 0) {
+        a.row_token[row] = static_cast<int32_t>(tok);
+        a.row_gate[row] = 1.f;
+      }
+      copy_row(tok, row);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Combine: y_t = sum over kept choices j (ascending) of the slot's row of Yp
 // (summed over its K-range partials in order).  A thread owns CU groups of 4
 // columns (grid-strided, so every load instruction of a warp is one run of
@@ -709,6 +921,45 @@ __global__ void selftest_timeout_kernel(unsigned int* err, uint64_t limit_ns) {
 
 cudaError_t launch_router(const RoutingArgs& a, cudaStream_t s) {
   return a.x_is_bf16 ? launch_router_x<__nv_bfloat16>(a, s) : launch_router_x<float>(a, s);
+}
+
+int route_small_chunks(int E, int d) {
+  int ds = (d + 255) / 256;
+  const int want = (2 * 148 + E - 1) / E;  // about two blocks per SM over all experts
+  if (ds > want) ds = want;
+  if (ds > SMALL_DS_MAX) ds = SMALL_DS_MAX;
+  return ds < 1 ? 1 : ds;
+}
+
+size_t route_small_partials_bytes(int E) {
+  return static_cast<size_t>(SMALL_DS_MAX) * SMALL_T * E * sizeof(float);
+}
+
+cudaError_t launch_route_small(const RoutingArgs& a, void* partials, cudaStream_t s) {
+  const int n_ds = route_small_chunks(a.E, a.d);
+  const int chunk = (a.d + n_ds - 1) / n_ds;
+  float* part = static_cast<float*>(partials);
+  const size_t smem = static_cast<size_t>(a.T) * a.E * sizeof(float);
+  cudaError_t e;
+  if (a.logits_in == nullptr) {  // the first kernel of the forward: an ordinary launch
+    if (a.x_is_bf16)
+      route_small_dot_kernel<__nv_bfloat16><<<dim3(n_ds, a.E), 256, 0, s>>>(a, chunk, part);
+    else
+      route_small_dot_kernel<float><<<dim3(n_ds, a.E), 256, 0, s>>>(a, chunk, part);
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (a.x_is_bf16)
+      return launch_pdl(route_small_kernel<__nv_bfloat16>, dim3(1), dim3(SCAN_T), smem, s, a, n_ds,
+                        static_cast<const float*>(part));
+    return launch_pdl(route_small_kernel<float>, dim3(1), dim3(SCAN_T), smem, s, a, n_ds,
+                      static_cast<const float*>(part));
+  }
+  if (a.x_is_bf16)
+    route_small_kernel<__nv_bfloat16><<<1, SCAN_T, smem, s>>>(a, 0, part);
+  else
+    route_small_kernel<float><<<1, SCAN_T, smem, s>>>(a, 0, part);
+  count_launch();
+  return cudaGetLastError();
 }
 
 cudaError_t launch_scan(const RoutingArgs& a, cudaStream_t s) {
