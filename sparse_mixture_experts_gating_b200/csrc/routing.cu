@@ -527,13 +527,13 @@ __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
       const uint4* src = reinterpret_cast<const uint4*>(x + tok * d);
       uint4* dst = reinterpret_cast<uint4*>(Xp + dest * d);
       const int nv = static_cast<int>(static_cast<size_t>(d) * sizeof(XT) / 16);
-      for (int v0 = lane; v0 < nv; v0 += 128) {  // up to four 16-byte loads in flight per lane
-        uint4 c[4];
+      for (int v0 = lane; v0 < nv; v0 += 256) {  // up to eight 16-byte loads in flight per lane
+        uint4 c[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 8; ++q)
           if (v0 + 32 * q < nv) c[q] = src[v0 + 32 * q];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 8; ++q)
           if (v0 + 32 * q < nv) dst[v0 + 32 * q] = c[q];
       }
     } else {
@@ -741,13 +741,13 @@ __global__ void __launch_bounds__(SCAN_T) route_small_kernel(RoutingArgs a, int 
       const uint4* src = reinterpret_cast<const uint4*>(x + tok * d);
       uint4* dst = reinterpret_cast<uint4*>(Xp + dest * d);
       const int nv = static_cast<int>(static_cast<size_t>(d) * sizeof(XT) / 16);
-      for (int v0 = lane; v0 < nv; v0 += 128) {
-        uint4 c[4];
+      for (int v0 = lane; v0 < nv; v0 += 256) {
+        uint4 c[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 8; ++q)
           if (v0 + 32 * q < nv) c[q] = src[v0 + 32 * q];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 8; ++q)
           if (v0 + 32 * q < nv) dst[v0 + 32 * q] = c[q];
       }
     } else {
