@@ -11,11 +11,8 @@
 // sharing a weight slab run at the same time and the slab is read from HBM once.
 //
 // Warp roles (192 threads, one CTA per SM):
-//   warp 0       TMA producer: A box [128 x 64] + two B boxes [128 x 64] per stage;
-//                with a single-plane A, a tile whose expert group ends inside it
-//                loads only the 16-row A boxes that hold rows of the group (the
-//                other smem rows keep stale data: they feed accumulator rows
-//                that are never stored)
+//   warp 0       TMA producer: A box [AR x 64] (both planes of a split A in one
+//                3D copy) + the B box(es) [256 x 64] per stage
 //   warp 1       TMEM allocator; lane 0 issues tcgen05.mma (M=128, N=256, K=16)
 //   warps 2..5   epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane per
 //                row), activation or gate, masked stores
@@ -43,7 +40,6 @@ constexpr int BK = 64;                   // bf16 per 128-byte smem row
 constexpr int MMA_N = 256;               // columns per MMA / accumulator
 constexpr int MAX_STAGES = 5;
 constexpr int A_BYTES = BM * BK * 2;     // 16 KB
-constexpr int A_SHORT = 16;              // rows per A box of a partly filled tile
 constexpr int B_HALF = 128 * BK * 2;     // 16 KB per B box
 constexpr int NUM_THREADS = 192;
 
@@ -163,7 +159,6 @@ template <int EPI, bool SPLIT, int AR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                         const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
-                        const __grid_constant__ CUtensorMap tmAs, const __grid_constant__ CUtensorMap tmAs2,
                         const Params p) {
   constexpr bool A_SPLIT = SPLIT && (EPI == EPI_GATE_F32 || EPI == EPI_GATE_SCATTER_BF16);
   constexpr bool OUT_SPLIT = SPLIT && (EPI == EPI_RELU_BF16 || EPI == EPI_SWIGLU_BF16);
@@ -188,8 +183,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (A_SPLIT) tma_prefetch_desc(&tmA2);
     tma_prefetch_desc(&tmB0);
     tma_prefetch_desc(&tmB1);
-    tma_prefetch_desc(&tmAs);
-    if (A_SPLIT) tma_prefetch_desc(&tmAs2);
   }
   if (warp == 1) tmem_alloc(&ctl->tmem_slot, TMEM_COLS);
   pdl_wait();  // tile offsets and the A rows come from the kernels before
@@ -218,28 +211,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int row0 = ctl->offsets[e] + mt * BM;
         const int brow = e * p.N + nt * p.bn;
         const int kb0 = w.kb0, kb1 = w.kb1;
-        // rows of the group in this tile (>= 1); 0 short boxes = one full box.
-        // Short boxes only for a single-plane A: with the hi + lo planes the
-        // extra copies cost more than the rows they save.
-        const int vrows = ctl->offsets[e + 1] - row0;
-        const int nshort = (A_SPLIT || vrows >= AR) ? 0 : (vrows + A_SHORT - 1) / A_SHORT;
-        const uint32_t a_bytes = nshort == 0 ? A_ST : nshort * A_SHORT * BK * 2;
-        const uint32_t tx = (A_SPLIT ? 2u : 1u) * a_bytes + 2u * B_HALF;
+        constexpr uint32_t tx = (A_SPLIT ? 2u : 1u) * A_ST + 2u * B_HALF;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_or_abort(ctl, &ctl->empty[stage], phase ^ 1u, p)) { ok = false; break; }
           uint8_t* sa = stages + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&ctl->full[stage], tx);
-          if (nshort == 0) {
-            if (A_SPLIT) tma_load_3d(sa, &tmA, &ctl->full[stage], kb * BK, row0, 0);  // hi and lo planes
-            else tma_load_2d(sa, &tmA, &ctl->full[stage], kb * BK, row0);
-          } else {
-            for (int j = 0; j < nshort; ++j) {
-              tma_load_2d(sa + j * A_SHORT * BK * 2, &tmAs, &ctl->full[stage], kb * BK, row0 + j * A_SHORT);
-              if (A_SPLIT)
-                tma_load_2d(sa + A_ST + j * A_SHORT * BK * 2, &tmAs2, &ctl->full[stage], kb * BK,
-                            row0 + j * A_SHORT);
-            }
-          }
+          if (A_SPLIT) tma_load_3d(sa, &tmA, &ctl->full[stage], kb * BK, row0, 0);  // hi and lo planes
+          else tma_load_2d(sa, &tmA, &ctl->full[stage], kb * BK, row0);
           if (EPI == EPI_SWIGLU_BF16) {
             tma_load_2d(sa + B_OFF, &tmB0, &ctl->full[stage], kb * BK, brow);
             tma_load_2d(sa + B_OFF + B_HALF, &tmB1, &ctl->full[stage], kb * BK, brow);
@@ -502,7 +480,7 @@ cudaError_t launch_t(const TcGemmPlan& pl, int num_sms, cudaStream_t s) {
                                       static_cast<int>(bytes));
   if (e != cudaSuccess) return e;
   return launch_pdl(grouped_gemm_kernel<EPI, SPLIT, AR>, dim3(num_sms), dim3(NUM_THREADS), bytes, s, pl.a, pl.a2,
-                    pl.b0, pl.b1, pl.as, pl.as2, pl.p);
+                    pl.b0, pl.b1, pl.p);
 }
 
 template <int EPI, bool SPLIT>
@@ -535,8 +513,7 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
   const bool maps_ok =
       (a_split ? make_map_planes_bf16(&pl->a, g.A, static_cast<uint64_t>(plane_stride), a_rows, K, ar)
                : make_map_bf16(&pl->a, g.A, a_rows, K, ar)) &&
-      make_map(&pl->a2, a_split ? g.A2 : g.A, a_rows, K) && make_map_bf16(&pl->as, g.A, a_rows, K, A_SHORT) &&
-      make_map_bf16(&pl->as2, a_split ? g.A2 : g.A, a_rows, K, A_SHORT) &&
+      make_map(&pl->a2, a_split ? g.A2 : g.A, a_rows, K) &&
       // B: two 128-row boxes (W1 and W3) for SwiGLU, else one 256-row box
       make_map_bf16(&pl->b0, g.B0, b_rows, K, swiglu ? 128 : 256) &&
       make_map(&pl->b1, swiglu ? g.B1 : g.B0, b_rows, K);

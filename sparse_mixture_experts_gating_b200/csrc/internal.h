@@ -144,7 +144,6 @@ struct TcParams {
 // Everything a tensor-core GEMM launch needs, prepared on the host up front.
 struct TcGemmPlan {
   CUtensorMap a, a2, b0, b1;
-  CUtensorMap as, as2;  // A and A2 with 16-row boxes, for tiles whose group ends inside the tile
   TcParams p;
   int epi;
   int split;
