@@ -639,8 +639,14 @@ __global__ void __launch_bounds__(SCAN_T) route_small_kernel(RoutingArgs a, int 
     if (a.logits_in != nullptr) {
       h = a.logits_in[i];
     } else {
+      float pv[SMALL_DS_MAX];  // all chunk loads in flight, then the sum in chunk order
+#pragma unroll
+      for (int ds = 0; ds < SMALL_DS_MAX; ++ds)
+        pv[ds] = ds < n_ds ? partial[(static_cast<int64_t>(ds) * T + t) * E + e] : 0.f;
       h = 0.f;
-      for (int ds = 0; ds < n_ds; ++ds) h += partial[(static_cast<int64_t>(ds) * T + t) * E + e];
+#pragma unroll
+      for (int ds = 0; ds < SMALL_DS_MAX; ++ds)
+        if (ds < n_ds) h += pv[ds];
       if (a.b_r != nullptr) h += a.b_r[e];
     }
     if (h != h) h = -INFINITY;  // NaN logits (out of contract) rank last
@@ -781,94 +787,97 @@ __global__ void __launch_bounds__(SCAN_T) route_small_kernel(RoutingArgs a, int 
 
 // ---------------------------------------------------------------------------
 // Combine: y_t = sum over kept choices j (ascending) of the slot's row of Yp
-// (summed over its K-range partials in order).  A thread owns CU groups of 4
-// columns (grid-strided, so every load instruction of a warp is one run of
-// 512 bytes); the destinations and all CU * K row loads are issued before the
-// ordered sums, so each thread keeps 8 loads in flight.  Small batches use
-// CU = 1 (WIDE false) to spread over more blocks.
-template <typename YT, int K, bool WIDE>
-__global__ void __launch_bounds__(256) combine_kernel(int64_t T, int d, const int32_t* __restrict__ dest_row,
+// (summed over its K-range partials in order), then the shared experts' rows.
+// A block takes one token at a time (grid-stride over tokens) and the
+// columns [blockIdx.y * cpb, +cpb) of it (small batches split a row over
+// several blocks): the token's destination rows are block-wide constants, so
+// each thread only streams its groups of 4 columns (VU of them per pass, all
+// loads issued before the ordered sums).
+template <typename YT, int K, int VU>
+__global__ void __launch_bounds__(256, 4) combine_kernel(int64_t T, int d, const int32_t* __restrict__ dest_row,
                                                       int n_shared, const int32_t* __restrict__ shared_base,
                                                       const float* __restrict__ Yp, int ksplit, int64_t split_stride,
-                                                      YT* __restrict__ y, float* __restrict__ yf) {
-  constexpr int CU = (!WIDE || K >= 8) ? 1 : 8 / K;
+                                                      int cpb, YT* __restrict__ y, float* __restrict__ yf) {
   pdl_wait();
   pdl_trigger();
-  const uint32_t vpr = static_cast<uint32_t>(d) >> 2;  // float4 groups per row (d % 4 == 0 on this path)
-  const uint32_t n = static_cast<uint32_t>(T) * vpr;   // T * d / 4 < 2^32 (checked on the host)
-  const uint32_t stride = gridDim.x * 256u;
-  uint32_t tok[CU];
-  int v[CU], dst[CU][K];
+  const int vpr = d >> 2;  // float4 groups per row (d % 4 == 0 on this path)
+  const int c_end = min(vpr, static_cast<int>(blockIdx.y + 1) * cpb);
+  const float4* Y4 = reinterpret_cast<const float4*>(Yp);
+  const int64_t sb = n_shared > 0 ? *shared_base : 0;
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    int64_t base[K];  // first float4 of each kept choice's row (-1: dropped)
 #pragma unroll
-  for (int u = 0; u < CU; ++u) {
-    const uint32_t i = blockIdx.x * 256u + threadIdx.x + u * stride;
-    tok[u] = i < n ? i / vpr : 0xffffffffu;
-    v[u] = i < n ? static_cast<int>(i - tok[u] * vpr) : 0;
-#pragma unroll
-    for (int j = 0; j < K; ++j) dst[u][j] = i < n ? dest_row[static_cast<int64_t>(tok[u]) * K + j] : -1;
-  }
-  float4 acc[CU];
-  if (ksplit == 1) {
-    float4 r[CU][K];
-#pragma unroll
-    for (int u = 0; u < CU; ++u)
-#pragma unroll
-      for (int j = 0; j < K; ++j)
-        r[u][j] = dst[u][j] >= 0 ? reinterpret_cast<const float4*>(Yp + static_cast<int64_t>(dst[u][j]) * d)[v[u]]
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int u = 0; u < CU; ++u) {
-      acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int j = 0; j < K; ++j) {
-        acc[u].x += r[u][j].x; acc[u].y += r[u][j].y; acc[u].z += r[u][j].z; acc[u].w += r[u][j].w;
-      }
+    for (int j = 0; j < K; ++j) {
+      const int dst = dest_row[t * K + j];
+      base[j] = dst >= 0 ? static_cast<int64_t>(dst) * vpr : -1;
     }
-  } else {
+    for (int v0 = static_cast<int>(blockIdx.y) * cpb + threadIdx.x; v0 < c_end; v0 += 256 * VU) {
+      float4 acc[VU];
+      if (ksplit == 1) {
+        float4 r[VU][K];
 #pragma unroll
-    for (int u = 0; u < CU; ++u) {
-      acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < VU; ++u) {
+          const int v = v0 + u * 256;
 #pragma unroll
-      for (int j = 0; j < K; ++j) {
-        if (dst[u][j] < 0) continue;
-        float4 sj = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int ks = 0; ks < ksplit; ++ks) {
-          const float4 q = reinterpret_cast<const float4*>(Yp + static_cast<int64_t>(ks) * split_stride +
-                                                           static_cast<int64_t>(dst[u][j]) * d)[v[u]];
-          sj.x += q.x; sj.y += q.y; sj.z += q.z; sj.w += q.w;
+          for (int j = 0; j < K; ++j)
+            r[u][j] = (v < c_end && base[j] >= 0) ? Y4[base[j] + v] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        acc[u].x += sj.x; acc[u].y += sj.y; acc[u].z += sj.z; acc[u].w += sj.w;
-      }
-    }
-  }
-  if (n_shared > 0) {  // the shared experts' rows, after the routed sum, in order s
-    const int64_t sb = *shared_base;
-    for (int si = 0; si < n_shared; ++si) {
 #pragma unroll
-      for (int u = 0; u < CU; ++u) {
-        if (tok[u] == 0xffffffffu) continue;
-        const int64_t row = sb + static_cast<int64_t>(si) * T + tok[u];
-        float4 sj = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int ks = 0; ks < ksplit; ++ks) {
-          const float4 q = reinterpret_cast<const float4*>(Yp + static_cast<int64_t>(ks) * split_stride + row * d)[v[u]];
-          sj.x += q.x; sj.y += q.y; sj.z += q.z; sj.w += q.w;
+        for (int u = 0; u < VU; ++u) {
+          acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int j = 0; j < K; ++j) {
+            acc[u].x += r[u][j].x; acc[u].y += r[u][j].y; acc[u].z += r[u][j].z; acc[u].w += r[u][j].w;
+          }
         }
-        acc[u].x += sj.x; acc[u].y += sj.y; acc[u].z += sj.z; acc[u].w += sj.w;
-      }
-    }
-  }
+      } else {
 #pragma unroll
-  for (int u = 0; u < CU; ++u) {
-    if (tok[u] == 0xffffffffu) continue;
-    const int64_t t = tok[u];
-    if (yf != nullptr) reinterpret_cast<float4*>(yf + t * d)[v[u]] = acc[u];
-    if constexpr (sizeof(YT) == 2) {
-      uint2 o;
-      o.x = pack_bf16x2(acc[u].x, acc[u].y);
-      o.y = pack_bf16x2(acc[u].z, acc[u].w);
-      reinterpret_cast<uint2*>(y + t * d)[v[u]] = o;
-    } else {
-      reinterpret_cast<float4*>(y + t * d)[v[u]] = acc[u];
+        for (int u = 0; u < VU; ++u) {
+          const int v = v0 + u * 256;
+          acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int j = 0; j < K; ++j) {
+            if (v >= c_end || base[j] < 0) continue;
+            float4 sj = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+            for (int ks = 0; ks < ksplit; ++ks) {
+              const float4 q = Y4[ks * (split_stride >> 2) + base[j] + v];
+              sj.x += q.x; sj.y += q.y; sj.z += q.z; sj.w += q.w;
+            }
+            acc[u].x += sj.x; acc[u].y += sj.y; acc[u].z += sj.z; acc[u].w += sj.w;
+          }
+        }
+      }
+      // shared experts' rows (offsets[E] + s * T + t), after the routed sum, in order s
+      for (int si = 0; si < n_shared; ++si) {
+        const int64_t rb = (sb + static_cast<int64_t>(si) * T + t) * vpr;
+#pragma unroll
+        for (int u = 0; u < VU; ++u) {
+          const int v = v0 + u * 256;
+          if (v >= c_end) continue;
+          float4 sj = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+          for (int ks = 0; ks < ksplit; ++ks) {
+            const float4 q = Y4[ks * (split_stride >> 2) + rb + v];
+            sj.x += q.x; sj.y += q.y; sj.z += q.z; sj.w += q.w;
+          }
+          acc[u].x += sj.x; acc[u].y += sj.y; acc[u].z += sj.z; acc[u].w += sj.w;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < VU; ++u) {
+        const int v = v0 + u * 256;
+        if (v >= c_end) continue;
+        if (yf != nullptr) reinterpret_cast<float4*>(yf + t * d)[v] = acc[u];
+        if constexpr (sizeof(YT) == 2) {
+          uint2 o;
+          o.x = pack_bf16x2(acc[u].x, acc[u].y);
+          o.y = pack_bf16x2(acc[u].z, acc[u].w);
+          reinterpret_cast<uint2*>(y + t * d)[v] = o;
+        } else {
+          reinterpret_cast<float4*>(y + t * d)[v] = acc[u];
+        }
+      }
     }
   }
 }
@@ -977,20 +986,22 @@ template <int K>
 cudaError_t launch_combine_k(int64_t T, int d, int y_is_bf16, const int32_t* dest_row, int n_shared,
                              const int32_t* shared_base, const float* Yp, int ksplit, int64_t split_stride, void* y,
                              float* y_f32, cudaStream_t s) {
-  constexpr int CU = K >= 8 ? 1 : 8 / K;
-  const int64_t groups = T * (d / 4);
-  // wide threads only when the grid still covers every SM several times over
-  const bool wide = groups >= static_cast<int64_t>(256) * CU * 148 * 4;
-  const int cu = wide ? CU : 1;
-  const dim3 grid(static_cast<unsigned>((groups + 256 * cu - 1) / (256 * cu)));
-  if (y_is_bf16) {
-    auto kern = wide ? combine_kernel<__nv_bfloat16, K, true> : combine_kernel<__nv_bfloat16, K, false>;
-    return launch_pdl(kern, grid, dim3(256), 0, s, T, d, dest_row, n_shared, shared_base, Yp, ksplit, split_stride,
-                      static_cast<__nv_bfloat16*>(y), y_f32);
-  }
-  auto kern = wide ? combine_kernel<float, K, true> : combine_kernel<float, K, false>;
-  return launch_pdl(kern, grid, dim3(256), 0, s, T, d, dest_row, n_shared, shared_base, Yp, ksplit, split_stride,
-                    static_cast<float*>(y), y_f32);
+  constexpr int VU = K <= 4 ? 2 : 1;  // column groups per thread and pass
+  const int64_t blocks = T < 148 * 16 ? T : 148 * 16;
+  // few tokens: split each row's groups of 4 columns over up to yc blocks
+  // (about two blocks per SM in all, at least 256 groups per block)
+  const int vpr = d / 4;
+  int yc = static_cast<int>((2 * 148 + blocks - 1) / (blocks > 0 ? blocks : 1));
+  const int yc_max = (vpr + 255) / 256;
+  if (yc > yc_max) yc = yc_max;
+  if (yc < 1) yc = 1;
+  const int cpb = (vpr + yc - 1) / yc;
+  const dim3 grid(static_cast<unsigned>(blocks > 0 ? blocks : 1), static_cast<unsigned>(yc));
+  if (y_is_bf16)
+    return launch_pdl(combine_kernel<__nv_bfloat16, K, VU>, grid, dim3(256), 0, s, T, d, dest_row, n_shared,
+                      shared_base, Yp, ksplit, split_stride, cpb, static_cast<__nv_bfloat16*>(y), y_f32);
+  return launch_pdl(combine_kernel<float, K, VU>, grid, dim3(256), 0, s, T, d, dest_row, n_shared, shared_base, Yp,
+                    ksplit, split_stride, cpb, static_cast<float*>(y), y_f32);
 }
 }  // namespace
 
