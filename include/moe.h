@@ -213,7 +213,7 @@ MOE_API int moe_balance_losses(moe_handle h, int64_t T, const void* workspace, f
  * scratch is a 32 MiB array compiled into the library, resident on every GPU
  * that loads it until the process exits.
  *   - A call needing more than 32 MiB (moe_workspace_bytes(h, T) > 32 MiB;
- *     e.g. the 8-expert top-2 d 4096 / d_ff 14336 SwiGLU layer up to T = 200)
+ *     e.g. the 8-expert top-2 d 4096 / d_ff 14336 SwiGLU layer up to T = 116)
  *     is rejected with MOE_ERR_UNSUPPORTED before any launch.
  *   - The first call on a device looks up the array's address on that device
  *     (with it current); make that first call before any stream capture.

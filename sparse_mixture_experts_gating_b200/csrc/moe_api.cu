@@ -139,14 +139,14 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   w.ksplit = ksplit_of(L, w.s_max);
   // Yp holds ksplit partials of s_max rows; reserve the most any smaller batch
   // needs as well, so a workspace sized for some T serves every smaller batch.
-  // ksplit(s) depends on s through the m-tile bound floor(s / 128) + min(groups, s),
-  // which changes at every s below the group count and then only at multiples
-  // of 128, and ksplit(s) = 1 once s > 148 * 128; the product ksplit(s) * s
+  // ksplit(s) depends on s through the m-tile bound min(G, s) + floor((s - min(G, s)) / 128)
+  // (G groups), which changes at every s up to G and then every 128 rows, and
+  // ksplit(s) = 1 once the bound reaches 148 tiles; the product ksplit(s) * s
   // peaks at the last s before each change.
   int64_t yp_rows = w.ksplit * w.s_max;
   const int64_t groups = L.E + L.n_shared;
   for (int64_t s = 1; s < w.s_max && s <= groups; ++s) yp_rows = std::max<int64_t>(yp_rows, ksplit_of(L, s) * s);
-  for (int64_t s = 127; s < w.s_max && s <= 148 * 128; s += 128)
+  for (int64_t s = groups + 127; s < w.s_max && s <= groups + 148 * 128; s += 128)
     yp_rows = std::max<int64_t>(yp_rows, ksplit_of(L, s) * s);
   w.Yp = take(w.need_yp ? sizeof(float) * static_cast<size_t>(yp_rows) * L.d : 0);
   w.total = o;
@@ -164,16 +164,27 @@ void record(const moe_debug* dbg, int stage, int which, cudaStream_t s) {
 void set_error_message(const char* msg) { t_err = msg; }
 
 int gemm2_ksplit(int64_t s_max, int E, int d, int d_ff) {
-  // most m-tiles the second projection can have: floor(S/128) full ones plus
-  // one partial per expert that holds rows
-  const int64_t mtiles = s_max / kTileM + std::min<int64_t>(E, s_max);
+  // Most m-tiles the second projection can have: a group of c rows takes
+  // 1 + floor((c - 1) / 128) tiles, so S rows over at most min(E, S) groups
+  // take at most min(E, S) + floor((S - min(E, S)) / 128).
+  const int64_t g = std::min<int64_t>(E, s_max);
+  const int64_t mtiles = g + (s_max - g) / kTileM;
   const int64_t base = mtiles * ((d + 255) / 256);
-  if (base <= 0 || base * 2 > kSplitTargetCtas) return 1;
+  if (base <= 0 || base >= kSplitTargetCtas) return 1;
+  // Fewer tiles than SMs: cut K into ranges so that every SM streams weights.
+  // Each persistent CTA takes every num_sms-th (tile, range) unit, so the
+  // longest CTA runs ceil(units / num_sms) ranges of `per` k-blocks; take the
+  // cut that shortens it, a cut with more ranges only when it saves over 3 %
+  // (each range adds an fp32 partial of the tile's rows).
   const int64_t num_kb = (d_ff + 63) / 64;
-  const int64_t ks = std::min<int64_t>(kSplitTargetCtas / base, num_kb / 4);
-  if (ks <= 1) return 1;
-  const int64_t per = (num_kb + ks - 1) / ks;  // no empty K range
-  return static_cast<int>((num_kb + per - 1) / per);
+  int64_t best = 1, best_len = num_kb;
+  for (int64_t ks = 2; ks <= num_kb / 4; ++ks) {
+    const int64_t per = (num_kb + ks - 1) / ks;
+    const int64_t ranges = (num_kb + per - 1) / per;  // no empty K range
+    const int64_t len = (base * ranges + kSplitTargetCtas - 1) / kSplitTargetCtas * per;
+    if (len * 32 < best_len * 31) { best = ranges; best_len = len; }
+  }
+  return static_cast<int>(best);
 }
 
 cudaError_t set_smem_limit_once(const void* kernel, int bytes) {

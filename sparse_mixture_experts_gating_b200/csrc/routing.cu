@@ -830,23 +830,44 @@ __global__ void __launch_bounds__(256, 4) combine_kernel(int64_t T, int d, const
             acc[u].x += r[u][j].x; acc[u].y += r[u][j].y; acc[u].z += r[u][j].z; acc[u].w += r[u][j].w;
           }
         }
-      } else {
+      } else if constexpr (VU == 1) {  // (the host launches K-range partials with VU = 1)
+        // K-range partials: each choice's ranges summed in order, then the
+        // choices in order.  Up to three choices: KU ranges of every choice
+        // in flight at a time; more: one choice at a time, four ranges.
+        constexpr int KC = K <= 3 ? K : 1;       // choices loaded together
+        constexpr int KU = K <= 3 ? 8 / K : 4;   // ranges loaded together
+        const int64_t ss4 = split_stride >> 2;
+        acc[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (v0 < c_end) {
 #pragma unroll
-        for (int u = 0; u < VU; ++u) {
-          const int v = v0 + u * 256;
-          acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int j0 = 0; j0 < K; j0 += KC) {
+            float4 sj[KC];
 #pragma unroll
-          for (int j = 0; j < K; ++j) {
-            if (v >= c_end || base[j] < 0) continue;
-            float4 sj = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-            for (int ks = 0; ks < ksplit; ++ks) {
-              const float4 q = Y4[ks * (split_stride >> 2) + base[j] + v];
-              sj.x += q.x; sj.y += q.y; sj.z += q.z; sj.w += q.w;
+            for (int j = 0; j < KC; ++j) sj[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int ks0 = 0; ks0 < ksplit; ks0 += KU) {
+              float4 q[KU][KC];
+#pragma unroll
+              for (int i = 0; i < KU; ++i)
+#pragma unroll
+                for (int j = 0; j < KC; ++j)
+                  q[i][j] = (ks0 + i < ksplit && base[j0 + j] >= 0) ? Y4[(ks0 + i) * ss4 + base[j0 + j] + v0]
+                                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+              for (int i = 0; i < KU; ++i)
+#pragma unroll
+                for (int j = 0; j < KC; ++j) {
+                  sj[j].x += q[i][j].x; sj[j].y += q[i][j].y; sj[j].z += q[i][j].z; sj[j].w += q[i][j].w;
+                }
             }
-            acc[u].x += sj.x; acc[u].y += sj.y; acc[u].z += sj.z; acc[u].w += sj.w;
+#pragma unroll
+            for (int j = 0; j < KC; ++j) {
+              acc[0].x += sj[j].x; acc[0].y += sj[j].y; acc[0].z += sj[j].z; acc[0].w += sj[j].w;
+            }
           }
         }
+      } else {
+#pragma unroll
+        for (int u = 0; u < VU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
       // shared experts' rows (offsets[E] + s * T + t), after the routed sum, in order s
       for (int si = 0; si < n_shared; ++si) {
@@ -986,7 +1007,6 @@ template <int K>
 cudaError_t launch_combine_k(int64_t T, int d, int y_is_bf16, const int32_t* dest_row, int n_shared,
                              const int32_t* shared_base, const float* Yp, int ksplit, int64_t split_stride, void* y,
                              float* y_f32, cudaStream_t s) {
-  constexpr int VU = K <= 4 ? 2 : 1;  // column groups per thread and pass
   const int64_t blocks = T < 148 * 16 ? T : 148 * 16;
   // few tokens: split each row's groups of 4 columns over up to yc blocks
   // (about two blocks per SM in all, at least 256 groups per block)
@@ -997,10 +1017,19 @@ cudaError_t launch_combine_k(int64_t T, int d, int y_is_bf16, const int32_t* des
   if (yc < 1) yc = 1;
   const int cpb = (vpr + yc - 1) / yc;
   const dim3 grid(static_cast<unsigned>(blocks > 0 ? blocks : 1), static_cast<unsigned>(yc));
+  // column groups per thread and pass: two for up to four choices, one where
+  // the loads of K-range partials take the registers
+  if (ksplit > 1 || K > 4) {
+    if (y_is_bf16)
+      return launch_pdl(combine_kernel<__nv_bfloat16, K, 1>, grid, dim3(256), 0, s, T, d, dest_row, n_shared,
+                        shared_base, Yp, ksplit, split_stride, cpb, static_cast<__nv_bfloat16*>(y), y_f32);
+    return launch_pdl(combine_kernel<float, K, 1>, grid, dim3(256), 0, s, T, d, dest_row, n_shared, shared_base,
+                      Yp, ksplit, split_stride, cpb, static_cast<float*>(y), y_f32);
+  }
   if (y_is_bf16)
-    return launch_pdl(combine_kernel<__nv_bfloat16, K, VU>, grid, dim3(256), 0, s, T, d, dest_row, n_shared,
+    return launch_pdl(combine_kernel<__nv_bfloat16, K, 2>, grid, dim3(256), 0, s, T, d, dest_row, n_shared,
                       shared_base, Yp, ksplit, split_stride, cpb, static_cast<__nv_bfloat16*>(y), y_f32);
-  return launch_pdl(combine_kernel<float, K, VU>, grid, dim3(256), 0, s, T, d, dest_row, n_shared, shared_base, Yp,
+  return launch_pdl(combine_kernel<float, K, 2>, grid, dim3(256), 0, s, T, d, dest_row, n_shared, shared_base, Yp,
                     ksplit, split_stride, cpb, static_cast<float*>(y), y_f32);
 }
 }  // namespace

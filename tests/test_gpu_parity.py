@@ -42,12 +42,12 @@ SMALL = [
     ("long_k_ragged", 333, 1032, 4, 2, 1160, S, RN, 0.0, BF, None),
     ("decode_splitk", 3, 256, 8, 2, 1024, S, RN, 0.0, BF, None),          # K ranges of GEMM2 split
     ("decode_splitk_ragged", 5, 136, 4, 2, 1160, R, SW, 0.0, BF, "normal"),
-    # grouped-GEMM stream-K tail: 1 < tiles / 148 < 2 (two pieces per tile) ...
-    ("stream_k_tail_relu", 600, 256, 8, 2, 4096, R, RN, 0.0, BF, None),
-    # ... and few tiles over long K (up to 6-7 pieces per tile), k = 1 scatter epilogue, SwiGLU
-    ("stream_k_switch_pieces", 700, 512, 16, 1, 1024, R, SW, 1.25, BF, "normal"),
-    ("stream_k_long_k", 2, 2048, 4, 1, 256, R, RN, 0.0, BF, None),
-    ("stream_k_swiglu_pieces", 4, 1536, 8, 2, 384, S, RN, 0.0, BF, None),
+    # grouped-GEMM wave tail: 1 < tiles / 148 < 2 ...
+    ("wave_tail_relu", 600, 256, 8, 2, 4096, R, RN, 0.0, BF, None),
+    # ... and few tiles over long K (K-range partials), k = 1 scatter epilogue, SwiGLU
+    ("few_tiles_switch", 700, 512, 16, 1, 1024, R, SW, 1.25, BF, "normal"),
+    ("few_tiles_long_k", 2, 2048, 4, 1, 256, R, RN, 0.0, BF, None),
+    ("few_tiles_swiglu", 4, 1536, 8, 2, 384, S, RN, 0.0, BF, None),
     # shared experts (last field: n_shared): k = 2; k = 1 Switch with drops (the
     # combine path, dropped tokens keep the shared output); fp32; a small batch
     # whose second projection is split into K-range partials
@@ -58,6 +58,8 @@ SMALL = [
     # 33 <= T <= 64: pipeline stages hold 64 rows of A (T <= 32: 32 rows)
     ("ar64_swiglu", 48, 256, 8, 2, 512, S, RN, 0.0, BF, None),
     ("ar64_switch_shared", 61, 192, 4, 1, 384, R, SW, 1.0, BF, "normal", 1),
+    # T <= 32 routes in two launches; here with fp32 rows (CUDA-core GEMMs), drops and a shared expert
+    ("small_batch_fp32", 20, 40, 6, 2, 48, S, RN, 1.0, F32, "normal", 1),
 ]
 
 
@@ -83,8 +85,8 @@ def test_small_layers_match_oracle(case):
 
 
 SINGLE = [c for c in SMALL if c[9] == BF and c[0] in ("swiglu_e8_k2", "switch_relu_drops", "k4_zipf_tails",
-                                                       "e128_k8_cap", "long_k_ragged", "stream_k_tail_relu",
-                                                       "stream_k_switch_pieces", "shared_switch_k1_drops",
+                                                       "e128_k8_cap", "long_k_ragged", "wave_tail_relu",
+                                                       "few_tiles_switch", "shared_switch_k1_drops",
                                                        "one_token", "ar64_swiglu")]
 
 
