@@ -76,11 +76,19 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // The second projection writes fp32 rows for the combine (k > 1, shared
 // experts, or fp32 layers) instead of scattering bf16 rows straight into y.
+// (A k = 1 layer keeps the scatter: splitting its K range would add a combine
+// pass over y that costs more than the split saves.)
+// The second projection splits its K range for at most this many tiles.
+constexpr int kSplitMaxTiles = 4 * kSplitTargetCtas;
+
 bool need_yp_of(const moe_layer& L) { return !(L.dtype == MOE_BF16 && L.k == 1 && L.n_shared == 0); }
 
 int ksplit_of(const moe_layer& L, int64_t s_max) {
   return (L.dtype == MOE_BF16 && need_yp_of(L)) ? gemm2_ksplit(s_max, L.E + L.n_shared, L.d, L.d_ff) : 1;
 }
+
+// Yp rows a batch of s rows needs (0: none, the bf16 rows go straight into y).
+int64_t yp_rows_of(const moe_layer& L, int64_t s) { return need_yp_of(L) ? ksplit_of(L, s) * s : 0; }
 
 int64_t capacity_of(const moe_layer& L, int64_t T) {
   if (!(L.capacity_factor > 0.0)) return -1;
@@ -110,7 +118,6 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   w.s_max += static_cast<int64_t>(L.n_shared) * T;  // every token's rows of the shared experts
   w.nblk = static_cast<int>((T + kRouterTokens - 1) / kRouterTokens);
   const size_t elt = L.dtype == MOE_BF16 ? 2 : 4;
-  w.need_yp = need_yp_of(L);
   w.split = L.dtype == MOE_BF16 && L.hidden == MOE_HIDDEN_BF16X2;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
@@ -137,18 +144,19 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   w.Hp = take(elt * static_cast<size_t>(w.s_max) * L.d_ff);
   w.Hp_lo = take(w.split ? elt * static_cast<size_t>(w.s_max) * L.d_ff : 0);
   w.ksplit = ksplit_of(L, w.s_max);
+  w.need_yp = need_yp_of(L);
   // Yp holds ksplit partials of s_max rows; reserve the most any smaller batch
   // needs as well, so a workspace sized for some T serves every smaller batch.
   // ksplit(s) depends on s through the m-tile bound min(G, s) + floor((s - min(G, s)) / 128)
   // (G groups), which changes at every s up to G and then every 128 rows, and
-  // ksplit(s) = 1 once the bound reaches 148 tiles; the product ksplit(s) * s
+  // ksplit(s) = 1 once the bound reaches kSplitMaxTiles; the product ksplit(s) * s
   // peaks at the last s before each change.
-  int64_t yp_rows = w.ksplit * w.s_max;
+  int64_t yp_rows = yp_rows_of(L, w.s_max);
   const int64_t groups = L.E + L.n_shared;
-  for (int64_t s = 1; s < w.s_max && s <= groups; ++s) yp_rows = std::max<int64_t>(yp_rows, ksplit_of(L, s) * s);
-  for (int64_t s = groups + 127; s < w.s_max && s <= groups + 148 * 128; s += 128)
-    yp_rows = std::max<int64_t>(yp_rows, ksplit_of(L, s) * s);
-  w.Yp = take(w.need_yp ? sizeof(float) * static_cast<size_t>(yp_rows) * L.d : 0);
+  for (int64_t s = 1; s < w.s_max && s <= groups; ++s) yp_rows = std::max<int64_t>(yp_rows, yp_rows_of(L, s));
+  for (int64_t s = groups + 127; s < w.s_max && s <= groups + int64_t{kSplitMaxTiles} * 128; s += 128)
+    yp_rows = std::max<int64_t>(yp_rows, yp_rows_of(L, s));
+  w.Yp = take(yp_rows > 0 ? sizeof(float) * static_cast<size_t>(yp_rows) * L.d : 0);
   w.total = o;
   return w;
 }
@@ -170,14 +178,14 @@ int gemm2_ksplit(int64_t s_max, int E, int d, int d_ff) {
   const int64_t g = std::min<int64_t>(E, s_max);
   const int64_t mtiles = g + (s_max - g) / kTileM;
   const int64_t base = mtiles * ((d + 255) / 256);
-  if (base <= 0 || base >= kSplitTargetCtas) return 1;
-  // Fewer tiles than SMs: cut K into ranges so that every SM streams weights.
-  // Each persistent CTA takes every num_sms-th (tile, range) unit, so the
-  // longest CTA runs ceil(units / num_sms) ranges of `per` k-blocks; take the
-  // cut that shortens it, a cut with more ranges only when it saves over 3 %
-  // (each range adds an fp32 partial of the tile's rows).
+  if (base <= 0 || base > kSplitMaxTiles) return 1;
+  // A few waves of tiles or less: cut K into ranges so that the last wave
+  // fills the SMs.  Each persistent CTA takes every num_sms-th (tile, range)
+  // unit, so the longest CTA runs ceil(units / num_sms) ranges of `per`
+  // k-blocks; take the cut that shortens it, a cut with more ranges only when
+  // it saves over 3 % (each range adds an fp32 partial of the tile's rows).
   const int64_t num_kb = (d_ff + 63) / 64;
-  int64_t best = 1, best_len = num_kb;
+  int64_t best = 1, best_len = (base + kSplitTargetCtas - 1) / kSplitTargetCtas * num_kb;
   for (int64_t ks = 2; ks <= num_kb / 4; ++ks) {
     const int64_t per = (num_kb + ks - 1) / ks;
     const int64_t ranges = (num_kb + per - 1) / per;  // no empty K range
