@@ -17,6 +17,7 @@
 #include "moe.h"
 #include "common.cuh"
 #include "internal.h"
+#include "scan_dispatch.h"
 
 struct moe_layer {
   int E, k, d, d_ff, act, gate_mode, dtype;
@@ -132,8 +133,9 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   w.part_lse2 = take(sizeof(float) * w.nblk);
   w.blockoff = take(sizeof(int32_t) * L.E * static_cast<size_t>(w.nblk));
   w.counts = take(sizeof(int32_t) * L.E);
-  w.offsets = take(sizeof(int32_t) * (L.E + 1));
-  w.mprefix = take(sizeof(int32_t) * (L.E + 1));
+  // [groups + 1]: the routed experts' groups, then one per shared expert
+  w.offsets = take(sizeof(int32_t) * (L.E + L.n_shared + 1));
+  w.mprefix = take(sizeof(int32_t) * (L.E + L.n_shared + 1));
   // scan totals [E] + [E], the scan ticket, the three balance statistics
   w.scal = take(sizeof(int32_t) * L.E + sizeof(float) * L.E + 64);
   const bool tc_router = L.dtype == MOE_BF16 && L.E <= kRouterTcMaxE;
@@ -438,12 +440,20 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
       return rc;
     }
     record(dbg, MOE_STAGE_ROUTER, 1, s);
-    record(dbg, MOE_STAGE_SCAN, 0, s);
-    if ((rc = check(launch_scan(r, s), "scan")) != MOE_OK) return rc;
-    record(dbg, MOE_STAGE_SCAN, 1, s);
-    record(dbg, MOE_STAGE_DISPATCH, 0, s);
-    if ((rc = check(launch_dispatch(r, s), "dispatch")) != MOE_OK) return rc;
-    record(dbg, MOE_STAGE_DISPATCH, 1, s);
+    if (scan_dispatch_fits(r)) {  // one launch (the scan stage of the debug events stays empty)
+      record(dbg, MOE_STAGE_SCAN, 0, s);
+      record(dbg, MOE_STAGE_SCAN, 1, s);
+      record(dbg, MOE_STAGE_DISPATCH, 0, s);
+      if ((rc = check(launch_scan_dispatch(r, s), "dispatch")) != MOE_OK) return rc;
+      record(dbg, MOE_STAGE_DISPATCH, 1, s);
+    } else {
+      record(dbg, MOE_STAGE_SCAN, 0, s);
+      if ((rc = check(launch_scan(r, s), "scan")) != MOE_OK) return rc;
+      record(dbg, MOE_STAGE_SCAN, 1, s);
+      record(dbg, MOE_STAGE_DISPATCH, 0, s);
+      if ((rc = check(launch_dispatch(r, s), "dispatch")) != MOE_OK) return rc;
+      record(dbg, MOE_STAGE_DISPATCH, 1, s);
+    }
   }
 
   record(dbg, MOE_STAGE_GEMM1, 0, s);

@@ -16,6 +16,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "scan_dispatch.h"
 
 namespace moe {
 namespace {
@@ -469,6 +470,30 @@ __global__ void __launch_bounds__(SCAN_T) scan_kernel(RoutingArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// One warp copies row `tok` of x to row `dest` of the expert-sorted buffer
+// (rows of 16-byte multiples: up to eight 16-byte loads in flight per lane).
+template <typename XT>
+__device__ __forceinline__ void copy_x_row(const XT* __restrict__ x, XT* __restrict__ Xp, int d, int64_t tok,
+                                           int64_t dest, int lane) {
+  if ((static_cast<size_t>(d) * sizeof(XT)) % 16 == 0) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + tok * d);
+    uint4* dst = reinterpret_cast<uint4*>(Xp + dest * d);
+    const int nv = static_cast<int>(static_cast<size_t>(d) * sizeof(XT) / 16);
+    for (int v0 = lane; v0 < nv; v0 += 256) {
+      uint4 c[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (v0 + 32 * q < nv) c[q] = src[v0 + 32 * q];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (v0 + 32 * q < nv) dst[v0 + 32 * q] = c[q];
+    }
+  } else {
+    for (int c = lane; c < d; c += 32) Xp[dest * d + c] = x[tok * d + c];
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Dispatch: one block per router block of BT tokens.  Warp 0 assigns the slot
 // rank of every (token, choice) of the block in token-major order (stable:
 // base = number of earlier assignments to the same expert in earlier blocks);
@@ -520,26 +545,7 @@ __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
   const XT* x = static_cast<const XT*>(a.x);
   XT* Xp = static_cast<XT*>(a.Xp);
   XT* yz = static_cast<XT*>(a.y_zero_dropped);
-  const bool vec = (static_cast<size_t>(d) * sizeof(XT)) % 16 == 0;
-  // one warp copies one row of x (token tok) to row `dest` of the sorted buffer
-  auto copy_row = [&](int64_t tok, int64_t dest) {
-    if (vec) {
-      const uint4* src = reinterpret_cast<const uint4*>(x + tok * d);
-      uint4* dst = reinterpret_cast<uint4*>(Xp + dest * d);
-      const int nv = static_cast<int>(static_cast<size_t>(d) * sizeof(XT) / 16);
-      for (int v0 = lane; v0 < nv; v0 += 256) {  // up to eight 16-byte loads in flight per lane
-        uint4 c[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (v0 + 32 * q < nv) c[q] = src[v0 + 32 * q];
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (v0 + 32 * q < nv) dst[v0 + 32 * q] = c[q];
-      }
-    } else {
-      for (int c = lane; c < d; c += 32) Xp[dest * d + c] = x[tok * d + c];
-    }
-  };
+  auto copy_row = [&](int64_t tok, int64_t dest) { copy_x_row(x, Xp, d, tok, dest, lane); };
   for (int ai = warp; ai < nA; ai += 8) {
     const int dest = dest_s[ai];
     const int64_t tok = t0 + ai / k;
@@ -563,6 +569,181 @@ __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
         a.row_gate[row] = 1.f;
       }
       copy_row(tok, row);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Scan and dispatch in one launch, for few experts times router blocks (each
+// warp loads at most kFusedLoads histogram entries per lane): block
+// (b, part) derives every expert's total and its prefix over the router
+// blocks before b itself (a warp per expert row, lanes over consecutive
+// blocks, four rows' loads in flight), takes the capacity-capped group sizes
+// and offsets the way scan_finalize does, ranks router block b's assignments
+// and copies its share of their rows (the warps of the gridDim.y parts stride
+// over them).  One more block, (nblk, 0), writes the scan's tables and
+// statistics (scan_finalize) alongside.  No per-block offsets table and no
+// second launch.
+constexpr int kFusedLoads = 16;  // (the Switch layer's 64 experts x 256 blocks, 64 loads per lane, ran no faster fused)
+constexpr int kFusedRows = 4;  // expert rows per batch of loads
+
+// Totals of kFusedRows expert rows e0, e0 + 8, ... (warp-uniform; rows past
+// E count zero) of a per-block table [E][nb], and their parts before block
+// blk: lanes over consecutive blocks, 256 blocks of every row per batch.
+template <typename V>
+__device__ __forceinline__ void rows_sums(const V* __restrict__ tab, int E, int nb, int e0, int blk, int lane,
+                                          V (&tot)[kFusedRows], V (&pre)[kFusedRows]) {
+#pragma unroll
+  for (int u = 0; u < kFusedRows; ++u) { tot[u] = V(0); pre[u] = V(0); }
+#pragma unroll 1
+  for (int c0 = 0; c0 < nb; c0 += 256) {
+    V v[kFusedRows][8];
+#pragma unroll
+    for (int u = 0; u < kFusedRows; ++u) {
+      const int e = e0 + 8 * u;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int b = c0 + 32 * j + lane;
+        v[u][j] = (e < E && b < nb) ? tab[static_cast<int64_t>(e) * nb + b] : V(0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kFusedRows; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        tot[u] += v[u][j];
+        if (c0 + 32 * j + lane < blk) pre[u] += v[u][j];
+      }
+  }
+}
+
+template <typename V>
+__device__ __forceinline__ V warp_total(V v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <typename XT>
+__global__ void __launch_bounds__(SCAN_T) scan_dispatch_kernel(RoutingArgs a) {
+  __shared__ int s_tot[256], s_pre[256], s_c1[256], s_off[257];
+  __shared__ float s_ps[256];
+  __shared__ int s_dest[BT * 8];
+  __shared__ int s_warp[2 * (SCAN_T / 32 + 1)];
+  __shared__ double s_red[6 * (SCAN_T / 32)];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int E = a.E, k = a.k, d = a.d, nb = a.nblk;
+  const int blk = blockIdx.x;
+  const bool stats = blk == nb;  // the block of the scan's tables and statistics
+  const int64_t t0 = static_cast<int64_t>(blk) * BT;
+  const int nt = stats ? 0 : static_cast<int>((a.T - t0) < BT ? (a.T - t0) : BT);
+  const int nA = nt * k;
+  pdl_wait();
+  pdl_trigger();
+  if (stats && blockIdx.y != 0) return;
+  // warp w: expert rows w + 8 i, kFusedRows of them per batch
+#pragma unroll 1
+  for (int e0 = warp; e0 < E; e0 += 8 * kFusedRows) {
+    int tot[kFusedRows], pre[kFusedRows];
+    rows_sums(a.part_hist, E, nb, e0, blk, lane, tot, pre);
+#pragma unroll
+    for (int u = 0; u < kFusedRows; ++u) {
+      const int t = warp_total(tot[u]), p = warp_total(pre[u]);
+      if (lane == 0 && e0 + 8 * u < E) { s_tot[e0 + 8 * u] = t; s_pre[e0 + 8 * u] = p; }
+    }
+    if (stats) {  // first-choice counts and probability sums for the statistics
+      int c1[kFusedRows], c1p[kFusedRows];
+      float ps[kFusedRows], psp[kFusedRows];
+      rows_sums(a.part_cnt1, E, nb, e0, 0, lane, c1, c1p);
+      rows_sums(a.part_psum, E, nb, e0, 0, lane, ps, psp);
+#pragma unroll
+      for (int u = 0; u < kFusedRows; ++u) {
+        const int c = warp_total(c1[u]);
+        const float q = warp_total(ps[u]);
+        if (lane == 0 && e0 + 8 * u < E) { s_c1[e0 + 8 * u] = c; s_ps[e0 + 8 * u] = q; }
+      }
+    }
+  }
+  __syncthreads();
+  if (stats) {
+    scan_finalize(a, tid < E ? s_tot[tid] : 0, tid < E ? s_c1[tid] : 0, tid < E ? s_ps[tid] : 0.f, s_warp, s_red);
+    return;
+  }
+  {  // group offsets, as scan_finalize computes them
+    const int groups = E + a.n_shared;
+    int kept = 0;
+    if (tid < E)
+      kept = (a.capacity < 0) ? s_tot[tid]
+                              : static_cast<int>((int64_t)s_tot[tid] < a.capacity ? (int64_t)s_tot[tid] : a.capacity);
+    else if (tid < groups)
+      kept = static_cast<int>(a.T);
+    int off, mp, total_rows, total_tiles;
+    block_exscan_int2(kept, (kept + kTileM - 1) / kTileM, s_warp, off, mp, total_rows, total_tiles);
+    if (tid < groups) s_off[tid] = off;
+    if (tid == 0) s_off[groups] = total_rows;
+  }
+  __syncthreads();
+  const bool writer = blockIdx.y == 0;  // one part writes the block's routing tables
+  if (warp == 0) {
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int a0 = 0; a0 < nA; a0 += 32) {
+      const int ai = a0 + lane;
+      const bool valid = ai < nA;
+      int e = valid ? a.topk_idx[t0 * k + ai] : -1;
+      if (e < 0 || e >= E) e = -1;  // never produced by the router; keeps smem indexing in range
+      const uint32_t peers = __match_any_sync(0xffffffffu, e);
+      const bool ok = valid && e >= 0;
+      const int base = ok ? s_pre[e] : 0;
+      const int rank = base + __popc(peers & lt);
+      __syncwarp();
+      if (ok && lane == __ffs(peers) - 1) s_pre[e] = base + __popc(peers);
+      __syncwarp();
+      if (valid && !ok) {
+        s_dest[ai] = -1;
+        if (writer) a.dest_row[t0 * k + ai] = -1;
+      } else if (valid) {
+        const bool kept = a.capacity < 0 || rank < a.capacity;
+        const int dest = kept ? s_off[e] + rank : -1;
+        s_dest[ai] = dest;
+        if (writer) {
+          a.dest_row[t0 * k + ai] = dest;
+          if (a.drop_mask != nullptr) a.drop_mask[t0 * k + ai] = kept ? 0 : 1;
+          if (kept) {
+            a.row_token[dest] = static_cast<int32_t>(t0 + ai / k);
+            a.row_gate[dest] = a.topk_gate[t0 * k + ai];
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const XT* x = static_cast<const XT*>(a.x);
+  XT* Xp = static_cast<XT*>(a.Xp);
+  XT* yz = static_cast<XT*>(a.y_zero_dropped);
+  const int gw = static_cast<int>(blockIdx.y) * (SCAN_T / 32) + warp, nw = static_cast<int>(gridDim.y) * (SCAN_T / 32);
+  for (int ai = gw; ai < nA; ai += nw) {
+    const int dest = s_dest[ai];
+    const int64_t tok = t0 + ai / k;
+    if (dest >= 0) {
+      copy_x_row(x, Xp, d, tok, dest, lane);
+    } else if (yz != nullptr) {  // k == 1: a dropped token's output row is zero
+      for (int c = lane; c < d; c += 32) yz[tok * d + c] = XT(0.f);
+      if (a.yf_zero_dropped != nullptr)
+        for (int c = lane; c < d; c += 32) a.yf_zero_dropped[tok * d + c] = 0.f;
+    }
+  }
+  // shared experts: every token of the block, gate 1, rows offsets[E] + s * T + t
+  if (a.n_shared > 0) {
+    const int64_t base = s_off[E];
+    for (int q = gw; q < nt * a.n_shared; q += nw) {
+      const int si = q / nt;
+      const int64_t tok = t0 + (q - si * nt);
+      const int64_t row = base + si * a.T + tok;
+      if (lane == 0) {
+        a.row_token[row] = static_cast<int32_t>(tok);
+        a.row_gate[row] = 1.f;
+      }
+      copy_x_row(x, Xp, d, tok, row, lane);
     }
   }
 }
@@ -741,25 +922,7 @@ __global__ void __launch_bounds__(SCAN_T) route_small_kernel(RoutingArgs a, int 
   const XT* x = static_cast<const XT*>(a.x);
   XT* Xp = static_cast<XT*>(a.Xp);
   XT* yz = static_cast<XT*>(a.y_zero_dropped);
-  const bool vec = (static_cast<size_t>(d) * sizeof(XT)) % 16 == 0;
-  auto copy_row = [&](int64_t tok, int64_t dest) {
-    if (vec) {
-      const uint4* src = reinterpret_cast<const uint4*>(x + tok * d);
-      uint4* dst = reinterpret_cast<uint4*>(Xp + dest * d);
-      const int nv = static_cast<int>(static_cast<size_t>(d) * sizeof(XT) / 16);
-      for (int v0 = lane; v0 < nv; v0 += 256) {
-        uint4 c[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (v0 + 32 * q < nv) c[q] = src[v0 + 32 * q];
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (v0 + 32 * q < nv) dst[v0 + 32 * q] = c[q];
-      }
-    } else {
-      for (int c = lane; c < d; c += 32) Xp[dest * d + c] = x[tok * d + c];
-    }
-  };
+  auto copy_row = [&](int64_t tok, int64_t dest) { copy_x_row(x, Xp, d, tok, dest, lane); };
   for (int i = warp; i < nA; i += SCAN_T / 32) {
     const int64_t tok = i / k;
     if (s_dest[i] >= 0) {
@@ -995,6 +1158,22 @@ cudaError_t launch_route_small(const RoutingArgs& a, void* partials, cudaStream_
 cudaError_t launch_scan(const RoutingArgs& a, cudaStream_t s) {
   if (a.nblk <= kScanSingleBlocks) return launch_pdl(scan_kernel<true>, dim3(1), dim3(SCAN_T), 0, s, a);
   return launch_pdl(scan_kernel<false>, dim3(a.E), dim3(SCAN_T), 0, s, a);
+}
+
+bool scan_dispatch_fits(const RoutingArgs& a) {
+  // histogram loads per lane: ceil(E / 8) rows of ceil(nblk / 32) entries
+  const int64_t loads = static_cast<int64_t>((a.E + 7) / 8) * ((a.nblk + 31) / 32);
+  return a.E <= 256 && loads <= kFusedLoads;
+}
+
+cudaError_t launch_scan_dispatch(const RoutingArgs& a, cudaStream_t s) {
+  // few router blocks: split each block's rows over up to 8 parts (about two
+  // blocks per SM in all)
+  int parts = (2 * 148) / (a.nblk > 0 ? a.nblk : 1);
+  parts = parts < 1 ? 1 : (parts > 8 ? 8 : parts);
+  const dim3 grid(static_cast<unsigned>(a.nblk + 1), static_cast<unsigned>(parts));  // + the statistics block
+  if (a.x_is_bf16) return launch_pdl(scan_dispatch_kernel<__nv_bfloat16>, grid, dim3(SCAN_T), 0, s, a);
+  return launch_pdl(scan_dispatch_kernel<float>, grid, dim3(SCAN_T), 0, s, a);
 }
 
 cudaError_t launch_dispatch(const RoutingArgs& a, cudaStream_t s) {

@@ -60,6 +60,12 @@ SMALL = [
     ("ar64_switch_shared", 61, 192, 4, 1, 384, R, SW, 1.0, BF, "normal", 1),
     # T <= 32 routes in two launches; here with fp32 rows (CUDA-core GEMMs), drops and a shared expert
     ("small_batch_fp32", 20, 40, 6, 2, 48, S, RN, 1.0, F32, "normal", 1),
+    # 256 groups: 255 routed experts and one shared expert
+    ("e255_shared", 300, 64, 255, 2, 64, R, RN, 0.0, BF, None, 1),
+    # 66 router blocks x 256 experts: too many histogram entries for the fused
+    # scan and dispatch, so the scan runs as its own launch (one block per
+    # expert); the other cases above route in the fused launch
+    ("e256_separate_scan", 2100, 64, 256, 1, 64, R, SW, 1.0, BF, "normal"),
 ]
 
 
