@@ -52,18 +52,20 @@ ACT_RELU, ACT_SWIGLU = 0, 1
 GATE_SWITCH, GATE_RENORM = 0, 1
 
 
-def router_logits(x, W_r, b_r=None) -> np.ndarray:
+def router_logits(x, W_r, b_r=None, dtype=np.float32) -> np.ndarray:
     """Router logits h = W_r x (+ b) per token, as fp32.
 
     "Replacing the feed-forward block": the router is one linear layer with E
     rows.  Accumulated in float64 and rounded once to float32 ("compute the
     router in float32", section "Implementation").
     x: [T][d], W_r: [E][d], b_r: [E] or None.  Returns float32 [T][E].
+    dtype=np.float64 skips the rounding (for finite-difference checks, whose
+    steps are far below float32 resolution).
     """
     h = np.asarray(x, np.float64) @ np.asarray(W_r, np.float64).T
     if b_r is not None:
         h = h + np.asarray(b_r, np.float64)[None, :]
-    return h.astype(np.float32)
+    return h.astype(dtype)
 
 
 def softmax_lse(h32: np.ndarray):
@@ -251,7 +253,7 @@ def balance_losses(p: np.ndarray, idx: np.ndarray, E: int) -> dict:
 def moe_forward(x, W_r, b_r, W1, W3, W2, *, k: int, gate_mode: int, act: int,
                 capacity_factor: float, rows: Optional[Sequence[int]] = None,
                 logits: Optional[np.ndarray] = None, hidden_bf16: bool = False,
-                shared: Optional[tuple] = None) -> dict:
+                shared: Optional[tuple] = None, logits_dtype=np.float32) -> dict:
     """The whole layer: routing for every token, y for every token or for ``rows``.
 
     x: [T][d]; W_r: [E][d]; b_r: [E] or None; W1, W3: [E][d_ff][d] (W3 None for
@@ -260,6 +262,7 @@ def moe_forward(x, W_r, b_r, W1, W3, W2, *, k: int, gate_mode: int, act: int,
     ``rows``: compute y only for these tokens (routing, capacity and losses are
     always global; y_t depends on x_t and the global routing only).
     ``hidden_bf16``: round each expert's hidden activation to bf16 (see expert_ffn).
+    ``logits_dtype``: np.float64 keeps the logits unrounded (finite differences).
     ``shared``: (W1s, W3s, W2s), each with n_s experts shaped like W1, W3, W2:
     shared experts that every token visits ("Mixture of experts", section
     "Total versus active parameters": "shared experts every token visits").
@@ -276,7 +279,7 @@ def moe_forward(x, W_r, b_r, W1, W3, W2, *, k: int, gate_mode: int, act: int,
     x = np.asarray(x)
     T = x.shape[0]
     E = np.asarray(W_r).shape[0]
-    h32 = router_logits(x, W_r, b_r) if logits is None else np.asarray(logits, np.float32)
+    h32 = router_logits(x, W_r, b_r, logits_dtype) if logits is None else np.asarray(logits, logits_dtype)
     p, lse = softmax_lse(h32)
     idx = top_k(h32, k)
     g = gates(h32, p, idx, gate_mode)

@@ -72,16 +72,16 @@ def _slots_choice_major(idx, E, C):
     return s
 
 
-def _logits_transposed_router(x, W_r, b_r=None):
+def _logits_transposed_router(x, W_r, b_r=None, dtype=np.float32):
     W = np.asarray(W_r, np.float64)
     h = np.asarray(x, np.float64) @ (W.T if W.shape[0] != W.shape[1] else W)
     if b_r is not None:
         h = h + b_r
-    return h.astype(np.float32)
+    return h.astype(dtype)
 
 
-def _logits_dropped_bias(x, W_r, b_r=None):
-    return _orig["router_logits"](x, W_r, None)
+def _logits_dropped_bias(x, W_r, b_r=None, dtype=np.float32):
+    return _orig["router_logits"](x, W_r, None, dtype)
 
 
 def _balance_sample_std(p, idx, E):
