@@ -8,4 +8,3 @@ from .moe_oracle import (  # noqa: F401
     aux_and_z, assign_slots, balance_losses, expert_capacity, expert_ffn, gates, moe_forward,
     round_to_bf16, router_logits, softmax_lse, top_k,
 )
-from .moe_backward import moe_backward  # noqa: F401,E402
