@@ -7,6 +7,10 @@ grouped GEMMs, combine, losses) over one batch of the workload's synthetic
 input, resident in HBM.  L2 is flushed between steps, outside the timed
 events: a 256 MiB write, then a 256 MiB read of another buffer.  Prints ONE JSON line on rank 0.
 
+--backward times a training step instead (the forward pass, then the
+backward pass of <dy, y> + 0.01 aux + 1e-3 z) on one GPU, with the
+backward's fp32 CUDA-core roofline.
+
 N > 1 (torchrun): every rank runs an independent replica of the layer on its
 own batch (the layer has no cross-batch exchange), so scaling is weak; the
 time is the max over ranks of each rank's device-timed total.
@@ -268,6 +272,8 @@ def main():
                     help="how the expert hidden activation is held (bf16 layers)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's token count (small cases for profiler captures)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time a training step instead: the forward pass, then the backward pass")
     args = ap.parse_args()
 
     import torch
@@ -295,6 +301,8 @@ def main():
     dev = torch.device("cuda", local)
 
     inp = make_inputs(w, device=dev)
+    if args.backward:
+        return backward_bench(args, w, inp, warmup, world, rank, local, dev)
     if rank > 0:
         inp["x"] = make_inputs(w.with_(seed=rank_seed(w.seed, rank)), device=dev, weights=False)["x"]
     layer = MoELayer(w.E, w.k, w.d, w.d_ff, act=w.act, gate_mode=w.gate, capacity_factor=w.capacity_factor,
@@ -450,6 +458,105 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def backward_flops(w, S, T):
+    """FP32 FLOPs of the backward pass for S kept rows (shared rows included):
+    per row and d x d_ff contraction 2 d d_ff; ReLU runs 5 of them (w1 x again,
+    W2^T dy, dXp, dW2, dW1), SwiGLU 8 (w1 x, w3 x, W2^T dy, two for dXp, dW2,
+    dW1, dW3); the router 3 T E d contractions (logits again, W_r^T dh, dW_r)."""
+    n = 8 if w.act == 1 else 5
+    return 2.0 * S * w.d * w.d_ff * n + 3 * 2.0 * T * w.E * w.d
+
+
+def backward_bench(args, w, inp, warmup, world, rank, local, dev):
+    """Training step = forward + backward (gradients of <dy, y> + 0.01 aux +
+    1e-3 z), inputs resident, L2 flushed before each step outside the events."""
+    import torch
+    from sparse_mixture_experts_gating_b200 import MoELayer, launch_count, status
+    from sparse_mixture_experts_gating_b200.workloads import torch_dtype
+    if world > 1 or rank > 0:
+        raise SystemExit("--backward runs on one GPU")
+    layer = MoELayer(w.E, w.k, w.d, w.d_ff, act=w.act, gate_mode=w.gate, capacity_factor=w.capacity_factor,
+                     dtype=torch_dtype(w.dtype), hidden=args.hidden, n_shared=w.n_shared)
+    ws = layer.workspace(w.T, dev)
+    gen = torch.Generator().manual_seed(w.seed + 17)
+    dy = torch.randn(w.T, w.d, generator=gen).to(inp["x"].dtype).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_rd = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
+
+    def flush_l2():  # as in the forward bench: a write, then a read of another buffer, both larger than L2
+        flush.zero_()
+        flush_rd.sum()
+    fw = (inp["x"], inp["W_r"], inp["b_r"], inp["W1"], inp["W3"], inp["W2"])
+    grads = None
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        nonlocal grads
+        y, counts, *_ = layer(*fw, workspace=ws)
+        if ev is not None:
+            ev.record(stream)
+        grads = layer.backward(*fw, dy, aux_coef=0.01, z_coef=1e-3, workspace=ws, grads=grads)
+        return counts
+
+    for _ in range(warmup):
+        flush_l2()
+        step()
+    status()
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    sampler = ClockSampler(vis.split(",")[local].strip() if vis else str(local))
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    n0 = launch_count()
+    wall0 = time.time()
+    gpu_hold(torch, 2.0 + 2.0 * K)
+    for i in range(K):
+        flush_l2()
+        evs[i][0].record(stream)
+        counts = step(evs[i][1])
+        evs[i][2].record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    n_launch = launch_count() - n0
+    time.sleep(0.15)
+    sampler.stop()
+    status()
+    step_s = sum(e[0].elapsed_time(e[2]) for e in evs) / 1e3
+    bw_s = sum(e[1].elapsed_time(e[2]) for e in evs) / 1e3
+    cap = layer.capacity(w.T)
+    kept = sum(c if cap is None else min(c, cap) for c in counts.cpu().tolist())
+    S = kept + w.n_shared * w.T
+    fl = backward_flops(w, S, w.T)
+    clocks = sampler.summary(wall0, wall1)
+    peak = 148 * 128 * 2 * (clocks["sm_max_mhz"] or 1965.0) * 1e6 / 1e12  # fp32 FMA lanes x 2 x max clock
+    ach = fl / (bw_s / K) / 1e12
+    line = {
+        "metric": "MoE-layer training step (forward + backward) tokens/s on 1 B200",
+        "value": round(w.T * K / step_s, 1),
+        "unit": "tokens/s",
+        "n_gpus": 1,
+        "steps": K,
+        "warmup": warmup,
+        "ms_per_step": round(step_s / K * 1e3, 5),
+        "backward_ms": round(bw_s / K * 1e3, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32 (backward), " + ("bf16" if w.dtype == 1 else "f32") + " (forward)",
+        "data": "synthetic (seeded; shapes and distributions of the workload, random-init weights)",
+        "config": dict(config_of(w, 1), hidden=args.hidden, loss="<dy, y> + 0.01 aux + 1e-3 z"),
+        "roofline": {"bound": "alu", "achieved": round(ach, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+                     "frac": round(ach / peak, 4), "kernel": "backward pass (fp32 CUDA-core GEMMs)",
+                     "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x clocks.max.sm", "traffic": None},
+        "gpu_launches": int(n_launch),
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
     return 0
 
 

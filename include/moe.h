@@ -228,6 +228,36 @@ MOE_API int moe_forward_static(moe_handle h, int64_t T, const void* x, const flo
                                void* stream);
 
 /*
+ * Backward pass ("Mixture of experts", rayaq.ca: section "Replacing the
+ * feed-forward block", the router learns through the gate values only, the
+ * choice of experts being discrete; section "The load-balancing loss", f_i
+ * is a count without gradient, P_i and the z-loss's lse have one).
+ *
+ * Gradients of L = sum_t <dy_t, y_t> + aux_coef * aux_loss + z_coef * z_loss
+ * (aux_loss and z_loss unscaled, as moe_forward reports them) with respect to
+ * x, W_r, b_r, W1, W3 and W2, the routing of the forward pass held fixed: the
+ * top-k choices, the capacity drops and the slots come from `workspace`,
+ * which must hold the moe_forward call of the same handle, T and inputs,
+ * issued earlier on `stream` with nothing written to it since (the
+ * moe_forward_static scratch cannot serve).  A dropped assignment passes no
+ * gradient; shared experts get gate 1.  Arithmetic in fp32 on CUDA cores,
+ * every sum in a fixed order (deterministic).
+ *   x, W1, W3, W2, dy in the layer's dtype (dy [T][d] like y); W_r, b_r fp32.
+ *   Outputs, fp32, overwritten: dx [T][d], dW_r [E][d], db_r [E] (NULL: not
+ *   wanted), dW1 / dW3 [E + n_shared][d_ff][d] (dW3 NULL for ReLU),
+ *   dW2 [E + n_shared][d][d_ff].
+ *   bw_workspace: device scratch of moe_backward_workspace_bytes(h, T) bytes,
+ *   256-byte aligned (never shrinks as T grows).
+ * Errors as moe_forward; T = 0 zeroes the weight gradients.  Asynchronous.
+ */
+MOE_API size_t moe_backward_workspace_bytes(moe_handle h, int64_t T);
+MOE_API int moe_backward(moe_handle h, int64_t T, const void* x, const float* W_r, const float* b_r,
+                         const void* W1, const void* W3, const void* W2, const void* dy, float aux_coef,
+                         float z_coef, float* dx, float* dW_r, float* db_r, float* dW1, float* dW3, float* dW2,
+                         const void* workspace, size_t workspace_bytes, void* bw_workspace,
+                         size_t bw_workspace_bytes, void* stream);
+
+/*
  * Synchronise `stream` and report the device error word of the current device:
  * MOE_OK, MOE_ERR_TIMEOUT (a kernel's bounded wait ran out and it returned
  * early; outputs of that call are undefined) or MOE_ERR_CUDA.  The error

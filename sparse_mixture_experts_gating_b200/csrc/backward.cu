@@ -1,0 +1,483 @@
+// Backward pass of the MoE layer on CUDA cores, fp32 arithmetic.
+//
+// Gradients of L = sum_t <dy_t, y_t> + aux_coef * aux + z_coef * z
+// ("Mixture of experts", rayaq.ca: section "Replacing the feed-forward
+// block" -- the router learns only through the gate values, the choice of
+// experts being discrete; section "The load-balancing loss" -- f_i is a count
+// without gradient, P_i has one, and the z-loss is the mean of lse^2).  The
+// routing of the forward pass (top-k, capacity drops, slots) is held fixed and
+// read from its workspace.  Per kept row r of expert e (token t, gate g):
+//   a1 = W1_e x_t, a3 = W3_e x_t (recomputed), hid = act(a1, a3)
+//   u = W2_e^T dy_t;  dg_r = <u, hid>;  dhid = g u
+//   ReLU: da1 = dhid [a1 > 0];  SwiGLU: da3 = dhid silu(a1),
+//         da1 = dhid a3 (s + a1 s (1 - s)), s = logistic(a1)
+//   dXp_r = W1_e^T da1 + W3_e^T da3;  dW2_e += g dy_t hid^T;  dW1_e += da1 x_t^T
+// and per token: dx_t = sum of its kept rows' dXp (and the shared experts'
+// rows) + W_r^T dh_t, with dh_t from the gates, the load-balancing loss and
+// the z-loss (Switch: through the full softmax; renormalised: through the
+// softmax over the chosen logits).  Every sum runs in a fixed order, so the
+// results are deterministic.
+//
+// The contractions run as tiled fp32 GEMMs (64 x 64 tiles, 16-deep k-steps,
+// 4 x 4 outputs per thread) over the expert groups of the sorted buffers.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "backward.h"
+#include "common.cuh"
+#include "internal.h"
+#include "moe.h"
+
+namespace moe {
+namespace {
+
+constexpr int TM = 64, TN = 64, TK = 16;
+constexpr int THREADS = 256;
+
+template <typename T>
+__device__ __forceinline__ float ldf(const T* p, int64_t i) {
+  return to_f32(p[i]);
+}
+
+__device__ __forceinline__ void group_rows(const int32_t* offsets, int e, int64_t single_rows, int64_t& r0,
+                                           int64_t& r1) {
+  if (offsets == nullptr) { r0 = 0; r1 = single_rows; }
+  else { r0 = offsets[e]; r1 = offsets[e + 1]; }
+}
+
+// 4 x 4 outputs per thread from shared tiles As[TK][TM], Bs[TK][TN].
+__device__ __forceinline__ void tile_fma(const float (*As)[TM + 4], const float (*Bs)[TN + 4], int ty, int tx,
+                                         float (&acc)[4][4]) {
+#pragma unroll
+  for (int kk = 0; kk < TK; ++kk) {
+    float av[4], bv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) av[i] = As[kk][ty * 4 + i];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+  }
+}
+
+// Row-grouped GEMM: C[r][n] = sum_k A(r, k) B_e(n, k) for the rows r of
+// group e = blockIdx.z, k over K0 terms of (A0, B0) then K1 terms of (A1, B1).
+//   A(r, k) = A0[ar * K0 + k] (A1[ar * K1 + k - K0]), ar = GATHER ? row_token[r] : r
+//   B_e(n, k) = KMAJOR ? B0[(e N + n) K0 + k] : B0[(e K0 + k) N + n]   (B1 likewise with K1)
+struct RowGemm {
+  int N, K0, K1;
+  const void* A0;
+  const void* A1;
+  const void* B0;
+  const void* B1;
+  float* C;  // [rows][N]
+  const int32_t* offsets;
+  const int32_t* row_token;
+};
+
+template <typename TA, typename TB, bool KMAJOR, bool GATHER>
+__global__ void __launch_bounds__(THREADS) bw_rowgemm_kernel(RowGemm g) {
+  __shared__ float As[TK][TM + 4];
+  __shared__ float Bs[TK][TN + 4];
+  const int e = blockIdx.z;
+  int64_t g0, g1;
+  group_rows(g.offsets, e, 0, g0, g1);
+  const int64_t r0 = g0 + static_cast<int64_t>(blockIdx.y) * TM;
+  if (r0 >= g1) return;
+  const int n0 = blockIdx.x * TN;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int K = g.K0 + g.K1;
+  const TA* A0 = static_cast<const TA*>(g.A0);
+  const TA* A1 = static_cast<const TA*>(g.A1);
+  const TB* B0 = static_cast<const TB*>(g.B0);
+  const TB* B1 = static_cast<const TB*>(g.B1);
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += TK) {
+#pragma unroll
+    for (int q = 0; q < (TM * TK) / THREADS; ++q) {  // A tile, k fastest
+      const int el = tid + q * THREADS;
+      const int i = el / TK, kk = el % TK;
+      const int64_t r = r0 + i;
+      const int k = k0 + kk;
+      float v = 0.f;
+      if (r < g1 && k < K) {
+        const int64_t ar = GATHER ? g.row_token[r] : r;
+        v = k < g.K0 ? ldf(A0, ar * g.K0 + k) : ldf(A1, ar * g.K1 + (k - g.K0));
+      }
+      As[kk][i] = v;
+    }
+#pragma unroll
+    for (int q = 0; q < (TN * TK) / THREADS; ++q) {  // B tile, along its contiguous index
+      const int el = tid + q * THREADS;
+      const int j = KMAJOR ? el / TK : el % TN;
+      const int kk = KMAJOR ? el % TK : el / TN;
+      const int n = n0 + j, k = k0 + kk;
+      float v = 0.f;
+      if (n < g.N && k < K) {
+        if (k < g.K0)
+          v = KMAJOR ? ldf(B0, (static_cast<int64_t>(e) * g.N + n) * g.K0 + k)
+                     : ldf(B0, (static_cast<int64_t>(e) * g.K0 + k) * g.N + n);
+        else
+          v = KMAJOR ? ldf(B1, (static_cast<int64_t>(e) * g.N + n) * g.K1 + (k - g.K0))
+                     : ldf(B1, (static_cast<int64_t>(e) * g.K1 + (k - g.K0)) * g.N + n);
+      }
+      Bs[kk][j] = v;
+    }
+    __syncthreads();
+    tile_fma(As, Bs, ty, tx, acc);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t r = r0 + ty * 4 + i;
+    if (r >= g1) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n < g.N) g.C[r * g.N + n] = acc[i][j];
+    }
+  }
+}
+
+// Gradient of a weight per group: C_e[m][n] = sum over the rows r of group e
+// of P(r, m) Q(r, n), rows in order; P(r, m) = P[pr * M + m] (times
+// row_gate[r] and pr = row_token[r] with GATHER_SCALE, else pr = r),
+// Q(r, n) = Q[r * N + n].  offsets NULL: one group of `rows` rows.  Groups
+// without rows get zeros.
+struct WGrad {
+  int M, N;
+  int64_t rows;
+  const void* P;
+  const void* Q;
+  float* C;  // [groups][M][N]
+  const int32_t* offsets;
+  const int32_t* row_token;
+  const float* row_gate;
+};
+
+template <typename TP, typename TQ, bool GATHER_SCALE>
+__global__ void __launch_bounds__(THREADS) bw_wgrad_kernel(WGrad g) {
+  __shared__ float As[TK][TM + 4];
+  __shared__ float Bs[TK][TN + 4];
+  const int e = blockIdx.z;
+  int64_t g0, g1;
+  group_rows(g.offsets, e, g.rows, g0, g1);
+  const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const TP* P = static_cast<const TP*>(g.P);
+  const TQ* Q = static_cast<const TQ*>(g.Q);
+  float acc[4][4] = {};
+  for (int64_t k0 = g0; k0 < g1; k0 += TK) {
+#pragma unroll
+    for (int q = 0; q < (TM * TK) / THREADS; ++q) {  // P tile, m fastest
+      const int el = tid + q * THREADS;
+      const int i = el % TM, kk = el / TM;
+      const int64_t r = k0 + kk;
+      const int m = m0 + i;
+      float v = 0.f;
+      if (r < g1 && m < g.M) {
+        if (GATHER_SCALE) v = ldf(P, static_cast<int64_t>(g.row_token[r]) * g.M + m) * g.row_gate[r];
+        else v = ldf(P, r * g.M + m);
+      }
+      As[kk][i] = v;
+    }
+#pragma unroll
+    for (int q = 0; q < (TN * TK) / THREADS; ++q) {  // Q tile, n fastest
+      const int el = tid + q * THREADS;
+      const int j = el % TN, kk = el / TN;
+      const int64_t r = k0 + kk;
+      const int n = n0 + j;
+      Bs[kk][j] = (r < g1 && n < g.N) ? ldf(Q, r * g.N + n) : 0.f;
+    }
+    __syncthreads();
+    tile_fma(As, Bs, ty, tx, acc);
+    __syncthreads();
+  }
+  float* C = g.C + static_cast<int64_t>(e) * g.M * g.N;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= g.M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n < g.N) C[static_cast<int64_t>(m) * g.N + n] = acc[i][j];
+    }
+  }
+}
+
+// Block-wide sum of one float per thread, in a fixed order.
+__device__ __forceinline__ float block_sum_f(float v, float* s_red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) s_red[warp] = v;
+  __syncthreads();
+  float t = 0.f;
+  for (int w = 0; w < THREADS / 32; ++w) t += s_red[w];
+  return t;
+}
+
+// One block per sorted row: the hidden activation (into A1), the gradients of
+// w1 x (into U) and w3 x (into A3), and dg_r = <W2^T dy_t, hid>.
+template <bool SWIGLU>
+__global__ void __launch_bounds__(THREADS) bw_act_kernel(int d_ff, const int32_t* offsets, int groups,
+                                                         const float* row_gate, float* A1, float* A3, float* U,
+                                                         float* dg) {
+  __shared__ float s_red[THREADS / 32];
+  const int64_t r = blockIdx.x;
+  if (r >= offsets[groups]) return;
+  const float g = row_gate[r];
+  float part = 0.f;
+  for (int n = threadIdx.x; n < d_ff; n += THREADS) {
+    const int64_t i = r * d_ff + n;
+    const float a1 = A1[i], u = U[i];
+    const float dhid = g * u;
+    if (SWIGLU) {
+      const float a3 = A3[i];
+      const float s = 1.f / (1.f + expf(-a1));
+      const float silu = a1 * s;
+      const float hid = silu * a3;
+      part = fmaf(u, hid, part);
+      A1[i] = hid;
+      A3[i] = dhid * silu;
+      U[i] = dhid * a3 * (s + a1 * s * (1.f - s));
+    } else {
+      const float hid = fmaxf(a1, 0.f);
+      part = fmaf(u, hid, part);
+      A1[i] = hid;
+      U[i] = a1 > 0.f ? dhid : 0.f;
+    }
+  }
+  const float t = block_sum_f(part, s_red);
+  if (threadIdx.x == 0) dg[r] = t;
+}
+
+// First-choice counts f_i * T (integer, so order-free).
+__global__ void bw_cnt1_kernel(int64_t T, int k, const int32_t* topk_idx, int32_t* cnt1) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
+  if (t < T) atomicAdd(cnt1 + topk_idx[t * k], 1);
+}
+
+// One block per token: the router logits again (fp32, bias added last), the
+// softmax and log-sum-exp, and the gradient reaching the logits.
+template <typename XT>
+__global__ void __launch_bounds__(THREADS) bw_router_kernel(BackwardArgs a) {
+  __shared__ float s_h[256], s_dp[256], s_dh[256];
+  __shared__ float s_red[THREADS / 32];
+  __shared__ float s_dgj[8];
+  const int64_t t = blockIdx.x;
+  const int E = a.E, d = a.d, k = a.k, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const XT* x = static_cast<const XT*>(a.x) + t * d;
+  for (int e = warp; e < E; e += THREADS / 32) {
+    const float* w = a.W_r + static_cast<int64_t>(e) * d;
+    float s = 0.f;
+    for (int c = lane; c < d; c += 32) s = fmaf(w[c], to_f32(x[c]), s);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) s_h[e] = a.b_r != nullptr ? s + a.b_r[e] : s;
+  }
+  if (tid < k) {
+    const int dst = a.dest_row[t * k + tid];
+    s_dgj[tid] = dst >= 0 ? a.dg[dst] : 0.f;  // a dropped choice passes nothing
+  }
+  __syncthreads();
+  float m = -INFINITY;
+  for (int e = tid; e < E; e += THREADS) m = fmaxf(m, s_h[e]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __syncthreads();
+  if (lane == 0) s_red[warp] = m;
+  __syncthreads();
+  m = -INFINITY;
+  for (int w = 0; w < THREADS / 32; ++w) m = fmaxf(m, s_red[w]);
+  float z = 0.f;
+  for (int e = tid; e < E; e += THREADS) z += expf(s_h[e] - m);
+  const float Z = block_sum_f(z, s_red);
+  const float lse = m + logf(Z);
+  const float inv_T = 1.f / static_cast<float>(a.T);
+  // dp (Switch gates and the load-balancing loss) and the renormalised gates' direct part
+  for (int e = tid; e < E; e += THREADS) {
+    float dp = a.aux_coef * static_cast<float>(E) * static_cast<float>(a.cnt1[e]) * inv_T * inv_T;
+    float dh = 0.f;
+    for (int j = 0; j < k; ++j) {
+      if (a.topk_idx[t * k + j] != e) continue;
+      if (a.gate_mode == MOE_GATE_SWITCH) {
+        dp += s_dgj[j];
+      } else {
+        float sg = 0.f;
+        for (int i = 0; i < k; ++i) sg = fmaf(a.topk_gate[t * k + i], s_dgj[i], sg);
+        dh = a.topk_gate[t * k + j] * (s_dgj[j] - sg);
+      }
+    }
+    s_dp[e] = dp;
+    s_dh[e] = dh;
+  }
+  __syncthreads();
+  float pd = 0.f;
+  for (int e = tid; e < E; e += THREADS) pd = fmaf(expf(s_h[e] - m) / Z, s_dp[e], pd);
+  const float dpp = block_sum_f(pd, s_red);
+  for (int e = tid; e < E; e += THREADS) {
+    const float p = expf(s_h[e] - m) / Z;
+    a.dh[t * E + e] = s_dh[e] + p * (s_dp[e] - dpp) + a.z_coef * 2.f * inv_T * lse * p;
+  }
+}
+
+// One block per token: dx_t = its kept rows' dXp (choices in order), then the
+// shared experts' rows, then W_r^T dh_t (experts in order).
+__global__ void __launch_bounds__(THREADS) bw_dx_kernel(BackwardArgs a) {
+  __shared__ float s_dh[256];
+  const int64_t t = blockIdx.x;
+  const int E = a.E, d = a.d, k = a.k;
+  for (int e = threadIdx.x; e < E; e += THREADS) s_dh[e] = a.dh[t * E + e];
+  __syncthreads();
+  const int64_t sbase = a.n_shared > 0 ? a.offsets[E] : 0;
+  for (int c = threadIdx.x; c < d; c += THREADS) {
+    float v = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int dst = a.dest_row[t * k + j];
+      if (dst >= 0) v += a.dXp[static_cast<int64_t>(dst) * d + c];
+    }
+    for (int si = 0; si < a.n_shared; ++si) v += a.dXp[(sbase + si * a.T + t) * d + c];
+    float r = 0.f;
+    for (int e = 0; e < E; ++e) r = fmaf(s_dh[e], a.W_r[static_cast<int64_t>(e) * d + c], r);
+    a.dx[t * d + c] = v + r;
+  }
+}
+
+// db_e = sum over tokens of dh[t][e], tokens in a fixed order.
+__global__ void __launch_bounds__(THREADS) bw_db_kernel(int64_t T, int E, const float* dh, float* db) {
+  __shared__ float s_red[THREADS / 32];
+  const int e = blockIdx.x;
+  float s = 0.f;
+  for (int64_t t = threadIdx.x; t < T; t += THREADS) s += dh[t * E + e];
+  const float tot = block_sum_f(s, s_red);
+  if (threadIdx.x == 0) db[e] = tot;
+}
+
+template <typename TA, typename TB, bool KMAJOR, bool GATHER>
+cudaError_t rowgemm(const RowGemm& g, int groups, int max_rows, cudaStream_t s) {
+  const dim3 grid((g.N + TN - 1) / TN, (max_rows + TM - 1) / TM, groups);
+  bw_rowgemm_kernel<TA, TB, KMAJOR, GATHER><<<grid, THREADS, 0, s>>>(g);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <typename TP, typename TQ, bool GATHER_SCALE>
+cudaError_t wgrad(const WGrad& g, int groups, cudaStream_t s) {
+  const dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM, groups);
+  bw_wgrad_kernel<TP, TQ, GATHER_SCALE><<<grid, THREADS, 0, s>>>(g);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <typename XT>
+cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
+  const int groups = a.E + a.n_shared;
+  const bool swiglu = a.act == MOE_ACT_SWIGLU;
+  cudaError_t e;
+  // first-choice counts for the load-balancing loss's gradient
+  if ((e = cudaMemsetAsync(a.cnt1, 0, sizeof(int32_t) * a.E, s)) != cudaSuccess) return e;
+  bw_cnt1_kernel<<<static_cast<unsigned>((a.T + THREADS - 1) / THREADS), THREADS, 0, s>>>(a.T, a.k, a.topk_idx,
+                                                                                          a.cnt1);
+  count_launch();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // a1 = W1 x, a3 = W3 x
+  RowGemm g{};
+  g.N = a.d_ff;
+  g.K0 = a.d;
+  g.A0 = a.Xp;
+  g.B0 = a.W1;
+  g.C = a.A1;
+  g.offsets = a.offsets;
+  g.row_token = a.row_token;
+  if ((e = rowgemm<XT, XT, true, false>(g, groups, a.max_group_rows, s)) != cudaSuccess) return e;
+  if (swiglu) {
+    g.B0 = a.W3;
+    g.C = a.A3;
+    if ((e = rowgemm<XT, XT, true, false>(g, groups, a.max_group_rows, s)) != cudaSuccess) return e;
+  }
+  // u = W2^T dy_t
+  g.K0 = a.d;
+  g.A0 = a.dy;
+  g.B0 = a.W2;
+  g.C = a.U;
+  if ((e = rowgemm<XT, XT, false, true>(g, groups, a.max_group_rows, s)) != cudaSuccess) return e;
+  // hidden activation, its gradients, dg
+  if (swiglu)
+    bw_act_kernel<true><<<static_cast<unsigned>(a.s_max), THREADS, 0, s>>>(a.d_ff, a.offsets, groups, a.row_gate,
+                                                                            a.A1, a.A3, a.U, a.dg);
+  else
+    bw_act_kernel<false><<<static_cast<unsigned>(a.s_max), THREADS, 0, s>>>(a.d_ff, a.offsets, groups, a.row_gate,
+                                                                             a.A1, a.A3, a.U, a.dg);
+  count_launch();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // dXp = W1^T da1 (+ W3^T da3)
+  RowGemm gx{};
+  gx.N = a.d;
+  gx.K0 = a.d_ff;
+  gx.K1 = swiglu ? a.d_ff : 0;
+  gx.A0 = a.U;
+  gx.A1 = a.A3;
+  gx.B0 = a.W1;
+  gx.B1 = a.W3;
+  gx.C = a.dXp;
+  gx.offsets = a.offsets;
+  if ((e = rowgemm<float, XT, false, false>(gx, groups, a.max_group_rows, s)) != cudaSuccess) return e;
+  // weight gradients
+  WGrad w{};
+  w.offsets = a.offsets;
+  w.row_token = a.row_token;
+  w.row_gate = a.row_gate;
+  w.M = a.d;  // dW2_e = sum_r (g_r dy_t) hid_r^T
+  w.N = a.d_ff;
+  w.P = a.dy;
+  w.Q = a.A1;
+  w.C = a.dW2;
+  if ((e = wgrad<XT, float, true>(w, groups, s)) != cudaSuccess) return e;
+  w.M = a.d_ff;  // dW1_e = sum_r da1_r x_r^T
+  w.N = a.d;
+  w.P = a.U;
+  w.Q = a.Xp;
+  w.C = a.dW1;
+  if ((e = wgrad<float, XT, false>(w, groups, s)) != cudaSuccess) return e;
+  if (swiglu) {
+    w.P = a.A3;
+    w.C = a.dW3;
+    if ((e = wgrad<float, XT, false>(w, groups, s)) != cudaSuccess) return e;
+  }
+  // router: dh, then dx, dW_r, db_r
+  bw_router_kernel<XT><<<static_cast<unsigned>(a.T), THREADS, 0, s>>>(a);
+  count_launch();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  bw_dx_kernel<<<static_cast<unsigned>(a.T), THREADS, 0, s>>>(a);
+  count_launch();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  WGrad wr{};
+  wr.M = a.E;
+  wr.N = a.d;
+  wr.rows = a.T;
+  wr.P = a.dh;
+  wr.Q = a.x;
+  wr.C = a.dW_r;
+  if ((e = wgrad<float, XT, false>(wr, 1, s)) != cudaSuccess) return e;
+  if (a.db_r != nullptr) {
+    bw_db_kernel<<<a.E, THREADS, 0, s>>>(a.T, a.E, a.dh, a.db_r);
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s) {
+  return a.x_is_bf16 ? backward_t<__nv_bfloat16>(a, s) : backward_t<float>(a, s);
+}
+
+}  // namespace moe

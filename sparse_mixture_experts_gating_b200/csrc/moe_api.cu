@@ -18,6 +18,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "scan_dispatch.h"
+#include "backward.h"
 
 struct moe_layer {
   int E, k, d, d_ff, act, gate_mode, dtype;
@@ -161,6 +162,28 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   w.Yp = take(yp_rows > 0 ? sizeof(float) * static_cast<size_t>(yp_rows) * L.d : 0);
   w.total = o;
   return w;
+}
+
+// Scratch of the backward pass (fp32): A1, U [S][d_ff] (and A3 for SwiGLU),
+// dg [S], dXp [S][d], dh [T][E], cnt1 [E].
+struct BwLayout {
+  size_t A1, A3, U, dg, dXp, dh, cnt1, total;
+};
+
+BwLayout make_bw_layout(const moe_layer& L, const Layout& w) {
+  BwLayout b;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
+  const size_t hid = sizeof(float) * static_cast<size_t>(w.s_max) * L.d_ff;
+  b.A1 = take(hid);
+  b.A3 = take(L.act == MOE_ACT_SWIGLU ? hid : 0);
+  b.U = take(hid);
+  b.dg = take(sizeof(float) * static_cast<size_t>(w.s_max));
+  b.dXp = take(sizeof(float) * static_cast<size_t>(w.s_max) * L.d);
+  b.dh = take(sizeof(float) * static_cast<size_t>(w.T) * L.E);
+  b.cnt1 = take(sizeof(int32_t) * L.E);
+  b.total = o;
+  return b;
 }
 
 void record(const moe_debug* dbg, int stage, int which, cudaStream_t s) {
@@ -515,6 +538,101 @@ int moe_selftest_timeout(int64_t limit_ns, void* stream) {
   const int64_t lim = std::min<int64_t>(std::max<int64_t>(limit_ns, 1000), 2000000000LL);
   ce = launch_selftest_timeout(di->err, lim, static_cast<cudaStream_t>(stream));
   if (ce != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_selftest_timeout: ") + cudaGetErrorString(ce));
+  return MOE_OK;
+}
+
+size_t moe_backward_workspace_bytes(moe_handle h, int64_t T) {
+  if (h == nullptr || T < 0) return 0;
+  return make_bw_layout(*h, make_layout(*h, T)).total;
+}
+
+int moe_backward(moe_handle h, int64_t T, const void* x, const float* W_r, const float* b_r, const void* W1,
+                 const void* W3, const void* W2, const void* dy, float aux_coef, float z_coef, float* dx,
+                 float* dW_r, float* db_r, float* dW1, float* dW3, float* dW2, const void* workspace,
+                 size_t workspace_bytes, void* bw_workspace, size_t bw_workspace_bytes, void* stream) {
+  if (h == nullptr) return fail(MOE_ERR_INVALID_ARG, "moe_backward: handle is NULL");
+  const moe_layer& L = *h;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "moe_backward: T < 0");
+  if (T * L.k > 2147483647LL / 2) return fail(MOE_ERR_UNSUPPORTED, "moe_backward: T * k too large");
+  if (W_r == nullptr || W1 == nullptr || W2 == nullptr || dW_r == nullptr || dW1 == nullptr || dW2 == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "moe_backward: W_r, W1, W2, dW_r, dW1 and dW2 must be non-NULL");
+  const bool swiglu = L.act == MOE_ACT_SWIGLU;
+  if (swiglu != (W3 != nullptr) || swiglu != (dW3 != nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "moe_backward: W3 and dW3 must be given for SwiGLU and NULL for ReLU");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int groups = L.E + L.n_shared;
+  const size_t wexp = sizeof(float) * static_cast<size_t>(groups) * L.d_ff * L.d;
+  if (T == 0) {  // L = 0: every gradient is zero
+    if (cudaMemsetAsync(dW_r, 0, sizeof(float) * L.E * static_cast<size_t>(L.d), s) != cudaSuccess ||
+        (db_r != nullptr && cudaMemsetAsync(db_r, 0, sizeof(float) * L.E, s) != cudaSuccess) ||
+        cudaMemsetAsync(dW1, 0, wexp, s) != cudaSuccess || cudaMemsetAsync(dW2, 0, wexp, s) != cudaSuccess ||
+        (swiglu && cudaMemsetAsync(dW3, 0, wexp, s) != cudaSuccess))
+      return fail(MOE_ERR_CUDA, std::string("moe_backward: ") + cudaGetErrorString(cudaGetLastError()));
+    t_err.clear();
+    return MOE_OK;
+  }
+  if (x == nullptr || dy == nullptr || dx == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "moe_backward: x, dy and dx must be non-NULL");
+  const Layout w = make_layout(L, T);
+  const BwLayout b = make_bw_layout(L, w);
+  if (workspace == nullptr || workspace_bytes < w.total)
+    return fail(MOE_ERR_INVALID_ARG, "moe_backward: forward workspace missing or smaller than moe_workspace_bytes()");
+  if (bw_workspace == nullptr || bw_workspace_bytes < b.total)
+    return fail(MOE_ERR_INVALID_ARG,
+                "moe_backward: backward workspace missing or smaller than moe_backward_workspace_bytes()");
+  if (((reinterpret_cast<uintptr_t>(workspace) | reinterpret_cast<uintptr_t>(bw_workspace)) & 255) != 0)
+    return fail(MOE_ERR_INVALID_ARG, "moe_backward: workspaces must be 256-byte aligned");
+
+  const uint8_t* ws = static_cast<const uint8_t*>(workspace);
+  uint8_t* bw = static_cast<uint8_t*>(bw_workspace);
+  BackwardArgs a;
+  memset(&a, 0, sizeof(a));
+  a.T = T;
+  a.E = L.E;
+  a.k = L.k;
+  a.d = L.d;
+  a.d_ff = L.d_ff;
+  a.act = L.act;
+  a.gate_mode = L.gate_mode;
+  a.n_shared = L.n_shared;
+  a.x_is_bf16 = L.dtype == MOE_BF16;
+  // a token takes an expert at most once, a shared expert's group has T rows
+  int64_t mg = T;
+  if (L.n_shared == 0 && w.capacity >= 0 && w.capacity < mg) mg = w.capacity;
+  a.max_group_rows = static_cast<int>(mg);
+  a.s_max = w.s_max;
+  a.x = x;
+  a.W_r = W_r;
+  a.b_r = b_r;
+  a.W1 = W1;
+  a.W3 = W3;
+  a.W2 = W2;
+  a.dy = dy;
+  a.aux_coef = aux_coef;
+  a.z_coef = z_coef;
+  a.topk_idx = reinterpret_cast<const int32_t*>(ws + w.idx);
+  a.topk_gate = reinterpret_cast<const float*>(ws + w.gate);
+  a.dest_row = reinterpret_cast<const int32_t*>(ws + w.dest);
+  a.offsets = reinterpret_cast<const int32_t*>(ws + w.offsets);
+  a.row_token = reinterpret_cast<const int32_t*>(ws + w.row_token);
+  a.row_gate = reinterpret_cast<const float*>(ws + w.row_gate);
+  a.Xp = ws + w.Xp;
+  a.A1 = reinterpret_cast<float*>(bw + b.A1);
+  a.A3 = swiglu ? reinterpret_cast<float*>(bw + b.A3) : nullptr;
+  a.U = reinterpret_cast<float*>(bw + b.U);
+  a.dg = reinterpret_cast<float*>(bw + b.dg);
+  a.dXp = reinterpret_cast<float*>(bw + b.dXp);
+  a.dh = reinterpret_cast<float*>(bw + b.dh);
+  a.cnt1 = reinterpret_cast<int32_t*>(bw + b.cnt1);
+  a.dx = dx;
+  a.dW_r = dW_r;
+  a.db_r = db_r;
+  a.dW1 = dW1;
+  a.dW3 = dW3;
+  a.dW2 = dW2;
+  const cudaError_t ce = launch_backward(a, s);
+  if (ce != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_backward: ") + cudaGetErrorString(ce));
+  t_err.clear();
   return MOE_OK;
 }
 

@@ -51,6 +51,7 @@ class MoELayer:
                                DTYPE[dtype], ctypes.byref(h)))
         self._h = h
         self._ws = None
+        self._bw = None  # backward scratch
         self.hidden = hidden
         check(lib().moe_set_hidden_precision(h, HIDDEN[hidden]))
         self.n_shared = int(n_shared)
@@ -112,6 +113,37 @@ class MoELayer:
         return y, counts, dropped, aux, z
 
     __call__ = forward
+
+    def backward_workspace_bytes(self, T: int) -> int:
+        return int(lib().moe_backward_workspace_bytes(self._h, T))
+
+    def backward(self, x, W_r, b_r, W1, W3, W2, dy, *, aux_coef=0.0, z_coef=0.0, workspace=None,
+                 bw_workspace=None, grads=None, stream=None) -> dict:
+        """Gradients of <dy, y> + aux_coef * aux + z_coef * z for the last
+        forward on ``workspace`` (default: this layer's own), routing held
+        fixed.  Returns fp32 device tensors dx, dW_r, db_r (None without a
+        bias), dW1, dW3 (None for ReLU), dW2; ``grads`` may supply them."""
+        T, dev = x.shape[0], x.device
+        ws = workspace if workspace is not None else self._ws
+        if bw_workspace is None:
+            n = self.backward_workspace_bytes(T)
+            if self._bw is None or self._bw.numel() < n or self._bw.device != dev:
+                self._bw = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
+            bw_workspace = self._bw
+        f32 = dict(dtype=torch.float32, device=dev)
+        g = dict(grads or {})
+        g.setdefault("dx", torch.empty((T, self.d), **f32))
+        g.setdefault("dW_r", torch.empty(W_r.shape, **f32))
+        g.setdefault("db_r", None if b_r is None else torch.empty(b_r.shape, **f32))
+        g.setdefault("dW1", torch.empty(W1.shape, **f32))
+        g.setdefault("dW3", None if W3 is None else torch.empty(W3.shape, **f32))
+        g.setdefault("dW2", torch.empty(W2.shape, **f32))
+        check(lib().moe_backward(
+            self._h, T, _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dy),
+            float(aux_coef), float(z_coef), _ptr(g["dx"]), _ptr(g["dW_r"]), _ptr(g["db_r"]), _ptr(g["dW1"]),
+            _ptr(g["dW3"]), _ptr(g["dW2"]), _ptr(ws), 0 if ws is None else ws.numel(), _ptr(bw_workspace),
+            bw_workspace.numel(), _stream_handle(stream)))
+        return g
 
     def balance_losses(self, T: int, workspace=None, out=None, stream=None) -> torch.Tensor:
         """The alternative balance statistics of the last forward on ``workspace``

@@ -160,3 +160,32 @@ def test_static_scratch_limit_stated_in_the_header_holds(L):
     lim = 32 << 20
     assert L.moe_workspace_bytes(h, stated) <= lim < L.moe_workspace_bytes(h, stated + 1)
     L.moe_destroy(h)
+
+
+def test_backward_validates_arguments_without_gpu(L):
+    rc, h = _create(L, 8, 2, 64, 64, 1, 1, 0.0, 1)  # SwiGLU
+    assert rc == 0
+    prev = 0
+    for T in range(0, 300):
+        n = L.moe_backward_workspace_bytes(h, T)
+        assert n >= prev and n % 256 == 0
+        prev = n
+    assert L.moe_backward_workspace_bytes(None, 4) == 0 and L.moe_backward_workspace_bytes(h, -1) == 0
+    p = ctypes.c_void_p(256)
+    big = 1 << 40
+
+    def call(hh=h, T=4, W3=p, dW3=p, ws=p, ws_n=big, bw=p, bw_n=big, x=p):
+        return L.moe_backward(hh, T, x, p, None, p, W3, p, p, 0.0, 0.0, p, p, None, p, dW3, p, ws, ws_n, bw,
+                              bw_n, None)
+
+    assert call(hh=None) == _lib.MOE_ERR_INVALID_ARG
+    assert call(T=-1) == _lib.MOE_ERR_INVALID_ARG
+    assert call(W3=None) == _lib.MOE_ERR_INVALID_ARG   # SwiGLU needs W3 ...
+    assert call(dW3=None) == _lib.MOE_ERR_INVALID_ARG  # ... and dW3
+    assert call(x=None) == _lib.MOE_ERR_INVALID_ARG
+    assert call(ws_n=16) == _lib.MOE_ERR_INVALID_ARG
+    assert "forward workspace" in L.moe_last_error().decode()
+    assert call(bw_n=16) == _lib.MOE_ERR_INVALID_ARG
+    assert "backward workspace" in L.moe_last_error().decode()
+    assert call(bw=ctypes.c_void_p(272)) == _lib.MOE_ERR_INVALID_ARG
+    L.moe_destroy(h)

@@ -1,0 +1,128 @@
+"""Parity of the backward pass (moe_backward through the C ABI) with the
+backward oracle (oracle/moe_backward.py, pinned by finite differences).
+
+Small seeded layers with dyadic router inputs, so that the routing of the
+forward pass is the oracle's (checked), then every gradient tensor is
+compared element by element.  Tolerance, per tensor: max|got - ref| <=
+2e-4 * max|ref|.  The kernels accumulate in fp32 sums of at most a few
+thousand products (relative error about sqrt(K) * 2^-24, below 1e-5 of the
+operands' scale); the router's gradient subtracts <dp, p> from dp, which
+loses a few more bits where the two are close.  A wrong term or sign moves a
+tensor by O(1) of its scale.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_backward as OB
+from sparse_mixture_experts_gating_b200 import status
+from sparse_mixture_experts_gating_b200.workloads import (ACT_RELU, ACT_SWIGLU, DTYPE_BF16, DTYPE_F32, GATE_RENORM,
+                                                          GATE_SWITCH, Workload, make_inputs)
+from tests._parity import layer_for, np32
+
+pytestmark = pytest.mark.gpu
+
+R, S = ACT_RELU, ACT_SWIGLU
+SW, RN = GATE_SWITCH, GATE_RENORM
+BF, F32 = DTYPE_BF16, DTYPE_F32
+AUX, ZC = 0.37, 0.21
+TOL = 2e-4
+
+# name, T, d, E, k, d_ff, act, gate, cf, dtype, bias, n_shared
+CASES = [
+    ("switch_relu_drops_bf16", 300, 64, 8, 1, 96, R, SW, 1.0, BF, "normal", 0),
+    ("renorm_swiglu_bf16", 257, 48, 6, 2, 80, S, RN, 0.0, BF, None, 0),
+    ("switch_k2_swiglu_fp32", 130, 40, 5, 2, 56, S, SW, 1.25, F32, "normal", 0),
+    ("shared_swiglu_drops_bf16", 150, 64, 4, 2, 64, S, RN, 1.0, BF, None, 1),
+    ("small_batch_bf16", 20, 64, 8, 2, 64, S, RN, 0.0, BF, "normal", 0),  # one launch routes T <= 32
+    ("e32_k4_zipf_relu", 200, 32, 32, 4, 40, R, RN, 1.0, BF, "zipf", 0),
+]
+
+
+def _w(case) -> Workload:
+    name, T, d, E, k, d_ff, act, gate, cf, dt, bias, ns = case
+    return Workload(name, T=T, d=d, E=E, k=k, d_ff=d_ff, act=act, gate=gate, capacity_factor=cf, dtype=dt,
+                    bias=bias, dyadic=True, seed=6000 + zlib.crc32(name.encode()) % 1000, n_shared=ns)
+
+
+def _run(w: Workload):
+    inp = make_inputs(w, device="cuda")
+    layer = layer_for(w)
+    dbg = layer.debug_buffers(w.T, inp["x"].device)
+    layer(inp["x"], inp["W_r"], inp["b_r"], inp["W1"], inp["W3"], inp["W2"], debug=dbg)
+    gen = torch.Generator().manual_seed(99)
+    dy = torch.randn(w.T, w.d, generator=gen).to(inp["x"].dtype).to(inp["x"].device)
+    g = layer.backward(inp["x"], inp["W_r"], inp["b_r"], inp["W1"], inp["W3"], inp["W2"], dy,
+                       aux_coef=AUX, z_coef=ZC)
+    status()
+    return inp, layer, dbg, dy, g
+
+
+def _oracle(w: Workload, inp: dict, dy):
+    E = w.E
+    W1, W2 = np32(inp["W1"]), np32(inp["W2"])
+    W3 = None if inp["W3"] is None else np32(inp["W3"])
+    shared = None
+    if w.n_shared:
+        shared = (W1[E:], None if W3 is None else W3[E:], W2[E:])
+    return OB.moe_backward(np32(inp["x"]), np32(inp["W_r"]), np32(inp["b_r"]), W1[:E],
+                           None if W3 is None else W3[:E], W2[:E], np32(dy), k=w.k, gate_mode=w.gate, act=w.act,
+                           capacity_factor=w.capacity_factor, aux_coef=AUX, z_coef=ZC, shared=shared)
+
+
+def _close(name, got, ref):
+    got = np.asarray(got, np.float64)
+    scale = float(np.abs(ref).max()) if ref.size else 0.0
+    err = float(np.abs(got - ref).max()) if ref.size else 0.0
+    assert err <= TOL * scale + 1e-30, f"{name}: max|d| {err:.3e} vs scale {scale:.3e}"
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_backward_matches_oracle(case):
+    w = _w(case)
+    inp, _, dbg, dy, g = _run(w)
+    o = _oracle(w, inp, dy)
+    np.testing.assert_array_equal(dbg["topk_idx"].cpu().numpy(), o["idx"])
+    np.testing.assert_array_equal(dbg["drop_mask"].cpu().numpy().astype(bool), ~o["kept"])
+    if w.capacity_factor > 0 and case[0] != "small_batch_bf16":
+        assert not o["kept"].all()
+    E = w.E
+    _close("dx", np32(g["dx"]), o["dx"])
+    _close("dW_r", np32(g["dW_r"]), o["dW_r"])
+    if inp["b_r"] is not None:
+        _close("db_r", np32(g["db_r"]), o["db_r"])
+    _close("dW1", np32(g["dW1"])[:E], o["dW1"])
+    _close("dW2", np32(g["dW2"])[:E], o["dW2"])
+    if w.act == S:
+        _close("dW3", np32(g["dW3"])[:E], o["dW3"])
+    if w.n_shared:
+        _close("dW1s", np32(g["dW1"])[E:], o["dW1s"])
+        _close("dW2s", np32(g["dW2"])[E:], o["dW2s"])
+        if w.act == S:
+            _close("dW3s", np32(g["dW3"])[E:], o["dW3s"])
+
+
+def test_backward_is_deterministic():
+    w = _w(CASES[1])
+    inp, layer, _, dy, g1 = _run(w)
+    g2 = layer.backward(inp["x"], inp["W_r"], inp["b_r"], inp["W1"], inp["W3"], inp["W2"], dy,
+                        aux_coef=AUX, z_coef=ZC)
+    status()
+    for key in ("dx", "dW_r", "dW1", "dW3", "dW2"):
+        assert torch.equal(g1[key], g2[key]), key
+
+
+def test_backward_zero_tokens():
+    w = _w(CASES[0])
+    inp = make_inputs(w, device="cuda")
+    layer = layer_for(w)
+    x0 = inp["x"][:0]
+    layer(x0, inp["W_r"], inp["b_r"], inp["W1"], inp["W3"], inp["W2"])
+    grads = {"dW1": torch.full(inp["W1"].shape, 7.0, device="cuda"),
+             "dW2": torch.full(inp["W2"].shape, 7.0, device="cuda")}
+    g = layer.backward(x0, inp["W_r"], inp["b_r"], inp["W1"], inp["W3"], inp["W2"], x0, grads=grads)
+    status()
+    for key in ("dW_r", "db_r", "dW1", "dW2"):
+        assert not torch.any(g[key]), key
