@@ -462,12 +462,16 @@ def main():
 
 
 def backward_flops(w, S, T):
-    """FP32 FLOPs of the backward pass for S kept rows (shared rows included):
-    per row and d x d_ff contraction 2 d d_ff; ReLU runs 5 of them (w1 x again,
-    W2^T dy, dXp, dW2, dW1), SwiGLU 8 (w1 x, w3 x, W2^T dy, two for dXp, dW2,
-    dW1, dW3); the router 3 T E d contractions (logits again, W_r^T dh, dW_r)."""
-    n = 8 if w.act == 1 else 5
-    return 2.0 * S * w.d * w.d_ff * n + 3 * 2.0 * T * w.E * w.d
+    """(row-product FLOPs, weight-gradient and router FLOPs) of the backward
+    pass for S kept rows (shared rows included).  Per row and d x d_ff
+    contraction 2 d d_ff: the row products are w1 x again, W2^T dy and dXp
+    (ReLU: 3; SwiGLU: w3 x and a second dXp term, 5) -- on the tensor cores for
+    bf16 layers; the weight gradients dW2, dW1 (and dW3) on the CUDA cores,
+    with the router's 3 T E d contractions (logits again, W_r^T dh, dW_r)."""
+    rows = 5 if w.act == 1 else 3
+    wgr = 3 if w.act == 1 else 2
+    c = 2.0 * S * w.d * w.d_ff
+    return c * rows, c * wgr + 3 * 2.0 * T * w.E * w.d
 
 
 def backward_bench(args, w, inp, warmup, world, rank, local, dev):
@@ -531,10 +535,14 @@ def backward_bench(args, w, inp, warmup, world, rank, local, dev):
     cap = layer.capacity(w.T)
     kept = sum(c if cap is None else min(c, cap) for c in counts.cpu().tolist())
     S = kept + w.n_shared * w.T
-    fl = backward_flops(w, S, w.T)
+    fl_rows, fl_alu = backward_flops(w, S, w.T)
+    if w.dtype != 1:  # fp32 layers: every product on the CUDA cores
+        fl_rows, fl_alu = 0.0, fl_rows + fl_alu
     clocks = sampler.summary(wall0, wall1)
     peak = 148 * 128 * 2 * (clocks["sm_max_mhz"] or 1965.0) * 1e6 / 1e12  # fp32 FMA lanes x 2 x max clock
-    ach = fl / (bw_s / K) / 1e12
+    peaks, _ = load_peaks()
+    floor_s = fl_rows / (peaks["bf16_tflops"] * 1e12) + fl_alu / (peak * 1e12)
+    ach = fl_alu / (bw_s / K) / 1e12
     line = {
         "metric": "MoE-layer training step (forward + backward) tokens/s on 1 B200",
         "value": round(w.T * K / step_s, 1),
@@ -550,9 +558,13 @@ def backward_bench(args, w, inp, warmup, world, rank, local, dev):
         "dtype": "f32 (backward), " + ("bf16" if w.dtype == 1 else "f32") + " (forward)",
         "data": "synthetic (seeded; shapes and distributions of the workload, random-init weights)",
         "config": dict(config_of(w, 1), hidden=args.hidden, loss="<dy, y> + 0.01 aux + 1e-3 z"),
+        # the CUDA-core weight gradients bound the step: their FLOPs over the whole backward time
         "roofline": {"bound": "alu", "achieved": round(ach, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
-                     "frac": round(ach / peak, 4), "kernel": "backward pass (fp32 CUDA-core GEMMs)",
+                     "frac": round(ach / peak, 4),
+                     "kernel": "backward pass (weight gradients on CUDA cores; row products on tensor cores)",
                      "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x clocks.max.sm", "traffic": None},
+        "backward_floor": {"tensor_flops": fl_rows, "alu_flops": fl_alu, "floor_ms": round(floor_s * 1e3, 4),
+                           "frac": round(floor_s / (bw_s / K), 4)},
         "gpu_launches": int(n_launch),
         "clocks": clocks,
     }

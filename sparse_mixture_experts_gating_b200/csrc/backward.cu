@@ -20,10 +20,18 @@
 //
 // The contractions run as tiled fp32 GEMMs (64 x 64 tiles, 16-deep k-steps,
 // 4 x 4 outputs per thread) over the expert groups of the sorted buffers.
+// For bf16 layers the three row-grouped products (w1 x and w3 x again,
+// W2^T dy, W1^T da1 + W3^T da3) run instead on the forward's tensor-core
+// grouped GEMM with its fp32 epilogue (gate 1): the weights are transposed
+// per expert into K-major copies, dy is gathered into expert-sorted rows, and
+// da1 / da3 enter as hi + lo bf16 planes (about 16 significant bits) like
+// the forward's hidden activation.  The weight gradients, whose reduction runs
+// over each expert's ragged rows, stay on the CUDA cores.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "backward.h"
 #include "common.cuh"
@@ -228,7 +236,8 @@ __device__ __forceinline__ float block_sum_f(float v, float* s_red) {
 template <bool SWIGLU>
 __global__ void __launch_bounds__(THREADS) bw_act_kernel(int d_ff, const int32_t* offsets, int groups,
                                                          const float* row_gate, float* A1, float* A3, float* U,
-                                                         float* dg) {
+                                                         float* dg, __nv_bfloat16* dA1p, __nv_bfloat16* dA3p,
+                                                         int64_t plane) {
   __shared__ float s_red[THREADS / 32];
   const int64_t r = blockIdx.x;
   if (r >= offsets[groups]) return;
@@ -238,6 +247,7 @@ __global__ void __launch_bounds__(THREADS) bw_act_kernel(int d_ff, const int32_t
     const int64_t i = r * d_ff + n;
     const float a1 = A1[i], u = U[i];
     const float dhid = g * u;
+    float da1, da3 = 0.f;
     if (SWIGLU) {
       const float a3 = A3[i];
       const float s = 1.f / (1.f + expf(-a1));
@@ -245,13 +255,25 @@ __global__ void __launch_bounds__(THREADS) bw_act_kernel(int d_ff, const int32_t
       const float hid = silu * a3;
       part = fmaf(u, hid, part);
       A1[i] = hid;
-      A3[i] = dhid * silu;
-      U[i] = dhid * a3 * (s + a1 * s * (1.f - s));
+      da3 = dhid * silu;
+      da1 = dhid * a3 * (s + a1 * s * (1.f - s));
+      A3[i] = da3;
     } else {
       const float hid = fmaxf(a1, 0.f);
       part = fmaf(u, hid, part);
       A1[i] = hid;
-      U[i] = a1 > 0.f ? dhid : 0.f;
+      da1 = a1 > 0.f ? dhid : 0.f;
+    }
+    U[i] = da1;
+    if (dA1p != nullptr) {  // hi = RNE(v), lo = RNE(v - hi)
+      const __nv_bfloat16 h1 = __float2bfloat16_rn(da1);
+      dA1p[i] = h1;
+      dA1p[plane + i] = __float2bfloat16_rn(da1 - __bfloat162float(h1));
+      if (SWIGLU) {
+        const __nv_bfloat16 h3 = __float2bfloat16_rn(da3);
+        dA3p[i] = h3;
+        dA3p[plane + i] = __float2bfloat16_rn(da3 - __bfloat162float(h3));
+      }
     }
   }
   const float t = block_sum_f(part, s_red);
@@ -330,10 +352,11 @@ __global__ void __launch_bounds__(THREADS) bw_router_kernel(BackwardArgs a) {
 
 // One block per token: dx_t = its kept rows' dXp (choices in order), then the
 // shared experts' rows, then W_r^T dh_t (experts in order).
-__global__ void __launch_bounds__(THREADS) bw_dx_kernel(BackwardArgs a) {
+__global__ void __launch_bounds__(THREADS) bw_dx_kernel(BackwardArgs a, int parts) {
   __shared__ float s_dh[256];
   const int64_t t = blockIdx.x;
   const int E = a.E, d = a.d, k = a.k;
+  const int64_t pstride = a.s_max * d;  // between the W1 and W3 parts of dXp
   for (int e = threadIdx.x; e < E; e += THREADS) s_dh[e] = a.dh[t * E + e];
   __syncthreads();
   const int64_t sbase = a.n_shared > 0 ? a.offsets[E] : 0;
@@ -341,9 +364,15 @@ __global__ void __launch_bounds__(THREADS) bw_dx_kernel(BackwardArgs a) {
     float v = 0.f;
     for (int j = 0; j < k; ++j) {
       const int dst = a.dest_row[t * k + j];
-      if (dst >= 0) v += a.dXp[static_cast<int64_t>(dst) * d + c];
+      if (dst < 0) continue;
+      v += a.dXp[static_cast<int64_t>(dst) * d + c];
+      if (parts == 2) v += a.dXp[pstride + static_cast<int64_t>(dst) * d + c];
     }
-    for (int si = 0; si < a.n_shared; ++si) v += a.dXp[(sbase + si * a.T + t) * d + c];
+    for (int si = 0; si < a.n_shared; ++si) {
+      const int64_t row = sbase + si * a.T + t;
+      v += a.dXp[row * d + c];
+      if (parts == 2) v += a.dXp[pstride + row * d + c];
+    }
     float r = 0.f;
     for (int e = 0; e < E; ++e) r = fmaf(s_dh[e], a.W_r[static_cast<int64_t>(e) * d + c], r);
     a.dx[t * d + c] = v + r;
@@ -358,6 +387,77 @@ __global__ void __launch_bounds__(THREADS) bw_db_kernel(int64_t T, int E, const 
   for (int64_t t = threadIdx.x; t < T; t += THREADS) s += dh[t * E + e];
   const float tot = block_sum_f(s, s_red);
   if (threadIdx.x == 0) db[e] = tot;
+}
+
+// out[g][c][r] = in[g][r][c] for bf16 matrices [G][R][C] (32 x 32 tiles).
+__global__ void __launch_bounds__(256) bw_transpose_kernel(const __nv_bfloat16* __restrict__ in,
+                                                           __nv_bfloat16* __restrict__ out, int R, int C) {
+  __shared__ __nv_bfloat16 tile[32][34];
+  const int64_t g = blockIdx.z;
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  const __nv_bfloat16* src = in + g * R * C;
+  __nv_bfloat16* dst = out + g * R * C;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < R && c < C) tile[i][threadIdx.x] = src[static_cast<int64_t>(r) * C + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < R && c < C) dst[static_cast<int64_t>(c) * R + r] = tile[threadIdx.x][i];
+  }
+}
+
+// dy rows into expert-sorted order (a warp per row, 16-byte copies) and the
+// gate 1 of every row for the fp32 epilogue.
+__global__ void __launch_bounds__(256) bw_gather_dy_kernel(int d, const int32_t* offsets, int groups,
+                                                           const int32_t* row_token, const uint4* dy, uint4* dYs,
+                                                           float* ones) {
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= offsets[groups]) return;
+  const int nv = d / 8;  // 16-byte groups of a bf16 row
+  const int64_t t = row_token[r];
+  for (int v = lane; v < nv; v += 32) dYs[r * nv + v] = dy[t * nv + v];
+  if (lane == 0) ones[r] = 1.f;
+}
+
+// One tensor-core grouped GEMM with the fp32 epilogue (gate 1):
+// out[r][n] = sum_k A[r][k] B_e[n][k] over the expert-sorted rows.
+cudaError_t tc_product(const BackwardArgs& a, const void* A, const void* A_lo, const void* B, int N, int K, float* out,
+                       cudaStream_t s) {
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.epi = EPI_GATE_F32;
+  g.E = a.E + a.n_shared;
+  g.N = N;
+  g.K = K;
+  g.a_rows = a.s_max;
+  g.max_group_rows = a.max_group_rows;
+  g.A = A;
+  g.A2 = A_lo;
+  g.split = A_lo != nullptr;
+  g.B0 = B;
+  g.out = out;
+  g.ksplit = 1;
+  g.offsets = a.offsets;
+  g.mprefix = a.mprefix;
+  g.row_gate = a.ones;
+  g.row_token = a.row_token;
+  g.err = a.err;
+  TcGemmPlan plan;
+  const char* why = nullptr;
+  cudaError_t e = plan_gemm_tc(g, &plan, &why);
+  if (e != cudaSuccess) return e;
+  return launch_gemm_tc(plan, a.num_sms, s);
+}
+
+cudaError_t transpose(const void* in, void* out, int G, int R, int C, cudaStream_t s) {
+  const dim3 grid((C + 31) / 32, (R + 31) / 32, G);
+  bw_transpose_kernel<<<grid, dim3(32, 8), 0, s>>>(static_cast<const __nv_bfloat16*>(in),
+                                                   static_cast<__nv_bfloat16*>(out), R, C);
+  count_launch();
+  return cudaGetLastError();
 }
 
 template <typename TA, typename TB, bool KMAJOR, bool GATHER>
@@ -387,48 +487,77 @@ cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
                                                                                           a.cnt1);
   count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // a1 = W1 x, a3 = W3 x
-  RowGemm g{};
-  g.N = a.d_ff;
-  g.K0 = a.d;
-  g.A0 = a.Xp;
-  g.B0 = a.W1;
-  g.C = a.A1;
-  g.offsets = a.offsets;
-  g.row_token = a.row_token;
-  if ((e = rowgemm<XT, XT, true, false>(g, groups, a.max_group_rows, s)) != cudaSuccess) return e;
-  if (swiglu) {
-    g.B0 = a.W3;
-    g.C = a.A3;
+  const bool tc = a.x_is_bf16 != 0;
+  const int64_t plane = a.s_max * static_cast<int64_t>(a.d_ff);
+  if (tc) {
+    // K-major copies of the weights for the transposed products, dy in sorted rows
+    if ((e = transpose(a.W2, a.W2t, groups, a.d, a.d_ff, s)) != cudaSuccess) return e;
+    if ((e = transpose(a.W1, a.W1t, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
+    if (swiglu && (e = transpose(a.W3, a.W3t, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
+    bw_gather_dy_kernel<<<static_cast<unsigned>((a.s_max + 7) / 8), 256, 0, s>>>(
+        a.d, a.offsets, groups, a.row_token, static_cast<const uint4*>(a.dy), static_cast<uint4*>(a.dYs), a.ones);
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // a1 = W1 x, a3 = W3 x, u = W2^T dy
+    if ((e = tc_product(a, a.Xp, nullptr, a.W1, a.d_ff, a.d, a.A1, s)) != cudaSuccess) return e;
+    if (swiglu && (e = tc_product(a, a.Xp, nullptr, a.W3, a.d_ff, a.d, a.A3, s)) != cudaSuccess) return e;
+    if ((e = tc_product(a, a.dYs, nullptr, a.W2t, a.d_ff, a.d, a.U, s)) != cudaSuccess) return e;
+  } else {
+    // a1 = W1 x, a3 = W3 x
+    RowGemm g{};
+    g.N = a.d_ff;
+    g.K0 = a.d;
+    g.A0 = a.Xp;
+    g.B0 = a.W1;
+    g.C = a.A1;
+    g.offsets = a.offsets;
+    g.row_token = a.row_token;
     if ((e = rowgemm<XT, XT, true, false>(g, groups, a.max_group_rows, s)) != cudaSuccess) return e;
+    if (swiglu) {
+      g.B0 = a.W3;
+      g.C = a.A3;
+      if ((e = rowgemm<XT, XT, true, false>(g, groups, a.max_group_rows, s)) != cudaSuccess) return e;
+    }
+    // u = W2^T dy_t
+    g.K0 = a.d;
+    g.A0 = a.dy;
+    g.B0 = a.W2;
+    g.C = a.U;
+    if ((e = rowgemm<XT, XT, false, true>(g, groups, a.max_group_rows, s)) != cudaSuccess) return e;
   }
-  // u = W2^T dy_t
-  g.K0 = a.d;
-  g.A0 = a.dy;
-  g.B0 = a.W2;
-  g.C = a.U;
-  if ((e = rowgemm<XT, XT, false, true>(g, groups, a.max_group_rows, s)) != cudaSuccess) return e;
   // hidden activation, its gradients, dg
+  __nv_bfloat16* p1 = tc ? static_cast<__nv_bfloat16*>(a.dA1p) : nullptr;
+  __nv_bfloat16* p3 = tc && swiglu ? static_cast<__nv_bfloat16*>(a.dA3p) : nullptr;
   if (swiglu)
     bw_act_kernel<true><<<static_cast<unsigned>(a.s_max), THREADS, 0, s>>>(a.d_ff, a.offsets, groups, a.row_gate,
-                                                                            a.A1, a.A3, a.U, a.dg);
+                                                                            a.A1, a.A3, a.U, a.dg, p1, p3, plane);
   else
     bw_act_kernel<false><<<static_cast<unsigned>(a.s_max), THREADS, 0, s>>>(a.d_ff, a.offsets, groups, a.row_gate,
-                                                                             a.A1, a.A3, a.U, a.dg);
+                                                                             a.A1, a.A3, a.U, a.dg, p1, p3, plane);
   count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // dXp = W1^T da1 (+ W3^T da3)
-  RowGemm gx{};
-  gx.N = a.d;
-  gx.K0 = a.d_ff;
-  gx.K1 = swiglu ? a.d_ff : 0;
-  gx.A0 = a.U;
-  gx.A1 = a.A3;
-  gx.B0 = a.W1;
-  gx.B1 = a.W3;
-  gx.C = a.dXp;
-  gx.offsets = a.offsets;
-  if ((e = rowgemm<float, XT, false, false>(gx, groups, a.max_group_rows, s)) != cudaSuccess) return e;
+  int parts = 1;
+  if (tc) {
+    if ((e = tc_product(a, p1, p1 + plane, a.W1t, a.d, a.d_ff, a.dXp, s)) != cudaSuccess) return e;
+    if (swiglu) {
+      if ((e = tc_product(a, p3, p3 + plane, a.W3t, a.d, a.d_ff, a.dXp + a.s_max * a.d, s)) != cudaSuccess)
+        return e;
+      parts = 2;
+    }
+  } else {
+    RowGemm gx{};
+    gx.N = a.d;
+    gx.K0 = a.d_ff;
+    gx.K1 = swiglu ? a.d_ff : 0;
+    gx.A0 = a.U;
+    gx.A1 = a.A3;
+    gx.B0 = a.W1;
+    gx.B1 = a.W3;
+    gx.C = a.dXp;
+    gx.offsets = a.offsets;
+    if ((e = rowgemm<float, XT, false, false>(gx, groups, a.max_group_rows, s)) != cudaSuccess) return e;
+  }
   // weight gradients
   WGrad w{};
   w.offsets = a.offsets;
@@ -455,7 +584,7 @@ cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
   bw_router_kernel<XT><<<static_cast<unsigned>(a.T), THREADS, 0, s>>>(a);
   count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bw_dx_kernel<<<static_cast<unsigned>(a.T), THREADS, 0, s>>>(a);
+  bw_dx_kernel<<<static_cast<unsigned>(a.T), THREADS, 0, s>>>(a, parts);
   count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   WGrad wr{};

@@ -35,9 +35,20 @@ struct BackwardArgs {
   float* A3;    // [s_max][d_ff]: w3 x, then its gradient (SwiGLU)
   float* U;     // [s_max][d_ff]: W2^T dy, then the gradient of w1 x
   float* dg;    // [s_max]: gradient reaching each row's gate
-  float* dXp;   // [s_max][d]
+  float* dXp;   // [s_max][d] (bf16 SwiGLU layers: [2][s_max][d], the W1 and W3 parts)
   float* dh;    // [T][E]: gradient reaching the router logits
   int32_t* cnt1;  // [E]: first-choice counts
+  // bf16 layers: the row-grouped products run on the tensor cores
+  int num_sms;
+  unsigned int* err;       // device error word (bounded waits of the tensor-core GEMM)
+  const int32_t* mprefix;  // [E + n_shared + 1] m-tile prefix of the forward's scan
+  float* ones;             // [s_max] gate 1 for the fp32 epilogue
+  void* dYs;               // [s_max][d] bf16: dy rows in expert-sorted order
+  void* W1t;               // [E + n_shared][d][d_ff] bf16: W1 transposed per expert
+  void* W3t;               // same for W3 (SwiGLU)
+  void* W2t;               // [E + n_shared][d_ff][d] bf16: W2 transposed per expert
+  void* dA1p;              // [2][s_max][d_ff] bf16: hi and lo planes of the gradient of w1 x
+  void* dA3p;              // same for w3 x (SwiGLU)
   // outputs (fp32)
   float* dx;    // [T][d]
   float* dW_r;  // [E][d]

@@ -164,24 +164,37 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   return w;
 }
 
-// Scratch of the backward pass (fp32): A1, U [S][d_ff] (and A3 for SwiGLU),
-// dg [S], dXp [S][d], dh [T][E], cnt1 [E].
+// Scratch of the backward pass: fp32 A1, U [S][d_ff] (and A3 for SwiGLU),
+// dg [S], dXp [S][d], dh [T][E], cnt1 [E]; for bf16 layers (tensor-core
+// products) also gate 1 [S], bf16 dy rows [S][d], the transposed weights
+// [G][d][d_ff] / [G][d_ff][d], the hi + lo planes of da1 (and da3)
+// [2][S][d_ff], and a second dXp part for SwiGLU.
 struct BwLayout {
-  size_t A1, A3, U, dg, dXp, dh, cnt1, total;
+  size_t A1, A3, U, dg, dXp, dh, cnt1, ones, dYs, W1t, W3t, W2t, dA1p, dA3p, total;
 };
 
 BwLayout make_bw_layout(const moe_layer& L, const Layout& w) {
   BwLayout b;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
-  const size_t hid = sizeof(float) * static_cast<size_t>(w.s_max) * L.d_ff;
+  const bool swiglu = L.act == MOE_ACT_SWIGLU, tc = L.dtype == MOE_BF16;
+  const size_t S = static_cast<size_t>(w.s_max), G = static_cast<size_t>(L.E + L.n_shared);
+  const size_t hid = sizeof(float) * S * L.d_ff;
   b.A1 = take(hid);
-  b.A3 = take(L.act == MOE_ACT_SWIGLU ? hid : 0);
+  b.A3 = take(swiglu ? hid : 0);
   b.U = take(hid);
-  b.dg = take(sizeof(float) * static_cast<size_t>(w.s_max));
-  b.dXp = take(sizeof(float) * static_cast<size_t>(w.s_max) * L.d);
+  b.dg = take(sizeof(float) * S);
+  b.dXp = take(sizeof(float) * S * L.d * (tc && swiglu ? 2 : 1));
   b.dh = take(sizeof(float) * static_cast<size_t>(w.T) * L.E);
   b.cnt1 = take(sizeof(int32_t) * L.E);
+  const size_t wsz = tc ? 2 * G * L.d * static_cast<size_t>(L.d_ff) : 0;
+  b.ones = take(tc ? sizeof(float) * S : 0);
+  b.dYs = take(tc ? 2 * S * L.d : 0);
+  b.W1t = take(wsz);
+  b.W3t = take(swiglu ? wsz : 0);
+  b.W2t = take(wsz);
+  b.dA1p = take(tc ? 2 * 2 * S * L.d_ff : 0);
+  b.dA3p = take(tc && swiglu ? 2 * 2 * S * L.d_ff : 0);
   b.total = o;
   return b;
 }
@@ -582,6 +595,13 @@ int moe_backward(moe_handle h, int64_t T, const void* x, const float* W_r, const
                 "moe_backward: backward workspace missing or smaller than moe_backward_workspace_bytes()");
   if (((reinterpret_cast<uintptr_t>(workspace) | reinterpret_cast<uintptr_t>(bw_workspace)) & 255) != 0)
     return fail(MOE_ERR_INVALID_ARG, "moe_backward: workspaces must be 256-byte aligned");
+  const uintptr_t al = reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy) |
+                       reinterpret_cast<uintptr_t>(W1) | reinterpret_cast<uintptr_t>(W2) |
+                       reinterpret_cast<uintptr_t>(W3);
+  if ((al & 15) != 0) return fail(MOE_ERR_INVALID_ARG, "moe_backward: x, dy and weights must be 16-byte aligned");
+  DeviceInfo* di = nullptr;
+  cudaError_t de = device_info(&di);
+  if (de != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_backward: ") + cudaGetErrorString(de));
 
   const uint8_t* ws = static_cast<const uint8_t*>(workspace);
   uint8_t* bw = static_cast<uint8_t*>(bw_workspace);
@@ -624,6 +644,18 @@ int moe_backward(moe_handle h, int64_t T, const void* x, const float* W_r, const
   a.dXp = reinterpret_cast<float*>(bw + b.dXp);
   a.dh = reinterpret_cast<float*>(bw + b.dh);
   a.cnt1 = reinterpret_cast<int32_t*>(bw + b.cnt1);
+  a.num_sms = di->num_sms;
+  a.err = di->err;
+  a.mprefix = reinterpret_cast<const int32_t*>(ws + w.mprefix);
+  if (L.dtype == MOE_BF16) {
+    a.ones = reinterpret_cast<float*>(bw + b.ones);
+    a.dYs = bw + b.dYs;
+    a.W1t = bw + b.W1t;
+    a.W3t = swiglu ? bw + b.W3t : nullptr;
+    a.W2t = bw + b.W2t;
+    a.dA1p = bw + b.dA1p;
+    a.dA3p = swiglu ? bw + b.dA3p : nullptr;
+  }
   a.dx = dx;
   a.dW_r = dW_r;
   a.db_r = db_r;
