@@ -461,17 +461,22 @@ def main():
     return 0
 
 
-def backward_flops(w, S, T):
-    """(row-product FLOPs, weight-gradient and router FLOPs) of the backward
-    pass for S kept rows (shared rows included).  Per row and d x d_ff
-    contraction 2 d d_ff: the row products are w1 x again, W2^T dy and dXp
-    (ReLU: 3; SwiGLU: w3 x and a second dXp term, 5) -- on the tensor cores for
-    bf16 layers; the weight gradients dW2, dW1 (and dW3) on the CUDA cores,
-    with the router's 3 T E d contractions (logits again, W_r^T dh, dW_r)."""
-    rows = 5 if w.act == 1 else 3
-    wgr = 3 if w.act == 1 else 2
-    c = 2.0 * S * w.d * w.d_ff
-    return c * rows, c * wgr + 3 * 2.0 * T * w.E * w.d
+def backward_work(w, S, T, active):
+    """Algorithmic work of the backward pass for S kept rows (shared rows
+    included) and `active` experts with rows.  FLOPs: per row and d x d_ff
+    contraction 2 d d_ff, 5 of them for ReLU (w1 x again, W2^T dy, dXp, dW2,
+    dW1) and 8 for SwiGLU (w3 x, a second dXp term, dW3 more), plus the
+    router's 3 T E d (logits again, W_r^T dh, dW_r).  Bytes: the active
+    experts' weights read once, the fp32 weight gradients of every expert
+    written once (zeros where no row came), x and dy read, dx and dW_r written."""
+    swiglu = w.act == 1
+    n_sh = getattr(w, "n_shared", 0)
+    flops = 2.0 * S * w.d * w.d_ff * (8 if swiglu else 5) + 3 * 2.0 * T * w.E * w.d
+    elt = 2 if w.dtype == 1 else 4
+    nproj = 3 if swiglu else 2
+    per = nproj * w.d * w.d_ff
+    nbytes = (active * per * elt + (w.E + n_sh) * per * 4 + 2 * T * w.d * elt + T * w.d * 4 + w.E * w.d * 4)
+    return flops, nbytes
 
 
 def backward_bench(args, w, inp, warmup, world, rank, local, dev):
@@ -535,14 +540,21 @@ def backward_bench(args, w, inp, warmup, world, rank, local, dev):
     cap = layer.capacity(w.T)
     kept = sum(c if cap is None else min(c, cap) for c in counts.cpu().tolist())
     S = kept + w.n_shared * w.T
-    fl_rows, fl_alu = backward_flops(w, S, w.T)
-    if w.dtype != 1:  # fp32 layers: every product on the CUDA cores
-        fl_rows, fl_alu = 0.0, fl_rows + fl_alu
+    active = sum(1 for c in counts.cpu().tolist() if c > 0) + w.n_shared
+    fl, nb = backward_work(w, S, w.T, active)
     clocks = sampler.summary(wall0, wall1)
-    peak = 148 * 128 * 2 * (clocks["sm_max_mhz"] or 1965.0) * 1e6 / 1e12  # fp32 FMA lanes x 2 x max clock
-    peaks, _ = load_peaks()
-    floor_s = fl_rows / (peaks["bf16_tflops"] * 1e12) + fl_alu / (peak * 1e12)
-    ach = fl_alu / (bw_s / K) / 1e12
+    peaks, peak_src = load_peaks()
+    t_bw = bw_s / K
+    if w.dtype == 1:  # bf16: every product on the tensor cores
+        roof = kernel_roofline(fl, nb, t_bw, peaks)
+        roof["peak_source"] = f"{peak_src} ({'bf16_tflops' if roof['bound'] == 'tensor' else 'hbm_gbs'}, burst)"
+    else:  # fp32: every product on the CUDA cores
+        peak = 148 * 128 * 2 * (clocks["sm_max_mhz"] or 1965.0) * 1e6 / 1e12  # fp32 FMA lanes x 2 x max clock
+        ach = fl / t_bw / 1e12
+        roof = {"bound": "alu", "achieved": round(ach, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+                "frac": round(ach / peak, 4), "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x clocks.max.sm"}
+    roof["kernel"] = "backward pass (all its launches)"
+    roof["traffic"] = None
     line = {
         "metric": "MoE-layer training step (forward + backward) tokens/s on 1 B200",
         "value": round(w.T * K / step_s, 1),
@@ -555,16 +567,11 @@ def backward_bench(args, w, inp, warmup, world, rank, local, dev):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32 (backward), " + ("bf16" if w.dtype == 1 else "f32") + " (forward)",
+        "dtype": "bf16" if w.dtype == 1 else "f32",  # operands of the products (bf16 as hi + lo pairs where fp32-derived)
         "data": "synthetic (seeded; shapes and distributions of the workload, random-init weights)",
         "config": dict(config_of(w, 1), hidden=args.hidden, loss="<dy, y> + 0.01 aux + 1e-3 z"),
-        # the CUDA-core weight gradients bound the step: their FLOPs over the whole backward time
-        "roofline": {"bound": "alu", "achieved": round(ach, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
-                     "frac": round(ach / peak, 4),
-                     "kernel": "backward pass (weight gradients on CUDA cores; row products on tensor cores)",
-                     "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x clocks.max.sm", "traffic": None},
-        "backward_floor": {"tensor_flops": fl_rows, "alu_flops": fl_alu, "floor_ms": round(floor_s * 1e3, 4),
-                           "frac": round(floor_s / (bw_s / K), 4)},
+        "roofline": roof,
+        "backward_work": {"flops": fl, "bytes": nb, "kept_rows": S, "active_experts": active},
         "gpu_launches": int(n_launch),
         "clocks": clocks,
     }

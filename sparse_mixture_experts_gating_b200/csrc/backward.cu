@@ -33,6 +33,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
+
 #include "backward.h"
 #include "common.cuh"
 #include "internal.h"
@@ -389,14 +391,15 @@ __global__ void __launch_bounds__(THREADS) bw_db_kernel(int64_t T, int E, const 
   if (threadIdx.x == 0) db[e] = tot;
 }
 
-// out[g][c][r] = in[g][r][c] for bf16 matrices [G][R][C] (32 x 32 tiles).
-__global__ void __launch_bounds__(256) bw_transpose_kernel(const __nv_bfloat16* __restrict__ in,
-                                                           __nv_bfloat16* __restrict__ out, int R, int C) {
-  __shared__ __nv_bfloat16 tile[32][34];
+// out[g][c][r] = in[g][r][c] for matrices [G][R][C] (32 x 32 tiles).
+template <typename T>
+__global__ void __launch_bounds__(256) bw_transpose_kernel(const T* __restrict__ in, T* __restrict__ out, int R,
+                                                           int C) {
+  __shared__ T tile[32][34];
   const int64_t g = blockIdx.z;
   const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
-  const __nv_bfloat16* src = in + g * R * C;
-  __nv_bfloat16* dst = out + g * R * C;
+  const T* src = in + g * R * C;
+  T* dst = out + g * R * C;
   for (int i = threadIdx.y; i < 32; i += 8) {
     const int r = r0 + i, c = c0 + threadIdx.x;
     if (r < R && c < C) tile[i][threadIdx.x] = src[static_cast<int64_t>(r) * C + c];
@@ -408,40 +411,38 @@ __global__ void __launch_bounds__(256) bw_transpose_kernel(const __nv_bfloat16* 
   }
 }
 
-// dy rows into expert-sorted order (a warp per row, 16-byte copies) and the
-// gate 1 of every row for the fp32 epilogue.
+// dy rows into expert-sorted order (a warp per row, 16-byte copies).
 __global__ void __launch_bounds__(256) bw_gather_dy_kernel(int d, const int32_t* offsets, int groups,
-                                                           const int32_t* row_token, const uint4* dy, uint4* dYs,
-                                                           float* ones) {
+                                                           const int32_t* row_token, const uint4* dy, uint4* dYs) {
   const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= offsets[groups]) return;
   const int nv = d / 8;  // 16-byte groups of a bf16 row
   const int64_t t = row_token[r];
   for (int v = lane; v < nv; v += 32) dYs[r * nv + v] = dy[t * nv + v];
-  if (lane == 0) ones[r] = 1.f;
 }
 
 // One tensor-core grouped GEMM with the fp32 epilogue (gate 1):
 // out[r][n] = sum_k A[r][k] B_e[n][k] over the expert-sorted rows.
 cudaError_t tc_product(const BackwardArgs& a, const void* A, const void* A_lo, const void* B, int N, int K, float* out,
-                       cudaStream_t s) {
+                       cudaStream_t s, const int32_t* offsets = nullptr, const int32_t* mprefix = nullptr,
+                       int64_t a_rows = 0, int max_rows = 0) {
   GemmArgs g;
   memset(&g, 0, sizeof(g));
   g.epi = EPI_GATE_F32;
   g.E = a.E + a.n_shared;
   g.N = N;
   g.K = K;
-  g.a_rows = a.s_max;
-  g.max_group_rows = a.max_group_rows;
+  g.a_rows = offsets != nullptr ? a_rows : a.s_max;
+  g.max_group_rows = offsets != nullptr ? max_rows : a.max_group_rows;
   g.A = A;
   g.A2 = A_lo;
   g.split = A_lo != nullptr;
   g.B0 = B;
   g.out = out;
   g.ksplit = 1;
-  g.offsets = a.offsets;
-  g.mprefix = a.mprefix;
+  g.offsets = offsets != nullptr ? offsets : a.offsets;
+  g.mprefix = offsets != nullptr ? mprefix : a.mprefix;
   g.row_gate = a.ones;
   g.row_token = a.row_token;
   g.err = a.err;
@@ -452,12 +453,70 @@ cudaError_t tc_product(const BackwardArgs& a, const void* A, const void* A_lo, c
   return launch_gemm_tc(plan, a.num_sms, s);
 }
 
+template <typename T>
 cudaError_t transpose(const void* in, void* out, int G, int R, int C, cudaStream_t s) {
   const dim3 grid((C + 31) / 32, (R + 31) / 32, G);
-  bw_transpose_kernel<<<grid, dim3(32, 8), 0, s>>>(static_cast<const __nv_bfloat16*>(in),
-                                                   static_cast<__nv_bfloat16*>(out), R, C);
+  bw_transpose_kernel<T><<<grid, dim3(32, 8), 0, s>>>(static_cast<const T*>(in), static_cast<T*>(out), R, C);
   count_launch();
   return cudaGetLastError();
+}
+
+// Per-expert operand of a weight gradient: out[e][f][kk] = v(off_e + kk, f)
+// for kk below the group's row count, 0 up to k_pad, where v(r, f) =
+// src[r][f] (times scale[r] when given); bf16, with SPLIT a lo plane at
+// out + plane holding v - hi.  32 x 32 tiles: rows read along f, written
+// along kk.
+template <typename ST, bool SPLIT>
+__global__ void __launch_bounds__(256) bw_pack_kernel(const ST* __restrict__ src, int F,
+                                                      const int32_t* __restrict__ offsets,
+                                                      const float* __restrict__ scale, int k_pad,
+                                                      __nv_bfloat16* __restrict__ out, int64_t plane) {
+  __shared__ float tile[32][33];
+  const int e = blockIdx.z;
+  const int f0 = blockIdx.x * 32, k0 = blockIdx.y * 32;
+  const int64_t off = offsets[e];
+  const int rows = static_cast<int>(offsets[e + 1] - off);
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int kk = k0 + i, f = f0 + threadIdx.x;
+    float v = 0.f;
+    if (kk < rows && f < F) {
+      v = to_f32(src[(off + kk) * F + f]);
+      if (scale != nullptr) v *= scale[off + kk];
+    }
+    tile[i][threadIdx.x] = v;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int f = f0 + i, kk = k0 + threadIdx.x;
+    if (f < F && kk < k_pad) {
+      const float v = tile[threadIdx.x][i];
+      const int64_t o = (static_cast<int64_t>(e) * F + f) * k_pad + kk;
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      out[o] = h;
+      if (SPLIT) out[plane + o] = __float2bfloat16_rn(v - __bfloat162float(h));
+    }
+  }
+}
+
+template <typename ST, bool SPLIT>
+cudaError_t pack(const void* src, int F, const int32_t* offsets, const float* scale, int G, int k_pad, void* out,
+                 int64_t plane, cudaStream_t s) {
+  const dim3 grid((F + 31) / 32, (k_pad + 31) / 32, G);
+  bw_pack_kernel<ST, SPLIT><<<grid, dim3(32, 8), 0, s>>>(static_cast<const ST*>(src), F, offsets, scale, k_pad,
+                                                         static_cast<__nv_bfloat16*>(out), plane);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// Gate 1 for n rows, and the group tables of the per-expert products
+// (groups of F rows each: offsets e F, m-tile prefix e ceil(F / 128)).
+__global__ void bw_tables_kernel(int64_t n, float* ones, int G, int F, int32_t* woff, int32_t* wpre) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  if (i < n) ones[i] = 1.f;
+  if (i <= G) {
+    woff[i] = static_cast<int32_t>(i * F);
+    wpre[i] = static_cast<int32_t>(i * ((F + kTileM - 1) / kTileM));
+  }
 }
 
 template <typename TA, typename TB, bool KMAJOR, bool GATHER>
@@ -491,11 +550,16 @@ cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
   const int64_t plane = a.s_max * static_cast<int64_t>(a.d_ff);
   if (tc) {
     // K-major copies of the weights for the transposed products, dy in sorted rows
-    if ((e = transpose(a.W2, a.W2t, groups, a.d, a.d_ff, s)) != cudaSuccess) return e;
-    if ((e = transpose(a.W1, a.W1t, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
-    if (swiglu && (e = transpose(a.W3, a.W3t, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
+    if ((e = transpose<__nv_bfloat16>(a.W2, a.W2t, groups, a.d, a.d_ff, s)) != cudaSuccess) return e;
+    if ((e = transpose<__nv_bfloat16>(a.W1, a.W1t, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
+    if (swiglu && (e = transpose<__nv_bfloat16>(a.W3, a.W3t, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
+    const int64_t n_ones = std::max<int64_t>(a.s_max, static_cast<int64_t>(groups) * a.d_ff);
+    bw_tables_kernel<<<static_cast<unsigned>((std::max<int64_t>(n_ones, groups + 1) + 255) / 256), 256, 0, s>>>(
+        n_ones, a.ones, groups, a.d_ff, a.woff, a.wpre);
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bw_gather_dy_kernel<<<static_cast<unsigned>((a.s_max + 7) / 8), 256, 0, s>>>(
-        a.d, a.offsets, groups, a.row_token, static_cast<const uint4*>(a.dy), static_cast<uint4*>(a.dYs), a.ones);
+        a.d, a.offsets, groups, a.row_token, static_cast<const uint4*>(a.dy), static_cast<uint4*>(a.dYs));
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // a1 = W1 x, a3 = W3 x, u = W2^T dy
@@ -559,6 +623,32 @@ cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
     if ((e = rowgemm<float, XT, false, false>(gx, groups, a.max_group_rows, s)) != cudaSuccess) return e;
   }
   // weight gradients
+  if (tc) {
+    // per expert: dW1_e = da1^T x, dW3_e = da3^T x, dW2_e^T = (g hid)^T dy over
+    // its rows, zero-padded to k_pad, as products of F-row groups
+    const int kp = a.k_pad;
+    const int64_t pl = static_cast<int64_t>(groups) * a.d_ff * kp;  // between the hi and lo planes
+    const int64_t arows = static_cast<int64_t>(groups) * a.d_ff;
+    auto* P1 = static_cast<__nv_bfloat16*>(a.P1);
+    auto* P3 = static_cast<__nv_bfloat16*>(a.P3);
+    auto* PH = static_cast<__nv_bfloat16*>(a.PH);
+    if ((e = pack<__nv_bfloat16, false>(a.Xp, a.d, a.offsets, nullptr, groups, kp, a.XT, 0, s)) != cudaSuccess)
+      return e;
+    if ((e = pack<__nv_bfloat16, false>(a.dYs, a.d, a.offsets, nullptr, groups, kp, a.DT, 0, s)) != cudaSuccess)
+      return e;
+    if ((e = pack<float, true>(a.U, a.d_ff, a.offsets, nullptr, groups, kp, P1, pl, s)) != cudaSuccess) return e;
+    if ((e = pack<float, true>(a.A1, a.d_ff, a.offsets, a.row_gate, groups, kp, PH, pl, s)) != cudaSuccess) return e;
+    if ((e = tc_product(a, P1, P1 + pl, a.XT, a.d, kp, a.dW1, s, a.woff, a.wpre, arows, a.d_ff)) != cudaSuccess)
+      return e;
+    if (swiglu) {
+      if ((e = pack<float, true>(a.A3, a.d_ff, a.offsets, nullptr, groups, kp, P3, pl, s)) != cudaSuccess) return e;
+      if ((e = tc_product(a, P3, P3 + pl, a.XT, a.d, kp, a.dW3, s, a.woff, a.wpre, arows, a.d_ff)) != cudaSuccess)
+        return e;
+    }
+    if ((e = tc_product(a, PH, PH + pl, a.DT, a.d, kp, a.dW2t, s, a.woff, a.wpre, arows, a.d_ff)) != cudaSuccess)
+      return e;
+    if ((e = transpose<float>(a.dW2t, a.dW2, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
+  } else {
   WGrad w{};
   w.offsets = a.offsets;
   w.row_token = a.row_token;
@@ -579,6 +669,7 @@ cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
     w.P = a.A3;
     w.C = a.dW3;
     if ((e = wgrad<float, XT, false>(w, groups, s)) != cudaSuccess) return e;
+  }
   }
   // router: dh, then dx, dW_r, db_r
   bw_router_kernel<XT><<<static_cast<unsigned>(a.T), THREADS, 0, s>>>(a);

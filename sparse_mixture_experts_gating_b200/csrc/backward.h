@@ -42,13 +42,24 @@ struct BackwardArgs {
   int num_sms;
   unsigned int* err;       // device error word (bounded waits of the tensor-core GEMM)
   const int32_t* mprefix;  // [E + n_shared + 1] m-tile prefix of the forward's scan
-  float* ones;             // [s_max] gate 1 for the fp32 epilogue
+  float* ones;             // [max(s_max, G d_ff)] gate 1 for the fp32 epilogue
   void* dYs;               // [s_max][d] bf16: dy rows in expert-sorted order
   void* W1t;               // [E + n_shared][d][d_ff] bf16: W1 transposed per expert
   void* W3t;               // same for W3 (SwiGLU)
   void* W2t;               // [E + n_shared][d_ff][d] bf16: W2 transposed per expert
   void* dA1p;              // [2][s_max][d_ff] bf16: hi and lo planes of the gradient of w1 x
   void* dA3p;              // same for w3 x (SwiGLU)
+  // bf16 layers: the weight gradients as per-expert products over K_pad
+  // (every expert's rows, zero-padded to the same count) on the tensor cores
+  int k_pad;               // max_group_rows rounded up to 8
+  void* P1;                // [2][G][d_ff][k_pad] bf16 planes: da1 per expert, transposed
+  void* P3;                // same for da3 (SwiGLU)
+  void* PH;                // same for g * hid
+  void* XT;                // [G][d][k_pad] bf16: Xp per expert, transposed
+  void* DT;                // [G][d][k_pad] bf16: dy (sorted rows) per expert, transposed
+  float* dW2t;             // [G][d_ff][d] fp32: dW2 transposed
+  int32_t* woff;           // [G + 1] rows of the per-expert products: e * d_ff
+  int32_t* wpre;           // [G + 1] their m-tile prefix: e * ceil(d_ff / 128)
   // outputs (fp32)
   float* dx;    // [T][d]
   float* dW_r;  // [E][d]

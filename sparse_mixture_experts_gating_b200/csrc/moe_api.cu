@@ -170,8 +170,18 @@ Layout make_layout(const moe_layer& L, int64_t T) {
 // [G][d][d_ff] / [G][d_ff][d], the hi + lo planes of da1 (and da3)
 // [2][S][d_ff], and a second dXp part for SwiGLU.
 struct BwLayout {
-  size_t A1, A3, U, dg, dXp, dh, cnt1, ones, dYs, W1t, W3t, W2t, dA1p, dA3p, total;
+  size_t A1, A3, U, dg, dXp, dh, cnt1, ones, dYs, W1t, W3t, W2t, dA1p, dA3p, P1, P3, PH, XT, DT, dW2t, woff, wpre,
+      total;
+  int max_group_rows, k_pad;
 };
+
+// No group has more rows: a token takes an expert at most once, and a shared
+// expert's group has T rows.
+int64_t max_group_rows_of(const moe_layer& L, const Layout& w) {
+  int64_t mg = w.T;
+  if (L.n_shared == 0 && w.capacity >= 0 && w.capacity < mg) mg = w.capacity;
+  return mg;
+}
 
 BwLayout make_bw_layout(const moe_layer& L, const Layout& w) {
   BwLayout b;
@@ -188,13 +198,26 @@ BwLayout make_bw_layout(const moe_layer& L, const Layout& w) {
   b.dh = take(sizeof(float) * static_cast<size_t>(w.T) * L.E);
   b.cnt1 = take(sizeof(int32_t) * L.E);
   const size_t wsz = tc ? 2 * G * L.d * static_cast<size_t>(L.d_ff) : 0;
-  b.ones = take(tc ? sizeof(float) * S : 0);
+  b.max_group_rows = static_cast<int>(max_group_rows_of(L, w));
+  b.k_pad = (b.max_group_rows + 7) / 8 * 8;
+  const size_t kp = static_cast<size_t>(b.k_pad);
+  b.ones = take(tc ? sizeof(float) * std::max(S, G * static_cast<size_t>(L.d_ff)) : 0);
   b.dYs = take(tc ? 2 * S * L.d : 0);
   b.W1t = take(wsz);
   b.W3t = take(swiglu ? wsz : 0);
   b.W2t = take(wsz);
   b.dA1p = take(tc ? 2 * 2 * S * L.d_ff : 0);
   b.dA3p = take(tc && swiglu ? 2 * 2 * S * L.d_ff : 0);
+  // the weight gradients' per-expert operands (rows zero-padded to k_pad)
+  const size_t plane2 = tc ? 2 * 2 * G * L.d_ff * kp : 0;
+  b.P1 = take(plane2);
+  b.P3 = take(swiglu ? plane2 : 0);
+  b.PH = take(plane2);
+  b.XT = take(tc ? 2 * G * L.d * kp : 0);
+  b.DT = take(tc ? 2 * G * L.d * kp : 0);
+  b.dW2t = take(tc ? sizeof(float) * G * L.d * static_cast<size_t>(L.d_ff) : 0);
+  b.woff = take(tc ? sizeof(int32_t) * (G + 1) : 0);
+  b.wpre = take(tc ? sizeof(int32_t) * (G + 1) : 0);
   b.total = o;
   return b;
 }
@@ -616,10 +639,8 @@ int moe_backward(moe_handle h, int64_t T, const void* x, const float* W_r, const
   a.gate_mode = L.gate_mode;
   a.n_shared = L.n_shared;
   a.x_is_bf16 = L.dtype == MOE_BF16;
-  // a token takes an expert at most once, a shared expert's group has T rows
-  int64_t mg = T;
-  if (L.n_shared == 0 && w.capacity >= 0 && w.capacity < mg) mg = w.capacity;
-  a.max_group_rows = static_cast<int>(mg);
+  a.max_group_rows = b.max_group_rows;
+  a.k_pad = b.k_pad;
   a.s_max = w.s_max;
   a.x = x;
   a.W_r = W_r;
@@ -655,6 +676,14 @@ int moe_backward(moe_handle h, int64_t T, const void* x, const float* W_r, const
     a.W2t = bw + b.W2t;
     a.dA1p = bw + b.dA1p;
     a.dA3p = swiglu ? bw + b.dA3p : nullptr;
+    a.P1 = bw + b.P1;
+    a.P3 = swiglu ? bw + b.P3 : nullptr;
+    a.PH = bw + b.PH;
+    a.XT = bw + b.XT;
+    a.DT = bw + b.DT;
+    a.dW2t = reinterpret_cast<float*>(bw + b.dW2t);
+    a.woff = reinterpret_cast<int32_t*>(bw + b.woff);
+    a.wpre = reinterpret_cast<int32_t*>(bw + b.wpre);
   }
   a.dx = dx;
   a.dW_r = dW_r;
