@@ -240,8 +240,10 @@ MOE_API int moe_forward_static(moe_handle h, int64_t T, const void* x, const flo
  * which must hold the moe_forward call of the same handle, T and inputs,
  * issued earlier on `stream` with nothing written to it since (the
  * moe_forward_static scratch cannot serve).  A dropped assignment passes no
- * gradient; shared experts get gate 1.  Arithmetic in fp32 on CUDA cores,
- * every sum in a fixed order (deterministic).
+ * gradient; shared experts get gate 1.  bf16 layers: every product on the
+ * tensor cores (bf16 operands, fp32-derived ones as hi + lo bf16 pairs, fp32
+ * accumulation); fp32 layers: fp32 on CUDA cores.  Every sum runs in a fixed
+ * order (deterministic).
  *   x, W1, W3, W2, dy in the layer's dtype (dy [T][d] like y); W_r, b_r fp32.
  *   Outputs, fp32, overwritten: dx [T][d], dW_r [E][d], db_r [E] (NULL: not
  *   wanted), dW1 / dW3 [E + n_shared][d_ff][d] (dW3 NULL for ReLU),
