@@ -53,10 +53,14 @@ __device__ __forceinline__ float ldf(const T* p, int64_t i) {
   return to_f32(p[i]);
 }
 
-__device__ __forceinline__ void group_rows(const int32_t* offsets, int e, int64_t single_rows, int64_t& r0,
-                                           int64_t& r1) {
-  if (offsets == nullptr) { r0 = 0; r1 = single_rows; }
-  else { r0 = offsets[e]; r1 = offsets[e + 1]; }
+// Rows of group e; without offsets, one group of single_rows rows cut into
+// chunks of `chunk` rows (0: whole), e being the chunk.
+__device__ __forceinline__ void group_rows(const int32_t* offsets, int e, int64_t single_rows, int64_t chunk,
+                                           int64_t& r0, int64_t& r1) {
+  if (offsets != nullptr) { r0 = offsets[e]; r1 = offsets[e + 1]; return; }
+  if (chunk <= 0) { r0 = 0; r1 = single_rows; return; }
+  r0 = e * chunk;
+  r1 = r0 + chunk < single_rows ? r0 + chunk : single_rows;
 }
 
 // 4 x 4 outputs per thread from shared tiles As[TK][TM], Bs[TK][TN].
@@ -97,7 +101,7 @@ __global__ void __launch_bounds__(THREADS) bw_rowgemm_kernel(RowGemm g) {
   __shared__ float Bs[TK][TN + 4];
   const int e = blockIdx.z;
   int64_t g0, g1;
-  group_rows(g.offsets, e, 0, g0, g1);
+  group_rows(g.offsets, e, 0, 0, g0, g1);
   const int64_t r0 = g0 + static_cast<int64_t>(blockIdx.y) * TM;
   if (r0 >= g1) return;
   const int n0 = blockIdx.x * TN;
@@ -158,11 +162,12 @@ __global__ void __launch_bounds__(THREADS) bw_rowgemm_kernel(RowGemm g) {
 // Gradient of a weight per group: C_e[m][n] = sum over the rows r of group e
 // of P(r, m) Q(r, n), rows in order; P(r, m) = P[pr * M + m] (times
 // row_gate[r] and pr = row_token[r] with GATHER_SCALE, else pr = r),
-// Q(r, n) = Q[r * N + n].  offsets NULL: one group of `rows` rows.  Groups
-// without rows get zeros.
+// Q(r, n) = Q[r * N + n].  offsets NULL: one group of `rows` rows, cut into
+// chunks of `chunk` rows whose partial products go to C + chunk * M * N (0:
+// whole).  Groups without rows get zeros.
 struct WGrad {
   int M, N;
-  int64_t rows;
+  int64_t rows, chunk;
   const void* P;
   const void* Q;
   float* C;  // [groups][M][N]
@@ -177,7 +182,7 @@ __global__ void __launch_bounds__(THREADS) bw_wgrad_kernel(WGrad g) {
   __shared__ float Bs[TK][TN + 4];
   const int e = blockIdx.z;
   int64_t g0, g1;
-  group_rows(g.offsets, e, g.rows, g0, g1);
+  group_rows(g.offsets, e, g.rows, g.chunk, g0, g1);
   const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const TP* P = static_cast<const TP*>(g.P);
@@ -383,6 +388,15 @@ __global__ void __launch_bounds__(THREADS) bw_dx_kernel(BackwardArgs a, int part
   }
 }
 
+// out[i] = sum over z < nz of part[z * n + i], z in order.
+__global__ void bw_sum_parts_kernel(int64_t n, int nz, const float* __restrict__ part, float* __restrict__ out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  if (i >= n) return;
+  float v = 0.f;
+  for (int z = 0; z < nz; ++z) v += part[z * n + i];
+  out[i] = v;
+}
+
 // db_e = sum over tokens of dh[t][e], tokens in a fixed order.
 __global__ void __launch_bounds__(THREADS) bw_db_kernel(int64_t T, int E, const float* dh, float* db) {
   __shared__ float s_red[THREADS / 32];
@@ -453,6 +467,44 @@ cudaError_t tc_product(const BackwardArgs& a, const void* A, const void* A_lo, c
   cudaError_t e = plan_gemm_tc(g, &plan, &why);
   if (e != cudaSuccess) return e;
   return launch_gemm_tc(plan, a.num_sms, s);
+}
+
+// bf16 [G][R][C] -> [G][C][R] with R and C even: 64 x 64 tiles, pairs of
+// columns read and pairs of rows written as 4-byte words.
+__global__ void __launch_bounds__(256) bw_transpose_bf16x2_kernel(const __nv_bfloat16* __restrict__ in,
+                                                                  __nv_bfloat16* __restrict__ out, int R, int C) {
+  __shared__ __nv_bfloat16 tile[64][66];
+  const int64_t g = blockIdx.z;
+  const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const __nv_bfloat16* src = in + g * R * C;
+  __nv_bfloat16* dst = out + g * R * C;
+  for (int i = ty; i < 64; i += 8) {
+    const int r = r0 + i, c = c0 + 2 * tx;
+    if (r < R && c < C) {
+      const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(src + static_cast<int64_t>(r) * C + c);
+      tile[i][2 * tx] = v.x;
+      tile[i][2 * tx + 1] = v.y;
+    }
+  }
+  __syncthreads();
+  for (int i = ty; i < 64; i += 8) {
+    const int c = c0 + i, r = r0 + 2 * tx;
+    if (c < C && r < R) {
+      __nv_bfloat162 v;
+      v.x = tile[2 * tx][i];
+      v.y = tile[2 * tx + 1][i];
+      *reinterpret_cast<__nv_bfloat162*>(dst + static_cast<int64_t>(c) * R + r) = v;
+    }
+  }
+}
+
+cudaError_t transpose_bf16(const void* in, void* out, int G, int R, int C, cudaStream_t s) {
+  const dim3 grid((C + 63) / 64, (R + 63) / 64, G);
+  bw_transpose_bf16x2_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(in),
+                                                  static_cast<__nv_bfloat16*>(out), R, C);
+  count_launch();
+  return cudaGetLastError();
 }
 
 template <typename T>
@@ -552,9 +604,9 @@ cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
   const int64_t plane = a.s_max * static_cast<int64_t>(a.d_ff);
   if (tc) {
     // K-major copies of the weights for the transposed products, dy in sorted rows
-    if ((e = transpose<__nv_bfloat16>(a.W2, a.W2t, groups, a.d, a.d_ff, s)) != cudaSuccess) return e;
-    if ((e = transpose<__nv_bfloat16>(a.W1, a.W1t, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
-    if (swiglu && (e = transpose<__nv_bfloat16>(a.W3, a.W3t, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
+    if ((e = transpose_bf16(a.W2, a.W2t, groups, a.d, a.d_ff, s)) != cudaSuccess) return e;
+    if ((e = transpose_bf16(a.W1, a.W1t, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
+    if (swiglu && (e = transpose_bf16(a.W3, a.W3t, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
     const int64_t n_ones = std::max<int64_t>(a.s_max, static_cast<int64_t>(groups) * a.d_ff);
     bw_tables_kernel<<<static_cast<unsigned>((std::max<int64_t>(n_ones, groups + 1) + 255) / 256), 256, 0, s>>>(
         n_ones, a.ones, groups, a.d_ff, a.woff, a.wpre);
@@ -680,14 +732,20 @@ cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
   bw_dx_kernel<<<static_cast<unsigned>(a.T), THREADS, 0, s>>>(a, parts);
   count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // dW_r = sum_t dh_t x_t^T: K = T cut into a.wr_chunks chunks of partials, summed in order
   WGrad wr{};
   wr.M = a.E;
   wr.N = a.d;
   wr.rows = a.T;
+  wr.chunk = (a.T + a.wr_chunks - 1) / a.wr_chunks;
   wr.P = a.dh;
   wr.Q = a.x;
-  wr.C = a.dW_r;
-  if ((e = wgrad<float, XT, false>(wr, 1, s)) != cudaSuccess) return e;
+  wr.C = a.wr_part;
+  if ((e = wgrad<float, XT, false>(wr, a.wr_chunks, s)) != cudaSuccess) return e;
+  const int64_t nwr = static_cast<int64_t>(a.E) * a.d;
+  bw_sum_parts_kernel<<<static_cast<unsigned>((nwr + 255) / 256), 256, 0, s>>>(nwr, a.wr_chunks, a.wr_part, a.dW_r);
+  count_launch();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.db_r != nullptr) {
     bw_db_kernel<<<a.E, THREADS, 0, s>>>(a.T, a.E, a.dh, a.db_r);
     count_launch();

@@ -60,6 +60,9 @@ struct BackwardArgs {
   float* dW2t;             // [G][d_ff][d] fp32: dW2 transposed
   int32_t* woff;           // [G + 1] rows of the per-expert products: e * d_ff
   int32_t* wpre;           // [G + 1] their m-tile prefix: e * ceil(d_ff / 128)
+  // dW_r: the sum over tokens cut into wr_chunks chunks of partials
+  int wr_chunks;
+  float* wr_part;          // [wr_chunks][E][d]
   // outputs (fp32)
   float* dx;    // [T][d]
   float* dW_r;  // [E][d]

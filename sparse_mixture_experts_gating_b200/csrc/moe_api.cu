@@ -171,8 +171,8 @@ Layout make_layout(const moe_layer& L, int64_t T) {
 // [2][S][d_ff], and a second dXp part for SwiGLU.
 struct BwLayout {
   size_t A1, A3, U, dg, dXp, dh, cnt1, ones, dYs, W1t, W3t, W2t, dA1p, dA3p, P1, P3, PH, XT, DT, dW2t, woff, wpre,
-      total;
-  int max_group_rows, k_pad;
+      wr_part, total;
+  int max_group_rows, k_pad, wr_chunks;
 };
 
 // No group has more rows: a token takes an expert at most once, and a shared
@@ -218,6 +218,10 @@ BwLayout make_bw_layout(const moe_layer& L, const Layout& w) {
   b.dW2t = take(tc ? sizeof(float) * G * L.d * static_cast<size_t>(L.d_ff) : 0);
   b.woff = take(tc ? sizeof(int32_t) * (G + 1) : 0);
   b.wpre = take(tc ? sizeof(int32_t) * (G + 1) : 0);
+  // dW_r's partials: chunks of at least 256 tokens, at most 64 of them
+  const int64_t ch = (w.T + 255) / 256;
+  b.wr_chunks = static_cast<int>(ch < 1 ? 1 : (ch > 64 ? 64 : ch));
+  b.wr_part = take(sizeof(float) * b.wr_chunks * static_cast<size_t>(L.E) * L.d);
   b.total = o;
   return b;
 }
@@ -641,6 +645,8 @@ int moe_backward(moe_handle h, int64_t T, const void* x, const float* W_r, const
   a.x_is_bf16 = L.dtype == MOE_BF16;
   a.max_group_rows = b.max_group_rows;
   a.k_pad = b.k_pad;
+  a.wr_chunks = b.wr_chunks;
+  a.wr_part = reinterpret_cast<float*>(bw + b.wr_part);
   a.s_max = w.s_max;
   a.x = x;
   a.W_r = W_r;
