@@ -18,17 +18,20 @@
 // softmax over the chosen logits).  Every sum runs in a fixed order, so the
 // results are deterministic.
 //
-// The contractions run as tiled fp32 GEMMs (64 x 64 tiles, 16-deep k-steps,
-// 4 x 4 outputs per thread) over the expert groups of the sorted buffers.
-// For bf16 layers every product runs instead on the forward's tensor-core
-// grouped GEMM with its fp32 epilogue (gate 1).  The row-grouped ones (w1 x
+// For fp32 layers the contractions run as tiled fp32 GEMMs on CUDA cores
+// (64 x 64 tiles, 16-deep k-steps, 4 x 4 outputs per thread) over the expert
+// groups of the sorted buffers.  For bf16 layers every product of the experts
+// runs on the forward's tensor-core grouped GEMM with its fp32 epilogue (gate
+// 1).  The row-grouped ones (w1 x
 // and w3 x again, W2^T dy, W1^T da1 + W3^T da3): the weights are transposed
 // per expert into K-major copies, dy is gathered into expert-sorted rows, and
 // da1 / da3 enter as hi + lo bf16 planes (about 16 significant bits) like the
 // forward's hidden activation.  The weight gradients reduce over each
 // expert's ragged rows: every expert's rows are packed transposed and
 // zero-padded to k_pad, so each gradient is a product of groups of d_ff rows
-// over K = k_pad (dW2 comes out transposed and is turned once more).
+// over K = k_pad (dW2 comes out transposed and is turned once more).  The
+// router's gradient dW_r, a sum over all tokens, runs on CUDA cores in chunks
+// of tokens whose partials are summed in chunk order.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
