@@ -69,3 +69,25 @@ def test_kernel_roofline_picks_the_binding_resource():
 
 def test_traffic_is_null_without_a_matching_profile(tmp_path, monkeypatch):
     assert bench.profiled_traffic("gemm1", "no_such_workload") is None
+
+
+def test_backward_work_closed_forms():
+    """Backward FLOPs: 5 (ReLU) or 8 (SwiGLU) d x d_ff contractions per kept
+    row plus the router's three T x E x d; bytes: active experts' weights read,
+    every expert's fp32 gradients written, x and dy read, dx and dW_r written."""
+    sw = WORKLOADS["switch_k1"]
+    f, b = bench.backward_work(sw, 4104, 8192, 57)
+    assert f == 2.0 * 4104 * 768 * 3072 * 5 + 3 * 2.0 * 8192 * 64 * 768
+    per = 2 * 768 * 3072
+    assert b == 57 * per * 2 + 64 * per * 4 + 2 * 8192 * 768 * 2 + 8192 * 768 * 4 + 64 * 768 * 4
+    mx = WORKLOADS["mixtral_prefill"]
+    f, b = bench.backward_work(mx, 16384, 8192, 8)
+    assert f == 2.0 * 16384 * 4096 * 14336 * 8 + 3 * 2.0 * 8192 * 8 * 4096
+    per = 3 * 4096 * 14336
+    assert b == 8 * per * 2 + 8 * per * 4 + 2 * 8192 * 4096 * 2 + 8192 * 4096 * 4 + 8 * 4096 * 4
+
+
+def test_profiled_traffic_matches_the_current_sources():
+    """The committed GEMM2 capture of the Switch workload names the sources it
+    was taken from; the bench reports its DRAM bytes while they are unchanged."""
+    assert bench.profiled_traffic("gemm2", "switch_k1") == 330019584.0
