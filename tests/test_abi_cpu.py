@@ -189,3 +189,36 @@ def test_backward_validates_arguments_without_gpu(L):
     assert "backward workspace" in L.moe_last_error().decode()
     assert call(bw=ctypes.c_void_p(272)) == _lib.MOE_ERR_INVALID_ARG
     L.moe_destroy(h)
+
+
+def test_header_compiles_and_links_as_plain_c(L, tmp_path):
+    """A C program (not C++) includes include/moe.h, links the library and
+    calls the host-only entry points."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_moe.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "moe.h"
+int main(void) {
+  moe_handle h = 0;
+  if (moe_create(64, 1, 768, 3072, MOE_ACT_RELU, MOE_GATE_SWITCH, 1.25, MOE_BF16, &h) != MOE_OK) return 1;
+  if (moe_capacity(h, 8192) != 160) return 2;
+  if (moe_workspace_bytes(h, 8192) == 0 || moe_backward_workspace_bytes(h, 8192) == 0) return 3;
+  if (moe_forward(NULL, 1, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0) != MOE_ERR_INVALID_ARG) return 4;
+  if (moe_destroy(h) != MOE_OK) return 5;
+  printf("ok\n");
+  return 0;
+}
+""")
+    lib_dir = os.path.dirname(L._name)
+    exe = tmp_path / "use_moe"
+    inc = os.path.dirname(HEADER)
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", inc, str(src), "-o", str(exe), "-L", lib_dir,
+                        "-l:" + os.path.basename(L._name), "-Wl,-rpath," + lib_dir], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", (run.returncode, run.stdout, run.stderr)
