@@ -410,26 +410,6 @@ __global__ void __launch_bounds__(THREADS) bw_db_kernel(int64_t T, int E, const 
   if (threadIdx.x == 0) db[e] = tot;
 }
 
-// out[g][c][r] = in[g][r][c] for matrices [G][R][C] (32 x 32 tiles).
-template <typename T>
-__global__ void __launch_bounds__(256) bw_transpose_kernel(const T* __restrict__ in, T* __restrict__ out, int R,
-                                                           int C) {
-  __shared__ T tile[32][34];
-  const int64_t g = blockIdx.z;
-  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
-  const T* src = in + g * R * C;
-  T* dst = out + g * R * C;
-  for (int i = threadIdx.y; i < 32; i += 8) {
-    const int r = r0 + i, c = c0 + threadIdx.x;
-    if (r < R && c < C) tile[i][threadIdx.x] = src[static_cast<int64_t>(r) * C + c];
-  }
-  __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += 8) {
-    const int c = c0 + i, r = r0 + threadIdx.x;
-    if (r < R && c < C) dst[static_cast<int64_t>(c) * R + r] = tile[threadIdx.x][i];
-  }
-}
-
 // dy rows into expert-sorted order (a warp per row, 16-byte copies).
 __global__ void __launch_bounds__(256) bw_gather_dy_kernel(int d, const int32_t* offsets, int groups,
                                                            const int32_t* row_token, const uint4* dy, uint4* dYs) {
@@ -502,6 +482,39 @@ __global__ void __launch_bounds__(256) bw_transpose_bf16x2_kernel(const __nv_bfl
   }
 }
 
+// fp32 [G][R][C] -> [G][C][R] with R and C even: 64 x 64 tiles, pairs of
+// columns read and pairs of rows written as 8-byte words.
+__global__ void __launch_bounds__(256) bw_transpose_f32x2_kernel(const float* __restrict__ in, float* __restrict__ out,
+                                                                 int R, int C) {
+  __shared__ float tile[64][65];
+  const int64_t g = blockIdx.z;
+  const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const float* src = in + g * R * C;
+  float* dst = out + g * R * C;
+  for (int i = ty; i < 64; i += 8) {
+    const int r = r0 + i, c = c0 + 2 * tx;
+    if (r < R && c < C) {
+      const float2 v = *reinterpret_cast<const float2*>(src + static_cast<int64_t>(r) * C + c);
+      tile[i][2 * tx] = v.x;
+      tile[i][2 * tx + 1] = v.y;
+    }
+  }
+  __syncthreads();
+  for (int i = ty; i < 64; i += 8) {
+    const int c = c0 + i, r = r0 + 2 * tx;
+    if (c < C && r < R)
+      *reinterpret_cast<float2*>(dst + static_cast<int64_t>(c) * R + r) = make_float2(tile[2 * tx][i], tile[2 * tx + 1][i]);
+  }
+}
+
+cudaError_t transpose_f32(const void* in, void* out, int G, int R, int C, cudaStream_t s) {
+  const dim3 grid((C + 63) / 64, (R + 63) / 64, G);
+  bw_transpose_f32x2_kernel<<<grid, 256, 0, s>>>(static_cast<const float*>(in), static_cast<float*>(out), R, C);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t transpose_bf16(const void* in, void* out, int G, int R, int C, cudaStream_t s) {
   const dim3 grid((C + 63) / 64, (R + 63) / 64, G);
   bw_transpose_bf16x2_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(in),
@@ -510,13 +523,6 @@ cudaError_t transpose_bf16(const void* in, void* out, int G, int R, int C, cudaS
   return cudaGetLastError();
 }
 
-template <typename T>
-cudaError_t transpose(const void* in, void* out, int G, int R, int C, cudaStream_t s) {
-  const dim3 grid((C + 31) / 32, (R + 31) / 32, G);
-  bw_transpose_kernel<T><<<grid, dim3(32, 8), 0, s>>>(static_cast<const T*>(in), static_cast<T*>(out), R, C);
-  count_launch();
-  return cudaGetLastError();
-}
 
 // Per-expert operand of a weight gradient: out[e][f][kk] = v(off_e + kk, f)
 // for kk below the group's row count, 0 up to k_pad, where v(r, f) =
@@ -704,7 +710,7 @@ cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
     }
     if ((e = tc_product(a, PH, PH + pl, a.DT, a.d, kp, a.dW2t, s, a.woff, a.wpre, arows, a.d_ff)) != cudaSuccess)
       return e;
-    if ((e = transpose<float>(a.dW2t, a.dW2, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
+    if ((e = transpose_f32(a.dW2t, a.dW2, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
   } else {
   WGrad w{};
   w.offsets = a.offsets;
