@@ -222,3 +222,24 @@ int main(void) {
     assert r.returncode == 0, r.stderr
     run = subprocess.run([str(exe)], capture_output=True, text=True)
     assert run.returncode == 0 and run.stdout.strip() == "ok", (run.returncode, run.stdout, run.stderr)
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    """No CPU fallback: with the library absent the binding raises instead of
+    computing anything."""
+    monkeypatch.setattr(_lib, "_LIB", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libmoe_b200.so"))
+    with pytest.raises(ImportError, match="no CPU fallback"):
+        _lib.lib()
+
+
+def test_product_path_never_imports_the_oracle():
+    """The package (binding, layer, workloads, build) and bench.py's timed arm
+    reference the oracle nowhere; only tests, smoke() and the CPU baseline do."""
+    pkg = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                       "sparse_mixture_experts_gating_b200")
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(root, f), encoding="utf-8").read()
+                assert "import oracle" not in src and "from oracle" not in src, f
