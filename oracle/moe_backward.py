@@ -1,7 +1,8 @@
 """CPU oracle for the backward pass of the sparse Mixture-of-Experts layer.
 
-TEST INFRASTRUCTURE ONLY (see moe_oracle.py): only tests/ and bench.py's
-CPU-baseline leg may import or run it.
+TEST INFRASTRUCTURE ONLY (see moe_oracle.py): only tests/,
+``__graft_entry__.smoke()`` and bench.py's CPU-baseline leg may import or run
+it; the product path never does.
 
 Gradients of the scalar
 
