@@ -125,6 +125,11 @@ MOE_API int moe_create(int num_experts, int k, int d, int d_ff, int act, int gat
  *     (about 16 significant bits); the second projection runs its tensor-core
  *     MMAs on both planes, twice the tensor work of that projection.
  *   MOE_HIDDEN_BF16: one bf16 number (8 significant bits, unit roundoff 2^-8).
+ *     OUTSIDE THE PARITY BAR for the maximum error: against an fp32 reference
+ *     on the same bf16 inputs, the rounding of the hidden activation alone
+ *     gives max|dy| of about 1.5e-2 * RMS(y) on layers with millions of
+ *     outputs (the bar is 1e-2 * RMS); the mean relative error (about 1.6e-3)
+ *     stays within 2e-3.  Use it only where that is acceptable.
  * Changes moe_workspace_bytes().  fp32 layers ignore it.  Returns MOE_OK or
  * MOE_ERR_INVALID_ARG.
  */
@@ -220,6 +225,10 @@ MOE_API int moe_balance_losses(moe_handle h, int64_t T, const void* workspace, f
  *   - Every call shares the array and leaves its contents there; calls that
  *     overlap on the GPU (other streams, other host threads) race on it.
  *     Nothing in it needs to start at zero.
+ *   - The looked-up address is kept for the life of the process.  A
+ *     cudaDeviceReset (or any other teardown of the device's primary
+ *     context) invalidates it, like the device error word every entry point
+ *     uses: make no further call of this library on that device afterwards.
  *   - Allocates nothing (no cudaMalloc / cudaFree or allocating routine).
  */
 MOE_API int moe_forward_static(moe_handle h, int64_t T, const void* x, const float* W_r, const float* b_r,

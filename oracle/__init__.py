@@ -6,5 +6,5 @@ import this package.  The CUDA library never links, imports or calls it.
 from .moe_oracle import (  # noqa: F401
     ACT_RELU, ACT_SWIGLU, GATE_RENORM, GATE_SWITCH,
     aux_and_z, assign_slots, balance_losses, expert_capacity, expert_ffn, gates, moe_forward,
-    round_to_bf16, router_logits, softmax_lse, top_k,
+    router_logits, softmax_lse, top_k,
 )

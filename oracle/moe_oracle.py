@@ -167,26 +167,13 @@ def assign_slots(idx: np.ndarray, E: int, C: Optional[int]):
     }
 
 
-def round_to_bf16(v: np.ndarray) -> np.ndarray:
-    """Round to the nearest bfloat16 (8 significant bits), ties to even.
-
-    The value is first rounded to float32 (as a float32 computation would hold
-    it), then the low 16 bits of the float32 pattern are rounded away with the
-    usual round-half-to-even bias.  Finite inputs only.  Returns float64.
-    """
-    u = np.asarray(v, np.float64).astype(np.float32).view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32).astype(np.float64)
-
-
-def expert_ffn(xr: np.ndarray, W1e, W3e, W2e, act: int, hidden_bf16: bool = False) -> np.ndarray:
+def expert_ffn(xr: np.ndarray, W1e, W3e, W2e, act: int) -> np.ndarray:
     """One expert on a batch of rows.
 
     SWIGLU ("Implementation"): w2(silu(w1 x) * w3 x), silu(u) = u / (1 + e^-u).
     RELU: w2(relu(w1 x)).  Weights in nn.Linear (out, in) layout:
-    W1e/W3e [d_ff][d], W2e [d][d_ff].  float64.
-    hidden_bf16: hold the hidden activation in bf16 between the two projections
-    (mixed precision: the page asks only the router to stay in float32).
+    W1e/W3e [d_ff][d], W2e [d][d_ff].  float64 throughout: the hidden
+    activation is never rounded (the page fixes only the router's precision).
     """
     a = xr @ np.asarray(W1e, np.float64).T
     if act == ACT_RELU:
@@ -194,8 +181,6 @@ def expert_ffn(xr: np.ndarray, W1e, W3e, W2e, act: int, hidden_bf16: bool = Fals
     else:
         b = xr @ np.asarray(W3e, np.float64).T
         hdn = a / (1.0 + np.exp(-a)) * b
-    if hidden_bf16:
-        hdn = round_to_bf16(hdn)
     return hdn @ np.asarray(W2e, np.float64).T
 
 
@@ -252,7 +237,7 @@ def balance_losses(p: np.ndarray, idx: np.ndarray, E: int) -> dict:
 
 def moe_forward(x, W_r, b_r, W1, W3, W2, *, k: int, gate_mode: int, act: int,
                 capacity_factor: float, rows: Optional[Sequence[int]] = None,
-                logits: Optional[np.ndarray] = None, hidden_bf16: bool = False,
+                logits: Optional[np.ndarray] = None,
                 shared: Optional[tuple] = None, logits_dtype=np.float32) -> dict:
     """The whole layer: routing for every token, y for every token or for ``rows``.
 
@@ -261,7 +246,6 @@ def moe_forward(x, W_r, b_r, W1, W3, W2, *, k: int, gate_mode: int, act: int,
     ``logits``: route from these fp32 logits instead of computing W_r x.
     ``rows``: compute y only for these tokens (routing, capacity and losses are
     always global; y_t depends on x_t and the global routing only).
-    ``hidden_bf16``: round each expert's hidden activation to bf16 (see expert_ffn).
     ``logits_dtype``: np.float64 keeps the logits unrounded (finite differences).
     ``shared``: (W1s, W3s, W2s), each with n_s experts shaped like W1, W3, W2:
     shared experts that every token visits ("Mixture of experts", section
@@ -299,7 +283,7 @@ def moe_forward(x, W_r, b_r, W1, W3, W2, *, k: int, gate_mode: int, act: int,
             continue
         ts = want[ii]
         out = expert_ffn(np.asarray(x[ts], np.float64), W1[e],
-                         None if W3 is None else W3[e], W2[e], act, hidden_bf16)
+                         None if W3 is None else W3[e], W2[e], act)
         contrib[ii, jj] = g[ts, jj][:, None] * out
     y = np.zeros((len(want), d), np.float64)
     for j in range(k):                  # slot order
@@ -308,7 +292,7 @@ def moe_forward(x, W_r, b_r, W1, W3, W2, *, k: int, gate_mode: int, act: int,
         W1s, W3s, W2s = shared
         xs = np.asarray(x[want], np.float64)
         for si in range(len(W1s)):      # shared-expert order, after the routed sum
-            y += expert_ffn(xs, W1s[si], None if W3s is None else W3s[si], W2s[si], act, hidden_bf16)
+            y += expert_ffn(xs, W1s[si], None if W3s is None else W3s[si], W2s[si], act)
     res = {"logits": h32, "p": p, "lse": lse, "idx": idx, "gate": g, "capacity": C,
            "y": y, "rows": want, "aux": aux, "z": z}
     res.update(balance_losses(p, idx, E))

@@ -5,16 +5,14 @@ Tolerances (derived from the arithmetic; see the design notes):
   * routing (top-k indices, expert counts, offsets, destination rows, drop
     mask, dropped count): bit-exact;
   * fp32 layers: max|dy| / max|y_ref| <= 1e-5;
-  * bf16 layers: on the fp32 value of y before its final cast,
-    max|dy| <= 1e-2 * RMS(y_ref) and sum|dy| / sum|y_ref| <= 2e-3 against the
-    plain oracle (default hidden precision: a hi + lo pair of bf16 planes);
-    with the hidden activation held in ONE bf16 plane its rounding alone
-    (unit roundoff 2^-8) pushes the max to ~1.5e-2 * RMS on large outputs, so
-    that mode asserts both bounds against the oracle holding the hidden
-    activation in bf16 like the kernel, and the mean bound against the plain one;
-    the tolerance applies to the fp32-accumulated result, and the stored bf16
-    output must be exactly its round-to-nearest-even image (the cast alone adds
-    about 1.3e-3 mean relative error);
+  * bf16 layers, always against the plain oracle (float64, nothing rounded
+    between its steps): max|dy| <= 1e-2 * RMS(y_ref) on the fp32-accumulated
+    value of y before its final cast, and sum|dy| / sum|y_ref| <= 2e-3 both on
+    that value and on the returned bf16 y; the returned y must be exactly the
+    round-to-nearest-even image of the fp32 value.  With the hidden activation
+    held in ONE bf16 plane (MOE_HIDDEN_BF16) its rounding alone (unit roundoff
+    2^-8) pushes the max to ~1.5e-2 * RMS on large outputs: that mode is held
+    to the mean bound only, its max error is reported;
   * gates: |dg| <= 2e-6 (fp32 exp of exact logit differences);
   * aux, z: relative 1e-5.
 """
@@ -92,7 +90,7 @@ class _Shift:
         return self.he[self.E + s]
 
 
-def run_oracle(w: Workload, host: dict, rows=None, logits=None, hidden_bf16=False):
+def run_oracle(w: Workload, host: dict, rows=None, logits=None):
     shared = None
     if w.n_shared:
         shared = (_Shift(host["W1"], w.E, w.n_shared),
@@ -100,7 +98,7 @@ def run_oracle(w: Workload, host: dict, rows=None, logits=None, hidden_bf16=Fals
                   _Shift(host["W2"], w.E, w.n_shared))
     return O.moe_forward(host["x"], host["W_r"], host["b_r"], host["W1"], host["W3"], host["W2"],
                          k=w.k, gate_mode=w.gate, act=w.act, capacity_factor=w.capacity_factor,
-                         rows=rows, logits=logits, hidden_bf16=hidden_bf16, shared=shared)
+                         rows=rows, logits=logits, shared=shared)
 
 
 def assert_routing_equal(g: dict, o: dict):
@@ -136,14 +134,14 @@ def y_errors(y_gpu: np.ndarray, y_ref: np.ndarray):
     }
 
 
-def assert_y_close(w: Workload, g: dict, y_ref: np.ndarray, rows=None, y_ref_bf16h=None):
-    """y of the CUDA path against the oracle.
+def assert_y_close(w: Workload, g: dict, y_ref: np.ndarray, rows=None, max_bound=True):
+    """y of the CUDA path against the plain oracle y_ref.
 
-    y_ref: the plain oracle (fp64, no intermediate rounding).  For bf16 layers
-    the max bound 1e-2 * RMS is asserted against y_ref, unless y_ref_bf16h (the
-    oracle holding the hidden activation in bf16, as the kernel does) is given,
-    in which case the max bound is asserted against it; the mean bound is
-    always asserted against y_ref.
+    fp32 layers: max|dy| / max|y_ref| <= 1e-5.  bf16 layers: the mean bound
+    on the fp32 value before the cast and on the returned bf16 y, the max
+    bound 1e-2 * RMS(y_ref) on the fp32 value unless max_bound is False (the
+    single-plane hidden mode, which is outside that bound), and the returned
+    y bit for bit the round-to-nearest-even image of the fp32 value.
     """
     sel = slice(None) if rows is None else np.asarray(rows)
     if w.dtype == DTYPE_F32:
@@ -152,21 +150,17 @@ def assert_y_close(w: Workload, g: dict, y_ref: np.ndarray, rows=None, y_ref_bf1
         return e
     yf = g["y_f32"][sel]
     e = y_errors(yf, y_ref)
+    e["bf16_output"] = y_errors(g["y"][sel], y_ref)
     assert e["mean_rel"] <= 2e-3, e
-    if y_ref_bf16h is None:
+    assert e["bf16_output"]["mean_rel"] <= 2e-3, e
+    if max_bound:
         assert e["max_over_rms"] <= 1e-2, e
-    else:
-        eh = y_errors(yf, y_ref_bf16h)
-        assert eh["max_over_rms"] <= 1e-2, eh
-        assert eh["mean_rel"] <= 2e-3, eh
-        e["vs_bf16_hidden"] = eh
     # the bf16 output is the RNE image of the fp32 value
     rne = torch.from_numpy(np.ascontiguousarray(yf)).to(torch.bfloat16)
     out = g["y_dev"].cpu()
     if rows is not None:
         out = out[torch.as_tensor(np.asarray(rows))]
     assert torch.equal(rne.view(torch.int16), out.view(torch.int16))
-    e["bf16_output"] = y_errors(g["y"][sel], y_ref)  # reported; the cast adds ~1.3e-3 mean relative
     return e
 
 

@@ -30,13 +30,13 @@ def _gates_not_renormalised(h32, p, idx, gate_mode):
     return p[np.arange(idx.shape[0])[:, None], idx]
 
 
-def _ffn_silu_sign(xr, W1e, W3e, W2e, act, hidden_bf16=False):
+def _ffn_silu_sign(xr, W1e, W3e, W2e, act):
     a = xr @ np.asarray(W1e, np.float64).T
     hdn = np.maximum(a, 0) if act == M.ACT_RELU else a / (1 + np.exp(a)) * (xr @ np.asarray(W3e, np.float64).T)
     return hdn @ np.asarray(W2e, np.float64).T
 
 
-def _ffn_w1_w3_swapped_roles(xr, W1e, W3e, W2e, act, hidden_bf16=False):
+def _ffn_w1_w3_swapped_roles(xr, W1e, W3e, W2e, act):
     if act == M.ACT_RELU:
         return _orig["expert_ffn"](xr, W1e, W3e, W2e, act)
     a = xr @ np.asarray(W3e, np.float64).T

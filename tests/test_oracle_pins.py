@@ -322,37 +322,6 @@ def test_sampled_rows_equal_full_rows_and_dropped_tokens_are_zero():
     np.testing.assert_allclose(full["y"][t], ref, rtol=1e-13)
 
 
-# ---------------------------------------------------------------- bf16 hidden activation
-def test_round_to_bf16_matches_torch_including_ties():
-    """The hidden-activation rounding equals torch's float32 -> bfloat16 (RNE) conversion."""
-    v = rng.normal(size=20000) * np.exp(rng.uniform(-20, 20, size=20000))
-    # exact halfway cases between two bf16 values, both parities of the kept bit
-    base = rng.integers(0x3F800000, 0x40800000, size=2000, dtype=np.int64) & ~0xFFFF
-    half = (base | 0x8000).astype(np.uint32).view(np.float32).astype(np.float64)
-    half = np.concatenate([half, -half, [0.0, -0.0, 1.0, 3.0e38, 1e-40]])
-    for arr in (v, half):
-        ref = torch.from_numpy(arr.astype(np.float32)).to(torch.bfloat16).double().numpy()
-        assert np.array_equal(O.round_to_bf16(arr), ref)
-
-
-def test_hidden_bf16_is_exact_when_the_hidden_values_are_bf16_numbers():
-    """ReLU layer with small-integer weights: hidden values are small integers,
-    exactly representable in bf16, so the rounding option changes nothing; with
-    general weights it changes each hidden value by at most 2^-8 relative."""
-    T, d, dff, E = 40, 6, 10, 3
-    x = rng.integers(-3, 4, size=(T, d)).astype(np.float64)
-    W_r = rng.normal(size=(E, d))
-    W1 = rng.integers(-2, 3, size=(E, dff, d)).astype(np.float64)
-    W2 = rng.normal(size=(E, d, dff))
-    a = O.moe_forward(x, W_r, None, W1, None, W2, k=2, gate_mode=O.GATE_RENORM, act=O.ACT_RELU,
-                      capacity_factor=0.0)
-    b = O.moe_forward(x, W_r, None, W1, None, W2, k=2, gate_mode=O.GATE_RENORM, act=O.ACT_RELU,
-                      capacity_factor=0.0, hidden_bf16=True)
-    np.testing.assert_array_equal(a["y"], b["y"])
-    h = rng.normal(size=5000) * 10
-    assert np.all(np.abs(O.round_to_bf16(h) - h) <= (2.0 ** -8 + 2.0 ** -23) * np.abs(h))  # unit roundoff 2^-8, via fp32
-
-
 # ---------------------------------------------------------------- shared experts
 @pytest.mark.parametrize("act", [O.ACT_RELU, O.ACT_SWIGLU])
 def test_shared_expert_with_silent_routed_experts_is_the_dense_ffn(act):
