@@ -5,11 +5,19 @@
 One step = one forward pass of the whole layer (router, scan, dispatch, two
 grouped GEMMs, combine, losses) over one batch of the workload's synthetic
 input, resident in HBM.  L2 is flushed between steps, outside the timed
-events: a 256 MiB write, then a 256 MiB read of another buffer.  Prints ONE JSON line on rank 0.
+events: a 256 MiB write, then a 256 MiB read of another buffer.
+
+Default run (no --workload, one GPU): one JSON line per workload on rank 0,
+the headline LAST: the Switch layer, the Mixtral-shaped decode layers at
+T = 1, 16 and 64 (each timed over at least 100 calls, with the p50 latency
+per call), the fine-grained 128-expert layer, and finally the Mixtral-shaped
+prefill layer (T 8192, d 4096, 8 experts, top-2, SwiGLU 14336), the largest
+single-GPU configuration, whose line also carries a summary of the others.
+With --workload NAME, or under torchrun with N > 1, only that workload (the
+prefill layer by default) is measured and printed.
 
 --backward times a training step instead (the forward pass, then the
-backward pass of <dy, y> + 0.01 aux + 1e-3 z) on one GPU, with the
-backward's fp32 CUDA-core roofline.
+backward pass of <dy, y> + 0.01 aux + 1e-3 z) on one GPU.
 
 N > 1 (torchrun): every rank runs an independent replica of the layer on its
 own batch (the layer has no cross-batch exchange), so scaling is weak; the
@@ -32,8 +40,13 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s on 1 B200 and % of roofline (TFLOP/s or HBM GB/s)"
-DEFAULT_WORKLOAD = "switch_k1"
+DEFAULT_WORKLOAD = "mixtral_prefill"
+# measured before the headline in the default one-GPU run
+SECONDARY = ["switch_k1", "mixtral_decode_t1", "mixtral_decode_t16", "mixtral_decode_t64", "fine_grained"]
+DECODE_MIN_CALLS = 100  # decode layers report the p50 latency over at least this many calls
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# the nominal B200 figures the layer's targets are quoted against (dense bf16, HBM3e)
+NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2200.0}
 STAGE_KERNEL = {"router": "router_kernel", "scan": "scan_kernel", "dispatch": "dispatch_kernel",
                 "gemm1": "grouped_gemm_kernel", "gemm2": "grouped_gemm_kernel", "combine": "combine_kernel"}
 # oracle tokens per CPU-baseline sample, per workload (bounded to ~10-30 s of CPU work)
@@ -51,45 +64,49 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def layer_work(w, kept_counts, hidden="bf16x2"):
+def layer_work(w, kept_counts):
     """Algorithmic FLOPs and bytes of the layer and of each grouped GEMM launch.
 
-    Counts kept assignments only, plus T rows per shared expert.  Bytes:
-    weights of experts with >= 1 kept row and of every shared expert (read
-    once), x read once, y written once, W_r; per GEMM also its own input and
-    output activations (the expert-sorted rows; the hidden activation at 4
-    bytes per element when held as a hi + lo bf16 pair).
+    FLOPs count kept assignments only (plus T rows per shared expert) and the
+    router.  Bytes are what the method must move, the expert-sorted
+    intermediates (sorted x, hidden activation, fp32 partial rows) excluded:
+    the layer reads W_r, the weights of every expert with at least one kept
+    row (and of every shared expert) once, x once, and writes y once.  Of
+    these, the first projection is charged its weights (W1, and W3 for
+    SwiGLU) and x, the second projection its weights (W2) and y.
     """
     elt = 2 if w.dtype == 1 else 4
-    h_elt = 4 if (w.dtype == 1 and hidden == "bf16x2") else elt
     n_sh = getattr(w, "n_shared", 0)
     S = int(sum(kept_counts)) + n_sh * w.T
     active = sum(1 for c in kept_counts if c > 0) + n_sh
     nproj1 = 2 if w.act == 1 else 1
     w1_bytes = active * nproj1 * w.d_ff * w.d * elt
     w2_bytes = active * w.d * w.d_ff * elt
+    act_bytes = w.T * w.d * elt
     flops_router = 2.0 * w.T * w.E * w.d
     flops1 = 2.0 * S * w.d * w.d_ff * nproj1
     flops2 = 2.0 * S * w.d_ff * w.d
-    gemm1_bytes = w1_bytes + S * w.d * elt + S * w.d_ff * h_elt
-    out2 = S * w.d * (elt if (w.k == 1 and n_sh == 0) else 4)
-    gemm2_bytes = w2_bytes + S * w.d_ff * h_elt + out2
-    layer_bytes = w1_bytes + w2_bytes + 2 * w.T * w.d * elt + w.E * w.d * 4
+    layer_bytes = w1_bytes + w2_bytes + 2 * act_bytes + w.E * w.d * 4
     return {"S": S, "active_experts": active, "flops_layer": flops_router + flops1 + flops2,
-            "bytes_layer": layer_bytes, "gemm1": {"flops": flops1, "bytes": gemm1_bytes},
-            "gemm2": {"flops": flops2, "bytes": gemm2_bytes}}
+            "bytes_layer": layer_bytes, "gemm1": {"flops": flops1, "bytes": w1_bytes + act_bytes},
+            "gemm2": {"flops": flops2, "bytes": w2_bytes + act_bytes}}
 
 
 def kernel_roofline(flops, nbytes, seconds, peaks):
+    """Roofline of one kernel: bound by whichever of its algorithmic FLOPs (at
+    the bf16 tensor peak) and bytes (at the HBM bandwidth) takes longer;
+    frac against the measured peak, frac_nominal against the nominal one."""
     t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     if t_tensor >= t_hbm:
         a = flops / seconds / 1e12
         return {"bound": "tensor", "achieved": round(a, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(a / peaks["bf16_tflops"], 4)}
+                "frac": round(a / peaks["bf16_tflops"], 4),
+                "frac_nominal": round(a / NOMINAL_PEAKS["bf16_tflops"], 4), "algorithmic": flops}
     a = nbytes / seconds / 1e9
     return {"bound": "hbm", "achieved": round(a, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(a / peaks["hbm_gbs"], 4)}
+            "frac": round(a / peaks["hbm_gbs"], 4), "frac_nominal": round(a / NOMINAL_PEAKS["hbm_gbs"], 4),
+            "algorithmic": nbytes}
 
 
 def source_sha(*rel):
@@ -260,49 +277,19 @@ def cpu_baseline(w, inp):
 
 
 # ----------------------------------------------------------------------------- GPU leg
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--hidden", choices=["bf16x2", "bf16"], default="bf16x2",
-                    help="how the expert hidden activation is held (bf16 layers)")
-    ap.add_argument("--tokens", type=int, default=None,
-                    help="override the workload's token count (small cases for profiler captures)")
-    ap.add_argument("--backward", action="store_true",
-                    help="time a training step instead: the forward pass, then the backward pass")
-    args = ap.parse_args()
-
+def measure_workload(args, w, dev, world, rank, local, K, warmup, cpu=True):
+    """Time K forward passes of workload w (inputs resident in HBM), the
+    per-stage breakdown in an untimed pass, and the end-to-end path with
+    pinned host buffers.  Returns the JSON line (rank 0) or None."""
     import torch
     import torch.distributed as dist
     from sparse_mixture_experts_gating_b200 import MoELayer, launch_count, status
-    from sparse_mixture_experts_gating_b200.workloads import WORKLOADS, make_inputs, torch_dtype
+    from sparse_mixture_experts_gating_b200.workloads import make_inputs, torch_dtype
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    w = WORKLOADS[args.workload]
-    if args.tokens is not None:
-        w = w.with_(T=args.tokens, x_rows_of=None)
-    warmup = max(3, args.warmup)
-
-    if args.impl == "reference":
-        if rank != 0:
-            return 0
-        return reference_arm(args, w, warmup)
-
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    dev = torch.device("cuda", local)
-
+    decode = w.name.startswith("mixtral_decode")
+    if decode:
+        K = max(K, DECODE_MIN_CALLS)
     inp = make_inputs(w, device=dev)
-    if args.backward:
-        return backward_bench(args, w, inp, warmup, world, rank, local, dev)
     if rank > 0:
         inp["x"] = make_inputs(w.with_(seed=rank_seed(w.seed, rank)), device=dev, weights=False)["x"]
     layer = MoELayer(w.E, w.k, w.d, w.d_ff, act=w.act, gate_mode=w.gate, capacity_factor=w.capacity_factor,
@@ -332,15 +319,15 @@ def main():
         step()
     status()
 
-    K = args.steps
     stage_names = ["router", "scan", "dispatch", "gemm1", "gemm2", "combine"]
-    active = [n for n in stage_names if not (n == "combine" and w.dtype == 1 and w.k == 1)]
+    active = [n for n in stage_names if not (n == "combine" and w.dtype == 1 and w.k == 1 and w.n_shared == 0)]
 
     # Untimed profiling pass: every stage bracketed by events -> per-kernel breakdown.
-    ev_stage = [[torch.cuda.Event(enable_timing=True) for _ in range(12)] for _ in range(K)]
+    Kp = min(K, 20)
+    ev_stage = [[torch.cuda.Event(enable_timing=True) for _ in range(12)] for _ in range(Kp)]
     torch.cuda.synchronize()
-    gpu_hold(torch, 2.0 + 0.3 * K)
-    for i in range(K):
+    gpu_hold(torch, 2.0 + 0.3 * Kp)
+    for i in range(Kp):
         flush_l2()
         step(events=ev_stage[i])
     torch.cuda.synchronize()
@@ -400,13 +387,14 @@ def main():
         x_dev.copy_(x_host, non_blocking=True)
         step(x=x_dev)
         y_host.copy_(y, non_blocking=True)
-        for h, s in zip(st_host, stats):
-            h.copy_(s, non_blocking=True)
+        for h, s_ in zip(st_host, stats):
+            h.copy_(s_, non_blocking=True)
         if i >= warmup:
             e2e_ev[i - warmup][1].record(stream)
     torch.cuda.synchronize()
     status()
-    e2e_s = sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3
+    e2e_ms = [a.elapsed_time(b) for a, b in e2e_ev]
+    e2e_s = sum(e2e_ms) / 1e3
 
     t_max, tokens = combine_ranks(total_s, w.T * K, dist if world > 1 else None)
     e2e_max, _ = combine_ranks(e2e_s, w.T * K, dist if world > 1 else None)
@@ -414,17 +402,24 @@ def main():
     counts = stats[0].cpu().tolist()
     cap = layer.capacity(w.T)
     kept = [c if cap is None else min(c, cap) for c in counts]
-    work = layer_work(w, kept, args.hidden)
+    work = layer_work(w, kept)
     peaks, peak_src = load_peaks()
     roof = kernel_roofline(work[dom]["flops"], work[dom]["bytes"], dom_ms / 1e3, peaks)
     roof["kernel"] = f"{STAGE_KERNEL[dom]} ({dom})"
     roof["peak_source"] = f"{peak_src} ({'bf16_tflops' if roof['bound'] == 'tensor' else 'hbm_gbs'}, burst)"
+    roof["nominal_peak"] = NOMINAL_PEAKS["bf16_tflops" if roof["bound"] == "tensor" else "hbm_gbs"]
     tr = profiled_traffic(dom, w.name)
     roof["traffic"] = tr
+    gemm_bytes = work[dom]["bytes"]
+    roof["traffic_ratio"] = None if tr is None else round(tr / gemm_bytes, 3)
+    roof["kernel_ms"] = round(dom_ms, 5)
     ms_step = total_s / K * 1e3
     floor_s = max(work["flops_layer"] / (peaks["bf16_tflops"] * 1e12), work["bytes_layer"] / (peaks["hbm_gbs"] * 1e9))
+    floor_nom = max(work["flops_layer"] / (NOMINAL_PEAKS["bf16_tflops"] * 1e12),
+                    work["bytes_layer"] / (NOMINAL_PEAKS["hbm_gbs"] * 1e9))
     clocks = sampler.summary(wall0, wall1)
 
+    line = None
     if rank == 0:
         line = {
             "metric": METRIC,
@@ -442,6 +437,8 @@ def main():
             "config": dict(config_of(w, world), hidden=args.hidden),
             "roofline": roof,
             "layer_roofline": {"floor_ms": round(floor_s * 1e3, 5), "frac": round(floor_s / (ms_step / 1e3), 4),
+                               "floor_ms_nominal": round(floor_nom * 1e3, 5),
+                               "frac_nominal": round(floor_nom / (ms_step / 1e3), 4),
                                "flops": work["flops_layer"], "bytes": work["bytes_layer"],
                                "kept_assignments": work["S"], "active_experts": work["active_experts"]},
             "kernels_ms": {k: round(v, 5) for k, v in stage_ms.items()},
@@ -452,8 +449,87 @@ def main():
             "gpu_launches": int(n_launch),
             "clocks": clocks,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if decode:
+            line["latency_ms"] = {"p50": round(statistics.median(step_ms), 5), "min": round(min(step_ms), 5),
+                                  "max": round(max(step_ms), 5), "calls": K,
+                                  "e2e_p50": round(statistics.median(e2e_ms), 5)}
+        if args.hidden != "bf16x2":
+            line["note"] = "hidden activation in one bf16 plane: outside the max-error parity bound"
+        if world == 1 and cpu and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, inp)
+    del inp, ws, y, flush, flush_rd, x_host, y_host, x_dev
+    layer = None
+    torch.cuda.empty_cache()
+    return line
+
+
+def summary_of(line):
+    """The few numbers of a workload's line that the headline line repeats."""
+    out = {"tokens_per_s": line["value"], "ms_per_step": line["ms_per_step"],
+           "dominant": line["roofline"]["kernel"], "dominant_bound": line["roofline"]["bound"],
+           "dominant_frac": line["roofline"]["frac"], "dominant_frac_nominal": line["roofline"]["frac_nominal"],
+           "layer_frac": line["layer_roofline"]["frac"], "layer_frac_nominal": line["layer_roofline"]["frac_nominal"],
+           "e2e_tokens_per_s": line["e2e"]["value"], "sm_mhz": line["clocks"].get("sm_mhz"),
+           "clock_reasons": line["clocks"].get("reasons")}
+    if "latency_ms" in line:
+        out["p50_ms"] = line["latency_ms"]["p50"]
+        out["calls"] = line["latency_ms"]["calls"]
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=None,
+                    help="measure only this workload (default: every workload, the Mixtral prefill layer last)")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--hidden", choices=["bf16x2", "bf16"], default="bf16x2",
+                    help="how the expert hidden activation is held (bf16 layers)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's token count (small cases for profiler captures)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time a training step instead: the forward pass, then the backward pass")
+    args = ap.parse_args()
+
+    import torch
+    import torch.distributed as dist
+    from sparse_mixture_experts_gating_b200.workloads import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    name = args.workload or DEFAULT_WORKLOAD
+    w = WORKLOADS[name]
+    if args.tokens is not None:
+        w = w.with_(T=args.tokens, x_rows_of=None)
+    warmup = max(3, args.warmup)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return reference_arm(args, w, warmup)
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+
+    if args.backward:
+        return backward_bench(args, w, make_inputs(w, device=dev), warmup, world, rank, local, dev)
+    others = []
+    if args.workload is None and args.tokens is None and world == 1:
+        for other in SECONDARY:
+            line = measure_workload(args, WORKLOADS[other], dev, world, rank, local, args.steps, warmup)
+            print(json.dumps(line), flush=True)
+            others.append(line)
+    line = measure_workload(args, w, dev, world, rank, local, args.steps, warmup)
+    if rank == 0:
+        if others:
+            line["workloads"] = {o["config"]["workload"]: summary_of(o) for o in others}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -596,7 +672,8 @@ def reference_arm(args, w, warmup):
         "metric": METRIC, "impl": "reference", "value": round(value, 3), "unit": "tokens/s",
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": warmup,
         "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "config": config_of(w, 1),
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": dict(config_of(w, int(os.environ.get("WORLD_SIZE", "1"))), hidden=args.hidden),
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"each step: oracle forward (float64 NumPy) on the first {n} of {w.T} tokens"},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

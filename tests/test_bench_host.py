@@ -57,6 +57,18 @@ def test_layer_work_mixtral_prefill_matches_the_closed_form():
     # 6 * d * d_ff * T * k for the experts (5.77 TFLOP) plus the router
     assert abs(work["flops_layer"] - (6 * 4096 * 14336 * 16384 + 2 * 8192 * 8 * 4096)) < 1
     assert work["bytes_layer"] == 3 * 8 * 4096 * 14336 * 2 + 2 * 8192 * 4096 * 2 + 8 * 4096 * 4
+    # per projection: its weights plus x (first) or y (second); no sorted or hidden rows
+    assert work["gemm1"]["bytes"] == 2 * 8 * 4096 * 14336 * 2 + 8192 * 4096 * 2
+    assert work["gemm2"]["bytes"] == 8 * 4096 * 14336 * 2 + 8192 * 4096 * 2
+
+
+def test_layer_work_switch_counts_only_experts_with_kept_rows():
+    w = WORKLOADS["switch_k1"]
+    kept = [160] * 25 + [0] * 7 + [100] * 32
+    work = bench.layer_work(w, kept)
+    assert work["active_experts"] == 57 and work["S"] == 25 * 160 + 32 * 100
+    assert work["gemm2"]["bytes"] == 57 * 768 * 3072 * 2 + 8192 * 768 * 2
+    assert work["gemm1"]["flops"] == 2.0 * work["S"] * 768 * 3072
 
 
 def test_kernel_roofline_picks_the_binding_resource():
@@ -65,6 +77,7 @@ def test_kernel_roofline_picks_the_binding_resource():
     assert r["bound"] == "tensor" and r["achieved"] == 1000.0 and abs(r["frac"] - 1000 / 1500) < 1e-4
     r = bench.kernel_roofline(flops=1e9, nbytes=3e9, seconds=1e-3, peaks=peaks)
     assert r["bound"] == "hbm" and r["achieved"] == 3000.0 and r["frac"] == 0.5
+    assert r["frac_nominal"] == round(3000.0 / bench.NOMINAL_PEAKS["hbm_gbs"], 4)
 
 
 def test_traffic_is_null_without_a_matching_profile(tmp_path, monkeypatch):
