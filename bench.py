@@ -49,9 +49,6 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2200.0}
 STAGE_KERNEL = {"router": "router_kernel", "scan": "scan_kernel", "dispatch": "dispatch_kernel",
                 "gemm1": "grouped_gemm_kernel", "gemm2": "grouped_gemm_kernel", "combine": "combine_kernel"}
-# oracle tokens per CPU-baseline sample, per workload (bounded to ~10-30 s of CPU work)
-CPU_SAMPLE_TOKENS = {"switch_k1": 8192, "mixtral_prefill": 128, "mixtral_decode_t1": 1, "mixtral_decode_t16": 16,
-                     "mixtral_decode_t64": 64, "fine_grained": 2048, "tiny_fp32": 64}
 
 
 # ----------------------------------------------------------------------------- helpers (host only)
@@ -229,51 +226,68 @@ def config_of(w, n_gpus):
 
 
 # ----------------------------------------------------------------------------- CPU (oracle) leg
-def cpu_oracle_run(w, inp, n_tokens):
-    """Time the oracle's forward on the first n_tokens tokens of the batch (full weights)."""
-    import numpy as np
-    import oracle
-
-    class Host:
-        def __init__(self, t):
-            self.t, self.c = t, {}
-
-        def __getitem__(self, e):
-            if e not in self.c:
-                self.c[e] = self.t[e].float().cpu().numpy()
-            return self.c[e]
-    x = inp["x"][:n_tokens].float().cpu().numpy()
-    W_r = inp["W_r"].float().cpu().numpy()
-    b_r = None if inp["b_r"] is None else inp["b_r"].float().cpu().numpy()
-    W1, W2 = Host(inp["W1"]), Host(inp["W2"])
-    W3 = None if inp["W3"] is None else Host(inp["W3"])
-    shared = None
-    if getattr(w, "n_shared", 0):
-        ids = range(w.E, w.E + w.n_shared)
-        shared = ([W1[e] for e in ids], None if W3 is None else [W3[e] for e in ids], [W2[e] for e in ids])
-    t0 = time.perf_counter()
-    oracle.moe_forward(x, W_r, b_r, W1, W3, W2, k=w.k, gate_mode=w.gate, act=w.act,
-                       capacity_factor=w.capacity_factor, shared=shared)
-    return time.perf_counter() - t0
+# Rows of y per host thread in one CPU-baseline sample (the routing always covers
+# every token): a few seconds of plain C++ loops per workload.
+CPU_ROWS_PER_THREAD = {"switch_k1": 256, "mixtral_prefill": 4, "fine_grained": 64, "fine_grained_shared": 48,
+                       "tiny_fp32": 64}
 
 
-def blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
-        if n:
-            return max(n)
-    except Exception:
-        pass
-    return os.cpu_count() or 1
+class CpuOracle:
+    """The C++ loop oracle on one workload's inputs, copied to host memory once."""
+
+    def __init__(self, w, inp):
+        from oracle import cpp
+        self.w = w
+        self.O = cpp.load()
+        self.host = {k: (None if v is None else v.detach().cpu()) for k, v in inp.items()}
+        self.hw_threads = self.O.hardware_threads() or (os.cpu_count() or 1)
+
+    def run(self, rows, threads):
+        """Seconds of one oracle forward: routing, capacity and losses over all T
+        tokens, y for the listed rows."""
+        w, h = self.w, self.host
+        shared = None
+        if w.n_shared:
+            ids = slice(w.E, w.E + w.n_shared)
+            shared = (h["W1"][ids], None if h["W3"] is None else h["W3"][ids], h["W2"][ids])
+        t0 = time.perf_counter()
+        self.O.moe_forward(h["x"], h["W_r"], h["b_r"], h["W1"], h["W3"], h["W2"], k=w.k, gate_mode=w.gate,
+                           act=w.act, capacity_factor=w.capacity_factor, rows=rows, shared=shared, threads=threads)
+        return time.perf_counter() - t0
+
+    def sample_rows(self, per_thread, threads):
+        n = min(self.w.T, max(1, per_thread * threads))
+        return list(range(n)), n
+
+
+def layer_rate(T, t_route, t_sample, n):
+    """Tokens/s of the whole layer on the host, from the seconds of routing all T
+    tokens (t_route) and of routing plus y for n of them (t_sample): y of the
+    other T - n tokens costs the same per row."""
+    per_row = max(t_sample - t_route, 0.0) / max(n, 1)
+    return T / (t_route + per_row * T)
 
 
 def cpu_baseline(w, inp):
-    n = min(w.T, CPU_SAMPLE_TOKENS.get(w.name, 256))
-    secs = cpu_oracle_run(w, inp, n)
-    return {"value": round(n / secs, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"oracle forward (float64 NumPy) on the first {n} of {w.T} tokens with the full weights; "
-                      f"{secs:.2f} s wall on the host"}
+    """The C++ oracle timed on the host cores, as tokens/s of the whole layer:
+    all hardware threads over tokens (the reported value), and one thread."""
+    co = CpuOracle(w, inp)
+    per = CPU_ROWS_PER_THREAD.get(w.name, w.T)
+    nt = co.hw_threads
+    out = {}
+    for threads, rows_per in ((nt, per), (1, max(1, per // 8))):
+        rows, n = co.sample_rows(rows_per, threads)
+        t_route = co.run([], threads)
+        t_sample = co.run(rows, threads)
+        out[threads] = (layer_rate(w.T, t_route, t_sample, n), n, t_route, t_sample)
+    v, n, tr, ts = out[nt]
+    v1, n1, tr1, ts1 = out[1]
+    return {"value": round(v, 3), "unit": "tokens/s", "cores": nt, "kind": "oracle",
+            "single_thread_value": round(v1, 3),
+            "sample": f"C++ loop oracle (oracle/moe_oracle.cpp, float64), {nt} threads over tokens: routing, "
+                      f"capacity and losses of all {w.T} tokens ({tr:.2f} s), plus y of the first {n} tokens "
+                      f"({ts - tr:.2f} s more), the y rows extrapolated to all {w.T}; single_thread_value: the same "
+                      f"on 1 thread with y of {n1} tokens ({tr1:.2f} s + {ts1 - tr1:.2f} s)"}
 
 
 # ----------------------------------------------------------------------------- GPU leg
@@ -656,26 +670,32 @@ def backward_bench(args, w, inp, warmup, world, rank, local, dev):
 
 
 def reference_arm(args, w, warmup):
-    """The oracle timed on the host cores (rank 0 only): the reference arm of this benchmark."""
+    """The C++ loop oracle timed on the host cores (rank 0 only): the reference
+    arm of this benchmark.  Each step routes all T tokens and computes y for a
+    bounded sample of them (one row per hardware thread at most)."""
     import torch
     from sparse_mixture_experts_gating_b200.workloads import make_inputs
 
-    n = min(w.T, max(1, CPU_SAMPLE_TOKENS.get(w.name, 256) // 4))
     inp = make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
-    for _ in range(warmup):
-        cpu_oracle_run(w, inp, n)
-    secs = [cpu_oracle_run(w, inp, n) for _ in range(args.steps)]
+    co = CpuOracle(w, inp)
+    del inp
+    nt = co.hw_threads
+    per = 1 if w.name in ("mixtral_prefill",) else max(1, CPU_ROWS_PER_THREAD.get(w.name, w.T) // 8)
+    rows, n = co.sample_rows(per, nt)
+    t_route = min(co.run([], nt) for _ in range(warmup))
+    secs = [co.run(rows, nt) for _ in range(args.steps)]
     total = sum(secs)
-    value = n * args.steps / total
-    cores = blas_threads()
+    value = layer_rate(w.T, t_route, total / args.steps, n)
     line = {
         "metric": METRIC, "impl": "reference", "value": round(value, 3), "unit": "tokens/s",
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": warmup,
         "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
         "config": dict(config_of(w, int(os.environ.get("WORLD_SIZE", "1"))), hidden=args.hidden),
-        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"each step: oracle forward (float64 NumPy) on the first {n} of {w.T} tokens"},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": nt, "kind": "oracle",
+                         "sample": f"each step: C++ loop oracle (float64), {nt} threads over tokens, routing all "
+                                   f"{w.T} tokens and computing y for the first {n}; value: tokens/s of the whole "
+                                   f"layer, y rows extrapolated to all {w.T} (routing alone: {t_route:.3f} s)"},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

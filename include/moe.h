@@ -125,11 +125,12 @@ MOE_API int moe_create(int num_experts, int k, int d, int d_ff, int act, int gat
  *     (about 16 significant bits); the second projection runs its tensor-core
  *     MMAs on both planes, twice the tensor work of that projection.
  *   MOE_HIDDEN_BF16: one bf16 number (8 significant bits, unit roundoff 2^-8).
- *     OUTSIDE THE PARITY BAR for the maximum error: against an fp32 reference
- *     on the same bf16 inputs, the rounding of the hidden activation alone
- *     gives max|dy| of about 1.5e-2 * RMS(y) on layers with millions of
- *     outputs (the bar is 1e-2 * RMS); the mean relative error (about 1.6e-3)
- *     stays within 2e-3.  Use it only where that is acceptable.
+ *     OUTSIDE THE PARITY BAR: against an fp32 reference on the same bf16
+ *     inputs, the rounding of the hidden activation alone gives max|dy| of
+ *     about 1.5e-2 * RMS(y) on layers with millions of outputs (the bar is
+ *     1e-2 * RMS) and a mean relative error of about 1.6e-3 before the final
+ *     cast, which the cast to bf16 raises to about 2.3e-3 in the returned y
+ *     (the bar is 2e-3).  Use it only where that is acceptable.
  * Changes moe_workspace_bytes().  fp32 layers ignore it.  Returns MOE_OK or
  * MOE_ERR_INVALID_ARG.
  */

@@ -11,8 +11,11 @@ Tolerances (derived from the arithmetic; see the design notes):
     that value and on the returned bf16 y; the returned y must be exactly the
     round-to-nearest-even image of the fp32 value.  With the hidden activation
     held in ONE bf16 plane (MOE_HIDDEN_BF16) its rounding alone (unit roundoff
-    2^-8) pushes the max to ~1.5e-2 * RMS on large outputs: that mode is held
-    to the mean bound only, its max error is reported;
+    2^-8) pushes the max to ~1.5e-2 * RMS on large outputs and adds ~1.6e-3 of
+    mean relative error, on top of the ~1.3e-3 of the final cast: that mode is
+    outside the bar; it is held to the mean bound on the fp32 value and to
+    3e-3 (the sum of the two terms) on the returned bf16 y, its max error is
+    reported;
   * gates: |dg| <= 2e-6 (fp32 exp of exact logit differences);
   * aux, z: relative 1e-5.
 """
@@ -134,14 +137,15 @@ def y_errors(y_gpu: np.ndarray, y_ref: np.ndarray):
     }
 
 
-def assert_y_close(w: Workload, g: dict, y_ref: np.ndarray, rows=None, max_bound=True):
+def assert_y_close(w: Workload, g: dict, y_ref: np.ndarray, rows=None, single_plane_hidden=False):
     """y of the CUDA path against the plain oracle y_ref.
 
     fp32 layers: max|dy| / max|y_ref| <= 1e-5.  bf16 layers: the mean bound
-    on the fp32 value before the cast and on the returned bf16 y, the max
-    bound 1e-2 * RMS(y_ref) on the fp32 value unless max_bound is False (the
-    single-plane hidden mode, which is outside that bound), and the returned
-    y bit for bit the round-to-nearest-even image of the fp32 value.
+    2e-3 on the fp32 value before the cast and on the returned bf16 y, the max
+    bound 1e-2 * RMS(y_ref) on the fp32 value, and the returned y bit for bit
+    the round-to-nearest-even image of the fp32 value.  single_plane_hidden
+    (the MOE_HIDDEN_BF16 mode, outside the bar): no max bound, and 3e-3 for
+    the mean of the returned bf16 y.
     """
     sel = slice(None) if rows is None else np.asarray(rows)
     if w.dtype == DTYPE_F32:
@@ -152,8 +156,8 @@ def assert_y_close(w: Workload, g: dict, y_ref: np.ndarray, rows=None, max_bound
     e = y_errors(yf, y_ref)
     e["bf16_output"] = y_errors(g["y"][sel], y_ref)
     assert e["mean_rel"] <= 2e-3, e
-    assert e["bf16_output"]["mean_rel"] <= 2e-3, e
-    if max_bound:
+    assert e["bf16_output"]["mean_rel"] <= (3e-3 if single_plane_hidden else 2e-3), e
+    if not single_plane_hidden:
         assert e["max_over_rms"] <= 1e-2, e
     # the bf16 output is the RNE image of the fp32 value
     rne = torch.from_numpy(np.ascontiguousarray(yf)).to(torch.bfloat16)

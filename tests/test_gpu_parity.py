@@ -99,14 +99,15 @@ SINGLE = [c for c in SMALL if c[9] == BF and c[0] in ("swiglu_e8_k2", "switch_re
 @pytest.mark.parametrize("case", SINGLE, ids=[c[0] for c in SINGLE])
 def test_small_layers_single_bf16_hidden(case):
     """Hidden activation held in one bf16 plane: same routing, y within the
-    mean bound against the plain oracle (this mode is outside the max bound)."""
+    mean bound against the plain oracle (this mode is outside the bar: see
+    assert_y_close)."""
     w = _small(case)
     inp = make_inputs(w, device="cuda")
     g = run_gpu(w, inp, layer=layer_for(w, hidden="bf16"))
     host = host_inputs(inp)
     o = run_oracle(w, host)
     assert_routing_equal(g, o)
-    assert_y_close(w, g, o["y"], max_bound=False)
+    assert_y_close(w, g, o["y"], single_plane_hidden=True)
 
 
 def test_ties_go_to_the_lower_expert_index():
@@ -295,4 +296,4 @@ def test_full_size_single_bf16_hidden(name):
     assert_routing_equal(g, o_route)
     rows = sample_rows(w, o_route["kept"], n=24, seed=3)
     o = run_oracle(w, host, rows=rows, logits=o_route["logits"])
-    assert_y_close(w, g, o["y"], rows=rows, max_bound=False)
+    assert_y_close(w, g, o["y"], rows=rows, single_plane_hidden=True)

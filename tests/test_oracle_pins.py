@@ -3,6 +3,10 @@
 No test here compares the oracle with itself: each check uses a closed form,
 brute force, a library routine (torch / scipy) or a value derived by hand from
 the page "Mixture of experts" (rayaq.ca), stored under tests/golden/.
+
+Every pin runs against both oracles: the NumPy restatement
+(oracle/moe_oracle.py) and the plain C++ loops (oracle/moe_oracle.cpp,
+through oracle/cpp.py).
 """
 import itertools
 import math
@@ -13,15 +17,24 @@ import scipy.special
 import torch
 import torch.nn.functional as F
 
-import oracle as O
+import oracle
+from oracle import cpp as oracle_cpp
 from tests._golden import load
+
+IMPLS = {"numpy": lambda: oracle, "cpp": lambda: oracle_cpp.load()}
+
+
+@pytest.fixture(params=sorted(IMPLS))
+def O(request):
+    """The oracle under test: the NumPy module or the C++ library binding."""
+    return IMPLS[request.param]()
 
 rng = np.random.default_rng(7)
 
 
 # ---------------------------------------------------------------- top-k
 @pytest.mark.parametrize("E", [1, 2, 3, 5, 7, 8])
-def test_top_k_matches_brute_force_with_ties(E):
+def test_top_k_matches_brute_force_with_ties(O, E):
     """Top-k gating: k largest logits, largest first; ties -> lower index.
 
     Brute force over all k-subsets: the chosen set has the maximal logit sum,
@@ -41,20 +54,20 @@ def test_top_k_matches_brute_force_with_ties(E):
             assert idx[t].tolist() == order
 
 
-def test_top_k_signed_zero_is_a_tie():
+def test_top_k_signed_zero_is_a_tie(O):
     h = np.array([[-0.0, 0.0], [0.0, -0.0]], np.float32)
     assert O.top_k(h, 1)[:, 0].tolist() == [0, 0]
 
 
 # ---------------------------------------------------------------- softmax, lse, logits
-def test_softmax_and_lse_match_scipy():
+def test_softmax_and_lse_match_scipy(O):
     h = rng.normal(size=(50, 9)).astype(np.float32) * 5
     p, lse = O.softmax_lse(h)
     np.testing.assert_allclose(p, scipy.special.softmax(h.astype(np.float64), axis=1), rtol=1e-13)
     np.testing.assert_allclose(lse, scipy.special.logsumexp(h.astype(np.float64), axis=1), rtol=1e-13)
 
 
-def test_router_logits_match_linear_and_are_order_free_on_dyadic_inputs():
+def test_router_logits_match_linear_and_are_order_free_on_dyadic_inputs(O):
     """h = W_r x + b (one linear layer with E rows); dyadic inputs give exact fp32."""
     x = np.clip(np.round(rng.normal(size=(33, 64)) * 64) / 64, -4, 4)
     W = np.clip(np.round(rng.normal(size=(6, 64)) / 8 * 1024) / 1024, -1, 1)
@@ -76,7 +89,7 @@ def test_router_logits_match_linear_and_are_order_free_on_dyadic_inputs():
 
 
 # ---------------------------------------------------------------- gates
-def test_renorm_gates_sum_to_one_and_equal_conditional_probabilities():
+def test_renorm_gates_sum_to_one_and_equal_conditional_probabilities(O):
     """Top-k gating, renormalised bullet: g = p_sel / sum(p_sel), sums to 1."""
     h = (rng.normal(size=(40, 8)) * 3).astype(np.float32)
     p = scipy.special.softmax(h.astype(np.float64), axis=1)
@@ -89,7 +102,7 @@ def test_renorm_gates_sum_to_one_and_equal_conditional_probabilities():
         assert np.all(np.diff(g, axis=1) <= 1e-15)  # largest first
 
 
-def test_switch_gate_is_max_probability_below_one():
+def test_switch_gate_is_max_probability_below_one(O):
     """Top-k gating, Switch bullet: gate = the argmax expert's full-softmax p < 1."""
     h = (rng.normal(size=(40, 8)) * 3).astype(np.float32)
     p = scipy.special.softmax(h.astype(np.float64), axis=1)
@@ -99,7 +112,7 @@ def test_switch_gate_is_max_probability_below_one():
     assert np.all(g < 1.0)
 
 
-def test_closed_form_golden_routing():
+def test_closed_form_golden_routing(O):
     G = load("closed_form_routing.txt")
     h = np.array([G["logits_t0"], G["logits_t1"]], np.float32)
     p, lse = O.softmax_lse(h)
@@ -124,7 +137,7 @@ def test_closed_form_golden_routing():
 
 
 # ---------------------------------------------------------------- losses
-def test_aux_is_one_under_uniform_routing():
+def test_aux_is_one_under_uniform_routing(O):
     """The load-balancing loss: uniform first choices give E*sum f P = 1 (so alpha*1)."""
     for E in (2, 4, 8, 64):
         T = 4 * E
@@ -135,7 +148,7 @@ def test_aux_is_one_under_uniform_routing():
         assert 0.01 * r["aux"] == pytest.approx(0.01, abs=1e-14)
 
 
-def test_aux_tends_to_E_when_collapsed():
+def test_aux_tends_to_E_when_collapsed(O):
     """Every token to one expert with probability ~1 gives E*sum f P -> E."""
     E, T = 8, 32
     x = rng.normal(size=(T, 16))
@@ -147,7 +160,7 @@ def test_aux_tends_to_E_when_collapsed():
     assert r["aux"] == pytest.approx(E, rel=1e-12)
 
 
-def test_z_loss_closed_form():
+def test_z_loss_closed_form(O):
     """All logits equal to c: lse = c + ln E, so z = (c + ln E)^2."""
     for E, c in [(4, 0.0), (8, 2.5), (128, -3.0)]:
         h = np.full((5, E), c, np.float32)
@@ -156,7 +169,7 @@ def test_z_loss_closed_form():
         assert z == pytest.approx((c + math.log(E)) ** 2, rel=1e-12)
 
 
-def test_balance_losses_are_zero_and_one_under_uniform_routing():
+def test_balance_losses_are_zero_and_one_under_uniform_routing(O):
     """Uniform routing: equal assignment counts and equal P_i give a coefficient
     of variation 0, cv^2 0, and the all-choices Switch loss E*sum f P = 1."""
     for E, k in [(4, 1), (8, 2), (16, 4)]:
@@ -169,7 +182,7 @@ def test_balance_losses_are_zero_and_one_under_uniform_routing():
         assert r["aux_all_choices"] == pytest.approx(1.0, abs=1e-12)
 
 
-def test_balance_losses_closed_forms_when_collapsed():
+def test_balance_losses_closed_forms_when_collapsed(O):
     """All T tokens to expert 0 with probability 1 (k = 1): counts (T, 0, ..., 0)
     have mean T/E and standard deviation (T/E) sqrt(E - 1), so CV = sqrt(E - 1);
     P = e_0 gives cv^2 = E - 1; the all-choices loss equals E."""
@@ -183,7 +196,7 @@ def test_balance_losses_closed_forms_when_collapsed():
         assert r["aux_all_choices"] == pytest.approx(E, rel=1e-12)
 
 
-def test_all_choices_loss_equals_switch_loss_at_k1_and_counts_every_choice():
+def test_all_choices_loss_equals_switch_loss_at_k1_and_counts_every_choice(O):
     """k = 1: first choices are all choices, so the two losses agree; k = 2 with
     second choices on one expert: f over all choices differs from first choices."""
     E, T, d = 6, 40, 9
@@ -205,7 +218,7 @@ def test_all_choices_loss_equals_switch_loss_at_k1_and_counts_every_choice():
 
 
 # ---------------------------------------------------------------- capacity
-def test_capacity_formula():
+def test_capacity_formula(O):
     """Capacity and dropped tokens: C = tokens/experts x factor (x k for top-k)."""
     assert O.expert_capacity(1.25, 8192, 1, 64) == 160
     assert O.expert_capacity(2.0, 16384, 4, 128) == 1024
@@ -215,7 +228,7 @@ def test_capacity_formula():
     assert O.expert_capacity(-1.0, 10, 2, 4) is None
 
 
-def test_dropless_keeps_everything():
+def test_dropless_keeps_everything(O):
     idx = rng.integers(0, 5, size=(300, 1))
     s = O.assign_slots(idx, 5, None)
     assert s["dropped"] == 0 and s["kept"].all()
@@ -223,7 +236,7 @@ def test_dropless_keeps_everything():
 
 
 @pytest.mark.parametrize("C", [1, 3, 17])
-def test_position_order_dropping_k1(C):
+def test_position_order_dropping_k1(O, C):
     """Slots fill in position order: the kept tokens of an expert are its first C."""
     T, E = 400, 6
     idx = rng.integers(0, E, size=(T, 1))
@@ -237,7 +250,7 @@ def test_position_order_dropping_k1(C):
     assert s["kept"].sum() + s["dropped"] == T
 
 
-def test_slot_priority_is_token_order_across_choices():
+def test_slot_priority_is_token_order_across_choices(O):
     """A token's second choice takes a slot before a later token's first choice."""
     idx = np.array([[1, 0], [0, 2], [0, 1]])  # expert 0: (t0,j1), (t1,j0), (t2,j0)
     s = O.assign_slots(idx, 3, 2)
@@ -248,7 +261,7 @@ def test_slot_priority_is_token_order_across_choices():
     assert s["dest_row"].tolist() == [[2, 0], [1, 4], [-1, 3]]
 
 
-def test_worked_example_reconstruction():
+def test_worked_example_reconstruction(O):
     G = load("worked_example_capacity.txt")
     idx = np.array(G["first_choice"])[:, None]
     for cf, cap, drops in [(1.0, G["cf1_capacity"], G["cf1_dropped_tokens"]),
@@ -267,13 +280,13 @@ def test_worked_example_reconstruction():
 # ---------------------------------------------------------------- whole-layer reductions
 def _torch_ffn(x, W1, W3, W2, act):
     a = F.linear(x, W1)
-    hdn = F.relu(a) if act == O.ACT_RELU else F.silu(a) * F.linear(x, W3)
+    hdn = F.relu(a) if act == oracle.ACT_RELU else F.silu(a) * F.linear(x, W3)
     return F.linear(hdn, W2)
 
 
-@pytest.mark.parametrize("act", [O.ACT_RELU, O.ACT_SWIGLU])
-@pytest.mark.parametrize("gate_mode", [O.GATE_RENORM, O.GATE_SWITCH])
-def test_single_expert_is_the_dense_ffn(act, gate_mode):
+@pytest.mark.parametrize("act", [oracle.ACT_RELU, oracle.ACT_SWIGLU])
+@pytest.mark.parametrize("gate_mode", [oracle.GATE_RENORM, oracle.GATE_SWITCH])
+def test_single_expert_is_the_dense_ffn(O, act, gate_mode):
     """E = 1, k = 1: the router always picks the only expert with gate 1 -> dense FFN."""
     T, d, dff = 23, 12, 20
     x = rng.normal(size=(T, d)); W_r = rng.normal(size=(1, d))
@@ -285,8 +298,8 @@ def test_single_expert_is_the_dense_ffn(act, gate_mode):
     assert r["gate"].tolist() == [[1.0]] * T
 
 
-@pytest.mark.parametrize("act", [O.ACT_RELU, O.ACT_SWIGLU])
-def test_k_equals_E_is_the_dense_softmax_mixture(act):
+@pytest.mark.parametrize("act", [oracle.ACT_RELU, oracle.ACT_SWIGLU])
+def test_k_equals_E_is_the_dense_softmax_mixture(O, act):
     """k = E, no capacity: y = sum_e softmax(h)_e E_e(x), every expert weighted."""
     T, d, dff, E = 17, 10, 14, 5
     x = rng.normal(size=(T, d)); W_r = rng.normal(size=(E, d)); b = rng.normal(size=E)
@@ -300,7 +313,7 @@ def test_k_equals_E_is_the_dense_softmax_mixture(act):
     np.testing.assert_allclose(r["y"], ref.numpy(), rtol=1e-10, atol=1e-12)
 
 
-def test_sampled_rows_equal_full_rows_and_dropped_tokens_are_zero():
+def test_sampled_rows_equal_full_rows_and_dropped_tokens_are_zero(O):
     T, d, dff, E, k = 60, 8, 12, 4, 2
     x = rng.normal(size=(T, d)); W_r = rng.normal(size=(E, d))
     W1 = rng.normal(size=(E, dff, d)); W2 = rng.normal(size=(E, d, dff))
@@ -323,8 +336,8 @@ def test_sampled_rows_equal_full_rows_and_dropped_tokens_are_zero():
 
 
 # ---------------------------------------------------------------- shared experts
-@pytest.mark.parametrize("act", [O.ACT_RELU, O.ACT_SWIGLU])
-def test_shared_expert_with_silent_routed_experts_is_the_dense_ffn(act):
+@pytest.mark.parametrize("act", [oracle.ACT_RELU, oracle.ACT_SWIGLU])
+def test_shared_expert_with_silent_routed_experts_is_the_dense_ffn(O, act):
     """Routed experts whose output is zero (W2 = 0): y is the sum of the shared
     experts' dense FFNs, for every token."""
     T, d, dff, E, ns = 19, 8, 12, 4, 2
@@ -338,7 +351,7 @@ def test_shared_expert_with_silent_routed_experts_is_the_dense_ffn(act):
     np.testing.assert_allclose(r["y"], ref.numpy(), rtol=1e-12, atol=1e-12)
 
 
-def test_shared_copy_of_the_single_expert_doubles_the_output():
+def test_shared_copy_of_the_single_expert_doubles_the_output(O):
     """E = 1, k = 1 (gate 1) and one shared expert with the same weights: y = 2 FFN(x)."""
     T, d, dff = 11, 6, 10
     x = rng.normal(size=(T, d)); W_r = rng.normal(size=(1, d))
@@ -349,7 +362,7 @@ def test_shared_copy_of_the_single_expert_doubles_the_output():
     np.testing.assert_allclose(r["y"], 2 * ref.numpy(), rtol=1e-12, atol=1e-12)
 
 
-def test_dropped_tokens_still_get_the_shared_experts():
+def test_dropped_tokens_still_get_the_shared_experts(O):
     """Capacity drops routed assignments only: a token with every routed choice
     dropped gets exactly the shared output; routing, counts and losses do not
     see the shared experts."""
