@@ -56,13 +56,14 @@ typedef struct moe_layer* moe_handle;
 enum { MOE_ACT_RELU = 0, MOE_ACT_SWIGLU = 1 };
 enum { MOE_GATE_SWITCH = 0, MOE_GATE_RENORM = 1 };
 enum { MOE_F32 = 0, MOE_BF16 = 1 };
-enum { MOE_HIDDEN_BF16X2 = 0, MOE_HIDDEN_BF16 = 1 };
+enum { MOE_HIDDEN_BF16X2 = 0, MOE_HIDDEN_BF16 = 1, MOE_HIDDEN_F16 = 2, MOE_HIDDEN_AUTO = 3 };
 enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1, /* bad shape, mode, null pointer or too small workspace */
   MOE_ERR_UNSUPPORTED = 2, /* valid layer this build cannot run (alignment, limits) */
   MOE_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
-  MOE_ERR_TIMEOUT = 4      /* a device-side bounded wait ran out (kernel gave up) */
+  MOE_ERR_TIMEOUT = 4,     /* a device-side bounded wait ran out (kernel gave up) */
+  MOE_ERR_RANGE = 5        /* MOE_HIDDEN_F16: a hidden value (or W2) beyond the fp16 range */
 };
 
 /* Kernel stages of one forward call, in launch order (see moe_debug.events). */
@@ -121,9 +122,20 @@ MOE_API int moe_create(int num_experts, int k, int d, int d_ff, int act, int gat
 /*
  * bf16 layers: how the hidden activation between the two expert projections
  * is held (no counterpart on the pages, which fix only the router at fp32):
- *   MOE_HIDDEN_BF16X2 (default): as the sum of two bf16 numbers hi + lo
- *     (about 16 significant bits); the second projection runs its tensor-core
- *     MMAs on both planes, twice the tensor work of that projection.
+ *   MOE_HIDDEN_BF16X2: as the sum of two bf16 numbers hi + lo (about 16
+ *     significant bits); the second projection runs its tensor-core MMAs on
+ *     both planes, twice the tensor work of that projection.
+ *   MOE_HIDDEN_F16: as one fp16 number (11 significant bits); the second
+ *     projection multiplies it by an fp16 image of W2 that each call makes
+ *     in the workspace while the first projection runs (bf16 -> fp16 is exact
+ *     for |w| in [2^-17, 65504]; smaller weights move by at most 2^-25).  One
+ *     plane of MMAs.  |hidden| and |W2| must stay below 65504: a larger value
+ *     makes moe_status() report MOE_ERR_RANGE and that call's outputs are
+ *     undefined.
+ *   MOE_HIDDEN_AUTO (default): MOE_HIDDEN_F16 when the batch averages at least
+ *     1024 rows per expert (shared experts counted), where the second
+ *     projection is bound by the tensor cores; MOE_HIDDEN_BF16X2 otherwise,
+ *     where it is bound by the weight stream and the pair costs no time.
  *   MOE_HIDDEN_BF16: one bf16 number (8 significant bits, unit roundoff 2^-8).
  *     OUTSIDE THE PARITY BAR: against an fp32 reference on the same bf16
  *     inputs, the rounding of the hidden activation alone gives max|dy| of
@@ -131,8 +143,9 @@ MOE_API int moe_create(int num_experts, int k, int d, int d_ff, int act, int gat
  *     1e-2 * RMS) and a mean relative error of about 1.6e-3 before the final
  *     cast, which the cast to bf16 raises to about 2.3e-3 in the returned y
  *     (the bar is 2e-3).  Use it only where that is acceptable.
- * Changes moe_workspace_bytes().  fp32 layers ignore it.  Returns MOE_OK or
- * MOE_ERR_INVALID_ARG.
+ * Changes moe_workspace_bytes() (MOE_HIDDEN_F16 and the automatic mode at
+ * large batches add the W2 image: (E + n_shared) * d * d_ff * 2 bytes).
+ * fp32 layers ignore it.  Returns MOE_OK or MOE_ERR_INVALID_ARG.
  */
 MOE_API int moe_set_hidden_precision(moe_handle h, int mode);
 
@@ -272,8 +285,9 @@ MOE_API int moe_backward(moe_handle h, int64_t T, const void* x, const float* W_
 /*
  * Synchronise `stream` and report the device error word of the current device:
  * MOE_OK, MOE_ERR_TIMEOUT (a kernel's bounded wait ran out and it returned
- * early; outputs of that call are undefined) or MOE_ERR_CUDA.  The error
- * word stays set until moe_clear_status().
+ * early; outputs of that call are undefined), MOE_ERR_RANGE (fp16 hidden mode:
+ * a value beyond the fp16 range; outputs of that call are undefined) or
+ * MOE_ERR_CUDA.  The error word stays set until moe_clear_status().
  */
 MOE_API int moe_status(void* stream);
 

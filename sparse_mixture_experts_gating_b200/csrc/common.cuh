@@ -4,12 +4,13 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace moe {
 
 // Device error codes written into the per-device error word (first one wins).
-enum : unsigned int { DEV_OK = 0, DEV_ERR_TIMEOUT = 4 };
+enum : unsigned int { DEV_OK = 0, DEV_ERR_TIMEOUT = 4, DEV_ERR_RANGE = 5 };
 
 // Default limit of every bounded wait in the pipelined kernels.  A healthy
 // wait lasts at most one tile (well under a millisecond).
@@ -158,7 +159,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
+// Instruction descriptor, kind::f16: fp16 A and B (both K-major), fp32 D.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4)                                   // D format: f32 (A and B format fields 0: f16)
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread (bf16 or fp16
+// operands, as the instruction descriptor says).
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
   asm volatile(
@@ -229,6 +238,14 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
 // ------------------------------------------------------------------ misc
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Two floats as an fp16 pair (round to nearest even); *bad is raised when a
+// value is beyond the fp16 range (it would round to infinity) or NaN.
+__device__ __forceinline__ uint32_t pack_f16x2_checked(float lo, float hi, bool& bad) {
+  bad |= !(fabsf(lo) < 65520.f) || !(fabsf(hi) < 65520.f);
+  __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 

@@ -59,7 +59,6 @@ struct Geo {
   static constexpr int STAGES = (200 * 1024 / STAGE_BYTES) < MAX_STAGES ? (200 * 1024 / STAGE_BYTES) : MAX_STAGES;
 };
 constexpr uint32_t TMEM_COLS = 2 * MMA_N;
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, MMA_N);
 constexpr int MAX_E = 256;
 
 using Params = TcParams;
@@ -152,16 +151,22 @@ __device__ __forceinline__ void split_bf16(float v0, float v1, uint32_t& hi, uin
   lo = pack_bf16x2(v0 - hf.x, v1 - hf.y);
 }
 
-// EPI: epilogue (internal.h GemmEpi).  SPLIT: for the first projection the
-// epilogue writes the hidden activation as hi/lo planes; for the second the
-// A operand is read as hi (tmA) + lo (tmA2) planes.
-template <int EPI, bool SPLIT, int AR>
+// EPI: epilogue (internal.h GemmEpi).  HID (internal.h HiddenKind): how the
+// hidden activation is held.  HID_BF16X2: the first projection's epilogue
+// writes it as hi/lo bf16 planes, the second reads its A operand as hi (tmA)
+// + lo (tmA2) planes.  HID_F16: the first projection writes it as fp16 (and
+// flags values beyond the fp16 range), the second multiplies fp16 A by an
+// fp16 image of its weights.
+template <int EPI, int HID, int AR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                         const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                         const Params p) {
-  constexpr bool A_SPLIT = SPLIT && (EPI == EPI_GATE_F32 || EPI == EPI_GATE_SCATTER_BF16);
-  constexpr bool OUT_SPLIT = SPLIT && (EPI == EPI_RELU_BF16 || EPI == EPI_SWIGLU_BF16);
+  constexpr bool GATE = EPI == EPI_GATE_F32 || EPI == EPI_GATE_SCATTER_BF16;
+  constexpr bool A_SPLIT = HID == HID_BF16X2 && GATE;
+  constexpr bool OUT_SPLIT = HID == HID_BF16X2 && !GATE;
+  constexpr bool OUT_F16 = HID == HID_F16 && !GATE;
+  constexpr uint32_t IDESC = (HID == HID_F16 && GATE) ? idesc_f16_f32(BM, MMA_N) : idesc_bf16_f32(BM, MMA_N);
   using G = Geo<A_SPLIT, AR>;
   constexpr int STAGES = G::STAGES;
   constexpr int STAGE_BYTES = G::STAGE_BYTES;
@@ -316,6 +321,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
       if (EPI == EPI_SWIGLU_BF16 || EPI == EPI_RELU_BF16 || EPI == EPI_GATE_SCATTER_BF16) {
         constexpr int NCH = (EPI == EPI_SWIGLU_BF16) ? 4 : 8;
+        bool out_of_range = false;  // OUT_F16: a hidden value beyond the fp16 range
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
         __nv_bfloat16* out_lo = static_cast<__nv_bfloat16*>(p.out_lo);
 #pragma unroll 1
@@ -332,6 +338,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const float h0 = silu_mul(__uint_as_float(ra[2 * i]), __uint_as_float(rb[2 * i]));
               const float h1 = silu_mul(__uint_as_float(ra[2 * i + 1]), __uint_as_float(rb[2 * i + 1]));
               if (OUT_SPLIT) split_bf16(h0, h1, hi[i], lo[i]);
+              else if (OUT_F16) hi[i] = pack_f16x2_checked(h0, h1, out_of_range);
               else hi[i] = pack_bf16x2(h0, h1);
             }
           } else {
@@ -348,6 +355,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 h1 *= g;
               }
               if (OUT_SPLIT) split_bf16(h0, h1, hi[i], lo[i]);
+              else if (OUT_F16) hi[i] = pack_f16x2_checked(h0, h1, out_of_range);
               else hi[i] = pack_bf16x2(h0, h1);
             }
             if (EPI == EPI_GATE_SCATTER_BF16 && p.out_f32 != nullptr && vrow) {  // debug copy
@@ -377,6 +385,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             __syncwarp();
           }
         }
+        if (OUT_F16 && __any_sync(0xffffffffu, out_of_range) && lane == 0) record_error(p.err, DEV_ERR_RANGE);
       } else {  // EPI_GATE_F32: gated fp32 rows of the expert-sorted buffer (partial ks)
         float* out = static_cast<float*>(p.out) + static_cast<int64_t>(ks) * p.split_stride;
 #pragma unroll 1
@@ -442,6 +451,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
   return make_map_bf16(m, base, rows, cols, 128);
 }
 
+// Row-major 16-bit matrix [rows][cols] of the given type -> map with box
+// [box_rows][64 cols], 128-byte swizzle.
+bool make_map_16(CUtensorMap* m, CUtensorMapDataType type, const void* base, uint64_t rows, uint64_t cols,
+                 uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 bool make_map_planes_bf16(CUtensorMap* m, const void* base, uint64_t plane_stride, uint64_t rows, uint64_t cols,
@@ -471,23 +495,65 @@ bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t col
 
 namespace {
 
-template <int EPI, bool SPLIT, int AR>
+template <int EPI, int HID, int AR>
 cudaError_t launch_t(const TcGemmPlan& pl, int num_sms, cudaStream_t s) {
-  constexpr bool A_SPLIT = SPLIT && (EPI == EPI_GATE_F32 || EPI == EPI_GATE_SCATTER_BF16);
+  constexpr bool A_SPLIT = HID == HID_BF16X2 && (EPI == EPI_GATE_F32 || EPI == EPI_GATE_SCATTER_BF16);
   constexpr size_t bytes = smem_bytes<A_SPLIT, AR>();
   static_assert(bytes <= 227 * 1024, "grouped GEMM shared memory");
-  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void*>(&grouped_gemm_kernel<EPI, SPLIT, AR>),
+  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void*>(&grouped_gemm_kernel<EPI, HID, AR>),
                                       static_cast<int>(bytes));
   if (e != cudaSuccess) return e;
-  return launch_pdl(grouped_gemm_kernel<EPI, SPLIT, AR>, dim3(num_sms), dim3(NUM_THREADS), bytes, s, pl.a, pl.a2,
+  return launch_pdl(grouped_gemm_kernel<EPI, HID, AR>, dim3(num_sms), dim3(NUM_THREADS), bytes, s, pl.a, pl.a2,
                     pl.b0, pl.b1, pl.p);
 }
 
-template <int EPI, bool SPLIT>
+template <int EPI, int HID>
 cudaError_t launch_ar(const TcGemmPlan& pl, int num_sms, cudaStream_t s) {
-  if (pl.ar == 32) return launch_t<EPI, SPLIT, 32>(pl, num_sms, s);
-  if (pl.ar == 64) return launch_t<EPI, SPLIT, 64>(pl, num_sms, s);
-  return launch_t<EPI, SPLIT, 128>(pl, num_sms, s);
+  if (pl.ar == 32) return launch_t<EPI, HID, 32>(pl, num_sms, s);
+  if (pl.ar == 64) return launch_t<EPI, HID, 64>(pl, num_sms, s);
+  return launch_t<EPI, HID, 128>(pl, num_sms, s);
+}
+
+template <int HID>
+cudaError_t launch_epi(const TcGemmPlan& pl, int num_sms, cudaStream_t s) {
+  switch (pl.epi) {
+    case EPI_RELU_BF16: return launch_ar<EPI_RELU_BF16, HID>(pl, num_sms, s);
+    case EPI_SWIGLU_BF16: return launch_ar<EPI_SWIGLU_BF16, HID>(pl, num_sms, s);
+    case EPI_GATE_F32: return launch_ar<EPI_GATE_F32, HID>(pl, num_sms, s);
+    default: return launch_ar<EPI_GATE_SCATTER_BF16, HID>(pl, num_sms, s);
+  }
+}
+
+// bf16 -> fp16, eight values per 16-byte access, four accesses in flight per
+// thread; see launch_convert_f16.
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v, bool& bad) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
+    w[i] = pack_f16x2_checked(lo, hi, bad);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__global__ void __launch_bounds__(256) convert_f16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                          int64_t n8, unsigned int* err) {
+  pdl_trigger();  // the second projection may be scheduled at once
+  bool bad = false;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n8; i += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = __ldcs(src + i + j * stride);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dst[i + j * stride] = bf16x8_to_f16x8(v[j], bad);
+  }
+  for (; i < n8; i += stride) dst[i] = bf16x8_to_f16x8(__ldcs(src + i), bad);
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) record_error(err, DEV_ERR_RANGE);
+  // complete only after the kernel before (the first projection): the kernel
+  // after this one waits for this one alone
+  pdl_wait();
 }
 
 }  // namespace
@@ -495,7 +561,10 @@ cudaError_t launch_ar(const TcGemmPlan& pl, int num_sms, cudaStream_t s) {
 cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
   *why = nullptr;
   if (g.E > MAX_E) { *why = "grouped GEMM supports at most 256 experts"; return cudaErrorInvalidValue; }
+  const bool gate = g.epi == EPI_GATE_F32 || g.epi == EPI_GATE_SCATTER_BF16;
+  if (g.f16 && g.split) { *why = "grouped GEMM: fp16 and split hidden modes exclude each other"; return cudaErrorInvalidValue; }
   const bool a_split = g.split && g.A2 != nullptr;
+  const bool ops_f16 = g.f16 && gate;  // A and B of the second projection in fp16
   const bool swiglu = g.epi == EPI_SWIGLU_BF16;
   // A rows per stage: every expert group has at most max_group_rows rows
   pl->ar = g.max_group_rows <= 32 ? 32 : g.max_group_rows <= 64 ? 64 : 128;
@@ -511,12 +580,17 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
     return cudaErrorInvalidValue;
   }
   const bool maps_ok =
-      (a_split ? make_map_planes_bf16(&pl->a, g.A, static_cast<uint64_t>(plane_stride), a_rows, K, ar)
-               : make_map_bf16(&pl->a, g.A, a_rows, K, ar)) &&
-      make_map(&pl->a2, a_split ? g.A2 : g.A, a_rows, K) &&
-      // B: two 128-row boxes (W1 and W3) for SwiGLU, else one 256-row box
-      make_map_bf16(&pl->b0, g.B0, b_rows, K, swiglu ? 128 : 256) &&
-      make_map(&pl->b1, swiglu ? g.B1 : g.B0, b_rows, K);
+      ops_f16
+          ? (make_map_16(&pl->a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.A, a_rows, K, ar) &&
+             make_map_16(&pl->a2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.A, a_rows, K, 128) &&
+             make_map_16(&pl->b0, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.B0, b_rows, K, 256) &&
+             make_map_16(&pl->b1, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.B0, b_rows, K, 128))
+          : ((a_split ? make_map_planes_bf16(&pl->a, g.A, static_cast<uint64_t>(plane_stride), a_rows, K, ar)
+                      : make_map_bf16(&pl->a, g.A, a_rows, K, ar)) &&
+             make_map(&pl->a2, a_split ? g.A2 : g.A, a_rows, K) &&
+             // B: two 128-row boxes (W1 and W3) for SwiGLU, else one 256-row box
+             make_map_bf16(&pl->b0, g.B0, b_rows, K, swiglu ? 128 : 256) &&
+             make_map(&pl->b1, swiglu ? g.B1 : g.B0, b_rows, K));
   if (!maps_ok) {
     *why = "cuTensorMapEncodeTiled failed (alignment or driver entry point)";
     return cudaErrorInvalidValue;
@@ -541,7 +615,7 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
   p.err = g.err;
   p.limit_ns = kWaitLimitNs;
   pl->epi = g.epi;
-  pl->split = g.split;
+  pl->hid = g.f16 ? HID_F16 : g.split ? HID_BF16X2 : HID_BF16;
   if (g.epi < EPI_RELU_BF16 || g.epi > EPI_GATE_SCATTER_BF16) {
     *why = "unknown epilogue";
     return cudaErrorInvalidValue;
@@ -550,20 +624,19 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
 }
 
 cudaError_t launch_gemm_tc(const TcGemmPlan& pl, int num_sms, cudaStream_t s) {
-  if (pl.split) {
-    switch (pl.epi) {
-      case EPI_RELU_BF16: return launch_ar<EPI_RELU_BF16, true>(pl, num_sms, s);
-      case EPI_SWIGLU_BF16: return launch_ar<EPI_SWIGLU_BF16, true>(pl, num_sms, s);
-      case EPI_GATE_F32: return launch_ar<EPI_GATE_F32, true>(pl, num_sms, s);
-      default: return launch_ar<EPI_GATE_SCATTER_BF16, true>(pl, num_sms, s);
-    }
-  }
-  switch (pl.epi) {
-    case EPI_RELU_BF16: return launch_ar<EPI_RELU_BF16, false>(pl, num_sms, s);
-    case EPI_SWIGLU_BF16: return launch_ar<EPI_SWIGLU_BF16, false>(pl, num_sms, s);
-    case EPI_GATE_F32: return launch_ar<EPI_GATE_F32, false>(pl, num_sms, s);
-    default: return launch_ar<EPI_GATE_SCATTER_BF16, false>(pl, num_sms, s);
-  }
+  if (pl.hid == HID_F16) return launch_epi<HID_F16>(pl, num_sms, s);
+  if (pl.hid == HID_BF16X2) return launch_epi<HID_BF16X2>(pl, num_sms, s);
+  return launch_epi<HID_BF16>(pl, num_sms, s);
+}
+
+cudaError_t launch_convert_f16(const void* src, void* dst, int64_t n, unsigned int* err, int num_sms,
+                               cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t n8 = n / 8;
+  int64_t blocks = (n8 + 255) / 256;
+  if (blocks > 4LL * num_sms) blocks = 4LL * num_sms;
+  return launch_pdl(convert_f16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
+                    static_cast<const uint4*>(src), static_cast<uint4*>(dst), n8, err);
 }
 
 }  // namespace moe

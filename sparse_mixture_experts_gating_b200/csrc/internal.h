@@ -111,6 +111,8 @@ struct GemmArgs {
   const void* A;   // [a_rows][K]  (the hi plane when split)
   const void* A2;  // [a_rows][K]  lo plane of a split A operand, else NULL
   int split;       // first projection: write hi/lo planes; second: read them
+  int f16;         // first projection: write the hidden activation as fp16; second:
+                   // A (that activation) and B (an fp16 image of W2) are fp16
   const void* B0;  // [E][N][K]  (W1, or W2)
   const void* B1;  // [E][N][K]  (W3 for SwiGLU, else unused)
   void* out;       // Hp [S][N] | Yp [S][N] fp32 | y [T][N]
@@ -141,14 +143,26 @@ struct TcParams {
   uint64_t limit_ns;
 };
 
+// How the hidden activation between the projections is held.
+enum HiddenKind { HID_BF16 = 0, HID_BF16X2 = 1, HID_F16 = 2 };
+
 // Everything a tensor-core GEMM launch needs, prepared on the host up front.
 struct TcGemmPlan {
   CUtensorMap a, a2, b0, b1;
   TcParams p;
   int epi;
-  int split;
-  int ar;  // A rows per pipeline stage: 32, 64 or 128
+  int hid;  // HiddenKind
+  int ar;   // A rows per pipeline stage: 32, 64 or 128
 };
+
+// fp16 image of n bf16 values (n a multiple of 8, both pointers 16-byte
+// aligned), for the second projection's B operand in the fp16 hidden mode.
+// Launched right after the first projection: it starts while that kernel
+// runs, and waits for it to complete before it ends itself, so the kernel
+// launched after it sees both complete.  A value beyond the fp16 range
+// records DEV_ERR_RANGE in *err.
+cudaError_t launch_convert_f16(const void* src, void* dst, int64_t n, unsigned int* err, int num_sms,
+                               cudaStream_t s);
 
 cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* plan, const char** why);
 cudaError_t launch_gemm_tc(const TcGemmPlan& plan, int num_sms, cudaStream_t s);

@@ -92,6 +92,20 @@ int ksplit_of(const moe_layer& L, int64_t s_max) {
 // Yp rows a batch of s rows needs (0: none, the bf16 rows go straight into y).
 int64_t yp_rows_of(const moe_layer& L, int64_t s) { return need_yp_of(L) ? ksplit_of(L, s) * s : 0; }
 
+// The automatic hidden mode holds the hidden activation in fp16 when the
+// batch averages at least this many rows per expert group: there the second
+// projection is bound by the tensor cores, and one fp16 plane halves its MMAs
+// against the hi + lo bf16 pair, which more than pays for the fp16 image of
+// W2 (made while the first projection runs).  Smaller batches are bound by
+// the weight stream, where the pair costs no time.
+constexpr int64_t kAutoF16RowsPerGroup = 1024;
+
+bool f16_hidden_of(const moe_layer& L, int64_t s_max) {
+  if (L.dtype != MOE_BF16) return false;
+  if (L.hidden == MOE_HIDDEN_F16) return true;
+  return L.hidden == MOE_HIDDEN_AUTO && s_max >= kAutoF16RowsPerGroup * (L.E + L.n_shared);
+}
+
 int64_t capacity_of(const moe_layer& L, int64_t T) {
   if (!(L.capacity_factor > 0.0)) return -1;
   const double c = ceil(L.capacity_factor * static_cast<double>(T) * static_cast<double>(L.k) /
@@ -104,10 +118,11 @@ struct Layout {
   int64_t T, s_max, capacity;
   int nblk;
   bool need_yp;
-  bool split;
+  bool split;  // hidden activation as a hi + lo bf16 pair
+  bool f16;    // hidden activation (and the second projection's operands) in fp16
   int ksplit;
   size_t idx, gate, dest, row_token, row_gate, part_hist, part_cnt1, part_psum, part_lse2, blockoff, counts,
-      offsets, mprefix, scal, wsplit, rpart, spart, Xp, Hp, Hp_lo, Yp, total;
+      offsets, mprefix, scal, wsplit, rpart, spart, Xp, Hp, Hp_lo, Yp, W2h, total;
 };
 
 Layout make_layout(const moe_layer& L, int64_t T) {
@@ -120,7 +135,8 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   w.s_max += static_cast<int64_t>(L.n_shared) * T;  // every token's rows of the shared experts
   w.nblk = static_cast<int>((T + kRouterTokens - 1) / kRouterTokens);
   const size_t elt = L.dtype == MOE_BF16 ? 2 : 4;
-  w.split = L.dtype == MOE_BF16 && L.hidden == MOE_HIDDEN_BF16X2;
+  w.f16 = f16_hidden_of(L, w.s_max);
+  w.split = L.dtype == MOE_BF16 && !w.f16 && (L.hidden == MOE_HIDDEN_BF16X2 || L.hidden == MOE_HIDDEN_AUTO);
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
   w.idx = take(sizeof(int32_t) * Tk);
@@ -145,7 +161,12 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   w.spart = take(route_small_partials_bytes(L.E));  // batches of <= 32 tokens (constant: sizes stay monotone)
   w.Xp = take(elt * static_cast<size_t>(w.s_max) * L.d);
   w.Hp = take(elt * static_cast<size_t>(w.s_max) * L.d_ff);
-  w.Hp_lo = take(w.split ? elt * static_cast<size_t>(w.s_max) * L.d_ff : 0);
+  // The automatic mode keeps the lo plane's room once it switches to fp16
+  // (the largest pair any smaller batch uses), so sizes never shrink as T grows.
+  int64_t lo_rows = w.split ? w.s_max : 0;
+  if (L.dtype == MOE_BF16 && L.hidden == MOE_HIDDEN_AUTO && w.f16)
+    lo_rows = kAutoF16RowsPerGroup * (L.E + L.n_shared) - 1;
+  w.Hp_lo = take(elt * static_cast<size_t>(lo_rows) * L.d_ff);
   w.ksplit = ksplit_of(L, w.s_max);
   w.need_yp = need_yp_of(L);
   // Yp holds ksplit partials of s_max rows; reserve the most any smaller batch
@@ -160,6 +181,8 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   for (int64_t s = groups + 127; s < w.s_max && s <= groups + int64_t{kSplitMaxTiles} * 128; s += 128)
     yp_rows = std::max<int64_t>(yp_rows, yp_rows_of(L, s));
   w.Yp = take(yp_rows > 0 ? sizeof(float) * static_cast<size_t>(yp_rows) * L.d : 0);
+  // fp16 image of W2 (every expert, shared ones included) for the fp16 mode
+  w.W2h = take(w.f16 ? sizeof(uint16_t) * static_cast<size_t>(L.E + L.n_shared) * L.d * L.d_ff : 0);
   w.total = o;
   return w;
 }
@@ -294,7 +317,7 @@ int moe_create(int num_experts, int k, int d, int d_ff, int act, int gate_mode, 
   if (dtype == MOE_BF16 && (d % 8 != 0 || d_ff % 8 != 0))
     return fail(MOE_ERR_UNSUPPORTED, "moe_create: bf16 layers need d and d_ff to be multiples of 8");
   moe_layer* L =
-      new moe_layer{num_experts, k, d, d_ff, act, gate_mode, dtype, capacity_factor, MOE_HIDDEN_BF16X2, 0};
+      new moe_layer{num_experts, k, d, d_ff, act, gate_mode, dtype, capacity_factor, MOE_HIDDEN_AUTO, 0};
   *out = L;
   t_err.clear();
   return MOE_OK;
@@ -302,7 +325,7 @@ int moe_create(int num_experts, int k, int d, int d_ff, int act, int gate_mode, 
 
 int moe_set_hidden_precision(moe_handle h, int mode) {
   if (h == nullptr) return fail(MOE_ERR_INVALID_ARG, "moe_set_hidden_precision: handle is NULL");
-  if (mode != MOE_HIDDEN_BF16X2 && mode != MOE_HIDDEN_BF16)
+  if (mode != MOE_HIDDEN_BF16X2 && mode != MOE_HIDDEN_BF16 && mode != MOE_HIDDEN_F16 && mode != MOE_HIDDEN_AUTO)
     return fail(MOE_ERR_INVALID_ARG, "moe_set_hidden_precision: unknown mode");
   h->hidden = mode;
   return MOE_OK;
@@ -447,6 +470,7 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   g1.B1 = W3;
   g1.out = ws + w.Hp;
   g1.split = w.split;
+  g1.f16 = w.f16;
   g1.out2 = w.split ? static_cast<void*>(ws + w.Hp_lo) : nullptr;
   g1.offsets = r.offsets;
   g1.mprefix = r.mprefix;
@@ -461,7 +485,7 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   g2.A = ws + w.Hp;
   g2.A2 = w.split ? static_cast<const void*>(ws + w.Hp_lo) : nullptr;
   g2.out2 = nullptr;
-  g2.B0 = W2;
+  g2.B0 = w.f16 ? static_cast<const void*>(ws + w.W2h) : W2;
   g2.B1 = nullptr;
   g2.out = w.need_yp ? static_cast<void*>(ws + w.Yp) : y;
   g2.out_f32 = (w.need_yp || dbg == nullptr) ? nullptr : dbg->y_f32;
@@ -522,6 +546,11 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   record(dbg, MOE_STAGE_GEMM1, 0, s);
   ce = tc ? launch_gemm_tc(plan1, di->num_sms, s) : launch_gemm_simt(g1, w.s_max, s);
   if ((rc = check(ce, "gemm1")) != MOE_OK) return rc;
+  if (w.f16) {  // the fp16 image of W2, made while the first projection runs
+    ce = launch_convert_f16(W2, ws + w.W2h, static_cast<int64_t>(L.E + L.n_shared) * L.d * L.d_ff, di->err,
+                            di->num_sms, s);
+    if ((rc = check(ce, "fp16 image of W2")) != MOE_OK) return rc;
+  }
   record(dbg, MOE_STAGE_GEMM1, 1, s);
   record(dbg, MOE_STAGE_GEMM2, 0, s);
   ce = tc ? launch_gemm_tc(plan2, di->num_sms, s) : launch_gemm_simt(g2, w.s_max, s);
@@ -556,6 +585,8 @@ int moe_status(void* stream) {
   e = cudaMemcpyFromSymbol(&word, g_moe_error_word, sizeof(word));
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_status: ") + cudaGetErrorString(e));
   if (word == DEV_ERR_TIMEOUT) return fail(MOE_ERR_TIMEOUT, "moe_status: a device-side bounded wait ran out");
+  if (word == DEV_ERR_RANGE)
+    return fail(MOE_ERR_RANGE, "moe_status: a value of the fp16 hidden mode was beyond the fp16 range");
   if (word != 0) return fail(MOE_ERR_CUDA, "moe_status: unknown device error word");
   return MOE_OK;
 }

@@ -16,7 +16,7 @@ from ._lib import MoEDebug, check, lib
 ACT = {"relu": 0, "swiglu": 1}
 GATE = {"switch": 0, "renorm": 1}
 DTYPE = {torch.float32: 0, torch.bfloat16: 1}
-HIDDEN = {"bf16x2": 0, "bf16": 1}
+HIDDEN = {"bf16x2": 0, "bf16": 1, "f16": 2, "auto": 3}
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -33,14 +33,16 @@ class MoELayer:
 
     act: "relu" | "swiglu" (or 0 / 1); gate_mode: "switch" | "renorm" (or 0 / 1);
     capacity_factor <= 0: dropless; dtype: torch.float32 or torch.bfloat16;
-    hidden (bf16 layers): "bf16x2" keeps the hidden activation as a hi + lo
-    pair of bf16 planes (default), "bf16" as one bf16 plane.
+    hidden (bf16 layers): "auto" (default) holds the hidden activation in fp16
+    for batches of at least 1024 rows per expert and as a hi + lo pair of
+    bf16 planes otherwise; "f16" and "bf16x2" force one of those; "bf16" is
+    one bf16 plane (outside the parity bar; see include/moe.h).
     n_shared: shared experts every token visits; W1, W3, W2 then hold
     num_experts + n_shared experts, the shared ones last.
     """
 
     def __init__(self, num_experts: int, k: int, d: int, d_ff: int, act="swiglu", gate_mode="renorm",
-                 capacity_factor: float = 0.0, dtype=torch.bfloat16, hidden="bf16x2", n_shared: int = 0):
+                 capacity_factor: float = 0.0, dtype=torch.bfloat16, hidden="auto", n_shared: int = 0):
         self.E, self.k, self.d, self.d_ff = num_experts, k, d, d_ff
         self.act = ACT[act] if isinstance(act, str) else int(act)
         self.gate_mode = GATE[gate_mode] if isinstance(gate_mode, str) else int(gate_mode)

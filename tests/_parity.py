@@ -46,7 +46,7 @@ class HostExperts:
         return self.cache[e]
 
 
-def layer_for(w: Workload, hidden: str = "bf16x2") -> MoELayer:
+def layer_for(w: Workload, hidden: str = "auto") -> MoELayer:
     return MoELayer(w.E, w.k, w.d, w.d_ff, act=w.act, gate_mode=w.gate,
                     capacity_factor=w.capacity_factor, dtype=torch_dtype(w.dtype), hidden=hidden,
                     n_shared=w.n_shared)

@@ -131,23 +131,47 @@ def test_shared_experts_and_balance_losses_validate_arguments(L):
 
 
 def test_workspace_sizing_is_defined_for_every_batch_size(L):
-    """Host-only sizing (no GPU): every T from 0 up, several layer shapes, both
-    hidden precisions; sizes never shrink as T grows."""
+    """Host-only sizing (no GPU): every T from 0 up, several layer shapes, every
+    hidden precision (the automatic one across its switch to fp16); sizes
+    never shrink as T grows."""
     shapes = [(8, 2, 4096, 14336, 1, 1, 0.0, 1), (64, 1, 768, 3072, 0, 0, 1.25, 1),
               (128, 4, 2048, 768, 1, 1, 2.0, 1), (4, 2, 32, 64, 0, 1, 0.0, 0), (256, 8, 64, 64, 0, 0, 0.5, 1),
               (3, 2, 1032, 1160, 1, 1, 0.0, 1)]
     for i, args in enumerate(shapes):
         rc, h = _create(L, *args)
         assert rc == 0
-        assert L.moe_set_shared_experts(h, min(i % 3, 256 - args[0])) == 0
-        for mode in (0, 1):
+        ns = min(i % 3, 256 - args[0])
+        assert L.moe_set_shared_experts(h, ns) == 0
+        E, k = args[0], args[1]
+        t_auto = 1024 * (E + ns) // (k + ns)  # near where the automatic mode turns to fp16
+        extra = sorted({t for t in range(t_auto - 3, t_auto + 4) if t > 0} | {511, 512, 513, 2047, 2048, 2049,
+                                                                               8192, 16384})
+        for mode in (0, 1, 2, 3):
             assert L.moe_set_hidden_precision(h, mode) == 0
             prev = 0
-            for T in list(range(0, 300)) + [511, 512, 513, 2047, 2048, 2049, 8192, 16384]:
+            for T in list(range(0, 300)) + extra:
                 n = L.moe_workspace_bytes(h, T)
                 assert n >= prev and n % 256 == 0, (args, mode, T, n)
                 prev = n
         L.moe_destroy(h)
+
+
+def test_automatic_hidden_mode_adds_the_fp16_weight_image_at_1024_rows_per_expert(L):
+    """The automatic mode holds the hidden activation in fp16 (and reserves the
+    fp16 image of W2) from 1024 rows per expert group on: for 8 experts, top-2,
+    dropless, that is T = 4096."""
+    rc, h = _create(L, 8, 2, 4096, 14336, 1, 1, 0.0, 1)
+    assert rc == 0
+    image = 8 * 4096 * 14336 * 2
+    assert L.moe_set_hidden_precision(h, 3) == 0
+    below, at = L.moe_workspace_bytes(h, 4095), L.moe_workspace_bytes(h, 4096)
+    assert at - below >= image
+    assert L.moe_set_hidden_precision(h, 2) == 0  # forced fp16: the image at any T
+    assert L.moe_workspace_bytes(h, 1) >= image
+    assert L.moe_set_hidden_precision(h, 0) == 0  # forced pair: no image
+    assert L.moe_workspace_bytes(h, 4096) < at
+    assert L.moe_set_hidden_precision(h, 4) == _lib.MOE_ERR_INVALID_ARG
+    L.moe_destroy(h)
 
 
 def test_static_scratch_limit_stated_in_the_header_holds(L):

@@ -1,5 +1,6 @@
 """Host-side logic of bench.py (no GPU): rank reduction over gloo with two
 ranks, per-rank seeding, algorithmic work and roofline arithmetic."""
+import hashlib
 import os
 import socket
 
@@ -100,7 +101,16 @@ def test_backward_work_closed_forms():
     assert b == 8 * per * 2 + 8 * per * 4 + 2 * 8192 * 4096 * 2 + 8192 * 4096 * 4 + 8 * 4096 * 4
 
 
-def test_profiled_traffic_matches_the_current_sources():
-    """The committed GEMM2 capture of the Switch workload names the sources it
-    was taken from; the bench reports its DRAM bytes while they are unchanged."""
-    assert bench.profiled_traffic("gemm2", "switch_k1") == 330019584.0
+def test_profiled_traffic_is_reported_only_while_its_sources_are_unchanged(tmp_path, monkeypatch):
+    """A committed ncu summary names the sources it was taken from and their
+    sha256; the bench reports its DRAM bytes only while they still match."""
+    src = tmp_path / "kernel.cu"
+    src.write_text("// kernel source\n")
+    (tmp_path / "profiles").mkdir()
+    prof = tmp_path / "profiles" / "gemm2_someload.txt"
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()
+    prof.write_text(f"dram_bytes_per_launch: 1234\nsource_files: kernel.cu\nsource_sha256: {sha}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("gemm2", "someload") == 1234.0
+    src.write_text("// kernel source, changed\n")
+    assert bench.profiled_traffic("gemm2", "someload") is None

@@ -38,6 +38,14 @@ CASES = [
     ("shared_swiglu_drops_bf16", 150, 64, 4, 2, 64, S, RN, 1.0, BF, None, 1),
     ("small_batch_bf16", 20, 64, 8, 2, 64, S, RN, 0.0, BF, "normal", 0),  # one launch routes T <= 32
     ("e32_k4_zipf_relu", 200, 32, 32, 4, 40, R, RN, 1.0, BF, "zipf", 0),
+    # at size: T >= 1024 sums dW_r over four or more token chunks; d >= 256 and
+    # d_ff >= 512 give several n-tiles and k-blocks in every product
+    ("chunks_relu_drops", 1100, 256, 8, 1, 512, R, SW, 1.25, BF, "normal", 0),
+    ("chunks_swiglu_k2", 1536, 384, 8, 2, 640, S, RN, 0.0, BF, None, 0),
+    # skewed loads: the largest expert group (and so the padded K of the
+    # weight-gradient products) is well above 512 rows
+    ("skewed_kpad_swiglu", 2048, 256, 4, 1, 512, S, SW, 0.0, BF, "zipf", 0),
+    ("chunks_shared_fp32", 1030, 64, 4, 2, 96, S, RN, 1.0, F32, "normal", 1),
 ]
 
 
@@ -102,6 +110,28 @@ def test_backward_matches_oracle(case):
         _close("dW2s", np32(g["dW2"])[E:], o["dW2s"])
         if w.act == S:
             _close("dW3s", np32(g["dW3"])[E:], o["dW3s"])
+
+
+def test_skewed_case_pads_k_beyond_512():
+    w = _w([c for c in CASES if c[0] == "skewed_kpad_swiglu"][0])
+    inp, _, dbg, dy, g = _run(w)
+    counts = np.bincount(dbg["topk_idx"].cpu().numpy().ravel(), minlength=w.E)
+    assert counts.max() > 512
+
+
+def test_full_size_switch_backward_matches_oracle():
+    """The Switch workload at full size (T 8192, d 768, 64 experts, ReLU 3072,
+    capacity 1.25) with dyadic router inputs: every gradient tensor, every
+    element, against the backward oracle."""
+    from sparse_mixture_experts_gating_b200.workloads import WORKLOADS
+    w = WORKLOADS["switch_k1"].with_(dyadic=True)
+    inp, _, dbg, dy, g = _run(w)
+    o = _oracle(w, inp, dy)
+    np.testing.assert_array_equal(dbg["topk_idx"].cpu().numpy(), o["idx"])
+    np.testing.assert_array_equal(dbg["drop_mask"].cpu().numpy().astype(bool), ~o["kept"])
+    assert not o["kept"].all()
+    for key in ("dx", "dW_r", "db_r", "dW1", "dW2"):
+        _close(key, np32(g[key]), o[key])
 
 
 def test_backward_is_deterministic():

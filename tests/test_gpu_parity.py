@@ -110,6 +110,42 @@ def test_small_layers_single_bf16_hidden(case):
     assert_y_close(w, g, o["y"], single_plane_hidden=True)
 
 
+F16 = [c for c in SMALL if c[9] == BF]
+
+
+@pytest.mark.parametrize("case", F16, ids=[c[0] for c in F16])
+def test_small_layers_f16_hidden(case):
+    """Hidden activation in fp16 and the second projection on fp16 operands
+    (an fp16 image of W2): routing bit-exact, y within the full bar."""
+    w = _small(case)
+    inp = make_inputs(w, device="cuda")
+    g = run_gpu(w, inp, layer=layer_for(w, hidden="f16"))
+    host = host_inputs(inp)
+    o = run_oracle(w, host)
+    assert_routing_equal(g, o)
+    assert_gates_and_losses(g, o)
+    assert_y_close(w, g, o["y"])
+
+
+def test_f16_hidden_out_of_range_is_reported_and_context_survives():
+    """A hidden value beyond the fp16 range (x scaled up 2^9) makes the fp16
+    mode report MOE_ERR_RANGE; the status clears and the next call is fine."""
+    w = _small(SMALL[1])
+    inp = make_inputs(w, device="cuda")
+    layer = layer_for(w, hidden="f16")
+    clear_status()
+    big = (inp["x"].float() * 512).to(torch.bfloat16)
+    layer(big, inp["W_r"], inp["b_r"], inp["W1"], inp["W3"], inp["W2"])
+    with pytest.raises(MoEError) as ei:
+        status()
+    assert ei.value.code == 5
+    clear_status()
+    g = run_gpu(w, inp, layer=layer)
+    o = run_oracle(w, host_inputs(inp))
+    assert_routing_equal(g, o)
+    assert_y_close(w, g, o["y"])
+
+
 def test_ties_go_to_the_lower_expert_index():
     w = Workload("ties", T=257, d=64, E=8, k=3, d_ff=128, act=S, gate=RN, capacity_factor=0.0, dtype=BF,
                  dyadic=True, seed=77)
@@ -281,6 +317,23 @@ def test_full_size_bench_configuration(name):
     rows = rows[same[rows]]
     assert len(rows) > 0
     o = run_oracle(w, host, rows=rows)
+    assert_y_close(w, g, o["y"], rows=rows)
+
+
+@pytest.mark.parametrize("name", ["switch_k1", "mixtral_prefill", "fine_grained", "mixtral_decode_t64"])
+@pytest.mark.parametrize("hidden", ["f16", "bf16x2"])
+def test_full_size_each_hidden_mode(name, hidden):
+    """Both in-bar hidden modes forced at full size (identical logits): the
+    automatic default picks one of them per batch, so each is checked on every
+    shape class."""
+    w = WORKLOADS[name]
+    inp = make_inputs(w, device="cuda")
+    host = host_inputs(inp)
+    o_route = run_oracle(w, host, rows=[])
+    g = run_gpu(w, inp, logits_in=torch.from_numpy(o_route["logits"]).cuda(), layer=layer_for(w, hidden=hidden))
+    assert_routing_equal(g, o_route)
+    rows = sample_rows(w, o_route["kept"], n=24, seed=4)
+    o = run_oracle(w, host, rows=rows, logits=o_route["logits"])
     assert_y_close(w, g, o["y"], rows=rows)
 
 
