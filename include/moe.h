@@ -204,6 +204,46 @@ MOE_API int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r
                 void* workspace, size_t workspace_bytes, const moe_debug* dbg, void* stream);
 
 /*
+ * 4-bit expert weights for serving ("Mixture of Experts (MoE)", inferensys.com,
+ * inference-optimization glossary, model quantization: post-training 4-bit
+ * quantization of a trained MoE's weights; "Mixture of experts", rayaq.ca,
+ * "Total versus active parameters": small-batch decoding is bound by reading
+ * the experts' weights, which quantization eases).  The pages fix no scheme;
+ * this library's format:
+ *   - each weight row [K] (K a multiple of 128) is cut into groups of 128
+ *     consecutive elements; group g has a bf16 scale s_g with at most 5
+ *     significant bits, and element k is w_k = (u_k - 8) * s_{k / 128} with a
+ *     4-bit code u_k in [0, 15] (so w_k is exact in bf16);
+ *   - codes: uint32 [rows][K / 8]; word m holds elements 8m .. 8m+7 of its
+ *     row, element 8m + 2j in bits 4j .. 4j+3 and element 8m + 2j + 1 in
+ *     bits 4j+16 .. 4j+19 (j = 0 .. 3);  scales: bf16 [rows][K / 128].
+ * Rows are the rows of the nn.Linear weights: W1 / W3 [E (+ n_shared)][d_ff]
+ * rows of K = d, W2 [E (+ n_shared)][d] rows of K = d_ff.
+ *
+ * moe_quantize_int4: codes and scales of a bf16 weight W [rows][K] (device
+ * pointers; W and codes 16-byte aligned, scales 2-byte aligned), by
+ * s = max|w| / 7 over the group in fp32, rounded up to 5 significant bits,
+ * and u = round-half-even(w / s) + 8 in fp32 (u = 8 when s = 0).  Asynchronous
+ * on `stream`.  K must be a multiple of 128, else MOE_ERR_UNSUPPORTED.
+ *
+ * moe_forward_w4: moe_forward of a bf16 layer (d and d_ff multiples of 128)
+ * whose expert weights are given in that format; the result is the layer
+ * with the dequantized weights.  The expert products run on the tensor
+ * cores with the weights dequantized on the fly (HBM carries the codes and
+ * scales only); the hidden activation is held as a hi + lo bf16 pair.  The
+ * workspace is moe_workspace_bytes_w4(h, T) bytes (256-byte aligned).
+ * Arguments, results and errors as moe_forward; W3_codes / W3_scales are
+ * NULL for ReLU layers.  moe_backward does not serve layers run this way.
+ */
+MOE_API int moe_quantize_int4(const void* W, int64_t rows, int64_t K, uint32_t* codes, void* scales, void* stream);
+MOE_API size_t moe_workspace_bytes_w4(moe_handle h, int64_t T);
+MOE_API int moe_forward_w4(moe_handle h, int64_t T, const void* x, const float* W_r, const float* b_r,
+                           const uint32_t* W1_codes, const void* W1_scales, const uint32_t* W3_codes,
+                           const void* W3_scales, const uint32_t* W2_codes, const void* W2_scales, void* y,
+                           int32_t* expert_counts, int32_t* dropped, float* aux_loss, float* z_loss, void* workspace,
+                           size_t workspace_bytes, const moe_debug* dbg, void* stream);
+
+/*
  * The alternative load-balancing statistics of the last moe_forward that used
  * `workspace` with T tokens (stream-ordered on `stream`), unscaled, written as
  * three fp32 values to the device pointer `out`:

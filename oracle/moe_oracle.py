@@ -298,3 +298,72 @@ def moe_forward(x, W_r, b_r, W1, W3, W2, *, k: int, gate_mode: int, act: int,
     res.update(balance_losses(p, idx, E))
     res.update(slots)
     return res
+
+
+# ----------------------------------------------------------------------------- 4-bit weights
+# "Mixture of Experts (MoE)" (inferensys.com, inference-optimization glossary),
+# model quantization paragraph: post-training quantization of a trained MoE's
+# weights to 4-bit integers; "Mixture of experts" (rayaq.ca), "Total versus
+# active parameters": small-batch decoding is bound by reading expert weights,
+# which quantization eases.  The pages fix no scheme; the reading here:
+#   * symmetric per-group quantization along the input dimension K of each
+#     weight row, groups of INT4_GROUP consecutive elements;
+#   * scale s = max|w| / 7 over the group, computed in float32 and rounded UP
+#     to 5 significant bits (so that every code times s is exact in bfloat16);
+#   * code q = round-half-even(w / s) in float32 (|w / s| <= 7, so q in [-7, 7];
+#     the stored range is [-8, 7]); s = 0 (an all-zero group) gives q = 0;
+#   * the dequantized weight is q * s, exactly.
+# Storage: codes u = q + 8 in 4 bits; each 32-bit word holds 8 consecutive
+# elements k0..k7 of a row, element k_{2j} in bits 4j..4j+3 and element
+# k_{2j+1} in bits 4j+16..4j+19 (j = 0..3); scales are bfloat16.
+INT4_GROUP = 128
+
+
+def _round_up_5_significant_bits(s32: np.ndarray) -> np.ndarray:
+    """Smallest float32 with at most 5 significant bits that is >= s (s >= 0)."""
+    u = np.asarray(s32, np.float32).view(np.uint32).astype(np.uint64)
+    low = u & ((1 << 19) - 1)
+    u = np.where(low != 0, (u | ((1 << 19) - 1)) + 1, u)
+    return u.astype(np.uint32).view(np.float32)
+
+
+def quantize_int4(W) -> tuple:
+    """Codes q [rows][K] (int8, -8..7) and float32 scales [rows][K / INT4_GROUP]
+    of a weight matrix W [rows][K] (bfloat16 values given as floats), by the
+    rule above; K must be a multiple of INT4_GROUP."""
+    W = np.asarray(W, np.float32)
+    rows, K = W.shape
+    assert K % INT4_GROUP == 0
+    g = W.reshape(rows, K // INT4_GROUP, INT4_GROUP)
+    amax = np.abs(g).max(axis=2).astype(np.float32)
+    s = _round_up_5_significant_bits((amax / np.float32(7.0)).astype(np.float32))
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = np.where(s[:, :, None] > 0, np.rint((g / s[:, :, None]).astype(np.float32)), 0.0)
+    q = np.clip(r, -8, 7).astype(np.int8).reshape(rows, K)
+    return q, s
+
+
+def pack_int4(q: np.ndarray) -> np.ndarray:
+    """Words [rows][K / 8] (uint32) of codes q [rows][K] in the storage layout above."""
+    q = np.asarray(q, np.int64)
+    rows, K = q.shape
+    u = (q + 8).reshape(rows, K // 8, 8).astype(np.uint64)
+    w = np.zeros((rows, K // 8), np.uint64)
+    for j in range(4):
+        w |= u[:, :, 2 * j] << (4 * j)
+        w |= u[:, :, 2 * j + 1] << (4 * j + 16)
+    return w.astype(np.uint32)
+
+
+def dequantize_int4(words, scales) -> np.ndarray:
+    """Weights [rows][K] (float64) from packed words [rows][K / 8] and scales
+    [rows][K / INT4_GROUP]: element k = (u_k - 8) * s_{k // INT4_GROUP}."""
+    w = np.asarray(words, np.uint64)
+    rows, K8 = w.shape
+    u = np.empty((rows, K8, 8), np.int64)
+    for j in range(4):
+        u[:, :, 2 * j] = (w >> (4 * j)) & 0xF
+        u[:, :, 2 * j + 1] = (w >> (4 * j + 16)) & 0xF
+    q = (u - 8).reshape(rows, K8 * 8).astype(np.float64)
+    s = np.repeat(np.asarray(scales, np.float64), INT4_GROUP, axis=1)
+    return q * s

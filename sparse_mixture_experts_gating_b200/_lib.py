@@ -32,6 +32,11 @@ SIGNATURES = {
     "moe_backward": (c_int, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                              c_void_p, c_float, c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                              c_void_p, c_void_p, c_size_t, c_void_p, c_size_t, c_void_p]),
+    "moe_quantize_int4": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
+    "moe_workspace_bytes_w4": (c_size_t, [c_void_p, c_int64]),
+    "moe_forward_w4": (c_int, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                               c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                               c_void_p, c_size_t, c_void_p, c_void_p]),
     "moe_status": (c_int, [c_void_p]),
     "moe_clear_status": (c_int, []),
     "moe_last_error": (c_char_p, []),

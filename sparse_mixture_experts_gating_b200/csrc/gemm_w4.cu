@@ -1,0 +1,479 @@
+// Grouped GEMM with 4-bit expert weights on the tcgen05 tensor cores, for
+// the weight-streaming batches of decoding ("Mixture of experts", rayaq.ca,
+// section "Total versus active parameters": at small batch sizes decoding is
+// limited by reading weights; "Mixture of Experts (MoE)", inferensys.com,
+// inference-optimization glossary: 4-bit post-training quantization of the
+// experts' weights).
+//
+// Weights arrive as 4-bit codes with one bf16 scale per 128 consecutive
+// elements of a row (format in include/moe.h, moe_quantize_int4).  The
+// product runs transposed: D[f][n] = sum_k W[f][k] X[n][k], with the weight
+// rows f as the M = 128 operand and the (few) activation rows n of the
+// expert as the N operand (16, 32 or 64 columns).  Dequantized weights never
+// touch shared or global memory: dequantizing warps turn each k-block of
+// codes into bf16 rows held in tensor memory (tcgen05.st), which the MMA
+// reads as its A operand, while the activation tile comes from shared memory
+// through TMA.  HBM then carries the codes and scales only.
+//
+// Warp roles (448 threads, one CTA per SM):
+//   warp 0        TMA producer: per stage the code tile(s) [128 rows x 32 B]
+//                 and the activation tile [NB rows x 64] (hi and lo planes
+//                 of the hidden activation for the second projection)
+//   warp 1        TMEM allocator; lane 0 issues the MMAs (M 128, N NB, K 16)
+//   warps 2..9    dequantize: warp w owns TMEM lanes 32 (w % 4) .. + 31 (one
+//                 weight row per lane) and half (w - 2) / 4 of each k-block
+//   warps 10..13  epilogue: activation (first projection) or gate (second)
+//                 and the stores, one weight row (output column) per lane
+// The dequantized values are exact: (code - 8) * scale with a scale of at
+// most 5 significant bits fits bf16 exactly, and both steps are exact bf16x2
+// operations.  Every wait is bounded as in the bf16 grouped GEMM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int WBM = 128;                 // weight rows per tile (TMEM lanes)
+constexpr int WBK = 64;                  // K per k-block
+constexpr int Q_TILE = WBM * WBK / 2;    // bytes of codes per weight tile and k-block (4 KB)
+constexpr int A_STAGES = 4;              // TMEM A ring
+constexpr int MAX_SMEM_STAGES = 8;
+constexpr int W4_THREADS = 448;
+constexpr int MAX_G = 256;
+
+template <int MODE>
+struct W4Geo {
+  static constexpr int NQ = MODE == W4_SWIGLU ? 2 : 1;      // weight matrices per tile (W1 and W3)
+  static constexpr int PLANES = MODE == W4_GATE ? 2 : 1;    // activation planes (hidden hi + lo)
+};
+
+template <int MODE, int NB>
+struct W4Stage {
+  static constexpr int BYTES = W4Geo<MODE>::NQ * Q_TILE + W4Geo<MODE>::PLANES * NB * 128;
+  static constexpr int N = (160 * 1024 / BYTES) < MAX_SMEM_STAGES ? (160 * 1024 / BYTES) : MAX_SMEM_STAGES;
+};
+
+struct W4Ctl {
+  uint64_t full[MAX_SMEM_STAGES];
+  uint64_t empty[MAX_SMEM_STAGES];
+  uint64_t afull[A_STAGES];
+  uint64_t aempty[A_STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_slot;
+  volatile int abort;
+  int nprefix[MAX_G + 1];  // prefix over groups of their n-tiles
+  int offsets[MAX_G + 1];
+};
+
+template <int MODE, int NB>
+constexpr size_t w4_smem_bytes() {
+  return W4Stage<MODE, NB>::N * W4Stage<MODE, NB>::BYTES + sizeof(W4Ctl) + 1024;
+}
+
+template <int MODE, int NB>
+constexpr uint32_t w4_tmem_cols() {
+  constexpr int used = A_STAGES * W4Geo<MODE>::NQ * 32 + 2 * W4Geo<MODE>::NQ * NB;
+  return used <= 32 ? 32 : used <= 64 ? 64 : used <= 128 ? 128 : used <= 256 ? 256 : 512;
+}
+
+// unit -> (group, m-tile over weight rows, n-tile over activation rows, K range)
+struct W4Item {
+  int e, mt, nt, ks, kb0, kb1;
+};
+
+__device__ __forceinline__ bool w4_item(const W4Ctl* c, const W4Params& p, int u, W4Item& w) {
+  const int units = c->nprefix[p.G] * p.m_tiles * p.ksplit;
+  if (u >= units) return false;
+  const int tile = u / p.ksplit;
+  w.ks = u - tile * p.ksplit;
+  int lo = 0, hi = p.G;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (c->nprefix[mid] * p.m_tiles <= tile) lo = mid; else hi = mid;
+  }
+  w.e = lo;
+  const int local = tile - c->nprefix[lo] * p.m_tiles;
+  const int nts = c->nprefix[lo + 1] - c->nprefix[lo];
+  w.mt = local / nts;
+  w.nt = local - w.mt * nts;
+  w.kb0 = w.ks * p.kb_per;
+  w.kb1 = min(p.num_kb, w.kb0 + p.kb_per);
+  return true;
+}
+
+__device__ __forceinline__ bool w4_wait(W4Ctl* c, uint64_t* bar, uint32_t parity, const W4Params& p) {
+  return mbar_wait_or_abort(bar, parity, &c->abort, p.err, p.limit_ns);
+}
+
+// A operand read from TMEM: D[tmem] (+)= A[tmem] * B[smem]^T, issued by one thread.
+__device__ __forceinline__ void umma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Eight codes of one 32-bit word (element 2j in bits 4j.., element 2j+1 in
+// bits 4j+16.., codes offset by 8) -> four bf16 pairs (code - 8) * s, exact.
+__device__ __forceinline__ void dequant_word(uint32_t w, __nv_bfloat162 s2, uint32_t* out) {
+  const __nv_bfloat162 bias = __floats2bfloat162_rn(136.f, 136.f);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t t = ((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u;  // bf16 pair 128 + code
+    __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&t);
+    v = __hmul2(__hsub2(v, bias), s2);
+    out[j] = *reinterpret_cast<const uint32_t*>(&v);
+  }
+}
+
+template <int MODE, int NB>
+__global__ void __launch_bounds__(W4_THREADS, 1)
+    w4_gemm_kernel(const __grid_constant__ CUtensorMap tmQ0, const __grid_constant__ CUtensorMap tmQ1,
+                   const __grid_constant__ CUtensorMap tmX, const W4Params p) {
+  using Geo = W4Geo<MODE>;
+  using St = W4Stage<MODE, NB>;
+  constexpr int NQ = Geo::NQ, PLANES = Geo::PLANES;
+  constexpr int STAGES = St::N, STAGE_BYTES = St::BYTES;
+  constexpr int X_OFF = NQ * Q_TILE;
+  constexpr uint32_t TMEM_COLS = w4_tmem_cols<MODE, NB>();
+  constexpr uint32_t ACC0 = A_STAGES * NQ * 32;  // first accumulator column
+  constexpr uint32_t IDESC = idesc_bf16_f32(WBM, NB);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* stages = smem_raw + pad;
+  W4Ctl* ctl = reinterpret_cast<W4Ctl*>(stages + STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
+    for (int a = 0; a < A_STAGES; ++a) { mbar_init(&ctl->afull[a], 8); mbar_init(&ctl->aempty[a], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&ctl->tfull[a], 1); mbar_init(&ctl->tempty[a], 128); }
+    mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tmQ0);
+    if (NQ == 2) tma_prefetch_desc(&tmQ1);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) tmem_alloc(&ctl->tmem_slot, TMEM_COLS);
+  pdl_wait();  // group offsets and the activation rows come from the kernels before
+  pdl_trigger();
+  if (threadIdx.x == 0) {
+    ctl->nprefix[0] = 0;
+    for (int g = 0; g < p.G; ++g) {
+      const int o0 = p.offsets[g], o1 = p.offsets[g + 1];
+      ctl->offsets[g] = o0;
+      ctl->nprefix[g + 1] = ctl->nprefix[g] + (o1 - o0 + NB - 1) / NB;
+    }
+    ctl->offsets[p.G] = p.offsets[p.G];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_phase = 0;
+      bool ok = true;
+      W4Item w;
+      for (int u = blockIdx.x; ok && w4_item(ctl, p, u, w); u += gridDim.x) {
+        const int qrow = w.e * p.N + w.mt * WBM;
+        const int xrow = ctl->offsets[w.e] + w.nt * NB;
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          if (!w4_wait(ctl, &ctl->empty[stage], phase ^ 1u, p)) { ok = false; break; }
+          uint8_t* st = stages + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
+          tma_load_2d(st, &tmQ0, &ctl->full[stage], kb * (WBK / 2), qrow);
+          if (NQ == 2) tma_load_2d(st + Q_TILE, &tmQ1, &ctl->full[stage], kb * (WBK / 2), qrow);
+          if (PLANES == 2) tma_load_3d(st + X_OFF, &tmX, &ctl->full[stage], kb * WBK, xrow, 0);
+          else tma_load_2d(st + X_OFF, &tmX, &ctl->full[stage], kb * WBK, xrow);
+          issued |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      for (int s = 0; s < STAGES; ++s)
+        if ((issued >> s) & 1u) mbar_wait(&ctl->full[s], (issued_phase >> s) & 1u, p.limit_ns);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0, astage = 0, acc = 0;
+      uint32_t phase = 0, aphase = 0, acc_phase = 0;
+      bool ok = true;
+      W4Item w;
+      for (int u = blockIdx.x; ok && w4_item(ctl, p, u, w); u += gridDim.x) {
+        if (!w4_wait(ctl, &ctl->tempty[acc], acc_phase ^ 1u, p)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + ACC0 + static_cast<uint32_t>(acc * NQ * NB);
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          if (!w4_wait(ctl, &ctl->full[stage], phase, p) || !w4_wait(ctl, &ctl->afull[astage], aphase, p)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sx = smem_u32(stages + stage * STAGE_BYTES + X_OFF);
+          const uint32_t a0 = tmem_base + static_cast<uint32_t>(astage * NQ * 32);
+#pragma unroll
+          for (int kk = 0; kk < WBK / 16; ++kk) {
+            const uint32_t acc_in = (kb != w.kb0 || kk != 0) ? 1u : 0u;
+            const uint64_t bd = sdesc_k_sw128(sx + kk * 32);
+            umma_tmem_a(d0, a0 + kk * 8, bd, IDESC, acc_in);
+            if (NQ == 2) umma_tmem_a(d0 + NB, a0 + 32 + kk * 8, bd, IDESC, acc_in);
+            if (PLANES == 2) umma_tmem_a(d0, a0 + kk * 8, sdesc_k_sw128(sx + NB * 128 + kk * 32), IDESC, 1u);
+          }
+          umma_commit(&ctl->empty[stage]);
+          umma_commit(&ctl->aempty[astage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++astage == A_STAGES) { astage = 0; aphase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&ctl->tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      umma_commit(&ctl->drain);
+      mbar_wait(&ctl->drain, 0, p.limit_ns);
+    }
+  } else if (warp < 10) {
+    // ------------------------------------------------------------ dequantize
+    const int q = warp & 3, half = (warp - 2) >> 2;
+    const int r = q * 32 + lane;  // weight row within the tile
+    const int groups = p.K / W4_GROUP;
+    int stage = 0, astage = 0;
+    uint32_t phase = 0, aphase = 0;
+    bool ok = true;
+    W4Item w;
+    for (int u = blockIdx.x; ok && w4_item(ctl, p, u, w); u += gridDim.x) {
+      const int64_t row = static_cast<int64_t>(w.e) * p.N + w.mt * WBM + r;
+      const bool vrow = w.mt * WBM + r < p.N;
+      for (int kb = w.kb0; kb < w.kb1; ++kb) {
+        // this half's 32 elements lie in one scale group
+        const int grp = (kb * WBK + half * 32) / W4_GROUP;
+        const __nv_bfloat16 s0 = vrow ? p.S0[row * groups + grp] : __float2bfloat16(0.f);
+        const __nv_bfloat16 s1 = (NQ == 2 && vrow) ? p.S1[row * groups + grp] : __float2bfloat16(0.f);
+        const bool got = __all_sync(0xffffffffu, w4_wait(ctl, &ctl->full[stage], phase, p) &&
+                                                     w4_wait(ctl, &ctl->aempty[astage], aphase ^ 1u, p));
+        if (!got) { ok = false; break; }
+        tc_fence_after();
+        const uint8_t* st = stages + stage * STAGE_BYTES;
+        const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                              static_cast<uint32_t>(astage * NQ * 32 + half * 16);
+#pragma unroll
+        for (int m = 0; m < NQ; ++m) {
+          const uint4 words = *reinterpret_cast<const uint4*>(st + m * Q_TILE + r * 32 + half * 16);
+          const __nv_bfloat162 s2 = __bfloat162bfloat162(m == 0 ? s0 : s1);
+          uint32_t v[16];
+          dequant_word(words.x, s2, v);
+          dequant_word(words.y, s2, v + 4);
+          dequant_word(words.z, s2, v + 8);
+          dequant_word(words.w, s2, v + 12);
+          tmem_st16(tcol + m * 32, v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->afull[astage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (++astage == A_STAGES) { astage = 0; aphase ^= 1u; }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    W4Item w;
+    for (int u = blockIdx.x; w4_item(ctl, p, u, w); u += gridDim.x) {
+      const bool got = __all_sync(0xffffffffu, w4_wait(ctl, &ctl->tfull[acc], acc_phase, p));
+      if (!got) break;
+      tc_fence_after();
+      const int f = w.mt * WBM + r;  // weight row = output column of this lane
+      const bool vcol = f < p.N;
+      const int g0 = ctl->offsets[w.e], grows = ctl->offsets[w.e + 1] - g0;
+      const int n0 = w.nt * NB;
+      const int nvalid = min(NB, grows - n0);
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ACC0 +
+                          static_cast<uint32_t>(acc * NQ * NB);
+#pragma unroll 1
+      for (int c = 0; c < NB; c += 16) {
+        uint32_t ra[16], rb[16];
+        tmem_ld16(tb + c, ra);
+        if (NQ == 2) tmem_ld16(tb + NB + c, rb);
+        tmem_ld_wait();
+        if (vcol) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int n = c + i;
+            if (n >= nvalid) break;
+            const int64_t row = g0 + n0 + n;  // expert-sorted row
+            const float a = __uint_as_float(ra[i]);
+            if (MODE == W4_GATE) {
+              float* out = static_cast<float*>(p.out) + static_cast<int64_t>(w.ks) * p.split_stride;
+              out[row * p.N + f] = a * p.row_gate[row];
+            } else {
+              const float h = MODE == W4_SWIGLU ? __fdividef(a, 1.f + __expf(-a)) * __uint_as_float(rb[i])
+                                                : fmaxf(a, 0.f);
+              const __nv_bfloat16 hi = __float2bfloat16_rn(h);
+              const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
+              static_cast<__nv_bfloat16*>(p.out)[row * p.N + f] = hi;
+              static_cast<__nv_bfloat16*>(p.out_lo)[row * p.N + f] = lo;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&ctl->tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Quantizer: one warp per (row, group of 128 elements).  Lane l holds
+// elements 4l .. 4l+3 of the group; scale = max|w| / 7 in fp32, rounded up to
+// 5 significant bits; code = round-half-even(w / scale) + 8 (0 if scale = 0).
+__device__ __forceinline__ uint32_t round_up_5_bits(float s) {
+  uint32_t u = __float_as_uint(s);
+  if (u & 0x7FFFFu) u = (u | 0x7FFFFu) + 1u;
+  return u;
+}
+
+__global__ void __launch_bounds__(256) quantize_int4_kernel(const __nv_bfloat16* __restrict__ W, int64_t rows,
+                                                            int K, uint32_t* __restrict__ codes,
+                                                            __nv_bfloat16* __restrict__ scales) {
+  const int groups = K / W4_GROUP;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (gw >= rows * groups) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = gw / groups;
+  const int grp = static_cast<int>(gw - row * groups);
+  const __nv_bfloat16* src = W + row * K + grp * W4_GROUP + lane * 4;
+  const uint2 raw = *reinterpret_cast<const uint2*>(src);
+  float v[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u), __uint_as_float(raw.y << 16),
+                __uint_as_float(raw.y & 0xFFFF0000u)};
+  float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float s = __uint_as_float(round_up_5_bits(__fdiv_rn(amax, 7.f)));
+  uint32_t u[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float qf = s > 0.f ? rintf(__fdiv_rn(v[i], s)) : 0.f;
+    u[i] = static_cast<uint32_t>(static_cast<int>(fminf(fmaxf(qf, -8.f), 7.f)) + 8);
+  }
+  // word m holds elements 8m .. 8m+7: element 2j in nibble j, element 2j+1 in nibble j + 4
+  const uint32_t part = (lane & 1) == 0 ? (u[0] | (u[1] << 16) | (u[2] << 4) | (u[3] << 20))
+                                        : ((u[0] << 8) | (u[1] << 24) | (u[2] << 12) | (u[3] << 28));
+  const uint32_t word = part | __shfl_xor_sync(0xffffffffu, part, 1);
+  if ((lane & 1) == 0) codes[(row * K + grp * W4_GROUP) / 8 + lane / 2] = word;
+  if (lane == 0) scales[row * groups + grp] = __float2bfloat16_rn(s);
+}
+
+// Row-major uint8 [rows][bytes] -> map with box [128 rows][32 bytes], no swizzle.
+bool make_map_codes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t bytes) {
+  return make_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, rows, bytes, 1, 32, WBM, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+template <int MODE, int NB>
+cudaError_t launch_w4_t(const W4Plan& pl, int num_sms, cudaStream_t s) {
+  constexpr size_t bytes = w4_smem_bytes<MODE, NB>();
+  static_assert(bytes <= 227 * 1024, "4-bit grouped GEMM shared memory");
+  cudaError_t e =
+      set_smem_limit_once(reinterpret_cast<const void*>(&w4_gemm_kernel<MODE, NB>), static_cast<int>(bytes));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(w4_gemm_kernel<MODE, NB>, dim3(num_sms), dim3(W4_THREADS), bytes, s, pl.q0, pl.q1, pl.x,
+                    pl.p);
+}
+
+template <int MODE>
+cudaError_t launch_w4_nb(const W4Plan& pl, int num_sms, cudaStream_t s) {
+  if (pl.nb == 16) return launch_w4_t<MODE, 16>(pl, num_sms, s);
+  if (pl.nb == 32) return launch_w4_t<MODE, 32>(pl, num_sms, s);
+  return launch_w4_t<MODE, 64>(pl, num_sms, s);
+}
+
+}  // namespace
+
+int w4_rows_per_tile(int64_t max_group_rows) { return max_group_rows <= 16 ? 16 : max_group_rows <= 32 ? 32 : 64; }
+
+cudaError_t plan_w4_gemm(const W4Args& g, W4Plan* pl, const char** why) {
+  *why = nullptr;
+  if (g.G > MAX_G) { *why = "4-bit grouped GEMM supports at most 256 expert groups"; return cudaErrorInvalidValue; }
+  if (g.K % W4_GROUP != 0) { *why = "4-bit weights need the input dimension to be a multiple of 128"; return cudaErrorInvalidValue; }
+  pl->nb = w4_rows_per_tile(g.max_group_rows);
+  const uint64_t qrows = static_cast<uint64_t>(g.G) * g.N;
+  const uint64_t qbytes = static_cast<uint64_t>(g.K) / 2;
+  bool ok = make_map_codes(&pl->q0, g.Q0, qrows, qbytes) &&
+            make_map_codes(&pl->q1, g.mode == W4_SWIGLU ? g.Q1 : g.Q0, qrows, qbytes);
+  if (g.mode == W4_GATE) {
+    const intptr_t stride = static_cast<const uint8_t*>(g.X_lo) - static_cast<const uint8_t*>(g.X);
+    if (stride <= 0 || stride % 16 != 0) { *why = "4-bit grouped GEMM: lo plane must follow the hi plane"; return cudaErrorInvalidValue; }
+    ok = ok && make_map_planes_bf16(&pl->x, g.X, static_cast<uint64_t>(stride), static_cast<uint64_t>(g.x_rows),
+                                    static_cast<uint64_t>(g.K), static_cast<uint32_t>(pl->nb));
+  } else {
+    ok = ok && make_map_bf16(&pl->x, g.X, static_cast<uint64_t>(g.x_rows), static_cast<uint64_t>(g.K),
+                             static_cast<uint32_t>(pl->nb));
+  }
+  if (!ok) { *why = "cuTensorMapEncodeTiled failed for the 4-bit grouped GEMM"; return cudaErrorInvalidValue; }
+  W4Params& p = pl->p;
+  p.G = g.G;
+  p.N = g.N;
+  p.K = g.K;
+  p.m_tiles = (g.N + WBM - 1) / WBM;
+  p.num_kb = g.K / WBK;
+  p.ksplit = g.mode == W4_GATE ? (g.ksplit < 1 ? 1 : (g.ksplit > p.num_kb ? p.num_kb : g.ksplit)) : 1;
+  p.kb_per = (p.num_kb + p.ksplit - 1) / p.ksplit;
+  p.ksplit = (p.num_kb + p.kb_per - 1) / p.kb_per;  // no empty K range
+  p.split_stride = g.split_stride;
+  p.S0 = static_cast<const __nv_bfloat16*>(g.S0);
+  p.S1 = static_cast<const __nv_bfloat16*>(g.mode == W4_SWIGLU ? g.S1 : g.S0);
+  p.out = g.out;
+  p.out_lo = g.out_lo;
+  p.offsets = g.offsets;
+  p.row_gate = g.row_gate;
+  p.err = g.err;
+  p.limit_ns = kWaitLimitNs;
+  pl->mode = g.mode;
+  return cudaSuccess;
+}
+
+cudaError_t launch_w4_gemm(const W4Plan& pl, int num_sms, cudaStream_t s) {
+  if (pl.mode == W4_SWIGLU) return launch_w4_nb<W4_SWIGLU>(pl, num_sms, s);
+  if (pl.mode == W4_RELU) return launch_w4_nb<W4_RELU>(pl, num_sms, s);
+  return launch_w4_nb<W4_GATE>(pl, num_sms, s);
+}
+
+cudaError_t launch_quantize_int4(const void* W, int64_t rows, int K, void* codes, void* scales, cudaStream_t s) {
+  const int64_t warps = rows * (K / W4_GROUP);
+  if (warps <= 0) return cudaSuccess;
+  const int64_t blocks = (warps + 7) / 8;
+  if (blocks > 2147483647LL) return cudaErrorInvalidValue;
+  quantize_int4_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(W), rows, K, static_cast<uint32_t*>(codes),
+      static_cast<__nv_bfloat16*>(scales));
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace moe

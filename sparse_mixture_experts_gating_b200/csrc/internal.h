@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -166,6 +167,59 @@ cudaError_t launch_convert_f16(const void* src, void* dst, int64_t n, unsigned i
 
 cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* plan, const char** why);
 cudaError_t launch_gemm_tc(const TcGemmPlan& plan, int num_sms, cudaStream_t s);
+
+// Any row-major 2D tensor [rows][cols] of elements of elem_bytes bytes -> map
+// with box [box_rows][box_cols] and the given swizzle.
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType type, const void* base, uint64_t rows, uint64_t cols,
+                 uint32_t elem_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle);
+
+// ---------------------------------------------------------------- 4-bit weights
+// Codes: uint32 [rows][K / 8], element 2j of each 8 in bits 4j.., element
+// 2j + 1 in bits 4j + 16.., code = q + 8; scales: bf16 [rows][K / W4_GROUP].
+constexpr int W4_GROUP = 128;
+enum W4Mode { W4_RELU = 0, W4_SWIGLU = 1, W4_GATE = 2 };
+
+struct W4Params {
+  int G, N, K, m_tiles, num_kb, ksplit, kb_per;
+  int64_t split_stride;              // W4_GATE: elements between K-range partials of the output
+  const __nv_bfloat16* S0;           // scales of W1 (or W2)
+  const __nv_bfloat16* S1;           // scales of W3 (SwiGLU)
+  void* out;                         // first projection: hidden hi plane [S][N] bf16; second: Yp fp32
+  void* out_lo;                      // first projection: hidden lo plane
+  const int32_t* offsets;            // [G + 1] rows of each expert group in the sorted buffers
+  const float* row_gate;             // [S] gate of each sorted row (second projection)
+  unsigned int* err;
+  uint64_t limit_ns;
+};
+
+struct W4Args {
+  int mode, G, N, K;
+  int64_t x_rows, max_group_rows;
+  const void* Q0;  // codes of W1 (or W2) [G * N][K / 8]
+  const void* Q1;  // codes of W3 (SwiGLU)
+  const void* S0;
+  const void* S1;
+  const void* X;     // activation rows [x_rows][K] bf16 (sorted x, or the hidden hi plane)
+  const void* X_lo;  // second projection: the hidden lo plane
+  int ksplit;
+  int64_t split_stride;
+  void* out;
+  void* out_lo;
+  const int32_t* offsets;
+  const float* row_gate;
+  unsigned int* err;
+};
+
+struct W4Plan {
+  CUtensorMap q0, q1, x;
+  W4Params p;
+  int mode, nb;
+};
+
+int w4_rows_per_tile(int64_t max_group_rows);
+cudaError_t plan_w4_gemm(const W4Args& g, W4Plan* plan, const char** why);
+cudaError_t launch_w4_gemm(const W4Plan& plan, int num_sms, cudaStream_t s);
+cudaError_t launch_quantize_int4(const void* W, int64_t rows, int K, void* codes, void* scales, cudaStream_t s);
 
 // Raise a kernel's dynamic shared memory limit, once per (kernel, device, size).
 cudaError_t set_smem_limit_once(const void* kernel, int bytes);

@@ -83,14 +83,35 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // The second projection splits its K range for at most this many tiles.
 constexpr int kSplitMaxTiles = 4 * kSplitTargetCtas;
 
-bool need_yp_of(const moe_layer& L) { return !(L.dtype == MOE_BF16 && L.k == 1 && L.n_shared == 0); }
+// (4-bit weights always go through the fp32 rows and the combine.)
+bool need_yp_of(const moe_layer& L, bool w4) {
+  return w4 || !(L.dtype == MOE_BF16 && L.k == 1 && L.n_shared == 0);
+}
 
-int ksplit_of(const moe_layer& L, int64_t s_max) {
-  return (L.dtype == MOE_BF16 && need_yp_of(L)) ? gemm2_ksplit(s_max, L.E + L.n_shared, L.d, L.d_ff) : 1;
+// K ranges of the 4-bit second projection: its tiles are (group, n-tile of
+// at most NB rows, 128 output columns); cut K until about two waves of
+// (tile, range) units cover the SMs.
+int w4_ksplit(int64_t s, int groups, int d, int d_ff) {
+  const int64_t nb = w4_rows_per_tile(s);
+  const int64_t g = std::min<int64_t>(groups, s);
+  const int64_t tiles = (g + (s - g) / nb) * ((d + 127) / 128);
+  const int64_t num_kb = d_ff / 64;
+  if (tiles <= 0 || tiles >= 2 * kSplitTargetCtas) return 1;
+  int64_t ks = (2 * kSplitTargetCtas + tiles - 1) / tiles;
+  ks = std::min<int64_t>(ks, std::max<int64_t>(num_kb / 4, 1));
+  const int64_t per = (num_kb + ks - 1) / ks;
+  return static_cast<int>((num_kb + per - 1) / per);
+}
+
+int ksplit_of(const moe_layer& L, int64_t s_max, bool w4) {
+  if (w4) return w4_ksplit(s_max, L.E + L.n_shared, L.d, L.d_ff);
+  return (L.dtype == MOE_BF16 && need_yp_of(L, false)) ? gemm2_ksplit(s_max, L.E + L.n_shared, L.d, L.d_ff) : 1;
 }
 
 // Yp rows a batch of s rows needs (0: none, the bf16 rows go straight into y).
-int64_t yp_rows_of(const moe_layer& L, int64_t s) { return need_yp_of(L) ? ksplit_of(L, s) * s : 0; }
+int64_t yp_rows_of(const moe_layer& L, int64_t s, bool w4) {
+  return need_yp_of(L, w4) ? ksplit_of(L, s, w4) * s : 0;
+}
 
 // The automatic hidden mode holds the hidden activation in fp16 when the
 // batch averages at least this many rows per expert group: there the second
@@ -125,7 +146,9 @@ struct Layout {
       offsets, mprefix, scal, wsplit, rpart, spart, Xp, Hp, Hp_lo, Yp, W2h, total;
 };
 
-Layout make_layout(const moe_layer& L, int64_t T) {
+// w4: the layout of moe_forward_w4 (4-bit weights: hidden as a hi + lo pair,
+// fp32 rows for the combine, no fp16 image of W2).
+Layout make_layout(const moe_layer& L, int64_t T, bool w4 = false) {
   Layout w;
   w.T = T;
   w.capacity = capacity_of(L, T);
@@ -135,8 +158,9 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   w.s_max += static_cast<int64_t>(L.n_shared) * T;  // every token's rows of the shared experts
   w.nblk = static_cast<int>((T + kRouterTokens - 1) / kRouterTokens);
   const size_t elt = L.dtype == MOE_BF16 ? 2 : 4;
-  w.f16 = f16_hidden_of(L, w.s_max);
-  w.split = L.dtype == MOE_BF16 && !w.f16 && (L.hidden == MOE_HIDDEN_BF16X2 || L.hidden == MOE_HIDDEN_AUTO);
+  w.f16 = !w4 && f16_hidden_of(L, w.s_max);
+  w.split = L.dtype == MOE_BF16 &&
+            (w4 || (!w.f16 && (L.hidden == MOE_HIDDEN_BF16X2 || L.hidden == MOE_HIDDEN_AUTO)));
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
   w.idx = take(sizeof(int32_t) * Tk);
@@ -164,22 +188,26 @@ Layout make_layout(const moe_layer& L, int64_t T) {
   // The automatic mode keeps the lo plane's room once it switches to fp16
   // (the largest pair any smaller batch uses), so sizes never shrink as T grows.
   int64_t lo_rows = w.split ? w.s_max : 0;
-  if (L.dtype == MOE_BF16 && L.hidden == MOE_HIDDEN_AUTO && w.f16)
+  if (!w4 && L.dtype == MOE_BF16 && L.hidden == MOE_HIDDEN_AUTO && w.f16)
     lo_rows = kAutoF16RowsPerGroup * (L.E + L.n_shared) - 1;
   w.Hp_lo = take(elt * static_cast<size_t>(lo_rows) * L.d_ff);
-  w.ksplit = ksplit_of(L, w.s_max);
-  w.need_yp = need_yp_of(L);
+  w.ksplit = ksplit_of(L, w.s_max, w4);
+  w.need_yp = need_yp_of(L, w4);
   // Yp holds ksplit partials of s_max rows; reserve the most any smaller batch
   // needs as well, so a workspace sized for some T serves every smaller batch.
   // ksplit(s) depends on s through the m-tile bound min(G, s) + floor((s - min(G, s)) / 128)
   // (G groups), which changes at every s up to G and then every 128 rows, and
   // ksplit(s) = 1 once the bound reaches kSplitMaxTiles; the product ksplit(s) * s
   // peaks at the last s before each change.
-  int64_t yp_rows = yp_rows_of(L, w.s_max);
+  int64_t yp_rows = yp_rows_of(L, w.s_max, w4);
   const int64_t groups = L.E + L.n_shared;
-  for (int64_t s = 1; s < w.s_max && s <= groups; ++s) yp_rows = std::max<int64_t>(yp_rows, yp_rows_of(L, s));
+  for (int64_t s = 1; s < w.s_max && s <= groups; ++s) yp_rows = std::max<int64_t>(yp_rows, yp_rows_of(L, s, w4));
   for (int64_t s = groups + 127; s < w.s_max && s <= groups + int64_t{kSplitMaxTiles} * 128; s += 128)
-    yp_rows = std::max<int64_t>(yp_rows, yp_rows_of(L, s));
+    yp_rows = std::max<int64_t>(yp_rows, yp_rows_of(L, s, w4));
+  if (w4) {  // the 4-bit split also changes at every 16 / 32 / 64 rows (n-tile sizes) up to two waves of tiles
+    for (int64_t s = groups + 1; s < w.s_max && s <= groups + int64_t{2 * kSplitTargetCtas} * 64; ++s)
+      yp_rows = std::max<int64_t>(yp_rows, yp_rows_of(L, s, w4));
+  }
   w.Yp = take(yp_rows > 0 ? sizeof(float) * static_cast<size_t>(yp_rows) * L.d : 0);
   // fp16 image of W2 (every expert, shared ones included) for the fp16 mode
   w.W2h = take(w.f16 ? sizeof(uint16_t) * static_cast<size_t>(L.E + L.n_shared) * L.d * L.d_ff : 0);
@@ -373,45 +401,72 @@ size_t moe_workspace_bytes(moe_handle h, int64_t T) {
   return make_layout(*h, T).total;
 }
 
-int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const float* b_r, const void* W1,
-                const void* W3, const void* W2, void* y, int32_t* expert_counts, int32_t* dropped, float* aux_loss,
-                float* z_loss, void* workspace, size_t workspace_bytes, const moe_debug* dbg, void* stream) {
-  if (h == nullptr) return fail(MOE_ERR_INVALID_ARG, "moe_forward: handle is NULL");
+}  // extern "C"
+
+namespace {
+
+// The expert weights of one forward call: bf16 / fp32 tensors, or 4-bit codes
+// with their scales (moe_forward_w4).
+struct ExpertWeights {
+  bool w4;
+  const void *W1, *W3, *W2;   // bf16 / fp32
+  const void *Q1, *Q3, *Q2;   // 4-bit codes
+  const void *S1, *S3, *S2;   // their scales
+};
+
+int forward_impl(moe_handle h, int64_t T, const void* x, const float* W_r, const float* b_r, const ExpertWeights& ew,
+                 void* y, int32_t* expert_counts, int32_t* dropped, float* aux_loss, float* z_loss, void* workspace,
+                 size_t workspace_bytes, const moe_debug* dbg, void* stream, const char* fn) {
+  const std::string F = std::string(fn) + ": ";
+  if (h == nullptr) return fail(MOE_ERR_INVALID_ARG, F + "handle is NULL");
   const moe_layer& L = *h;
-  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "moe_forward: T < 0");
-  if (T * L.k > 2147483647LL / 2) return fail(MOE_ERR_UNSUPPORTED, "moe_forward: T * k too large");
-  if (T * static_cast<int64_t>(L.d) >= 4294967296LL) return fail(MOE_ERR_UNSUPPORTED, "moe_forward: T * d too large");
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, F + "T < 0");
+  if (T * L.k > 2147483647LL / 2) return fail(MOE_ERR_UNSUPPORTED, F + "T * k too large");
+  if (T * static_cast<int64_t>(L.d) >= 4294967296LL) return fail(MOE_ERR_UNSUPPORTED, F + "T * d too large");
   if (expert_counts == nullptr || dropped == nullptr || aux_loss == nullptr || z_loss == nullptr)
-    return fail(MOE_ERR_INVALID_ARG, "moe_forward: a statistics output pointer is NULL");
+    return fail(MOE_ERR_INVALID_ARG, F + "a statistics output pointer is NULL");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (T == 0) {
     if (cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * L.E, s) != cudaSuccess ||
         cudaMemsetAsync(dropped, 0, sizeof(int32_t), s) != cudaSuccess ||
         cudaMemsetAsync(aux_loss, 0, sizeof(float), s) != cudaSuccess ||
         cudaMemsetAsync(z_loss, 0, sizeof(float), s) != cudaSuccess)
-      return fail(MOE_ERR_CUDA, std::string("moe_forward: ") + cudaGetErrorString(cudaGetLastError()));
+      return fail(MOE_ERR_CUDA, std::string(F + "") + cudaGetErrorString(cudaGetLastError()));
     t_err.clear();
     return MOE_OK;
   }
+  const void* W1 = ew.w4 ? ew.Q1 : ew.W1;
+  const void* W3 = ew.w4 ? ew.Q3 : ew.W3;
+  const void* W2 = ew.w4 ? ew.Q2 : ew.W2;
   if (x == nullptr || W_r == nullptr || W1 == nullptr || W2 == nullptr || y == nullptr)
-    return fail(MOE_ERR_INVALID_ARG, "moe_forward: x, W_r, W1, W2 and y must be non-NULL");
+    return fail(MOE_ERR_INVALID_ARG, F + "x, W_r, W1, W2 and y must be non-NULL");
   if ((L.act == MOE_ACT_SWIGLU) != (W3 != nullptr))
-    return fail(MOE_ERR_INVALID_ARG, "moe_forward: W3 must be given for SwiGLU and NULL for ReLU");
-  const Layout w = make_layout(L, T);
+    return fail(MOE_ERR_INVALID_ARG, F + "W3 must be given for SwiGLU and NULL for ReLU");
+  if (ew.w4) {
+    if (ew.S1 == nullptr || ew.S2 == nullptr || (W3 != nullptr && ew.S3 == nullptr))
+      return fail(MOE_ERR_INVALID_ARG, F + "every 4-bit weight needs its scales");
+    if (L.dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, F + "4-bit weights serve bf16 layers only");
+    if (L.d % W4_GROUP != 0 || L.d_ff % W4_GROUP != 0)
+      return fail(MOE_ERR_UNSUPPORTED, F + "4-bit weights need d and d_ff to be multiples of 128");
+    const uintptr_t sal = reinterpret_cast<uintptr_t>(ew.S1) | reinterpret_cast<uintptr_t>(ew.S2) |
+                          reinterpret_cast<uintptr_t>(ew.S3);
+    if ((sal & 1) != 0) return fail(MOE_ERR_INVALID_ARG, F + "scales must be 2-byte aligned");
+  }
+  const Layout w = make_layout(L, T, ew.w4);
   if (workspace == nullptr || workspace_bytes < w.total)
-    return fail(MOE_ERR_INVALID_ARG, "moe_forward: workspace missing or smaller than moe_workspace_bytes()");
+    return fail(MOE_ERR_INVALID_ARG, F + "workspace missing or smaller than moe_workspace_bytes()");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0)
-    return fail(MOE_ERR_INVALID_ARG, "moe_forward: workspace must be 256-byte aligned");
+    return fail(MOE_ERR_INVALID_ARG, F + "workspace must be 256-byte aligned");
   const uintptr_t al = reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y) |
                        reinterpret_cast<uintptr_t>(W1) | reinterpret_cast<uintptr_t>(W2) |
                        reinterpret_cast<uintptr_t>(W3);
-  if ((al & 15) != 0) return fail(MOE_ERR_INVALID_ARG, "moe_forward: x, y and weights must be 16-byte aligned");
+  if ((al & 15) != 0) return fail(MOE_ERR_INVALID_ARG, F + "x, y and weights must be 16-byte aligned");
   if (L.dtype == MOE_F32 && (w.s_max + 7) / 8 > 65535)
-    return fail(MOE_ERR_UNSUPPORTED, "moe_forward: fp32 layers are limited to 524280 assignments");
+    return fail(MOE_ERR_UNSUPPORTED, F + "fp32 layers are limited to 524280 assignments");
 
   DeviceInfo* di = nullptr;
   cudaError_t ce = device_info(&di);
-  if (ce != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_forward: ") + cudaGetErrorString(ce));
+  if (ce != cudaSuccess) return fail(MOE_ERR_CUDA, std::string(F + "") + cudaGetErrorString(ce));
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   RoutingArgs r;
@@ -495,16 +550,53 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
 
   // Host-side preparation of both GEMM launches happens before the first launch.
   TcGemmPlan plan1, plan2;
-  if (L.dtype == MOE_BF16) {
+  W4Plan wplan1, wplan2;
+  if (ew.w4) {
+    W4Args a1;
+    memset(&a1, 0, sizeof(a1));
+    a1.mode = L.act == MOE_ACT_SWIGLU ? W4_SWIGLU : W4_RELU;
+    a1.G = L.E + L.n_shared;
+    a1.N = L.d_ff;
+    a1.K = L.d;
+    a1.x_rows = w.s_max;
+    a1.max_group_rows = T;
+    a1.Q0 = ew.Q1;
+    a1.Q1 = ew.Q3;
+    a1.S0 = ew.S1;
+    a1.S1 = ew.S3;
+    a1.X = ws + w.Xp;
+    a1.out = ws + w.Hp;
+    a1.out_lo = ws + w.Hp_lo;
+    a1.offsets = r.offsets;
+    a1.row_gate = r.row_gate;
+    a1.err = di->err;
+    W4Args a2 = a1;
+    a2.mode = W4_GATE;
+    a2.N = L.d;
+    a2.K = L.d_ff;
+    a2.Q0 = ew.Q2;
+    a2.Q1 = nullptr;
+    a2.S0 = ew.S2;
+    a2.S1 = nullptr;
+    a2.X = ws + w.Hp;
+    a2.X_lo = ws + w.Hp_lo;
+    a2.out = ws + w.Yp;
+    a2.out_lo = nullptr;
+    a2.ksplit = w.ksplit;
+    a2.split_stride = static_cast<int64_t>(w.s_max) * L.d;
+    const char* why = nullptr;
+    if (plan_w4_gemm(a1, &wplan1, &why) != cudaSuccess || plan_w4_gemm(a2, &wplan2, &why) != cudaSuccess)
+      return fail(MOE_ERR_UNSUPPORTED, F + (why ? why : "4-bit GEMM plan failed"));
+  } else if (L.dtype == MOE_BF16) {
     const char* why = nullptr;
     if (plan_gemm_tc(g1, &plan1, &why) != cudaSuccess || plan_gemm_tc(g2, &plan2, &why) != cudaSuccess)
-      return fail(MOE_ERR_UNSUPPORTED, std::string("moe_forward: ") + (why ? why : "GEMM plan failed"));
+      return fail(MOE_ERR_UNSUPPORTED, std::string(F + "") + (why ? why : "GEMM plan failed"));
   }
 
-  const bool tc = L.dtype == MOE_BF16;
+  const bool tc = L.dtype == MOE_BF16 && !ew.w4;
   auto check = [&](cudaError_t e, const char* what) -> int {
     if (e == cudaSuccess) return MOE_OK;
-    return fail(MOE_ERR_CUDA, std::string("moe_forward: ") + what + ": " + cudaGetErrorString(e));
+    return fail(MOE_ERR_CUDA, std::string(F + "") + what + ": " + cudaGetErrorString(e));
   };
   int rc;
   record(dbg, MOE_STAGE_ROUTER, 0, s);
@@ -521,7 +613,7 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
     if (tc && L.E <= kRouterTcMaxE && r.logits_in == nullptr) {
       const char* why = nullptr;
       ce = launch_router_tc(r, ws + w.wsplit, ws + w.rpart, di->num_sms, di->err, s, &why);
-      if (why != nullptr) return fail(MOE_ERR_UNSUPPORTED, std::string("moe_forward: ") + why);
+      if (why != nullptr) return fail(MOE_ERR_UNSUPPORTED, std::string(F + "") + why);
       if ((rc = check(ce, "router")) != MOE_OK) return rc;
     } else if ((rc = check(launch_router(r, s), "router")) != MOE_OK) {
       return rc;
@@ -544,7 +636,8 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   }
 
   record(dbg, MOE_STAGE_GEMM1, 0, s);
-  ce = tc ? launch_gemm_tc(plan1, di->num_sms, s) : launch_gemm_simt(g1, w.s_max, s);
+  ce = ew.w4 ? launch_w4_gemm(wplan1, di->num_sms, s)
+             : tc ? launch_gemm_tc(plan1, di->num_sms, s) : launch_gemm_simt(g1, w.s_max, s);
   if ((rc = check(ce, "gemm1")) != MOE_OK) return rc;
   if (w.f16) {  // the fp16 image of W2, made while the first projection runs
     ce = launch_convert_f16(W2, ws + w.W2h, static_cast<int64_t>(L.E + L.n_shared) * L.d * L.d_ff, di->err,
@@ -553,7 +646,8 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   }
   record(dbg, MOE_STAGE_GEMM1, 1, s);
   record(dbg, MOE_STAGE_GEMM2, 0, s);
-  ce = tc ? launch_gemm_tc(plan2, di->num_sms, s) : launch_gemm_simt(g2, w.s_max, s);
+  ce = ew.w4 ? launch_w4_gemm(wplan2, di->num_sms, s)
+             : tc ? launch_gemm_tc(plan2, di->num_sms, s) : launch_gemm_simt(g2, w.s_max, s);
   if ((rc = check(ce, "gemm2")) != MOE_OK) return rc;
   record(dbg, MOE_STAGE_GEMM2, 1, s);
   if (w.need_yp) {
@@ -568,12 +662,71 @@ int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const 
   if (dbg != nullptr) {
     const size_t tk = static_cast<size_t>(T) * L.k;
     if (dbg->topk_idx && cudaMemcpyAsync(dbg->topk_idx, r.topk_idx, 4 * tk, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-      return fail(MOE_ERR_CUDA, "moe_forward: debug copy failed");
+      return fail(MOE_ERR_CUDA, F + "debug copy failed");
     if (dbg->topk_gate && cudaMemcpyAsync(dbg->topk_gate, r.topk_gate, 4 * tk, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-      return fail(MOE_ERR_CUDA, "moe_forward: debug copy failed");
+      return fail(MOE_ERR_CUDA, F + "debug copy failed");
     if (dbg->dest_row && cudaMemcpyAsync(dbg->dest_row, r.dest_row, 4 * tk, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-      return fail(MOE_ERR_CUDA, "moe_forward: debug copy failed");
+      return fail(MOE_ERR_CUDA, F + "debug copy failed");
   }
+  t_err.clear();
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r, const float* b_r, const void* W1,
+                const void* W3, const void* W2, void* y, int32_t* expert_counts, int32_t* dropped, float* aux_loss,
+                float* z_loss, void* workspace, size_t workspace_bytes, const moe_debug* dbg, void* stream) {
+  ExpertWeights ew;
+  memset(&ew, 0, sizeof(ew));
+  ew.W1 = W1;
+  ew.W3 = W3;
+  ew.W2 = W2;
+  return forward_impl(h, T, x, W_r, b_r, ew, y, expert_counts, dropped, aux_loss, z_loss, workspace,
+                      workspace_bytes, dbg, stream, "moe_forward");
+}
+
+size_t moe_workspace_bytes_w4(moe_handle h, int64_t T) {
+  if (h == nullptr || T < 0) return 0;
+  return make_layout(*h, T, true).total;
+}
+
+int moe_forward_w4(moe_handle h, int64_t T, const void* x, const float* W_r, const float* b_r,
+                   const uint32_t* W1_codes, const void* W1_scales, const uint32_t* W3_codes, const void* W3_scales,
+                   const uint32_t* W2_codes, const void* W2_scales, void* y, int32_t* expert_counts,
+                   int32_t* dropped, float* aux_loss, float* z_loss, void* workspace, size_t workspace_bytes,
+                   const moe_debug* dbg, void* stream) {
+  ExpertWeights ew;
+  memset(&ew, 0, sizeof(ew));
+  ew.w4 = true;
+  ew.Q1 = W1_codes;
+  ew.Q3 = W3_codes;
+  ew.Q2 = W2_codes;
+  ew.S1 = W1_scales;
+  ew.S3 = W3_scales;
+  ew.S2 = W2_scales;
+  return forward_impl(h, T, x, W_r, b_r, ew, y, expert_counts, dropped, aux_loss, z_loss, workspace,
+                      workspace_bytes, dbg, stream, "moe_forward_w4");
+}
+
+int moe_quantize_int4(const void* W, int64_t rows, int64_t K, uint32_t* codes, void* scales, void* stream) {
+  if (rows < 0 || K < 0) return fail(MOE_ERR_INVALID_ARG, "moe_quantize_int4: rows < 0 or K < 0");
+  if (K % W4_GROUP != 0) return fail(MOE_ERR_UNSUPPORTED, "moe_quantize_int4: K must be a multiple of 128");
+  if (K > 2147483647LL) return fail(MOE_ERR_UNSUPPORTED, "moe_quantize_int4: K too large");
+  if (rows == 0 || K == 0) {
+    t_err.clear();
+    return MOE_OK;
+  }
+  if (W == nullptr || codes == nullptr || scales == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "moe_quantize_int4: NULL pointer");
+  if (((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(codes)) & 15) != 0 ||
+      (reinterpret_cast<uintptr_t>(scales) & 1) != 0)
+    return fail(MOE_ERR_INVALID_ARG, "moe_quantize_int4: W and codes must be 16-byte aligned, scales 2-byte");
+  const cudaError_t e = launch_quantize_int4(W, rows, static_cast<int>(K), codes, scales,
+                                             static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_quantize_int4: ") + cudaGetErrorString(e));
   t_err.clear();
   return MOE_OK;
 }

@@ -116,6 +116,39 @@ class MoELayer:
 
     __call__ = forward
 
+    def workspace_bytes_w4(self, T: int) -> int:
+        return int(lib().moe_workspace_bytes_w4(self._h, T))
+
+    def forward_w4(self, x, W_r, b_r, W1q, W3q, W2q, *, out=None, stats=None, workspace=None,
+                   debug: Optional[dict] = None, stream=None):
+        """The layer with 4-bit expert weights: W1q, W3q (None for ReLU), W2q are
+        (codes, scales) pairs from quantize_int4.  Returns like forward()."""
+        T = x.shape[0]
+        dev = x.device
+        y = out if out is not None else torch.empty((T, self.d), dtype=x.dtype, device=dev)
+        if stats is None:
+            stats = (torch.empty(self.E, dtype=torch.int32, device=dev),
+                     torch.empty(1, dtype=torch.int32, device=dev),
+                     torch.empty(1, dtype=torch.float32, device=dev),
+                     torch.empty(1, dtype=torch.float32, device=dev))
+        counts, dropped, aux, z = stats
+        if workspace is None:
+            n = self.workspace_bytes_w4(T)
+            if self._ws is None or self._ws.numel() < n or self._ws.device != dev:
+                self._ws = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
+            workspace = self._ws
+        dbg = None
+        if debug is not None:
+            dbg = MoEDebug()
+            for name, t in debug.items():
+                setattr(dbg, name, _ptr(t))
+        q3, s3 = (None, None) if W3q is None else W3q
+        check(lib().moe_forward_w4(
+            self._h, T, _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(W1q[0]), _ptr(W1q[1]), _ptr(q3), _ptr(s3),
+            _ptr(W2q[0]), _ptr(W2q[1]), _ptr(y), _ptr(counts), _ptr(dropped), _ptr(aux), _ptr(z),
+            _ptr(workspace), workspace.numel(), None if dbg is None else ctypes.byref(dbg), _stream_handle(stream)))
+        return y, counts, dropped, aux, z
+
     def backward_workspace_bytes(self, T: int) -> int:
         return int(lib().moe_backward_workspace_bytes(self._h, T))
 
@@ -170,6 +203,19 @@ class MoELayer:
             "expert_offsets": torch.empty(E + 1, dtype=torch.int32, device=device),
             "y_f32": torch.empty((T, self.d), dtype=torch.float32, device=device),
         }
+
+
+def quantize_int4(W: torch.Tensor, stream=None):
+    """4-bit codes (int32 view of uint32 [rows][K / 8]) and bf16 scales
+    [rows][K / 128] of a bf16 weight [..., K] (rows = every leading index),
+    in the format of include/moe.h."""
+    K = W.shape[-1]
+    lead = W.shape[:-1]
+    rows = W.numel() // K if K else 0
+    codes = torch.empty(lead + (K // 8,), dtype=torch.int32, device=W.device)
+    scales = torch.empty(lead + (K // 128,), dtype=torch.bfloat16, device=W.device)
+    check(lib().moe_quantize_int4(_ptr(W.contiguous()), rows, K, _ptr(codes), _ptr(scales), _stream_handle(stream)))
+    return codes, scales
 
 
 def status(stream=None) -> None:
