@@ -43,6 +43,9 @@ METRIC = "MoE-layer tokens/s on 1 B200 and % of roofline (TFLOP/s or HBM GB/s)"
 DEFAULT_WORKLOAD = "mixtral_prefill"
 # measured before the headline in the default one-GPU run
 SECONDARY = ["switch_k1", "mixtral_decode_t1", "mixtral_decode_t16", "mixtral_decode_t64", "fine_grained"]
+# (workload, expert weights): the decode layers also with 4-bit weights
+SECONDARY_RUNS = [(n, "dense") for n in SECONDARY] + [
+    (n, "int4") for n in ("mixtral_decode_t1", "mixtral_decode_t16", "mixtral_decode_t64")]
 DECODE_MIN_CALLS = 100  # decode layers report the p50 latency over at least this many calls
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # the nominal B200 figures the layer's targets are quoted against (dense bf16, HBM3e)
@@ -61,7 +64,12 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def layer_work(w, kept_counts):
+# bytes per weight element of the 4-bit format: half a byte of code plus a
+# 2-byte scale per 128 elements
+W4_BYTES_PER_WEIGHT = 0.5 + 2.0 / 128
+
+
+def layer_work(w, kept_counts, weights="dense"):
     """Algorithmic FLOPs and bytes of the layer and of each grouped GEMM launch.
 
     FLOPs count kept assignments only (plus T rows per shared expert) and the
@@ -73,12 +81,13 @@ def layer_work(w, kept_counts):
     SwiGLU) and x, the second projection its weights (W2) and y.
     """
     elt = 2 if w.dtype == 1 else 4
+    welt = W4_BYTES_PER_WEIGHT if weights == "int4" else elt
     n_sh = getattr(w, "n_shared", 0)
     S = int(sum(kept_counts)) + n_sh * w.T
     active = sum(1 for c in kept_counts if c > 0) + n_sh
     nproj1 = 2 if w.act == 1 else 1
-    w1_bytes = active * nproj1 * w.d_ff * w.d * elt
-    w2_bytes = active * w.d * w.d_ff * elt
+    w1_bytes = active * nproj1 * w.d_ff * w.d * welt
+    w2_bytes = active * w.d * w.d_ff * welt
     act_bytes = w.T * w.d * elt
     flops_router = 2.0 * w.T * w.E * w.d
     flops1 = 2.0 * S * w.d * w.d_ff * nproj1
@@ -291,13 +300,15 @@ def cpu_baseline(w, inp):
 
 
 # ----------------------------------------------------------------------------- GPU leg
-def measure_workload(args, w, dev, world, rank, local, K, warmup, cpu=True):
+def measure_workload(args, w, dev, world, rank, local, K, warmup, cpu=True, weights="dense"):
     """Time K forward passes of workload w (inputs resident in HBM), the
     per-stage breakdown in an untimed pass, and the end-to-end path with
-    pinned host buffers.  Returns the JSON line (rank 0) or None."""
+    pinned host buffers.  weights "int4": the experts' weights quantized to
+    the 4-bit format once, before any timing (moe_forward_w4).  Returns the
+    JSON line (rank 0) or None."""
     import torch
     import torch.distributed as dist
-    from sparse_mixture_experts_gating_b200 import MoELayer, launch_count, status
+    from sparse_mixture_experts_gating_b200 import MoELayer, launch_count, quantize_int4, status
     from sparse_mixture_experts_gating_b200.workloads import make_inputs, torch_dtype
 
     decode = w.name.startswith("mixtral_decode")
@@ -308,7 +319,15 @@ def measure_workload(args, w, dev, world, rank, local, K, warmup, cpu=True):
         inp["x"] = make_inputs(w.with_(seed=rank_seed(w.seed, rank)), device=dev, weights=False)["x"]
     layer = MoELayer(w.E, w.k, w.d, w.d_ff, act=w.act, gate_mode=w.gate, capacity_factor=w.capacity_factor,
                      dtype=torch_dtype(w.dtype), hidden=args.hidden, n_shared=w.n_shared)
-    ws = layer.workspace(w.T, dev)
+    w4 = weights == "int4"
+    if w4:
+        qw = {k: (None if inp[k] is None else quantize_int4(inp[k])) for k in ("W1", "W3", "W2")}
+        status()
+        inp["W1"] = inp["W3"] = inp["W2"] = None  # only the 4-bit copies stay resident
+        torch.cuda.empty_cache()
+        ws = torch.empty(max(layer.workspace_bytes_w4(w.T), 256), dtype=torch.uint8, device=dev)
+    else:
+        ws = layer.workspace(w.T, dev)
     y = torch.empty((w.T, w.d), dtype=inp["x"].dtype, device=dev)
     stats = (torch.empty(w.E, dtype=torch.int32, device=dev), torch.empty(1, dtype=torch.int32, device=dev),
              torch.empty(1, dtype=torch.float32, device=dev), torch.empty(1, dtype=torch.float32, device=dev))
@@ -326,7 +345,11 @@ def measure_workload(args, w, dev, world, rank, local, K, warmup, cpu=True):
 
     def step(events=None, x=None):
         a = args_fw if x is None else (x,) + args_fw[1:]
-        layer(*a, out=y, stats=stats, workspace=ws, events=events)
+        if w4:
+            layer.forward_w4(a[0], a[1], a[2], qw["W1"], qw["W3"], qw["W2"], out=y, stats=stats, workspace=ws,
+                             events=events)
+        else:
+            layer(*a, out=y, stats=stats, workspace=ws, events=events)
 
     for _ in range(warmup):
         flush_l2()
@@ -334,7 +357,8 @@ def measure_workload(args, w, dev, world, rank, local, K, warmup, cpu=True):
     status()
 
     stage_names = ["router", "scan", "dispatch", "gemm1", "gemm2", "combine"]
-    active = [n for n in stage_names if not (n == "combine" and w.dtype == 1 and w.k == 1 and w.n_shared == 0)]
+    active = [n for n in stage_names
+              if not (n == "combine" and w.dtype == 1 and w.k == 1 and w.n_shared == 0 and not w4)]
 
     # Untimed profiling pass: every stage bracketed by events -> per-kernel breakdown.
     Kp = min(K, 20)
@@ -416,10 +440,10 @@ def measure_workload(args, w, dev, world, rank, local, K, warmup, cpu=True):
     counts = stats[0].cpu().tolist()
     cap = layer.capacity(w.T)
     kept = [c if cap is None else min(c, cap) for c in counts]
-    work = layer_work(w, kept)
+    work = layer_work(w, kept, "int4" if w4 else "dense")
     peaks, peak_src = load_peaks()
     roof = kernel_roofline(work[dom]["flops"], work[dom]["bytes"], dom_ms / 1e3, peaks)
-    roof["kernel"] = f"{STAGE_KERNEL[dom]} ({dom})"
+    roof["kernel"] = f"{'w4_gemm_kernel' if w4 else STAGE_KERNEL[dom]} ({dom})"
     roof["peak_source"] = f"{peak_src} ({'bf16_tflops' if roof['bound'] == 'tensor' else 'hbm_gbs'}, burst)"
     roof["nominal_peak"] = NOMINAL_PEAKS["bf16_tflops" if roof["bound"] == "tensor" else "hbm_gbs"]
     tr = profiled_traffic(dom, w.name)
@@ -448,7 +472,9 @@ def measure_workload(args, w, dev, world, rank, local, K, warmup, cpu=True):
             "vs_baseline": None,
             "dtype": "bf16" if w.dtype == 1 else "f32",
             "data": "synthetic (seeded; shapes and distributions of the workload, random-init weights)",
-            "config": dict(config_of(w, world), hidden=args.hidden),
+            "config": dict(config_of(w, world), hidden=args.hidden,
+                           **({"weights": "int4 (codes + bf16 scale per 128; quantized before timing)"}
+                              if w4 else {})),
             "roofline": roof,
             "layer_roofline": {"floor_ms": round(floor_s * 1e3, 5), "frac": round(floor_s / (ms_step / 1e3), 4),
                                "floor_ms_nominal": round(floor_nom * 1e3, 5),
@@ -469,9 +495,11 @@ def measure_workload(args, w, dev, world, rank, local, K, warmup, cpu=True):
                                   "e2e_p50": round(statistics.median(e2e_ms), 5)}
         if args.hidden != "bf16x2":
             line["note"] = "hidden activation in one bf16 plane: outside the max-error parity bound"
-        if world == 1 and cpu and not args.no_cpu_baseline:
+        if world == 1 and cpu and not args.no_cpu_baseline and not w4:
             line["cpu_baseline"] = cpu_baseline(w, inp)
     del inp, ws, y, flush, flush_rd, x_host, y_host, x_dev
+    if w4:
+        del qw
     layer = None
     torch.cuda.empty_cache()
     return line
@@ -485,6 +513,8 @@ def summary_of(line):
            "layer_frac": line["layer_roofline"]["frac"], "layer_frac_nominal": line["layer_roofline"]["frac_nominal"],
            "e2e_tokens_per_s": line["e2e"]["value"], "sm_mhz": line["clocks"].get("sm_mhz"),
            "clock_reasons": line["clocks"].get("reasons")}
+    if "weights" in line["config"]:
+        out["weights"] = "int4"
     if "latency_ms" in line:
         out["p50_ms"] = line["latency_ms"]["p50"]
         out["calls"] = line["latency_ms"]["calls"]
@@ -506,6 +536,8 @@ def main():
                     help="override the workload's token count (small cases for profiler captures)")
     ap.add_argument("--backward", action="store_true",
                     help="time a training step instead: the forward pass, then the backward pass")
+    ap.add_argument("--weights", choices=["dense", "int4"], default="dense",
+                    help="expert weights: the layer dtype, or the 4-bit format (moe_forward_w4)")
     args = ap.parse_args()
 
     import torch
@@ -536,14 +568,16 @@ def main():
         return backward_bench(args, w, make_inputs(w, device=dev), warmup, world, rank, local, dev)
     others = []
     if args.workload is None and args.tokens is None and world == 1:
-        for other in SECONDARY:
-            line = measure_workload(args, WORKLOADS[other], dev, world, rank, local, args.steps, warmup)
+        for other, wts in SECONDARY_RUNS:
+            line = measure_workload(args, WORKLOADS[other], dev, world, rank, local, args.steps, warmup,
+                                    weights=wts)
             print(json.dumps(line), flush=True)
             others.append(line)
-    line = measure_workload(args, w, dev, world, rank, local, args.steps, warmup)
+    line = measure_workload(args, w, dev, world, rank, local, args.steps, warmup, weights=args.weights)
     if rank == 0:
         if others:
-            line["workloads"] = {o["config"]["workload"]: summary_of(o) for o in others}
+            line["workloads"] = {o["config"]["workload"] + ("_int4" if "weights" in o["config"] else ""):
+                                 summary_of(o) for o in others}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -28,6 +28,22 @@ def _stream_handle(stream) -> int:
     return s.cuda_stream
 
 
+def _debug_struct(debug: Optional[dict], events, stream) -> Optional[MoEDebug]:
+    """moe_debug of the given device tensors and stage events (None if neither)."""
+    if debug is None and events is None:
+        return None
+    dbg = MoEDebug()
+    for name, t in (debug or {}).items():
+        setattr(dbg, name, _ptr(t))
+    if events is not None:
+        for i, ev in enumerate(events):
+            if ev is not None:
+                if not ev.cuda_event:  # torch creates its CUDA event lazily, on first record
+                    ev.record(torch.cuda.current_stream() if stream is None else stream)
+                dbg.events[i] = ev.cuda_event
+    return dbg
+
+
 class MoELayer:
     """One MoE layer description (E experts, top-k, d -> d_ff -> d experts).
 
@@ -97,17 +113,7 @@ class MoELayer:
                      torch.empty(1, dtype=torch.float32, device=dev))
         counts, dropped, aux, z = stats
         ws = workspace if workspace is not None else self.workspace(T, dev)
-        dbg = None
-        if debug is not None or events is not None:
-            dbg = MoEDebug()
-            for name, t in (debug or {}).items():
-                setattr(dbg, name, _ptr(t))
-            if events is not None:
-                for i, ev in enumerate(events):
-                    if ev is not None:
-                        if not ev.cuda_event:  # torch creates its CUDA event lazily, on first record
-                            ev.record(torch.cuda.current_stream() if stream is None else stream)
-                        dbg.events[i] = ev.cuda_event
+        dbg = _debug_struct(debug, events, stream)
         check(lib().moe_forward(
             self._h, T, _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(y),
             _ptr(counts), _ptr(dropped), _ptr(aux), _ptr(z), _ptr(ws), ws.numel(),
@@ -120,7 +126,7 @@ class MoELayer:
         return int(lib().moe_workspace_bytes_w4(self._h, T))
 
     def forward_w4(self, x, W_r, b_r, W1q, W3q, W2q, *, out=None, stats=None, workspace=None,
-                   debug: Optional[dict] = None, stream=None):
+                   debug: Optional[dict] = None, events=None, stream=None):
         """The layer with 4-bit expert weights: W1q, W3q (None for ReLU), W2q are
         (codes, scales) pairs from quantize_int4.  Returns like forward()."""
         T = x.shape[0]
@@ -137,11 +143,7 @@ class MoELayer:
             if self._ws is None or self._ws.numel() < n or self._ws.device != dev:
                 self._ws = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
             workspace = self._ws
-        dbg = None
-        if debug is not None:
-            dbg = MoEDebug()
-            for name, t in debug.items():
-                setattr(dbg, name, _ptr(t))
+        dbg = _debug_struct(debug, events, stream)
         q3, s3 = (None, None) if W3q is None else W3q
         check(lib().moe_forward_w4(
             self._h, T, _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(W1q[0]), _ptr(W1q[1]), _ptr(q3), _ptr(s3),

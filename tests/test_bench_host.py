@@ -72,6 +72,16 @@ def test_layer_work_switch_counts_only_experts_with_kept_rows():
     assert work["gemm1"]["flops"] == 2.0 * work["S"] * 768 * 3072
 
 
+def test_layer_work_counts_four_bit_weights_as_codes_plus_scales():
+    w = WORKLOADS["mixtral_decode_t1"]
+    work = bench.layer_work(w, [1, 1, 0, 0, 0, 0, 0, 0], "int4")
+    per = 4096 * 14336 * (0.5 + 2 / 128)
+    assert work["active_experts"] == 2
+    assert work["gemm1"]["bytes"] == 2 * 2 * per + 4096 * 2
+    assert work["gemm2"]["bytes"] == 2 * per + 4096 * 2
+    assert work["gemm1"]["flops"] == bench.layer_work(w, [1, 1, 0, 0, 0, 0, 0, 0])["gemm1"]["flops"]
+
+
 def test_kernel_roofline_picks_the_binding_resource():
     peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0}
     r = bench.kernel_roofline(flops=1e12, nbytes=1e9, seconds=1e-3, peaks=peaks)
