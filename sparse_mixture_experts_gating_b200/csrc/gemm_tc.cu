@@ -142,6 +142,17 @@ __device__ __forceinline__ bool wait_or_abort(Ctl* c, uint64_t* bar, uint32_t pa
 // silu(a) * b with the fast divide (2 ulp; 0 once 1 + e^-a overflows, the limit of silu).
 __device__ __forceinline__ float silu_mul(float a, float b) { return __fdividef(a, 1.f + __expf(-a)) * b; }
 
+// fp16 pair of (v0, v1); `valid`: the pair is a stored element of the hidden
+// activation (rows past an expert's group and columns past N hold whatever
+// the tile's stale operands gave and are never stored), and only then can it
+// raise *bad when out of the fp16 range.
+__device__ __forceinline__ uint32_t pack_f16x2_in_range(float v0, float v1, bool valid, bool& bad) {
+  bool b = false;
+  const uint32_t r = pack_f16x2_checked(v0, v1, b);
+  bad |= b && valid;
+  return r;
+}
+
 // bf16 pair (hi, lo) with hi = RNE(v) and lo = RNE(v - hi): hi + lo carries
 // about 16 significant bits of v.
 __device__ __forceinline__ void split_bf16(float v0, float v1, uint32_t& hi, uint32_t& lo) {
@@ -338,7 +349,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const float h0 = silu_mul(__uint_as_float(ra[2 * i]), __uint_as_float(rb[2 * i]));
               const float h1 = silu_mul(__uint_as_float(ra[2 * i + 1]), __uint_as_float(rb[2 * i + 1]));
               if (OUT_SPLIT) split_bf16(h0, h1, hi[i], lo[i]);
-              else if (OUT_F16) hi[i] = pack_f16x2_checked(h0, h1, out_of_range);
+              else if (OUT_F16) hi[i] = pack_f16x2_in_range(h0, h1, vrow && n0 + c * 32 + 2 * i < p.N, out_of_range);
               else hi[i] = pack_bf16x2(h0, h1);
             }
           } else {
@@ -355,7 +366,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 h1 *= g;
               }
               if (OUT_SPLIT) split_bf16(h0, h1, hi[i], lo[i]);
-              else if (OUT_F16) hi[i] = pack_f16x2_checked(h0, h1, out_of_range);
+              else if (OUT_F16) hi[i] = pack_f16x2_in_range(h0, h1, vrow && n0 + c * 32 + 2 * i < p.N, out_of_range);
               else hi[i] = pack_bf16x2(h0, h1);
             }
             if (EPI == EPI_GATE_SCATTER_BF16 && p.out_f32 != nullptr && vrow) {  // debug copy

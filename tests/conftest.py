@@ -8,3 +8,16 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (sm_100a); parity tests of the CUDA path")
+
+
+import pytest  # noqa: E402
+
+
+@pytest.fixture(autouse=True)
+def _fresh_device_status(request):
+    """GPU tests start with the library's device error word clear, so an error
+    one test provokes on purpose (or causes) is reported by that test alone."""
+    if request.node.get_closest_marker("gpu") is not None:
+        from sparse_mixture_experts_gating_b200 import clear_status
+        clear_status()
+    yield

@@ -121,8 +121,14 @@ def test_skewed_case_pads_k_beyond_512():
 
 def test_full_size_switch_backward_matches_oracle():
     """The Switch workload at full size (T 8192, d 768, 64 experts, ReLU 3072,
-    capacity 1.25) with dyadic router inputs: every gradient tensor, every
-    element, against the backward oracle."""
+    capacity 1.25) with dyadic router inputs, every element of every gradient
+    tensor against the backward oracle, except where the ReLU derivative is a
+    floating-point decision: relu'(a) flips between 0 and 1 at a = 0, and the
+    kernel decides it on its fp32 sum of w1 x while the oracle decides it on
+    the exact value.  Where |a| is within the fp32 summation bound of zero
+    (d 2^-24 sum_c |w1_c x_c|) either decision is correct; the gradient of x of
+    that token and row f of that expert's dW1 are then not unique and are left
+    out (dW2, dW_r and db_r see relu(a) itself, which is continuous there)."""
     from sparse_mixture_experts_gating_b200.workloads import WORKLOADS
     w = WORKLOADS["switch_k1"].with_(dyadic=True)
     inp, _, dbg, dy, g = _run(w)
@@ -130,7 +136,26 @@ def test_full_size_switch_backward_matches_oracle():
     np.testing.assert_array_equal(dbg["topk_idx"].cpu().numpy(), o["idx"])
     np.testing.assert_array_equal(dbg["drop_mask"].cpu().numpy().astype(bool), ~o["kept"])
     assert not o["kept"].all()
-    for key in ("dx", "dW_r", "db_r", "dW1", "dW2"):
+    x = np32(inp["x"]).astype(np.float64)
+    W1 = inp["W1"]
+    tok_unsure = np.zeros(w.T, bool)
+    row_unsure = np.zeros((w.E, w.d_ff), bool)
+    for e in range(w.E):
+        ts = np.nonzero((o["idx"][:, 0] == e) & o["kept"][:, 0])[0]
+        if ts.size == 0:
+            continue
+        We = W1[e].float().cpu().numpy().astype(np.float64)
+        a = x[ts] @ We.T
+        bound = w.d * 2.0 ** -24 * (np.abs(x[ts]) @ np.abs(We).T)
+        near = np.abs(a) <= bound
+        tok_unsure[ts[near.any(axis=1)]] = True
+        row_unsure[e, near.any(axis=0)] = True
+    assert tok_unsure.sum() < 0.01 * w.T and row_unsure.sum() < 0.01 * w.E * w.d_ff
+    sure = ~tok_unsure
+    _close("dx", np32(g["dx"])[sure], o["dx"][sure])
+    dW1 = np32(g["dW1"])[:w.E]
+    _close("dW1", dW1[~row_unsure], o["dW1"][~row_unsure])
+    for key in ("dW_r", "db_r", "dW2"):
         _close(key, np32(g[key]), o[key])
 
 
