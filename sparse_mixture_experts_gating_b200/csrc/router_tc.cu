@@ -610,7 +610,11 @@ cudaError_t launch_k(const RoutingArgs& a, void* wsplit, void* partials, int num
 int router_ksplit(int64_t T, int d) {
   const int64_t tiles = (T + BM - 1) / BM;
   const int64_t num_kb = (d + BK - 1) / BK;
-  if (tiles <= 0 || tiles > 16) return 1;  // none, or enough tiles: the exchange would cost more than it saves
+  if (tiles <= 0) return 1;
+  // Up to one wave of tiles with a long K (d >= 2048): two K ranges per tile
+  // fill the idle SMs and halve each CTA's MMAs (prefill d 4096: 55 -> 39 us);
+  // with a short K the exchange costs more than it saves (d 768: 21.5 -> 25.4 us).
+  if (tiles > 16) return (tiles <= kSplitTargetCtas && num_kb >= 32) ? 2 : 1;
   int64_t ks = kSplitTargetCtas / tiles;
   if (ks > 16) ks = 16;
   if (ks > num_kb / 2) ks = num_kb / 2;
@@ -624,7 +628,7 @@ size_t router_partials_bytes(int64_t T, int E, int d) {
   // some T serves every smaller batch too
   size_t best = 0;
   const int64_t max_tiles = (T + BM - 1) / BM;
-  for (int64_t tiles = 1; tiles <= max_tiles && tiles <= 16; ++tiles) {
+  for (int64_t tiles = 1; tiles <= max_tiles && tiles <= kSplitTargetCtas; ++tiles) {
     const int ks = router_ksplit(tiles * BM, d);
     if (ks <= 1) continue;
     const size_t need = static_cast<size_t>(tiles) * ks * BM * router_pad_e(E) * sizeof(float) +
