@@ -655,9 +655,12 @@ cudaError_t launch_gemm_tc(const TcGemmPlan& pl, int num_sms, cudaStream_t s) {
 cudaError_t launch_convert_f16(const void* src, void* dst, int64_t n, unsigned int* err, int num_sms,
                                cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
+  // one block per SM: it runs beside the first projection's CTA on each SM
+  // and should take few of its issue slots (four 16-byte loads in flight per
+  // thread keep ~1 MB in flight across the GPU, enough for the ~1 TB/s it needs)
   const int64_t n8 = n / 8;
   int64_t blocks = (n8 + 255) / 256;
-  if (blocks > 4LL * num_sms) blocks = 4LL * num_sms;
+  if (blocks > num_sms) blocks = num_sms;
   return launch_pdl(convert_f16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
                     static_cast<const uint4*>(src), static_cast<uint4*>(dst), n8, err);
 }

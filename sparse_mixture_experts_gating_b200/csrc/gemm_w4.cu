@@ -15,14 +15,17 @@
 // reads as its A operand, while the activation tile comes from shared memory
 // through TMA.  HBM then carries the codes and scales only.
 //
-// Warp roles (448 threads, one CTA per SM):
+// Warp roles (704 threads, one CTA per SM):
 //   warp 0        TMA producer: per stage the code tile(s) [128 rows x 32 B]
 //                 and the activation tile [NB rows x 64] (hi and lo planes
 //                 of the hidden activation for the second projection)
 //   warp 1        TMEM allocator; lane 0 issues the MMAs (M 128, N NB, K 16)
-//   warps 2..9    dequantize: warp w owns TMEM lanes 32 (w % 4) .. + 31 (one
-//                 weight row per lane) and half (w - 2) / 4 of each k-block
-//   warps 10..13  epilogue: activation (first projection) or gate (second)
+//   warps 2..17   dequantize: warp w owns TMEM lanes 32 (w % 4) .. + 31 (one
+//                 weight row per lane) and quarter (w - 2) / 4 of each
+//                 k-block (16 elements, 8 TMEM columns); it prefetches the
+//                 next scale group and keeps one k-block's tensor-memory
+//                 stores in flight while it dequantizes the next
+//   warps 18..21  epilogue: activation (first projection) or gate (second)
 //                 and the stores, one weight row (output column) per lane
 // The dequantized values are exact: (code - 8) * scale with a scale of at
 // most 5 significant bits fits bf16 exactly, and both steps are exact bf16x2
@@ -41,15 +44,29 @@ namespace {
 constexpr int WBM = 128;                 // weight rows per tile (TMEM lanes)
 constexpr int WBK = 64;                  // K per k-block
 constexpr int Q_TILE = WBM * WBK / 2;    // bytes of codes per weight tile and k-block (4 KB)
-constexpr int A_STAGES = 4;              // TMEM A ring
+constexpr int MAX_A_STAGES = 8;          // TMEM A ring
 constexpr int MAX_SMEM_STAGES = 8;
-constexpr int W4_THREADS = 448;
+constexpr int DQ_WARPS = 16;
+constexpr int EPI_WARP0 = 2 + DQ_WARPS;
+constexpr int W4_THREADS = 32 * (EPI_WARP0 + 4);
+constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_G = 256;
 
 template <int MODE>
 struct W4Geo {
   static constexpr int NQ = MODE == W4_SWIGLU ? 2 : 1;      // weight matrices per tile (W1 and W3)
   static constexpr int PLANES = MODE == W4_GATE ? 2 : 1;    // activation planes (hidden hi + lo)
+};
+
+// TMEM: two accumulators of NQ x NB columns, the rest (up to 8 stages of
+// NQ x 32 columns) for the dequantized A ring.
+template <int MODE, int NB>
+struct W4Tmem {
+  static constexpr int NQ = W4Geo<MODE>::NQ;
+  static constexpr int FREE = (static_cast<int>(TMEM_COLS) - 2 * NQ * NB) / (NQ * 32);
+  static constexpr int A_STAGES = FREE < MAX_A_STAGES ? FREE : MAX_A_STAGES;
+  static constexpr uint32_t ACC0 = A_STAGES * NQ * 32;  // first accumulator column
+  static_assert(A_STAGES >= 2, "tensor memory too small for the A ring");
 };
 
 template <int MODE, int NB>
@@ -61,8 +78,8 @@ struct W4Stage {
 struct W4Ctl {
   uint64_t full[MAX_SMEM_STAGES];
   uint64_t empty[MAX_SMEM_STAGES];
-  uint64_t afull[A_STAGES];
-  uint64_t aempty[A_STAGES];
+  uint64_t afull[MAX_A_STAGES];
+  uint64_t aempty[MAX_A_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -77,11 +94,6 @@ constexpr size_t w4_smem_bytes() {
   return W4Stage<MODE, NB>::N * W4Stage<MODE, NB>::BYTES + sizeof(W4Ctl) + 1024;
 }
 
-template <int MODE, int NB>
-constexpr uint32_t w4_tmem_cols() {
-  constexpr int used = A_STAGES * W4Geo<MODE>::NQ * 32 + 2 * W4Geo<MODE>::NQ * NB;
-  return used <= 32 ? 32 : used <= 64 ? 64 : used <= 128 ? 128 : used <= 256 ? 256 : 512;
-}
 
 // unit -> (group, m-tile over weight rows, n-tile over activation rows, K range)
 struct W4Item {
@@ -145,8 +157,8 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   constexpr int NQ = Geo::NQ, PLANES = Geo::PLANES;
   constexpr int STAGES = St::N, STAGE_BYTES = St::BYTES;
   constexpr int X_OFF = NQ * Q_TILE;
-  constexpr uint32_t TMEM_COLS = w4_tmem_cols<MODE, NB>();
-  constexpr uint32_t ACC0 = A_STAGES * NQ * 32;  // first accumulator column
+  constexpr int A_STAGES = W4Tmem<MODE, NB>::A_STAGES;
+  constexpr uint32_t ACC0 = W4Tmem<MODE, NB>::ACC0;
   constexpr uint32_t IDESC = idesc_bf16_f32(WBM, NB);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -156,7 +168,7 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
-    for (int a = 0; a < A_STAGES; ++a) { mbar_init(&ctl->afull[a], 8); mbar_init(&ctl->aempty[a], 1); }
+    for (int a = 0; a < A_STAGES; ++a) { mbar_init(&ctl->afull[a], DQ_WARPS); mbar_init(&ctl->aempty[a], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&ctl->tfull[a], 1); mbar_init(&ctl->tempty[a], 128); }
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
@@ -247,48 +259,69 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       umma_commit(&ctl->drain);
       mbar_wait(&ctl->drain, 0, p.limit_ns);
     }
-  } else if (warp < 10) {
+  } else if (warp < EPI_WARP0) {
     // ------------------------------------------------------------ dequantize
-    const int q = warp & 3, half = (warp - 2) >> 2;
+    const int q = warp & 3, part = (warp - 2) >> 2;  // 16 elements (8 columns) of each k-block
     const int r = q * 32 + lane;  // weight row within the tile
     const int groups = p.K / W4_GROUP;
-    int stage = 0, astage = 0;
+    const __nv_bfloat16 zero = __float2bfloat16(0.f);
+    int stage = 0, astage = 0, held = -1;  // held: A stage whose stores are still in flight
     uint32_t phase = 0, aphase = 0;
     bool ok = true;
     W4Item w;
     for (int u = blockIdx.x; ok && w4_item(ctl, p, u, w); u += gridDim.x) {
       const int64_t row = static_cast<int64_t>(w.e) * p.N + w.mt * WBM + r;
       const bool vrow = w.mt * WBM + r < p.N;
+      const __nv_bfloat16* s0p = p.S0 + row * groups;
+      const __nv_bfloat16* s1p = p.S1 + row * groups;
+      // scales of this k-block's group and the next one, loaded one group ahead
+      int g_cur = (w.kb0 * WBK + part * 16) / W4_GROUP;
+      __nv_bfloat16 sc0 = vrow ? s0p[g_cur] : zero, sc1 = (NQ == 2 && vrow) ? s1p[g_cur] : zero;
+      __nv_bfloat16 nx0 = (vrow && g_cur + 1 < groups) ? s0p[g_cur + 1] : zero;
+      __nv_bfloat16 nx1 = (NQ == 2 && vrow && g_cur + 1 < groups) ? s1p[g_cur + 1] : zero;
       for (int kb = w.kb0; kb < w.kb1; ++kb) {
-        // this half's 32 elements lie in one scale group
-        const int grp = (kb * WBK + half * 32) / W4_GROUP;
-        const __nv_bfloat16 s0 = vrow ? p.S0[row * groups + grp] : __float2bfloat16(0.f);
-        const __nv_bfloat16 s1 = (NQ == 2 && vrow) ? p.S1[row * groups + grp] : __float2bfloat16(0.f);
+        const int grp = (kb * WBK + part * 16) / W4_GROUP;
+        if (grp != g_cur) {
+          g_cur = grp;
+          sc0 = nx0;
+          sc1 = nx1;
+          nx0 = (vrow && grp + 1 < groups) ? s0p[grp + 1] : zero;
+          if (NQ == 2) nx1 = (vrow && grp + 1 < groups) ? s1p[grp + 1] : zero;
+        }
         const bool got = __all_sync(0xffffffffu, w4_wait(ctl, &ctl->full[stage], phase, p) &&
                                                      w4_wait(ctl, &ctl->aempty[astage], aphase ^ 1u, p));
         if (!got) { ok = false; break; }
         tc_fence_after();
         const uint8_t* st = stages + stage * STAGE_BYTES;
-        const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                              static_cast<uint32_t>(astage * NQ * 32 + half * 16);
+        uint32_t v[NQ][8];
 #pragma unroll
         for (int m = 0; m < NQ; ++m) {
-          const uint4 words = *reinterpret_cast<const uint4*>(st + m * Q_TILE + r * 32 + half * 16);
-          const __nv_bfloat162 s2 = __bfloat162bfloat162(m == 0 ? s0 : s1);
-          uint32_t v[16];
-          dequant_word(words.x, s2, v);
-          dequant_word(words.y, s2, v + 4);
-          dequant_word(words.z, s2, v + 8);
-          dequant_word(words.w, s2, v + 12);
-          tmem_st16(tcol + m * 32, v);
+          const uint2 words = *reinterpret_cast<const uint2*>(st + m * Q_TILE + r * 32 + part * 8);
+          const __nv_bfloat162 s2 = __bfloat162bfloat162(m == 0 ? sc0 : sc1);
+          dequant_word(words.x, s2, v[m]);
+          dequant_word(words.y, s2, v[m] + 4);
         }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->afull[astage]);
+        // the previous k-block's stores completed: hand that A stage to the MMA
+        if (held >= 0) {
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->afull[held]);
+        }
+        const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                              static_cast<uint32_t>(astage * NQ * 32 + part * 8);
+#pragma unroll
+        for (int m = 0; m < NQ; ++m) tmem_st8(tcol + m * 32, v[m]);
+        held = astage;
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         if (++astage == A_STAGES) { astage = 0; aphase ^= 1u; }
       }
+    }
+    if (held >= 0) {
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(&ctl->afull[held]);
     }
   } else {
     // ------------------------------------------------------------ epilogue

@@ -96,11 +96,17 @@ int w4_ksplit(int64_t s, int groups, int d, int d_ff) {
   const int64_t g = std::min<int64_t>(groups, s);
   const int64_t tiles = (g + (s - g) / nb) * ((d + 127) / 128);
   const int64_t num_kb = d_ff / 64;
-  if (tiles <= 0 || tiles >= 2 * kSplitTargetCtas) return 1;
-  int64_t ks = (2 * kSplitTargetCtas + tiles - 1) / tiles;
-  ks = std::min<int64_t>(ks, std::max<int64_t>(num_kb / 4, 1));
-  const int64_t per = (num_kb + ks - 1) / ks;
-  return static_cast<int>((num_kb + per - 1) / per);
+  if (tiles <= 0 || tiles >= 4 * kSplitTargetCtas) return 1;
+  // the cut whose longest CTA (ceil(units / SMs) ranges of `per` k-blocks) is
+  // shortest; more ranges only for a gain above 3 % (each adds fp32 partial rows)
+  int64_t best = 1, best_len = (tiles + kSplitTargetCtas - 1) / kSplitTargetCtas * num_kb;
+  for (int64_t ks = 2; ks <= num_kb / 4; ++ks) {
+    const int64_t per = (num_kb + ks - 1) / ks;
+    const int64_t ranges = (num_kb + per - 1) / per;
+    const int64_t len = (tiles * ranges + kSplitTargetCtas - 1) / kSplitTargetCtas * per;
+    if (len * 32 < best_len * 31) { best = ranges; best_len = len; }
+  }
+  return static_cast<int>(best);
 }
 
 int ksplit_of(const moe_layer& L, int64_t s_max, bool w4) {

@@ -611,10 +611,11 @@ int router_ksplit(int64_t T, int d) {
   const int64_t tiles = (T + BM - 1) / BM;
   const int64_t num_kb = (d + BK - 1) / BK;
   if (tiles <= 0) return 1;
-  // Up to one wave of tiles with a long K (d >= 2048): two K ranges per tile
-  // fill the idle SMs and halve each CTA's MMAs (prefill d 4096: 55 -> 39 us);
-  // with a short K the exchange costs more than it saves (d 768: 21.5 -> 25.4 us).
-  if (tiles > 16) return (tiles <= kSplitTargetCtas && num_kb >= 32) ? 2 : 1;
+  // Up to one wave of tiles with a long K (d >= 4096): two K ranges per tile
+  // fill the idle SMs and halve each CTA's MMAs (prefill d 4096, 64 tiles:
+  // 57 -> 41 us); with a shorter K the exchange costs more than it saves
+  // (d 768, 64 tiles: 21.5 -> 25.4 us; d 2048, 128 tiles: 52 -> 77 us).
+  if (tiles > 16) return (tiles <= kSplitTargetCtas && num_kb >= 64) ? 2 : 1;
   int64_t ks = kSplitTargetCtas / tiles;
   if (ks > 16) ks = 16;
   if (ks > num_kb / 2) ks = num_kb / 2;

@@ -122,13 +122,18 @@ def test_skewed_case_pads_k_beyond_512():
 def test_full_size_switch_backward_matches_oracle():
     """The Switch workload at full size (T 8192, d 768, 64 experts, ReLU 3072,
     capacity 1.25) with dyadic router inputs, every element of every gradient
-    tensor against the backward oracle, except where the ReLU derivative is a
-    floating-point decision: relu'(a) flips between 0 and 1 at a = 0, and the
-    kernel decides it on its fp32 sum of w1 x while the oracle decides it on
-    the exact value.  Where |a| is within the fp32 summation bound of zero
-    (d 2^-24 sum_c |w1_c x_c|) either decision is correct; the gradient of x of
-    that token and row f of that expert's dW1 are then not unique and are left
-    out (dW2, dW_r and db_r see relu(a) itself, which is continuous there)."""
+    tensor against the backward oracle.
+
+    The ReLU derivative is a floating-point decision: relu'(a) jumps from 0 to 1
+    at a = 0, and the kernel takes it on its fp32 tensor-core sum of w1 x while
+    the oracle takes it on the exact value.  Where |a| lies within the fp32
+    summation bound of 0 ((d / 16 + 16) 2^-23 sum_c |w1_c x_c|: fp32 partial
+    sums of 16 exact products, one rounding each, counted at double the unit
+    roundoff) either decision is correct, and the gradients that see it (dx of
+    that token, row f of that expert's dW1) may differ from the oracle's by
+    the whole term |U_tf| |W1[f]| (resp. |U_tf| |x_t|), U_tf = g_t (W2^T dy_t)_f;
+    they are checked to within that allowance, everything else to the usual
+    bound.  dW2, dW_r and db_r see relu(a) itself, continuous there."""
     from sparse_mixture_experts_gating_b200.workloads import WORKLOADS
     w = WORKLOADS["switch_k1"].with_(dyadic=True)
     inp, _, dbg, dy, g = _run(w)
@@ -137,24 +142,38 @@ def test_full_size_switch_backward_matches_oracle():
     np.testing.assert_array_equal(dbg["drop_mask"].cpu().numpy().astype(bool), ~o["kept"])
     assert not o["kept"].all()
     x = np32(inp["x"]).astype(np.float64)
-    W1 = inp["W1"]
-    tok_unsure = np.zeros(w.T, bool)
-    row_unsure = np.zeros((w.E, w.d_ff), bool)
+    dyh = np32(dy).astype(np.float64)
+    gate = dbg["topk_gate"].cpu().numpy().astype(np.float64)[:, 0]
+    allow_dx = np.zeros((w.T, w.d))
+    allow_dw1 = np.zeros((w.E, w.d_ff, w.d))
+    n_near_tokens = 0
     for e in range(w.E):
         ts = np.nonzero((o["idx"][:, 0] == e) & o["kept"][:, 0])[0]
         if ts.size == 0:
             continue
-        We = W1[e].float().cpu().numpy().astype(np.float64)
-        a = x[ts] @ We.T
-        bound = w.d * 2.0 ** -24 * (np.abs(x[ts]) @ np.abs(We).T)
+        W1e = inp["W1"][e].float().cpu().numpy().astype(np.float64)
+        W2e = inp["W2"][e].float().cpu().numpy().astype(np.float64)
+        a = x[ts] @ W1e.T
+        bound = (w.d / 16 + 16) * 2.0 ** -23 * (np.abs(x[ts]) @ np.abs(W1e).T)
         near = np.abs(a) <= bound
-        tok_unsure[ts[near.any(axis=1)]] = True
-        row_unsure[e, near.any(axis=0)] = True
-    assert tok_unsure.sum() < 0.01 * w.T and row_unsure.sum() < 0.01 * w.E * w.d_ff
-    sure = ~tok_unsure
-    _close("dx", np32(g["dx"])[sure], o["dx"][sure])
-    dW1 = np32(g["dW1"])[:w.E]
-    _close("dW1", dW1[~row_unsure], o["dW1"][~row_unsure])
+        rows = np.nonzero(near.any(axis=1))[0]
+        n_near_tokens += rows.size
+        if rows.size == 0:
+            continue
+        U = np.abs(gate[ts[rows], None] * (dyh[ts[rows]] @ W2e)) * near[rows]  # [n][d_ff], 0 where sure
+        allow_dx[ts[rows]] = U @ np.abs(W1e)
+        allow_dw1[e] = U.T @ np.abs(x[ts[rows]])
+    assert n_near_tokens < 0.5 * w.T
+
+    def close_with(name, got, ref, allow):
+        scale = float(np.abs(ref).max())
+        err = np.abs(np.asarray(got, np.float64) - ref)
+        assert (err <= TOL * scale + allow).all(), f"{name}: max excess {(err - TOL * scale - allow).max():.3e}"
+
+    close_with("dx", np32(g["dx"]), o["dx"], allow_dx)
+    close_with("dW1", np32(g["dW1"])[:w.E], o["dW1"], allow_dw1)
+    sure = allow_dx.max(axis=1) == 0
+    _close("dx (tokens whose ReLU decisions are unique)", np32(g["dx"])[sure], o["dx"][sure])
     for key in ("dW_r", "db_r", "dW2"):
         _close(key, np32(g[key]), o[key])
 

@@ -66,8 +66,8 @@ SMALL = [
     # scan and dispatch, so the scan runs as its own launch (one block per
     # expert); the other cases above route in the fused launch
     ("e256_separate_scan", 2100, 64, 256, 1, 64, R, SW, 1.0, BF, "normal"),
-    # 17..148 router tiles with d >= 2048: two K ranges per 128-token tile
-    ("router_two_k_ranges", 2500, 2048, 128, 4, 256, S, RN, 2.0, BF, "zipf"),
+    # 17..148 router tiles with d >= 4096: two K ranges per 128-token tile
+    ("router_two_k_ranges", 2500, 4096, 64, 2, 256, S, RN, 2.0, BF, "zipf"),
 ]
 
 
