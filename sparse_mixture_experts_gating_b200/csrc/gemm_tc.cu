@@ -97,26 +97,46 @@ __device__ __forceinline__ void decode_tile(int t, const Ctl* c, int E, int n_ti
 }
 
 // Work of one CTA, identical in every role: units u = blockIdx.x + j * gridDim.x
-// below tiles * ksplit; unit u is tile u / ksplit, K range u % ksplit
-// (ksplit > 1 only for the gated fp32 epilogue, whose partial outputs the
-// combine kernel sums in order).
+// below the unit count.  With ksplit > 1 (the gated fp32 epilogue only, whose
+// partial outputs the combine kernel sums in order) unit u is tile u / ksplit,
+// K range u % ksplit.  Otherwise, when the tiles leave a last wave at most
+// half full (p.split_tail: not SwiGLU, whose tile pairs W1 and W3 columns),
+// each tile of that last wave becomes two units of half its columns (N 128),
+// so the last wave takes half as long.
 struct Item {
   int tile, ks;    // tile and K-range index
   int kb0, kb1;    // k-blocks [kb0, kb1)
+  int half;        // -1: all of the tile's columns; 0 / 1: that half of them
 };
 struct ItemIter {
-  int u, units;
+  int u, units, whole;  // whole: units that are whole tiles (the rest are halves)
 };
 __device__ __forceinline__ ItemIter iter_begin(const Ctl* c, const Params& p) {
   ItemIter it;
   it.u = static_cast<int>(blockIdx.x);
-  it.units = c->mprefix[p.E] * p.n_tiles * p.ksplit;
+  const int tiles = c->mprefix[p.E] * p.n_tiles;
+  if (p.ksplit == 1 && p.split_tail) {
+    const int ctas = static_cast<int>(gridDim.x);
+    const int r = tiles % ctas;
+    it.whole = (r > 0 && 2 * r <= ctas) ? tiles - r : tiles;
+    it.units = it.whole + 2 * (tiles - it.whole);
+  } else {
+    it.whole = it.units = tiles * p.ksplit;
+  }
   return it;
 }
 __device__ __forceinline__ bool iter_next(ItemIter& it, const Params& p, Item& w) {
   if (it.u >= it.units) return false;
-  w.tile = it.u / p.ksplit;
-  w.ks = it.u - w.tile * p.ksplit;
+  if (it.u < it.whole) {
+    w.tile = it.u / p.ksplit;
+    w.ks = it.u - w.tile * p.ksplit;
+    w.half = -1;
+  } else {
+    const int v = it.u - it.whole;
+    w.tile = it.whole + (v >> 1);
+    w.ks = 0;
+    w.half = v & 1;
+  }
   w.kb0 = w.ks * p.kb_per;
   w.kb1 = min(p.num_kb, w.kb0 + p.kb_per);
   it.u += static_cast<int>(gridDim.x);
@@ -178,6 +198,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr bool OUT_SPLIT = HID == HID_BF16X2 && !GATE;
   constexpr bool OUT_F16 = HID == HID_F16 && !GATE;
   constexpr uint32_t IDESC = (HID == HID_F16 && GATE) ? idesc_f16_f32(BM, MMA_N) : idesc_bf16_f32(BM, MMA_N);
+  constexpr uint32_t IDESC_HALF =
+      (HID == HID_F16 && GATE) ? idesc_f16_f32(BM, MMA_N / 2) : idesc_bf16_f32(BM, MMA_N / 2);
   using G = Geo<A_SPLIT, AR>;
   constexpr int STAGES = G::STAGES;
   constexpr int STAGE_BYTES = G::STAGE_BYTES;
@@ -225,9 +247,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int e, mt, nt;
         decode_tile(w.tile, ctl, p.E, p.n_tiles, e, mt, nt);
         const int row0 = ctl->offsets[e] + mt * BM;
-        const int brow = e * p.N + nt * p.bn;
+        const int brow = e * p.N + nt * p.bn + (w.half > 0 ? 128 : 0);
         const int kb0 = w.kb0, kb1 = w.kb1;
-        constexpr uint32_t tx = (A_SPLIT ? 2u : 1u) * A_ST + 2u * B_HALF;
+        const uint32_t tx = (A_SPLIT ? 2u : 1u) * A_ST + (w.half >= 0 ? 1u : 2u) * B_HALF;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_or_abort(ctl, &ctl->empty[stage], phase ^ 1u, p)) { ok = false; break; }
           uint8_t* sa = stages + stage * STAGE_BYTES;
@@ -237,6 +259,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (EPI == EPI_SWIGLU_BF16) {
             tma_load_2d(sa + B_OFF, &tmB0, &ctl->full[stage], kb * BK, brow);
             tma_load_2d(sa + B_OFF + B_HALF, &tmB1, &ctl->full[stage], kb * BK, brow);
+          } else if (w.half >= 0) {
+            tma_load_2d(sa + B_OFF, &tmB1, &ctl->full[stage], kb * BK, brow);  // 128-row box
           } else {
             tma_load_2d(sa + B_OFF, &tmB0, &ctl->full[stage], kb * BK, brow);  // 256-row box
           }
@@ -267,14 +291,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
           const uint32_t sa = smem_u32(stages + stage * STAGE_BYTES);
           const uint32_t sb = sa + B_OFF;
+          const uint32_t idesc = w.half >= 0 ? IDESC_HALF : IDESC;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_bf16(d_tmem, sdesc_k_sw128(sa + k * 32), sdesc_k_sw128(sb + k * 32), IDESC,
+            umma_bf16(d_tmem, sdesc_k_sw128(sa + k * 32), sdesc_k_sw128(sb + k * 32), idesc,
                       (kb != kb0 || k != 0) ? 1u : 0u);
           if (A_SPLIT) {
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k)
-              umma_bf16(d_tmem, sdesc_k_sw128(sa + A_ST + k * 32), sdesc_k_sw128(sb + k * 32), IDESC, 1u);
+              umma_bf16(d_tmem, sdesc_k_sw128(sa + A_ST + k * 32), sdesc_k_sw128(sb + k * 32), idesc, 1u);
           }
           umma_commit(&ctl->empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -316,7 +341,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         continue;
       }
       const int row = ctl->offsets[e] + m_local;  // expert-sorted row of this lane
-      const int n0 = nt * p.bn;
+      const int n0 = nt * p.bn + (w.half > 0 ? 128 : 0);
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * MMA_N);
       // destination row of each 32-row block row this lane stores (for bf16: rows lane/4 + 8i)
       int drow[4];
@@ -331,7 +356,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
 
       if (EPI == EPI_SWIGLU_BF16 || EPI == EPI_RELU_BF16 || EPI == EPI_GATE_SCATTER_BF16) {
-        constexpr int NCH = (EPI == EPI_SWIGLU_BF16) ? 4 : 8;
+        const int NCH = (EPI == EPI_SWIGLU_BF16 || w.half >= 0) ? 4 : 8;
         bool out_of_range = false;  // OUT_F16: a hidden value beyond the fp16 range
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
         __nv_bfloat16* out_lo = static_cast<__nv_bfloat16*>(p.out_lo);
@@ -399,8 +424,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (OUT_F16 && __any_sync(0xffffffffu, out_of_range) && lane == 0) record_error(p.err, DEV_ERR_RANGE);
       } else {  // EPI_GATE_F32: gated fp32 rows of the expert-sorted buffer (partial ks)
         float* out = static_cast<float*>(p.out) + static_cast<int64_t>(ks) * p.split_stride;
+        const int nch = w.half >= 0 ? 4 : 8;
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < nch; ++c) {
           uint32_t ra[32];
           tmem_ld32(tb + c * 32, ra);
           tmem_ld_wait();
@@ -628,6 +654,7 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
   p.ksplit = g.epi == EPI_GATE_F32 ? (g.ksplit < 1 ? 1 : (g.ksplit > p.num_kb ? p.num_kb : g.ksplit)) : 1;
   p.kb_per = (p.num_kb + p.ksplit - 1) / p.ksplit;
   p.split_stride = g.split_stride;
+  p.split_tail = swiglu ? 0 : 1;
   p.out = g.out;
   p.out_lo = g.out2;
   p.out_f32 = g.out_f32;

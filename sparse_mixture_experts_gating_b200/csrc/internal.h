@@ -132,6 +132,7 @@ struct GemmArgs {
 struct TcParams {
   int E, N, K, n_tiles, bn, num_kb;
   int ksplit, kb_per;      // K ranges per (expert, m-tile, n-tile) and k-blocks in each
+  int split_tail;          // a last wave at most half full runs as half-width (N 128) units
   int64_t split_stride;    // elements between the partial outputs of consecutive K ranges
   void* out;
   void* out_lo;     // first projection with a split hidden activation: the lo plane
