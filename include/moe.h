@@ -214,17 +214,25 @@ MOE_API int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r
  *     consecutive elements; group g has a bf16 scale s_g with at most 5
  *     significant bits, and element k is w_k = (u_k - 8) * s_{k / 128} with a
  *     4-bit code u_k in [0, 15] (so w_k is exact in bf16);
- *   - codes: uint32 [rows][K / 8]; word m holds elements 8m .. 8m+7 of its
- *     row, element 8m + 2j in bits 4j .. 4j+3 and element 8m + 2j + 1 in
- *     bits 4j+16 .. 4j+19 (j = 0 .. 3);  scales: bf16 [rows][K / 128].
- * Rows are the rows of the nn.Linear weights: W1 / W3 [E (+ n_shared)][d_ff]
- * rows of K = d, W2 [E (+ n_shared)][d] rows of K = d_ff.
+ *   - a word holds 8 consecutive elements 8m .. 8m+7 of a row, element
+ *     8m + 2j in bits 4j .. 4j+3 and element 8m + 2j + 1 in bits
+ *     4j+16 .. 4j+19 (j = 0 .. 3);
+ *   - codes are stored in tiles of 128 rows x 64 elements (rows a multiple of
+ *     128), each tile 4 KB contiguous with its row r at byte 32 r:
+ *     uint32 [rows / 128][K / 64][128][8]; the word of (row, 8m) is at index
+ *     ((row / 128) (K / 64) + 8m / 64) 1024 + (row % 128) 8 + (m % 8);
+ *   - scales: bf16 [rows / 128][K / 128][128], the scale of (row, group g) at
+ *     ((row / 128) (K / 128) + g) 128 + row % 128.
+ * The tiles make each 64-element slice of 128 rows one contiguous read.  Rows
+ * are the rows of the nn.Linear weights: W1 / W3 [E (+ n_shared)][d_ff] rows of
+ * K = d, W2 [E (+ n_shared)][d] rows of K = d_ff, so an expert's codes and
+ * scales are contiguous.
  *
  * moe_quantize_int4: codes and scales of a bf16 weight W [rows][K] (device
  * pointers; W and codes 16-byte aligned, scales 2-byte aligned), by
  * s = max|w| / 7 over the group in fp32, rounded up to 5 significant bits,
  * and u = round-half-even(w / s) + 8 in fp32 (u = 8 when s = 0).  Asynchronous
- * on `stream`.  K must be a multiple of 128, else MOE_ERR_UNSUPPORTED.
+ * on `stream`.  rows and K must be multiples of 128, else MOE_ERR_UNSUPPORTED.
  *
  * moe_forward_w4: moe_forward of a bf16 layer (d and d_ff multiples of 128)
  * whose expert weights are given in that format; the result is the layer

@@ -315,7 +315,9 @@ def moe_forward(x, W_r, b_r, W1, W3, W2, *, k: int, gate_mode: int, act: int,
 #   * the dequantized weight is q * s, exactly.
 # Storage: codes u = q + 8 in 4 bits; each 32-bit word holds 8 consecutive
 # elements k0..k7 of a row, element k_{2j} in bits 4j..4j+3 and element
-# k_{2j+1} in bits 4j+16..4j+19 (j = 0..3); scales are bfloat16.
+# k_{2j+1} in bits 4j+16..4j+19 (j = 0..3); words stored in tiles of 128 rows x
+# 64 elements, [rows / 128][K / 64][128 rows][8 words]; scales are bfloat16,
+# [rows / 128][K / INT4_GROUP][128 rows].
 INT4_GROUP = 128
 
 
@@ -344,7 +346,8 @@ def quantize_int4(W) -> tuple:
 
 
 def pack_int4(q: np.ndarray) -> np.ndarray:
-    """Words [rows][K / 8] (uint32) of codes q [rows][K] in the storage layout above."""
+    """Words (uint32, flat, in tiles) of codes q [rows][K] in the storage layout
+    above; rows and K multiples of 128."""
     q = np.asarray(q, np.int64)
     rows, K = q.shape
     u = (q + 8).reshape(rows, K // 8, 8).astype(np.uint64)
@@ -352,18 +355,28 @@ def pack_int4(q: np.ndarray) -> np.ndarray:
     for j in range(4):
         w |= u[:, :, 2 * j] << (4 * j)
         w |= u[:, :, 2 * j + 1] << (4 * j + 16)
-    return w.astype(np.uint32)
+    # [rows][K/8] -> [rows/128][128][K/64][8] -> [rows/128][K/64][128][8]
+    tiles = w.reshape(rows // 128, 128, K // 64, 8).transpose(0, 2, 1, 3)
+    return np.ascontiguousarray(tiles).astype(np.uint32).reshape(-1)
 
 
-def dequantize_int4(words, scales) -> np.ndarray:
-    """Weights [rows][K] (float64) from packed words [rows][K / 8] and scales
-    [rows][K / INT4_GROUP]: element k = (u_k - 8) * s_{k // INT4_GROUP}."""
-    w = np.asarray(words, np.uint64)
-    rows, K8 = w.shape
-    u = np.empty((rows, K8, 8), np.int64)
+def tile_scales(s: np.ndarray) -> np.ndarray:
+    """Scales [rows][K / INT4_GROUP] in the storage layout (flat, in tiles)."""
+    s = np.asarray(s)
+    rows, G = s.shape
+    return np.ascontiguousarray(s.reshape(rows // 128, 128, G).transpose(0, 2, 1)).reshape(-1)
+
+
+def dequantize_int4(words, scales, rows: int, K: int) -> np.ndarray:
+    """Weights [rows][K] (float64) from the stored words and scales (flat, in
+    tiles): element k of a row = (u_k - 8) * s_{k // INT4_GROUP}."""
+    w = np.asarray(words, np.uint64).reshape(rows // 128, K // 64, 128, 8).transpose(0, 2, 1, 3)
+    w = w.reshape(rows, K // 8)
+    u = np.empty((rows, K // 8, 8), np.int64)
     for j in range(4):
         u[:, :, 2 * j] = (w >> (4 * j)) & 0xF
         u[:, :, 2 * j + 1] = (w >> (4 * j + 16)) & 0xF
-    q = (u - 8).reshape(rows, K8 * 8).astype(np.float64)
-    s = np.repeat(np.asarray(scales, np.float64), INT4_GROUP, axis=1)
+    q = (u - 8).reshape(rows, K).astype(np.float64)
+    sc = np.asarray(scales, np.float64).reshape(rows // 128, K // INT4_GROUP, 128).transpose(0, 2, 1)
+    s = np.repeat(sc.reshape(rows, K // INT4_GROUP), INT4_GROUP, axis=1)
     return q * s

@@ -6,7 +6,10 @@
 // experts' weights).
 //
 // Weights arrive as 4-bit codes with one bf16 scale per 128 consecutive
-// elements of a row (format in include/moe.h, moe_quantize_int4).  The
+// elements of a row (format in include/moe.h, moe_quantize_int4), stored in
+// tiles of 128 rows x 64 elements so that every k-block of a weight tile is
+// one contiguous 4 KB copy (a row-major layout would fetch 32-byte pieces of
+// 128 rows 2 KB or more apart).  The
 // product runs transposed: D[f][n] = sum_k W[f][k] X[n][k], with the weight
 // rows f as the M = 128 operand and the (few) activation rows n of the
 // expert as the N operand (16, 32 or 64 columns).  Dequantized weights never
@@ -16,9 +19,9 @@
 // through TMA.  HBM then carries the codes and scales only.
 //
 // Warp roles (704 threads, one CTA per SM):
-//   warp 0        TMA producer: per stage the code tile(s) [128 rows x 32 B]
-//                 and the activation tile [NB rows x 64] (hi and lo planes
-//                 of the hidden activation for the second projection)
+//   warp 0        producer: per stage the code tile(s) (one 4 KB bulk copy
+//                 each) and the activation tile [NB rows x 64] by TMA (hi and
+//                 lo planes of the hidden activation for the second projection)
 //   warp 1        TMEM allocator; lane 0 issues the MMAs (M 128, N NB, K 16)
 //   warps 2..17   dequantize: warp w owns TMEM lanes 32 (w % 4) .. + 31 (one
 //                 weight row per lane) and quarter (w - 2) / 4 of each
@@ -150,8 +153,7 @@ __device__ __forceinline__ void dequant_word(uint32_t w, __nv_bfloat162 s2, uint
 
 template <int MODE, int NB>
 __global__ void __launch_bounds__(W4_THREADS, 1)
-    w4_gemm_kernel(const __grid_constant__ CUtensorMap tmQ0, const __grid_constant__ CUtensorMap tmQ1,
-                   const __grid_constant__ CUtensorMap tmX, const W4Params p) {
+    w4_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const W4Params p) {
   using Geo = W4Geo<MODE>;
   using St = W4Stage<MODE, NB>;
   constexpr int NQ = Geo::NQ, PLANES = Geo::PLANES;
@@ -173,8 +175,6 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     fence_mbarrier_init();
-    tma_prefetch_desc(&tmQ0);
-    if (NQ == 2) tma_prefetch_desc(&tmQ1);
     tma_prefetch_desc(&tmX);
   }
   if (warp == 1) tmem_alloc(&ctl->tmem_slot, TMEM_COLS);
@@ -202,14 +202,16 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       bool ok = true;
       W4Item w;
       for (int u = blockIdx.x; ok && w4_item(ctl, p, u, w); u += gridDim.x) {
-        const int qrow = w.e * p.N + w.mt * WBM;
+        // the unit's first code tile: tile row (e, mt), k-block kb at + kb * Q_TILE
+        const int64_t qtile = (static_cast<int64_t>(w.e) * p.m_tiles + w.mt) * p.num_kb * Q_TILE;
         const int xrow = ctl->offsets[w.e] + w.nt * NB;
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!w4_wait(ctl, &ctl->empty[stage], phase ^ 1u, p)) { ok = false; break; }
           uint8_t* st = stages + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
-          tma_load_2d(st, &tmQ0, &ctl->full[stage], kb * (WBK / 2), qrow);
-          if (NQ == 2) tma_load_2d(st + Q_TILE, &tmQ1, &ctl->full[stage], kb * (WBK / 2), qrow);
+          bulk_load(st, p.Q0 + qtile + static_cast<int64_t>(kb) * Q_TILE, Q_TILE, &ctl->full[stage]);
+          if (NQ == 2)
+            bulk_load(st + Q_TILE, p.Q1 + qtile + static_cast<int64_t>(kb) * Q_TILE, Q_TILE, &ctl->full[stage]);
           if (PLANES == 2) tma_load_3d(st + X_OFF, &tmX, &ctl->full[stage], kb * WBK, xrow, 0);
           else tma_load_2d(st + X_OFF, &tmX, &ctl->full[stage], kb * WBK, xrow);
           issued |= 1u << stage;
@@ -270,23 +272,24 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
     bool ok = true;
     W4Item w;
     for (int u = blockIdx.x; ok && w4_item(ctl, p, u, w); u += gridDim.x) {
-      const int64_t row = static_cast<int64_t>(w.e) * p.N + w.mt * WBM + r;
-      const bool vrow = w.mt * WBM + r < p.N;
-      const __nv_bfloat16* s0p = p.S0 + row * groups;
-      const __nv_bfloat16* s1p = p.S1 + row * groups;
+      const bool vrow = true;  // N is a multiple of 128
+      // scales of tile row (e, mt): [groups][128], this lane's row r
+      const int64_t sbase = (static_cast<int64_t>(w.e) * p.m_tiles + w.mt) * groups * WBM + r;
+      const __nv_bfloat16* s0p = p.S0 + sbase;
+      const __nv_bfloat16* s1p = p.S1 + sbase;
       // scales of this k-block's group and the next one, loaded one group ahead
       int g_cur = (w.kb0 * WBK + part * 16) / W4_GROUP;
-      __nv_bfloat16 sc0 = vrow ? s0p[g_cur] : zero, sc1 = (NQ == 2 && vrow) ? s1p[g_cur] : zero;
-      __nv_bfloat16 nx0 = (vrow && g_cur + 1 < groups) ? s0p[g_cur + 1] : zero;
-      __nv_bfloat16 nx1 = (NQ == 2 && vrow && g_cur + 1 < groups) ? s1p[g_cur + 1] : zero;
+      __nv_bfloat16 sc0 = vrow ? s0p[g_cur * WBM] : zero, sc1 = (NQ == 2 && vrow) ? s1p[g_cur * WBM] : zero;
+      __nv_bfloat16 nx0 = (vrow && g_cur + 1 < groups) ? s0p[(g_cur + 1) * WBM] : zero;
+      __nv_bfloat16 nx1 = (NQ == 2 && vrow && g_cur + 1 < groups) ? s1p[(g_cur + 1) * WBM] : zero;
       for (int kb = w.kb0; kb < w.kb1; ++kb) {
         const int grp = (kb * WBK + part * 16) / W4_GROUP;
         if (grp != g_cur) {
           g_cur = grp;
           sc0 = nx0;
           sc1 = nx1;
-          nx0 = (vrow && grp + 1 < groups) ? s0p[grp + 1] : zero;
-          if (NQ == 2) nx1 = (vrow && grp + 1 < groups) ? s1p[grp + 1] : zero;
+          nx0 = (vrow && grp + 1 < groups) ? s0p[(grp + 1) * WBM] : zero;
+          if (NQ == 2) nx1 = (vrow && grp + 1 < groups) ? s1p[(grp + 1) * WBM] : zero;
         }
         const bool got = __all_sync(0xffffffffu, w4_wait(ctl, &ctl->full[stage], phase, p) &&
                                                      w4_wait(ctl, &ctl->aempty[astage], aphase ^ 1u, p));
@@ -419,14 +422,14 @@ __global__ void __launch_bounds__(256) quantize_int4_kernel(const __nv_bfloat16*
   const uint32_t part = (lane & 1) == 0 ? (u[0] | (u[1] << 16) | (u[2] << 4) | (u[3] << 20))
                                         : ((u[0] << 8) | (u[1] << 24) | (u[2] << 12) | (u[3] << 28));
   const uint32_t word = part | __shfl_xor_sync(0xffffffffu, part, 1);
-  if ((lane & 1) == 0) codes[(row * K + grp * W4_GROUP) / 8 + lane / 2] = word;
-  if (lane == 0) scales[row * groups + grp] = __float2bfloat16_rn(s);
+  // tiled layout: tile (row / 128, k-block), 128 rows x 8 words each
+  const int m = lane / 2;                      // word of the group, 0 .. 15
+  const int64_t trow = row / 128, rin = row % 128;
+  const int64_t kb = 2 * grp + m / 8;          // k-block of 64 elements
+  if ((lane & 1) == 0) codes[((trow * (K / 64) + kb) * 128 + rin) * 8 + (m % 8)] = word;
+  if (lane == 0) scales[(trow * groups + grp) * 128 + rin] = __float2bfloat16_rn(s);
 }
 
-// Row-major uint8 [rows][bytes] -> map with box [128 rows][32 bytes], no swizzle.
-bool make_map_codes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t bytes) {
-  return make_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, rows, bytes, 1, 32, WBM, CU_TENSOR_MAP_SWIZZLE_NONE);
-}
 
 template <int MODE, int NB>
 cudaError_t launch_w4_t(const W4Plan& pl, int num_sms, cudaStream_t s) {
@@ -435,8 +438,7 @@ cudaError_t launch_w4_t(const W4Plan& pl, int num_sms, cudaStream_t s) {
   cudaError_t e =
       set_smem_limit_once(reinterpret_cast<const void*>(&w4_gemm_kernel<MODE, NB>), static_cast<int>(bytes));
   if (e != cudaSuccess) return e;
-  return launch_pdl(w4_gemm_kernel<MODE, NB>, dim3(num_sms), dim3(W4_THREADS), bytes, s, pl.q0, pl.q1, pl.x,
-                    pl.p);
+  return launch_pdl(w4_gemm_kernel<MODE, NB>, dim3(num_sms), dim3(W4_THREADS), bytes, s, pl.x, pl.p);
 }
 
 template <int MODE>
@@ -454,11 +456,13 @@ cudaError_t plan_w4_gemm(const W4Args& g, W4Plan* pl, const char** why) {
   *why = nullptr;
   if (g.G > MAX_G) { *why = "4-bit grouped GEMM supports at most 256 expert groups"; return cudaErrorInvalidValue; }
   if (g.K % W4_GROUP != 0) { *why = "4-bit weights need the input dimension to be a multiple of 128"; return cudaErrorInvalidValue; }
+  if (g.N % WBM != 0) { *why = "4-bit weights need d and d_ff to be multiples of 128"; return cudaErrorInvalidValue; }
+  if (((reinterpret_cast<uintptr_t>(g.Q0) | reinterpret_cast<uintptr_t>(g.mode == W4_SWIGLU ? g.Q1 : g.Q0)) & 15) != 0) {
+    *why = "4-bit codes must be 16-byte aligned";
+    return cudaErrorInvalidValue;
+  }
   pl->nb = w4_rows_per_tile(g.max_group_rows);
-  const uint64_t qrows = static_cast<uint64_t>(g.G) * g.N;
-  const uint64_t qbytes = static_cast<uint64_t>(g.K) / 2;
-  bool ok = make_map_codes(&pl->q0, g.Q0, qrows, qbytes) &&
-            make_map_codes(&pl->q1, g.mode == W4_SWIGLU ? g.Q1 : g.Q0, qrows, qbytes);
+  bool ok = true;
   if (g.mode == W4_GATE) {
     const intptr_t stride = static_cast<const uint8_t*>(g.X_lo) - static_cast<const uint8_t*>(g.X);
     if (stride <= 0 || stride % 16 != 0) { *why = "4-bit grouped GEMM: lo plane must follow the hi plane"; return cudaErrorInvalidValue; }
@@ -479,6 +483,8 @@ cudaError_t plan_w4_gemm(const W4Args& g, W4Plan* pl, const char** why) {
   p.kb_per = (p.num_kb + p.ksplit - 1) / p.ksplit;
   p.ksplit = (p.num_kb + p.kb_per - 1) / p.kb_per;  // no empty K range
   p.split_stride = g.split_stride;
+  p.Q0 = static_cast<const uint8_t*>(g.Q0);
+  p.Q1 = static_cast<const uint8_t*>(g.mode == W4_SWIGLU ? g.Q1 : g.Q0);
   p.S0 = static_cast<const __nv_bfloat16*>(g.S0);
   p.S1 = static_cast<const __nv_bfloat16*>(g.mode == W4_SWIGLU ? g.S1 : g.S0);
   p.out = g.out;

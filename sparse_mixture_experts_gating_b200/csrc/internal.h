@@ -175,13 +175,18 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType type, const void* base, uin
                  uint32_t elem_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle);
 
 // ---------------------------------------------------------------- 4-bit weights
-// Codes: uint32 [rows][K / 8], element 2j of each 8 in bits 4j.., element
-// 2j + 1 in bits 4j + 16.., code = q + 8; scales: bf16 [rows][K / W4_GROUP].
+// Codes in tiles of 128 rows x 64 elements, each tile 4 KB contiguous (row r
+// of the tile at 32 r bytes): uint32 [rows / 128][K / 64][128][8]; in a word,
+// element 2j of its 8 in bits 4j.., element 2j + 1 in bits 4j + 16.., code =
+// q + 8.  Scales: bf16 [rows / 128][K / W4_GROUP][128].  rows and K multiples
+// of 128.
 constexpr int W4_GROUP = 128;
 enum W4Mode { W4_RELU = 0, W4_SWIGLU = 1, W4_GATE = 2 };
 
 struct W4Params {
   int G, N, K, m_tiles, num_kb, ksplit, kb_per;
+  const uint8_t* Q0;                 // codes of W1 (or W2), tiled
+  const uint8_t* Q1;                 // codes of W3 (SwiGLU)
   int64_t split_stride;              // W4_GATE: elements between K-range partials of the output
   const __nv_bfloat16* S0;           // scales of W1 (or W2)
   const __nv_bfloat16* S1;           // scales of W3 (SwiGLU)
@@ -212,7 +217,7 @@ struct W4Args {
 };
 
 struct W4Plan {
-  CUtensorMap q0, q1, x;
+  CUtensorMap x;
   W4Params p;
   int mode, nb;
 };

@@ -599,7 +599,8 @@ int forward_impl(moe_handle h, int64_t T, const void* x, const float* W_r, const
       return fail(MOE_ERR_UNSUPPORTED, std::string(F + "") + (why ? why : "GEMM plan failed"));
   }
 
-  const bool tc = L.dtype == MOE_BF16 && !ew.w4;
+  const bool tc = L.dtype == MOE_BF16 && !ew.w4;  // bf16 expert products on the tensor-core grouped GEMM
+  const bool tc_router = L.dtype == MOE_BF16;     // every bf16 layer routes on the tensor cores (E <= 128)
   auto check = [&](cudaError_t e, const char* what) -> int {
     if (e == cudaSuccess) return MOE_OK;
     return fail(MOE_ERR_CUDA, std::string(F + "") + what + ": " + cudaGetErrorString(e));
@@ -616,7 +617,7 @@ int forward_impl(moe_handle h, int64_t T, const void* x, const float* W_r, const
     record(dbg, MOE_STAGE_DISPATCH, 0, s);
     record(dbg, MOE_STAGE_DISPATCH, 1, s);
   } else {
-    if (tc && L.E <= kRouterTcMaxE && r.logits_in == nullptr) {
+    if (tc_router && L.E <= kRouterTcMaxE && r.logits_in == nullptr) {
       const char* why = nullptr;
       ce = launch_router_tc(r, ws + w.wsplit, ws + w.rpart, di->num_sms, di->err, s, &why);
       if (why != nullptr) return fail(MOE_ERR_UNSUPPORTED, std::string(F + "") + why);
@@ -719,7 +720,8 @@ int moe_forward_w4(moe_handle h, int64_t T, const void* x, const float* W_r, con
 
 int moe_quantize_int4(const void* W, int64_t rows, int64_t K, uint32_t* codes, void* scales, void* stream) {
   if (rows < 0 || K < 0) return fail(MOE_ERR_INVALID_ARG, "moe_quantize_int4: rows < 0 or K < 0");
-  if (K % W4_GROUP != 0) return fail(MOE_ERR_UNSUPPORTED, "moe_quantize_int4: K must be a multiple of 128");
+  if (K % W4_GROUP != 0 || rows % 128 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_quantize_int4: rows and K must be multiples of 128");
   if (K > 2147483647LL) return fail(MOE_ERR_UNSUPPORTED, "moe_quantize_int4: K too large");
   if (rows == 0 || K == 0) {
     t_err.clear();

@@ -31,7 +31,7 @@ def _words(codes: torch.Tensor) -> np.ndarray:
 
 def test_quantizer_matches_the_oracle_bit_for_bit():
     gen = torch.Generator(device="cuda").manual_seed(17)
-    W = (torch.randn(300, 1024, device="cuda", generator=gen) * 0.02)
+    W = (torch.randn(384, 1024, device="cuda", generator=gen) * 0.02)
     W[5, 128:256] = 0.0                        # an all-zero group: scale 0, codes 8
     W[7, :128] = torch.arange(128, device="cuda") - 64.0  # integer values: many exact halves after division
     W[9, :128] *= 1e-30                        # tiny values (subnormal scale region)
@@ -39,18 +39,19 @@ def test_quantizer_matches_the_oracle_bit_for_bit():
     codes, scales = quantize_int4(W)
     status()
     q, s = M.quantize_int4(W.float().cpu().numpy())
-    np.testing.assert_array_equal(_words(codes), M.pack_int4(q))
-    np.testing.assert_array_equal(scales.float().cpu().numpy(), s)
+    np.testing.assert_array_equal(_words(codes).reshape(-1), M.pack_int4(q))
+    np.testing.assert_array_equal(scales.float().cpu().numpy().reshape(-1), M.tile_scales(s))
     assert (s.view(np.uint32) & 0x7FFFF == 0).all()  # at most 5 significant bits
 
 
 def test_quantizer_round_trip_error_is_at_most_half_a_step():
-    W = (torch.randn(64, 512, device="cuda", generator=torch.Generator(device="cuda").manual_seed(3)) * 0.05)
+    W = (torch.randn(128, 512, device="cuda", generator=torch.Generator(device="cuda").manual_seed(3)) * 0.05)
     W = W.to(torch.bfloat16)
     codes, scales = quantize_int4(W)
     status()
-    Wd = M.dequantize_int4(_words(codes), scales.float().cpu().numpy())
-    step = np.repeat(scales.float().cpu().numpy().astype(np.float64), 128, axis=1)
+    Wd = M.dequantize_int4(_words(codes), scales.float().cpu().numpy(), 128, 512)
+    s_rows = scales.float().cpu().numpy().reshape(1, 4, 128).transpose(0, 2, 1).reshape(128, 4)
+    step = np.repeat(s_rows.astype(np.float64), 128, axis=1)
     assert (np.abs(Wd - W.float().cpu().numpy()) <= 0.5 * step + 1e-30).all()
 
 
@@ -63,7 +64,8 @@ class Dequant:
 
     def __getitem__(self, e):
         if e not in self.cache:
-            self.cache[e] = M.dequantize_int4(_words(self.codes[e]), self.scales[e].float().cpu().numpy())
+            rows, K = self.codes.shape[1], self.codes.shape[2] * 8
+            self.cache[e] = M.dequantize_int4(_words(self.codes[e]), self.scales[e].float().cpu().numpy(), rows, K)
         return self.cache[e]
 
     def __len__(self):

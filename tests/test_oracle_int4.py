@@ -18,11 +18,26 @@ rng = np.random.default_rng(23)
 
 
 def test_packing_matches_the_hand_derived_word():
-    q = np.array([G["codes_k0_to_k7"] * 16], np.int64)  # one row of 128 elements
+    q = np.tile(np.array(G["codes_k0_to_k7"], np.int64), (128, 32))  # 128 rows of 256 elements
     words = M.pack_int4(q)
-    assert words.shape == (1, 16) and (words == G["word"]).all()
-    back = M.dequantize_int4(words, np.ones((1, 1)))
-    assert back[0, :8].tolist() == G["codes_k0_to_k7"]
+    assert words.shape == (128 * 256 // 8,) and (words == G["word"]).all()
+    back = M.dequantize_int4(words, np.ones(128 * 2), 128, 256)
+    assert back[0, :8].tolist() == G["codes_k0_to_k7"] and (back == q).all()
+
+
+def test_tiles_hold_128_rows_by_64_elements_row_after_row():
+    """Storage order: tile (row // 128, k // 64), then the tile's row, then the
+    word; the word of (row 129, elements 64..71) is the first word of row 1 of
+    tile (1, 1)."""
+    rows, K = 256, 256
+    q = np.full((rows, K), -8, np.int64)
+    q[129, 64:72] = G["codes_k0_to_k7"]
+    words = M.pack_int4(q)
+    nz = np.nonzero(words)[0]
+    assert nz.tolist() == [((1 * (K // 64) + 1) * 128 + 1) * 8 + 0] and words[nz[0]] == G["word"]
+    s = np.arange(rows * 2, dtype=np.float64).reshape(rows, 2)
+    st = M.tile_scales(s)
+    assert st[(1 * 2 + 1) * 128 + 1] == s[129, 1]
 
 
 def test_quantization_matches_the_hand_derived_group():
@@ -37,15 +52,15 @@ def test_quantization_matches_the_hand_derived_group():
 
 
 def test_round_trip_bound_scale_bits_and_code_range():
-    W = (rng.normal(size=(40, 512)) * np.exp(rng.uniform(-8, 4, size=(40, 1)))).astype(np.float32)
+    W = (rng.normal(size=(128, 512)) * np.exp(rng.uniform(-8, 4, size=(128, 1)))).astype(np.float32)
     W[3, 128:256] = 0
     q, s = M.quantize_int4(W)
     assert q.min() >= -7 and q.max() <= 7
     assert (s.view(np.uint32) & 0x7FFFF == 0).all()
-    amax = np.abs(W.reshape(40, 4, 128)).max(axis=2)
+    amax = np.abs(W.reshape(128, 4, 128)).max(axis=2)
     assert (s >= amax / 7).all() and (s <= amax / 7 * (1 + 2 ** -4) + 1e-45).all()
     assert s[3, 1] == 0 and (q[3, 128:256] == 0).all()
-    Wd = M.dequantize_int4(M.pack_int4(q), s)
+    Wd = M.dequantize_int4(M.pack_int4(q), M.tile_scales(s), 128, 512)
     assert (np.abs(Wd - W) <= 0.5 * np.repeat(s, 128, axis=1).astype(np.float64) + 1e-45).all()
     # every dequantized value is exact in bfloat16 (at most 8 significant bits)
     mant = (Wd.astype(np.float32).view(np.uint32) & 0xFFFF)
@@ -55,7 +70,7 @@ def test_round_trip_bound_scale_bits_and_code_range():
 
 def test_values_on_the_grid_round_trip_exactly():
     s = np.float32(0.046875)  # 1.1b x 2^-5: 2 significant bits
-    q = rng.integers(-7, 8, size=(6, 256))
+    q = rng.integers(-7, 8, size=(128, 256))
     q[:, ::128] = 7  # each group's largest magnitude is 7 s, so its scale is s again
     W = (q * s).astype(np.float32)
     q2, s2 = M.quantize_int4(W)
@@ -70,7 +85,18 @@ def _pack_natural_order(q):
     w = np.zeros((rows, K // 8), np.uint64)
     for i in range(8):
         w |= u[:, :, i] << (4 * i)
-    return w.astype(np.uint32)
+    tiles = w.reshape(rows // 128, 128, K // 64, 8).transpose(0, 2, 1, 3)
+    return np.ascontiguousarray(tiles).astype(np.uint32).reshape(-1)
+
+
+_pack = M.pack_int4
+
+
+def _pack_row_major(q):
+    """Words in plain row order instead of 128 x 64 tiles."""
+    rows, K = np.shape(q)
+    t = _pack(q).reshape(rows // 128, K // 64, 128, 8).transpose(0, 2, 1, 3)
+    return np.ascontiguousarray(t).reshape(-1)
 
 
 def _scale_rounded_to_nearest(W):
@@ -98,13 +124,15 @@ def _codes_truncated(W):
 
 
 @pytest.mark.parametrize("name,attr,fn", [("natural nibble order", "pack_int4", _pack_natural_order),
+                                          ("words in row order, not tiles", "pack_int4", _pack_row_major),
                                           ("scale rounded to nearest", "quantize_int4", _scale_rounded_to_nearest),
                                           ("codes truncated", "quantize_int4", _codes_truncated)])
 def test_planted_mistake_fails_a_pin(name, attr, fn, monkeypatch):
     monkeypatch.setattr(M, attr, fn)
     failed = 0
-    for pin in (test_packing_matches_the_hand_derived_word, test_quantization_matches_the_hand_derived_group,
-                test_round_trip_bound_scale_bits_and_code_range, test_values_on_the_grid_round_trip_exactly):
+    for pin in (test_packing_matches_the_hand_derived_word, test_tiles_hold_128_rows_by_64_elements_row_after_row,
+                test_quantization_matches_the_hand_derived_group, test_round_trip_bound_scale_bits_and_code_range,
+                test_values_on_the_grid_round_trip_exactly):
         try:
             pin()
         except AssertionError:
