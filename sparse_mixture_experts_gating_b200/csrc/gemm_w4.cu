@@ -18,10 +18,16 @@
 // reads as its A operand, while the activation tile comes from shared memory
 // through TMA.  HBM then carries the codes and scales only.
 //
-// Warp roles (704 threads, one CTA per SM):
-//   warp 0        producer: per stage the code tile(s) (one 4 KB bulk copy
-//                 each) and the activation tile [NB rows x 64] by TMA (hi and
-//                 lo planes of the hidden activation for the second projection)
+// Warp roles (736 threads, one CTA per SM):
+//   warp 0        code producer: bulk copies of KS = 4 consecutive k-blocks of
+//                 each code tile (NQ x 16 KB per stage, one contiguous copy
+//                 per weight matrix) into a ring of stages that only the
+//                 dequantizing warps release, so the HBM stream keeps about
+//                 128 KB in flight per SM, independent of the MMAs
+//   warp 22       activation producer: the [NB rows x 64] activation tile of
+//                 every k-block by TMA (hi and lo planes of the hidden
+//                 activation for the second projection) into a ring the MMAs
+//                 release
 //   warp 1        TMEM allocator; lane 0 issues the MMAs (M 128, N NB, K 16)
 //   warps 2..17   dequantize: warp w owns TMEM lanes 32 (w % 4) .. + 31 (one
 //                 weight row per lane) and quarter (w - 2) / 4 of each
@@ -48,10 +54,15 @@ constexpr int WBM = 128;                 // weight rows per tile (TMEM lanes)
 constexpr int WBK = 64;                  // K per k-block
 constexpr int Q_TILE = WBM * WBK / 2;    // bytes of codes per weight tile and k-block (4 KB)
 constexpr int MAX_A_STAGES = 8;          // TMEM A ring
-constexpr int MAX_SMEM_STAGES = 8;
+constexpr int KS = 4;                    // k-blocks per code stage
+constexpr int MAX_Q_STAGES = 8;
+constexpr int MAX_X_STAGES = 6;
+constexpr int Q_RING_BYTES = 128 * 1024;
+constexpr int X_RING_BYTES = 64 * 1024;
 constexpr int DQ_WARPS = 16;
 constexpr int EPI_WARP0 = 2 + DQ_WARPS;
-constexpr int W4_THREADS = 32 * (EPI_WARP0 + 4);
+constexpr int XPROD_WARP = EPI_WARP0 + 4;
+constexpr int W4_THREADS = 32 * (XPROD_WARP + 1);
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_G = 256;
 
@@ -72,15 +83,22 @@ struct W4Tmem {
   static_assert(A_STAGES >= 2, "tensor memory too small for the A ring");
 };
 
+// Two shared-memory rings: code stages (KS k-blocks of every weight matrix of
+// the tile) and activation stages (one k-block).
 template <int MODE, int NB>
 struct W4Stage {
-  static constexpr int BYTES = W4Geo<MODE>::NQ * Q_TILE + W4Geo<MODE>::PLANES * NB * 128;
-  static constexpr int N = (160 * 1024 / BYTES) < MAX_SMEM_STAGES ? (160 * 1024 / BYTES) : MAX_SMEM_STAGES;
+  static constexpr int Q_BYTES = W4Geo<MODE>::NQ * KS * Q_TILE;
+  static constexpr int QN = (Q_RING_BYTES / Q_BYTES) < MAX_Q_STAGES ? (Q_RING_BYTES / Q_BYTES) : MAX_Q_STAGES;
+  static constexpr int X_BYTES = W4Geo<MODE>::PLANES * NB * 128;
+  static constexpr int XN = (X_RING_BYTES / X_BYTES) < MAX_X_STAGES ? (X_RING_BYTES / X_BYTES) : MAX_X_STAGES;
+  static constexpr int BYTES = QN * Q_BYTES + XN * X_BYTES;
 };
 
 struct W4Ctl {
-  uint64_t full[MAX_SMEM_STAGES];
-  uint64_t empty[MAX_SMEM_STAGES];
+  uint64_t qfull[MAX_Q_STAGES];
+  uint64_t qempty[MAX_Q_STAGES];
+  uint64_t xfull[MAX_X_STAGES];
+  uint64_t xempty[MAX_X_STAGES];
   uint64_t afull[MAX_A_STAGES];
   uint64_t aempty[MAX_A_STAGES];
   uint64_t tfull[2];
@@ -94,7 +112,7 @@ struct W4Ctl {
 
 template <int MODE, int NB>
 constexpr size_t w4_smem_bytes() {
-  return W4Stage<MODE, NB>::N * W4Stage<MODE, NB>::BYTES + sizeof(W4Ctl) + 1024;
+  return W4Stage<MODE, NB>::BYTES + sizeof(W4Ctl) + 1024;
 }
 
 
@@ -157,19 +175,20 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   using Geo = W4Geo<MODE>;
   using St = W4Stage<MODE, NB>;
   constexpr int NQ = Geo::NQ, PLANES = Geo::PLANES;
-  constexpr int STAGES = St::N, STAGE_BYTES = St::BYTES;
-  constexpr int X_OFF = NQ * Q_TILE;
+  constexpr int QN = St::QN, XN = St::XN, Q_BYTES = St::Q_BYTES, X_BYTES = St::X_BYTES;
   constexpr int A_STAGES = W4Tmem<MODE, NB>::A_STAGES;
   constexpr uint32_t ACC0 = W4Tmem<MODE, NB>::ACC0;
   constexpr uint32_t IDESC = idesc_bf16_f32(WBM, NB);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
-  uint8_t* stages = smem_raw + pad;
-  W4Ctl* ctl = reinterpret_cast<W4Ctl*>(stages + STAGES * STAGE_BYTES);
+  uint8_t* xring = smem_raw + pad;          // activation stages first: 1024-byte aligned for the swizzle
+  uint8_t* qring = xring + XN * X_BYTES;
+  W4Ctl* ctl = reinterpret_cast<W4Ctl*>(qring + QN * Q_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
+    for (int s = 0; s < QN; ++s) { mbar_init(&ctl->qfull[s], 1); mbar_init(&ctl->qempty[s], DQ_WARPS); }
+    for (int s = 0; s < XN; ++s) { mbar_init(&ctl->xfull[s], 1); mbar_init(&ctl->xempty[s], 1); }
     for (int a = 0; a < A_STAGES; ++a) { mbar_init(&ctl->afull[a], DQ_WARPS); mbar_init(&ctl->aempty[a], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&ctl->tfull[a], 1); mbar_init(&ctl->tempty[a], 128); }
     mbar_init(&ctl->drain, 1);
@@ -195,32 +214,54 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   const uint32_t tmem_base = ctl->tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ code producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_phase = 0;
       bool ok = true;
       W4Item w;
       for (int u = blockIdx.x; ok && w4_item(ctl, p, u, w); u += gridDim.x) {
-        // the unit's first code tile: tile row (e, mt), k-block kb at + kb * Q_TILE
+        // tile row (e, mt): its k-blocks are Q_TILE apart, contiguous
         const int64_t qtile = (static_cast<int64_t>(w.e) * p.m_tiles + w.mt) * p.num_kb * Q_TILE;
-        const int xrow = ctl->offsets[w.e] + w.nt * NB;
-        for (int kb = w.kb0; kb < w.kb1; ++kb) {
-          if (!w4_wait(ctl, &ctl->empty[stage], phase ^ 1u, p)) { ok = false; break; }
-          uint8_t* st = stages + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
-          bulk_load(st, p.Q0 + qtile + static_cast<int64_t>(kb) * Q_TILE, Q_TILE, &ctl->full[stage]);
+        for (int kb = w.kb0; kb < w.kb1; kb += KS) {
+          const int nkb = min(KS, w.kb1 - kb);
+          if (!w4_wait(ctl, &ctl->qempty[stage], phase ^ 1u, p)) { ok = false; break; }
+          uint8_t* st = qring + stage * Q_BYTES;
+          const uint32_t bytes = static_cast<uint32_t>(nkb * Q_TILE);
+          mbar_arrive_expect_tx(&ctl->qfull[stage], NQ * bytes);
+          bulk_load(st, p.Q0 + qtile + static_cast<int64_t>(kb) * Q_TILE, bytes, &ctl->qfull[stage]);
           if (NQ == 2)
-            bulk_load(st + Q_TILE, p.Q1 + qtile + static_cast<int64_t>(kb) * Q_TILE, Q_TILE, &ctl->full[stage]);
-          if (PLANES == 2) tma_load_3d(st + X_OFF, &tmX, &ctl->full[stage], kb * WBK, xrow, 0);
-          else tma_load_2d(st + X_OFF, &tmX, &ctl->full[stage], kb * WBK, xrow);
+            bulk_load(st + KS * Q_TILE, p.Q1 + qtile + static_cast<int64_t>(kb) * Q_TILE, bytes, &ctl->qfull[stage]);
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == QN) { stage = 0; phase ^= 1u; }
         }
       }
-      for (int s = 0; s < STAGES; ++s)
-        if ((issued >> s) & 1u) mbar_wait(&ctl->full[s], (issued_phase >> s) & 1u, p.limit_ns);
+      for (int s = 0; s < QN; ++s)
+        if ((issued >> s) & 1u) mbar_wait(&ctl->qfull[s], (issued_phase >> s) & 1u, p.limit_ns);
+    }
+  } else if (warp == XPROD_WARP) {
+    // ------------------------------------------------------------ activation producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_phase = 0;
+      bool ok = true;
+      W4Item w;
+      for (int u = blockIdx.x; ok && w4_item(ctl, p, u, w); u += gridDim.x) {
+        const int xrow = ctl->offsets[w.e] + w.nt * NB;
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          if (!w4_wait(ctl, &ctl->xempty[stage], phase ^ 1u, p)) { ok = false; break; }
+          uint8_t* st = xring + stage * X_BYTES;
+          mbar_arrive_expect_tx(&ctl->xfull[stage], X_BYTES);
+          if (PLANES == 2) tma_load_3d(st, &tmX, &ctl->xfull[stage], kb * WBK, xrow, 0);
+          else tma_load_2d(st, &tmX, &ctl->xfull[stage], kb * WBK, xrow);
+          issued |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == XN) { stage = 0; phase ^= 1u; }
+        }
+      }
+      for (int s = 0; s < XN; ++s)
+        if ((issued >> s) & 1u) mbar_wait(&ctl->xfull[s], (issued_phase >> s) & 1u, p.limit_ns);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -234,12 +275,12 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         tc_fence_after();
         const uint32_t d0 = tmem_base + ACC0 + static_cast<uint32_t>(acc * NQ * NB);
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
-          if (!w4_wait(ctl, &ctl->full[stage], phase, p) || !w4_wait(ctl, &ctl->afull[astage], aphase, p)) {
+          if (!w4_wait(ctl, &ctl->xfull[stage], phase, p) || !w4_wait(ctl, &ctl->afull[astage], aphase, p)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sx = smem_u32(stages + stage * STAGE_BYTES + X_OFF);
+          const uint32_t sx = smem_u32(xring + stage * X_BYTES);
           const uint32_t a0 = tmem_base + static_cast<uint32_t>(astage * NQ * 32);
 #pragma unroll
           for (int kk = 0; kk < WBK / 16; ++kk) {
@@ -249,9 +290,9 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
             if (NQ == 2) umma_tmem_a(d0 + NB, a0 + 32 + kk * 8, bd, IDESC, acc_in);
             if (PLANES == 2) umma_tmem_a(d0, a0 + kk * 8, sdesc_k_sw128(sx + NB * 128 + kk * 32), IDESC, 1u);
           }
-          umma_commit(&ctl->empty[stage]);
+          umma_commit(&ctl->xempty[stage]);
           umma_commit(&ctl->aempty[astage]);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == XN) { stage = 0; phase ^= 1u; }
           if (++astage == A_STAGES) { astage = 0; aphase ^= 1u; }
         }
         if (!ok) break;
@@ -272,37 +313,42 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
     bool ok = true;
     W4Item w;
     for (int u = blockIdx.x; ok && w4_item(ctl, p, u, w); u += gridDim.x) {
-      const bool vrow = true;  // N is a multiple of 128
       // scales of tile row (e, mt): [groups][128], this lane's row r
       const int64_t sbase = (static_cast<int64_t>(w.e) * p.m_tiles + w.mt) * groups * WBM + r;
       const __nv_bfloat16* s0p = p.S0 + sbase;
       const __nv_bfloat16* s1p = p.S1 + sbase;
       // scales of this k-block's group and the next one, loaded one group ahead
       int g_cur = (w.kb0 * WBK + part * 16) / W4_GROUP;
-      __nv_bfloat16 sc0 = vrow ? s0p[g_cur * WBM] : zero, sc1 = (NQ == 2 && vrow) ? s1p[g_cur * WBM] : zero;
-      __nv_bfloat16 nx0 = (vrow && g_cur + 1 < groups) ? s0p[(g_cur + 1) * WBM] : zero;
-      __nv_bfloat16 nx1 = (NQ == 2 && vrow && g_cur + 1 < groups) ? s1p[(g_cur + 1) * WBM] : zero;
+      __nv_bfloat16 sc0 = s0p[g_cur * WBM], sc1 = NQ == 2 ? s1p[g_cur * WBM] : zero;
+      __nv_bfloat16 nx0 = g_cur + 1 < groups ? s0p[(g_cur + 1) * WBM] : zero;
+      __nv_bfloat16 nx1 = (NQ == 2 && g_cur + 1 < groups) ? s1p[(g_cur + 1) * WBM] : zero;
       for (int kb = w.kb0; kb < w.kb1; ++kb) {
+        const int j = (kb - w.kb0) % KS;  // k-block within the code stage
+        if (j == 0 && !__all_sync(0xffffffffu, w4_wait(ctl, &ctl->qfull[stage], phase, p))) { ok = false; break; }
         const int grp = (kb * WBK + part * 16) / W4_GROUP;
         if (grp != g_cur) {
           g_cur = grp;
           sc0 = nx0;
           sc1 = nx1;
-          nx0 = (vrow && grp + 1 < groups) ? s0p[(grp + 1) * WBM] : zero;
-          if (NQ == 2) nx1 = (vrow && grp + 1 < groups) ? s1p[(grp + 1) * WBM] : zero;
+          nx0 = grp + 1 < groups ? s0p[(grp + 1) * WBM] : zero;
+          if (NQ == 2) nx1 = grp + 1 < groups ? s1p[(grp + 1) * WBM] : zero;
         }
-        const bool got = __all_sync(0xffffffffu, w4_wait(ctl, &ctl->full[stage], phase, p) &&
-                                                     w4_wait(ctl, &ctl->aempty[astage], aphase ^ 1u, p));
-        if (!got) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, w4_wait(ctl, &ctl->aempty[astage], aphase ^ 1u, p))) { ok = false; break; }
         tc_fence_after();
-        const uint8_t* st = stages + stage * STAGE_BYTES;
+        const uint8_t* st = qring + stage * Q_BYTES + j * Q_TILE;
         uint32_t v[NQ][8];
 #pragma unroll
         for (int m = 0; m < NQ; ++m) {
-          const uint2 words = *reinterpret_cast<const uint2*>(st + m * Q_TILE + r * 32 + part * 8);
+          const uint2 words = *reinterpret_cast<const uint2*>(st + m * KS * Q_TILE + r * 32 + part * 8);
           const __nv_bfloat162 s2 = __bfloat162bfloat162(m == 0 ? sc0 : sc1);
           dequant_word(words.x, s2, v[m]);
           dequant_word(words.y, s2, v[m] + 4);
+        }
+        // the code stage is read once its last k-block's codes are in registers
+        if (j == KS - 1 || kb + 1 == w.kb1) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->qempty[stage]);
+          if (++stage == QN) { stage = 0; phase ^= 1u; }
         }
         // the previous k-block's stores completed: hand that A stage to the MMA
         if (held >= 0) {
@@ -316,7 +362,6 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
 #pragma unroll
         for (int m = 0; m < NQ; ++m) tmem_st8(tcol + m * 32, v[m]);
         held = astage;
-        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         if (++astage == A_STAGES) { astage = 0; aphase ^= 1u; }
       }
     }
