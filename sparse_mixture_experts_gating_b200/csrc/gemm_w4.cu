@@ -23,11 +23,13 @@
 //                 each code tile (NQ x 16 KB per stage, one contiguous copy
 //                 per weight matrix) into a ring of stages that only the
 //                 dequantizing warps release, so the HBM stream keeps about
-//                 128 KB in flight per SM, independent of the MMAs
+//                 96 KB in flight per SM, independent of the MMAs
 //   warp 22       activation producer: the [NB rows x 64] activation tile of
 //                 every k-block by TMA (hi and lo planes of the hidden
 //                 activation for the second projection) into a ring the MMAs
-//                 release
+//                 release, up to 32 stages deep: these small copies have the
+//                 same latency as the code stream, and a shallow ring of them
+//                 (6 stages) held the whole pipeline to a third of its rate
 //   warp 1        TMEM allocator; lane 0 issues the MMAs (M 128, N NB, K 16)
 //   warps 2..17   dequantize: warp w owns TMEM lanes 32 (w % 4) .. + 31 (one
 //                 weight row per lane) and quarter (w - 2) / 4 of each
@@ -56,9 +58,9 @@ constexpr int Q_TILE = WBM * WBK / 2;    // bytes of codes per weight tile and k
 constexpr int MAX_A_STAGES = 8;          // TMEM A ring
 constexpr int KS = 4;                    // k-blocks per code stage
 constexpr int MAX_Q_STAGES = 8;
-constexpr int MAX_X_STAGES = 6;
-constexpr int Q_RING_BYTES = 128 * 1024;
-constexpr int X_RING_BYTES = 64 * 1024;
+constexpr int MAX_X_STAGES = 32;
+constexpr int Q_RING_BYTES = 96 * 1024;
+constexpr int X_RING_BYTES = 96 * 1024;
 constexpr int DQ_WARPS = 16;
 constexpr int EPI_WARP0 = 2 + DQ_WARPS;
 constexpr int XPROD_WARP = EPI_WARP0 + 4;
