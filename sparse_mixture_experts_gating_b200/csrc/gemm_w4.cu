@@ -55,9 +55,8 @@ namespace {
 constexpr int WBM = 128;                 // weight rows per tile (TMEM lanes)
 constexpr int WBK = 64;                  // K per k-block
 constexpr int Q_TILE = WBM * WBK / 2;    // bytes of codes per weight tile and k-block (4 KB)
-constexpr int KA = 2;                    // k-blocks per step: one A stage, one activation stage, one handshake
-constexpr int MAX_A_STAGES = 8;          // TMEM A ring (steps)
-constexpr int KS = 4;                    // k-blocks per code stage (a multiple of KA)
+constexpr int MAX_A_STAGES = 8;          // TMEM A ring
+constexpr int KS = 4;                    // k-blocks per code stage
 constexpr int MAX_Q_STAGES = 8;
 constexpr int MAX_X_STAGES = 32;
 constexpr int Q_RING_BYTES = 96 * 1024;
@@ -76,13 +75,13 @@ struct W4Geo {
 };
 
 // TMEM: two accumulators of NQ x NB columns, the rest (up to 8 stages of
-// KA x NQ x 32 columns) for the dequantized A ring.
+// NQ x 32 columns) for the dequantized A ring.
 template <int MODE, int NB>
 struct W4Tmem {
   static constexpr int NQ = W4Geo<MODE>::NQ;
-  static constexpr int FREE = (static_cast<int>(TMEM_COLS) - 2 * NQ * NB) / (KA * NQ * 32);
+  static constexpr int FREE = (static_cast<int>(TMEM_COLS) - 2 * NQ * NB) / (NQ * 32);
   static constexpr int A_STAGES = FREE < MAX_A_STAGES ? FREE : MAX_A_STAGES;
-  static constexpr uint32_t ACC0 = A_STAGES * KA * NQ * 32;  // first accumulator column
+  static constexpr uint32_t ACC0 = A_STAGES * NQ * 32;  // first accumulator column
   static_assert(A_STAGES >= 2, "tensor memory too small for the A ring");
 };
 
@@ -92,7 +91,7 @@ template <int MODE, int NB>
 struct W4Stage {
   static constexpr int Q_BYTES = W4Geo<MODE>::NQ * KS * Q_TILE;
   static constexpr int QN = (Q_RING_BYTES / Q_BYTES) < MAX_Q_STAGES ? (Q_RING_BYTES / Q_BYTES) : MAX_Q_STAGES;
-  static constexpr int X_BYTES = KA * W4Geo<MODE>::PLANES * NB * 128;  // one step's activation tiles
+  static constexpr int X_BYTES = W4Geo<MODE>::PLANES * NB * 128;
   static constexpr int XN = (X_RING_BYTES / X_BYTES) < MAX_X_STAGES ? (X_RING_BYTES / X_BYTES) : MAX_X_STAGES;
   static constexpr int BYTES = QN * Q_BYTES + XN * X_BYTES;
 };
@@ -252,16 +251,12 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       W4Item w;
       for (int u = blockIdx.x; ok && w4_item(ctl, p, u, w); u += gridDim.x) {
         const int xrow = ctl->offsets[w.e] + w.nt * NB;
-        for (int kb = w.kb0; kb < w.kb1; kb += KA) {
-          const int nk = min(KA, w.kb1 - kb);
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!w4_wait(ctl, &ctl->xempty[stage], phase ^ 1u, p)) { ok = false; break; }
           uint8_t* st = xring + stage * X_BYTES;
-          mbar_arrive_expect_tx(&ctl->xfull[stage], nk * (X_BYTES / KA));
-          for (int t = 0; t < nk; ++t) {
-            uint8_t* dst = st + t * (X_BYTES / KA);
-            if (PLANES == 2) tma_load_3d(dst, &tmX, &ctl->xfull[stage], (kb + t) * WBK, xrow, 0);
-            else tma_load_2d(dst, &tmX, &ctl->xfull[stage], (kb + t) * WBK, xrow);
-          }
+          mbar_arrive_expect_tx(&ctl->xfull[stage], X_BYTES);
+          if (PLANES == 2) tma_load_3d(st, &tmX, &ctl->xfull[stage], kb * WBK, xrow, 0);
+          else tma_load_2d(st, &tmX, &ctl->xfull[stage], kb * WBK, xrow);
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == XN) { stage = 0; phase ^= 1u; }
@@ -281,26 +276,21 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         if (!w4_wait(ctl, &ctl->tempty[acc], acc_phase ^ 1u, p)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + ACC0 + static_cast<uint32_t>(acc * NQ * NB);
-        for (int kb = w.kb0; kb < w.kb1; kb += KA) {
-          const int nk = min(KA, w.kb1 - kb);
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!w4_wait(ctl, &ctl->xfull[stage], phase, p) || !w4_wait(ctl, &ctl->afull[astage], aphase, p)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sx0 = smem_u32(xring + stage * X_BYTES);
-          const uint32_t a00 = tmem_base + static_cast<uint32_t>(astage * KA * NQ * 32);
-          for (int t = 0; t < nk; ++t) {
-            const uint32_t sx = sx0 + t * (X_BYTES / KA);
+          const uint32_t sx = smem_u32(xring + stage * X_BYTES);
+          const uint32_t a0 = tmem_base + static_cast<uint32_t>(astage * NQ * 32);
 #pragma unroll
-            for (int kk = 0; kk < WBK / 16; ++kk) {
-              const uint32_t acc_in = (kb + t != w.kb0 || kk != 0) ? 1u : 0u;
-              const uint64_t bd = sdesc_k_sw128(sx + kk * 32);
-              umma_tmem_a(d0, a00 + t * 32 + kk * 8, bd, IDESC, acc_in);
-              if (NQ == 2) umma_tmem_a(d0 + NB, a00 + (KA + t) * 32 + kk * 8, bd, IDESC, acc_in);
-              if (PLANES == 2)
-                umma_tmem_a(d0, a00 + t * 32 + kk * 8, sdesc_k_sw128(sx + NB * 128 + kk * 32), IDESC, 1u);
-            }
+          for (int kk = 0; kk < WBK / 16; ++kk) {
+            const uint32_t acc_in = (kb != w.kb0 || kk != 0) ? 1u : 0u;
+            const uint64_t bd = sdesc_k_sw128(sx + kk * 32);
+            umma_tmem_a(d0, a0 + kk * 8, bd, IDESC, acc_in);
+            if (NQ == 2) umma_tmem_a(d0 + NB, a0 + 32 + kk * 8, bd, IDESC, acc_in);
+            if (PLANES == 2) umma_tmem_a(d0, a0 + kk * 8, sdesc_k_sw128(sx + NB * 128 + kk * 32), IDESC, 1u);
           }
           umma_commit(&ctl->xempty[stage]);
           umma_commit(&ctl->aempty[astage]);
@@ -334,42 +324,35 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       __nv_bfloat16 sc0 = s0p[g_cur * WBM], sc1 = NQ == 2 ? s1p[g_cur * WBM] : zero;
       __nv_bfloat16 nx0 = g_cur + 1 < groups ? s0p[(g_cur + 1) * WBM] : zero;
       __nv_bfloat16 nx1 = (NQ == 2 && g_cur + 1 < groups) ? s1p[(g_cur + 1) * WBM] : zero;
-      for (int kb0s = w.kb0; kb0s < w.kb1; kb0s += KA) {  // one step: KA k-blocks, one A stage
-        const int nk = min(KA, w.kb1 - kb0s);
-        if (!__all_sync(0xffffffffu, w4_wait(ctl, &ctl->aempty[astage], aphase ^ 1u, p))) { ok = false; break; }
-        uint32_t v[KA][NQ][8];
-#pragma unroll
-        for (int t = 0; t < KA; ++t) {
-          if (t >= nk) break;
-          const int kb = kb0s + t;
-          const int j = (kb - w.kb0) % KS;  // k-block within the code stage
-          if (j == 0 && !__all_sync(0xffffffffu, w4_wait(ctl, &ctl->qfull[stage], phase, p))) { ok = false; break; }
-          const int grp = (kb * WBK + part * 16) / W4_GROUP;
-          if (grp != g_cur) {
-            g_cur = grp;
-            sc0 = nx0;
-            sc1 = nx1;
-            nx0 = grp + 1 < groups ? s0p[(grp + 1) * WBM] : zero;
-            if (NQ == 2) nx1 = grp + 1 < groups ? s1p[(grp + 1) * WBM] : zero;
-          }
-          const uint8_t* st = qring + stage * Q_BYTES + j * Q_TILE;
-#pragma unroll
-          for (int m = 0; m < NQ; ++m) {
-            const uint2 words = *reinterpret_cast<const uint2*>(st + m * KS * Q_TILE + r * 32 + part * 8);
-            const __nv_bfloat162 s2 = __bfloat162bfloat162(m == 0 ? sc0 : sc1);
-            dequant_word(words.x, s2, v[t][m]);
-            dequant_word(words.y, s2, v[t][m] + 4);
-          }
-          // the code stage is read once its last k-block's codes are in registers
-          if (j == KS - 1 || kb + 1 == w.kb1) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->qempty[stage]);
-            if (++stage == QN) { stage = 0; phase ^= 1u; }
-          }
+      for (int kb = w.kb0; kb < w.kb1; ++kb) {
+        const int j = (kb - w.kb0) % KS;  // k-block within the code stage
+        if (j == 0 && !__all_sync(0xffffffffu, w4_wait(ctl, &ctl->qfull[stage], phase, p))) { ok = false; break; }
+        const int grp = (kb * WBK + part * 16) / W4_GROUP;
+        if (grp != g_cur) {
+          g_cur = grp;
+          sc0 = nx0;
+          sc1 = nx1;
+          nx0 = grp + 1 < groups ? s0p[(grp + 1) * WBM] : zero;
+          if (NQ == 2) nx1 = grp + 1 < groups ? s1p[(grp + 1) * WBM] : zero;
         }
-        if (!ok) break;
+        if (!__all_sync(0xffffffffu, w4_wait(ctl, &ctl->aempty[astage], aphase ^ 1u, p))) { ok = false; break; }
         tc_fence_after();
-        // the previous step's stores completed: hand that A stage to the MMA
+        const uint8_t* st = qring + stage * Q_BYTES + j * Q_TILE;
+        uint32_t v[NQ][8];
+#pragma unroll
+        for (int m = 0; m < NQ; ++m) {
+          const uint2 words = *reinterpret_cast<const uint2*>(st + m * KS * Q_TILE + r * 32 + part * 8);
+          const __nv_bfloat162 s2 = __bfloat162bfloat162(m == 0 ? sc0 : sc1);
+          dequant_word(words.x, s2, v[m]);
+          dequant_word(words.y, s2, v[m] + 4);
+        }
+        // the code stage is read once its last k-block's codes are in registers
+        if (j == KS - 1 || kb + 1 == w.kb1) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->qempty[stage]);
+          if (++stage == QN) { stage = 0; phase ^= 1u; }
+        }
+        // the previous k-block's stores completed: hand that A stage to the MMA
         if (held >= 0) {
           tmem_st_wait();
           tc_fence_before();
@@ -377,13 +360,9 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
           if (lane == 0) mbar_arrive(&ctl->afull[held]);
         }
         const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                              static_cast<uint32_t>(astage * KA * NQ * 32 + part * 8);
+                              static_cast<uint32_t>(astage * NQ * 32 + part * 8);
 #pragma unroll
-        for (int t = 0; t < KA; ++t) {
-          if (t >= nk) break;
-#pragma unroll
-          for (int m = 0; m < NQ; ++m) tmem_st8(tcol + (m * KA + t) * 32, v[t][m]);
-        }
+        for (int m = 0; m < NQ; ++m) tmem_st8(tcol + m * 32, v[m]);
         held = astage;
         if (++astage == A_STAGES) { astage = 0; aphase ^= 1u; }
       }
