@@ -50,6 +50,18 @@ DECODE_MIN_CALLS = 100  # decode layers report the p50 latency over at least thi
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # the nominal B200 figures the layer's targets are quoted against (dense bf16, HBM3e)
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2200.0}
+# Batches of at most this many tokens run the 4-bit layer on the few-row
+# products (w4_small_kernel; the first projection's stage also holds
+# w4_hidden_kernel), larger ones on the tcgen05 grouped GEMM (w4_gemm_kernel).
+W4_SMALL_MAX_T = 16
+
+
+def w4_kernel_name(T, stage):
+    if T > W4_SMALL_MAX_T:
+        return "w4_gemm_kernel"
+    return "w4_small_kernel + w4_hidden_kernel" if stage == "gemm1" else "w4_small_kernel"
+
+
 STAGE_KERNEL = {"router": "router_kernel", "scan": "scan_kernel", "dispatch": "dispatch_kernel",
                 "gemm1": "grouped_gemm_kernel", "gemm2": "grouped_gemm_kernel", "combine": "combine_kernel"}
 
@@ -443,7 +455,7 @@ def measure_workload(args, w, dev, world, rank, local, K, warmup, cpu=True, weig
     work = layer_work(w, kept, "int4" if w4 else "dense")
     peaks, peak_src = load_peaks()
     roof = kernel_roofline(work[dom]["flops"], work[dom]["bytes"], dom_ms / 1e3, peaks)
-    roof["kernel"] = f"{'w4_gemm_kernel' if w4 else STAGE_KERNEL[dom]} ({dom})"
+    roof["kernel"] = f"{w4_kernel_name(w.T, dom) if w4 else STAGE_KERNEL[dom]} ({dom})"
     roof["peak_source"] = f"{peak_src} ({'bf16_tflops' if roof['bound'] == 'tensor' else 'hbm_gbs'}, burst)"
     roof["nominal_peak"] = NOMINAL_PEAKS["bf16_tflops" if roof["bound"] == "tensor" else "hbm_gbs"]
     tr = profiled_traffic(dom, w.name)

@@ -161,7 +161,10 @@ __device__ __forceinline__ void umma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, ui
 // Eight codes of one 32-bit word (element 2j in bits 4j.., element 2j+1 in
 // bits 4j+16.., codes offset by 8) -> four bf16 pairs (code - 8) * s, exact.
 __device__ __forceinline__ void dequant_word(uint32_t w, __nv_bfloat162 s2, uint32_t* out) {
-  const __nv_bfloat162 bias = __floats2bfloat162_rn(136.f, 136.f);
+  __nv_bfloat162_raw braw;  // 136 as bits: no conversion instruction
+  braw.x = 0x4308;
+  braw.y = 0x4308;
+  const __nv_bfloat162 bias(braw);
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t t = ((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u;  // bf16 pair 128 + code

@@ -225,6 +225,50 @@ struct W4Plan {
 int w4_rows_per_tile(int64_t max_group_rows);
 cudaError_t plan_w4_gemm(const W4Args& g, W4Plan* plan, const char** why);
 cudaError_t launch_w4_gemm(const W4Plan& plan, int num_sms, cudaStream_t s);
+
+// Few-row 4-bit products (register-fed warp MMAs) for expert groups of at most
+// kW4SmallRows rows; they write fp32 partial rows per K range.
+constexpr int kW4SmallRows = 16;
+
+struct W4SmallParams {
+  int G, N, K, m_tiles, row_blocks, num_g, gp, ksplit;  // gp: scale groups (128 elements) per K range
+  int two_mats;                       // SwiGLU: W1 and W3 rows of one m-tile per unit
+  int rows_cap;                       // activation rows of one group at most
+  int stage_bytes, nstage;            // pipeline stages (codes, scales and activation columns)
+  const uint8_t* Q0;
+  const uint8_t* Q1;
+  const __nv_bfloat16* S0;
+  const __nv_bfloat16* S1;
+  const __nv_bfloat16* X;     // activation rows [x_rows][K] (sorted x, or the hidden hi plane)
+  const __nv_bfloat16* X_lo;  // second projection: the hidden lo plane
+  float* out;                 // partials [ksplit][split_stride] of W1 x, or of gate * W2 h
+  float* out3;                // partials of W3 x (SwiGLU)
+  int64_t split_stride;
+  const int32_t* offsets;
+  const float* row_gate;      // second projection only
+  unsigned int* err;
+  uint64_t limit_ns;
+};
+
+struct W4SmallPlan {
+  W4SmallParams p;
+  int planes, nt;
+};
+
+struct W4SmallSplit {
+  int row_blocks, gp, ksplit;
+};
+
+// K ranges of a few-row product (mode W4Mode; x_rows bounds the groups with
+// rows; rows_cap the rows of one group) spread over `ctas` CTAs.
+W4SmallSplit w4_small_split(int mode, int G, int64_t x_rows, int64_t rows_cap, int N, int K, int ctas);
+cudaError_t plan_w4_small(const W4Args& g, int ctas, W4SmallPlan* plan, const char** why);
+cudaError_t launch_w4_small(const W4SmallPlan& plan, int num_sms, cudaStream_t s);
+// Hidden bf16 hi + lo planes [rows][N] from the first projection's partials
+// (rows = *total_rows <= max_rows, read on the device).
+cudaError_t launch_w4_hidden(int act, const float* P1, const float* P3, int ksplit, int64_t split_stride,
+                             const int32_t* total_rows, int64_t max_rows, int N, void* H, void* H_lo, int num_sms,
+                             cudaStream_t s);
 cudaError_t launch_quantize_int4(const void* W, int64_t rows, int K, void* codes, void* scales, cudaStream_t s);
 
 // Raise a kernel's dynamic shared memory limit, once per (kernel, device, size).

@@ -147,10 +147,39 @@ struct Layout {
   bool need_yp;
   bool split;  // hidden activation as a hi + lo bf16 pair
   bool f16;    // hidden activation (and the second projection's operands) in fp16
+  bool small;  // 4-bit weights, at most kW4SmallMaxT tokens: the few-row products
   int ksplit;
+  int ks1;     // few-row products: K ranges of the first projection
   size_t idx, gate, dest, row_token, row_gate, part_hist, part_cnt1, part_psum, part_lse2, blockoff, counts,
-      offsets, mprefix, scal, wsplit, rpart, spart, Xp, Hp, Hp_lo, Yp, W2h, total;
+      offsets, mprefix, scal, wsplit, rpart, spart, Xp, Hp, Hp_lo, Yp, W2h, P, total;
 };
+
+// Batches of 4-bit layers up to this many tokens (so no expert group above
+// kW4SmallRows rows) take the few-row products.
+constexpr int64_t kW4SmallMaxT = kW4SmallRows;
+
+int64_t s_max_of(const moe_layer& L, int64_t T) {
+  const int64_t cap = capacity_of(L, T);
+  int64_t s = T * L.k;
+  if (cap >= 0) s = std::min<int64_t>(s, static_cast<int64_t>(L.E) * cap);
+  return s + static_cast<int64_t>(L.n_shared) * T;
+}
+
+// The K ranges of both few-row products for a batch of T tokens.
+struct SmallSplits {
+  W4SmallSplit g1, g2;
+  int64_t s_max;
+};
+
+SmallSplits small_splits_of(const moe_layer& L, int64_t T) {
+  SmallSplits r;
+  r.s_max = s_max_of(L, T);
+  const int G = L.E + L.n_shared;
+  const int mode1 = L.act == MOE_ACT_SWIGLU ? W4_SWIGLU : W4_RELU;
+  r.g1 = w4_small_split(mode1, G, r.s_max, T, L.d_ff, L.d, kSplitTargetCtas);
+  r.g2 = w4_small_split(W4_GATE, G, r.s_max, T, L.d, L.d_ff, kSplitTargetCtas);
+  return r;
+}
 
 // w4: the layout of moe_forward_w4 (4-bit weights: hidden as a hi + lo pair,
 // fp32 rows for the combine, no fp16 image of W2).
@@ -214,9 +243,30 @@ Layout make_layout(const moe_layer& L, int64_t T, bool w4 = false) {
     for (int64_t s = groups + 1; s < w.s_max && s <= groups + int64_t{2 * kSplitTargetCtas} * 64; ++s)
       yp_rows = std::max<int64_t>(yp_rows, yp_rows_of(L, s, w4));
   }
-  w.Yp = take(yp_rows > 0 ? sizeof(float) * static_cast<size_t>(yp_rows) * L.d : 0);
   // fp16 image of W2 (every expert, shared ones included) for the fp16 mode
   w.W2h = take(w.f16 ? sizeof(uint16_t) * static_cast<size_t>(L.E + L.n_shared) * L.d * L.d_ff : 0);
+  // Few-row products: fp32 partials of the first projection [nq][ks1][s_max][d_ff],
+  // and the second projection's partials in Yp; sized for every batch up to
+  // kW4SmallMaxT tokens, so sizes stay monotone in T.
+  w.small = w4 && T <= kW4SmallMaxT;
+  w.ks1 = 1;
+  size_t p_bytes = 0;
+  if (w4) {
+    const size_t nq = L.act == MOE_ACT_SWIGLU ? 2 : 1;
+    for (int64_t t = 1; t <= std::min<int64_t>(T, kW4SmallMaxT); ++t) {
+      const SmallSplits sp = small_splits_of(L, t);
+      p_bytes = std::max(p_bytes, nq * sizeof(float) * static_cast<size_t>(sp.g1.ksplit) *
+                                      static_cast<size_t>(sp.s_max) * L.d_ff);
+      yp_rows = std::max<int64_t>(yp_rows, static_cast<int64_t>(sp.g2.ksplit) * sp.s_max);
+    }
+    if (w.small) {
+      const SmallSplits sp = small_splits_of(L, T);
+      w.ks1 = sp.g1.ksplit;
+      w.ksplit = sp.g2.ksplit;
+    }
+  }
+  w.Yp = take(yp_rows > 0 ? sizeof(float) * static_cast<size_t>(yp_rows) * L.d : 0);
+  w.P = take(p_bytes);
   w.total = o;
   return w;
 }
@@ -456,7 +506,7 @@ int forward_impl(moe_handle h, int64_t T, const void* x, const float* W_r, const
       return fail(MOE_ERR_UNSUPPORTED, F + "4-bit weights need d and d_ff to be multiples of 128");
     const uintptr_t sal = reinterpret_cast<uintptr_t>(ew.S1) | reinterpret_cast<uintptr_t>(ew.S2) |
                           reinterpret_cast<uintptr_t>(ew.S3);
-    if ((sal & 1) != 0) return fail(MOE_ERR_INVALID_ARG, F + "scales must be 2-byte aligned");
+    if ((sal & 15) != 0) return fail(MOE_ERR_INVALID_ARG, F + "scales must be 16-byte aligned");
   }
   const Layout w = make_layout(L, T, ew.w4);
   if (workspace == nullptr || workspace_bytes < w.total)
@@ -557,6 +607,7 @@ int forward_impl(moe_handle h, int64_t T, const void* x, const float* W_r, const
   // Host-side preparation of both GEMM launches happens before the first launch.
   TcGemmPlan plan1, plan2;
   W4Plan wplan1, wplan2;
+  W4SmallPlan splan1, splan2;
   if (ew.w4) {
     W4Args a1;
     memset(&a1, 0, sizeof(a1));
@@ -591,8 +642,21 @@ int forward_impl(moe_handle h, int64_t T, const void* x, const float* W_r, const
     a2.ksplit = w.ksplit;
     a2.split_stride = static_cast<int64_t>(w.s_max) * L.d;
     const char* why = nullptr;
-    if (plan_w4_gemm(a1, &wplan1, &why) != cudaSuccess || plan_w4_gemm(a2, &wplan2, &why) != cudaSuccess)
+    if (w.small) {
+      // few-row products: fp32 partials of W1 x (and W3 x), then the hidden
+      // planes, then gated partials of W2 h in Yp
+      const size_t p1 = static_cast<size_t>(w.ks1) * static_cast<size_t>(w.s_max) * L.d_ff;
+      a1.out = ws + w.P;
+      a1.out_lo = reinterpret_cast<float*>(ws + w.P) + p1;
+      a1.split_stride = static_cast<int64_t>(w.s_max) * L.d_ff;
+      if (plan_w4_small(a1, kSplitTargetCtas, &splan1, &why) != cudaSuccess ||
+          plan_w4_small(a2, kSplitTargetCtas, &splan2, &why) != cudaSuccess)
+        return fail(MOE_ERR_UNSUPPORTED, F + (why ? why : "4-bit few-row plan failed"));
+      if (splan1.p.ksplit != w.ks1 || splan2.p.ksplit != w.ksplit)
+        return fail(MOE_ERR_UNSUPPORTED, F + "4-bit few-row plan disagrees with the workspace layout");
+    } else if (plan_w4_gemm(a1, &wplan1, &why) != cudaSuccess || plan_w4_gemm(a2, &wplan2, &why) != cudaSuccess) {
       return fail(MOE_ERR_UNSUPPORTED, F + (why ? why : "4-bit GEMM plan failed"));
+    }
   } else if (L.dtype == MOE_BF16) {
     const char* why = nullptr;
     if (plan_gemm_tc(g1, &plan1, &why) != cudaSuccess || plan_gemm_tc(g2, &plan2, &why) != cudaSuccess)
@@ -643,8 +707,17 @@ int forward_impl(moe_handle h, int64_t T, const void* x, const float* W_r, const
   }
 
   record(dbg, MOE_STAGE_GEMM1, 0, s);
-  ce = ew.w4 ? launch_w4_gemm(wplan1, di->num_sms, s)
-             : tc ? launch_gemm_tc(plan1, di->num_sms, s) : launch_gemm_simt(g1, w.s_max, s);
+  if (w.small) {
+    ce = launch_w4_small(splan1, di->num_sms, s);
+    if ((rc = check(ce, "gemm1")) != MOE_OK) return rc;
+    const float* P1 = reinterpret_cast<const float*>(ws + w.P);
+    ce = launch_w4_hidden(L.act, P1, P1 + static_cast<size_t>(w.ks1) * static_cast<size_t>(w.s_max) * L.d_ff, w.ks1,
+                          static_cast<int64_t>(w.s_max) * L.d_ff, r.offsets + (L.E + L.n_shared), w.s_max, L.d_ff,
+                          ws + w.Hp, ws + w.Hp_lo, di->num_sms, s);
+  } else {
+    ce = ew.w4 ? launch_w4_gemm(wplan1, di->num_sms, s)
+               : tc ? launch_gemm_tc(plan1, di->num_sms, s) : launch_gemm_simt(g1, w.s_max, s);
+  }
   if ((rc = check(ce, "gemm1")) != MOE_OK) return rc;
   if (w.f16) {  // the fp16 image of W2, made while the first projection runs
     ce = launch_convert_f16(W2, ws + w.W2h, static_cast<int64_t>(L.E + L.n_shared) * L.d * L.d_ff, di->err,
@@ -653,8 +726,10 @@ int forward_impl(moe_handle h, int64_t T, const void* x, const float* W_r, const
   }
   record(dbg, MOE_STAGE_GEMM1, 1, s);
   record(dbg, MOE_STAGE_GEMM2, 0, s);
-  ce = ew.w4 ? launch_w4_gemm(wplan2, di->num_sms, s)
-             : tc ? launch_gemm_tc(plan2, di->num_sms, s) : launch_gemm_simt(g2, w.s_max, s);
+  ce = w.small ? launch_w4_small(splan2, di->num_sms, s)
+       : ew.w4  ? launch_w4_gemm(wplan2, di->num_sms, s)
+       : tc     ? launch_gemm_tc(plan2, di->num_sms, s)
+                : launch_gemm_simt(g2, w.s_max, s);
   if ((rc = check(ce, "gemm2")) != MOE_OK) return rc;
   record(dbg, MOE_STAGE_GEMM2, 1, s);
   if (w.need_yp) {

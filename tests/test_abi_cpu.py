@@ -156,6 +156,23 @@ def test_workspace_sizing_is_defined_for_every_batch_size(L):
         L.moe_destroy(h)
 
 
+def test_4bit_workspace_never_shrinks_as_T_grows(L):
+    """moe_workspace_bytes_w4 across the switch from the few-row products
+    (T <= 16, fp32 partials of the first projection) to the grouped GEMM."""
+    shapes = [(8, 2, 4096, 14336, 1, 1, 0.0, 1), (64, 1, 768, 3072, 0, 0, 1.25, 1),
+              (16, 4, 1024, 2048, 1, 1, 0.0, 1), (2, 2, 384, 640, 0, 0, 0.0, 1)]
+    for i, args in enumerate(shapes):
+        rc, h = _create(L, *args)
+        assert rc == 0
+        assert L.moe_set_shared_experts(h, i % 2) == 0
+        prev = 0
+        for T in list(range(0, 300)) + [511, 512, 513, 4096]:
+            n = L.moe_workspace_bytes_w4(h, T)
+            assert n >= prev and n % 256 == 0, (args, T, n)
+            prev = n
+        L.moe_destroy(h)
+
+
 def test_automatic_hidden_mode_adds_the_fp16_weight_image_at_1024_rows_per_expert(L):
     """The automatic mode holds the hidden activation in fp16 (and reserves the
     fp16 image of W2) from 1024 rows per expert group on: for 8 experts, top-2,

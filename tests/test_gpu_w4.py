@@ -6,6 +6,8 @@ quantize_int4 and pack_int4, the same rule in float32) bit for bit.  The
 4-bit forward must equal the layer computed by the oracle with the
 dequantized weights (exact in bf16): routing bit-exact on dyadic router
 inputs, y within the bf16 bar (max|dy| <= 1e-2 RMS, mean relative 2e-3).
+Batches of at most 16 tokens run the few-row products (warp MMAs fed from
+registers), larger ones the tcgen05 grouped GEMM; the cases cover both.
 """
 import zlib
 
@@ -124,6 +126,15 @@ CASES = [
     ("w4_shared", 40, 256, 4, 2, 256, S, RN, 1.0, None, 1),
     # groups of more than 64 rows: several n-tiles per expert
     ("w4_large_groups", 300, 256, 4, 2, 384, S, RN, 0.0, "normal", 0),
+    # few-row products: 12 rows per group (two n-tiles of the first projection,
+    # three of the second), odd m-tile counts (a unit with one slot), ReLU
+    ("w4_small_relu_odd_tiles", 12, 384, 2, 2, 640, R, RN, 0.0, "normal", 0),
+    # few-row products with a shared expert (a group of every token)
+    ("w4_small_shared", 5, 256, 8, 2, 384, S, RN, 0.0, None, 1),
+    # few-row products with capacity drops (at most 8 rows per expert)
+    ("w4_small_capacity", 16, 512, 4, 2, 256, S, RN, 1.0, None, 0),
+    # few-row products over a long K range (d_ff 2048: 16 scale groups)
+    ("w4_small_long_k", 3, 1024, 16, 4, 2048, S, RN, 0.0, "normal", 0),
 ]
 
 
