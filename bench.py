@@ -53,7 +53,7 @@ NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2200.0}
 # Batches of at most this many tokens run the 4-bit layer on the few-row
 # products (w4_small_kernel; the first projection's stage also holds
 # w4_hidden_kernel), larger ones on the tcgen05 grouped GEMM (w4_gemm_kernel).
-W4_SMALL_MAX_T = 16
+W4_SMALL_MAX_T = 64
 
 
 def w4_kernel_name(T, stage):

@@ -239,7 +239,7 @@ MOE_API int moe_forward(moe_handle h, int64_t T, const void* x, const float* W_r
  * with the dequantized weights.  The expert products run on the tensor
  * cores with the weights dequantized on the fly (HBM carries the codes and
  * scales only); the hidden activation is held as a hi + lo bf16 pair.
- * Batches of T <= 16 tokens take warp-level MMAs fed from registers, larger
+ * Batches of T <= 64 tokens take warp-level MMAs fed from registers, larger
  * ones the tcgen05 grouped GEMM.  Codes and scales must be 16-byte aligned.
  * The workspace is moe_workspace_bytes_w4(h, T) bytes (256-byte aligned).
  * Arguments, results and errors as moe_forward; W3_codes / W3_scales are

@@ -1,8 +1,8 @@
-// Expert products with 4-bit weights for batches of at most 16 tokens
+// Expert products with 4-bit weights for batches of at most 64 tokens
 // ("Mixture of experts", rayaq.ca, section "Total versus active parameters":
 // decoding a few tokens is bound by reading the active experts' weights).
 //
-// With at most 16 activation rows per expert the products are a handful of
+// With a few activation rows per expert the products are a handful of
 // matrix-vector products.  The tcgen05 path (gemm_w4.cu) cycles every
 // dequantized k-block through tensor memory and waits for the MMA's commit
 // before reusing it; at these sizes that round trip, not HBM, sets its pace.
@@ -78,15 +78,19 @@ struct SmCtl {
   uint64_t full[MAX_STAGE];
   uint64_t empty[MAX_STAGE];
   volatile int abort;
-  int nprefix[MAX_G + 1];  // prefix over groups of 1 for a group with rows
+  int nprefix[MAX_G + 1];  // prefix over groups of their row chunks
   int offsets[MAX_G + 1];
   uint4 zero[XROW / 16];   // a zero activation row: B fragments of rows past the group's
 };
 
 struct SmItem {
   int e, b, ks, g0, g1;  // group, row block, K range, scale groups [g0, g1)
+  int row0, rows;        // the unit's activation rows (one chunk of the group's)
 };
 
+// Unit u -> (group e, row block b, chunk c of at most rows_cap rows, K range
+// ks), K ranges innermost, then chunks (the chunks of one code tile run side
+// by side, so the later ones find its codes in L2).
 __device__ __forceinline__ bool sm_item(const SmCtl* c, const W4SmallParams& p, int u, SmItem& w) {
   const int units = c->nprefix[p.G] * p.row_blocks * p.ksplit;
   if (u >= units) return false;
@@ -98,7 +102,12 @@ __device__ __forceinline__ bool sm_item(const SmCtl* c, const W4SmallParams& p, 
     if (c->nprefix[mid] * p.row_blocks <= tile) lo = mid; else hi = mid;
   }
   w.e = lo;  // the largest lo with nprefix[lo] <= tile / row_blocks: a group with rows
-  w.b = tile - c->nprefix[lo] * p.row_blocks;
+  const int local = tile - c->nprefix[lo] * p.row_blocks;
+  const int chunks = c->nprefix[lo + 1] - c->nprefix[lo];
+  w.b = local / chunks;
+  const int ch = local - w.b * chunks;
+  w.row0 = c->offsets[lo] + ch * p.rows_cap;
+  w.rows = min(p.rows_cap, c->offsets[lo + 1] - w.row0);
   w.g0 = w.ks * p.gp;
   w.g1 = min(p.num_g, w.g0 + p.gp);
   return true;
@@ -180,7 +189,15 @@ __device__ __forceinline__ void a_frag(uint32_t w, uint32_t v, uint32_t (&a)[4])
 // + 16).  Every load of the stage is issued first; the body is straight-line.
 template <int NT, int NTA, int NG>
 __device__ __forceinline__ void stage_mma(uint32_t q, const uint32_t (&xa)[NT], uint32_t sadr, float (&acc)[NT][4]) {
-  constexpr int PAR = NTA >= 4 ? 1 : 2;  // accumulator chains per n-tile (one when registers are short)
+  if constexpr (NG == 2 && NTA > 2) {  // registers are short: one scale group at a time
+    uint32_t xa2[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) xa2[j] = xa[j] + W4_GROUP * 2;
+    stage_mma<NT, NTA, 1>(q, xa, sadr, acc);
+    stage_mma<NT, NTA, 1>(q + GROUP_CODES, xa2, sadr + GROUP_SCALES, acc);
+    return;
+  }
+  constexpr int PAR = NTA >= 3 ? 1 : 2;  // accumulator chains per n-tile (one when registers are short)
   uint2 cw[NG][2][2];
   float sc[NG][2];
 #pragma unroll
@@ -277,7 +294,7 @@ __global__ void __launch_bounds__(SM_THREADS, 1) w4_small_kernel(const W4SmallPa
     for (int g = 0; g < p.G; ++g) {
       const int o0 = p.offsets[g], o1 = p.offsets[g + 1];
       ctl->offsets[g] = o0;
-      ctl->nprefix[g + 1] = ctl->nprefix[g] + (o1 > o0 ? 1 : 0);
+      ctl->nprefix[g + 1] = ctl->nprefix[g] + (o1 - o0 + p.rows_cap - 1) / p.rows_cap;
     }
     ctl->offsets[p.G] = p.offsets[p.G];
   }
@@ -291,12 +308,7 @@ __global__ void __launch_bounds__(SM_THREADS, 1) w4_small_kernel(const W4SmallPa
       bool ok = true;
       SmItem w;
       for (int u = blockIdx.x; ok && sm_item(ctl, p, u, w); u += gridDim.x) {
-        const int row0 = ctl->offsets[w.e];
-        int rows = ctl->offsets[w.e + 1] - row0;
-        if (rows > p.rows_cap) {  // the host sizes rows_cap from the largest possible group
-          record_error(p.err, DEV_ERR_RANGE);
-          rows = p.rows_cap;
-        }
+        const int row0 = w.row0, rows = w.rows;
         const int mt0 = slot_mtile(p, w.b, 0), mt1 = slot_mtile(p, w.b, 1);
         const bool has1 = p.two_mats || mt1 < p.m_tiles;
         const int64_t t0 = static_cast<int64_t>(w.e) * p.m_tiles + mt0;
@@ -350,8 +362,7 @@ __global__ void __launch_bounds__(SM_THREADS, 1) w4_small_kernel(const W4SmallPa
   SmItem w;
   bool ok = true;
   for (int u = blockIdx.x; ok && sm_item(ctl, p, u, w); u += gridDim.x) {
-    const int row0 = ctl->offsets[w.e];
-    const int rows = min(ctl->offsets[w.e + 1] - row0, p.rows_cap);
+    const int row0 = w.row0, rows = w.rows;
     const int nt = (rows + RPT - 1) / RPT;
     const int mt = slot_mtile(p, w.b, slot);
     const bool active = p.two_mats || mt < p.m_tiles;
@@ -463,14 +474,23 @@ int small_groups_per_range(int64_t tiles, int num_g, int64_t rows, int ctas) {
 
 }  // namespace
 
-W4SmallSplit w4_small_split(int mode, int G, int64_t x_rows, int64_t rows_cap, int N, int K, int ctas) {
+// Activation rows of one unit: four n-tiles (32 rows of the first
+// projection, 16 of the second's two planes); a larger group is cut into
+// chunks of that many rows, each its own unit.
+int small_chunk_rows(int mode) { return mode == W4_GATE ? 16 : 32; }
+
+W4SmallSplit w4_small_split(int mode, int G, int64_t x_rows, int64_t max_group_rows, int N, int K, int ctas) {
   W4SmallSplit sp;
   const int m_tiles = N / SB;
   sp.row_blocks = mode == W4_SWIGLU ? m_tiles : (m_tiles + 1) / 2;
   const int num_g = K / W4_GROUP;
-  const int64_t rc = rows_cap < 1 ? 1 : rows_cap;
-  const int64_t groups = x_rows < G ? x_rows : G;  // groups with rows
-  sp.gp = small_groups_per_range(groups * sp.row_blocks, num_g, rc, ctas);
+  int64_t rc = max_group_rows < small_chunk_rows(mode) ? max_group_rows : small_chunk_rows(mode);
+  if (rc < 1) rc = 1;
+  sp.rows_cap = static_cast<int>(rc);
+  // (group, chunk) pairs: at most min(G, x_rows) groups with rows, ceil(rows / rc) chunks each
+  const int64_t groups = x_rows < G ? x_rows : G;
+  const int64_t chunks = (x_rows + groups * (rc - 1)) / rc;
+  sp.gp = small_groups_per_range(chunks * sp.row_blocks, num_g, rc, ctas);
   sp.ksplit = (num_g + sp.gp - 1) / sp.gp;
   return sp;
 }
@@ -480,10 +500,6 @@ cudaError_t plan_w4_small(const W4Args& g, int ctas, W4SmallPlan* pl, const char
   if (g.G > MAX_G) { *why = "4-bit products support at most 256 expert groups"; return cudaErrorInvalidValue; }
   if (g.K % W4_GROUP != 0 || g.N % SB != 0) {
     *why = "4-bit weights need d and d_ff to be multiples of 128";
-    return cudaErrorInvalidValue;
-  }
-  if (g.max_group_rows > kW4SmallRows) {
-    *why = "4-bit few-row products: expert groups may exceed 16 rows";
     return cudaErrorInvalidValue;
   }
   const bool two = g.mode == W4_SWIGLU;
@@ -507,7 +523,7 @@ cudaError_t plan_w4_small(const W4Args& g, int ctas, W4SmallPlan* pl, const char
   p.gp = sp.gp;
   p.ksplit = sp.ksplit;
   p.two_mats = two ? 1 : 0;
-  p.rows_cap = static_cast<int>(g.max_group_rows < 1 ? 1 : g.max_group_rows);
+  p.rows_cap = sp.rows_cap;
   const int planes = g.mode == W4_GATE ? 2 : 1;
   p.stage_bytes = X_OFF + planes * p.rows_cap * XROW;
   p.nstage = static_cast<int>((SMEM_BUDGET - sizeof(SmCtl)) / static_cast<size_t>(p.stage_bytes));
@@ -537,7 +553,8 @@ cudaError_t plan_w4_small(const W4Args& g, int ctas, W4SmallPlan* pl, const char
 cudaError_t launch_w4_small(const W4SmallPlan& pl, int num_sms, cudaStream_t s) {
   if (pl.planes == 1) {
     if (pl.nt <= 1) return launch_small_t<1, 1>(pl.p, num_sms, s);
-    return launch_small_t<1, 2>(pl.p, num_sms, s);
+    if (pl.nt <= 2) return launch_small_t<1, 2>(pl.p, num_sms, s);
+    return launch_small_t<1, 4>(pl.p, num_sms, s);
   }
   if (pl.nt <= 1) return launch_small_t<2, 1>(pl.p, num_sms, s);
   if (pl.nt <= 2) return launch_small_t<2, 2>(pl.p, num_sms, s);

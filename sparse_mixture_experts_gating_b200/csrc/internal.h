@@ -226,9 +226,10 @@ int w4_rows_per_tile(int64_t max_group_rows);
 cudaError_t plan_w4_gemm(const W4Args& g, W4Plan* plan, const char** why);
 cudaError_t launch_w4_gemm(const W4Plan& plan, int num_sms, cudaStream_t s);
 
-// Few-row 4-bit products (register-fed warp MMAs) for expert groups of at most
-// kW4SmallRows rows; they write fp32 partial rows per K range.
-constexpr int kW4SmallRows = 16;
+// Few-row 4-bit products (register-fed warp MMAs) for batches of at most
+// kW4SmallMaxT tokens (groups of more than 32 / 16 rows run as several
+// units); they write fp32 partial rows per K range.
+constexpr int kW4SmallMaxT = 64;
 
 struct W4SmallParams {
   int G, N, K, m_tiles, row_blocks, num_g, gp, ksplit;  // gp: scale groups (128 elements) per K range
@@ -256,12 +257,13 @@ struct W4SmallPlan {
 };
 
 struct W4SmallSplit {
-  int row_blocks, gp, ksplit;
+  int row_blocks, gp, ksplit, rows_cap;
 };
 
-// K ranges of a few-row product (mode W4Mode; x_rows bounds the groups with
-// rows; rows_cap the rows of one group) spread over `ctas` CTAs.
-W4SmallSplit w4_small_split(int mode, int G, int64_t x_rows, int64_t rows_cap, int N, int K, int ctas);
+// Units and K ranges of a few-row product (mode W4Mode; x_rows activation
+// rows in all; max_group_rows the rows of the largest group) spread over
+// `ctas` CTAs.
+W4SmallSplit w4_small_split(int mode, int G, int64_t x_rows, int64_t max_group_rows, int N, int K, int ctas);
 cudaError_t plan_w4_small(const W4Args& g, int ctas, W4SmallPlan* plan, const char** why);
 cudaError_t launch_w4_small(const W4SmallPlan& plan, int num_sms, cudaStream_t s);
 // Hidden bf16 hi + lo planes [rows][N] from the first projection's partials

@@ -154,9 +154,7 @@ struct Layout {
       offsets, mprefix, scal, wsplit, rpart, spart, Xp, Hp, Hp_lo, Yp, W2h, P, total;
 };
 
-// Batches of 4-bit layers up to this many tokens (so no expert group above
-// kW4SmallRows rows) take the few-row products.
-constexpr int64_t kW4SmallMaxT = kW4SmallRows;
+// Batches of 4-bit layers up to kW4SmallMaxT tokens take the few-row products.
 
 int64_t s_max_of(const moe_layer& L, int64_t T) {
   const int64_t cap = capacity_of(L, T);

@@ -6,8 +6,9 @@ quantize_int4 and pack_int4, the same rule in float32) bit for bit.  The
 4-bit forward must equal the layer computed by the oracle with the
 dequantized weights (exact in bf16): routing bit-exact on dyadic router
 inputs, y within the bf16 bar (max|dy| <= 1e-2 RMS, mean relative 2e-3).
-Batches of at most 16 tokens run the few-row products (warp MMAs fed from
-registers), larger ones the tcgen05 grouped GEMM; the cases cover both.
+Batches of at most 64 tokens run the few-row products (warp MMAs fed from
+registers; groups above 32 / 16 rows in several chunks), larger ones the
+tcgen05 grouped GEMM; the cases cover both.
 """
 import zlib
 
@@ -135,6 +136,12 @@ CASES = [
     ("w4_small_capacity", 16, 512, 4, 2, 256, S, RN, 1.0, None, 0),
     # few-row products over a long K range (d_ff 2048: 16 scale groups)
     ("w4_small_long_k", 3, 1024, 16, 4, 2048, S, RN, 0.0, "normal", 0),
+    # few-row products with groups of 64 rows (two chunks of the first
+    # projection, four of the second) and a shared expert of 64 rows
+    ("w4_small_chunks", 64, 256, 2, 2, 384, S, RN, 0.0, None, 1),
+    # the tcgen05 grouped GEMM just above the few-row range, ReLU, shared expert
+    ("w4_tc_t65_relu_shared", 65, 256, 4, 2, 256, R, RN, 0.0, "normal", 1),
+    ("w4_tc_t128", 128, 384, 8, 2, 640, S, RN, 1.0, None, 0),
 ]
 
 
