@@ -76,7 +76,9 @@ template <int EP>
 struct RtGeo {
   static constexpr int B_PLANE = EP * BK * 2;  // one plane box: EP rows x 128 B
   static constexpr int STAGE_BYTES = A_BYTES + 3 * B_PLANE;
-  static constexpr int STAGES = (190 * 1024 / STAGE_BYTES) < MAX_STAGES ? (190 * 1024 / STAGE_BYTES) : MAX_STAGES;
+  // as many stages as fit beside the control block (E_pad 128: three of 64 KB)
+  static constexpr int FIT = static_cast<int>((227 * 1024 - 1024 - sizeof(RtCtl)) / STAGE_BYTES);
+  static constexpr int STAGES = FIT < MAX_STAGES ? FIT : MAX_STAGES;
   static constexpr uint32_t TMEM_COLS = (2 * EP) <= 32 ? 32 : (2 * EP) <= 64 ? 64 : (2 * EP) <= 128 ? 128
                                         : (2 * EP) <= 256 ? 256 : 512;
   static constexpr size_t SMEM = STAGES * STAGE_BYTES + sizeof(RtCtl) + 1024;
@@ -383,14 +385,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       } else {
 #pragma unroll 1
-        for (int c0 = 0; c0 < H; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(tq + c_lo + c0, r);
+        for (int c0 = 0; c0 < H; c0 += 32) {  // 32 columns per wait
+          uint32_t r[2][16];
+          tmem_ld16(tq + c_lo + c0, r[0]);
+          tmem_ld16(tq + c_lo + c0 + 16, r[1]);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < 32; ++i) {
             const int e = c_lo + c0 + i;
-            if (e < E) consider(logit(__uint_as_float(r[i]), e), e);
+            if (e < E) consider(logit(__uint_as_float(r[i / 16][i % 16]), e), e);
           }
         }
       }
@@ -442,14 +445,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       } else {
 #pragma unroll 1
-        for (int c0 = 0; c0 < H; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(tq + c_lo + c0, r);
+        for (int c0 = 0; c0 < H; c0 += 32) {  // 32 columns per wait
+          uint32_t r[2][16];
+          tmem_ld16(tq + c_lo + c0, r[0]);
+          tmem_ld16(tq + c_lo + c0 + 16, r[1]);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < 32; ++i) {
             const int e = c_lo + c0 + i;
-            s4[i & 3] += e < E ? expf(logit(__uint_as_float(r[i]), e) - m) : 0.f;
+            s4[i & 3] += e < E ? expf(logit(__uint_as_float(r[i / 16][i % 16]), e) - m) : 0.f;
           }
         }
       }
