@@ -135,9 +135,11 @@ def source_sha(*rel):
     return h.hexdigest()
 
 
-def profiled_traffic(stage, workload):
-    """dram bytes per launch from the committed ncu summary, if the kernel is unchanged since."""
-    p = os.path.join(ROOT, "profiles", f"{stage}_{workload}.txt")
+def profiled_traffic(stage, workload, weights="dense"):
+    """dram bytes per launch from the committed ncu summary, if the kernel is unchanged since.
+    Summaries of the 4-bit kernels carry the suffix _int4."""
+    suffix = "_int4" if weights == "int4" else ""
+    p = os.path.join(ROOT, "profiles", f"{stage}_{workload}{suffix}.txt")
     if not os.path.exists(p):
         return None
     vals = {}
@@ -458,7 +460,7 @@ def measure_workload(args, w, dev, world, rank, local, K, warmup, cpu=True, weig
     roof["kernel"] = f"{w4_kernel_name(w.T, dom) if w4 else STAGE_KERNEL[dom]} ({dom})"
     roof["peak_source"] = f"{peak_src} ({'bf16_tflops' if roof['bound'] == 'tensor' else 'hbm_gbs'}, burst)"
     roof["nominal_peak"] = NOMINAL_PEAKS["bf16_tflops" if roof["bound"] == "tensor" else "hbm_gbs"]
-    tr = profiled_traffic(dom, w.name)
+    tr = profiled_traffic(dom, w.name, "int4" if w4 else "dense")
     roof["traffic"] = tr
     gemm_bytes = work[dom]["bytes"]
     roof["traffic_ratio"] = None if tr is None else round(tr / gemm_bytes, 3)

@@ -122,5 +122,11 @@ def test_profiled_traffic_is_reported_only_while_its_sources_are_unchanged(tmp_p
     prof.write_text(f"dram_bytes_per_launch: 1234\nsource_files: kernel.cu\nsource_sha256: {sha}\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.profiled_traffic("gemm2", "someload") == 1234.0
+    # the 4-bit line of the same workload reads its own summary only
+    assert bench.profiled_traffic("gemm2", "someload", "int4") is None
+    (tmp_path / "profiles" / "gemm2_someload_int4.txt").write_text(
+        f"dram_bytes_per_launch: 99\nsource_files: kernel.cu\nsource_sha256: {sha}\n")
+    assert bench.profiled_traffic("gemm2", "someload", "int4") == 99.0
     src.write_text("// kernel source, changed\n")
     assert bench.profiled_traffic("gemm2", "someload") is None
+    assert bench.profiled_traffic("gemm2", "someload", "int4") is None
