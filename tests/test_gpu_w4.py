@@ -142,6 +142,10 @@ CASES = [
     # the tcgen05 grouped GEMM just above the few-row range, ReLU, shared expert
     ("w4_tc_t65_relu_shared", 65, 256, 4, 2, 256, R, RN, 0.0, "normal", 1),
     ("w4_tc_t128", 128, 384, 8, 2, 640, S, RN, 1.0, None, 0),
+    # few-row products over many groups (64 experts, top-4: up to 64 groups with rows)
+    ("w4_small_many_experts", 32, 256, 64, 4, 256, S, RN, 0.0, "zipf", 0),
+    # few-row products with capacity drops and a shared expert, Switch gate
+    ("w4_small_drops_shared", 48, 384, 8, 1, 384, R, SW, 0.5, "normal", 1),
 ]
 
 
@@ -182,6 +186,21 @@ def test_w4_full_size_decode(name):
     rows = sample_rows(w, None, n=16)
     o = _oracle_w4(w, inp, qw, rows=rows, logits=o_route["logits"])
     assert_y_close(w, g, o["y"], rows=rows)
+
+
+def test_w4_empty_batch():
+    """T = 0: no launch of the expert products; zeroed counts and losses."""
+    w = _w(("w4_empty", 0, 256, 8, 2, 256, S, RN, 0.0, None, 0))
+    inp = make_inputs(Workload("w4_empty_src", T=1, d=256, E=8, k=2, d_ff=256, act=S, gate=RN, capacity_factor=0.0,
+                               dtype=DTYPE_BF16, dyadic=True, seed=3), device="cuda")
+    qw = _quantized(inp)
+    layer = layer_for(w)
+    x = inp["x"][:0]
+    y, counts, dropped, aux, z = layer.forward_w4(x, inp["W_r"], inp["b_r"], qw["W1"], qw["W3"], qw["W2"])
+    status()
+    assert y.shape == (0, 256)
+    assert int(counts.sum().item()) == 0 and int(dropped.item()) == 0
+    assert float(aux.item()) == 0.0 and float(z.item()) == 0.0
 
 
 def test_w4_rejects_dimensions_off_the_group_size():
