@@ -11,10 +11,11 @@
 //
 // One CTA per 128-token tile (persistent over tiles): warp 0 issues TMA (x box
 // 128 x 64, three plane boxes E_pad x 64), warp 1 issues the MMAs (M 128,
-// N E_pad, K 16; 4 per plane per k-block), warps 2..5 run the epilogue with one
-// token per thread (TMEM lane = token): bias, max, one-pass top-k (ties to the
-// lower expert index), log-sum-exp, gates, and the per-32-token partial counts
-// and sums that the scan kernel reduces (each epilogue warp owns one 32-token
+// N E_pad, K 16; 4 per plane per k-block), and 4 NP epilogue warps take each
+// token (TMEM lane) with NP threads, one per part of the experts (NP = 2, or 4
+// for E_pad 128): bias, max, one-pass top-k (ties to the lower expert index),
+// log-sum-exp, gates, and the per-32-token partial counts and sums that the
+// scan kernel reduces (the warps of one TMEM lane quarter own one 32-token
 // router block, the same partition as the CUDA-core router).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -30,7 +31,14 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int NUM_THREADS = 320;  // producer, MMA, 8 epilogue warps
+// Epilogue threads per token (expert parts) and block size: two parts of up
+// to 32 experts; for E_pad 128, four parts of 32, so that each thread keeps its
+// logits in registers and the top-k and exponential chains stay short.
+template <int EP>
+struct RtShape {
+  static constexpr int NP = EP >= 128 ? 4 : 2;
+  static constexpr int THREADS = 64 + 128 * NP;  // producer, MMA, 4 NP epilogue warps
+};
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int MAX_STAGES = 8;  // small router tiles: a deep ring hides the TMA round trip
 
@@ -53,6 +61,7 @@ struct RtParams {
   uint64_t limit_ns;
 };
 
+template <int NP, int K>
 struct RtCtl {
   uint64_t full[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
@@ -64,24 +73,28 @@ struct RtCtl {
   int last;  // this CTA finished the last K range of the tile
   int hist[4][kRouterTcMaxE];
   int cnt1[4][kRouterTcMaxE];
-  float pstage[8][32][17];  // per epilogue warp: 32 tokens x 16 experts of probabilities
-  float xm[4][2][32];       // per lane quarter and half: partial max of each token
-  float xs[4][2][32];       // partial exp sums
-  float xtv[4][8][32];      // half 1's top-k list (values, indices)
-  int xte[4][8][32];
+  // per epilogue warp: 32 tokens x SW experts of probabilities (SW 16, or 4
+  // with four parts, where the smaller block lets a third 64 KB stage fit)
+  static constexpr int SW = NP == 4 ? 4 : 16;
+  float pstage[4 * NP][32][SW + 1];
+  float xm[4][NP][32];           // per lane quarter and part: partial max of each token
+  float xs[4][NP][32];           // partial exp sums
+  float xtv[4][NP - 1][K][32];   // parts 1.. : their top-k lists (values, indices)
+  int xte[4][NP - 1][K][32];
   float bias[kRouterTcMaxE];
 };
 
-template <int EP>
+template <int EP, int K>
 struct RtGeo {
   static constexpr int B_PLANE = EP * BK * 2;  // one plane box: EP rows x 128 B
   static constexpr int STAGE_BYTES = A_BYTES + 3 * B_PLANE;
   // as many stages as fit beside the control block (E_pad 128: three of 64 KB)
-  static constexpr int FIT = static_cast<int>((227 * 1024 - 1024 - sizeof(RtCtl)) / STAGE_BYTES);
+  using Ctl = RtCtl<RtShape<EP>::NP, K>;
+  static constexpr int FIT = static_cast<int>((227 * 1024 - 1024 - sizeof(Ctl)) / STAGE_BYTES);
   static constexpr int STAGES = FIT < MAX_STAGES ? FIT : MAX_STAGES;
   static constexpr uint32_t TMEM_COLS = (2 * EP) <= 32 ? 32 : (2 * EP) <= 64 ? 64 : (2 * EP) <= 128 ? 128
                                         : (2 * EP) <= 256 ? 256 : 512;
-  static constexpr size_t SMEM = STAGES * STAGE_BYTES + sizeof(RtCtl) + 1024;
+  static constexpr size_t SMEM = STAGES * STAGE_BYTES + sizeof(Ctl) + 1024;
 };
 
 __device__ __forceinline__ float warp_sum_f(float v) {
@@ -114,21 +127,24 @@ __global__ void __launch_bounds__(256) split_router_kernel(const float* __restri
 // K (= top-k) is a template parameter so the running k-best list is indexed
 // statically and lives in registers.
 template <int EP, int K>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(RtShape<EP>::THREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const RtParams p) {
-  using G = RtGeo<EP>;
+  using G = RtGeo<EP, K>;
+  using RtCtlT = typename G::Ctl;
+  constexpr int NP = RtShape<EP>::NP;
+  constexpr int NUM_THREADS = RtShape<EP>::THREADS;
   constexpr int STAGES = G::STAGES;
   constexpr uint32_t IDESC = idesc_bf16_f32(BM, EP);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* stages = smem_raw + pad;
-  RtCtl* ctl = reinterpret_cast<RtCtl*>(stages + STAGES * G::STAGE_BYTES);
+  RtCtlT* ctl = reinterpret_cast<RtCtlT*>(stages + STAGES * G::STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&ctl->tfull[a], 1); mbar_init(&ctl->tempty[a], 256); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&ctl->tfull[a], 1); mbar_init(&ctl->tempty[a], 128 * NP); }
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     fence_mbarrier_init();
@@ -218,19 +234,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait(&ctl->drain, 0, p.limit_ns);
     }
   } else {  // ---------------------------------------------------------- epilogue
-    // Eight warps, two per TMEM lane quarter q (= 32-token router block of the
-    // tile).  Warp half hf takes expert columns [c_lo, c_hi): the pair splits
-    // the experts and exchanges, per token, the partial max, the partial top-k
-    // list (half 1 -> half 0) and the partial exp sums through shared memory;
-    // the lower-expert half goes first in every merge and sum, so ties and
+    // 4 NP warps, NP per TMEM lane quarter q (= 32-token router block of the
+    // tile).  Warp part hf takes expert columns [c_lo, c_lo + H): the parts
+    // split the experts and exchange, per token, the partial max, the partial
+    // top-k lists (parts 1.. -> part 0) and the partial exp sums through shared
+    // memory; lower-expert parts go first in every merge and sum, so ties and
     // summation order are fixed.
-    const int wi = warp - 2;       // 0..7
+    const int wi = warp - 2;       // 0 .. 4 NP - 1
     const int q = warp & 3;        // TMEM lane quarter
-    const int hf = wi >> 2;        // 0: lower experts, 1: upper experts
-    constexpr int H = EP / 2 < 16 ? 16 : EP / 2;  // columns per half (EP = 16: half 1 has none)
+    const int hf = wi >> 2;        // expert part: 0 = lowest experts
+    constexpr int H = EP / NP < 16 ? 16 : EP / NP;  // columns per part (EP = 16: part 1 has none)
     const int c_lo = hf * H;
     const bool has_cols = c_lo < EP;
-    const int pair_bar = 2 + q;    // named barrier of the warp pair (64 threads)
+    const int pair_bar = 2 + q;    // named barrier of the quarter's NP warps
     int acc = 0;
     uint32_t acc_phase = 0;
     const int E = p.E;
@@ -264,9 +280,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         __threadfence();
-        named_barrier(1, 256);  // all 128 rows of this range are written
+        named_barrier(1, 128 * NP);  // all 128 rows of this range are written
         if (threadIdx.x == 64) ctl->last = (atomicAdd(p.tickets + tile, 1) == p.ksplit - 1) ? 1 : 0;
-        named_barrier(1, 256);
+        named_barrier(1, 128 * NP);
         if (!ctl->last) {
           tc_fence_before();
           mbar_arrive(&ctl->tempty[acc]);
@@ -397,20 +413,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      // 3. exchange: both halves' max; half 1's list to half 0, which merges
-      // (half 0's experts have the lower indices, so it wins equal values)
+      // 3. exchange: every part's max; the lists of parts 1.. to part 0, which
+      // merges them in part order (lower parts hold the lower expert indices,
+      // so the earlier list wins equal values)
       ctl->xm[q][hf][lane] = m;
-      if (hf == 1) {
+      if (hf > 0) {
 #pragma unroll
-        for (int j = 0; j < K; ++j) { ctl->xtv[q][j][lane] = tv[j]; ctl->xte[q][j][lane] = te[j]; }
+        for (int j = 0; j < K; ++j) { ctl->xtv[q][hf - 1][j][lane] = tv[j]; ctl->xte[q][hf - 1][j][lane] = te[j]; }
       }
-      named_barrier(pair_bar, 64);
-      m = fmaxf(ctl->xm[q][0][lane], ctl->xm[q][1][lane]);
-      if (hf == 0) {
+      named_barrier(pair_bar, 32 * NP);
+      m = ctl->xm[q][0][lane];
+#pragma unroll
+      for (int pp = 1; pp < NP; ++pp) m = fmaxf(m, ctl->xm[q][pp][lane]);
+#pragma unroll
+      for (int pp = 1; pp < NP; ++pp) {
+        if (hf != 0) break;
         float bv[K];
         int be[K];
 #pragma unroll
-        for (int j = 0; j < K; ++j) { bv[j] = ctl->xtv[q][j][lane]; be[j] = ctl->xte[q][j][lane]; }
+        for (int j = 0; j < K; ++j) { bv[j] = ctl->xtv[q][pp - 1][j][lane]; be[j] = ctl->xte[q][pp - 1][j][lane]; }
         float mv[K];
         int me[K];
         int ia = 0, ib = 0;
@@ -433,8 +454,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int j = 0; j < K; ++j) { tv[j] = mv[j]; te[j] = me[j]; }
       }
-      // 4. s = sum_e exp(h - m): four partial sums per half in a fixed order,
-      // then half 0 + half 1 (registers: each exponential once, kept in h)
+      // 4. s = sum_e exp(h - m): four partial sums per part in a fixed order,
+      // then the parts in order (registers: each exponential once, kept in h)
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
       if constexpr (REG) {
 #pragma unroll
@@ -458,20 +479,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       ctl->xs[q][hf][lane] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      named_barrier(pair_bar, 64);
-      const float s = ctl->xs[q][0][lane] + ctl->xs[q][1][lane];
+      named_barrier(pair_bar, 32 * NP);
+      float s = ctl->xs[q][0][lane];
+#pragma unroll
+      for (int pp = 1; pp < NP; ++pp) s += ctl->xs[q][pp][lane];
       const float inv_s = 1.f / s;
       const float lse = m + logf(s);
-      // 5. per-expert probability sums of this 32-token block for this half's
-      // experts: 32 tokens x 16 experts through shared memory, lane j < 16
-      // sums column j over the tokens in order (fixed order: deterministic)
+      // 5. per-expert probability sums of this 32-token block for this part's
+      // experts: 32 tokens x SW experts at a time through shared memory, lane
+      // j < SW sums column j over the tokens in order (fixed order: deterministic)
       float* stg = &ctl->pstage[wi][0][0];
 #pragma unroll
       for (int c0 = 0; c0 < H; c0 += 16) {
+        float pv[16];
         if constexpr (REG) {
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            stg[lane * 17 + i] = (valid && has_cols && c_lo + c0 + i < E) ? h[(c0 + i) & (H - 1)] * inv_s : 0.f;
+            pv[i] = (valid && has_cols && c_lo + c0 + i < E) ? h[(c0 + i) & (H - 1)] * inv_s : 0.f;
         } else {
           uint32_t r[16];
           tmem_ld16(tq + c_lo + c0, r);
@@ -479,29 +503,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int e = c_lo + c0 + i;
-            stg[lane * 17 + i] = (valid && e < E) ? expf(logit(__uint_as_float(r[i]), e) - m) * inv_s : 0.f;
+            pv[i] = (valid && e < E) ? expf(logit(__uint_as_float(r[i]), e) - m) * inv_s : 0.f;
           }
         }
-        __syncwarp();
-        if (lane < 16 && has_cols && c_lo + c0 + lane < E && blk_valid) {
-          float a0 = 0.f, a1 = 0.f;
+        constexpr int SW = RtCtlT::SW;
 #pragma unroll
-          for (int t = 0; t < 32; t += 2) {
-            a0 += stg[t * 17 + lane];
-            a1 += stg[(t + 1) * 17 + lane];
+        for (int hh = 0; hh < 16 / SW; ++hh) {
+#pragma unroll
+          for (int i = 0; i < SW; ++i) stg[lane * (SW + 1) + i] = pv[hh * SW + i];
+          __syncwarp();
+          const int e = c_lo + c0 + hh * SW + lane;
+          if (lane < SW && has_cols && e < E && blk_valid) {
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int t = 0; t < 32; t += 2) {
+              a0 += stg[t * (SW + 1) + lane];
+              a1 += stg[(t + 1) * (SW + 1) + lane];
+            }
+            p.part_psum[e * p.nblk + blk] = a0 + a1;
           }
-          p.part_psum[(c_lo + c0 + lane) * p.nblk + blk] = a0 + a1;
+          __syncwarp();
         }
-        __syncwarp();
       }
       if constexpr (!REG) {
         tc_fence_before();
         mbar_arrive(&ctl->tempty[acc]);  // accumulator consumed
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
-      if (hf == 1) continue;
+      if (hf != 0) continue;  // part 0 alone writes the outputs
 
-      // 6. (half 0) gates, outputs and block counts
+      // 6. (part 0) gates, outputs and block counts
       if (valid) {
         float den = 0.f;
         if (p.gate_mode != 0) {
@@ -545,7 +576,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 template <int EP, int K>
 cudaError_t launch_ep(const RoutingArgs& a, void* wsplit, void* partials, int num_sms, unsigned int* err,
                       cudaStream_t s, const char** why) {
-  using G = RtGeo<EP>;
+  using G = RtGeo<EP, K>;
   static_assert(G::STAGES >= 2, "router stages");
   CUtensorMap mx, mw;
   if (!make_map_bf16(&mx, a.x, static_cast<uint64_t>(a.T), static_cast<uint64_t>(a.d), BM) ||
@@ -591,7 +622,7 @@ cudaError_t launch_ep(const RoutingArgs& a, void* wsplit, void* partials, int nu
   if (e != cudaSuccess) return e;
   const int units = p.n_tiles * p.ksplit;
   const int grid = units < num_sms ? units : num_sms;
-  return launch_pdl(router_tc_kernel<EP, K>, dim3(grid), dim3(NUM_THREADS), G::SMEM, s, mx, mw, p);
+  return launch_pdl(router_tc_kernel<EP, K>, dim3(grid), dim3(RtShape<EP>::THREADS), G::SMEM, s, mx, mw, p);
 }
 
 template <int EP>
