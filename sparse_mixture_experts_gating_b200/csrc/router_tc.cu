@@ -73,10 +73,6 @@ struct RtCtl {
   int last;  // this CTA finished the last K range of the tile
   int hist[4][kRouterTcMaxE];
   int cnt1[4][kRouterTcMaxE];
-  // per epilogue warp: 32 tokens x SW experts of probabilities (SW 16, or 4
-  // with four parts, where the smaller block lets a third 64 KB stage fit)
-  static constexpr int SW = NP == 4 ? 4 : 16;
-  float pstage[4 * NP][32][SW + 1];
   float xm[4][NP][32];           // per lane quarter and part: partial max of each token
   float xs[4][NP][32];           // partial exp sums
   float xtv[4][NP - 1][K][32];   // parts 1.. : their top-k lists (values, indices)
@@ -97,6 +93,33 @@ struct RtGeo {
   static constexpr size_t SMEM = STAGES * STAGE_BYTES + sizeof(Ctl) + 1024;
 };
 
+// Sums of 16 columns over the 32 lanes of a warp: step b (offsets 16, 8, 4,
+// 2) keeps the half of the columns selected by lane bit b and adds the other
+// lane's copy of it, so after four steps lane l holds its 16-lane partial of
+// column l >> 1; the last step (offset 1) completes it.  Returns column
+// (lane >> 1)'s sum.
+__device__ __forceinline__ float column_sums16(const float (&v)[16], int lane) {
+  float a[8], b[4], c[2];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool up = (lane & 16) != 0;
+    a[i] = (up ? v[i + 8] : v[i]) + __shfl_xor_sync(0xffffffffu, up ? v[i] : v[i + 8], 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool up = (lane & 8) != 0;
+    b[i] = (up ? a[i + 4] : a[i]) + __shfl_xor_sync(0xffffffffu, up ? a[i] : a[i + 4], 8);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool up = (lane & 4) != 0;
+    c[i] = (up ? b[i + 2] : b[i]) + __shfl_xor_sync(0xffffffffu, up ? b[i] : b[i + 2], 4);
+  }
+  const bool up = (lane & 2) != 0;
+  const float d = (up ? c[1] : c[0]) + __shfl_xor_sync(0xffffffffu, up ? c[0] : c[1], 2);
+  return d + __shfl_xor_sync(0xffffffffu, d, 1);
+}
+
 __device__ __forceinline__ float warp_sum_f(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -108,6 +131,7 @@ __global__ void __launch_bounds__(256) split_router_kernel(const float* __restri
                                                            __nv_bfloat16* __restrict__ planes, int* tickets,
                                                            int n_tickets, int* scan_ticket) {
   const int64_t n = static_cast<int64_t>(EP) * d;
+  pdl_trigger();  // the router may be scheduled at once (it waits for this grid before reading)
   if (blockIdx.x == 0 && threadIdx.x == 0) *scan_ticket = 0;
   if (tickets != nullptr)
     for (int i = blockIdx.x * 256 + threadIdx.x; i < n_tickets; i += gridDim.x * 256) tickets[i] = 0;
@@ -486,9 +510,9 @@ __global__ void __launch_bounds__(RtShape<EP>::THREADS, 1)
       const float inv_s = 1.f / s;
       const float lse = m + logf(s);
       // 5. per-expert probability sums of this 32-token block for this part's
-      // experts: 32 tokens x SW experts at a time through shared memory, lane
-      // j < SW sums column j over the tokens in order (fixed order: deterministic)
-      float* stg = &ctl->pstage[wi][0][0];
+      // experts, 16 at a time: a fixed shuffle tree over the 32 tokens (lanes),
+      // halving the columns at each step, leaves column lane / 2 in lanes
+      // 2c and 2c + 1 (deterministic)
 #pragma unroll
       for (int c0 = 0; c0 < H; c0 += 16) {
         float pv[16];
@@ -506,24 +530,9 @@ __global__ void __launch_bounds__(RtShape<EP>::THREADS, 1)
             pv[i] = (valid && e < E) ? expf(logit(__uint_as_float(r[i]), e) - m) * inv_s : 0.f;
           }
         }
-        constexpr int SW = RtCtlT::SW;
-#pragma unroll
-        for (int hh = 0; hh < 16 / SW; ++hh) {
-#pragma unroll
-          for (int i = 0; i < SW; ++i) stg[lane * (SW + 1) + i] = pv[hh * SW + i];
-          __syncwarp();
-          const int e = c_lo + c0 + hh * SW + lane;
-          if (lane < SW && has_cols && e < E && blk_valid) {
-            float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-            for (int t = 0; t < 32; t += 2) {
-              a0 += stg[t * (SW + 1) + lane];
-              a1 += stg[(t + 1) * (SW + 1) + lane];
-            }
-            p.part_psum[e * p.nblk + blk] = a0 + a1;
-          }
-          __syncwarp();
-        }
+        const float ps = column_sums16(pv, lane);
+        const int e = c_lo + c0 + (lane >> 1);
+        if ((lane & 1) == 0 && has_cols && e < E && blk_valid) p.part_psum[e * p.nblk + blk] = ps;
       }
       if constexpr (!REG) {
         tc_fence_before();
