@@ -405,14 +405,14 @@ __device__ __forceinline__ void scan_finalize(const RoutingArgs& a, int cnt, int
 }
 
 // SINGLE (few router blocks): one block, thread e walks expert e's blocks in
-// order.  Otherwise one block per expert as described above.
+// order, then finalises.  Otherwise one block per expert as described above
+// (the dispatch launch finalises).
 template <bool SINGLE>
 __global__ void __launch_bounds__(SCAN_T) scan_kernel(RoutingArgs a) {
   __shared__ int s_warp[2 * (SCAN_T / 32 + 1)];
   __shared__ float s_redf[SCAN_T / 32];
   __shared__ int s_redi[SCAN_T / 32];
   __shared__ double s_redd[6 * (SCAN_T / 32)];
-  __shared__ int s_last;
   const int tid = threadIdx.x;
   const int E = a.E, nb = a.nblk;
   pdl_wait();
@@ -453,20 +453,11 @@ __global__ void __launch_bounds__(SCAN_T) scan_kernel(RoutingArgs a) {
   }
   const int c1_tot = block_sum<int>(c1, s_redi);
   const float ps_tot = block_sum<float>(ps, s_redf);
-  if (tid == 0) {
+  if (tid == 0) {  // the totals; the dispatch launch finalises (scan_finalize) alongside its copies
     a.counts[e] = count;
     a.tot_cnt1[e] = c1_tot;
     a.tot_psum[e] = ps_tot;
-    __threadfence();
-    s_last = atomicAdd(a.scan_ticket, 1) == E - 1;
   }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  // the last block
-  scan_finalize(a, tid < E ? __ldcg(a.counts + tid) : 0, tid < E ? __ldcg(a.tot_cnt1 + tid) : 0,
-                tid < E ? __ldcg(a.tot_psum + tid) : 0.f, s_warp, s_redd);
-  if (tid == 0) *a.scan_ticket = 0;  // ready for the next call
 }
 
 // ---------------------------------------------------------------------------
@@ -494,29 +485,62 @@ __device__ __forceinline__ void copy_x_row(const XT* __restrict__ x, XT* __restr
 }
 
 // ---------------------------------------------------------------------------
-// Dispatch: one block per router block of BT tokens.  Warp 0 assigns the slot
-// rank of every (token, choice) of the block in token-major order (stable:
-// base = number of earlier assignments to the same expert in earlier blocks);
-// then all warps copy the kept rows of x into the expert-sorted buffer.
+// Dispatch: one block per router block of BT tokens.  The block derives the
+// group offsets from the scan's per-expert counts itself (as scan_finalize
+// does), while its (token, choice) experts and gates, and its per-expert rank
+// bases, load alongside.  Warp 0 assigns the slot rank of every (token,
+// choice) of the block in token-major order (stable: base = number of earlier
+// assignments to the same expert in earlier blocks); then all warps copy the
+// kept rows of x into the expert-sorted buffer.  With `finalize` one more
+// block, nblk, runs scan_finalize (offsets and tile prefix for the GEMMs,
+// counts, losses and statistics) beside them.
 template <typename XT>
 __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
   __shared__ int run_s[256];
+  __shared__ int off_s[256];
   __shared__ int dest_s[BT * 8];
+  __shared__ int e_s[BT * 8];
+  __shared__ float g_s[BT * 8];
+  __shared__ int s_warp[2 * (SCAN_T / 32 + 1)];
+  __shared__ double s_red[6 * (SCAN_T / 32)];
+  static_assert(SCAN_T == 256, "the dispatch block is the scan's block size");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = a.E, k = a.k, d = a.d, nb = a.nblk;
+  pdl_wait();
+  pdl_trigger();
+  if (static_cast<int>(blockIdx.x) == nb) {  // the scan's finalisation
+    scan_finalize(a, tid < E ? a.counts[tid] : 0, tid < E ? a.tot_cnt1[tid] : 0, tid < E ? a.tot_psum[tid] : 0.f,
+                  s_warp, s_red);
+    return;
+  }
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * BT;
   const int nt = static_cast<int>((a.T - t0) < BT ? (a.T - t0) : BT);
   const int nA = nt * k;
-  pdl_wait();
-  pdl_trigger();
-  for (int e = tid; e < E; e += 256) run_s[e] = a.blockoff[e * nb + blockIdx.x];
+  {
+    const int groups = E + a.n_shared;
+    int kept = 0;
+    if (tid < E) {
+      const int cnt = a.counts[tid];
+      run_s[tid] = a.blockoff[tid * nb + blockIdx.x];
+      kept = (a.capacity < 0) ? cnt : static_cast<int>((int64_t)cnt < a.capacity ? (int64_t)cnt : a.capacity);
+    } else if (tid < groups) {
+      kept = static_cast<int>(a.T);
+    }
+    for (int i = tid; i < nA; i += 256) {
+      e_s[i] = a.topk_idx[t0 * k + i];
+      g_s[i] = a.topk_gate[t0 * k + i];
+    }
+    int off, mp, total_rows, total_tiles;
+    block_exscan_int2(kept, (kept + kTileM - 1) / kTileM, s_warp, off, mp, total_rows, total_tiles);  // syncs
+    if (tid < groups) off_s[tid] = off;
+  }
   __syncthreads();
   if (warp == 0) {
     const uint32_t lt = (1u << lane) - 1u;
     for (int a0 = 0; a0 < nA; a0 += 32) {
       const int ai = a0 + lane;
       const bool valid = ai < nA;
-      int e = valid ? a.topk_idx[t0 * k + ai] : -1;
+      int e = valid ? e_s[ai] : -1;
       if (e < 0 || e >= E) e = -1;  // never produced by the router; keeps smem indexing in range
       const uint32_t peers = __match_any_sync(0xffffffffu, e);
       const bool ok = valid && e >= 0;
@@ -530,13 +554,13 @@ __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
         a.dest_row[t0 * k + ai] = -1;
       } else if (valid) {
         const bool kept = a.capacity < 0 || rank < a.capacity;
-        const int dest = kept ? a.offsets[e] + rank : -1;
+        const int dest = kept ? off_s[e] + rank : -1;
         dest_s[ai] = dest;
         a.dest_row[t0 * k + ai] = dest;
         if (a.drop_mask != nullptr) a.drop_mask[t0 * k + ai] = kept ? 0 : 1;
         if (kept) {
           a.row_token[dest] = static_cast<int32_t>(t0 + ai / k);
-          a.row_gate[dest] = a.topk_gate[t0 * k + ai];
+          a.row_gate[dest] = g_s[ai];
         }
       }
     }
@@ -559,7 +583,7 @@ __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
   }
   // shared experts: every token of the block, gate 1, rows offsets[E] + s * T + t
   if (a.n_shared > 0) {
-    const int64_t base = a.offsets[E];
+    const int64_t base = off_s[E];
     for (int q = warp; q < nt * a.n_shared; q += 8) {
       const int si = q / nt;
       const int64_t tok = t0 + (q - si * nt);
@@ -1177,8 +1201,11 @@ cudaError_t launch_scan_dispatch(const RoutingArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_dispatch(const RoutingArgs& a, cudaStream_t s) {
-  if (a.x_is_bf16) return launch_pdl(dispatch_kernel<__nv_bfloat16>, dim3(a.nblk), dim3(256), 0, s, a);
-  return launch_pdl(dispatch_kernel<float>, dim3(a.nblk), dim3(256), 0, s, a);
+  // one more block finalises the scan when its per-expert blocks did not
+  // (the single-block scan finalises itself)
+  const unsigned grid = static_cast<unsigned>(a.nblk + (a.nblk > kScanSingleBlocks ? 1 : 0));
+  if (a.x_is_bf16) return launch_pdl(dispatch_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, a);
+  return launch_pdl(dispatch_kernel<float>, dim3(grid), dim3(256), 0, s, a);
 }
 
 namespace {
