@@ -13,7 +13,7 @@
 // 128 x 64, three plane boxes E_pad x 64), warp 1 issues the MMAs (M 128,
 // N E_pad, K 16; 4 per plane per k-block), and 4 NP epilogue warps take each
 // token (TMEM lane) with NP threads, one per part of the experts (NP = 2, or 4
-// for E_pad 128): bias, max, one-pass top-k (ties to the lower expert index),
+// for E_pad 64 and 128): bias, max, one-pass top-k (ties to the lower expert index),
 // log-sum-exp, gates, and the per-32-token partial counts and sums that the
 // scan kernel reduces (the warps of one TMEM lane quarter own one 32-token
 // router block, the same partition as the CUDA-core router).
@@ -32,11 +32,12 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;
 // Epilogue threads per token (expert parts) and block size: two parts of up
-// to 32 experts; for E_pad 128, four parts of 32, so that each thread keeps its
-// logits in registers and the top-k and exponential chains stay short.
+// to 16 experts (E_pad 16, 32); for E_pad 64 and 128, four parts of 16 or 32,
+// so that each thread keeps its logits in registers and the top-k and
+// exponential chains stay short.
 template <int EP>
 struct RtShape {
-  static constexpr int NP = EP >= 128 ? 4 : 2;
+  static constexpr int NP = EP >= 64 ? 4 : 2;
   static constexpr int THREADS = 64 + 128 * NP;  // producer, MMA, 4 NP epilogue warps
 };
 constexpr int A_BYTES = BM * BK * 2;
@@ -359,10 +360,10 @@ __global__ void __launch_bounds__(RtShape<EP>::THREADS, 1)
       const int blk = tile * 4 + q;
       const bool blk_valid = blk < p.nblk;
 
-      // 1. this half's logits: for up to 32 columns (E_pad <= 64) one batch of
-      // TMEM loads into registers, after which the accumulator is released;
-      // for 64 columns (E_pad = 128) passes over 16-column chunks re-read TMEM
-      // (the register budget of ten warps does not hold 64 logits per thread)
+      // 1. this part's logits: up to 32 columns (every E_pad at NP parts) in
+      // one batch of TMEM loads into registers, after which the accumulator is
+      // released; wider parts would take passes over 16-column chunks that
+      // re-read TMEM
       constexpr bool REG = H <= 32;
       float h[REG ? H : 1];
       if constexpr (REG) {
@@ -551,13 +552,23 @@ __global__ void __launch_bounds__(RtShape<EP>::THREADS, 1)
 #pragma unroll
         for (int j = 0; j < K; ++j) {
           const float g = (p.gate_mode == 0) ? expf(tv[j] - m) * inv_s : expf(tv[j] - tv[0]) / den;
-          const int e = (te[j] >= 0 && te[j] < E) ? te[j] : 0;
           p.topk_idx[tok * K + j] = te[j];
           p.topk_gate[tok * K + j] = g;
-          atomicAdd(&ctl->hist[q][e], 1);
-          if (j == 0) atomicAdd(&ctl->cnt1[q][e], 1);
         }
         if (p.lse_out != nullptr) p.lse_out[tok] = lse;
+      }
+      // block counts: per choice j, one shared-memory update per distinct
+      // expert by the lowest lane choosing it (no contended atomics)
+#pragma unroll
+      for (int j = 0; j < K; ++j) {
+        const int e = valid ? ((te[j] >= 0 && te[j] < E) ? te[j] : 0) : -1;
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && lane == __ffs(peers) - 1) {
+          const int n = __popc(peers);
+          ctl->hist[q][e] += n;
+          if (j == 0) ctl->cnt1[q][e] += n;
+        }
+        __syncwarp();
       }
       const float l2 = warp_sum_f(valid ? lse * lse : 0.f);
       __syncwarp();
