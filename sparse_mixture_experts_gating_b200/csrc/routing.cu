@@ -361,6 +361,8 @@ __device__ __forceinline__ void scan_finalize(const RoutingArgs& a, int cnt, int
   const int tid = threadIdx.x, E = a.E, nb = a.nblk;
   const int groups = E + a.n_shared;
   const bool routed = tid < E;
+  double zs = 0.0;  // this thread's share of sum lse^2 (loaded before the scans below)
+  for (int b = tid; b < nb; b += SCAN_T) zs += static_cast<double>(a.part_lse2[b]);
   int kept = 0;
   if (routed) kept = (a.capacity < 0) ? cnt : static_cast<int>((int64_t)cnt < a.capacity ? (int64_t)cnt : a.capacity);
   else if (tid < groups) kept = static_cast<int>(a.T);
@@ -381,8 +383,6 @@ __device__ __forceinline__ void scan_finalize(const RoutingArgs& a, int cnt, int
   const double T = static_cast<double>(a.T);
   const double c = routed ? static_cast<double>(cnt) : 0.0;
   const double Pe = routed ? static_cast<double>(ps) / T : 0.0;  // mean router probability of e
-  double zs = 0.0;
-  for (int b = tid; b < nb; b += SCAN_T) zs += static_cast<double>(a.part_lse2[b]);
   // dropped, sum f1*P (first choices), sum of counts, sum of P, sum counts*P, sum lse^2
   double v[6] = {routed ? static_cast<double>(cnt - kept) : 0.0,
                  routed ? static_cast<double>(c1) * static_cast<double>(ps) : 0.0, c, Pe, c * Pe, zs};
@@ -457,6 +457,18 @@ __global__ void __launch_bounds__(SCAN_T) scan_kernel(RoutingArgs a) {
     a.counts[e] = count;
     a.tot_cnt1[e] = c1_tot;
     a.tot_psum[e] = ps_tot;
+  }
+}
+
+// One warp zeroes row `tok` of y (16-byte stores where the row allows).
+template <typename XT>
+__device__ __forceinline__ void zero_row(XT* __restrict__ y, int d, int64_t tok, int lane) {
+  if ((static_cast<size_t>(d) * sizeof(XT)) % 16 == 0) {
+    uint4* dst = reinterpret_cast<uint4*>(y + tok * d);
+    const int nv = static_cast<int>(static_cast<size_t>(d) * sizeof(XT) / 16);
+    for (int v = lane; v < nv; v += 32) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+  } else {
+    for (int c = lane; c < d; c += 32) y[tok * d + c] = XT(0.f);
   }
 }
 
@@ -576,7 +588,7 @@ __global__ void __launch_bounds__(256) dispatch_kernel(RoutingArgs a) {
     if (dest >= 0) {
       copy_row(tok, dest);
     } else if (yz != nullptr) {  // k == 1: a dropped token's output row is zero
-      for (int c = lane; c < d; c += 32) yz[tok * d + c] = XT(0.f);
+      zero_row(yz, d, tok, lane);
       if (a.yf_zero_dropped != nullptr)
         for (int c = lane; c < d; c += 32) a.yf_zero_dropped[tok * d + c] = 0.f;
     }
@@ -751,7 +763,7 @@ __global__ void __launch_bounds__(SCAN_T) scan_dispatch_kernel(RoutingArgs a) {
     if (dest >= 0) {
       copy_x_row(x, Xp, d, tok, dest, lane);
     } else if (yz != nullptr) {  // k == 1: a dropped token's output row is zero
-      for (int c = lane; c < d; c += 32) yz[tok * d + c] = XT(0.f);
+      zero_row(yz, d, tok, lane);
       if (a.yf_zero_dropped != nullptr)
         for (int c = lane; c < d; c += 32) a.yf_zero_dropped[tok * d + c] = 0.f;
     }
@@ -952,7 +964,7 @@ __global__ void __launch_bounds__(SCAN_T) route_small_kernel(RoutingArgs a, int 
     if (s_dest[i] >= 0) {
       copy_row(tok, s_dest[i]);
     } else if (yz != nullptr) {  // k == 1: a dropped token's output row is zero
-      for (int c = lane; c < d; c += 32) yz[tok * d + c] = XT(0.f);
+      zero_row(yz, d, tok, lane);
       if (a.yf_zero_dropped != nullptr)
         for (int c = lane; c < d; c += 32) a.yf_zero_dropped[tok * d + c] = 0.f;
     }
