@@ -38,7 +38,6 @@ struct RoutingArgs {
   int32_t* mprefix;    // [E+1] prefix of ceil(kept_e / kTileM)
   int32_t* tot_cnt1;   // [E]   first-choice count of each expert (scan)
   float* tot_psum;     // [E]   probability sum of each expert (scan)
-  int32_t* scan_ticket;  // zeroed by the router; the scan's last block resets it
   float* balance_out;    // [3] aux over all choices, CV of counts, cv^2 of P (scan)
   int n_shared;          // shared experts: groups E .. E + n_shared - 1 of T rows each
   int32_t* row_token;  // [S_max]

@@ -210,7 +210,7 @@ Layout make_layout(const moe_layer& L, int64_t T, bool w4 = false) {
   // [groups + 1]: the routed experts' groups, then one per shared expert
   w.offsets = take(sizeof(int32_t) * (L.E + L.n_shared + 1));
   w.mprefix = take(sizeof(int32_t) * (L.E + L.n_shared + 1));
-  // scan totals [E] + [E], the scan ticket, the three balance statistics
+  // scan totals [E] + [E], 16 spare bytes, the three balance statistics
   w.scal = take(sizeof(int32_t) * L.E + sizeof(float) * L.E + 64);
   const bool tc_router = L.dtype == MOE_BF16 && L.E <= kRouterTcMaxE;
   w.wsplit = take(tc_router ? 3 * sizeof(uint16_t) * router_pad_e(L.E) * static_cast<size_t>(L.d) : 0);
@@ -551,7 +551,6 @@ int forward_impl(moe_handle h, int64_t T, const void* x, const float* W_r, const
   r.row_token = reinterpret_cast<int32_t*>(ws + w.row_token);
   r.tot_cnt1 = reinterpret_cast<int32_t*>(ws + w.scal);
   r.tot_psum = reinterpret_cast<float*>(ws + w.scal + sizeof(int32_t) * L.E);
-  r.scan_ticket = reinterpret_cast<int32_t*>(ws + w.scal + (sizeof(int32_t) + sizeof(float)) * L.E);
   r.balance_out = reinterpret_cast<float*>(ws + w.scal + (sizeof(int32_t) + sizeof(float)) * L.E + 16);
   r.n_shared = L.n_shared;
   r.row_gate = reinterpret_cast<float*>(ws + w.row_gate);

@@ -130,10 +130,9 @@ __device__ __forceinline__ float warp_sum_f(float v) {
 // Split W_r (fp32 [E][d]) into bf16 planes [3][EP][d]; rows E..EP-1 are zero.
 __global__ void __launch_bounds__(256) split_router_kernel(const float* __restrict__ W, int E, int EP, int d,
                                                            __nv_bfloat16* __restrict__ planes, int* tickets,
-                                                           int n_tickets, int* scan_ticket) {
+                                                           int n_tickets) {
   const int64_t n = static_cast<int64_t>(EP) * d;
   pdl_trigger();  // the router may be scheduled at once (it waits for this grid before reading)
-  if (blockIdx.x == 0 && threadIdx.x == 0) *scan_ticket = 0;
   if (tickets != nullptr)
     for (int i = blockIdx.x * 256 + threadIdx.x; i < n_tickets; i += gridDim.x * 256) tickets[i] = 0;
   for (int64_t i = blockIdx.x * 256ll + threadIdx.x; i < n; i += static_cast<int64_t>(gridDim.x) * 256) {
@@ -634,7 +633,7 @@ cudaError_t launch_ep(const RoutingArgs& a, void* wsplit, void* partials, int nu
   const int64_t n = static_cast<int64_t>(EP) * a.d;
   const int sblocks = static_cast<int>((n + 255) / 256 < 4 * num_sms ? (n + 255) / 256 : 4 * num_sms);
   split_router_kernel<<<sblocks, 256, 0, s>>>(a.W_r, a.E, EP, a.d, static_cast<__nv_bfloat16*>(wsplit),
-                                              p.ksplit > 1 ? p.tickets : nullptr, p.n_tiles, a.scan_ticket);
+                                              p.ksplit > 1 ? p.tickets : nullptr, p.n_tiles);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

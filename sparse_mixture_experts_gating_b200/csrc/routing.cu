@@ -74,7 +74,6 @@ __global__ void __launch_bounds__(RT) router_kernel(RoutingArgs a) {
   const XT* x = static_cast<const XT*>(a.x);
 
   for (int e = tid; e < EP; e += RT) { cnt1_s[e] = 0; hist_s[e] = 0; }
-  if (blockIdx.x == 0 && tid == 0) *a.scan_ticket = 0;
 
   if (a.logits_in == nullptr) {
     const int tg = tid >> 4, eg = tid & 15;
