@@ -508,17 +508,79 @@ __global__ void __launch_bounds__(256) bw_transpose_f32x2_kernel(const float* __
   }
 }
 
+// [G][R][C] -> [G][C][R] for elements of 2 or 4 bytes (T = uint16_t / float)
+// with R and C multiples of 16 / sizeof(T) and 16-byte aligned buffers: 64 x
+// 64 tiles, 16-byte reads along the input rows; each 16-byte write holds
+// 16 / sizeof(T) consecutive input rows of one input column, and the threads
+// of a warp write whole output row segments (64 elements) side by side.
+template <typename T>
+__global__ void __launch_bounds__(256) bw_transpose16_kernel(const T* __restrict__ in, T* __restrict__ out, int R,
+                                                             int C) {
+  constexpr int V = 16 / static_cast<int>(sizeof(T));  // elements per 16-byte word
+  constexpr int NW = 64 * 64 / V / 256;                // words per thread and phase
+  __shared__ T tile[64][64 + 4 / static_cast<int>(sizeof(T))];  // rows padded by one 4-byte word
+  const int64_t g = blockIdx.z;
+  const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64;
+  const T* src = in + g * R * C;
+  T* dst = out + g * R * C;
+  uint4 v[NW];
+#pragma unroll
+  for (int p = 0; p < NW; ++p) {  // word p of this thread: row id / (64 / V), column chunk id % (64 / V)
+    const int id = threadIdx.x + 256 * p;
+    const int r = id / (64 / V), c = (id % (64 / V)) * V;
+    v[p] = (r0 + r < R && c0 + c < C)
+               ? *reinterpret_cast<const uint4*>(src + static_cast<int64_t>(r0 + r) * C + c0 + c)
+               : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int p = 0; p < NW; ++p) {
+    const int id = threadIdx.x + 256 * p;
+    const int r = id / (64 / V), c = (id % (64 / V)) * V;
+    const uint32_t w[4] = {v[p].x, v[p].y, v[p].z, v[p].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) *reinterpret_cast<uint32_t*>(&tile[r][c + j * (4 / sizeof(T))]) = w[j];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int p = 0; p < NW; ++p) {  // output row c0 + oc, input rows r0 + q V .. + V - 1
+    const int id = threadIdx.x + 256 * p;
+    const int oc = id / (64 / V), q = id % (64 / V);
+    if (c0 + oc < C && r0 + q * V < R) {
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if constexpr (sizeof(T) == 2)
+          w[j] = static_cast<uint32_t>(tile[q * V + 2 * j][oc]) | (static_cast<uint32_t>(tile[q * V + 2 * j + 1][oc]) << 16);
+        else
+          w[j] = __float_as_uint(tile[q * V + j][oc]);
+      }
+      *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(c0 + oc) * R + r0 + q * V) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+bool aligned16(const void* a, const void* b) {
+  return ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 15) == 0;
+}
+
 cudaError_t transpose_f32(const void* in, void* out, int G, int R, int C, cudaStream_t s) {
   const dim3 grid((C + 63) / 64, (R + 63) / 64, G);
-  bw_transpose_f32x2_kernel<<<grid, 256, 0, s>>>(static_cast<const float*>(in), static_cast<float*>(out), R, C);
+  if (aligned16(in, out) && R % 4 == 0 && C % 4 == 0)
+    bw_transpose16_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(in), static_cast<float*>(out), R, C);
+  else  // a gradient output without 16-byte alignment
+    bw_transpose_f32x2_kernel<<<grid, 256, 0, s>>>(static_cast<const float*>(in), static_cast<float*>(out), R, C);
   count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t transpose_bf16(const void* in, void* out, int G, int R, int C, cudaStream_t s) {
   const dim3 grid((C + 63) / 64, (R + 63) / 64, G);
-  bw_transpose_bf16x2_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(in),
-                                                  static_cast<__nv_bfloat16*>(out), R, C);
+  if (aligned16(in, out) && R % 8 == 0 && C % 8 == 0)
+    bw_transpose16_kernel<uint16_t><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(in), static_cast<uint16_t*>(out),
+                                                        R, C);
+  else
+    bw_transpose_bf16x2_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(in),
+                                                    static_cast<__nv_bfloat16*>(out), R, C);
   count_launch();
   return cudaGetLastError();
 }
