@@ -298,8 +298,9 @@ __global__ void bw_cnt1_kernel(int64_t T, int k, const int32_t* topk_idx, int32_
   if (t < T) atomicAdd(cnt1 + topk_idx[t * k], 1);
 }
 
-// One block per token: the router logits again (fp32, bias added last), the
-// softmax and log-sum-exp, and the gradient reaching the logits.
+// One block per token: the router logits (given: the forward's router kernel
+// run again, the same fp32 values; else recomputed here, fp32, bias added
+// last), the softmax and log-sum-exp, and the gradient reaching the logits.
 template <typename XT>
 __global__ void __launch_bounds__(THREADS) bw_router_kernel(BackwardArgs a) {
   __shared__ float s_h[256], s_dp[256], s_dh[256];
@@ -308,13 +309,17 @@ __global__ void __launch_bounds__(THREADS) bw_router_kernel(BackwardArgs a) {
   const int64_t t = blockIdx.x;
   const int E = a.E, d = a.d, k = a.k, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const XT* x = static_cast<const XT*>(a.x) + t * d;
-  for (int e = warp; e < E; e += THREADS / 32) {
-    const float* w = a.W_r + static_cast<int64_t>(e) * d;
-    float s = 0.f;
-    for (int c = lane; c < d; c += 32) s = fmaf(w[c], to_f32(x[c]), s);
+  if (a.logits != nullptr) {  // computed again by the forward's router kernel
+    for (int e = tid; e < E; e += THREADS) s_h[e] = a.logits[t * E + e];
+  } else {
+    for (int e = warp; e < E; e += THREADS / 32) {
+      const float* w = a.W_r + static_cast<int64_t>(e) * d;
+      float s = 0.f;
+      for (int c = lane; c < d; c += 32) s = fmaf(w[c], to_f32(x[c]), s);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) s_h[e] = a.b_r != nullptr ? s + a.b_r[e] : s;
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) s_h[e] = a.b_r != nullptr ? s + a.b_r[e] : s;
+    }
   }
   if (tid < k) {
     const int dst = a.dest_row[t * k + tid];
@@ -359,6 +364,80 @@ __global__ void __launch_bounds__(THREADS) bw_router_kernel(BackwardArgs a) {
   for (int e = tid; e < E; e += THREADS) {
     const float p = expf(s_h[e] - m) / Z;
     a.dh[t * E + e] = s_dh[e] + p * (s_dp[e] - dpp) + a.z_coef * 2.f * inv_T * lse * p;
+  }
+}
+
+// dx for 64 tokens x 64 columns per block (16 x 16 threads, 4 x 4 outputs
+// each, 16-byte accesses): the router term W_r^T dh_t from 32-expert chunks
+// of dh and W_r staged in shared memory, experts in order, then the same sum
+// as bw_dx_kernel (kept rows' dXp, choices in order, then the shared
+// experts' rows) plus that term: the same operations in the same order.
+// Needs d % 4 == 0 and 16-byte aligned dXp and dx.
+__global__ void __launch_bounds__(256) bw_dx_tiled_kernel(BackwardArgs a, int parts) {
+  __shared__ float s_dh[64][33];
+  __shared__ __align__(16) float s_w[32][68];
+  const int E = a.E, d = a.d, k = a.k;
+  const int64_t T = a.T;
+  const int t0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int ne = min(32, E - e0);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {  // dh [64 tokens][32 experts]
+      const int idx = tid + 256 * q, r = idx >> 5, e = idx & 31;
+      s_dh[r][e] = (t0 + r < T && e < ne) ? a.dh[(static_cast<int64_t>(t0) + r) * E + e0 + e] : 0.f;
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {  // W_r [32 experts][64 columns], 16-byte loads
+      const int idx = tid + 256 * q, e = idx >> 4, c = (idx & 15) * 4;
+      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e < ne && c0 + c < d) w = *reinterpret_cast<const float4*>(a.W_r + static_cast<int64_t>(e0 + e) * d + c0 + c);
+      *reinterpret_cast<float4*>(&s_w[e][c]) = w;
+    }
+    __syncthreads();
+    for (int e = 0; e < ne; ++e) {
+      const float4 w = *reinterpret_cast<const float4*>(&s_w[e][tx * 4]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float h = s_dh[ty * 4 + i][e];
+        acc[i][0] = fmaf(h, w.x, acc[i][0]);
+        acc[i][1] = fmaf(h, w.y, acc[i][1]);
+        acc[i][2] = fmaf(h, w.z, acc[i][2]);
+        acc[i][3] = fmaf(h, w.w, acc[i][3]);
+      }
+    }
+    __syncthreads();
+  }
+  const int c = c0 + tx * 4;
+  if (c >= d) return;
+  const int64_t pstride = a.s_max * d;  // between the W1 and W3 parts of dXp
+  const int64_t sbase = a.n_shared > 0 ? a.offsets[E] : 0;
+  const float4* X4 = reinterpret_cast<const float4*>(a.dXp);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t t = t0 + ty * 4 + i;
+    if (t >= T) break;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto add_row = [&](int64_t row) {
+      const float4 p = X4[(row * d + c) >> 2];
+      v.x += p.x; v.y += p.y; v.z += p.z; v.w += p.w;
+      if (parts == 2) {
+        const float4 p2 = X4[(pstride + row * d + c) >> 2];
+        v.x += p2.x; v.y += p2.y; v.z += p2.z; v.w += p2.w;
+      }
+    };
+    for (int j = 0; j < k; ++j) {
+      const int dst = a.dest_row[t * k + j];
+      if (dst >= 0) add_row(dst);
+    }
+    for (int si = 0; si < a.n_shared; ++si) add_row(sbase + si * T + t);
+    *reinterpret_cast<float4*>(a.dx + t * d + c) =
+        make_float4(v.x + acc[i][0], v.y + acc[i][1], v.z + acc[i][2], v.w + acc[i][3]);
   }
 }
 
@@ -800,7 +879,14 @@ cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
   bw_router_kernel<XT><<<static_cast<unsigned>(a.T), THREADS, 0, s>>>(a);
   count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bw_dx_kernel<<<static_cast<unsigned>(a.T), THREADS, 0, s>>>(a, parts);
+  const bool tiled = a.d % 4 == 0 && (a.T + 63) / 64 <= 65535 &&
+                     ((reinterpret_cast<uintptr_t>(a.W_r) | reinterpret_cast<uintptr_t>(a.dXp) |
+                       reinterpret_cast<uintptr_t>(a.dx)) & 15) == 0;
+  if (tiled)
+    bw_dx_tiled_kernel<<<dim3(static_cast<unsigned>((a.d + 63) / 64), static_cast<unsigned>((a.T + 63) / 64)), 256, 0,
+                         s>>>(a, parts);
+  else
+    bw_dx_kernel<<<static_cast<unsigned>(a.T), THREADS, 0, s>>>(a, parts);
   count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // dW_r = sum_t dh_t x_t^T: K = T cut into a.wr_chunks chunks of partials, summed in order

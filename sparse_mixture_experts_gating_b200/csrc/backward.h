@@ -16,6 +16,7 @@ struct BackwardArgs {
   int64_t s_max;       // rows of the expert-sorted buffers
   const void* x;       // [T][d]
   const float* W_r;    // [E][d]
+  const float* logits;  // [T][E] the forward's router logits (bias added), or NULL: recomputed here
   const float* b_r;    // [E] or NULL
   const void* W1;      // [E + n_shared][d_ff][d]
   const void* W3;      // same, SwiGLU only

@@ -277,6 +277,9 @@ Layout make_layout(const moe_layer& L, int64_t T, bool w4 = false) {
 struct BwLayout {
   size_t A1, A3, U, dg, dXp, dh, cnt1, ones, dYs, W1t, W3t, W2t, dA1p, dA3p, P1, P3, PH, XT, DT, dW2t, woff, wpre,
       wr_part, total;
+  // the forward's router kernel run again for its logits (bf16, E <= kRouterTcMaxE)
+  bool rt;
+  size_t rt_idx, rt_gate, rt_hist, rt_cnt1, rt_psum, rt_lse2, rt_logits, rt_wsplit, rt_rpart;
   int max_group_rows, k_pad, wr_chunks;
 };
 
@@ -327,6 +330,17 @@ BwLayout make_bw_layout(const moe_layer& L, const Layout& w) {
   const int64_t ch = (w.T + 255) / 256;
   b.wr_chunks = static_cast<int>(ch < 1 ? 1 : (ch > 64 ? 64 : ch));
   b.wr_part = take(sizeof(float) * b.wr_chunks * static_cast<size_t>(L.E) * L.d);
+  b.rt = tc && L.E <= kRouterTcMaxE;
+  const size_t Tk = static_cast<size_t>(w.T) * L.k, EB = static_cast<size_t>(L.E) * w.nblk;
+  b.rt_idx = take(b.rt ? sizeof(int32_t) * Tk : 0);
+  b.rt_gate = take(b.rt ? sizeof(float) * Tk : 0);
+  b.rt_hist = take(b.rt ? sizeof(int32_t) * EB : 0);
+  b.rt_cnt1 = take(b.rt ? sizeof(int32_t) * EB : 0);
+  b.rt_psum = take(b.rt ? sizeof(float) * EB : 0);
+  b.rt_lse2 = take(b.rt ? sizeof(float) * w.nblk : 0);
+  b.rt_logits = take(b.rt ? sizeof(float) * static_cast<size_t>(w.T) * L.E : 0);
+  b.rt_wsplit = take(b.rt ? 3 * sizeof(uint16_t) * router_pad_e(L.E) * static_cast<size_t>(L.d) : 0);
+  b.rt_rpart = take(b.rt ? router_partials_bytes(w.T, L.E, L.d) : 0);
   b.total = o;
   return b;
 }
@@ -961,7 +975,34 @@ int moe_backward(moe_handle h, int64_t T, const void* x, const float* W_r, const
   a.dW1 = dW1;
   a.dW3 = dW3;
   a.dW2 = dW2;
-  const cudaError_t ce = launch_backward(a, s);
+  cudaError_t ce = cudaSuccess;
+  if (b.rt) {  // the router logits, as the forward computed them (its top-k and tables go to scratch)
+    RoutingArgs r;
+    memset(&r, 0, sizeof(r));
+    r.T = T;
+    r.E = L.E;
+    r.k = L.k;
+    r.d = L.d;
+    r.gate_mode = L.gate_mode;
+    r.capacity = w.capacity;
+    r.nblk = w.nblk;
+    r.x_is_bf16 = 1;
+    r.x = x;
+    r.W_r = W_r;
+    r.b_r = b_r;
+    r.topk_idx = reinterpret_cast<int32_t*>(bw + b.rt_idx);
+    r.topk_gate = reinterpret_cast<float*>(bw + b.rt_gate);
+    r.part_hist = reinterpret_cast<int32_t*>(bw + b.rt_hist);
+    r.part_cnt1 = reinterpret_cast<int32_t*>(bw + b.rt_cnt1);
+    r.part_psum = reinterpret_cast<float*>(bw + b.rt_psum);
+    r.part_lse2 = reinterpret_cast<float*>(bw + b.rt_lse2);
+    r.logits_out = reinterpret_cast<float*>(bw + b.rt_logits);
+    const char* why = nullptr;
+    ce = launch_router_tc(r, bw + b.rt_wsplit, bw + b.rt_rpart, di->num_sms, di->err, s, &why);
+    if (why != nullptr) return fail(MOE_ERR_UNSUPPORTED, std::string("moe_backward: ") + why);
+    a.logits = r.logits_out;
+  }
+  if (ce == cudaSuccess) ce = launch_backward(a, s);
   if (ce != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_backward: ") + cudaGetErrorString(ce));
   t_err.clear();
   return MOE_OK;
