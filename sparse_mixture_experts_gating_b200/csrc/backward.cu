@@ -504,7 +504,7 @@ __global__ void __launch_bounds__(256) bw_gather_dy_kernel(int d, const int32_t*
 // out[r][n] = sum_k A[r][k] B_e[n][k] over the expert-sorted rows.
 cudaError_t tc_product(const BackwardArgs& a, const void* A, const void* A_lo, const void* B, int N, int K, float* out,
                        cudaStream_t s, const int32_t* offsets = nullptr, const int32_t* mprefix = nullptr,
-                       int64_t a_rows = 0, int max_rows = 0) {
+                       int64_t a_rows = 0, int max_rows = 0, const int32_t* k_rows = nullptr) {
   GemmArgs g;
   memset(&g, 0, sizeof(g));
   g.epi = EPI_GATE_F32;
@@ -524,6 +524,7 @@ cudaError_t tc_product(const BackwardArgs& a, const void* A, const void* A_lo, c
   g.row_gate = a.ones;
   g.row_token = a.row_token;
   g.err = a.err;
+  g.k_rows = k_rows;
   TcGemmPlan plan;
   const char* why = nullptr;
   cudaError_t e = plan_gemm_tc(g, &plan, &why);
@@ -666,7 +667,8 @@ cudaError_t transpose_bf16(const void* in, void* out, int G, int R, int C, cudaS
 
 
 // Per-expert operand of a weight gradient: out[e][f][kk] = v(off_e + kk, f)
-// for kk below the group's row count, 0 up to k_pad, where v(r, f) =
+// for kk below the group's row count, 0 up to the next multiple of 64 (the
+// product's k-blocks; no further than k_pad), where v(r, f) =
 // src[r][f] (times scale[r] when given); bf16, with SPLIT a lo plane at
 // out + plane holding v - hi.  32 x 32 tiles: rows read along f, written
 // along kk.
@@ -680,6 +682,7 @@ __global__ void __launch_bounds__(256) bw_pack_kernel(const ST* __restrict__ src
   const int f0 = blockIdx.x * 32, k0 = blockIdx.y * 32;
   const int64_t off = offsets[e];
   const int rows = static_cast<int>(offsets[e + 1] - off);
+  if (k0 >= (rows + 63) / 64 * 64) return;  // the product reads k-blocks of 64 below the group's rows only
   for (int i = threadIdx.y; i < 32; i += 8) {
     const int kk = k0 + i, f = f0 + threadIdx.x;
     float v = 0.f;
@@ -842,14 +845,14 @@ cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
       return e;
     if ((e = pack<float, true>(a.U, a.d_ff, a.offsets, nullptr, groups, kp, P1, pl, s)) != cudaSuccess) return e;
     if ((e = pack<float, true>(a.A1, a.d_ff, a.offsets, a.row_gate, groups, kp, PH, pl, s)) != cudaSuccess) return e;
-    if ((e = tc_product(a, P1, P1 + pl, a.XT, a.d, kp, a.dW1, s, a.woff, a.wpre, arows, a.d_ff)) != cudaSuccess)
+    if ((e = tc_product(a, P1, P1 + pl, a.XT, a.d, kp, a.dW1, s, a.woff, a.wpre, arows, a.d_ff, a.offsets)) != cudaSuccess)
       return e;
     if (swiglu) {
       if ((e = pack<float, true>(a.A3, a.d_ff, a.offsets, nullptr, groups, kp, P3, pl, s)) != cudaSuccess) return e;
-      if ((e = tc_product(a, P3, P3 + pl, a.XT, a.d, kp, a.dW3, s, a.woff, a.wpre, arows, a.d_ff)) != cudaSuccess)
+      if ((e = tc_product(a, P3, P3 + pl, a.XT, a.d, kp, a.dW3, s, a.woff, a.wpre, arows, a.d_ff, a.offsets)) != cudaSuccess)
         return e;
     }
-    if ((e = tc_product(a, PH, PH + pl, a.DT, a.d, kp, a.dW2t, s, a.woff, a.wpre, arows, a.d_ff)) != cudaSuccess)
+    if ((e = tc_product(a, PH, PH + pl, a.DT, a.d, kp, a.dW2t, s, a.woff, a.wpre, arows, a.d_ff, a.offsets)) != cudaSuccess)
       return e;
     if ((e = transpose_f32(a.dW2t, a.dW2, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
   } else {

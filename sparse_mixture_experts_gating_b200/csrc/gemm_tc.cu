@@ -102,7 +102,9 @@ __device__ __forceinline__ void decode_tile(int t, const Ctl* c, int E, int n_ti
 // K range u % ksplit.  Otherwise, when the tiles leave a last wave at most
 // half full (p.split_tail: not SwiGLU, whose tile pairs W1 and W3 columns),
 // each tile of that last wave becomes two units of half its columns (N 128),
-// so the last wave takes half as long.
+// so the last wave takes half as long.  With a per-group K (p.k_rows, the
+// weight gradients over each expert's rows) a tile runs only its group's
+// k-blocks, none for an empty group (whose output the epilogue writes as 0).
 struct Item {
   int tile, ks;    // tile and K-range index
   int kb0, kb1;    // k-blocks [kb0, kb1)
@@ -125,7 +127,7 @@ __device__ __forceinline__ ItemIter iter_begin(const Ctl* c, const Params& p) {
   }
   return it;
 }
-__device__ __forceinline__ bool iter_next(ItemIter& it, const Params& p, Item& w) {
+__device__ __forceinline__ bool iter_next(ItemIter& it, const Params& p, const Ctl* ctl, Item& w) {
   if (it.u >= it.units) return false;
   if (it.u < it.whole) {
     w.tile = it.u / p.ksplit;
@@ -139,6 +141,11 @@ __device__ __forceinline__ bool iter_next(ItemIter& it, const Params& p, Item& w
   }
   w.kb0 = w.ks * p.kb_per;
   w.kb1 = min(p.num_kb, w.kb0 + p.kb_per);
+  if (p.k_rows != nullptr) {  // this group's own K (no K ranges): its k-blocks only, possibly none
+    int e, mt, nt;
+    decode_tile(w.tile, ctl, p.E, p.n_tiles, e, mt, nt);
+    w.kb1 = min(w.kb1, (p.k_rows[e + 1] - p.k_rows[e] + BK - 1) / BK);
+  }
   it.u += static_cast<int>(gridDim.x);
   return true;
 }
@@ -243,7 +250,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       ItemIter it = iter_begin(ctl, p);
       Item w;
-      while (ok && iter_next(it, p, w)) {
+      while (ok && iter_next(it, p, ctl, w)) {
         int e, mt, nt;
         decode_tile(w.tile, ctl, p.E, p.n_tiles, e, mt, nt);
         const int row0 = ctl->offsets[e] + mt * BM;
@@ -281,7 +288,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       ItemIter it = iter_begin(ctl, p);
       Item w;
-      while (ok && iter_next(it, p, w)) {
+      while (ok && iter_next(it, p, ctl, w)) {
         if (!wait_or_abort(ctl, &ctl->tempty[acc], acc_phase ^ 1u, p)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * MMA_N);
@@ -325,7 +332,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t acc_phase = 0;
     ItemIter it = iter_begin(ctl, p);
     Item w;
-    while (iter_next(it, p, w)) {
+    while (iter_next(it, p, ctl, w)) {
       int e, mt, nt;
       decode_tile(w.tile, ctl, p.E, p.n_tiles, e, mt, nt);
       const int ks = w.ks;
@@ -428,8 +435,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll 1
         for (int c = 0; c < nch; ++c) {
           uint32_t ra[32];
-          tmem_ld32(tb + c * 32, ra);
-          tmem_ld_wait();
+          if (w.kb1 > w.kb0) {
+            tmem_ld32(tb + c * 32, ra);
+            tmem_ld_wait();
+          } else {  // a group with no k-blocks (per-group K of 0): the product is zero
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ra[i] = 0u;
+          }
           float4* srow = reinterpret_cast<float4*>(stg + lane * 144);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
@@ -664,6 +676,11 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
   p.row_token = g.row_token;
   p.err = g.err;
   p.limit_ns = kWaitLimitNs;
+  p.k_rows = g.k_rows;
+  if (g.k_rows != nullptr && (g.epi != EPI_GATE_F32 || p.ksplit != 1)) {
+    *why = "grouped GEMM: a per-group K needs the gated fp32 epilogue without K ranges";
+    return cudaErrorInvalidValue;
+  }
   pl->epi = g.epi;
   pl->hid = g.f16 ? HID_F16 : g.split ? HID_BF16X2 : HID_BF16;
   if (g.epi < EPI_RELU_BF16 || g.epi > EPI_GATE_SCATTER_BF16) {

@@ -125,6 +125,7 @@ struct GemmArgs {
   const float* row_gate;
   const int32_t* row_token;
   unsigned int* err;
+  const int32_t* k_rows;  // gated fp32 epilogue: group e's K is k_rows[e + 1] - k_rows[e] (NULL: K)
 };
 
 // Kernel parameters of the tensor-core grouped GEMM.
@@ -142,6 +143,7 @@ struct TcParams {
   const int32_t* row_token;
   unsigned int* err;
   uint64_t limit_ns;
+  const int32_t* k_rows;  // per-group K (k-blocks ceil(K_e / 64)), NULL: K for every group
 };
 
 // How the hidden activation between the projections is held.
