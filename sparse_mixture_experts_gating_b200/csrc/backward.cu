@@ -367,68 +367,80 @@ __global__ void __launch_bounds__(THREADS) bw_router_kernel(BackwardArgs a) {
   }
 }
 
-// dx for 64 tokens x 64 columns per block (16 x 16 threads, 4 x 4 outputs
-// each, 16-byte accesses): the router term W_r^T dh_t from 32-expert chunks
-// of dh and W_r staged in shared memory, experts in order, then the same sum
-// as bw_dx_kernel (kept rows' dXp, choices in order, then the shared
-// experts' rows) plus that term: the same operations in the same order.
-// Needs d % 4 == 0 and 16-byte aligned dXp and dx.
+// dx for 128 tokens x 128 columns per block (16 x 16 threads, 8 x 8 outputs
+// each): the router term W_r^T dh_t from 32-expert chunks of dh (transposed)
+// and W_r staged in shared memory, experts in order, then the same sum as
+// bw_dx_kernel (kept rows' dXp, choices in order, then the shared experts'
+// rows) plus that term: the same operations in the same order.  Needs
+// d % 8 == 0, E % 4 == 0 and 16-byte aligned dh, W_r, dXp and dx.
 __global__ void __launch_bounds__(256) bw_dx_tiled_kernel(BackwardArgs a, int parts) {
-  __shared__ float s_dh[64][33];
-  __shared__ __align__(16) float s_w[32][68];
+  __shared__ __align__(16) float s_h[32][132];  // [expert][token]
+  __shared__ __align__(16) float s_w[32][132];  // [expert][column]
   const int E = a.E, d = a.d, k = a.k;
   const int64_t T = a.T;
-  const int t0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.y) * 128;
+  const int c0 = blockIdx.x * 128;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  float acc[4][4];
+  float acc[8][8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
   for (int e0 = 0; e0 < E; e0 += 32) {
     const int ne = min(32, E - e0);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {  // dh [64 tokens][32 experts]
-      const int idx = tid + 256 * q, r = idx >> 5, e = idx & 31;
-      s_dh[r][e] = (t0 + r < T && e < ne) ? a.dh[(static_cast<int64_t>(t0) + r) * E + e0 + e] : 0.f;
+    for (int q = 0; q < 4; ++q) {  // dh [128 tokens][32 experts] -> s_h[expert][token]
+      const int id = tid + 256 * q, t = id >> 3, e4 = (id & 7) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t0 + t < T && e4 < ne) v = *reinterpret_cast<const float4*>(a.dh + (t0 + t) * E + e0 + e4);
+      s_h[e4][t] = v.x;
+      s_h[e4 + 1][t] = v.y;
+      s_h[e4 + 2][t] = v.z;
+      s_h[e4 + 3][t] = v.w;
     }
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {  // W_r [32 experts][64 columns], 16-byte loads
-      const int idx = tid + 256 * q, e = idx >> 4, c = (idx & 15) * 4;
+    for (int q = 0; q < 4; ++q) {  // W_r [32 experts][128 columns]
+      const int id = tid + 256 * q, e = id >> 5, c = (id & 31) * 4;
       float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
       if (e < ne && c0 + c < d) w = *reinterpret_cast<const float4*>(a.W_r + static_cast<int64_t>(e0 + e) * d + c0 + c);
       *reinterpret_cast<float4*>(&s_w[e][c]) = w;
     }
     __syncthreads();
     for (int e = 0; e < ne; ++e) {
-      const float4 w = *reinterpret_cast<const float4*>(&s_w[e][tx * 4]);
+      const float4 h0 = *reinterpret_cast<const float4*>(&s_h[e][ty * 8]);
+      const float4 h1 = *reinterpret_cast<const float4*>(&s_h[e][ty * 8 + 4]);
+      const float4 w0 = *reinterpret_cast<const float4*>(&s_w[e][tx * 8]);
+      const float4 w1 = *reinterpret_cast<const float4*>(&s_w[e][tx * 8 + 4]);
+      const float h[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+      const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float h = s_dh[ty * 4 + i][e];
-        acc[i][0] = fmaf(h, w.x, acc[i][0]);
-        acc[i][1] = fmaf(h, w.y, acc[i][1]);
-        acc[i][2] = fmaf(h, w.z, acc[i][2]);
-        acc[i][3] = fmaf(h, w.w, acc[i][3]);
-      }
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(h[i], w[j], acc[i][j]);
     }
     __syncthreads();
   }
-  const int c = c0 + tx * 4;
+  const int c = c0 + tx * 8;
   if (c >= d) return;
   const int64_t pstride = a.s_max * d;  // between the W1 and W3 parts of dXp
   const int64_t sbase = a.n_shared > 0 ? a.offsets[E] : 0;
-  const float4* X4 = reinterpret_cast<const float4*>(a.dXp);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t t = t0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const int64_t t = t0 + ty * 8 + i;
     if (t >= T) break;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = 0.f;
     auto add_row = [&](int64_t row) {
-      const float4 p = X4[(row * d + c) >> 2];
-      v.x += p.x; v.y += p.y; v.z += p.z; v.w += p.w;
+      const float4* p = reinterpret_cast<const float4*>(a.dXp + row * d + c);
+      const float4 p0 = p[0], p1 = p[1];
+      v[0] += p0.x; v[1] += p0.y; v[2] += p0.z; v[3] += p0.w;
+      v[4] += p1.x; v[5] += p1.y; v[6] += p1.z; v[7] += p1.w;
       if (parts == 2) {
-        const float4 p2 = X4[(pstride + row * d + c) >> 2];
-        v.x += p2.x; v.y += p2.y; v.z += p2.z; v.w += p2.w;
+        const float4* p2 = reinterpret_cast<const float4*>(a.dXp + pstride + row * d + c);
+        const float4 q0 = p2[0], q1 = p2[1];
+        v[0] += q0.x; v[1] += q0.y; v[2] += q0.z; v[3] += q0.w;
+        v[4] += q1.x; v[5] += q1.y; v[6] += q1.z; v[7] += q1.w;
       }
     };
     for (int j = 0; j < k; ++j) {
@@ -436,8 +448,9 @@ __global__ void __launch_bounds__(256) bw_dx_tiled_kernel(BackwardArgs a, int pa
       if (dst >= 0) add_row(dst);
     }
     for (int si = 0; si < a.n_shared; ++si) add_row(sbase + si * T + t);
-    *reinterpret_cast<float4*>(a.dx + t * d + c) =
-        make_float4(v.x + acc[i][0], v.y + acc[i][1], v.z + acc[i][2], v.w + acc[i][3]);
+    float4* o = reinterpret_cast<float4*>(a.dx + t * d + c);
+    o[0] = make_float4(v[0] + acc[i][0], v[1] + acc[i][1], v[2] + acc[i][2], v[3] + acc[i][3]);
+    o[1] = make_float4(v[4] + acc[i][4], v[5] + acc[i][5], v[6] + acc[i][6], v[7] + acc[i][7]);
   }
 }
 
@@ -705,12 +718,89 @@ __global__ void __launch_bounds__(256) bw_pack_kernel(const ST* __restrict__ src
   }
 }
 
+// The same operand in 64 (kk) x 64 (f) tiles with 16-byte accesses: rows of
+// src read along f (fp32 tile in shared memory), 16-byte writes of eight
+// consecutive kk of one f, the threads of a warp writing whole 128-byte row
+// segments.  Needs F % 8 == 0, k_pad % 8 == 0 and 16-byte aligned buffers.
+template <typename ST, bool SPLIT>
+__global__ void __launch_bounds__(256) bw_pack16_kernel(const ST* __restrict__ src, int F,
+                                                        const int32_t* __restrict__ offsets,
+                                                        const float* __restrict__ scale, int k_pad,
+                                                        __nv_bfloat16* __restrict__ out, int64_t plane) {
+  constexpr int V = 16 / static_cast<int>(sizeof(ST));  // source elements per 16-byte load
+  constexpr int NL = 64 * 64 / V / 256;                  // loads per thread
+  __shared__ float tile[64][65];
+  const int e = blockIdx.z;
+  const int f0 = blockIdx.x * 64, k0 = blockIdx.y * 64;
+  const int64_t off = offsets[e];
+  const int rows = static_cast<int>(offsets[e + 1] - off);
+  if (k0 >= (rows + 63) / 64 * 64) return;  // the product reads k-blocks of 64 below the group's rows only
+#pragma unroll
+  for (int p = 0; p < NL; ++p) {
+    const int id = threadIdx.x + 256 * p;
+    const int r = id / (64 / V), c = (id % (64 / V)) * V;
+    float v[V];
+    if (k0 + r < rows && f0 + c < F) {
+      const uint4 u = *reinterpret_cast<const uint4*>(src + (off + k0 + r) * F + f0 + c);
+      const float sc = scale != nullptr ? scale[off + k0 + r] : 1.f;
+      if constexpr (sizeof(ST) == 2) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[2 * j] = __uint_as_float(w[j] << 16);
+          v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+      } else {
+        v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y); v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+      }
+      if (scale != nullptr)
+#pragma unroll
+        for (int j = 0; j < V; ++j) v[j] *= sc;
+    } else {
+#pragma unroll
+      for (int j = 0; j < V; ++j) v[j] = 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < V; ++j) tile[r][c + j] = v[j];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {  // output row f0 + oc, kk = k0 + 8 q .. + 7
+    const int id = threadIdx.x + 256 * p;
+    const int oc = id / 8, q = id % 8;
+    if (f0 + oc >= F || k0 + 8 * q >= k_pad) continue;
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float a = tile[8 * q + 2 * j][oc], b = tile[8 * q + 2 * j + 1][oc];
+      const __nv_bfloat16 ha = __float2bfloat16_rn(a), hb = __float2bfloat16_rn(b);
+      hi[j] = static_cast<uint32_t>(__bfloat16_as_ushort(ha)) | (static_cast<uint32_t>(__bfloat16_as_ushort(hb)) << 16);
+      if (SPLIT) {
+        const __nv_bfloat16 la = __float2bfloat16_rn(a - __bfloat162float(ha));
+        const __nv_bfloat16 lb = __float2bfloat16_rn(b - __bfloat162float(hb));
+        lo[j] = static_cast<uint32_t>(__bfloat16_as_ushort(la)) | (static_cast<uint32_t>(__bfloat16_as_ushort(lb)) << 16);
+      }
+    }
+    const int64_t o = (static_cast<int64_t>(e) * F + f0 + oc) * k_pad + k0 + 8 * q;
+    *reinterpret_cast<uint4*>(out + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    if (SPLIT) *reinterpret_cast<uint4*>(out + plane + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+}
+
 template <typename ST, bool SPLIT>
 cudaError_t pack(const void* src, int F, const int32_t* offsets, const float* scale, int G, int k_pad, void* out,
                  int64_t plane, cudaStream_t s) {
-  const dim3 grid((F + 31) / 32, (k_pad + 31) / 32, G);
-  bw_pack_kernel<ST, SPLIT><<<grid, dim3(32, 8), 0, s>>>(static_cast<const ST*>(src), F, offsets, scale, k_pad,
-                                                         static_cast<__nv_bfloat16*>(out), plane);
+  const bool wide = F % 8 == 0 && k_pad % 8 == 0 && plane % 8 == 0 &&
+                    ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(out)) & 15) == 0;
+  if (wide) {
+    const dim3 grid((F + 63) / 64, (k_pad + 63) / 64, G);
+    bw_pack16_kernel<ST, SPLIT><<<grid, 256, 0, s>>>(static_cast<const ST*>(src), F, offsets, scale, k_pad,
+                                                     static_cast<__nv_bfloat16*>(out), plane);
+  } else {
+    const dim3 grid((F + 31) / 32, (k_pad + 31) / 32, G);
+    bw_pack_kernel<ST, SPLIT><<<grid, dim3(32, 8), 0, s>>>(static_cast<const ST*>(src), F, offsets, scale, k_pad,
+                                                           static_cast<__nv_bfloat16*>(out), plane);
+  }
   count_launch();
   return cudaGetLastError();
 }
@@ -882,12 +972,12 @@ cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
   bw_router_kernel<XT><<<static_cast<unsigned>(a.T), THREADS, 0, s>>>(a);
   count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const bool tiled = a.d % 4 == 0 && (a.T + 63) / 64 <= 65535 &&
+  const bool tiled = a.d % 8 == 0 && a.E % 4 == 0 && (a.T + 127) / 128 <= 65535 &&
                      ((reinterpret_cast<uintptr_t>(a.W_r) | reinterpret_cast<uintptr_t>(a.dXp) |
-                       reinterpret_cast<uintptr_t>(a.dx)) & 15) == 0;
+                       reinterpret_cast<uintptr_t>(a.dx) | reinterpret_cast<uintptr_t>(a.dh)) & 15) == 0;
   if (tiled)
-    bw_dx_tiled_kernel<<<dim3(static_cast<unsigned>((a.d + 63) / 64), static_cast<unsigned>((a.T + 63) / 64)), 256, 0,
-                         s>>>(a, parts);
+    bw_dx_tiled_kernel<<<dim3(static_cast<unsigned>((a.d + 127) / 128), static_cast<unsigned>((a.T + 127) / 128)), 256,
+                         0, s>>>(a, parts);
   else
     bw_dx_kernel<<<static_cast<unsigned>(a.T), THREADS, 0, s>>>(a, parts);
   count_launch();
