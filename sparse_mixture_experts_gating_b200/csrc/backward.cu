@@ -545,6 +545,39 @@ cudaError_t tc_product(const BackwardArgs& a, const void* A, const void* A_lo, c
   return launch_gemm_tc(plan, a.num_sms, s);
 }
 
+// The per-expert product with a single-plane A and B as hi + lo planes
+// (EPI_GATE_F32_B2, gate 1): out[r][n] = sum_k A[r][k] (B_hi + B_lo)_e[n][k]
+// over groups of max_rows rows (offsets / mprefix), group e's K = its rows
+// in k_rows.
+cudaError_t tc_product_b2(const BackwardArgs& a, const void* A, const void* B_hi, const void* B_lo, int N, int K,
+                          float* out, cudaStream_t s, const int32_t* offsets, const int32_t* mprefix, int64_t a_rows,
+                          int max_rows, const int32_t* k_rows) {
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.epi = EPI_GATE_F32_B2;
+  g.E = a.E + a.n_shared;
+  g.N = N;
+  g.K = K;
+  g.a_rows = a_rows;
+  g.max_group_rows = max_rows;
+  g.A = A;
+  g.B0 = B_hi;
+  g.B1 = B_lo;
+  g.out = out;
+  g.ksplit = 1;
+  g.offsets = offsets;
+  g.mprefix = mprefix;
+  g.row_gate = a.ones;
+  g.row_token = a.row_token;
+  g.err = a.err;
+  g.k_rows = k_rows;
+  TcGemmPlan plan;
+  const char* why = nullptr;
+  cudaError_t e = plan_gemm_tc(g, &plan, &why);
+  if (e != cudaSuccess) return e;
+  return launch_gemm_tc(plan, a.num_sms, s);
+}
+
 // bf16 [G][R][C] -> [G][C][R] with R and C even: 64 x 64 tiles, pairs of
 // columns read and pairs of rows written as 4-byte words.
 __global__ void __launch_bounds__(256) bw_transpose_bf16x2_kernel(const __nv_bfloat16* __restrict__ in,
@@ -572,32 +605,6 @@ __global__ void __launch_bounds__(256) bw_transpose_bf16x2_kernel(const __nv_bfl
       v.y = tile[2 * tx + 1][i];
       *reinterpret_cast<__nv_bfloat162*>(dst + static_cast<int64_t>(c) * R + r) = v;
     }
-  }
-}
-
-// fp32 [G][R][C] -> [G][C][R] with R and C even: 64 x 64 tiles, pairs of
-// columns read and pairs of rows written as 8-byte words.
-__global__ void __launch_bounds__(256) bw_transpose_f32x2_kernel(const float* __restrict__ in, float* __restrict__ out,
-                                                                 int R, int C) {
-  __shared__ float tile[64][65];
-  const int64_t g = blockIdx.z;
-  const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const float* src = in + g * R * C;
-  float* dst = out + g * R * C;
-  for (int i = ty; i < 64; i += 8) {
-    const int r = r0 + i, c = c0 + 2 * tx;
-    if (r < R && c < C) {
-      const float2 v = *reinterpret_cast<const float2*>(src + static_cast<int64_t>(r) * C + c);
-      tile[i][2 * tx] = v.x;
-      tile[i][2 * tx + 1] = v.y;
-    }
-  }
-  __syncthreads();
-  for (int i = ty; i < 64; i += 8) {
-    const int c = c0 + i, r = r0 + 2 * tx;
-    if (c < C && r < R)
-      *reinterpret_cast<float2*>(dst + static_cast<int64_t>(c) * R + r) = make_float2(tile[2 * tx][i], tile[2 * tx + 1][i]);
   }
 }
 
@@ -654,16 +661,6 @@ __global__ void __launch_bounds__(256) bw_transpose16_kernel(const T* __restrict
 
 bool aligned16(const void* a, const void* b) {
   return ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 15) == 0;
-}
-
-cudaError_t transpose_f32(const void* in, void* out, int G, int R, int C, cudaStream_t s) {
-  const dim3 grid((C + 63) / 64, (R + 63) / 64, G);
-  if (aligned16(in, out) && R % 4 == 0 && C % 4 == 0)
-    bw_transpose16_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(in), static_cast<float*>(out), R, C);
-  else  // a gradient output without 16-byte alignment
-    bw_transpose_f32x2_kernel<<<grid, 256, 0, s>>>(static_cast<const float*>(in), static_cast<float*>(out), R, C);
-  count_launch();
-  return cudaGetLastError();
 }
 
 cudaError_t transpose_bf16(const void* in, void* out, int G, int R, int C, cudaStream_t s) {
@@ -806,13 +803,17 @@ cudaError_t pack(const void* src, int F, const int32_t* offsets, const float* sc
 }
 
 // Gate 1 for n rows, and the group tables of the per-expert products
-// (groups of F rows each: offsets e F, m-tile prefix e ceil(F / 128)).
-__global__ void bw_tables_kernel(int64_t n, float* ones, int G, int F, int32_t* woff, int32_t* wpre) {
+// (groups of F rows each: offsets e F, m-tile prefix e ceil(F / 128)), for
+// F = F1 and F = F2.
+__global__ void bw_tables_kernel(int64_t n, float* ones, int G, int F1, int32_t* woff1, int32_t* wpre1, int F2,
+                                 int32_t* woff2, int32_t* wpre2) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   if (i < n) ones[i] = 1.f;
   if (i <= G) {
-    woff[i] = static_cast<int32_t>(i * F);
-    wpre[i] = static_cast<int32_t>(i * ((F + kTileM - 1) / kTileM));
+    woff1[i] = static_cast<int32_t>(i * F1);
+    wpre1[i] = static_cast<int32_t>(i * ((F1 + kTileM - 1) / kTileM));
+    woff2[i] = static_cast<int32_t>(i * F2);
+    wpre2[i] = static_cast<int32_t>(i * ((F2 + kTileM - 1) / kTileM));
   }
 }
 
@@ -850,9 +851,9 @@ cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
     if ((e = transpose_bf16(a.W2, a.W2t, groups, a.d, a.d_ff, s)) != cudaSuccess) return e;
     if ((e = transpose_bf16(a.W1, a.W1t, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
     if (swiglu && (e = transpose_bf16(a.W3, a.W3t, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
-    const int64_t n_ones = std::max<int64_t>(a.s_max, static_cast<int64_t>(groups) * a.d_ff);
+    const int64_t n_ones = std::max<int64_t>(a.s_max, static_cast<int64_t>(groups) * std::max(a.d_ff, a.d));
     bw_tables_kernel<<<static_cast<unsigned>((std::max<int64_t>(n_ones, groups + 1) + 255) / 256), 256, 0, s>>>(
-        n_ones, a.ones, groups, a.d_ff, a.woff, a.wpre);
+        n_ones, a.ones, groups, a.d_ff, a.woff, a.wpre, a.d, a.woff_d, a.wpre_d);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bw_gather_dy_kernel<<<static_cast<unsigned>((a.s_max + 7) / 8), 256, 0, s>>>(
@@ -942,9 +943,10 @@ cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
       if ((e = tc_product(a, P3, P3 + pl, a.XT, a.d, kp, a.dW3, s, a.woff, a.wpre, arows, a.d_ff, a.offsets)) != cudaSuccess)
         return e;
     }
-    if ((e = tc_product(a, PH, PH + pl, a.DT, a.d, kp, a.dW2t, s, a.woff, a.wpre, arows, a.d_ff, a.offsets)) != cudaSuccess)
+    // dW2_e [d][d_ff] directly: A = dy^T (d rows per expert), B = (g hid)^T as hi + lo planes
+    if ((e = tc_product_b2(a, a.DT, PH, PH + pl, a.d_ff, kp, a.dW2, s, a.woff_d, a.wpre_d,
+                           static_cast<int64_t>(groups) * a.d, a.d, a.offsets)) != cudaSuccess)
       return e;
-    if ((e = transpose_f32(a.dW2t, a.dW2, groups, a.d_ff, a.d, s)) != cudaSuccess) return e;
   } else {
   WGrad w{};
   w.offsets = a.offsets;

@@ -58,9 +58,10 @@ struct BackwardArgs {
   void* PH;                // same for g * hid
   void* XT;                // [G][d][k_pad] bf16: Xp per expert, transposed
   void* DT;                // [G][d][k_pad] bf16: dy (sorted rows) per expert, transposed
-  float* dW2t;             // [G][d_ff][d] fp32: dW2 transposed
   int32_t* woff;           // [G + 1] rows of the per-expert products: e * d_ff
   int32_t* wpre;           // [G + 1] their m-tile prefix: e * ceil(d_ff / 128)
+  int32_t* woff_d;         // [G + 1] the same for products of d rows (dW2): e * d
+  int32_t* wpre_d;         // [G + 1] e * ceil(d / 128)
   // dW_r: the sum over tokens cut into wr_chunks chunks of partials
   int wr_chunks;
   float* wr_part;          // [wr_chunks][E][d]

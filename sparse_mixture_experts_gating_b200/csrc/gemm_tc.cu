@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mbar_arrive_expect_tx(&ctl->full[stage], tx);
           if (A_SPLIT) tma_load_3d(sa, &tmA, &ctl->full[stage], kb * BK, row0, 0);  // hi and lo planes
           else tma_load_2d(sa, &tmA, &ctl->full[stage], kb * BK, row0);
-          if (EPI == EPI_SWIGLU_BF16) {
+          if (EPI == EPI_SWIGLU_BF16 || EPI == EPI_GATE_F32_B2) {  // W1 / W3, or B's hi / lo planes
             tma_load_2d(sa + B_OFF, &tmB0, &ctl->full[stage], kb * BK, brow);
             tma_load_2d(sa + B_OFF + B_HALF, &tmB1, &ctl->full[stage], kb * BK, brow);
           } else if (w.half >= 0) {
@@ -353,7 +353,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // destination row of each 32-row block row this lane stores (for bf16: rows lane/4 + 8i)
       int drow[4];
       bool dval[4];
-      const float g = (EPI == EPI_GATE_F32 || EPI == EPI_GATE_SCATTER_BF16) && vrow ? p.row_gate[row] : 0.f;
+      const float g =
+          (EPI == EPI_GATE_F32 || EPI == EPI_GATE_SCATTER_BF16 || EPI == EPI_GATE_F32_B2) && vrow ? p.row_gate[row] : 0.f;
       const int my_dst = (EPI == EPI_GATE_SCATTER_BF16) ? (vrow ? p.row_token[row] : 0) : row;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -429,13 +430,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         if (OUT_F16 && __any_sync(0xffffffffu, out_of_range) && lane == 0) record_error(p.err, DEV_ERR_RANGE);
-      } else {  // EPI_GATE_F32: gated fp32 rows of the expert-sorted buffer (partial ks)
+      } else {  // EPI_GATE_F32(_B2): gated fp32 rows of the expert-sorted buffer (partial ks)
         float* out = static_cast<float*>(p.out) + static_cast<int64_t>(ks) * p.split_stride;
-        const int nch = w.half >= 0 ? 4 : 8;
+        const int nch = (w.half >= 0 || EPI == EPI_GATE_F32_B2) ? 4 : 8;
 #pragma unroll 1
         for (int c = 0; c < nch; ++c) {
           uint32_t ra[32];
-          if (w.kb1 > w.kb0) {
+          if (w.kb1 > w.kb0 && EPI == EPI_GATE_F32_B2) {  // hi-plane and lo-plane products summed
+            uint32_t rb[32];
+            tmem_ld32(tb + c * 32, ra);
+            tmem_ld32(tb + 128 + c * 32, rb);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ra[i] = __float_as_uint(__uint_as_float(ra[i]) + __uint_as_float(rb[i]));
+          } else if (w.kb1 > w.kb0) {
             tmem_ld32(tb + c * 32, ra);
             tmem_ld_wait();
           } else {  // a group with no k-blocks (per-group K of 0): the product is zero
@@ -581,6 +589,9 @@ cudaError_t launch_epi(const TcGemmPlan& pl, int num_sms, cudaStream_t s) {
     case EPI_RELU_BF16: return launch_ar<EPI_RELU_BF16, HID>(pl, num_sms, s);
     case EPI_SWIGLU_BF16: return launch_ar<EPI_SWIGLU_BF16, HID>(pl, num_sms, s);
     case EPI_GATE_F32: return launch_ar<EPI_GATE_F32, HID>(pl, num_sms, s);
+    case EPI_GATE_F32_B2:
+      if constexpr (HID == HID_BF16) return launch_ar<EPI_GATE_F32_B2, HID>(pl, num_sms, s);
+      return cudaErrorInvalidValue;
     default: return launch_ar<EPI_GATE_SCATTER_BF16, HID>(pl, num_sms, s);
   }
 }
@@ -627,6 +638,11 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
   const bool a_split = g.split && g.A2 != nullptr;
   const bool ops_f16 = g.f16 && gate;  // A and B of the second projection in fp16
   const bool swiglu = g.epi == EPI_SWIGLU_BF16;
+  const bool b2 = g.epi == EPI_GATE_F32_B2;  // B as hi + lo planes, like W1 / W3: two 128-row boxes
+  if (b2 && (g.split || g.f16 || g.B1 == nullptr)) {
+    *why = "grouped GEMM: a split B operand takes a single-plane bf16 A and both B planes";
+    return cudaErrorInvalidValue;
+  }
   // A rows per stage: every expert group has at most max_group_rows rows
   pl->ar = g.max_group_rows <= 32 ? 32 : g.max_group_rows <= 64 ? 64 : 128;
   const uint32_t ar = static_cast<uint32_t>(pl->ar);
@@ -650,8 +666,8 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
                       : make_map_bf16(&pl->a, g.A, a_rows, K, ar)) &&
              make_map(&pl->a2, a_split ? g.A2 : g.A, a_rows, K) &&
              // B: two 128-row boxes (W1 and W3) for SwiGLU, else one 256-row box
-             make_map_bf16(&pl->b0, g.B0, b_rows, K, swiglu ? 128 : 256) &&
-             make_map(&pl->b1, swiglu ? g.B1 : g.B0, b_rows, K));
+             make_map_bf16(&pl->b0, g.B0, b_rows, K, swiglu || b2 ? 128 : 256) &&
+             make_map(&pl->b1, swiglu || b2 ? g.B1 : g.B0, b_rows, K));
   if (!maps_ok) {
     *why = "cuTensorMapEncodeTiled failed (alignment or driver entry point)";
     return cudaErrorInvalidValue;
@@ -660,13 +676,13 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
   p.E = g.E;
   p.N = g.N;
   p.K = g.K;
-  p.bn = (g.epi == EPI_SWIGLU_BF16) ? 128 : 256;
+  p.bn = (swiglu || b2) ? 128 : 256;
   p.n_tiles = (g.N + p.bn - 1) / p.bn;
   p.num_kb = (g.K + BK - 1) / BK;
   p.ksplit = g.epi == EPI_GATE_F32 ? (g.ksplit < 1 ? 1 : (g.ksplit > p.num_kb ? p.num_kb : g.ksplit)) : 1;
   p.kb_per = (p.num_kb + p.ksplit - 1) / p.ksplit;
   p.split_stride = g.split_stride;
-  p.split_tail = swiglu ? 0 : 1;
+  p.split_tail = (swiglu || b2) ? 0 : 1;
   p.out = g.out;
   p.out_lo = g.out2;
   p.out_f32 = g.out_f32;
@@ -677,13 +693,13 @@ cudaError_t plan_gemm_tc(const GemmArgs& g, TcGemmPlan* pl, const char** why) {
   p.err = g.err;
   p.limit_ns = kWaitLimitNs;
   p.k_rows = g.k_rows;
-  if (g.k_rows != nullptr && (g.epi != EPI_GATE_F32 || p.ksplit != 1)) {
+  if (g.k_rows != nullptr && ((g.epi != EPI_GATE_F32 && !b2) || p.ksplit != 1)) {
     *why = "grouped GEMM: a per-group K needs the gated fp32 epilogue without K ranges";
     return cudaErrorInvalidValue;
   }
   pl->epi = g.epi;
   pl->hid = g.f16 ? HID_F16 : g.split ? HID_BF16X2 : HID_BF16;
-  if (g.epi < EPI_RELU_BF16 || g.epi > EPI_GATE_SCATTER_BF16) {
+  if (g.epi < EPI_RELU_BF16 || g.epi > EPI_GATE_F32_B2) {
     *why = "unknown epilogue";
     return cudaErrorInvalidValue;
   }

@@ -99,7 +99,10 @@ constexpr int kSplitTargetCtas = 148;
 int gemm2_ksplit(int64_t s_max, int E, int d, int d_ff);
 
 // Grouped GEMM epilogues
-enum GemmEpi { EPI_RELU_BF16 = 0, EPI_SWIGLU_BF16 = 1, EPI_GATE_F32 = 2, EPI_GATE_SCATTER_BF16 = 3 };
+// EPI_GATE_F32_B2: the gated fp32 epilogue with B given as hi + lo bf16 planes
+// (B0, B1): one N 256 MMA per step over a 128-row box of each, the two
+// halves of the accumulator summed per output column (128 columns per tile).
+enum GemmEpi { EPI_RELU_BF16 = 0, EPI_SWIGLU_BF16 = 1, EPI_GATE_F32 = 2, EPI_GATE_SCATTER_BF16 = 3, EPI_GATE_F32_B2 = 4 };
 
 struct GemmArgs {
   int epi;

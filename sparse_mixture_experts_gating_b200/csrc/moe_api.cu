@@ -275,7 +275,7 @@ Layout make_layout(const moe_layer& L, int64_t T, bool w4 = false) {
 // [G][d][d_ff] / [G][d_ff][d], the hi + lo planes of da1 (and da3)
 // [2][S][d_ff], and a second dXp part for SwiGLU.
 struct BwLayout {
-  size_t A1, A3, U, dg, dXp, dh, cnt1, ones, dYs, W1t, W3t, W2t, dA1p, dA3p, P1, P3, PH, XT, DT, dW2t, woff, wpre,
+  size_t A1, A3, U, dg, dXp, dh, cnt1, ones, dYs, W1t, W3t, W2t, dA1p, dA3p, P1, P3, PH, XT, DT, woff, wpre, woff_d, wpre_d,
       wr_part, total;
   // the forward's router kernel run again for its logits (bf16, E <= kRouterTcMaxE)
   bool rt;
@@ -309,7 +309,8 @@ BwLayout make_bw_layout(const moe_layer& L, const Layout& w) {
   b.max_group_rows = static_cast<int>(max_group_rows_of(L, w));
   b.k_pad = (b.max_group_rows + 7) / 8 * 8;
   const size_t kp = static_cast<size_t>(b.k_pad);
-  b.ones = take(tc ? sizeof(float) * std::max(S, G * static_cast<size_t>(L.d_ff)) : 0);
+  // gate 1 for every row of the products: the sorted rows, and G groups of d_ff or d rows
+  b.ones = take(tc ? sizeof(float) * std::max(S, G * static_cast<size_t>(std::max(L.d_ff, L.d))) : 0);
   b.dYs = take(tc ? 2 * S * L.d : 0);
   b.W1t = take(wsz);
   b.W3t = take(swiglu ? wsz : 0);
@@ -323,9 +324,10 @@ BwLayout make_bw_layout(const moe_layer& L, const Layout& w) {
   b.PH = take(plane2);
   b.XT = take(tc ? 2 * G * L.d * kp : 0);
   b.DT = take(tc ? 2 * G * L.d * kp : 0);
-  b.dW2t = take(tc ? sizeof(float) * G * L.d * static_cast<size_t>(L.d_ff) : 0);
   b.woff = take(tc ? sizeof(int32_t) * (G + 1) : 0);
   b.wpre = take(tc ? sizeof(int32_t) * (G + 1) : 0);
+  b.woff_d = take(tc ? sizeof(int32_t) * (G + 1) : 0);
+  b.wpre_d = take(tc ? sizeof(int32_t) * (G + 1) : 0);
   // dW_r's partials: chunks of at least 256 tokens, at most 64 of them
   const int64_t ch = (w.T + 255) / 256;
   b.wr_chunks = static_cast<int>(ch < 1 ? 1 : (ch > 64 ? 64 : ch));
@@ -902,8 +904,11 @@ int moe_backward(moe_handle h, int64_t T, const void* x, const float* W_r, const
     return fail(MOE_ERR_INVALID_ARG, "moe_backward: workspaces must be 256-byte aligned");
   const uintptr_t al = reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy) |
                        reinterpret_cast<uintptr_t>(W1) | reinterpret_cast<uintptr_t>(W2) |
-                       reinterpret_cast<uintptr_t>(W3);
-  if ((al & 15) != 0) return fail(MOE_ERR_INVALID_ARG, "moe_backward: x, dy and weights must be 16-byte aligned");
+                       reinterpret_cast<uintptr_t>(W3) | reinterpret_cast<uintptr_t>(dx) |
+                       reinterpret_cast<uintptr_t>(dW1) | reinterpret_cast<uintptr_t>(dW2) |
+                       reinterpret_cast<uintptr_t>(dW3);
+  if ((al & 15) != 0)
+    return fail(MOE_ERR_INVALID_ARG, "moe_backward: x, dy, weights, dx and the expert-weight gradients must be 16-byte aligned");
   DeviceInfo* di = nullptr;
   cudaError_t de = device_info(&di);
   if (de != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("moe_backward: ") + cudaGetErrorString(de));
@@ -965,9 +970,10 @@ int moe_backward(moe_handle h, int64_t T, const void* x, const float* W_r, const
     a.PH = bw + b.PH;
     a.XT = bw + b.XT;
     a.DT = bw + b.DT;
-    a.dW2t = reinterpret_cast<float*>(bw + b.dW2t);
     a.woff = reinterpret_cast<int32_t*>(bw + b.woff);
     a.wpre = reinterpret_cast<int32_t*>(bw + b.wpre);
+    a.woff_d = reinterpret_cast<int32_t*>(bw + b.woff_d);
+    a.wpre_d = reinterpret_cast<int32_t*>(bw + b.wpre_d);
   }
   a.dx = dx;
   a.dW_r = dW_r;
