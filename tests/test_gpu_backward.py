@@ -200,3 +200,32 @@ def test_backward_zero_tokens():
     status()
     for key in ("dW_r", "db_r", "dW1", "dW2"):
         assert not torch.any(g[key]), key
+
+
+def test_expert_no_token_chooses_gets_zero_weight_gradients():
+    """An expert that no token routes to has an empty group: the weight
+    gradients' products run none of its k-blocks, and its dW1 / dW2 rows must
+    come out exactly zero (the oracle's sum over no rows), the rest as usual.
+    A router bias of -64 on expert 3 (dyadic, so the logits stay exact) keeps
+    every token away from it."""
+    w = _w(CASES[0])
+    inp = make_inputs(w, device="cuda")
+    inp["b_r"][3] = -64.0
+    layer = layer_for(w)
+    dbg = layer.debug_buffers(w.T, inp["x"].device)
+    layer(inp["x"], inp["W_r"], inp["b_r"], inp["W1"], inp["W3"], inp["W2"], debug=dbg)
+    gen = torch.Generator().manual_seed(99)
+    dy = torch.randn(w.T, w.d, generator=gen).to(inp["x"].dtype).to(inp["x"].device)
+    g = layer.backward(inp["x"], inp["W_r"], inp["b_r"], inp["W1"], inp["W3"], inp["W2"], dy,
+                       aux_coef=AUX, z_coef=ZC)
+    status()
+    idx = dbg["topk_idx"].cpu().numpy()
+    assert not (idx == 3).any()
+    o = _oracle(w, inp, dy)
+    np.testing.assert_array_equal(idx, o["idx"])
+    assert not np.any(np32(g["dW1"])[3]) and not np.any(np32(g["dW2"])[3])
+    E = w.E
+    _close("dx", np32(g["dx"]), o["dx"])
+    _close("dW_r", np32(g["dW_r"]), o["dW_r"])
+    _close("dW1", np32(g["dW1"])[:E], o["dW1"])
+    _close("dW2", np32(g["dW2"])[:E], o["dW2"])
