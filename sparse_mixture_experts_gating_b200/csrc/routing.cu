@@ -1,10 +1,12 @@
 // Routing kernels of the MoE layer forward pass:
 //   router   - fp32 router logits h = W_r x (+ b), softmax, log-sum-exp, top-k
 //              (ties -> lower expert index), gates, per-block counts and sums
-//   scan     - per-expert totals, stable per-block rank bases, capacity,
-//              expert offsets, tile prefix, aux loss and z-loss
-//   dispatch - slot rank of each (token, choice) in token order, drop mask,
-//              permute of the kept token rows into expert-sorted order
+//   scan     - per-expert totals and stable per-block rank bases
+//   dispatch - capacity and expert offsets from the totals, slot rank of each
+//              (token, choice) in token order, drop mask, permute of the kept
+//              token rows into expert-sorted order; one extra block finalises
+//              the scan (offsets and tile prefix for the GEMMs, dropped count,
+//              aux loss, z-loss and the other balance statistics)
 //   combine  - y_t = sum over kept choices j (in order j) of the gated expert rows
 // Layer definition: "Mixture of experts" (rayaq.ca), sections "Replacing the
 // feed-forward block", "Top-k gating", "The load-balancing loss", "Capacity
@@ -250,10 +252,10 @@ cudaError_t launch_router_x(const RoutingArgs& a, cudaStream_t s) {
 // Scan: one block per expert e.  Each thread takes a contiguous run of the
 // router blocks, so the exclusive prefix of e's per-block counts (the stable
 // rank base of each block, in token order) is one block-wide scan; e's totals
-// (routed count, first-choice count, probability sum) go to the workspace.
-// The block that finishes last (ticket) turns the totals into capacity,
-// expert offsets, tile prefix, dropped count, aux loss and z-loss, all summed
-// in a fixed order.
+// (routed count, first-choice count, probability sum) go to the workspace,
+// where the dispatch launch turns them into capacity, expert offsets, tile
+// prefix, dropped count, aux loss and z-loss (scan_finalize), all summed in a
+// fixed order.
 constexpr int SCAN_T = 256;
 constexpr int kScanSingleBlocks = 8;  // up to 256 tokens: one block, one expert per thread
 
